@@ -1,0 +1,181 @@
+"""Float64 CPU oracle for one MMDiT block's joint-attention core.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke``
+and by the CPU-baseline leg of ``bench.py``.  Nothing in the product package
+imports it, and it imports nothing from the product package.
+
+The arithmetic lives in ``oracle.c`` (plain C loops in double precision); this
+module only marshals NumPy float64 arrays.  Which page and section each step
+follows is stated beside each function in ``oracle.c``:
+Vimoo 1.0 research page, section 2.2 (QK-RMSNorm, 3D RoPE 16/56/56 on the
+visual stream, joint attention over the concatenated streams with the output
+split back, adaLN modulate, gated residual) and the Wan 2.1 report, sections
+4.2.1 (raster flatten of the patched latent) and 4.3.1 (non-causal attention).
+
+Parity status: every function is pinned by tests in tests/test_oracle_pins.py
+(brute force with explicit rotation matrices and physically concatenated
+sequences, library routines for the special cases that reduce to them,
+closed forms and invariants).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional, Tuple
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+class _Grid(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("pos_scale", ctypes.c_double * 3), ("rope_base", ctypes.c_double),
+                ("split", ctypes.c_int * 3)]
+
+
+def _configure(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.oracle_rmsnorm.argtypes = [dp, dp, dp, ctypes.c_long, ctypes.c_int, ctypes.c_double]
+    lib.oracle_rope3d.argtypes = [dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                  ctypes.POINTER(_Grid)]
+    lib.oracle_joint_attention_rows.argtypes = (
+        [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [ctypes.c_int] * 5 +
+        [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp])
+    lib.oracle_adaln_modulate.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3 + [ctypes.c_double]
+    lib.oracle_gated_residual.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _configure(ctypes.CDLL(_build.build()))
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def rmsnorm(x, g, eps: float = 1e-6) -> np.ndarray:
+    """RMS-normalise the last axis of ``x`` (length D) and scale by ``g`` [D]."""
+    x = _f64(x)
+    g = _f64(g)
+    y = np.empty_like(x)
+    D = x.shape[-1]
+    _load().oracle_rmsnorm(_p(x), _p(y), _p(g), x.size // D, D, eps)
+    return y
+
+
+def rope3d(x, grid: Tuple[int, int, int], pos_scale=(1.0, 1.0, 1.0), base: float = 10000.0,
+           split=(16, 56, 56)) -> np.ndarray:
+    """Rotate visual rows x [B, N, H, D] by their (t, h, w) grid position."""
+    x = _f64(x).copy()
+    B, N, H, D = x.shape
+    if N != grid[0] * grid[1] * grid[2] or sum(split) != D:
+        raise ValueError("grid / split do not match x")
+    gr = _Grid(grid[0], grid[1], grid[2], (ctypes.c_double * 3)(*pos_scale), base,
+               (ctypes.c_int * 3)(*split))
+    _load().oracle_rope3d(_p(x), B, N, H, D, ctypes.byref(gr))
+    return x
+
+
+def qk_norm_rope(q, k, gq, gk, grid=None, pos_scale=(1.0, 1.0, 1.0), eps: float = 1e-6,
+                 base: float = 10000.0, split=(16, 56, 56)):
+    """QK-RMSNorm of q and k [B, N, H, D] with their own scales, then (when a
+    grid is given, i.e. for the visual stream) 3D RoPE."""
+    qn = rmsnorm(q, gq, eps)
+    kn = rmsnorm(k, gk, eps)
+    if grid is not None:
+        qn = rope3d(qn, grid, pos_scale, base, split)
+        kn = rope3d(kn, grid, pos_scale, base, split)
+    return qn, kn
+
+
+def joint_attention_rows(qv, kv, vv, qc, kc, vc, ctx_len, rows, scale: Optional[float] = None):
+    """Attention output for selected query rows.  ``rows`` is an int array of
+    (b, h, i) triplets with i the joint index (< Nv visual, else cond)."""
+    qv, kv, vv, qc, kc, vc = (_f64(a) for a in (qv, kv, vv, qc, kc, vc))
+    B, Nv, H, D = qv.shape
+    Nc = qc.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    out = np.zeros((rows.shape[0], D), dtype=np.float64)
+    if ctx_len is None:
+        cl_p = ctypes.POINTER(ctypes.c_int)()
+    else:
+        cl = np.ascontiguousarray(ctx_len, dtype=np.int32)
+        cl_p = cl.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+    if rows.shape[0]:
+        _load().oracle_joint_attention_rows(
+            _p(qv), _p(kv), _p(vv), _p(qc), _p(kc), _p(vc), cl_p, B, Nv, Nc, H, D, scale,
+            rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), rows.shape[0], _p(out))
+    return out
+
+
+def joint_attention(qv, kv, vv, qc, kc, vc, ctx_len=None, scale: Optional[float] = None):
+    """Full joint attention; returns (o_vis [B,Nv,H,D], o_ctx [B,Nc,H,D])."""
+    B, Nv, H, D = np.shape(qv)
+    Nc = np.shape(qc)[1]
+    bb, hh, ii = np.meshgrid(np.arange(B), np.arange(H), np.arange(Nv + Nc), indexing="ij")
+    rows = np.stack([bb.ravel(), hh.ravel(), ii.ravel()], axis=1)
+    out = joint_attention_rows(qv, kv, vv, qc, kc, vc, ctx_len, rows, scale)
+    out = out.reshape(B, H, Nv + Nc, D).transpose(0, 2, 1, 3)
+    return np.ascontiguousarray(out[:, :Nv]), np.ascontiguousarray(out[:, Nv:])
+
+
+def adaln_modulate(x, shift, scale, eps: float = 1e-6) -> np.ndarray:
+    """LN(x) * (1 + scale) + shift for x [B, N, C], shift/scale [B, C]."""
+    x = _f64(x)
+    shift = _f64(shift)
+    scale = _f64(scale)
+    B, N, C = x.shape
+    y = np.empty_like(x)
+    _load().oracle_adaln_modulate(_p(x), _p(shift), _p(scale), _p(y), B, N, C, eps)
+    return y
+
+
+def gated_residual(x, branch, gate) -> np.ndarray:
+    """x + gate * branch for x, branch [B, N, C], gate [B, C]."""
+    x = _f64(x)
+    branch = _f64(branch)
+    gate = _f64(gate)
+    B, N, C = x.shape
+    out = np.empty_like(x)
+    _load().oracle_gated_residual(_p(x), _p(branch), _p(gate), _p(out), B, N, C)
+    return out
+
+
+def block(inp: dict, eps: float = 1e-6):
+    """One pass of the whole path on the arrays of ``mmdit_joint_attention_b200.inputs
+    .make_inputs``: modulate both streams, QK-norm (+RoPE on the visual stream),
+    joint attention, and the gated residual with the attention output as the
+    branch (the projections around attention are outside this path).
+
+    Returns a dict with y_vis, y_ctx, q_vis, k_vis, q_ctx, k_ctx (normalised),
+    o_vis, o_ctx, x_vis, x_ctx (after the residual)."""
+    w = inp["workload"]
+    B, Nv, Nc, H, D = w.B, w.Nv, w.Nc, w.H, w.D
+    r = {}
+    for s in ("vis", "ctx"):
+        r["y_" + s] = adaln_modulate(inp["x_" + s].f64, inp["shift_" + s], inp["scale_" + s], eps)
+    r["q_vis"], r["k_vis"] = qk_norm_rope(inp["q_vis"].f64, inp["k_vis"].f64, inp["gq_vis"],
+                                          inp["gk_vis"], grid=w.grid, pos_scale=w.pos_scale,
+                                          eps=eps)
+    r["q_ctx"], r["k_ctx"] = qk_norm_rope(inp["q_ctx"].f64, inp["k_ctx"].f64, inp["gq_ctx"],
+                                          inp["gk_ctx"], grid=None, eps=eps)
+    r["o_vis"], r["o_ctx"] = joint_attention(r["q_vis"], r["k_vis"], inp["v_vis"].f64,
+                                             r["q_ctx"], r["k_ctx"], inp["v_ctx"].f64,
+                                             inp["ctx_len"])
+    r["x_vis"] = gated_residual(inp["x_vis"].f64, r["o_vis"].reshape(B, Nv, H * D), inp["gate_vis"])
+    r["x_ctx"] = gated_residual(inp["x_ctx"].f64, r["o_ctx"].reshape(B, Nc, H * D), inp["gate_ctx"])
+    return r

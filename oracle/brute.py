@@ -1,0 +1,94 @@
+"""Brute-force float64 restatement of the block, for tiny inputs only.
+
+TEST INFRASTRUCTURE ONLY: a second, structurally different formulation used
+to pin the C oracle (``oracle.c``).  It shares no code with it:
+
+  * RoPE is built as an explicit D x D block-diagonal rotation matrix per token
+    (one 2x2 rotation block per pair) and applied as a matrix product;
+  * joint attention physically concatenates [visual ; cond] Q, K, V, forms the
+    whole score matrix with one matrix product, applies an additive -inf key
+    mask, and normalises every row of exp(S - rowmax);
+  * LayerNorm uses numpy's mean / var.
+
+Sources: Vimoo 1.0 research page, section 2.2 (dual-stream joint attention,
+QK-RMSNorm, 3D RoPE 16/56/56, adaLN, gated residual); Wan 2.1 report section
+4.2.1 (raster flatten of the patched latent).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def rotation_matrix(pos_thw, D=128, split=(16, 56, 56), base=10000.0, pos_scale=(1.0, 1.0, 1.0)):
+    """D x D block-diagonal rotation for a token at grid position (t, h, w)."""
+    R = np.zeros((D, D))
+    off = 0
+    for a in range(3):
+        d_a = split[a]
+        p = pos_thw[a] * pos_scale[a]
+        for j in range(d_a // 2):
+            ang = p * base ** (-2.0 * j / d_a)
+            c, s = np.cos(ang), np.sin(ang)
+            i0 = off + 2 * j
+            R[i0:i0 + 2, i0:i0 + 2] = [[c, -s], [s, c]]
+        off += d_a
+    return R
+
+
+def grid_positions(grid):
+    T, Hp, Wp = grid
+    t, h, w = np.meshgrid(np.arange(T), np.arange(Hp), np.arange(Wp), indexing="ij")
+    return np.stack([t.ravel(), h.ravel(), w.ravel()], axis=1)   # [N, 3] raster order
+
+
+def rope3d(x, grid, pos_scale=(1.0, 1.0, 1.0), base=10000.0, split=(16, 56, 56)):
+    x = np.asarray(x, dtype=np.float64)
+    B, N, H, D = x.shape
+    out = np.empty_like(x)
+    for n, pos in enumerate(grid_positions(grid)):
+        R = rotation_matrix(pos, D, split, base, pos_scale)
+        out[:, n] = x[:, n] @ R.T
+    return out
+
+
+def rmsnorm(x, g, eps=1e-6):
+    x = np.asarray(x, dtype=np.float64)
+    norm = np.linalg.norm(x, axis=-1, keepdims=True)
+    D = x.shape[-1]
+    return x * (np.sqrt(D) / np.sqrt(norm ** 2 + D * eps)) * np.asarray(g, dtype=np.float64)
+
+
+def joint_attention(qv, kv, vv, qc, kc, vc, ctx_len=None, scale=None):
+    qv, kv, vv, qc, kc, vc = (np.asarray(a, dtype=np.float64) for a in (qv, kv, vv, qc, kc, vc))
+    B, Nv, H, D = qv.shape
+    Nc = qc.shape[1]
+    if scale is None:
+        scale = D ** -0.5
+    if ctx_len is None:
+        ctx_len = [Nc] * B
+    Q = np.concatenate([qv, qc], axis=1)       # [B, N, H, D]
+    K = np.concatenate([kv, kc], axis=1)
+    V = np.concatenate([vv, vc], axis=1)
+    O = np.zeros_like(Q)
+    for b in range(B):
+        valid = np.concatenate([np.ones(Nv, bool), np.arange(Nc) < ctx_len[b]])
+        bias = np.where(valid, 0.0, -np.inf)
+        for h in range(H):
+            S = Q[b, :, h] @ K[b, :, h].T * scale + bias[None, :]
+            P = np.exp(S - S.max(axis=1, keepdims=True))
+            P /= P.sum(axis=1, keepdims=True)
+            O[b, :, h] = P @ V[b, :, h]
+        O[b, Nv:][~valid[Nv:]] = 0.0
+    return O[:, :Nv], O[:, Nv:]
+
+
+def adaln_modulate(x, shift, scale, eps=1e-6):
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = x.var(axis=-1, keepdims=True)
+    ln = (x - mu) / np.sqrt(var + eps)
+    return ln * (1.0 + np.asarray(scale, np.float64)[:, None, :]) + np.asarray(shift, np.float64)[:, None, :]
+
+
+def gated_residual(x, branch, gate):
+    return np.asarray(x, np.float64) + np.asarray(gate, np.float64)[:, None, :] * np.asarray(branch, np.float64)

@@ -1,0 +1,181 @@
+/*
+ * Float64 CPU oracle for one MMDiT block's joint-attention core.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA library, and the CUDA library never
+ * calls it.
+ *
+ * Every function is the plain definition written out with loops in double
+ * precision, parallelised over independent rows with OpenMP and nothing else
+ * (no blocking, no fusion, no reordering of a row's arithmetic beyond the
+ * definition).  Sources, cited by page title and section:
+ *
+ *   [V]  "Vimoo 1.0: Video Generation for Compact, Lightweight, and High-Speed",
+ *        section 2.2 "Dual-Stream MMDiT Backbone":
+ *          - each stream projects its own Q/K/V; the sequences are concatenated
+ *            for joint attention and the outputs are split back per stream;
+ *          - 3D RoPE over temporal / vertical / horizontal positions, the 128
+ *            head dims split 16 / 56 / 56, applied to the visual Q and K only;
+ *          - Q and K RMS-normalised within each head with distinct learned
+ *            scales;
+ *          - LayerNorm before attention with timestep shift / scale, and gates
+ *            that control each branch's residual contribution.
+ *   [W4] "Wan 2.1" technical report (Chinese translation), section 4.2.1
+ *        (patchify + flatten of the (T, H, W) latent into a token sequence) and
+ *        section 4.3.1 (DiT attention is non-causal).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - RoPE pairs are adjacent (2j, 2j+1) inside each axis chunk, chunk order
+ *     T, H, W; frequency of pair j on an axis of width d is base^(-2j/d);
+ *     rotation (x, y) -> (x cos a - y sin a, x sin a + y cos a).
+ *   - token n of the visual stream sits at t = n / (Hp*Wp), h = (n / Wp) % Hp,
+ *     w = n % Wp (raster flatten); the rotation angle uses pos * pos_scale.
+ *   - joint key order is [visual ; conditioning]; cond keys at index
+ *     >= ctx_len[b] are excluded; cond query rows >= ctx_len[b] output zero.
+ *   - LayerNorm has no affine, biased variance; modulate is
+ *     LN(x) * (1 + scale) + shift.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "oracle.h"
+
+/* ---- QK-RMSNorm [V] -------------------------------------------------------
+ * For each row r of D values: y = x / sqrt(mean(x^2) + eps) * g.             */
+void oracle_rmsnorm(const double* x, double* y, const double* g,
+                    long rows, int D, double eps)
+{
+    #pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        const double* xr = x + r * (long)D;
+        double* yr = y + r * (long)D;
+        double ss = 0.0;
+        for (int d = 0; d < D; ++d) ss += xr[d] * xr[d];
+        double rms = sqrt(ss / (double)D + eps);
+        for (int d = 0; d < D; ++d) yr[d] = xr[d] / rms * g[d];
+    }
+}
+
+/* ---- 3D RoPE [V], flatten order [W4] ---------------------------------------
+ * x: [B, N, H, D] visual rows, rotated in place.  N must equal T*Hp*Wp.      */
+void oracle_rope3d(double* x, int B, int N, int H, int D, const oracle_grid* grid)
+{
+    const int HW = grid->H * grid->W;
+    #pragma omp parallel for schedule(static)
+    for (long bn = 0; bn < (long)B * N; ++bn) {
+        int n = (int)(bn % N);
+        int pos[3];
+        pos[0] = n / HW;                 /* t */
+        pos[1] = (n / grid->W) % grid->H; /* h */
+        pos[2] = n % grid->W;            /* w */
+        for (int hd = 0; hd < H; ++hd) {
+            double* row = x + (bn * H + hd) * (long)D;
+            int offset = 0;
+            for (int a = 0; a < 3; ++a) {
+                int d_a = grid->split[a];
+                double p = (double)pos[a] * grid->pos_scale[a];
+                for (int j = 0; j < d_a / 2; ++j) {
+                    double freq = pow(grid->rope_base, -2.0 * (double)j / (double)d_a);
+                    double ang = p * freq;
+                    double c = cos(ang), s = sin(ang);
+                    double u = row[offset + 2 * j];
+                    double v = row[offset + 2 * j + 1];
+                    row[offset + 2 * j]     = u * c - v * s;
+                    row[offset + 2 * j + 1] = u * s + v * c;
+                }
+                offset += d_a;
+            }
+        }
+    }
+}
+
+/* ---- joint attention [V], non-causal [W4] ----------------------------------
+ * Per (b, h): Q = [Qv; Qc], K = [Kv; Kc], V = [Vv; Vc] (joint index i < Nv is
+ * visual row i, otherwise cond row i - Nv).  For each requested query row:
+ *   s_j = q . k_j * scale over valid keys j, m = max s_j, p_j = exp(s_j - m),
+ *   o = sum_j p_j v_j / sum_j p_j.
+ * Requested rows are triplets (b, h, i); out is [nrows, D].                   */
+void oracle_joint_attention_rows(const double* qv, const double* kv, const double* vv,
+                                 const double* qc, const double* kc, const double* vc,
+                                 const int* ctx_len, int B, int Nv, int Nc, int H, int D,
+                                 double scale, const long* rows, long nrows, double* out)
+{
+    (void)B;
+    #pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)(Nv + Nc + 1));
+        #pragma omp for schedule(dynamic, 4)
+        for (long r = 0; r < nrows; ++r) {
+            long b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+            int L = ctx_len ? ctx_len[b] : Nc;
+            double* o = out + r * (long)D;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            const double* q;
+            if (i < Nv) {
+                q = qv + ((b * Nv + i) * H + h) * (long)D;
+            } else {
+                if (i - Nv >= L) continue;        /* padded cond query: zero */
+                q = qc + ((b * Nc + (i - Nv)) * H + h) * (long)D;
+            }
+            int nk = Nv + L;
+            double m = -INFINITY;
+            for (int j = 0; j < nk; ++j) {
+                const double* k = (j < Nv) ? kv + ((b * Nv + j) * H + h) * (long)D
+                                           : kc + ((b * Nc + (j - Nv)) * H + h) * (long)D;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += q[d] * k[d];
+                s[j] = acc * scale;
+                if (s[j] > m) m = s[j];
+            }
+            if (nk == 0) continue;
+            double den = 0.0;
+            for (int j = 0; j < nk; ++j) {
+                double p = exp(s[j] - m);
+                den += p;
+                const double* v = (j < Nv) ? vv + ((b * Nv + j) * H + h) * (long)D
+                                           : vc + ((b * Nc + (j - Nv)) * H + h) * (long)D;
+                for (int d = 0; d < D; ++d) o[d] += p * v[d];
+            }
+            for (int d = 0; d < D; ++d) o[d] /= den;
+        }
+        free(s);
+    }
+}
+
+/* ---- adaLN modulate [V] ------------------------------------------------------
+ * Per row of C values of sample b: mu = mean, var = mean((x - mu)^2),
+ * y = (x - mu) / sqrt(var + eps) * (1 + scale[b, c]) + shift[b, c].          */
+void oracle_adaln_modulate(const double* x, const double* shift, const double* scale,
+                           double* y, int B, int N, int C, double eps)
+{
+    #pragma omp parallel for schedule(static)
+    for (long bn = 0; bn < (long)B * N; ++bn) {
+        long b = bn / N;
+        const double* xr = x + bn * (long)C;
+        double* yr = y + bn * (long)C;
+        double mu = 0.0;
+        for (int c = 0; c < C; ++c) mu += xr[c];
+        mu /= (double)C;
+        double var = 0.0;
+        for (int c = 0; c < C; ++c) var += (xr[c] - mu) * (xr[c] - mu);
+        var /= (double)C;
+        double rstd = 1.0 / sqrt(var + eps);
+        for (int c = 0; c < C; ++c)
+            yr[c] = (xr[c] - mu) * rstd * (1.0 + scale[b * C + c]) + shift[b * C + c];
+    }
+}
+
+/* ---- gated residual [V] -------------------------------------------------------
+ * out[b, n, c] = x[b, n, c] + gate[b, c] * branch[b, n, c].                   */
+void oracle_gated_residual(const double* x, const double* branch, const double* gate,
+                           double* out, int B, int N, int C)
+{
+    #pragma omp parallel for schedule(static)
+    for (long bn = 0; bn < (long)B * N; ++bn) {
+        long b = bn / N;
+        for (int c = 0; c < C; ++c)
+            out[bn * C + c] = x[bn * C + c] + gate[b * C + c] * branch[bn * C + c];
+    }
+}

@@ -1,0 +1,25 @@
+/* Float64 CPU oracle (test infrastructure only): declarations.
+ * Argument meaning mirrors the CUDA library's entry points, but every array is
+ * a host float64 array and every result is written to a separate output. */
+#ifndef MMDIT_ORACLE_H
+#define MMDIT_ORACLE_H
+
+typedef struct {
+    int T, H, W;            /* visual token grid */
+    double pos_scale[3];    /* per-axis position multiplier (T, H, W) */
+    double rope_base;       /* RoPE frequency base */
+    int split[3];           /* head dims per axis; sums to D */
+} oracle_grid;
+
+void oracle_rmsnorm(const double* x, double* y, const double* g, long rows, int D, double eps);
+void oracle_rope3d(double* x, int B, int N, int H, int D, const oracle_grid* grid);
+void oracle_joint_attention_rows(const double* qv, const double* kv, const double* vv,
+                                 const double* qc, const double* kc, const double* vc,
+                                 const int* ctx_len, int B, int Nv, int Nc, int H, int D,
+                                 double scale, const long* rows, long nrows, double* out);
+void oracle_adaln_modulate(const double* x, const double* shift, const double* scale,
+                           double* y, int B, int N, int C, double eps);
+void oracle_gated_residual(const double* x, const double* branch, const double* gate,
+                           double* out, int B, int N, int C);
+
+#endif

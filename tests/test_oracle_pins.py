@@ -1,0 +1,454 @@
+"""Pins for the float64 oracle, independent of the oracle itself.
+
+Each pin checks the oracle against something the pages or mathematics fix:
+a brute-force restatement with explicit rotation matrices and physically
+concatenated sequences (oracle/brute.py), a library routine in a special case
+the definition reduces to (torch float64 scaled_dot_product_attention and
+layer_norm), closed forms (tests/golden/rope_closed_form.json) and invariants
+(RoPE preserves norms and is relative; softmax rows sum to one; identical keys
+give mean(V); masked keys have no influence; constant-scale RMSNorm has RMS
+equal to the scale).  Sources: Vimoo 1.0 research page, section 2.2; Wan 2.1
+report sections 4.2.1 and 4.3.1.
+
+``test_mutants_are_caught`` plants plausible mistakes in copies of the
+oracle's C source and checks that at least one pin fails for each.
+"""
+import ctypes
+import json
+import math
+import os
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import brute
+from mmdit_joint_attention_b200 import inputs as I
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = lambda s: np.random.Generator(np.random.PCG64(s))  # noqa: E731
+
+PINS = {}
+
+
+def pin(f):
+    PINS[f.__name__] = f
+    return f
+
+
+def _close(a, b, tol=1e-12):
+    a, b = np.asarray(a), np.asarray(b)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    assert err <= tol, f"max abs err {err} > {tol}"
+
+
+# --------------------------------------------------------------------- RMSNorm
+
+@pin
+def pin_rmsnorm_constant_scale_rms():
+    """A constant scale g*1 gives output RMS g * sqrt(ms / (ms + eps))."""
+    x = RNG(1).standard_normal((3, 7, 2, 128))
+    for g, eps in ((0.7, 1e-6), (1.3, 0.0), (2.0, 0.5)):
+        y = oracle.rmsnorm(x, np.full(128, g), eps)
+        ms = np.mean(x * x, axis=-1)
+        _close(np.sqrt(np.mean(y * y, axis=-1)), g * np.sqrt(ms / (ms + eps)))
+
+
+@pin
+def pin_rmsnorm_closed_form():
+    """x = a*1 -> y = a / sqrt(a^2 + eps) * g, element by element."""
+    g = RNG(2).uniform(0.5, 1.5, 128)
+    for a in (1.0, -3.0, 0.25):
+        y = oracle.rmsnorm(np.full((1, 128), a), g, 1e-6)
+        _close(y[0], a / math.sqrt(a * a + 1e-6) * g)
+
+
+@pin
+def pin_rmsnorm_per_dim_scale_and_homogeneity():
+    """With eps = 0: y(x; g) = y(x; 1) * g per dim, and y(c x) = y(x) for c > 0."""
+    r = RNG(3)
+    x = r.standard_normal((5, 128))
+    g = r.uniform(0.5, 1.5, 128)
+    y1 = oracle.rmsnorm(x, np.ones(128), 0.0)
+    _close(oracle.rmsnorm(x, g, 0.0), y1 * g)
+    _close(oracle.rmsnorm(3.5 * x, np.ones(128), 0.0), y1)
+
+
+@pin
+def pin_rmsnorm_brute():
+    r = RNG(4)
+    x = r.standard_normal((2, 9, 3, 128))
+    g = r.uniform(0.5, 1.5, 128)
+    _close(oracle.rmsnorm(x, g, 1e-6), brute.rmsnorm(x, g, 1e-6))
+
+
+# ------------------------------------------------------------------------ RoPE
+
+GRID = (4, 5, 6)
+
+
+def _unit_rows(grid, D=128, H=1, seed=5):
+    N = grid[0] * grid[1] * grid[2]
+    return RNG(seed).standard_normal((2, N, H, D))
+
+
+@pin
+def pin_rope_norm_preserved():
+    """A rotation keeps the norm of every head vector and of every pair."""
+    x = _unit_rows(GRID, H=2)
+    y = oracle.rope3d(x, GRID, pos_scale=(1.0, 0.5, 2.0))
+    _close(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), 1e-11)
+    xp = x.reshape(*x.shape[:-1], 64, 2)
+    yp = y.reshape(*y.shape[:-1], 64, 2)
+    _close(np.linalg.norm(yp, axis=-1), np.linalg.norm(xp, axis=-1), 1e-11)
+
+
+@pin
+def pin_rope_identity_at_origin():
+    x = _unit_rows(GRID)
+    y = oracle.rope3d(x, GRID)
+    _close(y[:, 0], x[:, 0], 0.0)
+
+
+@pin
+def pin_rope_relative_position():
+    """<R(p1) q, R(p2) k> depends only on p1 - p2: shifting both tokens by the
+    same grid offset leaves every score unchanged."""
+    T, Hp, Wp = GRID
+    r = RNG(6)
+    q = r.standard_normal(128)
+    k = r.standard_normal(128)
+    N = T * Hp * Wp
+    xq = np.broadcast_to(q, (1, N, 1, 128)).copy()
+    xk = np.broadcast_to(k, (1, N, 1, 128)).copy()
+    rq = oracle.rope3d(xq, GRID, pos_scale=(1.0, 0.75, 1.25))[0, :, 0]
+    rk = oracle.rope3d(xk, GRID, pos_scale=(1.0, 0.75, 1.25))[0, :, 0]
+    idx = lambda t, h, w: (t * Hp + h) * Wp + w  # noqa: E731
+    pairs = [((0, 0, 0), (1, 2, 3)), ((2, 1, 0), (0, 4, 5)), ((1, 3, 2), (1, 0, 4))]
+    for p1, p2 in pairs:
+        base_score = rq[idx(*p1)] @ rk[idx(*p2)]
+        for d in ((1, 0, 0), (0, 1, 0), (0, 0, 1), (1, 1, 0)):
+            s1 = tuple(a + b for a, b in zip(p1, d))
+            s2 = tuple(a + b for a, b in zip(p2, d))
+            if all(s1[i] < GRID[i] and s2[i] < GRID[i] for i in range(3)):
+                assert abs(rq[idx(*s1)] @ rk[idx(*s2)] - base_score) < 1e-10
+
+
+@pin
+def pin_rope_axis_chunks():
+    """Moving along one axis only changes that axis's chunk of dims:
+    T -> [0, 16), H -> [16, 72), W -> [72, 128)."""
+    T, Hp, Wp = GRID
+    x = _unit_rows(GRID)
+    y = oracle.rope3d(x, GRID)
+    idx = lambda t, h, w: (t * Hp + h) * Wp + w  # noqa: E731
+    chunks = {0: (0, 16), 1: (16, 72), 2: (72, 128)}
+    for axis, pos in ((0, (2, 0, 0)), (1, (0, 3, 0)), (2, (0, 0, 4))):
+        n = idx(*pos)
+        lo, hi = chunks[axis]
+        changed = np.any(np.abs(y[:, n, 0] - x[:, n, 0]) > 0, axis=0)
+        assert changed[lo:hi].sum() >= (hi - lo) - 2
+        assert not changed[:lo].any() and not changed[hi:].any()
+
+
+def _eval(expr):
+    return eval(expr, {"cos": math.cos, "sin": math.sin})
+
+
+@pin
+def pin_rope_golden_closed_form():
+    with open(os.path.join(GOLDEN, "rope_closed_form.json")) as f:
+        gold = json.load(f)
+    grid = tuple(gold["grid"])
+    T, Hp, Wp = grid
+    N = T * Hp * Wp
+    for block, scale in ((gold["cases"], (1.0, 1.0, 1.0)),
+                         (gold["scaled"]["cases"], tuple(gold["scaled"]["pos_scale"]))):
+        for c in block:
+            x = np.zeros((1, N, 1, 128))
+            n = (c["pos"][0] * Hp + c["pos"][1]) * Wp + c["pos"][2]
+            x[0, n, 0, c["in_dim"]] = 1.0
+            y = oracle.rope3d(x, grid, pos_scale=scale)[0, n, 0]
+            want = [_eval(e) for e in c["expect"]]
+            _close(y[c["out_dims"]], want, 1e-13)
+            rest = np.delete(y, c["out_dims"])
+            _close(rest, np.zeros_like(rest), 0.0)
+
+
+@pin
+def pin_rope_brute():
+    x = _unit_rows((2, 3, 4), H=2)
+    for ps in ((1.0, 1.0, 1.0), (1.0, 1 / 1.5, 1 / 1.5)):
+        _close(oracle.rope3d(x, (2, 3, 4), pos_scale=ps), brute.rope3d(x, (2, 3, 4), pos_scale=ps),
+               1e-12)
+
+
+# ------------------------------------------------------------------- attention
+
+def _qkv(B, Nv, Nc, H, seed, D=128):
+    r = RNG(seed)
+    return [r.standard_normal((B, n, H, D)) for n in (Nv, Nv, Nv, Nc, Nc, Nc)]
+
+
+def _sdpa(Q, K, V, mask=None):
+    """torch float64 SDPA on [B, N, H, D] tensors (heads moved to dim 1)."""
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).permute(0, 2, 1, 3)  # noqa: E731
+    o = torch.nn.functional.scaled_dot_product_attention(t(Q), t(K), t(V), attn_mask=mask)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+@pin
+def pin_attention_brute():
+    for (B, Nv, Nc, H, cl) in ((1, 32, 8, 2, None), (2, 20, 9, 3, [0, 5]), (2, 17, 6, 1, [6, 1])):
+        a = _qkv(B, Nv, Nc, H, seed=7 + B + Nv)
+        ov, oc = oracle.joint_attention(*a, ctx_len=cl)
+        bv, bc = brute.joint_attention(*a, ctx_len=cl)
+        _close(ov, bv, 1e-12)
+        _close(oc, bc, 1e-12)
+
+
+@pin
+def pin_attention_sdpa_on_concatenation():
+    """With every cond token valid, joint attention is plain attention over
+    the physically concatenated sequence (torch float64 SDPA, scale 1/sqrt(D))."""
+    qv, kv, vv, qc, kc, vc = _qkv(2, 24, 10, 3, seed=11)
+    ov, oc = oracle.joint_attention(qv, kv, vv, qc, kc, vc)
+    o = _sdpa(*(np.concatenate(p, axis=1) for p in ((qv, qc), (kv, kc), (vv, vc))))
+    _close(np.concatenate([ov, oc], axis=1), o, 1e-12)
+
+
+@pin
+def pin_attention_sdpa_key_padding():
+    """Ragged cond lengths equal SDPA with a boolean key mask, per sample."""
+    B, Nv, Nc, H = 2, 16, 12, 2
+    a = _qkv(B, Nv, Nc, H, seed=12)
+    cl = [3, 12]
+    ov, oc = oracle.joint_attention(*a, ctx_len=cl)
+    for b in range(B):
+        Q, K, V = (np.concatenate([a[i][b:b + 1], a[i + 3][b:b + 1]], axis=1) for i in range(3))
+        keep = torch.tensor(np.concatenate([np.ones(Nv, bool), np.arange(Nc) < cl[b]]))
+        o = _sdpa(Q, K, V, mask=keep[None, None, None, :])
+        _close(ov[b], o[0, :Nv], 1e-12)
+        _close(oc[b, :cl[b]], o[0, Nv:Nv + cl[b]], 1e-12)
+        _close(oc[b, cl[b]:], np.zeros_like(oc[b, cl[b]:]), 0.0)
+
+
+@pin
+def pin_attention_self_when_no_cond():
+    """Nc = 0 reduces joint attention to self-attention over the visual stream."""
+    qv, kv, vv = _qkv(1, 30, 0, 2, seed=13)[:3]
+    empty = np.zeros((1, 0, 2, 128))
+    ov, oc = oracle.joint_attention(qv, kv, vv, empty, empty, empty)
+    _close(ov, _sdpa(qv, kv, vv), 1e-12)
+    assert oc.shape == (1, 0, 2, 128)
+
+
+@pin
+def pin_attention_rows_sum_to_one():
+    """V = 1 for every key: each valid output row is exactly the weight sum, 1."""
+    qv, kv, vv, qc, kc, vc = _qkv(2, 19, 7, 2, seed=14)
+    ov, oc = oracle.joint_attention(qv, kv, np.ones_like(vv), qc, kc, np.ones_like(vc),
+                                    ctx_len=[7, 2])
+    _close(ov, np.ones_like(ov), 1e-13)
+    _close(oc[0], np.ones_like(oc[0]), 1e-13)
+    _close(oc[1, :2], np.ones_like(oc[1, :2]), 1e-13)
+
+
+@pin
+def pin_attention_identical_keys_mean_v():
+    """All keys equal -> uniform weights -> output = mean of the valid V rows."""
+    B, Nv, Nc, H = 2, 13, 6, 2
+    qv, kv, vv, qc, kc, vc = _qkv(B, Nv, Nc, H, seed=15)
+    kvec = RNG(16).standard_normal((1, 1, H, 128))
+    kv = np.broadcast_to(kvec, kv.shape).copy()
+    kc = np.broadcast_to(kvec, kc.shape).copy()
+    cl = [6, 4]
+    ov, oc = oracle.joint_attention(qv, kv, vv, qc, kc, vc, ctx_len=cl)
+    for b in range(B):
+        m = np.concatenate([vv[b], vc[b, :cl[b]]], axis=0).mean(axis=0)  # [H, D]
+        _close(ov[b], np.broadcast_to(m, ov[b].shape), 1e-12)
+        _close(oc[b, :cl[b]], np.broadcast_to(m, oc[b, :cl[b]].shape), 1e-12)
+
+
+@pin
+def pin_attention_mask_no_influence():
+    """Changing padded cond keys / values leaves every output bit-identical."""
+    B, Nv, Nc, H = 2, 11, 9, 2
+    a = _qkv(B, Nv, Nc, H, seed=17)
+    cl = [4, 0]
+    ov, oc = oracle.joint_attention(*a, ctx_len=cl)
+    a2 = [x.copy() for x in a]
+    for b in range(B):
+        a2[4][b, cl[b]:] = 1e3 * RNG(18).standard_normal(a2[4][b, cl[b]:].shape)
+        a2[5][b, cl[b]:] = -7.0
+    ov2, oc2 = oracle.joint_attention(*a2, ctx_len=cl)
+    assert np.array_equal(ov, ov2) and np.array_equal(oc, oc2)
+
+
+@pin
+def pin_attention_two_keys_closed_form():
+    """One query, two keys: o = (e^s1 v1 + e^s2 v2) / (e^s1 + e^s2), s = q.k / sqrt(128)."""
+    r = RNG(19)
+    q = r.standard_normal((1, 1, 1, 128))
+    k1, k2 = r.standard_normal((2, 128))
+    v1, v2 = r.standard_normal((2, 128))
+    kv = k1.reshape(1, 1, 1, 128)
+    vv = v1.reshape(1, 1, 1, 128)
+    kc = k2.reshape(1, 1, 1, 128)
+    vc = v2.reshape(1, 1, 1, 128)
+    ov, _ = oracle.joint_attention(q, kv, vv, q, kc, vc)
+    s1 = float(q.ravel() @ k1) / math.sqrt(128)
+    s2 = float(q.ravel() @ k2) / math.sqrt(128)
+    want = (math.exp(s1) * v1 + math.exp(s2) * v2) / (math.exp(s1) + math.exp(s2))
+    _close(ov[0, 0, 0], want, 1e-13)
+
+
+@pin
+def pin_attention_large_scores_stable():
+    """Scores in the thousands (the softmax is shift-invariant, so the exact
+    result is well defined) must come out finite and equal brute force,
+    which subtracts the row maximum."""
+    a = _qkv(1, 12, 5, 2, seed=25)
+    a[0] = a[0] * 1000.0
+    a[3] = a[3] * 1000.0
+    ov, oc = oracle.joint_attention(*a)
+    bv, bc = brute.joint_attention(*a)
+    assert np.all(np.isfinite(ov)) and np.all(np.isfinite(oc))
+    _close(ov, bv, 1e-9)
+    _close(oc, bc, 1e-9)
+
+
+@pin
+def pin_attention_rows_subset_matches_full():
+    """The row-subset entry point returns the same rows as the full call."""
+    w = I.Workload("t", "f32", B=2, H=2, grid=(2, 3, 5), Nc=9, ctx_len=(9, 3))
+    a = _qkv(2, w.Nv, w.Nc, 2, seed=20)
+    ov, oc = oracle.joint_attention(*a, ctx_len=w.ctx_lengths())
+    full = np.concatenate([ov, oc], axis=1)
+    for b in range(2):
+        for h in range(2):
+            rows = I.parity_rows(w, b, h, n_random=8)
+            trip = np.stack([np.full_like(rows, b), np.full_like(rows, h), rows], axis=1)
+            got = oracle.joint_attention_rows(*a, w.ctx_lengths(), trip)
+            _close(got, full[b, rows, h], 0.0)
+
+
+# ------------------------------------------------------------- adaLN / residual
+
+@pin
+def pin_modulate_zero_is_layer_norm():
+    """scale = shift = 0 leaves plain LayerNorm (torch float64 layer_norm)."""
+    x = RNG(21).standard_normal((2, 7, 3072)) * 3.0 + 1.5
+    z = np.zeros((2, 3072))
+    y = oracle.adaln_modulate(x, z, z, 1e-6)
+    ln = torch.nn.functional.layer_norm(torch.from_numpy(x), (3072,), eps=1e-6).numpy()
+    _close(y, ln, 1e-12)
+    _close(y.mean(axis=-1), np.zeros((2, 7)), 1e-12)
+
+
+@pin
+def pin_modulate_closed_form():
+    """Row (a, -a, a, -a, ...) + m: mean m, variance a^2, so
+    y = +-a / sqrt(a^2 + eps) * (1 + scale) + shift."""
+    C = 3072
+    a, m, eps = 2.0, 0.75, 1e-6
+    x = (np.where(np.arange(C) % 2 == 0, a, -a) + m).reshape(1, 1, C)
+    r = RNG(22)
+    shift = r.standard_normal((1, C)) * 0.1
+    scale = r.standard_normal((1, C)) * 0.1
+    sign = np.where(np.arange(C) % 2 == 0, 1.0, -1.0)
+    want = sign * a / math.sqrt(a * a + eps) * (1 + scale[0]) + shift[0]
+    _close(oracle.adaln_modulate(x, shift, scale, eps)[0, 0], want, 1e-12)
+
+
+@pin
+def pin_modulate_brute():
+    r = RNG(23)
+    x = r.standard_normal((2, 5, 256))
+    shift = r.standard_normal((2, 256)) * 0.1
+    scale = r.standard_normal((2, 256)) * 0.1
+    _close(oracle.adaln_modulate(x, shift, scale), brute.adaln_modulate(x, shift, scale), 1e-12)
+
+
+@pin
+def pin_residual_special_gates():
+    r = RNG(24)
+    x = r.standard_normal((2, 5, 64))
+    br = r.standard_normal((2, 5, 64))
+    _close(oracle.gated_residual(x, br, np.zeros((2, 64))), x, 0.0)
+    _close(oracle.gated_residual(x, br, np.ones((2, 64))), x + br, 0.0)
+    g = r.standard_normal((2, 64))
+    _close(oracle.gated_residual(x, x, g), x * (1.0 + g[:, None, :]), 1e-14)
+    g2 = np.zeros((2, 64))
+    g2[1] = 1.0
+    out = oracle.gated_residual(x, br, g2)
+    _close(out[0], x[0], 0.0)
+    _close(out[1], x[1] + br[1], 0.0)
+
+
+@pin
+def pin_block_brute():
+    """The composed block equals the brute-force composition on the tiny workload."""
+    w = I.WORKLOADS["tiny"]
+    inp = I.make_inputs(w, seed=0)
+    r = oracle.block(inp)
+    qv, kv = brute.rmsnorm(inp["q_vis"].f64, inp["gq_vis"]), brute.rmsnorm(inp["k_vis"].f64, inp["gk_vis"])
+    qv, kv = brute.rope3d(qv, w.grid), brute.rope3d(kv, w.grid)
+    qc, kc = brute.rmsnorm(inp["q_ctx"].f64, inp["gq_ctx"]), brute.rmsnorm(inp["k_ctx"].f64, inp["gk_ctx"])
+    ov, oc = brute.joint_attention(qv, kv, inp["v_vis"].f64, qc, kc, inp["v_ctx"].f64)
+    _close(r["o_vis"], ov, 1e-12)
+    _close(r["o_ctx"], oc, 1e-12)
+    _close(r["x_vis"], brute.gated_residual(inp["x_vis"].f64, ov.reshape(1, w.Nv, w.C), inp["gate_vis"]), 1e-12)
+    _close(r["y_ctx"], brute.adaln_modulate(inp["x_ctx"].f64, inp["shift_ctx"], inp["scale_ctx"]), 1e-12)
+
+
+@pytest.mark.parametrize("name", sorted(PINS))
+def test_pin(name):
+    PINS[name]()
+
+
+# --------------------------------------------------------------- mutation check
+
+MUTANTS = {
+    "rope_sign": ("row[offset + 2 * j]     = u * c - v * s;", "row[offset + 2 * j]     = u * c + v * s;"),
+    "rope_freq": ("-2.0 * (double)j / (double)d_a", "-1.0 * (double)j / (double)d_a"),
+    "rope_axis_order": ("pos[0] = n / HW;", "pos[0] = n % grid->W;"),
+    "rope_pairing": ("double v = row[offset + 2 * j + 1];", "double v = row[offset + j + d_a / 2];"),
+    "rms_missing_mean": ("sqrt(ss / (double)D + eps)", "sqrt(ss + eps)"),
+    "rms_scale_reversed": ("yr[d] = xr[d] / rms * g[d];", "yr[d] = xr[d] / rms * g[D - 1 - d];"),
+    "attn_no_scale": ("s[j] = acc * scale;", "s[j] = acc;"),
+    "attn_mask_off_by_one": ("int nk = Nv + L;", "int nk = Nv + L + (L < Nc ? 1 : 0);"),
+    "attn_padded_rows_not_zero": ("if (i - Nv >= L) continue;", "if (i - Nv >= Nc) continue;"),
+    "attn_no_max_sub": ("double p = exp(s[j] - m);", "double p = exp(s[j] - 0.5 * m);"),
+    "ln_unbiased_var": ("var /= (double)C;", "var /= (double)(C - 1);"),
+    "ln_missing_one_plus": ("* (1.0 + scale[b * C + c])", "* (scale[b * C + c])"),
+    "residual_gate_index": ("gate[b * C + c] * branch", "gate[c] * branch"),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_mutants_are_caught(mutant, tmp_path):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "oracle.c")).read()
+    old, new = MUTANTS[mutant]
+    assert src.count(old) == 1, f"mutation anchor not found: {old}"
+    (tmp_path / "oracle.c").write_text(src.replace(old, new))
+    hdr = os.path.join(os.path.dirname(oracle.__file__), "oracle.h")
+    (tmp_path / "oracle.h").write_text(open(hdr).read())
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-std=c99", "-O2", "-fopenmp", "-shared", "-fPIC", "-o", str(so),
+                           str(tmp_path / "oracle.c"), "-lm"])
+    saved = oracle._load()
+    oracle._lib = oracle._configure(ctypes.CDLL(str(so)))
+    failed = []
+    try:
+        for name, f in PINS.items():
+            try:
+                f()
+            except AssertionError:
+                failed.append(name)
+    finally:
+        oracle._lib = saved
+    assert failed, f"mutant {mutant} passed every pin"
