@@ -1,0 +1,143 @@
+/*
+ * mmdit.h — C ABI of libmmdit.so: one dual-stream MMDiT block's joint-attention
+ * core on NVIDIA B200 (sm_100a).
+ *
+ * What the block computes is stated in "Vimoo 1.0: Video Generation for
+ * Compact, Lightweight, and High-Speed", section 2.2 "Dual-Stream MMDiT
+ * Backbone" (cited below as [Vimoo §2.2]); the token order of the visual
+ * stream follows the patchify-and-flatten step of the Wan 2.1 report, section
+ * 4.2.1, and the attention is non-causal (Wan 2.1 report, section 4.3.1).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers to contiguous row-major arrays,
+ *     16-byte aligned.  The caller owns all memory; the library allocates no
+ *     device memory and keeps no state between calls.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on it; the return value reports
+ *     argument validation and launch errors only.  A kernel that gives up on a
+ *     bounded device-side wait records MMDIT_ERR_TIMEOUT in a device status
+ *     word, read back (and cleared) by mmdit_device_status().
+ *   - Element type of q/k/v/x/branch/outputs is given by `dt`; every scale,
+ *     shift, gate and RMSNorm weight is fp32.  Arithmetic is fp32 (tensor-core
+ *     products of bf16 operands accumulate in fp32).
+ *   - Head dim D must be 128.  Tokens are laid out [B, N, H, D] for q/k/v/o
+ *     and [B, N, C] with C = H*D for x/branch/y.
+ *   - On any error nothing is enqueued and no output is touched.
+ */
+#ifndef MMDIT_H
+#define MMDIT_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MMDIT_API __attribute__((visibility("default")))
+#else
+#define MMDIT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MMDIT_F32 = 0, MMDIT_BF16 = 1 } mmdit_dtype;
+
+enum {
+    MMDIT_OK = 0,
+    MMDIT_ERR_ARG = -1,          /* null pointer, negative size, bad dtype/eps/scale */
+    MMDIT_ERR_SHAPE = -2,        /* sizes inconsistent (e.g. N != T*H*W, split sum != D) */
+    MMDIT_ERR_ALIGN = -3,        /* a pointer is not 16-byte aligned */
+    MMDIT_ERR_UNSUPPORTED = -4,  /* valid but not implemented (D != 128, C % 8 != 0, ...) */
+    MMDIT_ERR_CUDA = -5,         /* a CUDA runtime / driver call failed */
+    MMDIT_ERR_TIMEOUT = -6       /* a device-side bounded wait expired */
+};
+
+/* Visual token grid and RoPE parameters [Vimoo §2.2]: the visual stream holds
+ * T*H*W tokens in raster order n = (t*H + h)*W + w.  Axis a in (T, H, W) owns
+ * split[a] consecutive head dims (16, 56, 56 in the paper), pair j of that
+ * chunk (dims 2j, 2j+1) turns by pos_a * pos_scale[a] * rope_base^(-2j/split[a]).
+ * pos_scale is a per-axis position multiplier (1 = integer grid positions). */
+typedef struct {
+    int T, H, W;
+    float pos_scale[3];
+    float rope_base;
+    int split[3];
+} mmdit_grid;
+
+/* QK-RMSNorm, then 3D RoPE [Vimoo §2.2: Q and K are RMS-normalised per head,
+ * Q and K each with its own learned scale; the rotary embedding touches the
+ * visual stream's Q and K and leaves the conditioning stream unrotated].
+ *
+ * For every (b, n, h) row of D values of q_in and of k_in:
+ *   y = x / sqrt(mean(x^2) + eps) * scale[d]   (q_scale for q, k_scale for k)
+ * and, when grid != NULL, y is then rotated by the RoPE of token n's (t, h, w).
+ * grid == NULL is the conditioning stream (no rotation).
+ *   q_in, k_in   [B, N, H, D] dt, read
+ *   q_out, k_out [B, N, H, D] dt, written; may equal q_in / k_in (in place)
+ *   q_scale, k_scale  [D] fp32
+ *   grid: host pointer, read during the call only; requires N == T*H*W,
+ *         split[] even and summing to D, positions (T-1,H-1,W-1) * pos_scale
+ *         finite.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                       const float* q_scale, const float* k_scale,
+                       int B, int N, int H, int D, const mmdit_grid* grid, float eps,
+                       mmdit_dtype dt, void* stream);
+
+/* Joint non-causal attention over the concatenated streams, output split back
+ * [Vimoo §2.2: each stream projects its own Q/K/V, one attention runs over the
+ * two sequences joined end to end, and its output rows return to the stream
+ * they came from].
+ *
+ * Per (b, h), with joint sequences Q = [q_vis; q_ctx], K = [k_vis; k_ctx],
+ * V = [v_vis; v_ctx] (visual first; never materialised) and key j valid when
+ * j < Nv or j - Nv < ctx_len[b]:
+ *   O_i = sum_j softmax_j(Q_i . K_j * softmax_scale) V_j   over valid keys j,
+ * rows i < Nv written to o_vis, the rest to o_ctx.  Cond query rows at index
+ * >= ctx_len[b] (padding) are written as zeros.  A row with no valid key is 0.
+ *   q_vis, k_vis, v_vis  [B, Nv, H, D] dt      q_ctx, k_ctx, v_ctx [B, Nc, H, D] dt
+ *   ctx_len  DEVICE int32 [B], each clamped to [0, Nc]; NULL = all Nc valid
+ *   o_vis [B, Nv, H, D] dt, o_ctx [B, Nc, H, D] dt  (written; must not alias inputs)
+ *   softmax_scale > 0 (1/sqrt(D) in the usual form)
+ * bf16 runs on the tcgen05 tensor cores (fp32 accumulation in tensor memory);
+ * f32 runs an fp32 CUDA-core kernel.  Nv or Nc may be 0 (the ctx pointers may
+ * then be NULL).
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vis,
+                          const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                          const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                          int B, int Nv, int Nc, int H, int D, float softmax_scale,
+                          mmdit_dtype dt, void* stream);
+
+/* adaLN modulate [Vimoo §2.2: a LayerNorm sits before attention and the FFN,
+ * and the timestep embedding supplies a shift and a scale for its output]:
+ *   y = LN(x) * (1 + scale[b]) + shift[b], LN over C without an affine,
+ *   biased variance.
+ *   x [B, N, C] dt read;  y [B, N, C] dt written (may equal x)
+ *   shift, scale [B, C] fp32;  C % 8 == 0 and C <= 4096 (bf16) / 2048 (f32)
+ * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_adaln_modulate(const void* x, const float* shift, const float* scale, void* y,
+                         int B, int N, int C, float eps, mmdit_dtype dt, void* stream);
+
+/* Gated residual [Vimoo §2.2: a per-channel gate from the timestep embedding
+ * weighs each branch before it is added back to the residual stream]:
+ *   out = x + gate[b] * branch.
+ *   x, branch [B, N, C] dt read;  out [B, N, C] dt written (may equal x)
+ *   gate [B, C] fp32;  C % 8 == 0
+ * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_gated_residual(const void* x, const void* branch, const float* gate, void* out,
+                         int B, int N, int C, mmdit_dtype dt, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word of the
+ * current device: MMDIT_OK, or MMDIT_ERR_TIMEOUT if a kernel gave up on a
+ * bounded wait since the last call (its outputs are then undefined), or
+ * MMDIT_ERR_CUDA if the synchronisation failed. */
+MMDIT_API int mmdit_device_status(void* stream);
+
+/* Human-readable text of a status code (static storage). */
+MMDIT_API const char* mmdit_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MMDIT_H */

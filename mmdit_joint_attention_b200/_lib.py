@@ -1,0 +1,74 @@
+"""ctypes binding of libmmdit.so (declared in include/mmdit.h).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+Loading fails loudly (ImportError) when the library has not been built; there
+is no fallback implementation."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmmdit.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "mmdit.h")
+
+MMDIT_F32 = 0
+MMDIT_BF16 = 1
+
+STATUS = {0: "MMDIT_OK", -1: "MMDIT_ERR_ARG", -2: "MMDIT_ERR_SHAPE", -3: "MMDIT_ERR_ALIGN",
+          -4: "MMDIT_ERR_UNSUPPORTED", -5: "MMDIT_ERR_CUDA", -6: "MMDIT_ERR_TIMEOUT"}
+
+
+class Grid(ctypes.Structure):
+    """mmdit_grid: visual token grid (T, H, W) and RoPE parameters."""
+    _fields_ = [("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("pos_scale", ctypes.c_float * 3), ("rope_base", ctypes.c_float),
+                ("split", ctypes.c_int * 3)]
+
+
+class MmditError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} "
+                         f"({lib().mmdit_status_string(status).decode()})")
+
+
+_LIB = None
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+
+def declared_functions():
+    """Names of the functions include/mmdit.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^MMDIT_API\s+(?:int|const char\*)\s+(mmdit_\w+)\s*\(", text, re.M)))
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m mmdit_joint_attention_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.mmdit_qk_norm_rope.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                         ctypes.POINTER(Grid), _f, _i, _vp]
+        L.mmdit_joint_attention.argtypes = [_vp] * 9 + [_i] * 5 + [_f, _i, _vp]
+        L.mmdit_adaln_modulate.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp]
+        L.mmdit_gated_residual.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+        L.mmdit_device_status.argtypes = [_vp]
+        L.mmdit_status_string.argtypes = [_i]
+        L.mmdit_status_string.restype = ctypes.c_char_p
+        for name in ("mmdit_qk_norm_rope", "mmdit_joint_attention", "mmdit_adaln_modulate",
+                     "mmdit_gated_residual", "mmdit_device_status"):
+            getattr(L, name).restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def check(fn: str, status: int) -> None:
+    if status != 0:
+        raise MmditError(fn, status)

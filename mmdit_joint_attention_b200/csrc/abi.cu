@@ -1,0 +1,151 @@
+// C ABI of libmmdit.so (declared in include/mmdit.h): argument validation, then
+// one launch per call on the caller's stream.  No device memory is allocated.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/mmdit.h"
+#include "internal.h"
+
+using namespace mmdit;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MMDIT_OK : MMDIT_ERR_CUDA; }
+
+bool dtype_ok(mmdit_dtype dt) { return dt == MMDIT_F32 || dt == MMDIT_BF16; }
+
+// Elements per 16-byte vector.
+int vec_elems(mmdit_dtype dt) { return dt == MMDIT_BF16 ? 8 : 4; }
+
+}  // namespace
+
+extern "C" {
+
+int mmdit_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                       const float* q_scale, const float* k_scale, int B, int N, int H, int D,
+                       const mmdit_grid* grid, float eps, mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || N < 0 || H < 0 || !(eps >= 0.f) || !std::isfinite(eps))
+        return MMDIT_ERR_ARG;
+    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * N * H == 0) return MMDIT_OK;
+    if (!q_in || !k_in || !q_out || !k_out || !q_scale || !k_scale) return MMDIT_ERR_ARG;
+    if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(q_out) || !aligned16(k_out) ||
+        !aligned16(q_scale) || !aligned16(k_scale))
+        return MMDIT_ERR_ALIGN;
+    if ((long long)B * N * H > (1LL << 40)) return MMDIT_ERR_UNSUPPORTED;
+    RopeGrid g{};
+    if (grid) {
+        if (grid->T < 1 || grid->H < 1 || grid->W < 1) return MMDIT_ERR_SHAPE;
+        if ((long long)grid->T * grid->H * grid->W != (long long)N) return MMDIT_ERR_SHAPE;
+        int sum = 0;
+        for (int a = 0; a < 3; ++a) {
+            if (grid->split[a] < 0 || (grid->split[a] & 1)) return MMDIT_ERR_SHAPE;
+            sum += grid->split[a];
+            if (!std::isfinite(grid->pos_scale[a])) return MMDIT_ERR_ARG;
+        }
+        if (sum != D) return MMDIT_ERR_SHAPE;
+        if (!(grid->rope_base > 0.f) || !std::isfinite(grid->rope_base)) return MMDIT_ERR_ARG;
+        // every 16-byte vector of head dims must sit inside one axis chunk
+        const int E = vec_elems(dt);
+        if (grid->split[0] % E || (grid->split[0] + grid->split[1]) % E)
+            return MMDIT_ERR_UNSUPPORTED;
+        g.T = grid->T;
+        g.H = grid->H;
+        g.W = grid->W;
+        for (int a = 0; a < 3; ++a) {
+            g.pos_scale[a] = grid->pos_scale[a];
+            g.split[a] = grid->split[a];
+        }
+        g.base = grid->rope_base;
+    }
+    return cuda_status(launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_scale, k_scale, B, N, H,
+                                           grid ? &g : nullptr, eps, dt == MMDIT_BF16,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vis,
+                          const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                          const int32_t* ctx_len, void* o_vis, void* o_ctx, int B, int Nv, int Nc,
+                          int H, int D, float softmax_scale, mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || Nv < 0 || Nc < 0 || H < 0) return MMDIT_ERR_ARG;
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MMDIT_ERR_ARG;
+    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * H * (Nv + (long long)Nc) == 0) return MMDIT_OK;
+    if (B > 65535 || H > 65535) return MMDIT_ERR_UNSUPPORTED;
+    if (Nv > 0) {
+        if (!q_vis || !k_vis || !v_vis || !o_vis) return MMDIT_ERR_ARG;
+        if (!aligned16(q_vis) || !aligned16(k_vis) || !aligned16(v_vis) || !aligned16(o_vis))
+            return MMDIT_ERR_ALIGN;
+    }
+    if (Nc > 0) {
+        if (!q_ctx || !k_ctx || !v_ctx || !o_ctx) return MMDIT_ERR_ARG;
+        if (!aligned16(q_ctx) || !aligned16(k_ctx) || !aligned16(v_ctx) || !aligned16(o_ctx))
+            return MMDIT_ERR_ALIGN;
+    }
+    if (ctx_len && (reinterpret_cast<uintptr_t>(ctx_len) & 3u)) return MMDIT_ERR_ALIGN;
+    if ((long long)Nv + Nc > (1LL << 30)) return MMDIT_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == MMDIT_F32)
+        return cuda_status(launch_joint_attention_f32(
+            static_cast<const float*>(q_vis), static_cast<const float*>(k_vis),
+            static_cast<const float*>(v_vis), static_cast<const float*>(q_ctx),
+            static_cast<const float*>(k_ctx), static_cast<const float*>(v_ctx), ctx_len,
+            static_cast<float*>(o_vis), static_cast<float*>(o_ctx), B, Nv, Nc, H, softmax_scale,
+            s));
+    const int r = launch_joint_attention_bf16(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len,
+                                              o_vis, o_ctx, B, Nv, Nc, H, softmax_scale, s);
+    return r == 0 ? MMDIT_OK : MMDIT_ERR_CUDA;
+}
+
+int mmdit_adaln_modulate(const void* x, const float* shift, const float* scale, void* y, int B,
+                         int N, int C, float eps, mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || N < 0 || C < 0 || !(eps >= 0.f) || !std::isfinite(eps))
+        return MMDIT_ERR_ARG;
+    const int E = vec_elems(dt);
+    if (C == 0 || C % 8 != 0 || C / E > 512) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * N == 0) return MMDIT_OK;
+    if (B > 65535) return MMDIT_ERR_UNSUPPORTED;
+    if (!x || !shift || !scale || !y) return MMDIT_ERR_ARG;
+    if (!aligned16(x) || !aligned16(shift) || !aligned16(scale) || !aligned16(y))
+        return MMDIT_ERR_ALIGN;
+    return cuda_status(launch_adaln_modulate(x, shift, scale, y, B, N, C, eps, dt == MMDIT_BF16,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+int mmdit_gated_residual(const void* x, const void* branch, const float* gate, void* out, int B,
+                         int N, int C, mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || N < 0 || C < 0) return MMDIT_ERR_ARG;
+    if (C == 0 || C % 8 != 0) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * N == 0) return MMDIT_OK;
+    if (!x || !branch || !gate || !out) return MMDIT_ERR_ARG;
+    if (!aligned16(x) || !aligned16(branch) || !aligned16(gate) || !aligned16(out))
+        return MMDIT_ERR_ALIGN;
+    return cuda_status(launch_gated_residual(x, branch, gate, out, B, N, C, dt == MMDIT_BF16,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+int mmdit_device_status(void* stream) {
+    unsigned int w = 0;
+    if (read_and_clear_device_status(&w, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return MMDIT_ERR_CUDA;
+    return w ? MMDIT_ERR_TIMEOUT : MMDIT_OK;
+}
+
+const char* mmdit_status_string(int status) {
+    switch (status) {
+        case MMDIT_OK: return "ok";
+        case MMDIT_ERR_ARG: return "invalid argument";
+        case MMDIT_ERR_SHAPE: return "inconsistent shapes";
+        case MMDIT_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case MMDIT_ERR_UNSUPPORTED: return "unsupported size or layout";
+        case MMDIT_ERR_CUDA: return "CUDA error";
+        case MMDIT_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,527 @@
+// Bandwidth-bound kernels of the block:
+//   * fused QK-RMSNorm + 3D RoPE (one read and one write of q and k),
+//   * adaLN modulate  y = LN(x) * (1 + scale) + shift,
+//   * gated residual  out = x + gate * branch.
+// What they compute: "Vimoo 1.0" research page, section 2.2 (QK-RMSNorm within
+// each head with distinct learned scales; 3D RoPE over T/H/W with the 128 head
+// dims split 16/56/56, visual stream only; LayerNorm with timestep shift and
+// scale; gated residual).  The fusion of normalisation and RoPE into one pass
+// over memory follows the Seaweed-7B report, section 3.4 "Fused Kernel".
+//
+// Every kernel moves 16 bytes per thread per access (8 bf16 or 4 fp32) so a
+// warp touches whole 128-byte lines, and keeps all arithmetic in fp32.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+
+namespace mmdit {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+template <typename T>
+struct Elems;
+template <>
+struct Elems<__nv_bfloat16> {
+    static constexpr int E = 8;  // elements per 16-byte vector
+};
+template <>
+struct Elems<float> {
+    static constexpr int E = 4;
+};
+
+__device__ __forceinline__ void unpack(const uint4& u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void unpack(const uint4& u, float (&f)[4]) {
+    f[0] = __uint_as_float(u.x);
+    f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z);
+    f[3] = __uint_as_float(u.w);
+}
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint4 pack(const float (&f)[8]) {
+    return make_uint4(bf16x2(f[0], f[1]), bf16x2(f[2], f[3]), bf16x2(f[4], f[5]),
+                      bf16x2(f[6], f[7]));
+}
+__device__ __forceinline__ uint4 pack(const float (&f)[4]) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+}
+
+// Plain (coherent) 16-byte accesses: outputs may alias inputs.
+template <typename T>
+__device__ __forceinline__ uint4 ld16(const T* p) {
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+template <typename T>
+__device__ __forceinline__ void st16(T* p, const uint4& v) {
+    __stcs(reinterpret_cast<uint4*>(p), v);
+}
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+// ======================================================================
+// QK-RMSNorm + 3D RoPE
+// ======================================================================
+
+struct RopeParams {
+    int T, Hg, Wg;
+    int split[3];
+    int off[3];        // first head dim of each axis chunk
+    int stride[3];     // table row length of each axis (pairs, rounded up to even)
+    int tab_off[3];    // first table entry of each axis
+    int tab_entries;
+    double pos_scale[3];
+    double freq[64];   // frequency of pair j of axis a at index off[a]/2 + j
+};
+
+// One group of 128/E lanes owns one (token, head): its q row and its k row.
+// Lane g of the group holds head dims [g*E, g*E + E), which lie inside a single
+// RoPE axis chunk (the host checks that every chunk boundary is a multiple of
+// E), so each lane needs the (cos, sin) of E/2 consecutive pairs of one axis.
+template <typename T, bool ROPE, bool TABLE>
+__global__ void __launch_bounds__(256)
+qk_norm_rope_kernel(const T* __restrict__ q_in, const T* __restrict__ k_in, T* q_out, T* k_out,
+                    const float* __restrict__ gq, const float* __restrict__ gk, long long units,
+                    int N, int H, float eps, const RopeParams rp) {
+    constexpr int E = Elems<T>::E;
+    constexpr int LPR = kHeadDim / E;  // lanes per row
+    constexpr int GPW = 32 / LPR;      // (token, head) units per warp
+    extern __shared__ float4 rope_tab4[];
+    const float2* tab = reinterpret_cast<const float2*>(rope_tab4);
+
+    if (ROPE && TABLE) {
+        float2* wtab = reinterpret_cast<float2*>(rope_tab4);
+        for (int e = threadIdx.x; e < rp.tab_entries; e += blockDim.x) {
+            const int a = e < rp.tab_off[1] ? 0 : (e < rp.tab_off[2] ? 1 : 2);
+            const int local = e - rp.tab_off[a];
+            const int pos = local / rp.stride[a];
+            const int j = local - pos * rp.stride[a];
+            float c = 1.f, s = 0.f;
+            if (j < rp.split[a] / 2) {
+                const float ang =
+                    (float)((double)pos * rp.pos_scale[a] * rp.freq[rp.off[a] / 2 + j]);
+                sincosf(ang, &s, &c);
+            }
+            wtab[e] = make_float2(c, s);
+        }
+        __syncthreads();
+    }
+
+    const int lane = threadIdx.x & 31;
+    const int g = lane % LPR;
+    const int grp = lane / LPR;
+    const int d0 = g * E;
+    float wq[E], wk[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        wq[i] = gq[d0 + i];
+        wk[i] = gk[d0 + i];
+    }
+    const int axis = d0 < rp.off[1] ? 0 : (d0 < rp.off[2] ? 1 : 2);
+    const int jb = (d0 - rp.off[axis]) >> 1;
+    const int HW = rp.Hg * rp.Wg;
+
+    const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+    for (long long uw = warp0 * GPW; uw < units; uw += nwarps * GPW) {
+        const long long u = uw + grp;
+        const bool valid = u < units;
+        const long long base = (valid ? u : 0) * kHeadDim + d0;
+        float xq[E], xk[E];
+        uint4 rq4 = make_uint4(0, 0, 0, 0), rk4 = make_uint4(0, 0, 0, 0);
+        if (valid) {
+            rq4 = ld16(q_in + base);
+            rk4 = ld16(k_in + base);
+        }
+        unpack(rq4, xq);
+        unpack(rk4, xk);
+        float sq = 0.f, sk = 0.f;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            sq = fmaf(xq[i], xq[i], sq);
+            sk = fmaf(xk[i], xk[i], sk);
+        }
+#pragma unroll
+        for (int o = LPR / 2; o >= 1; o >>= 1) {
+            sq += __shfl_xor_sync(kFull, sq, o);
+            sk += __shfl_xor_sync(kFull, sk, o);
+        }
+        const float iq = rsqrtf(sq * (1.0f / kHeadDim) + eps);
+        const float ik = rsqrtf(sk * (1.0f / kHeadDim) + eps);
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            xq[i] *= iq * wq[i];
+            xk[i] *= ik * wk[i];
+        }
+        if (ROPE) {
+            const int n = (int)((valid ? u : 0) / H % N);
+            const int pos = axis == 0 ? n / HW : (axis == 1 ? (n / rp.Wg) % rp.Hg : n % rp.Wg);
+            float cs[E];  // (cos, sin) of the lane's E/2 pairs
+            if (TABLE) {
+                const float4* p4 = reinterpret_cast<const float4*>(
+                    tab + rp.tab_off[axis] + pos * rp.stride[axis] + jb);
+#pragma unroll
+                for (int i = 0; i < E / 4; ++i) {
+                    const float4 v = p4[i];
+                    cs[4 * i] = v.x;
+                    cs[4 * i + 1] = v.y;
+                    cs[4 * i + 2] = v.z;
+                    cs[4 * i + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int p = 0; p < E / 2; ++p) {
+                    const float ang = (float)((double)pos * rp.pos_scale[axis] *
+                                              rp.freq[rp.off[axis] / 2 + jb + p]);
+                    sincosf(ang, &cs[2 * p + 1], &cs[2 * p]);
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < E / 2; ++p) {
+                const float c = cs[2 * p], s = cs[2 * p + 1];
+                const float q0 = xq[2 * p], q1 = xq[2 * p + 1];
+                const float k0 = xk[2 * p], k1 = xk[2 * p + 1];
+                xq[2 * p] = q0 * c - q1 * s;
+                xq[2 * p + 1] = q0 * s + q1 * c;
+                xk[2 * p] = k0 * c - k1 * s;
+                xk[2 * p + 1] = k0 * s + k1 * c;
+            }
+        }
+        if (valid) {
+            st16(q_out + base, pack(xq));
+            st16(k_out + base, pack(xk));
+        }
+    }
+}
+
+template <typename T, bool ROPE, bool TABLE>
+cudaError_t run_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, const float* gq,
+                   const float* gk, long long units, int N, int H, float eps,
+                   const RopeParams& rp, size_t smem, cudaStream_t s) {
+    auto kern = qk_norm_rope_kernel<T, ROPE, TABLE>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    constexpr int GPW = 32 / (kHeadDim / Elems<T>::E);
+    const long long need = (units + 8LL * GPW - 1) / (8LL * GPW);
+    long long blocks = (long long)sm_count() * per_sm;
+    if (need < blocks) blocks = need;
+    if (blocks < 1) blocks = 1;
+    kern<<<(unsigned)blocks, 256, smem, s>>>(
+        static_cast<const T*>(q_in), static_cast<const T*>(k_in), static_cast<T*>(q_out),
+        static_cast<T*>(k_out), gq, gk, units, N, H, eps, rp);
+    return cudaGetLastError();
+}
+
+// ======================================================================
+// adaLN modulate
+// ======================================================================
+
+// Pieces of 16 bytes holding (1 + scale) and shift for one 16-byte chunk of x.
+template <typename T>
+struct ModLayout {
+    static constexpr int E = Elems<T>::E;
+    static constexpr int PIECES = 2 * E / 4;  // bf16: 4, f32: 2
+    // XOR swizzle so the 8 lanes of a quarter-warp, which read the same piece
+    // of 8 consecutive chunks, hit 8 different 16-byte bank groups.
+    __device__ static __forceinline__ int slot(int c, int k) {
+        constexpr int chunks_per_128B = 128 / (PIECES * 16);
+        return c * PIECES + (k ^ ((c / chunks_per_128B) & (PIECES - 1)));
+    }
+};
+
+// One warp per row of C elements.  The row stays in registers (packed), so x
+// is read from HBM once; mean and variance are two exact passes over the
+// registers with warp-shuffle reductions.
+template <typename T, int CPL>
+__global__ void __launch_bounds__(256)
+adaln_modulate_kernel(const T* x, const float* __restrict__ shift,
+                      const float* __restrict__ scale, T* y, int N, int C, float eps) {
+    using L = ModLayout<T>;
+    constexpr int E = L::E;
+    constexpr int P = L::PIECES;
+    extern __shared__ float4 mod[];
+    const int b = blockIdx.y;
+    const int nch = C / E;
+    for (int idx = threadIdx.x; idx < nch * P; idx += blockDim.x) {
+        const int c = idx / P, k = idx - (idx / P) * P;
+        float4 v;
+        if (k < P / 2) {
+            v = *reinterpret_cast<const float4*>(scale + (size_t)b * C + c * E + 4 * k);
+            v.x += 1.f;
+            v.y += 1.f;
+            v.z += 1.f;
+            v.w += 1.f;
+        } else {
+            v = *reinterpret_cast<const float4*>(shift + (size_t)b * C + c * E + 4 * (k - P / 2));
+        }
+        mod[L::slot(c, k)] = v;
+    }
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int warps = blockDim.x >> 5;
+    const float invC = 1.0f / (float)C;
+    for (int n = blockIdx.x * warps + (threadIdx.x >> 5); n < N; n += gridDim.x * warps) {
+        const size_t row = ((size_t)b * N + n) * (size_t)C;
+        uint4 raw[CPL];
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int c = lane + 32 * i;
+            raw[i] = c < nch ? ld16(x + row + (size_t)c * E) : make_uint4(0, 0, 0, 0);
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            float f[E];
+            unpack(raw[i], f);
+#pragma unroll
+            for (int e = 0; e < E; ++e) sum += f[e];
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
+        const float mean = sum * invC;
+        float sq = 0.f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            if (lane + 32 * i < nch) {
+                float f[E];
+                unpack(raw[i], f);
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const float d = f[e] - mean;
+                    sq = fmaf(d, d, sq);
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) sq += __shfl_xor_sync(kFull, sq, o);
+        const float rstd = rsqrtf(sq * invC + eps);
+        const float nmr = -mean * rstd;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int c = lane + 32 * i;
+            if (c < nch) {
+                float f[E];
+                unpack(raw[i], f);
+                float m[2 * E];
+#pragma unroll
+                for (int k = 0; k < P; ++k) {
+                    const float4 v = mod[L::slot(c, k)];
+                    m[4 * k] = v.x;
+                    m[4 * k + 1] = v.y;
+                    m[4 * k + 2] = v.z;
+                    m[4 * k + 3] = v.w;
+                }
+#pragma unroll
+                for (int e = 0; e < E; ++e) f[e] = fmaf(fmaf(f[e], rstd, nmr), m[e], m[E + e]);
+                st16(y + row + (size_t)c * E, pack(f));
+            }
+        }
+    }
+}
+
+template <typename T, int CPL>
+cudaError_t run_modulate(const void* x, const float* shift, const float* scale, void* y, int B,
+                         int N, int C, float eps, cudaStream_t s) {
+    auto kern = adaln_modulate_kernel<T, CPL>;
+    const size_t smem = (size_t)C * 8;  // (1 + scale, shift) per column, fp32
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    long long bx = ((long long)sm_count() * per_sm + B - 1) / B;
+    const long long need = (N + 7) / 8;
+    if (need < bx) bx = need;
+    if (bx < 1) bx = 1;
+    dim3 grid((unsigned)bx, (unsigned)B);
+    kern<<<grid, 256, smem, s>>>(static_cast<const T*>(x), shift, scale, static_cast<T*>(y), N, C,
+                                 eps);
+    return cudaGetLastError();
+}
+
+// ======================================================================
+// gated residual
+// ======================================================================
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+gated_residual_kernel(const T* x, const T* br, const float* __restrict__ gate, T* out,
+                      long long total, int nch_row, long long nch_sample, int C) {
+    constexpr int E = Elems<T>::E;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    // two independent chunks per iteration keep more loads in flight
+    for (; i + stride < total; i += 2 * stride) {
+        const long long i2 = i + stride;
+        const uint4 xa = ld16(x + i * E), ba = ld16(br + i * E);
+        const uint4 xb = ld16(x + i2 * E), bb = ld16(br + i2 * E);
+        const float* ga = gate + (i / nch_sample) * C + (int)(i % nch_row) * E;
+        const float* gb = gate + (i2 / nch_sample) * C + (int)(i2 % nch_row) * E;
+        float fx[E], fb[E], gx[E], gy[E], fy[E], fz[E];
+        unpack(xa, fx);
+        unpack(ba, fb);
+        unpack(xb, fy);
+        unpack(bb, fz);
+#pragma unroll
+        for (int k = 0; k < E / 4; ++k) {
+            const float4 u = __ldg(reinterpret_cast<const float4*>(ga) + k);
+            const float4 v = __ldg(reinterpret_cast<const float4*>(gb) + k);
+            gx[4 * k] = u.x; gx[4 * k + 1] = u.y; gx[4 * k + 2] = u.z; gx[4 * k + 3] = u.w;
+            gy[4 * k] = v.x; gy[4 * k + 1] = v.y; gy[4 * k + 2] = v.z; gy[4 * k + 3] = v.w;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            fx[e] = fmaf(gx[e], fb[e], fx[e]);
+            fy[e] = fmaf(gy[e], fz[e], fy[e]);
+        }
+        st16(out + i * E, pack(fx));
+        st16(out + i2 * E, pack(fy));
+    }
+    if (i < total) {
+        const uint4 xa = ld16(x + i * E), ba = ld16(br + i * E);
+        const float* ga = gate + (i / nch_sample) * C + (int)(i % nch_row) * E;
+        float fx[E], fb[E];
+        unpack(xa, fx);
+        unpack(ba, fb);
+#pragma unroll
+        for (int e = 0; e < E; ++e) fx[e] = fmaf(__ldg(ga + e), fb[e], fx[e]);
+        st16(out + i * E, pack(fx));
+    }
+}
+
+template <typename T>
+cudaError_t run_residual(const void* x, const void* br, const float* gate, void* out, int B,
+                         int N, int C, cudaStream_t s) {
+    constexpr int E = Elems<T>::E;
+    const int nch_row = C / E;
+    const long long nch_sample = (long long)N * nch_row;
+    const long long total = (long long)B * nch_sample;
+    if (total == 0) return cudaSuccess;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm,
+                                                                  gated_residual_kernel<T>, 256, 0);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    long long blocks = (long long)sm_count() * per_sm;
+    const long long need = (total + 255) / 256;
+    if (need < blocks) blocks = need;
+    gated_residual_kernel<T><<<(unsigned)blocks, 256, 0, s>>>(
+        static_cast<const T*>(x), static_cast<const T*>(br), gate, static_cast<T*>(out), total,
+        nch_row, nch_sample, C);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// ----------------------------------------------------------------------
+cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                                const float* gq, const float* gk, int B, int N, int H,
+                                const RopeGrid* grid, float eps, bool bf16, cudaStream_t s) {
+    const long long units = (long long)B * N * H;
+    if (units == 0) return cudaSuccess;
+    RopeParams rp{};
+    size_t smem = 0;
+    bool table = false;
+    if (grid) {
+        rp.T = grid->T;
+        rp.Hg = grid->H;
+        rp.Wg = grid->W;
+        const int extent[3] = {grid->T, grid->H, grid->W};
+        int off = 0, toff = 0;
+        for (int a = 0; a < 3; ++a) {
+            rp.split[a] = grid->split[a];
+            rp.off[a] = off;
+            rp.pos_scale[a] = grid->pos_scale[a];
+            const int half = grid->split[a] / 2;
+            for (int j = 0; j < half; ++j)
+                rp.freq[off / 2 + j] = std::pow(grid->base, -2.0 * j / (double)grid->split[a]);
+            rp.stride[a] = (half + 1) & ~1;
+            rp.tab_off[a] = toff;
+            toff += extent[a] * rp.stride[a];
+            off += grid->split[a];
+        }
+        rp.tab_entries = toff;
+        smem = (size_t)toff * sizeof(float2);
+        table = smem <= 64 * 1024;
+        if (!table) smem = 0;
+    } else {
+        rp.off[1] = rp.off[2] = kHeadDim;  // every lane on "axis 0", unused
+        rp.Hg = rp.Wg = 1;
+    }
+    if (bf16) {
+        using T = __nv_bfloat16;
+        if (!grid) return run_qk<T, false, false>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, 0, s);
+        if (table) return run_qk<T, true, true>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, smem, s);
+        return run_qk<T, true, false>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, 0, s);
+    }
+    using T = float;
+    if (!grid) return run_qk<T, false, false>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, 0, s);
+    if (table) return run_qk<T, true, true>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, smem, s);
+    return run_qk<T, true, false>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, 0, s);
+}
+
+cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float* scale,
+                                  void* y, int B, int N, int C, float eps, bool bf16,
+                                  cudaStream_t s) {
+    if ((long long)B * N == 0) return cudaSuccess;
+    const int E = bf16 ? 8 : 4;
+    const int cpl = (C / E + 31) / 32;
+#define MMDIT_MOD_CASE(V)                                                                 \
+    if (cpl <= V)                                                                         \
+        return bf16 ? run_modulate<__nv_bfloat16, V>(x, shift, scale, y, B, N, C, eps, s) \
+                    : run_modulate<float, V>(x, shift, scale, y, B, N, C, eps, s);
+    MMDIT_MOD_CASE(1)
+    MMDIT_MOD_CASE(2)
+    MMDIT_MOD_CASE(4)
+    MMDIT_MOD_CASE(8)
+    MMDIT_MOD_CASE(12)
+    MMDIT_MOD_CASE(16)
+#undef MMDIT_MOD_CASE
+    return cudaErrorInvalidValue;  // the C-ABI layer rejects such C before this point
+}
+
+cudaError_t launch_gated_residual(const void* x, const void* branch, const float* gate,
+                                  void* out, int B, int N, int C, bool bf16, cudaStream_t s) {
+    return bf16 ? run_residual<__nv_bfloat16>(x, branch, gate, out, B, N, C, s)
+                : run_residual<float>(x, branch, gate, out, B, N, C, s);
+}
+
+}  // namespace mmdit

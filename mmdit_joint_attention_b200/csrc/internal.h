@@ -1,0 +1,46 @@
+// Launchers shared between the C-ABI layer (abi.cu) and the kernel files.
+// Arguments arrive already validated by abi.cu.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mmdit {
+
+struct RopeGrid {
+    int T, H, W;
+    double pos_scale[3];
+    double base;
+    int split[3];
+};
+
+// 0 or a cudaError_t value
+cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                                const float* gq, const float* gk, int B, int N, int H,
+                                const RopeGrid* grid, float eps, bool bf16, cudaStream_t s);
+
+cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float* scale,
+                                  void* y, int B, int N, int C, float eps, bool bf16,
+                                  cudaStream_t s);
+
+cudaError_t launch_gated_residual(const void* x, const void* branch, const float* gate,
+                                  void* out, int B, int N, int C, bool bf16, cudaStream_t s);
+
+// Returns 0 on success, a cudaError_t value on CUDA failure, or -1 if the
+// driver entry point for tensor-map encoding is unavailable.
+int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv,
+                                const void* qc, const void* kc, const void* vc,
+                                const int32_t* ctx_len, void* ov, void* oc, int B, int Nv,
+                                int Nc, int H, float softmax_scale, cudaStream_t s);
+
+cudaError_t launch_joint_attention_f32(const float* qv, const float* kv, const float* vv,
+                                       const float* qc, const float* kc, const float* vc,
+                                       const int32_t* ctx_len, float* ov, float* oc, int B,
+                                       int Nv, int Nc, int H, float softmax_scale,
+                                       cudaStream_t s);
+
+// Device status word (bit set = a bounded wait expired): read-and-clear.
+cudaError_t read_and_clear_device_status(unsigned int* out, cudaStream_t s);
+
+constexpr int kHeadDim = 128;
+
+}  // namespace mmdit
