@@ -346,6 +346,7 @@ def run_ours(args):
     # ---- device-resident timing
     clocks = ClockSampler(local)
     clocks.start()
+    time.sleep(1.0)   # let nvidia-smi start sampling before the timed region
     barrier(group, dev)
     torch.cuda.synchronize(dev)
     ev = [[] for _ in range(5)]

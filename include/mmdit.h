@@ -133,6 +133,12 @@ MMDIT_API int mmdit_gated_residual(const void* x, const void* branch, const floa
  * MMDIT_ERR_CUDA if the synchronisation failed. */
 MMDIT_API int mmdit_device_status(void* stream);
 
+/* Text of the CUDA error behind the calling thread's most recent
+ * MMDIT_ERR_CUDA return (which call failed and the CUDA error name), or "" if
+ * none.  Thread-local storage owned by the library, valid until the thread's
+ * next call into the library. */
+MMDIT_API const char* mmdit_last_error(void);
+
 /* Human-readable text of a status code (static storage). */
 MMDIT_API const char* mmdit_status_string(int status);
 

@@ -30,8 +30,10 @@ class Grid(ctypes.Structure):
 class MmditError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {STATUS.get(status, status)} "
-                         f"({lib().mmdit_status_string(status).decode()})")
+        detail = lib().mmdit_status_string(status).decode()
+        if status == -5:
+            detail += ": " + lib().mmdit_last_error().decode()
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({detail})")
 
 
 _LIB = None
@@ -60,6 +62,8 @@ def lib():
         L.mmdit_adaln_modulate.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp]
         L.mmdit_gated_residual.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
         L.mmdit_device_status.argtypes = [_vp]
+        L.mmdit_last_error.argtypes = []
+        L.mmdit_last_error.restype = ctypes.c_char_p
         L.mmdit_status_string.argtypes = [_i]
         L.mmdit_status_string.restype = ctypes.c_char_p
         for name in ("mmdit_qk_norm_rope", "mmdit_joint_attention", "mmdit_adaln_modulate",

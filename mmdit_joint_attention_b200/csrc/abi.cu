@@ -4,6 +4,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 
 #include "../../include/mmdit.h"
 #include "internal.h"
@@ -12,9 +13,26 @@ using namespace mmdit;
 
 namespace {
 
+thread_local char g_last_error[256] = "";
+
+}  // namespace
+
+void mmdit::set_last_error(const char* where, int code) {
+    const char* name = code >= 1000 ? "cuTensorMapEncodeTiled rejected a tensor map"
+                       : code > 0   ? cudaGetErrorName(static_cast<cudaError_t>(code))
+                                    : "driver entry point cuTensorMapEncodeTiled unavailable";
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, name, code);
+}
+
+namespace {
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? MMDIT_OK : MMDIT_ERR_CUDA; }
+int cuda_status(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return MMDIT_OK;
+    set_last_error(where, (int)e);
+    return MMDIT_ERR_CUDA;
+}
 
 bool dtype_ok(mmdit_dtype dt) { return dt == MMDIT_F32 || dt == MMDIT_BF16; }
 
@@ -64,7 +82,8 @@ int mmdit_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_
     }
     return cuda_status(launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_scale, k_scale, B, N, H,
                                            grid ? &g : nullptr, eps, dt == MMDIT_BF16,
-                                           static_cast<cudaStream_t>(stream)));
+                                           static_cast<cudaStream_t>(stream)),
+                       "qk_norm_rope");
 }
 
 int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vis,
@@ -95,10 +114,12 @@ int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vi
             static_cast<const float*>(v_vis), static_cast<const float*>(q_ctx),
             static_cast<const float*>(k_ctx), static_cast<const float*>(v_ctx), ctx_len,
             static_cast<float*>(o_vis), static_cast<float*>(o_ctx), B, Nv, Nc, H, softmax_scale,
-            s));
+            s), "joint_attention_f32");
     const int r = launch_joint_attention_bf16(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len,
                                               o_vis, o_ctx, B, Nv, Nc, H, softmax_scale, s);
-    return r == 0 ? MMDIT_OK : MMDIT_ERR_CUDA;
+    if (r == 0) return MMDIT_OK;
+    set_last_error("joint_attention_bf16", r);
+    return MMDIT_ERR_CUDA;
 }
 
 int mmdit_adaln_modulate(const void* x, const float* shift, const float* scale, void* y, int B,
@@ -113,7 +134,8 @@ int mmdit_adaln_modulate(const void* x, const float* shift, const float* scale, 
     if (!aligned16(x) || !aligned16(shift) || !aligned16(scale) || !aligned16(y))
         return MMDIT_ERR_ALIGN;
     return cuda_status(launch_adaln_modulate(x, shift, scale, y, B, N, C, eps, dt == MMDIT_BF16,
-                                             static_cast<cudaStream_t>(stream)));
+                                             static_cast<cudaStream_t>(stream)),
+                       "adaln_modulate");
 }
 
 int mmdit_gated_residual(const void* x, const void* branch, const float* gate, void* out, int B,
@@ -125,15 +147,18 @@ int mmdit_gated_residual(const void* x, const void* branch, const float* gate, v
     if (!aligned16(x) || !aligned16(branch) || !aligned16(gate) || !aligned16(out))
         return MMDIT_ERR_ALIGN;
     return cuda_status(launch_gated_residual(x, branch, gate, out, B, N, C, dt == MMDIT_BF16,
-                                             static_cast<cudaStream_t>(stream)));
+                                             static_cast<cudaStream_t>(stream)),
+                       "gated_residual");
 }
 
 int mmdit_device_status(void* stream) {
     unsigned int w = 0;
-    if (read_and_clear_device_status(&w, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return MMDIT_ERR_CUDA;
+    const cudaError_t e = read_and_clear_device_status(&w, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e, "device_status");
     return w ? MMDIT_ERR_TIMEOUT : MMDIT_OK;
 }
+
+const char* mmdit_last_error(void) { return g_last_error; }
 
 const char* mmdit_status_string(int status) {
     switch (status) {

@@ -124,7 +124,7 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t tile, int s) {
     return smem_desc_sw128(tile + s * 2048, kHalfBytes, 1024);
 }
 
-__global__ void __maxnreg__(200) joint_attn_bf16_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -477,12 +477,12 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
     if (Nv > 0) {
         if (!encode_tokens(&p.tm_q[0], qv, B, Nv, H) || !encode_tokens(&p.tm_k[0], kv, B, Nv, H) ||
             !encode_tokens(&p.tm_v[0], vv, B, Nv, H))
-            return (int)cudaErrorInvalidValue;
+            return 1000 + (int)cudaErrorInvalidValue;
     }
     if (Nc > 0) {
         if (!encode_tokens(&p.tm_q[1], qc, B, Nc, H) || !encode_tokens(&p.tm_k[1], kc, B, Nc, H) ||
             !encode_tokens(&p.tm_v[1], vc, B, Nc, H))
-            return (int)cudaErrorInvalidValue;
+            return 1000 + (int)cudaErrorInvalidValue;
     }
     p.out[0] = static_cast<__nv_bfloat16*>(ov);
     p.out[1] = static_cast<__nv_bfloat16*>(oc);

@@ -43,4 +43,7 @@ cudaError_t read_and_clear_device_status(unsigned int* out, cudaStream_t s);
 
 constexpr int kHeadDim = 128;
 
+// Records the CUDA error behind an MMDIT_ERR_CUDA return for mmdit_last_error().
+void set_last_error(const char* where, int code);
+
 }  // namespace mmdit
