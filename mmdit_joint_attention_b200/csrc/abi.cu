@@ -54,7 +54,7 @@ int mmdit_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_
     if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(q_out) || !aligned16(k_out) ||
         !aligned16(q_scale) || !aligned16(k_scale))
         return MMDIT_ERR_ALIGN;
-    if ((long long)B * N * H > (1LL << 40)) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * N * H >= (1LL << 31)) return MMDIT_ERR_UNSUPPORTED;
     RopeGrid g{};
     if (grid) {
         if (grid->T < 1 || grid->H < 1 || grid->W < 1) return MMDIT_ERR_SHAPE;

@@ -89,8 +89,26 @@ int sm_count() {
 // QK-RMSNorm + 3D RoPE
 // ======================================================================
 
+// Unsigned 32-bit division by a run-time constant d >= 1, exact for n < 2^31:
+// with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1 (computed on the
+// host), n / d = (umulhi(n, m) + n) >> l.  (Multiply-high division by an
+// invariant integer, Granlund & Montgomery, PLDI 1994.)
+struct FastDiv {
+    uint32_t d, m, l;
+};
+FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while ((1ull << l) < d) ++l;
+    const uint64_t m = ((1ull << 32) * ((1ull << l) - d)) / d + 1;
+    return FastDiv{d, (uint32_t)m, l};
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+    return (__umulhi(n, f.m) + n) >> f.l;
+}
+
 struct RopeParams {
-    int T, Hg, Wg;
+    FastDiv H, N, HW, W;   // heads, tokens per sample, Hg*Wg, Wg
+    int Hg;
     int split[3];
     int off[3];        // first head dim of each axis chunk
     int stride[3];     // table row length of each axis (pairs, rounded up to even)
@@ -104,14 +122,20 @@ struct RopeParams {
 // Lane g of the group holds head dims [g*E, g*E + E), which lie inside a single
 // RoPE axis chunk (the host checks that every chunk boundary is a multiple of
 // E), so each lane needs the (cos, sin) of E/2 consecutive pairs of one axis.
-template <typename T, bool ROPE, bool TABLE>
-__global__ void __launch_bounds__(256)
-qk_norm_rope_kernel(const T* __restrict__ q_in, const T* __restrict__ k_in, T* q_out, T* k_out,
-                    const float* __restrict__ gq, const float* __restrict__ gk, long long units,
-                    int N, int H, float eps, const RopeParams rp) {
+// Each warp handles UNR groups of consecutive units per iteration and issues
+// all of their loads before any arithmetic, to keep enough bytes in flight.
+// 8 units in flight per warp and 2 CTAs of 256 threads per SM measured best at
+// 480p (5.5 TB/s, vs 3.6 TB/s with one unit per group and 64-bit index math).
+constexpr int kQkUnroll = 8;
+
+template <typename T, bool ROPE, bool TABLE, int UNR>
+__global__ void __launch_bounds__(256, 2)
+qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
+                    const float* __restrict__ gq, const float* __restrict__ gk, uint32_t units,
+                    float eps, const RopeParams rp) {
     constexpr int E = Elems<T>::E;
     constexpr int LPR = kHeadDim / E;  // lanes per row
-    constexpr int GPW = 32 / LPR;      // (token, head) units per warp
+    constexpr int GPW = 32 / LPR;      // (token, head) units per warp per round
     extern __shared__ float4 rope_tab4[];
     const float2* tab = reinterpret_cast<const float2*>(rope_tab4);
 
@@ -145,86 +169,101 @@ qk_norm_rope_kernel(const T* __restrict__ q_in, const T* __restrict__ k_in, T* q
     }
     const int axis = d0 < rp.off[1] ? 0 : (d0 < rp.off[2] ? 1 : 2);
     const int jb = (d0 - rp.off[axis]) >> 1;
-    const int HW = rp.Hg * rp.Wg;
 
-    const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-    for (long long uw = warp0 * GPW; uw < units; uw += nwarps * GPW) {
-        const long long u = uw + grp;
-        const bool valid = u < units;
-        const long long base = (valid ? u : 0) * kHeadDim + d0;
-        float xq[E], xk[E];
-        uint4 rq4 = make_uint4(0, 0, 0, 0), rk4 = make_uint4(0, 0, 0, 0);
-        if (valid) {
-            rq4 = ld16(q_in + base);
-            rk4 = ld16(k_in + base);
-        }
-        unpack(rq4, xq);
-        unpack(rk4, xk);
-        float sq = 0.f, sk = 0.f;
+    const uint32_t warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t uw = warp0 * (GPW * UNR); uw < units; uw += nwarps * (GPW * UNR)) {
+        uint4 rq[UNR], rk[UNR];
 #pragma unroll
-        for (int i = 0; i < E; ++i) {
-            sq = fmaf(xq[i], xq[i], sq);
-            sk = fmaf(xk[i], xk[i], sk);
-        }
-#pragma unroll
-        for (int o = LPR / 2; o >= 1; o >>= 1) {
-            sq += __shfl_xor_sync(kFull, sq, o);
-            sk += __shfl_xor_sync(kFull, sk, o);
-        }
-        const float iq = rsqrtf(sq * (1.0f / kHeadDim) + eps);
-        const float ik = rsqrtf(sk * (1.0f / kHeadDim) + eps);
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-            xq[i] *= iq * wq[i];
-            xk[i] *= ik * wk[i];
-        }
-        if (ROPE) {
-            const int n = (int)((valid ? u : 0) / H % N);
-            const int pos = axis == 0 ? n / HW : (axis == 1 ? (n / rp.Wg) % rp.Hg : n % rp.Wg);
-            float cs[E];  // (cos, sin) of the lane's E/2 pairs
-            if (TABLE) {
-                const float4* p4 = reinterpret_cast<const float4*>(
-                    tab + rp.tab_off[axis] + pos * rp.stride[axis] + jb);
-#pragma unroll
-                for (int i = 0; i < E / 4; ++i) {
-                    const float4 v = p4[i];
-                    cs[4 * i] = v.x;
-                    cs[4 * i + 1] = v.y;
-                    cs[4 * i + 2] = v.z;
-                    cs[4 * i + 3] = v.w;
-                }
+        for (int r = 0; r < UNR; ++r) {
+            const uint32_t u = uw + r * GPW + grp;
+            if (u < units) {
+                const size_t base = (size_t)u * kHeadDim + d0;
+                rq[r] = ld16(q_in + base);
+                rk[r] = ld16(k_in + base);
             } else {
+                rq[r] = make_uint4(0, 0, 0, 0);
+                rk[r] = make_uint4(0, 0, 0, 0);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < UNR; ++r) {
+            const uint32_t u = uw + r * GPW + grp;
+            float xq[E], xk[E];
+            unpack(rq[r], xq);
+            unpack(rk[r], xk);
+            float sq = 0.f, sk = 0.f;
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                sq = fmaf(xq[i], xq[i], sq);
+                sk = fmaf(xk[i], xk[i], sk);
+            }
+#pragma unroll
+            for (int o = LPR / 2; o >= 1; o >>= 1) {
+                sq += __shfl_xor_sync(kFull, sq, o);
+                sk += __shfl_xor_sync(kFull, sk, o);
+            }
+            const float iq = rsqrtf(sq * (1.0f / kHeadDim) + eps);
+            const float ik = rsqrtf(sk * (1.0f / kHeadDim) + eps);
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                xq[i] *= iq * wq[i];
+                xk[i] *= ik * wk[i];
+            }
+            if (ROPE) {
+                const uint32_t uu = u < units ? u : 0;
+                const uint32_t bn = fdiv(uu, rp.H);
+                const uint32_t n = bn - fdiv(bn, rp.N) * rp.N.d;
+                const uint32_t t = fdiv(n, rp.HW);
+                const uint32_t rem = n - t * rp.HW.d;
+                const uint32_t hh = fdiv(rem, rp.W);
+                const uint32_t pos = axis == 0 ? t : (axis == 1 ? hh : rem - hh * rp.W.d);
+                float cs[E];  // (cos, sin) of the lane's E/2 pairs
+                if (TABLE) {
+                    const float4* p4 = reinterpret_cast<const float4*>(
+                        tab + rp.tab_off[axis] + pos * rp.stride[axis] + jb);
+#pragma unroll
+                    for (int i = 0; i < E / 4; ++i) {
+                        const float4 v = p4[i];
+                        cs[4 * i] = v.x;
+                        cs[4 * i + 1] = v.y;
+                        cs[4 * i + 2] = v.z;
+                        cs[4 * i + 3] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int p = 0; p < E / 2; ++p) {
+                        const float ang = (float)((double)pos * rp.pos_scale[axis] *
+                                                  rp.freq[rp.off[axis] / 2 + jb + p]);
+                        sincosf(ang, &cs[2 * p + 1], &cs[2 * p]);
+                    }
+                }
 #pragma unroll
                 for (int p = 0; p < E / 2; ++p) {
-                    const float ang = (float)((double)pos * rp.pos_scale[axis] *
-                                              rp.freq[rp.off[axis] / 2 + jb + p]);
-                    sincosf(ang, &cs[2 * p + 1], &cs[2 * p]);
+                    const float c = cs[2 * p], s = cs[2 * p + 1];
+                    const float q0 = xq[2 * p], q1 = xq[2 * p + 1];
+                    const float k0 = xk[2 * p], k1 = xk[2 * p + 1];
+                    xq[2 * p] = q0 * c - q1 * s;
+                    xq[2 * p + 1] = q0 * s + q1 * c;
+                    xk[2 * p] = k0 * c - k1 * s;
+                    xk[2 * p + 1] = k0 * s + k1 * c;
                 }
             }
-#pragma unroll
-            for (int p = 0; p < E / 2; ++p) {
-                const float c = cs[2 * p], s = cs[2 * p + 1];
-                const float q0 = xq[2 * p], q1 = xq[2 * p + 1];
-                const float k0 = xk[2 * p], k1 = xk[2 * p + 1];
-                xq[2 * p] = q0 * c - q1 * s;
-                xq[2 * p + 1] = q0 * s + q1 * c;
-                xk[2 * p] = k0 * c - k1 * s;
-                xk[2 * p + 1] = k0 * s + k1 * c;
+            if (u < units) {
+                const size_t base = (size_t)u * kHeadDim + d0;
+                st16(q_out + base, pack(xq));
+                st16(k_out + base, pack(xk));
             }
-        }
-        if (valid) {
-            st16(q_out + base, pack(xq));
-            st16(k_out + base, pack(xk));
         }
     }
 }
 
 template <typename T, bool ROPE, bool TABLE>
 cudaError_t run_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, const float* gq,
-                   const float* gk, long long units, int N, int H, float eps,
-                   const RopeParams& rp, size_t smem, cudaStream_t s) {
-    auto kern = qk_norm_rope_kernel<T, ROPE, TABLE>;
+                   const float* gk, uint32_t units, float eps, const RopeParams& rp, size_t smem,
+                   cudaStream_t s) {
+    constexpr int UNR = kQkUnroll;
+    auto kern = qk_norm_rope_kernel<T, ROPE, TABLE, UNR>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -235,13 +274,13 @@ cudaError_t run_qk(const void* q_in, const void* k_in, void* q_out, void* k_out,
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     constexpr int GPW = 32 / (kHeadDim / Elems<T>::E);
-    const long long need = (units + 8LL * GPW - 1) / (8LL * GPW);
+    const long long need = ((long long)units + 8LL * GPW * UNR - 1) / (8LL * GPW * UNR);
     long long blocks = (long long)sm_count() * per_sm;
     if (need < blocks) blocks = need;
     if (blocks < 1) blocks = 1;
     kern<<<(unsigned)blocks, 256, smem, s>>>(
         static_cast<const T*>(q_in), static_cast<const T*>(k_in), static_cast<T*>(q_out),
-        static_cast<T*>(k_out), gq, gk, units, N, H, eps, rp);
+        static_cast<T*>(k_out), gq, gk, units, eps, rp);
     return cudaGetLastError();
 }
 
@@ -263,10 +302,84 @@ struct ModLayout {
 };
 
 // One warp per row of C elements.  The row stays in registers (packed), so x
-// is read from HBM once; mean and variance are two exact passes over the
-// registers with warp-shuffle reductions.
+// is read from HBM once; both moments come from one pass over the registers
+// and one warp-shuffle reduction.
 template <typename T, int CPL>
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void mod_load(uint4 (&raw)[CPL], const T* x, size_t row, int nch,
+                                         int lane) {
+    constexpr int E = Elems<T>::E;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        const int c = lane + 32 * i;
+        raw[i] = c < nch ? ld16(x + row + (size_t)c * E) : make_uint4(0, 0, 0, 0);
+    }
+}
+
+template <typename T, int CPL>
+__device__ __forceinline__ void mod_row(const uint4 (&raw)[CPL], T* y, size_t row, int nch,
+                                        int lane, float invC, float eps, const float4* mod) {
+    using L = ModLayout<T>;
+    constexpr int E = L::E;
+    constexpr int P = L::PIECES;
+    // One pass over the row for both moments, shifted by a pivot (the row's
+    // first element) so that E[(x-p)^2] - E[x-p]^2 does not cancel when the
+    // row mean is large compared to its spread.
+    float pivot;
+    {
+        float f[E];
+        unpack(raw[0], f);
+        pivot = __shfl_sync(kFull, f[0], 0);
+    }
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        if (lane + 32 * i < nch) {
+            float f[E];
+            unpack(raw[i], f);
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const float d = f[e] - pivot;
+                s1 += d;
+                s2 = fmaf(d, d, s2);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        s1 += __shfl_xor_sync(kFull, s1, o);
+        s2 += __shfl_xor_sync(kFull, s2, o);
+    }
+    const float dm = s1 * invC;
+    const float var = fmaxf(s2 * invC - dm * dm, 0.f);
+    const float mean = pivot + dm;
+    const float rstd = rsqrtf(var + eps);
+    const float nmr = -mean * rstd;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        const int c = lane + 32 * i;
+        if (c < nch) {
+            float f[E];
+            unpack(raw[i], f);
+            float m[2 * E];
+#pragma unroll
+            for (int k = 0; k < P; ++k) {
+                const float4 v = mod[L::slot(c, k)];
+                m[4 * k] = v.x;
+                m[4 * k + 1] = v.y;
+                m[4 * k + 2] = v.z;
+                m[4 * k + 3] = v.w;
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) f[e] = fmaf(fmaf(f[e], rstd, nmr), m[e], m[E + e]);
+            st16(y + row + (size_t)c * E, pack(f));
+        }
+    }
+}
+
+// Two CTAs of 256 threads per SM (about 127 registers, 16 warps): measured
+// best at 480p among 1-3 CTAs per SM with and without double-buffered rows.
+template <typename T, int CPL>
+__global__ void __launch_bounds__(256, 2)
 adaln_modulate_kernel(const T* x, const float* __restrict__ shift,
                       const float* __restrict__ scale, T* y, int N, int C, float eps) {
     using L = ModLayout<T>;
@@ -294,63 +407,15 @@ adaln_modulate_kernel(const T* x, const float* __restrict__ shift,
     const int lane = threadIdx.x & 31;
     const int warps = blockDim.x >> 5;
     const float invC = 1.0f / (float)C;
-    for (int n = blockIdx.x * warps + (threadIdx.x >> 5); n < N; n += gridDim.x * warps) {
-        const size_t row = ((size_t)b * N + n) * (size_t)C;
-        uint4 raw[CPL];
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int c = lane + 32 * i;
-            raw[i] = c < nch ? ld16(x + row + (size_t)c * E) : make_uint4(0, 0, 0, 0);
-        }
-        float sum = 0.f;
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            float f[E];
-            unpack(raw[i], f);
-#pragma unroll
-            for (int e = 0; e < E; ++e) sum += f[e];
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
-        const float mean = sum * invC;
-        float sq = 0.f;
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            if (lane + 32 * i < nch) {
-                float f[E];
-                unpack(raw[i], f);
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const float d = f[e] - mean;
-                    sq = fmaf(d, d, sq);
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) sq += __shfl_xor_sync(kFull, sq, o);
-        const float rstd = rsqrtf(sq * invC + eps);
-        const float nmr = -mean * rstd;
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int c = lane + 32 * i;
-            if (c < nch) {
-                float f[E];
-                unpack(raw[i], f);
-                float m[2 * E];
-#pragma unroll
-                for (int k = 0; k < P; ++k) {
-                    const float4 v = mod[L::slot(c, k)];
-                    m[4 * k] = v.x;
-                    m[4 * k + 1] = v.y;
-                    m[4 * k + 2] = v.z;
-                    m[4 * k + 3] = v.w;
-                }
-#pragma unroll
-                for (int e = 0; e < E; ++e) f[e] = fmaf(fmaf(f[e], rstd, nmr), m[e], m[E + e]);
-                st16(y + row + (size_t)c * E, pack(f));
-            }
-        }
+    const int stride = gridDim.x * warps;
+    const size_t base = (size_t)b * N * (size_t)C;
+    int n = blockIdx.x * warps + (threadIdx.x >> 5);
+    for (; n < N; n += stride) {
+        uint4 buf[CPL];
+        mod_load<T, CPL>(buf, x, base + (size_t)n * C, nch, lane);
+        mod_row<T, CPL>(buf, y, base + (size_t)n * C, nch, lane, invC, eps, mod);
     }
+
 }
 
 template <typename T, int CPL>
@@ -455,15 +520,19 @@ cudaError_t run_residual(const void* x, const void* br, const float* gate, void*
 cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
                                 const float* gq, const float* gk, int B, int N, int H,
                                 const RopeGrid* grid, float eps, bool bf16, cudaStream_t s) {
-    const long long units = (long long)B * N * H;
-    if (units == 0) return cudaSuccess;
+    const long long units_ll = (long long)B * N * H;
+    if (units_ll == 0) return cudaSuccess;
+    if (units_ll >= (1LL << 31)) return cudaErrorInvalidValue;  // rejected by the C-ABI layer
+    const uint32_t units = (uint32_t)units_ll;
     RopeParams rp{};
+    rp.H = make_fastdiv((uint32_t)H);
+    rp.N = make_fastdiv((uint32_t)N);
     size_t smem = 0;
     bool table = false;
     if (grid) {
-        rp.T = grid->T;
         rp.Hg = grid->H;
-        rp.Wg = grid->W;
+        rp.HW = make_fastdiv((uint32_t)grid->H * (uint32_t)grid->W);
+        rp.W = make_fastdiv((uint32_t)grid->W);
         const int extent[3] = {grid->T, grid->H, grid->W};
         int off = 0, toff = 0;
         for (int a = 0; a < 3; ++a) {
@@ -484,18 +553,19 @@ cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out,
         if (!table) smem = 0;
     } else {
         rp.off[1] = rp.off[2] = kHeadDim;  // every lane on "axis 0", unused
-        rp.Hg = rp.Wg = 1;
+        rp.Hg = 1;
+        rp.HW = rp.W = make_fastdiv(1);
     }
     if (bf16) {
         using T = __nv_bfloat16;
-        if (!grid) return run_qk<T, false, false>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, 0, s);
-        if (table) return run_qk<T, true, true>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, smem, s);
-        return run_qk<T, true, false>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, 0, s);
+        if (!grid) return run_qk<T, false, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, s);
+        if (table) return run_qk<T, true, true>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, smem, s);
+        return run_qk<T, true, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, s);
     }
     using T = float;
-    if (!grid) return run_qk<T, false, false>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, 0, s);
-    if (table) return run_qk<T, true, true>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, smem, s);
-    return run_qk<T, true, false>(q_in, k_in, q_out, k_out, gq, gk, units, N, H, eps, rp, 0, s);
+    if (!grid) return run_qk<T, false, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, s);
+    if (table) return run_qk<T, true, true>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, smem, s);
+    return run_qk<T, true, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, s);
 }
 
 cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float* scale,
