@@ -45,12 +45,25 @@ namespace attn {
 
 constexpr int kBlockM = 128;         // query rows per tile
 constexpr int kBlockN = 128;         // keys per tile
-constexpr int kStages = 2;           // K and V ring depth
+constexpr int kStages = 2;           // K and V ring depth (the MMA issuer assumes 2)
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kHalfBytes = kTileBytes / 2;  // one 64-column TMA box (128 B per row)
-constexpr int kThreads = 320;        // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA
+// Warpgroups: 0 = softmax of query tile 0 (warps 0-3), 1 = softmax of tile 1
+// (warps 4-7), 2 = warp 8 TMA of Q and K, warp 9 MMA issuer, warp 10 TMA of V,
+// warp 11 idle.  K and V have their own producers so that neither waits for
+// the other's ring slot: a tile takes about one KV iteration to arrive.
+constexpr int kThreads = 384;
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
+constexpr int kWarpLoadV = 10;
+// Register split: launched with kRegsLaunch per thread (64512 in total); the
+// producer warpgroup drops to kRegsProducer, the softmax warpgroups rise to
+// kRegsSoftmax: 2*128*216 + 128*72 = 64512, the launch total.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsProducer = 72;
+constexpr int kRegsSoftmax = 216;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsProducer == kThreads * kRegsLaunch,
+              "register split must add up to the launch allocation");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per pipeline wait
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s per drain wait after an abort
 
@@ -80,7 +93,8 @@ struct Bars {
     uint64_t q_full;
     uint64_t k_full[kStages], k_empty[kStages];
     uint64_t v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t s_full[2], o_done[2];
+    uint64_t p_full[4];  // [2 i + h]: half h (keys 64h..64h+63) of P_i is in tensor memory
     uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
@@ -124,6 +138,70 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t tile, int s) {
     return smem_desc_sw128(tile + s * 2048, kHalfBytes, 1024);
 }
 
+// Streams the n_kv 128-key tiles of one operand (K or V) of the joint key
+// sequence (visual tiles first, then conditioning tiles) through its ring of
+// kStages shared-memory slots.  On an abort, waits (bounded) for the copies
+// it issued before returning.
+__device__ __forceinline__ void stream_tiles(const CUtensorMap* tm, uint8_t* ring, uint64_t* full,
+                                             uint64_t* empty, int n_kv, int kv_vis, int h, int b,
+                                             Bars* bars) {
+    int issued = 0;
+    for (int j = 0; j < n_kv; ++j) {
+        const int st = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        const int seg = j < kv_vis ? 0 : 1;
+        const int row = (seg == 0 ? j : j - kv_vis) * kBlockN;
+        if (!wait(&empty[st], ph ^ 1, bars)) break;
+        uint8_t* t = ring + st * kTileBytes;
+        mbar_arrive_expect_tx(&full[st], kTileBytes);
+        tma_load_4d(t, &tm[seg], &full[st], 0, h, row, b);
+        tma_load_4d(t + kHalfBytes, &tm[seg], &full[st], 64, h, row, b);
+        ++issued;
+    }
+    if (bars->abort) {
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+            mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1, nullptr, kDrainLimitNs);
+    }
+}
+
+// O row of this thread *= f, 32 tensor-memory columns at a time.
+__device__ __forceinline__ void rescale_o(uint32_t tO, float f) {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+        tmem_st32(tO + 32 * c, o);
+    }
+}
+
+// P = 2^(s * scale_log2 - m) for keys [64 h, 64 h + 64) of one score row,
+// packed two bf16 keys per 32-bit column into rh (column c holds keys
+// 64 h + 2c, 64 h + 2c + 1); returns their sum.  Products and sums use the
+// packed fp32x2 pipe, the partial sums run in four independent chains.
+__device__ __forceinline__ float exp_half(const float (&sv)[128], uint32_t (&rh)[32], int h,
+                                          uint64_t sl2x2, uint64_t negm2) {
+    uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const int k = 64 * h + 2 * c;
+        const uint64_t x2 = f2_fma(f2_pack(sv[k], sv[k + 1]), sl2x2, negm2);
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        const uint64_t e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        acc[c & 3] = f2_add(acc[c & 3], e2);
+        float a0, a1;
+        f2_unpack(e2, a0, a1);
+        rh[c] = pack_bf16x2(a0, a1);
+    }
+    const uint64_t s2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+    float lo, hi;
+    f2_unpack(s2, lo, hi);
+    return lo + hi;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -154,7 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->s_full[i], 1);
-            mbar_init(&bars->p_full[i], 128);
+            mbar_init(&bars->p_full[2 * i], 4);      // one elected lane per softmax warp
+            mbar_init(&bars->p_full[2 * i + 1], 4);
             mbar_init(&bars->o_done[i], 1);
         }
         mbar_init(&bars->drain, 1);
@@ -191,17 +270,19 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         return;
     }
 
+    // Each role's whole body sits inside the branch that set its register
+    // budget, so the compiler allocates each region with its own limit.
+    if (warp >= 8) {
+        regs_dec<kRegsProducer>();
     if (warp == kWarpLoad) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ TMA: Q and K
         if (lane == 0) {
             for (int seg = 0; seg < 2; ++seg) {
                 if (p.N[seg] > 0) {
                     tma_prefetch_desc(&p.tm_q[seg]);
                     tma_prefetch_desc(&p.tm_k[seg]);
-                    tma_prefetch_desc(&p.tm_v[seg]);
                 }
             }
-            int jk = 0, jv = 0;  // K / V tile loads issued
             int s0, r0, s1 = 0, r1 = 0;
             tile_of(p, t0, s0, r0);
             if (has1) tile_of(p, t0 + 1, s1, r1);
@@ -213,99 +294,100 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                 tma_load_4d(smem + Smem::q_off + kTileBytes + kHalfBytes, &p.tm_q[s1], &bars->q_full,
                             64, h, r1, b);
             }
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j % kStages;
-                const uint32_t ph = (j / kStages) & 1;
-                const int seg = j < kv_vis ? 0 : 1;
-                const int row = (seg == 0 ? j : j - kv_vis) * kBlockN;
-                if (!wait(&bars->k_empty[st], ph ^ 1, bars)) break;
-                uint8_t* kt = smem + Smem::k_off + st * kTileBytes;
-                mbar_arrive_expect_tx(&bars->k_full[st], kTileBytes);
-                tma_load_4d(kt, &p.tm_k[seg], &bars->k_full[st], 0, h, row, b);
-                tma_load_4d(kt + kHalfBytes, &p.tm_k[seg], &bars->k_full[st], 64, h, row, b);
-                ++jk;
-                if (!wait(&bars->v_empty[st], ph ^ 1, bars)) break;
-                uint8_t* vt = smem + Smem::v_off + st * kTileBytes;
-                mbar_arrive_expect_tx(&bars->v_full[st], kTileBytes);
-                tma_load_4d(vt, &p.tm_v[seg], &bars->v_full[st], 0, h, row, b);
-                tma_load_4d(vt + kHalfBytes, &p.tm_v[seg], &bars->v_full[st], 64, h, row, b);
-                ++jv;
-            }
-            if (bars->abort) {
-                // let every copy already issued land before the CTA exits
-                volatile uint32_t never = 0;
-                mbar_wait_bounded(&bars->q_full, 0, &never, kDrainLimitNs);
-                for (int j = (jk > kStages ? jk - kStages : 0); j < jk; ++j)
-                    mbar_wait_bounded(&bars->k_full[j % kStages], (j / kStages) & 1, &never,
-                                      kDrainLimitNs);
-                for (int j = (jv > kStages ? jv - kStages : 0); j < jv; ++j)
-                    mbar_wait_bounded(&bars->v_full[j % kStages], (j / kStages) & 1, &never,
-                                      kDrainLimitNs);
-            }
+            stream_tiles(p.tm_k, smem + Smem::k_off, bars->k_full, bars->k_empty, n_kv, kv_vis, h,
+                         b, bars);
+            if (bars->abort) mbar_wait_bounded(&bars->q_full, 0, nullptr, kDrainLimitNs);
         }
-    } else if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == kWarpLoadV) {
+        // ------------------------------------------------------------ TMA: V
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-            const uint32_t tS[2] = {tmem + 0, tmem + 128};
-            const uint32_t tO[2] = {tmem + 256, tmem + 384};
-            const int ntile = has1 ? 2 : 1;
-            bool ok = wait(&bars->q_full, 0, bars);
-            auto qk = [&](int i, int st) {
-                const uint32_t q = sQ + i * kTileBytes;
-                const uint32_t k = sK + st * kTileBytes;
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_ss(tS[i], desc_kmajor(q, s), desc_kmajor(k, s), idesc_qk, s > 0 ? 1u : 0u);
-            };
-            auto pv = [&](int i, int st, bool acc) {
-                const uint32_t v = sV + st * kTileBytes;
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_ts(tO[i], tS[i] + s * 8, desc_v(v, s), idesc_pv, (acc || s > 0) ? 1u : 0u);
-            };
-            for (int j = 0; ok && j < n_kv; ++j) {
-                const int st = j % kStages;
-                const uint32_t ph = (j / kStages) & 1;
-                const int pst = (j + kStages - 1) % kStages;
-                const uint32_t pph = ((j - 1) / kStages) & 1;
-                if (!(ok = wait(&bars->k_full[st], ph, bars))) break;
-                if (j > 0 && !(ok = wait(&bars->v_full[pst], pph, bars))) break;
-                for (int i = 0; i < ntile; ++i) {
-                    if (j > 0) {
-                        if (!(ok = wait(&bars->p_full[i], (j - 1) & 1, bars))) break;
-                        tc_fence_after();
-                        pv(i, pst, j > 1);
-                    }
-                    tc_fence_after();
-                    qk(i, st);
-                    mma_commit(&bars->s_full[i]);
-                }
-                if (!ok) break;
-                if (j > 0) mma_commit(&bars->v_empty[pst]);
-                mma_commit(&bars->k_empty[st]);
-            }
-            if (ok) {
-                const int j = n_kv;
-                const int pst = (j - 1) % kStages;
-                const uint32_t pph = ((j - 1) / kStages) & 1;
-                ok = wait(&bars->v_full[pst], pph, bars);
-                for (int i = 0; ok && i < ntile; ++i) {
-                    if (!(ok = wait(&bars->p_full[i], (j - 1) & 1, bars))) break;
-                    tc_fence_after();
-                    pv(i, pst, j > 1);
-                    mma_commit(&bars->o_done[i]);
-                }
-                if (ok) mma_commit(&bars->v_empty[pst]);
-            }
-            // make sure nothing this thread issued is still running before TMEM is freed
-            mma_commit(&bars->drain);
-            volatile uint32_t never = 0;
-            if (!mbar_wait_bounded(&bars->drain, 0, &never, kDrainLimitNs))
-                atomicOr(&g_device_status, 1u);
+            for (int seg = 0; seg < 2; ++seg)
+                if (p.N[seg] > 0) tma_prefetch_desc(&p.tm_v[seg]);
+            stream_tiles(p.tm_v, smem + Smem::v_off, bars->v_full, bars->v_empty, n_kv, kv_vis, h,
+                         b, bars);
         }
+    } else if (warp == kWarpMma && lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        // One thread issues every MMA, in the order PV_0(j-1), QK_0(j),
+        // PV_1(j-1), QK_1(j): QK_i(j) overwrites the tensor memory PV_i(j-1)
+        // reads, and one thread's MMAs execute in issue order.  (Two issuing
+        // threads, one per tile, measured 14 % slower: the tensor core then
+        // interleaves the two tiles' batches and both S tiles arrive later.)
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+        const int ntile = has1 ? 2 : 1;
+        bool ok = wait(&bars->q_full, 0, bars);
+        // Descriptor bases are computed once; a k-step only adds a constant to
+        // the start-address field (shared addresses stay below 256 KB, so the
+        // 14-bit field never carries).  This keeps the issuing thread, which
+        // shares its SM sub-partition with softmax warps, to a few
+        // instructions per MMA.
+        const uint64_t dq0 = desc_kmajor(sQ, 0), dq1 = desc_kmajor(sQ + kTileBytes, 0);
+        const uint64_t dk0 = desc_kmajor(sK, 0), dk1 = desc_kmajor(sK + kTileBytes, 0);
+        const uint64_t dv0 = desc_v(sV, 0), dv1 = desc_v(sV + kTileBytes, 0);
+        // tile i: S_i (and P_i over its first 64 columns) at column 128 i, O_i at 256 + 128 i
+        auto qk = [&](int i, int st) {
+            const uint64_t dq = i == 0 ? dq0 : dq1;
+            const uint64_t dk = st == 0 ? dk0 : dk1;
+            const uint32_t d = tmem + 128 * i;
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint64_t off = (uint64_t)((s >> 2) * (kHalfBytes >> 4) + (s & 3) * 2);
+                mma_ss(d, dq + off, dk + off, idesc_qk, s > 0 ? 1u : 0u);
+            }
+        };
+        // O_i += P_i V in two halves of 64 keys, each issued as soon as the
+        // softmax has written that half of P_i; false if a wait gave up.
+        auto pv = [&](int i, int st, bool acc, uint32_t par) -> bool {
+            const uint64_t dv = st == 0 ? dv0 : dv1;
+            const uint32_t d = tmem + 256 + 128 * i;
+            const uint32_t a = tmem + 128 * i;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                if (!wait(&bars->p_full[2 * i + hh], par, bars)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int s = 4 * hh; s < 4 * hh + 4; ++s)
+                    mma_ts(d, a + s * 8, dv + (uint64_t)(s * (2048 >> 4)), idesc_pv,
+                           (acc || s > 0) ? 1u : 0u);
+            }
+            return true;
+        };
+        for (int j = 0; ok && j < n_kv; ++j) {
+            const int st = j % kStages;
+            const uint32_t ph = (j / kStages) & 1;
+            const int pst = (j + kStages - 1) % kStages;
+            const uint32_t pph = ((j - 1) / kStages) & 1;
+            if (!(ok = wait(&bars->k_full[st], ph, bars))) break;
+            if (j > 0 && !(ok = wait(&bars->v_full[pst], pph, bars))) break;
+            for (int i = 0; i < ntile; ++i) {
+                if (j > 0 && !(ok = pv(i, pst, j > 1, (j - 1) & 1))) break;
+                tc_fence_after();
+                qk(i, st);
+                mma_commit(&bars->s_full[i]);
+            }
+            if (!ok) break;
+            if (j > 0) mma_commit(&bars->v_empty[pst]);
+            mma_commit(&bars->k_empty[st]);
+        }
+        if (ok) {
+            const int j = n_kv;
+            const int pst = (j - 1) % kStages;
+            const uint32_t pph = ((j - 1) / kStages) & 1;
+            ok = wait(&bars->v_full[pst], pph, bars);
+            for (int i = 0; ok && i < ntile; ++i) {
+                if (!(ok = pv(i, pst, j > 1, (j - 1) & 1))) break;
+                mma_commit(&bars->o_done[i]);
+            }
+            if (ok) mma_commit(&bars->v_empty[pst]);
+        }
+        // make sure nothing this thread issued is still running before TMEM is freed
+        mma_commit(&bars->drain);
+        if (!mbar_wait_bounded(&bars->drain, 0, nullptr, kDrainLimitNs))
+            atomicOr(&g_device_status, 1u);
+    }
     } else {
+        regs_inc<kRegsSoftmax>();
         // ------------------------------------------------------------ softmax warpgroups
         const int i = warp >> 2;        // query tile of this warpgroup
         const int quarter = warp & 3;   // TMEM lanes [32 quarter, 32 quarter + 32)
@@ -314,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
             const uint32_t tS = tmem + i * 128 + lane_off;
             const uint32_t tO = tmem + 256 + i * 128 + lane_off;
             const float sl2 = p.scale_log2;
+            const uint64_t sl2x2 = f2_pack(sl2, sl2);
             float m_run = -INFINITY, l_run = 0.f;
             bool ok = true;
             for (int j = 0; j < n_kv; ++j) {
@@ -332,53 +415,46 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                     for (int c = 0; c < 128; ++c)
                         if (c >= valid) sv[c] = -INFINITY;
                 }
-                float mx = sv[0];
+                // row maximum in 8 independent chains
+                float mk[8];
 #pragma unroll
-                for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
-                const float m_tile = mx * sl2;
+                for (int k = 0; k < 8; ++k) mk[k] = fmaxf(sv[k], sv[k + 8]);
+#pragma unroll
+                for (int c = 16; c < 128; c += 16)
+#pragma unroll
+                    for (int k = 0; k < 8; k += 2)
+                        mk[k] = fmax3(mk[k], sv[c + k], sv[c + k + 1]),
+                        mk[k + 1] = fmax3(mk[k + 1], sv[c + k + 8], sv[c + k + 9]);
+                const float m_tile = fmaxf(fmax3(mk[0], mk[1], mk[2]),
+                                           fmaxf(fmax3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]))) *
+                                     sl2;
                 // Raise the running maximum only when some row of this warp grew
-                // by more than 8 (log2 units); O is then rescaled after P is out
-                // of the registers (the two steps are independent).
-                bool rescale = false;
-                float f = 1.f;
+                // by more than 8 (log2 units); O (which holds PV up to the
+                // previous tile: S(j) ready implies it completed) is rescaled
+                // before any half of this tile's P is released to the MMA.
                 if (j == 0) {
                     m_run = m_tile;
                 } else if (__any_sync(0xffffffffu, m_tile > m_run + 8.0f)) {
                     const float m_new = fmaxf(m_run, m_tile);
-                    f = ex2_approx(m_run - m_new);
+                    const float f = ex2_approx(m_run - m_new);
                     m_run = m_new;
                     l_run *= f;
-                    rescale = true;
+                    rescale_o(tO, f);
                 }
-                const float neg_m = -m_run;
+                // P in two halves of 64 keys: the MMA starts the first half of
+                // P V while the second half of the exponentials is computed.
+                const uint64_t negm2 = f2_pack(-m_run, -m_run);
                 float sum = 0.f;
-                // P packs two keys per 32-bit column; column c only overwrites
-                // register slot c, whose score (slot c <= 2c) is already consumed.
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const float a0 = ex2_approx(fmaf(sv[2 * c], sl2, neg_m));
-                    const float a1 = ex2_approx(fmaf(sv[2 * c + 1], sl2, neg_m));
-                    sum += a0 + a1;
-                    r[c >> 5][c & 31] = pack_bf16x2(a0, a1);
+                for (int h = 0; h < 2; ++h) {
+                    sum += exp_half(sv, r[h], h, sl2x2, negm2);
+                    tmem_st32(tS + 32 * h, r[h]);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->p_full[2 * i + h]);
                 }
                 l_run += sum;
-                tmem_st32(tS, r[0]);
-                tmem_st32(tS + 32, r[1]);
-                if (rescale) {
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + 32 * c, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                        tmem_st32(tO + 32 * c, o);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&bars->p_full[i]);
             }
             // epilogue: O / l  ->  bf16 row of the owning stream
             if (ok) ok = wait_warp(&bars->o_done[i], 0, bars);
@@ -494,12 +570,23 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
     p.q_tiles = q_tiles;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     const int smem = Smem::total + 1024;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(joint_attn_bf16_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return (int)e;
+    static bool attr_set[64] = {false};
+    if (dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        // The register split inside the kernel assumes the launch allocation
+        // is exactly kRegsLaunch per thread; refuse to launch otherwise (a
+        // smaller allocation would leave the increase waiting for ever).
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, joint_attn_bf16_kernel);
         if (e != cudaSuccess) return (int)e;
-        attr_set = true;
+        if (fa.numRegs != kRegsLaunch) return (int)cudaErrorInvalidKernelImage;
+        e = cudaFuncSetAttribute(joint_attn_bf16_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return (int)e;
+        attr_set[dev] = true;
     }
     dim3 grid((q_tiles + 1) / 2, H, B);
     joint_attn_bf16_kernel<<<grid, kThreads, smem, s>>>(p);
