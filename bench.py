@@ -387,6 +387,32 @@ def run_ours(args):
     barrier(group, dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), group, dev) / e2e_steps
 
+    # ---- "next" rows, timed outside the step on the same tensors
+    def time_ms(fn, reps=20):
+        for _ in range(3):
+            fn()
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        z.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(z) / reps
+
+    y_next = torch.empty_like(t["x_vis"])
+    x_next = torch.empty_like(t["x_vis"])
+    rm_ms = time_ms(lambda: api.residual_modulate(
+        t["x_vis"], t["o_vis"].view(B, Nv, C), t["gate_vis"], t["shift_ctx"], t["scale_ctx"],
+        x_out=x_next, y=y_next))
+    q_txt = torch.empty_like(t["q_ctx"])
+    k_txt = torch.empty_like(t["k_ctx"])
+    txt_ms = time_ms(lambda: api.qk_norm_rope_text(
+        t["q_ctx"], t["k_ctx"], t["gq_ctx"], t["gk_ctx"], pos_offset=float(max(w.grid)),
+        q_out=q_txt, k_out=k_txt))
+    if api.device_status() != 0:
+        raise SystemExit("device-side wait timed out in the next-row kernels")
+
     flops = w.attention_flops()
     pk, pk_src = peaks()
     attn_tflops = flops / (kern_ms["joint_attention"] * 1e-3) / 1e12
@@ -434,6 +460,14 @@ def run_ours(args):
                      "peak_kind": f"bf16_tflops_sustained ({pk_src}); attention is timed "
                                   f"inside a multi-second loop of steps"},
         "kernels": kernels,
+        "next_rows": {
+            "residual_modulate_vis": {
+                "ms": rm_ms, "GB/s": 4 * B * Nv * C * 2 / (rm_ms * 1e-3) / 1e9,
+                "frac_hbm": 4 * B * Nv * C * 2 / (rm_ms * 1e-3) / 1e9 / hbm,
+                "unfused_ms": (kern_ms["gated_residual"] + kern_ms["adaln_modulate"]) *
+                              Nv / (Nv + Nc)},
+            "qk_norm_rope_text_ctx": {
+                "ms": txt_ms, "GB/s": 4 * B * Nc * C * 2 / (txt_ms * 1e-3) / 1e9}},
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,

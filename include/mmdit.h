@@ -83,6 +83,30 @@ MMDIT_API int mmdit_qk_norm_rope(const void* q_in, const void* k_in, void* q_out
                        int B, int N, int H, int D, const mmdit_grid* grid, float eps,
                        mmdit_dtype dt, void* stream);
 
+/* Text-token positions of MM-RoPE ["Seaweed-7B: Cost-Effective Training of
+ * Video Generation Foundation Model", section 3.2: text tokens get a 1D
+ * position compatible with the video's 3D one, shared by its three
+ * components]: conditioning token n sits at pos_offset + n on each of the T,
+ * H and W axis chunks (split[] head dims each, frequencies rope_base^(-2j/d)
+ * as for mmdit_grid).  Where the 1D positions start is the caller's choice. */
+typedef struct {
+    float pos_offset;
+    float rope_base;
+    int split[3];
+} mmdit_text_rope;
+
+/* QK-RMSNorm, then the MM-RoPE rotation of text tokens (see mmdit_text_rope):
+ * the same normalisation and rotation as mmdit_qk_norm_rope, with every axis
+ * chunk of token n rotated by the shared position pos_offset + n.  An
+ * alternative to leaving the conditioning stream unrotated.
+ *   q_in, k_in, q_out, k_out, q_scale, k_scale, eps, dt: as mmdit_qk_norm_rope
+ *   rope: host pointer, read during the call only; split[] even, summing to D
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_qk_norm_rope_text(const void* q_in, const void* k_in, void* q_out,
+                                      void* k_out, const float* q_scale, const float* k_scale,
+                                      int B, int N, int H, int D, const mmdit_text_rope* rope,
+                                      float eps, mmdit_dtype dt, void* stream);
+
 /* Joint non-causal attention over the concatenated streams, output split back
  * [Vimoo §2.2: each stream projects its own Q/K/V, one attention runs over the
  * two sequences joined end to end, and its output rows return to the stream
@@ -126,6 +150,24 @@ MMDIT_API int mmdit_adaln_modulate(const void* x, const float* shift, const floa
  * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
 MMDIT_API int mmdit_gated_residual(const void* x, const void* branch, const float* gate, void* out,
                          int B, int N, int C, mmdit_dtype dt, void* stream);
+
+/* Gated residual fused with the adaLN modulate that follows it, in one pass
+ * over memory [Vimoo §2.2: a branch's gated contribution is added to the
+ * residual stream, and the next branch starts from a LayerNorm of that stream
+ * modulated by its own shift and scale]:
+ *   x_out = x + gate[b] * branch                      (stored in dt)
+ *   y     = LN(x_out) * (1 + scale[b]) + shift[b]     (LN of x_out as stored)
+ * Equal to mmdit_gated_residual followed by mmdit_adaln_modulate, with one
+ * read of x fewer.
+ *   x, branch [B, N, C] dt read;  x_out [B, N, C] written (may equal x);
+ *   y [B, N, C] written (must not alias x, branch or x_out)
+ *   gate [B, C] fp32 (this branch);  shift, scale [B, C] fp32 (next branch)
+ *   C % 8 == 0 and C <= 3072 (bf16) / 1536 (f32)
+ * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_residual_modulate(const void* x, const void* branch, const float* gate,
+                                      const float* shift, const float* scale, void* x_out,
+                                      void* y, int B, int N, int C, float eps, mmdit_dtype dt,
+                                      void* stream);
 
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device: MMDIT_OK, or MMDIT_ERR_TIMEOUT if a kernel gave up on a

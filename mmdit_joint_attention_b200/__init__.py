@@ -7,8 +7,8 @@ package does not load the library; the first use of an ``api`` function does,
 and fails loudly if it has not been built."""
 import importlib
 
-_API = ("qk_norm_rope", "joint_attention", "adaln_modulate", "gated_residual",
-        "block_forward", "device_status")
+_API = ("qk_norm_rope", "qk_norm_rope_text", "joint_attention", "adaln_modulate", "gated_residual",
+        "residual_modulate", "block_forward", "device_status")
 __all__ = list(_API)
 
 

@@ -27,6 +27,12 @@ class Grid(ctypes.Structure):
                 ("split", ctypes.c_int * 3)]
 
 
+class TextRope(ctypes.Structure):
+    """mmdit_text_rope: MM-RoPE text positions pos_offset + n on every axis."""
+    _fields_ = [("pos_offset", ctypes.c_float), ("rope_base", ctypes.c_float),
+                ("split", ctypes.c_int * 3)]
+
+
 class MmditError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
@@ -58,16 +64,19 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         L.mmdit_qk_norm_rope.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                          ctypes.POINTER(Grid), _f, _i, _vp]
+        L.mmdit_qk_norm_rope_text.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                              ctypes.POINTER(TextRope), _f, _i, _vp]
         L.mmdit_joint_attention.argtypes = [_vp] * 9 + [_i] * 5 + [_f, _i, _vp]
         L.mmdit_adaln_modulate.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp]
         L.mmdit_gated_residual.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+        L.mmdit_residual_modulate.argtypes = [_vp] * 7 + [_i, _i, _i, _f, _i, _vp]
         L.mmdit_device_status.argtypes = [_vp]
         L.mmdit_last_error.argtypes = []
         L.mmdit_last_error.restype = ctypes.c_char_p
         L.mmdit_status_string.argtypes = [_i]
         L.mmdit_status_string.restype = ctypes.c_char_p
-        for name in ("mmdit_qk_norm_rope", "mmdit_joint_attention", "mmdit_adaln_modulate",
-                     "mmdit_gated_residual", "mmdit_device_status"):
+        for name in ("mmdit_qk_norm_rope", "mmdit_qk_norm_rope_text", "mmdit_joint_attention", "mmdit_adaln_modulate",
+                     "mmdit_gated_residual", "mmdit_residual_modulate", "mmdit_device_status"):
             getattr(L, name).restype = ctypes.c_int
         _LIB = L
     return _LIB

@@ -82,6 +82,32 @@ def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, q_scale: torch.Tensor, k_scal
     return q_out, k_out
 
 
+def qk_norm_rope_text(q: torch.Tensor, k: torch.Tensor, q_scale: torch.Tensor,
+                      k_scale: torch.Tensor, pos_offset: float = 0.0, eps: float = 1e-6,
+                      rope_base: float = 10000.0, split=(16, 56, 56),
+                      q_out: Optional[torch.Tensor] = None, k_out: Optional[torch.Tensor] = None,
+                      stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-head RMSNorm of q and k, then MM-RoPE text positions: token n at
+    pos_offset + n on all three axis chunks.  In place unless outputs are given."""
+    dt = _dtype(q, k)
+    _f32(q_scale, k_scale)
+    B, N, H, D = q.shape
+    if k.shape != q.shape:
+        raise ValueError("q and k shapes differ")
+    q_out = q if q_out is None else q_out
+    k_out = k if k_out is None else k_out
+    r = _lib.TextRope()
+    r.pos_offset = float(pos_offset)
+    r.rope_base = float(rope_base)
+    for a in range(3):
+        r.split[a] = int(split[a])
+    st = _lib.lib().mmdit_qk_norm_rope_text(
+        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _ptr(q_scale), _ptr(k_scale), B, N, H, D,
+        ctypes.byref(r), eps, dt, _stream(stream))
+    check("mmdit_qk_norm_rope_text", st)
+    return q_out, k_out
+
+
 def joint_attention(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
                     softmax_scale: Optional[float] = None, o_vis=None, o_ctx=None,
                     stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
@@ -131,6 +157,24 @@ def gated_residual(x: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor,
                                          dt, _stream(stream))
     check("mmdit_gated_residual", st)
     return out
+
+
+def residual_modulate(x: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor,
+                      shift: torch.Tensor, scale: torch.Tensor, eps: float = 1e-6,
+                      x_out: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                      stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """x_out = x + gate * branch (in place into x unless ``x_out`` is given), then
+    y = LN(x_out) * (1 + scale) + shift, in one pass over memory."""
+    dt = _dtype(x, branch)
+    _f32(gate, shift, scale)
+    B, N, C = x.shape
+    x_out = x if x_out is None else x_out
+    y = torch.empty_like(x) if y is None else y
+    st = _lib.lib().mmdit_residual_modulate(_ptr(x), _ptr(branch), _ptr(gate), _ptr(shift),
+                                            _ptr(scale), _ptr(x_out), _ptr(y), B, N, C, eps, dt,
+                                            _stream(stream))
+    check("mmdit_residual_modulate", st)
+    return x_out, y
 
 
 def device_status(stream=None) -> int:

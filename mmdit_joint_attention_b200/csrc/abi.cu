@@ -81,9 +81,41 @@ int mmdit_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_
         g.base = grid->rope_base;
     }
     return cuda_status(launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_scale, k_scale, B, N, H,
-                                           grid ? &g : nullptr, eps, dt == MMDIT_BF16,
+                                           grid ? &g : nullptr, nullptr, eps, dt == MMDIT_BF16,
                                            static_cast<cudaStream_t>(stream)),
                        "qk_norm_rope");
+}
+
+int mmdit_qk_norm_rope_text(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                            const float* q_scale, const float* k_scale, int B, int N, int H, int D,
+                            const mmdit_text_rope* rope, float eps, mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || N < 0 || H < 0 || !(eps >= 0.f) || !std::isfinite(eps) || !rope)
+        return MMDIT_ERR_ARG;
+    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * N * H == 0) return MMDIT_OK;
+    if (!q_in || !k_in || !q_out || !k_out || !q_scale || !k_scale) return MMDIT_ERR_ARG;
+    if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(q_out) || !aligned16(k_out) ||
+        !aligned16(q_scale) || !aligned16(k_scale))
+        return MMDIT_ERR_ALIGN;
+    if ((long long)B * N * H >= (1LL << 31)) return MMDIT_ERR_UNSUPPORTED;
+    if (!std::isfinite(rope->pos_offset)) return MMDIT_ERR_ARG;
+    if (!(rope->rope_base > 0.f) || !std::isfinite(rope->rope_base)) return MMDIT_ERR_ARG;
+    int sum = 0;
+    for (int a = 0; a < 3; ++a) {
+        if (rope->split[a] < 0 || (rope->split[a] & 1)) return MMDIT_ERR_SHAPE;
+        sum += rope->split[a];
+    }
+    if (sum != D) return MMDIT_ERR_SHAPE;
+    const int E = vec_elems(dt);
+    if (rope->split[0] % E || (rope->split[0] + rope->split[1]) % E) return MMDIT_ERR_UNSUPPORTED;
+    RopeText t{};
+    t.pos_offset = rope->pos_offset;
+    t.base = rope->rope_base;
+    for (int a = 0; a < 3; ++a) t.split[a] = rope->split[a];
+    return cuda_status(launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_scale, k_scale, B, N, H,
+                                           nullptr, &t, eps, dt == MMDIT_BF16,
+                                           static_cast<cudaStream_t>(stream)),
+                       "qk_norm_rope_text");
 }
 
 int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vis,
@@ -149,6 +181,26 @@ int mmdit_gated_residual(const void* x, const void* branch, const float* gate, v
     return cuda_status(launch_gated_residual(x, branch, gate, out, B, N, C, dt == MMDIT_BF16,
                                              static_cast<cudaStream_t>(stream)),
                        "gated_residual");
+}
+
+int mmdit_residual_modulate(const void* x, const void* branch, const float* gate,
+                            const float* shift, const float* scale, void* x_out, void* y, int B,
+                            int N, int C, float eps, mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || N < 0 || C < 0 || !(eps >= 0.f) || !std::isfinite(eps))
+        return MMDIT_ERR_ARG;
+    const int E = vec_elems(dt);
+    if (C == 0 || C % 8 != 0 || C / E > 384) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * N == 0) return MMDIT_OK;
+    if (B > 65535) return MMDIT_ERR_UNSUPPORTED;
+    if (!x || !branch || !gate || !shift || !scale || !x_out || !y) return MMDIT_ERR_ARG;
+    if (y == x || y == branch || y == x_out) return MMDIT_ERR_ARG;
+    if (!aligned16(x) || !aligned16(branch) || !aligned16(gate) || !aligned16(shift) ||
+        !aligned16(scale) || !aligned16(x_out) || !aligned16(y))
+        return MMDIT_ERR_ALIGN;
+    return cuda_status(launch_residual_modulate(x, branch, gate, shift, scale, x_out, y, B, N, C,
+                                                eps, dt == MMDIT_BF16,
+                                                static_cast<cudaStream_t>(stream)),
+                       "residual_modulate");
 }
 
 int mmdit_device_status(void* stream) {

@@ -115,8 +115,14 @@ struct RopeParams {
     int tab_off[3];    // first table entry of each axis
     int tab_entries;
     double pos_scale[3];
+    double pos_offset; // text mode: token n sits at pos_offset + n on every axis
     double freq[64];   // frequency of pair j of axis a at index off[a]/2 + j
 };
+
+// RoPE modes of the norm kernel
+constexpr int kRopeNone = 0;   // conditioning stream without positions
+constexpr int kRopeGrid = 1;   // visual stream: (t, h, w) from the token's grid cell
+constexpr int kRopeText = 2;   // text tokens, MM-RoPE: one position shared by the three axes
 
 // One group of 128/E lanes owns one (token, head): its q row and its k row.
 // Lane g of the group holds head dims [g*E, g*E + E), which lie inside a single
@@ -128,7 +134,7 @@ struct RopeParams {
 // 480p (5.5 TB/s, vs 3.6 TB/s with one unit per group and 64-bit index math).
 constexpr int kQkUnroll = 8;
 
-template <typename T, bool ROPE, bool TABLE, int UNR>
+template <typename T, int ROPE, bool TABLE, int UNR>
 __global__ void __launch_bounds__(256, 2)
 qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
                     const float* __restrict__ gq, const float* __restrict__ gk, uint32_t units,
@@ -139,7 +145,7 @@ qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
     extern __shared__ float4 rope_tab4[];
     const float2* tab = reinterpret_cast<const float2*>(rope_tab4);
 
-    if (ROPE && TABLE) {
+    if (ROPE == kRopeGrid && TABLE) {
         float2* wtab = reinterpret_cast<float2*>(rope_tab4);
         for (int e = threadIdx.x; e < rp.tab_entries; e += blockDim.x) {
             const int a = e < rp.tab_off[1] ? 0 : (e < rp.tab_off[2] ? 1 : 2);
@@ -210,31 +216,40 @@ qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
                 xq[i] *= iq * wq[i];
                 xk[i] *= ik * wk[i];
             }
-            if (ROPE) {
+            if (ROPE != kRopeNone) {
                 const uint32_t uu = u < units ? u : 0;
                 const uint32_t bn = fdiv(uu, rp.H);
                 const uint32_t n = bn - fdiv(bn, rp.N) * rp.N.d;
-                const uint32_t t = fdiv(n, rp.HW);
-                const uint32_t rem = n - t * rp.HW.d;
-                const uint32_t hh = fdiv(rem, rp.W);
-                const uint32_t pos = axis == 0 ? t : (axis == 1 ? hh : rem - hh * rp.W.d);
                 float cs[E];  // (cos, sin) of the lane's E/2 pairs
-                if (TABLE) {
-                    const float4* p4 = reinterpret_cast<const float4*>(
-                        tab + rp.tab_off[axis] + pos * rp.stride[axis] + jb);
+                if (ROPE == kRopeGrid) {
+                    const uint32_t t = fdiv(n, rp.HW);
+                    const uint32_t rem = n - t * rp.HW.d;
+                    const uint32_t hh = fdiv(rem, rp.W);
+                    const uint32_t pos = axis == 0 ? t : (axis == 1 ? hh : rem - hh * rp.W.d);
+                    if (TABLE) {
+                        const float4* p4 = reinterpret_cast<const float4*>(
+                            tab + rp.tab_off[axis] + pos * rp.stride[axis] + jb);
 #pragma unroll
-                    for (int i = 0; i < E / 4; ++i) {
-                        const float4 v = p4[i];
-                        cs[4 * i] = v.x;
-                        cs[4 * i + 1] = v.y;
-                        cs[4 * i + 2] = v.z;
-                        cs[4 * i + 3] = v.w;
+                        for (int i = 0; i < E / 4; ++i) {
+                            const float4 v = p4[i];
+                            cs[4 * i] = v.x;
+                            cs[4 * i + 1] = v.y;
+                            cs[4 * i + 2] = v.z;
+                            cs[4 * i + 3] = v.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int p = 0; p < E / 2; ++p) {
+                            const float ang = (float)((double)pos * rp.pos_scale[axis] *
+                                                      rp.freq[rp.off[axis] / 2 + jb + p]);
+                            sincosf(ang, &cs[2 * p + 1], &cs[2 * p]);
+                        }
                     }
                 } else {
+                    const double pos = rp.pos_offset + (double)n;
 #pragma unroll
                     for (int p = 0; p < E / 2; ++p) {
-                        const float ang = (float)((double)pos * rp.pos_scale[axis] *
-                                                  rp.freq[rp.off[axis] / 2 + jb + p]);
+                        const float ang = (float)(pos * rp.freq[rp.off[axis] / 2 + jb + p]);
                         sincosf(ang, &cs[2 * p + 1], &cs[2 * p]);
                     }
                 }
@@ -258,7 +273,7 @@ qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
     }
 }
 
-template <typename T, bool ROPE, bool TABLE>
+template <typename T, int ROPE, bool TABLE>
 cudaError_t run_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, const float* gq,
                    const float* gk, uint32_t units, float eps, const RopeParams& rp, size_t smem,
                    cudaStream_t s) {
@@ -418,6 +433,97 @@ adaln_modulate_kernel(const T* x, const float* __restrict__ shift,
 
 }
 
+// Gated residual followed by the next adaLN modulate, one pass over memory:
+//   x' = x + gate[b] * branch   (stored, rounded to T)
+//   y  = LN(x') * (1 + scale[b]) + shift[b]
+// The statistics use x' as stored (rounded to T), so the result equals the
+// two separate kernels run back to back.  One warp per row, as above; gate is
+// read through L1, (1 + scale, shift) are staged in shared memory.
+template <typename T, int CPL>
+__global__ void __launch_bounds__(256, 2)
+residual_modulate_kernel(const T* x, const T* br, const float* __restrict__ gate,
+                         const float* __restrict__ shift, const float* __restrict__ scale,
+                         T* x_out, T* y, int N, int C, float eps) {
+    using L = ModLayout<T>;
+    constexpr int E = L::E;
+    constexpr int P = L::PIECES;
+    extern __shared__ float4 mod[];
+    const int b = blockIdx.y;
+    const int nch = C / E;
+    for (int idx = threadIdx.x; idx < nch * P; idx += blockDim.x) {
+        const int c = idx / P, k = idx - (idx / P) * P;
+        float4 v;
+        if (k < P / 2) {
+            v = *reinterpret_cast<const float4*>(scale + (size_t)b * C + c * E + 4 * k);
+            v.x += 1.f;
+            v.y += 1.f;
+            v.z += 1.f;
+            v.w += 1.f;
+        } else {
+            v = *reinterpret_cast<const float4*>(shift + (size_t)b * C + c * E + 4 * (k - P / 2));
+        }
+        mod[L::slot(c, k)] = v;
+    }
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int warps = blockDim.x >> 5;
+    const float invC = 1.0f / (float)C;
+    const size_t base = (size_t)b * N * (size_t)C;
+    const float* g = gate + (size_t)b * C;
+    for (int n = blockIdx.x * warps + (threadIdx.x >> 5); n < N; n += gridDim.x * warps) {
+        const size_t row = base + (size_t)n * C;
+        uint4 raw[CPL], rb[CPL];
+        mod_load<T, CPL>(raw, x, row, nch, lane);
+        mod_load<T, CPL>(rb, br, row, nch, lane);
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int c = lane + 32 * i;
+            if (c < nch) {
+                float fx[E], fb[E];
+                unpack(raw[i], fx);
+                unpack(rb[i], fb);
+#pragma unroll
+                for (int k = 0; k < E / 4; ++k) {
+                    const float4 gv = __ldg(reinterpret_cast<const float4*>(g + c * E) + k);
+                    fx[4 * k] = fmaf(gv.x, fb[4 * k], fx[4 * k]);
+                    fx[4 * k + 1] = fmaf(gv.y, fb[4 * k + 1], fx[4 * k + 1]);
+                    fx[4 * k + 2] = fmaf(gv.z, fb[4 * k + 2], fx[4 * k + 2]);
+                    fx[4 * k + 3] = fmaf(gv.w, fb[4 * k + 3], fx[4 * k + 3]);
+                }
+                raw[i] = pack(fx);
+                st16(x_out + row + (size_t)c * E, raw[i]);
+            }
+        }
+        mod_row<T, CPL>(raw, y, row, nch, lane, invC, eps, mod);
+    }
+}
+
+template <typename T, int CPL>
+cudaError_t run_residual_modulate(const void* x, const void* br, const float* gate,
+                                  const float* shift, const float* scale, void* x_out, void* y,
+                                  int B, int N, int C, float eps, cudaStream_t s) {
+    auto kern = residual_modulate_kernel<T, CPL>;
+    const size_t smem = (size_t)C * 8;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    long long bx = ((long long)sm_count() * per_sm + B - 1) / B;
+    const long long need = (N + 7) / 8;
+    if (need < bx) bx = need;
+    if (bx < 1) bx = 1;
+    dim3 grid((unsigned)bx, (unsigned)B);
+    kern<<<grid, 256, smem, s>>>(static_cast<const T*>(x), static_cast<const T*>(br), gate, shift,
+                                 scale, static_cast<T*>(x_out), static_cast<T*>(y), N, C, eps);
+    return cudaGetLastError();
+}
+
 template <typename T, int CPL>
 cudaError_t run_modulate(const void* x, const float* shift, const float* scale, void* y, int B,
                          int N, int C, float eps, cudaStream_t s) {
@@ -519,7 +625,8 @@ cudaError_t run_residual(const void* x, const void* br, const float* gate, void*
 // ----------------------------------------------------------------------
 cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
                                 const float* gq, const float* gk, int B, int N, int H,
-                                const RopeGrid* grid, float eps, bool bf16, cudaStream_t s) {
+                                const RopeGrid* grid, const RopeText* text, float eps, bool bf16,
+                                cudaStream_t s) {
     const long long units_ll = (long long)B * N * H;
     if (units_ll == 0) return cudaSuccess;
     if (units_ll >= (1LL << 31)) return cudaErrorInvalidValue;  // rejected by the C-ABI layer
@@ -551,21 +658,39 @@ cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out,
         smem = (size_t)toff * sizeof(float2);
         table = smem <= 64 * 1024;
         if (!table) smem = 0;
+    } else if (text) {
+        int off = 0;
+        for (int a = 0; a < 3; ++a) {
+            rp.split[a] = text->split[a];
+            rp.off[a] = off;
+            for (int j = 0; j < text->split[a] / 2; ++j)
+                rp.freq[off / 2 + j] = std::pow(text->base, -2.0 * j / (double)text->split[a]);
+            off += text->split[a];
+        }
+        rp.pos_offset = text->pos_offset;
+        rp.Hg = 1;
+        rp.HW = rp.W = make_fastdiv(1);
     } else {
         rp.off[1] = rp.off[2] = kHeadDim;  // every lane on "axis 0", unused
         rp.Hg = 1;
         rp.HW = rp.W = make_fastdiv(1);
     }
+#define MMDIT_QK_DISPATCH(T)                                                                   \
+    if (text)                                                                                  \
+        return run_qk<T, kRopeText, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, \
+                                           s);                                                  \
+    if (!grid)                                                                                 \
+        return run_qk<T, kRopeNone, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, \
+                                           s);                                                  \
+    if (table)                                                                                 \
+        return run_qk<T, kRopeGrid, true>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp,     \
+                                          smem, s);                                             \
+    return run_qk<T, kRopeGrid, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, s);
     if (bf16) {
-        using T = __nv_bfloat16;
-        if (!grid) return run_qk<T, false, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, s);
-        if (table) return run_qk<T, true, true>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, smem, s);
-        return run_qk<T, true, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, s);
+        MMDIT_QK_DISPATCH(__nv_bfloat16)
     }
-    using T = float;
-    if (!grid) return run_qk<T, false, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, s);
-    if (table) return run_qk<T, true, true>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, smem, s);
-    return run_qk<T, true, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, s);
+    MMDIT_QK_DISPATCH(float)
+#undef MMDIT_QK_DISPATCH
 }
 
 cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float* scale,
@@ -585,6 +710,27 @@ cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float
     MMDIT_MOD_CASE(12)
     MMDIT_MOD_CASE(16)
 #undef MMDIT_MOD_CASE
+    return cudaErrorInvalidValue;  // the C-ABI layer rejects such C before this point
+}
+
+cudaError_t launch_residual_modulate(const void* x, const void* branch, const float* gate,
+                                     const float* shift, const float* scale, void* x_out, void* y,
+                                     int B, int N, int C, float eps, bool bf16, cudaStream_t s) {
+    if ((long long)B * N == 0) return cudaSuccess;
+    const int E = bf16 ? 8 : 4;
+    const int cpl = (C / E + 31) / 32;
+#define MMDIT_RM_CASE(V)                                                                        \
+    if (cpl <= V)                                                                               \
+        return bf16 ? run_residual_modulate<__nv_bfloat16, V>(x, branch, gate, shift, scale,     \
+                                                              x_out, y, B, N, C, eps, s)        \
+                    : run_residual_modulate<float, V>(x, branch, gate, shift, scale, x_out, y,  \
+                                                      B, N, C, eps, s);
+    MMDIT_RM_CASE(1)
+    MMDIT_RM_CASE(2)
+    MMDIT_RM_CASE(4)
+    MMDIT_RM_CASE(8)
+    MMDIT_RM_CASE(12)
+#undef MMDIT_RM_CASE
     return cudaErrorInvalidValue;  // the C-ABI layer rejects such C before this point
 }
 

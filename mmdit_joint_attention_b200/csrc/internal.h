@@ -13,14 +13,26 @@ struct RopeGrid {
     int split[3];
 };
 
-// 0 or a cudaError_t value
+// MM-RoPE positions of text tokens: token n at pos_offset + n on all three axes.
+struct RopeText {
+    double pos_offset;
+    double base;
+    int split[3];
+};
+
+// 0 or a cudaError_t value.  At most one of grid / text is non-null.
 cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
                                 const float* gq, const float* gk, int B, int N, int H,
-                                const RopeGrid* grid, float eps, bool bf16, cudaStream_t s);
+                                const RopeGrid* grid, const RopeText* text, float eps, bool bf16,
+                                cudaStream_t s);
 
 cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float* scale,
                                   void* y, int B, int N, int C, float eps, bool bf16,
                                   cudaStream_t s);
+
+cudaError_t launch_residual_modulate(const void* x, const void* branch, const float* gate,
+                                     const float* shift, const float* scale, void* x_out, void* y,
+                                     int B, int N, int C, float eps, bool bf16, cudaStream_t s);
 
 cudaError_t launch_gated_residual(const void* x, const void* branch, const float* gate,
                                   void* out, int B, int N, int C, bool bf16, cudaStream_t s);

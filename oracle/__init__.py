@@ -42,6 +42,9 @@ def _configure(lib):
     lib.oracle_rmsnorm.argtypes = [dp, dp, dp, ctypes.c_long, ctypes.c_int, ctypes.c_double]
     lib.oracle_rope3d.argtypes = [dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.POINTER(_Grid)]
+    lib.oracle_rope_positions.argtypes = [dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, dp, ctypes.c_double,
+                                          ctypes.POINTER(ctypes.c_int)]
     lib.oracle_joint_attention_rows.argtypes = (
         [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [ctypes.c_int] * 5 +
         [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp])
@@ -86,6 +89,34 @@ def rope3d(x, grid: Tuple[int, int, int], pos_scale=(1.0, 1.0, 1.0), base: float
                (ctypes.c_int * 3)(*split))
     _load().oracle_rope3d(_p(x), B, N, H, D, ctypes.byref(gr))
     return x
+
+
+def rope_positions(x, pos, base: float = 10000.0, split=(16, 56, 56)) -> np.ndarray:
+    """Rotate rows x [B, N, H, D] by explicit per-axis positions pos [N, 3]."""
+    x = _f64(x).copy()
+    B, N, H, D = x.shape
+    pos = _f64(pos).reshape(N, 3)
+    if sum(split) != D:
+        raise ValueError("split does not match D")
+    sp = (ctypes.c_int * 3)(*split)
+    _load().oracle_rope_positions(_p(x), B, N, H, D, _p(pos), base, sp)
+    return x
+
+
+def text_positions(N: int, offset: float = 0.0) -> np.ndarray:
+    """MM-RoPE positions of N text tokens: token n at (offset + n) on all three axes."""
+    p = offset + np.arange(N, dtype=np.float64)
+    return np.stack([p, p, p], axis=1)
+
+
+def qk_norm_rope_text(q, k, gq, gk, offset: float = 0.0, eps: float = 1e-6,
+                      base: float = 10000.0, split=(16, 56, 56)):
+    """QK-RMSNorm, then MM-RoPE with shared 1D text positions (Seaweed-7B report,
+    section 3.2) for the conditioning stream."""
+    qn = rmsnorm(q, gq, eps)
+    kn = rmsnorm(k, gk, eps)
+    pos = text_positions(np.shape(q)[1], offset)
+    return rope_positions(qn, pos, base, split), rope_positions(kn, pos, base, split)
 
 
 def qk_norm_rope(q, k, gq, gk, grid=None, pos_scale=(1.0, 1.0, 1.0), eps: float = 1e-6,
@@ -153,6 +184,15 @@ def gated_residual(x, branch, gate) -> np.ndarray:
     out = np.empty_like(x)
     _load().oracle_gated_residual(_p(x), _p(branch), _p(gate), _p(out), B, N, C)
     return out
+
+
+def residual_modulate(x, branch, gate, shift, scale, eps: float = 1e-6, round_to=None):
+    """Gated residual, then the adaLN modulate of the next branch on its result.
+    ``round_to`` (a function) rounds x' to the storage type before the
+    LayerNorm, as a pipeline that stores x' and reads it back does."""
+    xo = gated_residual(x, branch, gate)
+    xs = round_to(xo) if round_to is not None else xo
+    return xo, adaln_modulate(xs, shift, scale, eps)
 
 
 def block(inp: dict, eps: float = 1e-6):

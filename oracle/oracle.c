@@ -21,6 +21,9 @@
  *            scales;
  *          - LayerNorm before attention with timestep shift / scale, and gates
  *            that control each branch's residual contribution.
+ *   [S]  "Seaweed-7B: Cost-Effective Training of Video Generation Foundation
+ *        Model", section 3.2: MM-RoPE gives text tokens a 1D position that the
+ *        three RoPE components (T, H, W) share.
  *   [W4] "Wan 2.1" technical report (Chinese translation), section 4.2.1
  *        (patchify + flatten of the (T, H, W) latent into a token sequence) and
  *        section 4.3.1 (DiT attention is non-causal).
@@ -84,6 +87,37 @@ void oracle_rope3d(double* x, int B, int N, int H, int D, const oracle_grid* gri
                     double v = row[offset + 2 * j + 1];
                     row[offset + 2 * j]     = u * c - v * s;
                     row[offset + 2 * j + 1] = u * s + v * c;
+                }
+                offset += d_a;
+            }
+        }
+    }
+}
+
+/* ---- RoPE at explicit positions ----------------------------------------------
+ * Same rotation as oracle_rope3d, but token n of x [B, N, H, D] sits at the
+ * per-axis positions pos[3n + a] given by the caller (already scaled).  With
+ * pos = (p, p, p) this is the text-token case of the Seaweed-7B report's
+ * MM-RoPE (section 3.2): a 1D position shared by the three components.        */
+void oracle_rope_positions(double* x, int B, int N, int H, int D, const double* pos,
+                           double rope_base, const int* split)
+{
+    #pragma omp parallel for schedule(static)
+    for (long bn = 0; bn < (long)B * N; ++bn) {
+        int n = (int)(bn % N);
+        for (int hd = 0; hd < H; ++hd) {
+            double* row = x + (bn * H + hd) * (long)D;
+            int offset = 0;
+            for (int a = 0; a < 3; ++a) {
+                int d_a = split[a];
+                double p = pos[3 * (long)n + a];
+                for (int j = 0; j < d_a / 2; ++j) {
+                    double ang = p * pow(rope_base, -2.0 * (double)j / (double)d_a);
+                    double c = cos(ang), sn = sin(ang);
+                    double u = row[offset + 2 * j];
+                    double v = row[offset + 2 * j + 1];
+                    row[offset + 2 * j]     = u * c - v * sn;
+                    row[offset + 2 * j + 1] = u * sn + v * c;
                 }
                 offset += d_a;
             }

@@ -13,6 +13,8 @@ typedef struct {
 
 void oracle_rmsnorm(const double* x, double* y, const double* g, long rows, int D, double eps);
 void oracle_rope3d(double* x, int B, int N, int H, int D, const oracle_grid* grid);
+void oracle_rope_positions(double* x, int B, int N, int H, int D, const double* pos,
+                           double rope_base, const int* split);
 void oracle_joint_attention_rows(const double* qv, const double* kv, const double* vv,
                                  const double* qc, const double* kc, const double* vc,
                                  const int* ctx_len, int B, int Nv, int Nc, int H, int D,

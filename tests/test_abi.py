@@ -17,7 +17,8 @@ def L():
 def test_exports_every_declared_symbol(L):
     names = _lib.declared_functions()
     assert set(names) >= {"mmdit_qk_norm_rope", "mmdit_joint_attention", "mmdit_adaln_modulate",
-                          "mmdit_gated_residual", "mmdit_status_string", "mmdit_device_status"}
+                          "mmdit_gated_residual", "mmdit_residual_modulate",
+                          "mmdit_status_string", "mmdit_device_status", "mmdit_last_error"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -71,3 +72,29 @@ def test_modulate_residual_validation(L):
     assert r(P, P, None, P, 1, 4, 3072, 1, None) == -1
     assert r(P, P, P, U, 1, 4, 3072, 1, None) == -3
     assert r(P, P, P, P, 1, 0, 3072, 1, None) == 0
+
+
+def test_residual_modulate_validation(L):
+    f = L.mmdit_residual_modulate
+    Q = ctypes.c_void_p(32)
+    assert f(P, P, P, P, P, P, Q, 1, 4, 4096, 1e-6, 1, None) == -4     # above 3072 for bf16
+    assert f(P, P, P, P, P, P, Q, 1, 4, 3070, 1e-6, 1, None) == -4
+    assert f(P, P, P, P, P, P, P, 1, 4, 3072, 1e-6, 1, None) == -1     # y aliases x
+    assert f(P, None, P, P, P, P, Q, 1, 4, 3072, 1e-6, 1, None) == -1
+    assert f(P, P, P, U, P, P, Q, 1, 4, 3072, 1e-6, 1, None) == -3
+    assert f(P, P, P, P, P, P, Q, 1, 0, 3072, 1e-6, 1, None) == 0
+
+
+def test_qk_norm_rope_text_validation(L):
+    f = L.mmdit_qk_norm_rope_text
+    r = _lib.TextRope(3.0, 10000.0, (ctypes.c_int * 3)(16, 56, 56))
+    assert f(P, P, P, P, P, P, 1, 8, 2, 128, None, 1e-6, 1, None) == -1          # no rope
+    assert f(P, P, P, P, P, P, 1, 8, 2, 64, ctypes.byref(r), 1e-6, 1, None) == -4
+    r.split[1] = 58
+    assert f(P, P, P, P, P, P, 1, 8, 2, 128, ctypes.byref(r), 1e-6, 1, None) == -2
+    r.split[0], r.split[1] = 12, 60
+    assert f(P, P, P, P, P, P, 1, 8, 2, 128, ctypes.byref(r), 1e-6, 1, None) == -4
+    r.split[0], r.split[1] = 16, 56
+    r.pos_offset = float("inf")
+    assert f(P, P, P, P, P, P, 1, 8, 2, 128, ctypes.byref(r), 1e-6, 1, None) == -1
+    assert f(U, P, P, P, P, P, 1, 8, 2, 128, ctypes.byref(r), 1e-6, 1, None) == -3

@@ -205,3 +205,54 @@ def test_api_rejects_bad_arguments():
     with pytest.raises(api._lib.MmditError) as e:
         api.qk_norm_rope(q, q.clone(), g, g, grid=(2, 4, 5))
     assert e.value.status == -2
+
+
+# ---------------------------------------------------------------- fused residual + modulate
+
+@pytest.mark.parametrize("name", ["tiny", "block", "480p"])
+def test_residual_modulate_fused(name):
+    """x' = x + gate * branch and y = LN(x') (1 + scale) + shift of the next
+    branch in one pass; the LayerNorm reads x' as stored (rounded to the
+    storage type), like the two separate kernels run back to back."""
+    w = W[name]
+    inp = I.make_inputs(w, parts=("qkv", "adaln"))
+    rnd = I.round_f64_to_bf16 if w.dtype == "bf16" else I.round_f64_to_f32
+    n = w.Nv
+    x = to_dev(inp["x_vis"])
+    br = to_dev(inp["v_vis"]).view(w.B, n, w.C)
+    gate, shift, scale = (to_dev(inp[k]) for k in ("gate_vis", "shift_ctx", "scale_ctx"))
+    xo, y = api.residual_modulate(x, br, gate, shift, scale, x_out=torch.empty_like(x))
+    # the unfused pair on the same inputs
+    xo2 = api.gated_residual(x, br, gate, out=torch.empty_like(x))
+    y2 = api.adaln_modulate(xo2, shift, scale)
+    torch.cuda.synchronize()
+    assert torch.equal(xo, xo2) and torch.equal(y, y2)
+    rxo, ry = oracle.residual_modulate(inp["x_vis"].f64, inp["v_vis"].f64.reshape(w.B, n, w.C),
+                                       inp["gate_vis"], inp["shift_ctx"], inp["scale_ctx"],
+                                       round_to=rnd)
+    parity(from_dev(xo), rxo, w.dtype, f"{name} x_out")
+    parity(from_dev(y), ry, w.dtype, f"{name} y")
+    # in place into x
+    api.residual_modulate(x, br, gate, shift, scale, y=y)
+    torch.cuda.synchronize()
+    assert torch.equal(x, xo)
+
+
+# ---------------------------------------------------------------- MM-RoPE text positions
+
+@pytest.mark.parametrize("name,offset", [("tiny", 0.0), ("block", 52.0), ("ragged", 3.0),
+                                         ("480p", 80.0)])
+def test_qk_norm_rope_text(name, offset):
+    """QK-RMSNorm + MM-RoPE text positions (token n at offset + n on all three
+    axis chunks) on the conditioning stream."""
+    w = W[name]
+    inp = I.make_inputs(w, parts=("qkv", "scales"))
+    q, k = to_dev(inp["q_ctx"]), to_dev(inp["k_ctx"])
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+    api.qk_norm_rope_text(q, k, to_dev(inp["gq_ctx"]), to_dev(inp["gk_ctx"]), pos_offset=offset,
+                          q_out=qo, k_out=ko)
+    torch.cuda.synchronize()
+    rq, rk = oracle.qk_norm_rope_text(inp["q_ctx"].f64, inp["k_ctx"].f64, inp["gq_ctx"],
+                                      inp["gk_ctx"], offset=offset)
+    parity(from_dev(qo), rq, w.dtype, f"{name} q_ctx")
+    parity(from_dev(ko), rk, w.dtype, f"{name} k_ctx")

@@ -186,6 +186,47 @@ def pin_rope_brute():
                1e-12)
 
 
+@pin
+def pin_rope_positions_matches_grid_and_brute():
+    """Explicit-position RoPE equals the grid RoPE at the grid's (scaled)
+    positions, and brute-force rotation matrices at arbitrary positions."""
+    g = (2, 3, 4)
+    ps = (1.0, 0.5, 1.5)
+    x = _unit_rows(g, H=2)
+    pos = brute.grid_positions(g) * np.asarray(ps)
+    _close(oracle.rope_positions(x, pos), oracle.rope3d(x, g, pos_scale=ps), 1e-12)
+    rnd = RNG(31).uniform(-20, 60, size=(g[0] * g[1] * g[2], 3))
+    want = np.stack([x[:, n] @ brute.rotation_matrix(rnd[n]).T for n in range(len(rnd))], axis=1)
+    _close(oracle.rope_positions(x, rnd), want, 1e-11)
+
+
+@pin
+def pin_text_rope_shared_position():
+    """MM-RoPE text tokens: position offset + n on all three axes.  Pair 0 of
+    each chunk (dims 0, 16, 72) turns by exactly that position; pair d/4 of the
+    H and W chunks by 0.01 of it; scores depend only on position differences."""
+    N, off = 6, 7.0
+    pos = oracle.text_positions(N, off)
+    assert np.array_equal(pos[:, 0], pos[:, 1]) and np.array_equal(pos[:, 0], pos[:, 2])
+    for d0, dd in ((0, 0), (16, 0), (72, 0), (44, 0.01), (100, 0.01)):
+        x = np.zeros((1, N, 1, 128))
+        x[0, :, 0, d0] = 1.0
+        y = oracle.rope_positions(x, pos)[0, :, 0]
+        for n in range(N):
+            p = (off + n) * (dd if dd else 1.0)
+            _close(y[n, d0:d0 + 2], [math.cos(p), math.sin(p)], 1e-13)
+    r = RNG(32)
+    q, k = r.standard_normal(128), r.standard_normal(128)
+    xq = np.broadcast_to(q, (1, N, 1, 128)).copy()
+    xk = np.broadcast_to(k, (1, N, 1, 128)).copy()
+    rq = oracle.rope_positions(xq, pos)[0, :, 0]
+    rk = oracle.rope_positions(xk, pos)[0, :, 0]
+    for d in (1, 2, 3):
+        s0 = rq[d] @ rk[0]
+        for a in range(1, N - d):
+            assert abs(rq[a + d] @ rk[a] - s0) < 1e-10
+
+
 # ------------------------------------------------------------------- attention
 
 def _qkv(B, Nv, Nc, H, seed, D=128):
@@ -414,9 +455,15 @@ def test_pin(name):
 
 MUTANTS = {
     "rope_sign": ("row[offset + 2 * j]     = u * c - v * s;", "row[offset + 2 * j]     = u * c + v * s;"),
-    "rope_freq": ("-2.0 * (double)j / (double)d_a", "-1.0 * (double)j / (double)d_a"),
+    "rope_freq": ("double freq = pow(grid->rope_base, -2.0 * (double)j / (double)d_a);",
+                  "double freq = pow(grid->rope_base, -1.0 * (double)j / (double)d_a);"),
     "rope_axis_order": ("pos[0] = n / HW;", "pos[0] = n % grid->W;"),
-    "rope_pairing": ("double v = row[offset + 2 * j + 1];", "double v = row[offset + j + d_a / 2];"),
+    "rope_pairing": ("""                    double v = row[offset + 2 * j + 1];
+                    row[offset + 2 * j]     = u * c - v * s;""", """                    double v = row[offset + j + d_a / 2];
+                    row[offset + 2 * j]     = u * c - v * s;"""),
+    "posrope_sign": ("row[offset + 2 * j]     = u * c - v * sn;", "row[offset + 2 * j]     = u * c + v * sn;"),
+    "posrope_freq": ("double ang = p * pow(rope_base, -2.0 * (double)j / (double)d_a);",
+                     "double ang = p * pow(rope_base, -1.0 * (double)j / (double)d_a);"),
     "rms_missing_mean": ("sqrt(ss / (double)D + eps)", "sqrt(ss + eps)"),
     "rms_scale_reversed": ("yr[d] = xr[d] / rms * g[d];", "yr[d] = xr[d] / rms * g[D - 1 - d];"),
     "attn_no_scale": ("s[j] = acc * scale;", "s[j] = acc;"),
@@ -452,3 +499,14 @@ def test_mutants_are_caught(mutant, tmp_path):
     finally:
         oracle._lib = saved
     assert failed, f"mutant {mutant} passed every pin"
+
+
+def test_residual_modulate_is_the_composition():
+    """The fused oracle entry is literally the two defined steps in a row."""
+    r = RNG(30)
+    x = r.standard_normal((2, 5, 64))
+    br = r.standard_normal((2, 5, 64))
+    g, sh, sc = (r.standard_normal((2, 64)) * 0.1 for _ in range(3))
+    xo, y = oracle.residual_modulate(x, br, g, sh, sc)
+    _close(xo, x + g[:, None, :] * br, 1e-14)
+    _close(y, brute.adaln_modulate(x + g[:, None, :] * br, sh, sc), 1e-12)
