@@ -175,6 +175,15 @@ MMDIT_API int mmdit_residual_modulate(const void* x, const void* branch, const f
  * MMDIT_ERR_CUDA if the synchronisation failed. */
 MMDIT_API int mmdit_device_status(void* stream);
 
+/* Sets the limit of one bounded wait inside the attention kernel for launches
+ * made after the call, process-wide: 0 restores the default (2 s).  A wait that
+ * runs out makes every role of the kernel stop (outputs undefined), drain the
+ * copies and tensor-core work it issued, free its tensor memory and return;
+ * the next mmdit_device_status() then reports MMDIT_ERR_TIMEOUT.  No fault or
+ * trap is involved, so the CUDA context stays usable.  Meant for diagnostics
+ * and for testing that path; the default never expires on a healthy GPU. */
+MMDIT_API void mmdit_set_wait_timeout_ns(unsigned long long ns);
+
 /* Text of the CUDA error behind the calling thread's most recent
  * MMDIT_ERR_CUDA return (which call failed and the CUDA error name), or "" if
  * none.  Thread-local storage owned by the library, valid until the thread's

@@ -20,6 +20,9 @@ STATUS = {0: "MMDIT_OK", -1: "MMDIT_ERR_ARG", -2: "MMDIT_ERR_SHAPE", -3: "MMDIT_
           -4: "MMDIT_ERR_UNSUPPORTED", -5: "MMDIT_ERR_CUDA", -6: "MMDIT_ERR_TIMEOUT"}
 
 
+STATUS_CODES = {v: k for k, v in STATUS.items()}
+
+
 class Grid(ctypes.Structure):
     """mmdit_grid: visual token grid (T, H, W) and RoPE parameters."""
     _fields_ = [("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
@@ -52,7 +55,8 @@ def declared_functions():
     """Names of the functions include/mmdit.h declares."""
     with open(HEADER) as f:
         text = f.read()
-    return sorted(set(re.findall(r"^MMDIT_API\s+(?:int|const char\*)\s+(mmdit_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^MMDIT_API\s+(?:int|void|const char\*)\s+(mmdit_\w+)\s*\(",
+                                 text, re.M)))
 
 
 def lib():
@@ -71,6 +75,8 @@ def lib():
         L.mmdit_gated_residual.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
         L.mmdit_residual_modulate.argtypes = [_vp] * 7 + [_i, _i, _i, _f, _i, _vp]
         L.mmdit_device_status.argtypes = [_vp]
+        L.mmdit_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
+        L.mmdit_set_wait_timeout_ns.restype = None
         L.mmdit_last_error.argtypes = []
         L.mmdit_last_error.restype = ctypes.c_char_p
         L.mmdit_status_string.argtypes = [_i]

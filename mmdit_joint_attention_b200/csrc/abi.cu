@@ -210,6 +210,8 @@ int mmdit_device_status(void* stream) {
     return w ? MMDIT_ERR_TIMEOUT : MMDIT_OK;
 }
 
+void mmdit_set_wait_timeout_ns(unsigned long long ns) { set_wait_timeout_ns(ns); }
+
 const char* mmdit_last_error(void) { return g_last_error; }
 
 const char* mmdit_status_string(int status) {

@@ -30,6 +30,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -64,7 +65,7 @@ constexpr int kRegsProducer = 72;
 constexpr int kRegsSoftmax = 216;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsProducer == kThreads * kRegsLaunch,
               "register split must add up to the launch allocation");
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per pipeline wait
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // default: 2 s per pipeline wait
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s per drain wait after an abort
 
 struct Smem {
@@ -87,6 +88,7 @@ struct Params {
     int q_tiles_vis;    // ceil(Nv / 128)
     int q_tiles;        // ceil(Nv / 128) + ceil(Nc / 128)
     float scale_log2;   // softmax_scale * log2(e)
+    uint64_t wait_ns;   // limit of one pipeline wait
 };
 
 struct Bars {
@@ -96,6 +98,7 @@ struct Bars {
     uint64_t s_full[2], o_done[2];
     uint64_t p_full[4];  // [2 i + h]: half h (keys 64h..64h+63) of P_i is in tensor memory
     uint64_t drain;
+    uint64_t wait_ns;   // limit of one pipeline wait (copied from the parameters)
     uint32_t tmem_base;
     uint32_t abort;
 };
@@ -111,7 +114,7 @@ __device__ __forceinline__ void tile_of(const Params& p, int t, int& s, int& row
 }
 
 __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Bars* bars) {
-    if (mbar_wait_bounded(bar, parity, &bars->abort, kWaitLimitNs)) return true;
+    if (mbar_wait_bounded(bar, parity, &bars->abort, bars->wait_ns)) return true;
     bars->abort = 1;
     atomicOr(&g_device_status, 1u);
     return false;
@@ -238,6 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
+        bars->wait_ns = p.wait_ns;
         fence_barrier_init();
     }
     if (warp == kWarpLoad && n_kv > 0) {
@@ -503,6 +507,13 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
 
 namespace {
 
+std::atomic<unsigned long long> g_wait_timeout_ns{0};  // 0: default
+
+uint64_t wait_timeout_ns() {
+    const unsigned long long v = g_wait_timeout_ns.load(std::memory_order_relaxed);
+    return v ? v : attn::kWaitLimitNs;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -569,6 +580,7 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
     p.q_tiles_vis = (Nv + kBlockM - 1) / kBlockM;
     p.q_tiles = q_tiles;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.wait_ns = wait_timeout_ns();
     const int smem = Smem::total + 1024;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -591,6 +603,10 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
     dim3 grid((q_tiles + 1) / 2, H, B);
     joint_attn_bf16_kernel<<<grid, kThreads, smem, s>>>(p);
     return (int)cudaGetLastError();
+}
+
+void set_wait_timeout_ns(unsigned long long ns) {
+    g_wait_timeout_ns.store(ns, std::memory_order_relaxed);
 }
 
 cudaError_t read_and_clear_device_status(unsigned int* out, cudaStream_t s) {

@@ -50,6 +50,9 @@ cudaError_t launch_joint_attention_f32(const float* qv, const float* kv, const f
                                        int Nv, int Nc, int H, float softmax_scale,
                                        cudaStream_t s);
 
+// Limit of one bounded pipeline wait in the attention kernel (0 = default).
+void set_wait_timeout_ns(unsigned long long ns);
+
 // Device status word (bit set = a bounded wait expired): read-and-clear.
 cudaError_t read_and_clear_device_status(unsigned int* out, cudaStream_t s);
 

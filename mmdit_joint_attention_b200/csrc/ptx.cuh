@@ -45,33 +45,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Like mbar_wait_bounded, but polls without letting the thread be suspended
-// (lower wake-up latency, at the cost of issue slots while it spins).
-__device__ __forceinline__ bool mbar_spin_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile uint32_t* abort, uint64_t limit_ns) {
-    if (mbar_test_wait(bar, parity)) return true;
-    const uint64_t start = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_test_wait(bar, parity)) return true;
-        if ((it & 255u) == 0) {
-            if (abort != nullptr && *abort) return false;
-            if (global_timer_ns() - start > limit_ns) return false;
-        }
-    }
-}
-
 // Wait for the phase with the given parity to complete.  Gives up after
 // `limit_ns` of wall time or as soon as *abort (if given) becomes non-zero;
 // returns false then.  Every wait in the kernels goes through here, so no kernel can spin
@@ -79,13 +52,11 @@ __device__ __forceinline__ bool mbar_spin_bounded(uint64_t* bar, uint32_t parity
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile uint32_t* abort, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
-    uint64_t start = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
+    const uint64_t start = global_timer_ns();
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
-            if (abort != nullptr && *abort) return false;
-            if (global_timer_ns() - start > limit_ns) return false;
-        }
+        if (abort != nullptr && *abort) return false;
+        if (global_timer_ns() - start > limit_ns) return false;
     }
 }
 

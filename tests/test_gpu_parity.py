@@ -256,3 +256,42 @@ def test_qk_norm_rope_text(name, offset):
                                       inp["gk_ctx"], offset=offset)
     parity(from_dev(qo), rq, w.dtype, f"{name} q_ctx")
     parity(from_dev(ko), rk, w.dtype, f"{name} k_ctx")
+
+
+# ---------------------------------------------------------------- invariants on the GPU
+
+def test_attention_padded_keys_have_no_influence():
+    """Changing the padded cond keys / values leaves every output bit-identical."""
+    w = SMALL["ragged_small"]
+    inp = I.make_inputs(w, parts=("qkv",))
+    t = device_inputs(inp)
+    a = api.joint_attention(t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"],
+                            t["v_ctx"], t["ctx_len"])
+    for b, L in enumerate(w.ctx_lengths()):
+        t["k_ctx"][b, L:] = 50.0
+        t["v_ctx"][b, L:] = -7.0
+    c = api.joint_attention(t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"],
+                            t["v_ctx"], t["ctx_len"])
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], c[0]) and torch.equal(a[1], c[1])
+
+
+def test_attention_identical_keys_give_mean_v_and_unit_v_gives_one():
+    w = _ws(W["block"], B=2, H=2, grid=(2, 9, 15), Nc=70, ctx_len=(70, 31))
+    inp = I.make_inputs(w, parts=("qkv",))
+    t = device_inputs(inp)
+    t["k_vis"][:] = t["k_vis"][0, 0]
+    t["k_ctx"][:] = t["k_vis"][0, 0]
+    ov, oc = api.joint_attention(t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"],
+                                 t["v_ctx"], t["ctx_len"])
+    v = from_dev(t["v_vis"])
+    vc = from_dev(t["v_ctx"])
+    for b, L in enumerate(w.ctx_lengths()):
+        mean = np.concatenate([v[b], vc[b, :L]], axis=0).mean(axis=0)      # [H, D]
+        parity(from_dev(ov)[b], np.broadcast_to(mean, ov[b].shape), "bf16", "o_vis = mean(V)")
+        parity(from_dev(oc)[b, :L], np.broadcast_to(mean, oc[b, :L].shape), "bf16",
+               "o_ctx = mean(V)")
+    ones_v, ones_c = torch.ones_like(t["v_vis"]), torch.ones_like(t["v_ctx"])
+    ov, oc = api.joint_attention(t["q_vis"], t["k_vis"], ones_v, t["q_ctx"], t["k_ctx"], ones_c,
+                                 t["ctx_len"])
+    parity(from_dev(ov), np.ones(ov.shape), "bf16", "rows sum to one")
