@@ -9,8 +9,10 @@ module only marshals NumPy float64 arrays.  Which page and section each step
 follows is stated beside each function in ``oracle.c``:
 Vimoo 1.0 research page, section 2.2 (QK-RMSNorm, 3D RoPE 16/56/56 on the
 visual stream, joint attention over the concatenated streams with the output
-split back, adaLN modulate, gated residual) and the Wan 2.1 report, sections
-4.2.1 (raster flatten of the patched latent) and 4.3.1 (non-causal attention).
+split back, adaLN modulate, gated residual); the Wan 2.1 report, sections
+4.2.1 (raster flatten of the patched latent) and 4.3.1 (non-causal attention);
+the Seaweed-7B report, section 3.2 (MM-RoPE text positions, 3D window
+attention).
 
 Parity status: every function is pinned by tests in tests/test_oracle_pins.py
 (brute force with explicit rotation matrices and physically concatenated
@@ -47,6 +49,12 @@ def _configure(lib):
                                           ctypes.POINTER(ctypes.c_int)]
     lib.oracle_joint_attention_rows.argtypes = (
         [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [ctypes.c_int] * 5 +
+        [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp])
+    lib.oracle_window_of_tokens.argtypes = [ctypes.POINTER(_Grid), ctypes.POINTER(ctypes.c_int),
+                                            ctypes.POINTER(ctypes.c_int)]
+    lib.oracle_window_attention_rows.argtypes = (
+        [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [ctypes.c_int] * 5 +
+        [ctypes.POINTER(_Grid), ctypes.POINTER(ctypes.c_int)] +
         [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp])
     lib.oracle_adaln_modulate.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3 + [ctypes.c_double]
     lib.oracle_gated_residual.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3
@@ -160,6 +168,69 @@ def joint_attention(qv, kv, vv, qc, kc, vc, ctx_len=None, scale: Optional[float]
     bb, hh, ii = np.meshgrid(np.arange(B), np.arange(H), np.arange(Nv + Nc), indexing="ij")
     rows = np.stack([bb.ravel(), hh.ravel(), ii.ravel()], axis=1)
     out = joint_attention_rows(qv, kv, vv, qc, kc, vc, ctx_len, rows, scale)
+    out = out.reshape(B, H, Nv + Nc, D).transpose(0, 2, 1, 3)
+    return np.ascontiguousarray(out[:, :Nv]), np.ascontiguousarray(out[:, Nv:])
+
+
+def _grid_struct(grid) -> _Grid:
+    return _Grid(grid[0], grid[1], grid[2], (ctypes.c_double * 3)(1.0, 1.0, 1.0), 10000.0,
+                 (ctypes.c_int * 3)(16, 56, 56))
+
+
+def window_of_tokens(grid: Tuple[int, int, int], parts: Tuple[int, int, int]) -> np.ndarray:
+    """Window index of every visual token (raster order) when the (T, H, W) grid
+    is split into parts[a] windows along axis a (Seaweed-7B report, section 3.2;
+    the first extent % parts windows of an axis are one position longer)."""
+    if any(p < 1 or p > e for p, e in zip(parts, grid)):
+        raise ValueError("each axis needs 1 <= parts <= extent")
+    win = np.empty(grid[0] * grid[1] * grid[2], dtype=np.int32)
+    pa = (ctypes.c_int * 3)(*parts)
+    gr = _grid_struct(grid)
+    _load().oracle_window_of_tokens(ctypes.byref(gr), pa,
+                                    win.ctypes.data_as(ctypes.POINTER(ctypes.c_int)))
+    return win
+
+
+def window_attention_rows(qv, kv, vv, qc, kc, vc, ctx_len, grid, parts, rows,
+                          scale: Optional[float] = None):
+    """3D window joint attention for selected query rows (inputs and joint
+    indices in raster order): a visual query sees the visual keys of its own
+    window and every valid conditioning key; a conditioning query sees every
+    valid key."""
+    qv, kv, vv, qc, kc, vc = (_f64(a) for a in (qv, kv, vv, qc, kc, vc))
+    B, Nv, H, D = qv.shape
+    Nc = qc.shape[1]
+    if Nv != grid[0] * grid[1] * grid[2]:
+        raise ValueError("grid does not match Nv")
+    if any(p < 1 or p > e for p, e in zip(parts, grid)):
+        raise ValueError("each axis needs 1 <= parts <= extent")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    out = np.zeros((rows.shape[0], D), dtype=np.float64)
+    if ctx_len is None:
+        cl_p = ctypes.POINTER(ctypes.c_int)()
+    else:
+        cl = np.ascontiguousarray(ctx_len, dtype=np.int32)
+        cl_p = cl.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+    gr = _grid_struct(grid)
+    pa = (ctypes.c_int * 3)(*parts)
+    if rows.shape[0]:
+        _load().oracle_window_attention_rows(
+            _p(qv), _p(kv), _p(vv), _p(qc), _p(kc), _p(vc), cl_p, B, Nv, Nc, H, D,
+            ctypes.byref(gr), pa, scale, rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)),
+            rows.shape[0], _p(out))
+    return out
+
+
+def window_attention(qv, kv, vv, qc, kc, vc, grid, parts, ctx_len=None,
+                     scale: Optional[float] = None):
+    """Full 3D window joint attention; returns (o_vis, o_ctx) in raster order."""
+    B, Nv, H, D = np.shape(qv)
+    Nc = np.shape(qc)[1]
+    bb, hh, ii = np.meshgrid(np.arange(B), np.arange(H), np.arange(Nv + Nc), indexing="ij")
+    rows = np.stack([bb.ravel(), hh.ravel(), ii.ravel()], axis=1)
+    out = window_attention_rows(qv, kv, vv, qc, kc, vc, ctx_len, grid, parts, rows, scale)
     out = out.reshape(B, H, Nv + Nc, D).transpose(0, 2, 1, 3)
     return np.ascontiguousarray(out[:, :Nv]), np.ascontiguousarray(out[:, Nv:])
 

@@ -8,7 +8,10 @@ to pin the C oracle (``oracle.c``).  It shares no code with it:
   * joint attention physically concatenates [visual ; cond] Q, K, V, forms the
     whole score matrix with one matrix product, applies an additive -inf key
     mask, and normalises every row of exp(S - rowmax);
-  * LayerNorm uses numpy's mean / var.
+  * LayerNorm uses numpy's mean / var;
+  * window attention physically gathers each window's tokens (numpy's
+    array_split of the (T, H, W) grid along each axis) and runs the
+    concatenated-sequence attention above on every window separately.
 
 Sources: Vimoo 1.0 research page, section 2.2 (dual-stream joint attention,
 QK-RMSNorm, 3D RoPE 16/56/56, adaLN, gated residual); Wan 2.1 report section
@@ -80,6 +83,31 @@ def joint_attention(qv, kv, vv, qc, kc, vc, ctx_len=None, scale=None):
             O[b, :, h] = P @ V[b, :, h]
         O[b, Nv:][~valid[Nv:]] = 0.0
     return O[:, :Nv], O[:, Nv:]
+
+
+def window_token_lists(grid, parts):
+    """Raster indices of the visual tokens of each window, window-major
+    (T part slowest), each list in raster order."""
+    T, Hp, Wp = grid
+    idx = np.arange(T * Hp * Wp).reshape(T, Hp, Wp)
+    out = []
+    for ts in np.array_split(np.arange(T), parts[0]):
+        for hs in np.array_split(np.arange(Hp), parts[1]):
+            for ws in np.array_split(np.arange(Wp), parts[2]):
+                out.append(idx[np.ix_(ts, hs, ws)].ravel())
+    return out
+
+
+def window_attention(qv, kv, vv, qc, kc, vc, grid, parts, ctx_len=None, scale=None):
+    """Each window's visual rows attend to [window visual ; cond]; cond rows
+    attend to the whole joint sequence."""
+    qv, kv, vv = (np.asarray(a, dtype=np.float64) for a in (qv, kv, vv))
+    ov = np.zeros_like(qv)
+    for toks in window_token_lists(grid, parts):
+        o, _ = joint_attention(qv[:, toks], kv[:, toks], vv[:, toks], qc, kc, vc, ctx_len, scale)
+        ov[:, toks] = o
+    _, oc = joint_attention(qv, kv, vv, qc, kc, vc, ctx_len, scale)
+    return ov, oc
 
 
 def adaln_modulate(x, shift, scale, eps=1e-6):

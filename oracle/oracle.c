@@ -23,7 +23,8 @@
  *            that control each branch's residual contribution.
  *   [S]  "Seaweed-7B: Cost-Effective Training of Video Generation Foundation
  *        Model", section 3.2: MM-RoPE gives text tokens a 1D position that the
- *        three RoPE components (T, H, W) share.
+ *        three RoPE components (T, H, W) share; 3D window attention restricts
+ *        attention to w_t x w_h x w_w windows of the visual grid.
  *   [W4] "Wan 2.1" technical report (Chinese translation), section 4.2.1
  *        (patchify + flatten of the (T, H, W) latent into a token sequence) and
  *        section 4.3.1 (DiT attention is non-causal).
@@ -212,4 +213,98 @@ void oracle_gated_residual(const double* x, const double* branch, const double* 
         for (int c = 0; c < C; ++c)
             out[bn * C + c] = x[bn * C + c] + gate[b * C + c] * branch[bn * C + c];
     }
+}
+
+/* ---- 3D window attention [S] ----------------------------------------------
+ * Seaweed-7B report, section 3.2: the visual tokens are partitioned into
+ * w_t x w_h x w_w windows and attention is computed only within a window
+ * (even layers 1 x 2 x 2, odd layers 4 x 1 x 1).  Readings where the report is
+ * silent:
+ *   - parts[a] is the number of windows along axis a; an axis of extent X
+ *     split into p parts gives the first X % p parts X / p + 1 positions and
+ *     the others X / p (part k starts at k * (X / p) + min(k, X % p));
+ *   - a visual query attends to the visual keys of its own window and to every
+ *     valid conditioning key; a conditioning query attends to every valid key
+ *     (the joint attention above, unchanged).
+ * Inputs are in raster order; rows are (b, h, i) triplets as above.           */
+static int oracle_part_of(int x, int extent, int parts)
+{
+    const int q = extent / parts, r = extent % parts;
+    for (int k = 0; k < parts; ++k) {
+        const int start = k * q + (k < r ? k : r);
+        const int size = q + (k < r ? 1 : 0);
+        if (x >= start && x < start + size) return k;
+    }
+    return -1;
+}
+
+void oracle_window_of_tokens(const oracle_grid* grid, const int* parts, int* win)
+{
+    for (int t = 0; t < grid->T; ++t)
+        for (int h = 0; h < grid->H; ++h)
+            for (int w = 0; w < grid->W; ++w) {
+                const int kt = oracle_part_of(t, grid->T, parts[0]);
+                const int kh = oracle_part_of(h, grid->H, parts[1]);
+                const int kw = oracle_part_of(w, grid->W, parts[2]);
+                win[(t * grid->H + h) * grid->W + w] = (kt * parts[1] + kh) * parts[2] + kw;
+            }
+}
+
+void oracle_window_attention_rows(const double* qv, const double* kv, const double* vv,
+                                  const double* qc, const double* kc, const double* vc,
+                                  const int* ctx_len, int B, int Nv, int Nc, int H, int D,
+                                  const oracle_grid* grid, const int* parts, double scale,
+                                  const long* rows, long nrows, double* out)
+{
+    (void)B;
+    int* win = (int*)malloc(sizeof(int) * (size_t)(Nv > 0 ? Nv : 1));
+    oracle_window_of_tokens(grid, parts, win);
+    #pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)(Nv + Nc + 1));
+        int* key = (int*)malloc(sizeof(int) * (size_t)(Nv + Nc + 1));
+        #pragma omp for schedule(dynamic, 4)
+        for (long r = 0; r < nrows; ++r) {
+            long b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+            int L = ctx_len ? ctx_len[b] : Nc;
+            double* o = out + r * (long)D;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            const double* q;
+            if (i < Nv) {
+                q = qv + ((b * Nv + i) * H + h) * (long)D;
+            } else {
+                if (i >= Nv + L) continue;        /* padded conditioning query: zero */
+                q = qc + ((b * Nc + (i - Nv)) * H + h) * (long)D;
+            }
+            /* the keys this query sees, as joint indices */
+            int nk = 0;
+            for (int j = 0; j < Nv; ++j)
+                if (i >= Nv || win[j] == win[i]) key[nk++] = j;
+            for (int j = 0; j < L; ++j) key[nk++] = Nv + j;
+            if (nk == 0) continue;
+            double m = -INFINITY;
+            for (int e = 0; e < nk; ++e) {
+                const int j = key[e];
+                const double* k = (j < Nv) ? kv + ((b * Nv + j) * H + h) * (long)D
+                                           : kc + ((b * Nc + (j - Nv)) * H + h) * (long)D;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += q[d] * k[d];
+                s[e] = acc * scale;
+                if (s[e] > m) m = s[e];
+            }
+            double den = 0.0;
+            for (int e = 0; e < nk; ++e) {
+                const int j = key[e];
+                double p = exp(s[e] - m);
+                den += p;
+                const double* v = (j < Nv) ? vv + ((b * Nv + j) * H + h) * (long)D
+                                           : vc + ((b * Nc + (j - Nv)) * H + h) * (long)D;
+                for (int d = 0; d < D; ++d) o[d] += p * v[d];
+            }
+            for (int d = 0; d < D; ++d) o[d] /= den;
+        }
+        free(key);
+        free(s);
+    }
+    free(win);
 }

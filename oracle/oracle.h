@@ -19,6 +19,14 @@ void oracle_joint_attention_rows(const double* qv, const double* kv, const doubl
                                  const double* qc, const double* kc, const double* vc,
                                  const int* ctx_len, int B, int Nv, int Nc, int H, int D,
                                  double scale, const long* rows, long nrows, double* out);
+/* Window index (window-major: T part slowest, W part fastest) of every visual
+ * token of the grid, in raster order; parts = windows along T, H, W. */
+void oracle_window_of_tokens(const oracle_grid* grid, const int* parts, int* win);
+void oracle_window_attention_rows(const double* qv, const double* kv, const double* vv,
+                                  const double* qc, const double* kc, const double* vc,
+                                  const int* ctx_len, int B, int Nv, int Nc, int H, int D,
+                                  const oracle_grid* grid, const int* parts, double scale,
+                                  const long* rows, long nrows, double* out);
 void oracle_adaln_modulate(const double* x, const double* shift, const double* scale,
                            double* y, int B, int N, int C, double eps);
 void oracle_gated_residual(const double* x, const double* branch, const double* gate,

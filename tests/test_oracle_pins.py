@@ -7,8 +7,9 @@ the definition reduces to (torch float64 scaled_dot_product_attention and
 layer_norm), closed forms (tests/golden/rope_closed_form.json) and invariants
 (RoPE preserves norms and is relative; softmax rows sum to one; identical keys
 give mean(V); masked keys have no influence; constant-scale RMSNorm has RMS
-equal to the scale).  Sources: Vimoo 1.0 research page, section 2.2; Wan 2.1
-report sections 4.2.1 and 4.3.1.
+equal to the scale; a window sees nothing outside itself).  Sources: Vimoo
+1.0 research page, section 2.2; Wan 2.1 report sections 4.2.1 and 4.3.1;
+Seaweed-7B report, section 3.2.
 
 ``test_mutants_are_caught`` plants plausible mistakes in copies of the
 oracle's C source and checks that at least one pin fails for each.
@@ -446,6 +447,89 @@ def pin_block_brute():
     _close(r["y_ctx"], brute.adaln_modulate(inp["x_ctx"].f64, inp["shift_ctx"], inp["scale_ctx"]), 1e-12)
 
 
+# ------------------------------------------------------- 3D window attention
+
+def _window_case(seed, grid, Nc=6, B=2, H=2, ctx_len=(6, 3)):
+    r = RNG(seed)
+    Nv = grid[0] * grid[1] * grid[2]
+    qv, kv, vv = (r.standard_normal((B, Nv, H, 128)) for _ in range(3))
+    qc, kc, vc = (r.standard_normal((B, Nc, H, 128)) for _ in range(3))
+    return (qv, kv, vv, qc, kc, vc), (None if ctx_len is None else np.array(ctx_len, np.int32))
+
+
+@pin
+def pin_window_brute():
+    """Seaweed-7B section 3.2 windows against a brute force that gathers each
+    window with numpy's array_split and attends over [window ; cond]."""
+    grid = (5, 6, 7)
+    t, cl = _window_case(40, grid)
+    for parts in ((1, 2, 2), (4, 1, 1), (2, 3, 2), (5, 1, 3)):
+        ov, oc = oracle.window_attention(*t, grid, parts, cl)
+        bv, bc = brute.window_attention(*t, grid, parts, cl)
+        _close(ov, bv, 1e-12)
+        _close(oc, bc, 1e-12)
+
+
+@pin
+def pin_window_single_is_joint():
+    """One window over the whole grid is plain joint attention."""
+    grid = (3, 4, 5)
+    t, cl = _window_case(41, grid)
+    ov, oc = oracle.window_attention(*t, grid, (1, 1, 1), cl)
+    jv, jc = brute.joint_attention(*t, cl)
+    _close(ov, jv, 1e-12)
+    _close(oc, jc, 1e-12)
+
+
+@pin
+def pin_window_singletons():
+    """parts = grid extents puts every token in its own window: with no
+    conditioning keys a visual row sees only itself, so its output is its V."""
+    grid = (2, 3, 4)
+    t, _ = _window_case(42, grid, Nc=0, ctx_len=None)
+    ov, _ = oracle.window_attention(*t, grid, grid)
+    _close(ov, t[2], 1e-15)
+
+
+@pin
+def pin_window_locality():
+    """Changing K and V of the tokens outside a window leaves that window's
+    visual rows unchanged but changes the conditioning rows."""
+    grid = (4, 6, 6)
+    parts = (2, 2, 3)
+    t, cl = _window_case(43, grid)
+    win = brute.window_token_lists(grid, parts)
+    inside = win[5]
+    outside = np.setdiff1d(np.arange(grid[0] * grid[1] * grid[2]), inside)
+    qv, kv, vv, qc, kc, vc = t
+    kv2, vv2 = kv.copy(), vv.copy()
+    kv2[:, outside] += 3.0
+    vv2[:, outside] *= -2.0
+    a_v, a_c = oracle.window_attention(qv, kv, vv, qc, kc, vc, grid, parts, cl)
+    b_v, b_c = oracle.window_attention(qv, kv2, vv2, qc, kc, vc, grid, parts, cl)
+    _close(a_v[:, inside], b_v[:, inside], 0.0)
+    assert np.max(np.abs(a_c - b_c)) > 1e-3
+    assert np.max(np.abs(a_v[:, outside] - b_v[:, outside])) > 1e-3
+
+
+@pin
+def pin_window_sizes():
+    """Window sizes of the pages' 480p latent grid (21 x 30 x 52): 1x2x2 gives
+    four windows of 21*15*26 tokens; 4x1x1 splits the 21 frames 6/5/5/5."""
+    win = oracle.window_of_tokens((21, 30, 52), (1, 2, 2))
+    assert win.min() == 0 and win.max() == 3
+    assert np.bincount(win).tolist() == [8190] * 4
+    win = oracle.window_of_tokens((21, 30, 52), (4, 1, 1))
+    assert win.min() == 0
+    assert np.bincount(win).tolist() == [6 * 1560, 5 * 1560, 5 * 1560, 5 * 1560]
+    assert win[0] == 0 and win[6 * 1560 - 1] == 0 and win[6 * 1560] == 1
+    # 720p: 45 rows split 23/22, 80 columns 40/40; raster token (t, h, w) = (0, 23, 40)
+    win = oracle.window_of_tokens((21, 45, 80), (1, 2, 2))
+    assert win.min() == 0
+    assert np.bincount(win).tolist() == [21 * 23 * 40, 21 * 23 * 40, 21 * 22 * 40, 21 * 22 * 40]
+    assert win[23 * 80 + 40] == 3 and win[22 * 80 + 39] == 0
+
+
 @pytest.mark.parametrize("name", sorted(PINS))
 def test_pin(name):
     PINS[name]()
@@ -473,6 +557,16 @@ MUTANTS = {
     "ln_unbiased_var": ("var /= (double)C;", "var /= (double)(C - 1);"),
     "ln_missing_one_plus": ("* (1.0 + scale[b * C + c])", "* (scale[b * C + c])"),
     "residual_gate_index": ("gate[b * C + c] * branch", "gate[c] * branch"),
+    "window_no_remainder": ("const int size = q + (k < r ? 1 : 0);", "const int size = q;"),
+    "window_remainder_last": ("const int start = k * q + (k < r ? k : r);",
+                              "const int start = k * q + (k > parts - 1 - r ? k - (parts - r) : 0);"),
+    "window_axis_parts": ("const int kh = oracle_part_of(h, grid->H, parts[1]);",
+                          "const int kh = oracle_part_of(h, grid->H, parts[2]);"),
+    "window_cond_queries_windowed": ("if (i >= Nv || win[j] == win[i]) key[nk++] = j;",
+                                     "if (win[j] == win[i < Nv ? i : 0]) key[nk++] = j;"),
+    "window_padded_rows_not_zero": ("if (i >= Nv + L) continue;", "if (i >= Nv + Nc) continue;"),
+    "window_no_cond_keys": ("for (int j = 0; j < L; ++j) key[nk++] = Nv + j;",
+                            "for (int j = 0; j < L && i >= Nv; ++j) key[nk++] = Nv + j;"),
 }
 
 
