@@ -79,6 +79,23 @@ def recorded_traffic():
     return float(m.group(1))
 
 
+def window_sizes(grid, parts):
+    """Token counts of the 3D windows (parts windows per axis, the first
+    extent % parts of an axis one position longer)."""
+    ext = [[X // p + (1 if k < X % p else 0) for k in range(p)] for X, p in zip(grid, parts)]
+    return [a * b * c for a in ext[0] for b in ext[1] for c in ext[2]]
+
+
+def window_attention_flops(w: I.Workload, parts) -> float:
+    """4 * D per (query, key) pair over valid pairs: visual rows see their
+    window plus the valid cond keys, cond rows see every valid key."""
+    sizes = window_sizes(w.grid, parts)
+    total = 0
+    for L in w.ctx_lengths():
+        total += sum(n * (n + L) for n in sizes) + L * (w.Nv + L)
+    return 4.0 * w.D * w.H * total
+
+
 def workload_bytes(w: I.Workload):
     """Algorithmic HBM bytes per step of each bandwidth-bound kernel (bf16)."""
     e = 2
@@ -410,6 +427,32 @@ def run_ours(args):
     txt_ms = time_ms(lambda: api.qk_norm_rope_text(
         t["q_ctx"], t["k_ctx"], t["gq_ctx"], t["gk_ctx"], pos_offset=float(max(w.grid)),
         q_out=q_txt, k_out=k_txt))
+    # 3D window attention (1x2x2 and 4x1x1 windows): permuting prologue for
+    # q/k, row permutation of v, windowed attention back to raster order
+    win_rows = {}
+    for parts in ((1, 2, 2), (4, 1, 1)):
+        tag = "x".join(map(str, parts))
+        qw, kw = api.qk_norm_rope_window(t["q_vis"], t["k_vis"], t["gq_vis"], t["gk_vis"],
+                                         w.grid, parts, pos_scale=w.pos_scale)
+        vw = api.window_permute(t["v_vis"], w.grid, parts)
+        pro_ms = time_ms(lambda: api.qk_norm_rope_window(
+            t["q_vis"], t["k_vis"], t["gq_vis"], t["gk_vis"], w.grid, parts,
+            pos_scale=w.pos_scale, q_out=qw, k_out=kw))
+        perm_ms = time_ms(lambda: api.window_permute(t["v_vis"], w.grid, parts, out=vw))
+        att_ms = time_ms(lambda: api.joint_window_attention(
+            qw, kw, vw, t["q_ctx"], t["k_ctx"], t["v_ctx"], w.grid, parts, t["ctx_len"],
+            o_vis=t["o_vis"], o_ctx=t["o_ctx"]), reps=10)
+        wfl = window_attention_flops(w, parts)
+        vbytes = 2 * B * Nv * C * 2
+        win_rows["window_" + tag] = {
+            "attention_ms": att_ms, "attention_TFLOP/s": wfl / (att_ms * 1e-3) / 1e12,
+            "frac_bf16_sustained": wfl / (att_ms * 1e-3) / 1e12 / float(
+                peaks()[0]["bf16_tflops_sustained"]),
+            "attention_flops": wfl, "density_vs_full": wfl / w.attention_flops(),
+            "qk_norm_rope_window_ms": pro_ms,
+            "qk_norm_rope_window_GB/s": 2 * vbytes / (pro_ms * 1e-3) / 1e9,
+            "v_permute_ms": perm_ms, "v_permute_GB/s": vbytes / (perm_ms * 1e-3) / 1e9}
+        del qw, kw, vw
     if api.device_status() != 0:
         raise SystemExit("device-side wait timed out in the next-row kernels")
 
@@ -467,7 +510,8 @@ def run_ours(args):
                 "unfused_ms": (kern_ms["gated_residual"] + kern_ms["adaln_modulate"]) *
                               Nv / (Nv + Nc)},
             "qk_norm_rope_text_ctx": {
-                "ms": txt_ms, "GB/s": 4 * B * Nc * C * 2 / (txt_ms * 1e-3) / 1e9}},
+                "ms": txt_ms, "GB/s": 4 * B * Nc * C * 2 / (txt_ms * 1e-3) / 1e9},
+            **win_rows},
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,

@@ -132,6 +132,60 @@ MMDIT_API int mmdit_joint_attention(const void* q_vis, const void* k_vis, const 
                           int B, int Nv, int Nc, int H, int D, float softmax_scale,
                           mmdit_dtype dt, void* stream);
 
+/* 3D window partition of the visual grid ["Seaweed-7B", section 3.2: attention
+ * restricted to w_t x w_h x w_w windows, e.g. 1x2x2 and 4x1x1 in alternating
+ * layers].  parts[a] is the number of windows along axis a (T, H, W), each in
+ * [1, extent of the axis], product at most 64.  An axis of extent X split into
+ * p windows: window k starts at k*(X/p) + min(k, X%p); the first X%p windows
+ * are one position longer.
+ * Window-major token order: windows one after another, T part slowest, W part
+ * fastest; inside a window its tokens keep raster order. */
+typedef struct {
+    int parts[3];
+} mmdit_window;
+
+/* mmdit_qk_norm_rope for the visual stream, storing the rows in window-major
+ * order for mmdit_joint_window_attention: row (b, n, h) of q_in / k_in
+ * (raster order, RoPE at its grid position) is written to row
+ * (b, window_major(n), h) of q_out / k_out.
+ *   Arguments as mmdit_qk_norm_rope (grid required); win: host pointer.
+ *   q_out, k_out must not overlap q_in or k_in.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_qk_norm_rope_window(const void* q_in, const void* k_in, void* q_out,
+                                        void* k_out, const float* q_scale, const float* k_scale,
+                                        int B, int N, int H, int D, const mmdit_grid* grid,
+                                        const mmdit_window* win, float eps, mmdit_dtype dt,
+                                        void* stream);
+
+/* Reorders rows of C elements between raster and window-major order:
+ * inverse == 0: y[b, window_major(n)] = x[b, n]; otherwise
+ * y[b, n] = x[b, window_major(n)].  Used for v (C = H*D) before
+ * mmdit_joint_window_attention; a pure copy.
+ *   x, y [B, N, C] dt, N == T*H*W of grid, C*sizeof(dt) a multiple of 16;
+ *   y must not overlap x.  grid, win: host pointers (only T, H, W are read).
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_window_permute(const void* x, void* y, int B, int N, int C,
+                                   const mmdit_grid* grid, const mmdit_window* win, int inverse,
+                                   mmdit_dtype dt, void* stream);
+
+/* Joint attention restricted to 3D windows ["Seaweed-7B", section 3.2, with
+ * the joint streams of Vimoo §2.2]: a visual query row attends to the visual
+ * keys of its own window and to every valid conditioning key; a conditioning
+ * query row attends to every valid key, as in mmdit_joint_attention.
+ *   q_vis, k_vis, v_vis  [B, Nv, H, D] dt in WINDOW-MAJOR order (as written
+ *                        by mmdit_qk_norm_rope_window / mmdit_window_permute)
+ *   o_vis [B, Nv, H, D] dt written in RASTER order
+ *   grid, win: host pointers; Nv == T*H*W (only T, H, W are read)
+ *   everything else as mmdit_joint_attention.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_joint_window_attention(const void* q_vis, const void* k_vis,
+                                           const void* v_vis, const void* q_ctx,
+                                           const void* k_ctx, const void* v_ctx,
+                                           const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                                           int B, int Nv, int Nc, int H, int D,
+                                           const mmdit_grid* grid, const mmdit_window* win,
+                                           float softmax_scale, mmdit_dtype dt, void* stream);
+
 /* adaLN modulate [Vimoo §2.2: a LayerNorm sits before attention and the FFN,
  * and the timestep embedding supplies a shift and a scale for its output]:
  *   y = LN(x) * (1 + scale[b]) + shift[b], LN over C without an affine,

@@ -36,6 +36,11 @@ class TextRope(ctypes.Structure):
                 ("split", ctypes.c_int * 3)]
 
 
+class Window(ctypes.Structure):
+    """mmdit_window: number of 3D windows along T, H, W."""
+    _fields_ = [("parts", ctypes.c_int * 3)]
+
+
 class MmditError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
@@ -70,7 +75,15 @@ def lib():
                                          ctypes.POINTER(Grid), _f, _i, _vp]
         L.mmdit_qk_norm_rope_text.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                               ctypes.POINTER(TextRope), _f, _i, _vp]
+        L.mmdit_qk_norm_rope_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                                ctypes.POINTER(Grid), ctypes.POINTER(Window),
+                                                _f, _i, _vp]
+        L.mmdit_window_permute.argtypes = [_vp, _vp, _i, _i, _i, ctypes.POINTER(Grid),
+                                           ctypes.POINTER(Window), _i, _i, _vp]
         L.mmdit_joint_attention.argtypes = [_vp] * 9 + [_i] * 5 + [_f, _i, _vp]
+        L.mmdit_joint_window_attention.argtypes = ([_vp] * 9 + [_i] * 5 +
+                                                   [ctypes.POINTER(Grid), ctypes.POINTER(Window),
+                                                    _f, _i, _vp])
         L.mmdit_adaln_modulate.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp]
         L.mmdit_gated_residual.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
         L.mmdit_residual_modulate.argtypes = [_vp] * 7 + [_i, _i, _i, _f, _i, _vp]
@@ -81,7 +94,9 @@ def lib():
         L.mmdit_last_error.restype = ctypes.c_char_p
         L.mmdit_status_string.argtypes = [_i]
         L.mmdit_status_string.restype = ctypes.c_char_p
-        for name in ("mmdit_qk_norm_rope", "mmdit_qk_norm_rope_text", "mmdit_joint_attention", "mmdit_adaln_modulate",
+        for name in ("mmdit_qk_norm_rope", "mmdit_qk_norm_rope_text", "mmdit_qk_norm_rope_window",
+                     "mmdit_window_permute", "mmdit_joint_attention",
+                     "mmdit_joint_window_attention", "mmdit_adaln_modulate",
                      "mmdit_gated_residual", "mmdit_residual_modulate", "mmdit_device_status"):
             getattr(L, name).restype = ctypes.c_int
         _LIB = L

@@ -132,6 +132,86 @@ def joint_attention(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
     return o_vis, o_ctx
 
 
+def make_window(parts: Sequence[int]) -> _lib.Window:
+    w = _lib.Window()
+    for a in range(3):
+        w.parts[a] = int(parts[a])
+    return w
+
+
+def qk_norm_rope_window(q: torch.Tensor, k: torch.Tensor, q_scale: torch.Tensor,
+                        k_scale: torch.Tensor, grid: Sequence[int], parts: Sequence[int],
+                        pos_scale=(1.0, 1.0, 1.0), eps: float = 1e-6, rope_base: float = 10000.0,
+                        split=(16, 56, 56), q_out: Optional[torch.Tensor] = None,
+                        k_out: Optional[torch.Tensor] = None,
+                        stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """qk_norm_rope of the visual stream (raster order in) with the rows stored
+    in the window-major order of the 3D window partition ``parts`` = (windows
+    along T, H, W).  Outputs are new tensors unless q_out / k_out are given
+    (never the inputs)."""
+    dt = _dtype(q, k)
+    _f32(q_scale, k_scale)
+    B, N, H, D = q.shape
+    if k.shape != q.shape:
+        raise ValueError("q and k shapes differ")
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    g = make_grid(grid, pos_scale, rope_base, split)
+    w = make_window(parts)
+    st = _lib.lib().mmdit_qk_norm_rope_window(
+        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _ptr(q_scale), _ptr(k_scale), B, N, H, D,
+        ctypes.byref(g), ctypes.byref(w), eps, dt, _stream(stream))
+    check("mmdit_qk_norm_rope_window", st)
+    return q_out, k_out
+
+
+def window_permute(x: torch.Tensor, grid: Sequence[int], parts: Sequence[int],
+                   inverse: bool = False, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Reorder the token rows of x [B, N, ...] (N = T*H*W) from raster to
+    window-major order (inverse: back to raster)."""
+    dt = _dtype(x)
+    B, N = x.shape[0], x.shape[1]
+    C = x.numel() // max(B * N, 1)
+    y = torch.empty_like(x) if out is None else out
+    g = make_grid(grid)
+    w = make_window(parts)
+    st = _lib.lib().mmdit_window_permute(_ptr(x), _ptr(y), B, N, C, ctypes.byref(g),
+                                         ctypes.byref(w), 1 if inverse else 0, dt,
+                                         _stream(stream))
+    check("mmdit_window_permute", st)
+    return y
+
+
+def joint_window_attention(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, grid: Sequence[int],
+                           parts: Sequence[int], ctx_len=None,
+                           softmax_scale: Optional[float] = None, o_vis=None, o_ctx=None,
+                           stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """3D window joint attention.  The visual q/k/v are in window-major order
+    (as qk_norm_rope_window / window_permute write them); o_vis comes back in
+    raster order.  A visual row sees its own window plus the valid
+    conditioning keys; a conditioning row sees every valid key."""
+    dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx)
+    B, Nv, H, D = q_vis.shape
+    Nc = q_ctx.shape[1]
+    if o_vis is None:
+        o_vis = torch.empty_like(q_vis)
+    if o_ctx is None:
+        o_ctx = torch.empty_like(q_ctx)
+    if ctx_len is not None and (ctx_len.dtype != torch.int32 or not ctx_len.is_cuda):
+        raise TypeError("ctx_len must be an int32 CUDA tensor")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    g = make_grid(grid)
+    w = make_window(parts)
+    st = _lib.lib().mmdit_joint_window_attention(
+        _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), B, Nv, Nc, H, D, ctypes.byref(g),
+        ctypes.byref(w), softmax_scale, dt, _stream(stream))
+    check("mmdit_joint_window_attention", st)
+    return o_vis, o_ctx
+
+
 def adaln_modulate(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
                    eps: float = 1e-6, out: Optional[torch.Tensor] = None,
                    stream=None) -> torch.Tensor:

@@ -39,6 +39,51 @@ bool dtype_ok(mmdit_dtype dt) { return dt == MMDIT_F32 || dt == MMDIT_BF16; }
 // Elements per 16-byte vector.
 int vec_elems(mmdit_dtype dt) { return dt == MMDIT_BF16 ? 8 : 4; }
 
+int elem_bytes(mmdit_dtype dt) { return dt == MMDIT_BF16 ? 2 : 4; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+// Validates a RoPE grid for N tokens of head dim D and converts it.
+int check_grid(const mmdit_grid* grid, long long N, int D, mmdit_dtype dt, RopeGrid& g) {
+    if (grid->T < 1 || grid->H < 1 || grid->W < 1) return MMDIT_ERR_SHAPE;
+    if ((long long)grid->T * grid->H * grid->W != N) return MMDIT_ERR_SHAPE;
+    int sum = 0;
+    for (int a = 0; a < 3; ++a) {
+        if (grid->split[a] < 0 || (grid->split[a] & 1)) return MMDIT_ERR_SHAPE;
+        sum += grid->split[a];
+        if (!std::isfinite(grid->pos_scale[a])) return MMDIT_ERR_ARG;
+    }
+    if (sum != D) return MMDIT_ERR_SHAPE;
+    if (!(grid->rope_base > 0.f) || !std::isfinite(grid->rope_base)) return MMDIT_ERR_ARG;
+    // every 16-byte vector of head dims must sit inside one axis chunk
+    const int E = vec_elems(dt);
+    if (grid->split[0] % E || (grid->split[0] + grid->split[1]) % E) return MMDIT_ERR_UNSUPPORTED;
+    g.T = grid->T;
+    g.H = grid->H;
+    g.W = grid->W;
+    for (int a = 0; a < 3; ++a) {
+        g.pos_scale[a] = grid->pos_scale[a];
+        g.split[a] = grid->split[a];
+    }
+    g.base = grid->rope_base;
+    return MMDIT_OK;
+}
+
+// Validates a window partition of the grid's T, H, W extents.
+int check_window(const mmdit_grid* grid, const mmdit_window* win) {
+    const int extent[3] = {grid->T, grid->H, grid->W};
+    long long count = 1;
+    for (int a = 0; a < 3; ++a) {
+        if (extent[a] < 1) return MMDIT_ERR_SHAPE;
+        if (win->parts[a] < 1 || win->parts[a] > extent[a]) return MMDIT_ERR_SHAPE;
+        count *= win->parts[a];
+    }
+    return count <= kMaxWindows ? MMDIT_OK : MMDIT_ERR_UNSUPPORTED;
+}
+
 }  // namespace
 
 extern "C" {
@@ -57,33 +102,66 @@ int mmdit_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_
     if ((long long)B * N * H >= (1LL << 31)) return MMDIT_ERR_UNSUPPORTED;
     RopeGrid g{};
     if (grid) {
-        if (grid->T < 1 || grid->H < 1 || grid->W < 1) return MMDIT_ERR_SHAPE;
-        if ((long long)grid->T * grid->H * grid->W != (long long)N) return MMDIT_ERR_SHAPE;
-        int sum = 0;
-        for (int a = 0; a < 3; ++a) {
-            if (grid->split[a] < 0 || (grid->split[a] & 1)) return MMDIT_ERR_SHAPE;
-            sum += grid->split[a];
-            if (!std::isfinite(grid->pos_scale[a])) return MMDIT_ERR_ARG;
-        }
-        if (sum != D) return MMDIT_ERR_SHAPE;
-        if (!(grid->rope_base > 0.f) || !std::isfinite(grid->rope_base)) return MMDIT_ERR_ARG;
-        // every 16-byte vector of head dims must sit inside one axis chunk
-        const int E = vec_elems(dt);
-        if (grid->split[0] % E || (grid->split[0] + grid->split[1]) % E)
-            return MMDIT_ERR_UNSUPPORTED;
-        g.T = grid->T;
-        g.H = grid->H;
-        g.W = grid->W;
-        for (int a = 0; a < 3; ++a) {
-            g.pos_scale[a] = grid->pos_scale[a];
-            g.split[a] = grid->split[a];
-        }
-        g.base = grid->rope_base;
+        const int r = check_grid(grid, N, D, dt, g);
+        if (r != MMDIT_OK) return r;
     }
     return cuda_status(launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_scale, k_scale, B, N, H,
-                                           grid ? &g : nullptr, nullptr, eps, dt == MMDIT_BF16,
-                                           static_cast<cudaStream_t>(stream)),
+                                           grid ? &g : nullptr, nullptr, nullptr, eps,
+                                           dt == MMDIT_BF16, static_cast<cudaStream_t>(stream)),
                        "qk_norm_rope");
+}
+
+int mmdit_qk_norm_rope_window(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                              const float* q_scale, const float* k_scale, int B, int N, int H,
+                              int D, const mmdit_grid* grid, const mmdit_window* win, float eps,
+                              mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || N < 0 || H < 0 || !(eps >= 0.f) || !std::isfinite(eps) ||
+        !grid || !win)
+        return MMDIT_ERR_ARG;
+    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
+    RopeGrid g{};
+    int r = check_grid(grid, N, D, dt, g);
+    if (r != MMDIT_OK) return r;
+    if ((r = check_window(grid, win)) != MMDIT_OK) return r;
+    if ((long long)B * N * H == 0) return MMDIT_OK;
+    if (!q_in || !k_in || !q_out || !k_out || !q_scale || !k_scale) return MMDIT_ERR_ARG;
+    if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(q_out) || !aligned16(k_out) ||
+        !aligned16(q_scale) || !aligned16(k_scale))
+        return MMDIT_ERR_ALIGN;
+    if ((long long)B * N * H >= (1LL << 31)) return MMDIT_ERR_UNSUPPORTED;
+    const size_t bytes = (size_t)B * N * H * D * elem_bytes(dt);
+    if (overlap(q_out, bytes, q_in, bytes) || overlap(q_out, bytes, k_in, bytes) ||
+        overlap(k_out, bytes, q_in, bytes) || overlap(k_out, bytes, k_in, bytes) ||
+        overlap(q_out, bytes, k_out, bytes))
+        return MMDIT_ERR_ARG;
+    return cuda_status(launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_scale, k_scale, B, N, H,
+                                           &g, nullptr, win->parts, eps, dt == MMDIT_BF16,
+                                           static_cast<cudaStream_t>(stream)),
+                       "qk_norm_rope_window");
+}
+
+int mmdit_window_permute(const void* x, void* y, int B, int N, int C, const mmdit_grid* grid,
+                         const mmdit_window* win, int inverse, mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || N < 0 || C < 0 || !grid || !win) return MMDIT_ERR_ARG;
+    if (grid->T < 1 || grid->H < 1 || grid->W < 1) return MMDIT_ERR_SHAPE;
+    if ((long long)grid->T * grid->H * grid->W != (long long)N) return MMDIT_ERR_SHAPE;
+    int r = check_window(grid, win);
+    if (r != MMDIT_OK) return r;
+    const long long row_bytes = (long long)C * elem_bytes(dt);
+    if (C == 0 || row_bytes % 16 != 0) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * N == 0) return MMDIT_OK;
+    if ((long long)B * N >= (1LL << 31) || row_bytes >= (1LL << 31)) return MMDIT_ERR_UNSUPPORTED;
+    if (!x || !y) return MMDIT_ERR_ARG;
+    if (!aligned16(x) || !aligned16(y)) return MMDIT_ERR_ALIGN;
+    const size_t bytes = (size_t)B * N * row_bytes;
+    if (overlap(x, bytes, y, bytes)) return MMDIT_ERR_ARG;
+    RopeGrid g{};
+    g.T = grid->T;
+    g.H = grid->H;
+    g.W = grid->W;
+    return cuda_status(launch_window_permute(x, y, B, N, (int)row_bytes, g, win->parts,
+                                             inverse != 0, static_cast<cudaStream_t>(stream)),
+                       "window_permute");
 }
 
 int mmdit_qk_norm_rope_text(const void* q_in, const void* k_in, void* q_out, void* k_out,
@@ -113,15 +191,20 @@ int mmdit_qk_norm_rope_text(const void* q_in, const void* k_in, void* q_out, voi
     t.base = rope->rope_base;
     for (int a = 0; a < 3; ++a) t.split[a] = rope->split[a];
     return cuda_status(launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_scale, k_scale, B, N, H,
-                                           nullptr, &t, eps, dt == MMDIT_BF16,
+                                           nullptr, &t, nullptr, eps, dt == MMDIT_BF16,
                                            static_cast<cudaStream_t>(stream)),
                        "qk_norm_rope_text");
 }
 
-int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vis,
-                          const void* q_ctx, const void* k_ctx, const void* v_ctx,
-                          const int32_t* ctx_len, void* o_vis, void* o_ctx, int B, int Nv, int Nc,
-                          int H, int D, float softmax_scale, mmdit_dtype dt, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int joint_attention_impl(const void* q_vis, const void* k_vis, const void* v_vis,
+                         const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                         const int32_t* ctx_len, void* o_vis, void* o_ctx, int B, int Nv, int Nc,
+                         int H, int D, float softmax_scale, const WindowTable* win,
+                         mmdit_dtype dt, void* stream) {
     if (!dtype_ok(dt) || B < 0 || Nv < 0 || Nc < 0 || H < 0) return MMDIT_ERR_ARG;
     if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MMDIT_ERR_ARG;
     if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
@@ -146,12 +229,40 @@ int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vi
             static_cast<const float*>(v_vis), static_cast<const float*>(q_ctx),
             static_cast<const float*>(k_ctx), static_cast<const float*>(v_ctx), ctx_len,
             static_cast<float*>(o_vis), static_cast<float*>(o_ctx), B, Nv, Nc, H, softmax_scale,
-            s), "joint_attention_f32");
+            win, s), "joint_attention_f32");
     const int r = launch_joint_attention_bf16(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len,
-                                              o_vis, o_ctx, B, Nv, Nc, H, softmax_scale, s);
+                                              o_vis, o_ctx, B, Nv, Nc, H, softmax_scale, win, s);
     if (r == 0) return MMDIT_OK;
     set_last_error("joint_attention_bf16", r);
     return MMDIT_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vis,
+                          const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                          const int32_t* ctx_len, void* o_vis, void* o_ctx, int B, int Nv, int Nc,
+                          int H, int D, float softmax_scale, mmdit_dtype dt, void* stream) {
+    return joint_attention_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx, B,
+                                Nv, Nc, H, D, softmax_scale, nullptr, dt, stream);
+}
+
+int mmdit_joint_window_attention(const void* q_vis, const void* k_vis, const void* v_vis,
+                                 const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                 const int32_t* ctx_len, void* o_vis, void* o_ctx, int B, int Nv,
+                                 int Nc, int H, int D, const mmdit_grid* grid,
+                                 const mmdit_window* win, float softmax_scale, mmdit_dtype dt,
+                                 void* stream) {
+    if (!grid || !win || Nv < 0) return MMDIT_ERR_ARG;
+    if (grid->T < 1 || grid->H < 1 || grid->W < 1) return MMDIT_ERR_SHAPE;
+    if ((long long)grid->T * grid->H * grid->W != (long long)Nv) return MMDIT_ERR_SHAPE;
+    const int r = check_window(grid, win);
+    if (r != MMDIT_OK) return r;
+    const WindowTable tab = make_window_table(grid->T, grid->H, grid->W, win->parts);
+    return joint_attention_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx, B,
+                                Nv, Nc, H, D, softmax_scale, &tab, dt, stream);
 }
 
 int mmdit_adaln_modulate(const void* x, const float* shift, const float* scale, void* y, int B,

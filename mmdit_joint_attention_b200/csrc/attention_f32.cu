@@ -8,6 +8,12 @@
 // warp-shuffle sum, and the softmax runs online (running max, rescaled sum and
 // accumulator) over the valid keys of the visual stream, then of the
 // conditioning stream.
+//
+// Window mode (Seaweed-7B report, section 3.2, 3D window attention): the
+// visual q/k/v are in window-major order (window.h); a visual query row takes
+// the visual keys of its own window only (a contiguous range in that order)
+// plus the conditioning keys, a conditioning row takes every key, and the
+// visual output row is written back at its raster position.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -22,7 +28,7 @@ joint_attn_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv
                       const float* __restrict__ vv, const float* __restrict__ qc,
                       const float* __restrict__ kc, const float* __restrict__ vc,
                       const int32_t* __restrict__ ctx_len, float* ov, float* oc, int Nv, int Nc,
-                      int H, float scale) {
+                      int H, float scale, bool windowed, const __grid_constant__ WindowTable win) {
     const int lane = threadIdx.x & 31;
     const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // joint query row
     const int h = blockIdx.y;
@@ -35,7 +41,17 @@ joint_attn_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv
     }
     const bool vis = i < Nv;
     const size_t qrow = vis ? ((size_t)b * Nv + i) * H + h : ((size_t)b * Nc + (i - Nv)) * H + h;
-    float4* dst = reinterpret_cast<float4*>((vis ? ov : oc) + qrow * kHeadDim) + lane;
+    int k0 = 0, k1 = Nv;   // visual keys [k0, k1)
+    size_t orow = qrow;    // output row
+    if (windowed && vis) {
+        int w = 0;
+        while (w + 1 < win.count && win.w[w + 1].start <= i) ++w;
+        const WindowGeom& g = win.w[w];
+        k0 = g.start;
+        k1 = g.start + g.te * g.he * g.we;
+        orow = ((size_t)b * Nv + window_to_raster(g, i - g.start, win.Hg, win.Wg)) * H + h;
+    }
+    float4* dst = reinterpret_cast<float4*>((vis ? ov : oc) + orow * kHeadDim) + lane;
     if (!vis && i - Nv >= L) {  // padded conditioning query: zero output
         *dst = make_float4(0.f, 0.f, 0.f, 0.f);
         return;
@@ -44,11 +60,12 @@ joint_attn_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv
     float m = -INFINITY, l = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int seg = 0; seg < 2; ++seg) {
-        const int nk = seg == 0 ? Nv : L;
+        const int j0 = seg == 0 ? k0 : 0;
+        const int nk = seg == 0 ? k1 : L;
         const float* K = seg == 0 ? kv : kc;
         const float* V = seg == 0 ? vv : vc;
         const int Ns = seg == 0 ? Nv : Nc;
-        for (int j = 0; j < nk; ++j) {
+        for (int j = j0; j < nk; ++j) {
             const size_t krow = ((size_t)b * Ns + j) * H + h;
             const float4 k = reinterpret_cast<const float4*>(K + krow * kHeadDim)[lane];
             float d = q.x * k.x + q.y * k.y + q.z * k.z + q.w * k.w;
@@ -77,12 +94,14 @@ cudaError_t launch_joint_attention_f32(const float* qv, const float* kv, const f
                                        const float* qc, const float* kc, const float* vc,
                                        const int32_t* ctx_len, float* ov, float* oc, int B,
                                        int Nv, int Nc, int H, float softmax_scale,
-                                       cudaStream_t s) {
+                                       const WindowTable* win, cudaStream_t s) {
     const int rows = Nv + Nc;
     if (rows == 0 || B == 0) return cudaSuccess;
     dim3 grid((rows + 7) / 8, H, B);
+    WindowTable tab{};
+    if (win) tab = *win;
     joint_attn_f32_kernel<<<grid, 256, 0, s>>>(qv, kv, vv, qc, kc, vc, ctx_len, ov, oc, Nv, Nc, H,
-                                               softmax_scale);
+                                               softmax_scale, win != nullptr, tab);
     return cudaGetLastError();
 }
 

@@ -26,6 +26,14 @@
 //     maximum, which is exact after the final division by the row sum and
 //     keeps every P below 256.
 // Tensor memory: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) columns.
+//
+// Window mode (Seaweed-7B report, section 3.2, 3D window attention): the
+// visual q/k/v arrive in window-major order (window.h), so each window is a
+// contiguous key range.  A CTA then owns two query tiles of one window and
+// streams that window's visual keys followed by the conditioning keys; the
+// conditioning query tiles stream every key.  The grid is one-dimensional with
+// the conditioning tiles first (they run longest), and the epilogue writes
+// each visual row back at its raster position.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -89,6 +97,25 @@ struct Params {
     int q_tiles;        // ceil(Nv / 128) + ceil(Nc / 128)
     float scale_log2;   // softmax_scale * log2(e)
     uint64_t wait_ns;   // limit of one pipeline wait
+    // window mode only
+    int windowed;
+    int B;
+    int cond_pairs;     // query-tile pairs of the conditioning stream per (b, h)
+    int vis_pairs;      // query-tile pairs of all windows per (b, h)
+    int pair_start[kMaxWindows + 1];  // first pair of each window
+    WindowTable win;
+};
+
+
+// What one CTA works on: query tiles (seg, row) of stream seg (0 visual,
+// 1 conditioning), the visual key range [vis_start, vis_start + vis_len), and
+// the window of its visual rows (-1: rows are stored in place).
+struct Work {
+    int b, h;
+    int seg0, row0, seg1, row1;
+    bool has1;
+    int vis_start, vis_len;
+    int wi;
 };
 
 struct Bars {
@@ -101,7 +128,11 @@ struct Bars {
     uint64_t wait_ns;   // limit of one pipeline wait (copied from the parameters)
     uint32_t tmem_base;
     uint32_t abort;
+    Work work;          // this CTA's work item, decoded once by thread 0
 };
+
+static_assert(sizeof(Params) <= 4096, "kernel parameters must fit the 4 KB parameter space");
+static_assert(sizeof(Bars) <= 256, "barrier block must fit its shared-memory slot");
 
 __device__ __forceinline__ void tile_of(const Params& p, int t, int& s, int& row0) {
     if (t < p.q_tiles_vis) {
@@ -111,6 +142,64 @@ __device__ __forceinline__ void tile_of(const Params& p, int t, int& s, int& row
         s = 1;
         row0 = (t - p.q_tiles_vis) * kBlockM;
     }
+}
+
+__device__ __forceinline__ Work decode_work(const Params& p) {
+    Work w;
+    w.vis_start = 0;
+    w.vis_len = p.N[0];
+    w.wi = -1;
+    if (!p.windowed) {
+        w.h = blockIdx.y;
+        w.b = blockIdx.z;
+        const int t0 = 2 * blockIdx.x;
+        w.has1 = t0 + 1 < p.q_tiles;
+        tile_of(p, t0, w.seg0, w.row0);
+        w.seg1 = w.seg0;
+        w.row1 = w.row0;
+        if (w.has1) tile_of(p, t0 + 1, w.seg1, w.row1);
+        return w;
+    }
+    int idx = blockIdx.x;
+    const int cond_items = p.B * p.H * p.cond_pairs;
+    int bh;
+    if (idx < cond_items) {
+        bh = idx / p.cond_pairs;
+        const int pr = idx - bh * p.cond_pairs;
+        w.seg0 = w.seg1 = 1;
+        w.row0 = 2 * kBlockM * pr;
+        w.row1 = w.row0 + kBlockM;
+        w.has1 = w.row1 < p.N[1];
+    } else {
+        idx -= cond_items;
+        bh = idx / p.vis_pairs;
+        const int q = idx - bh * p.vis_pairs;
+        int wi = 0;
+        while (wi + 1 < p.win.count && p.pair_start[wi + 1] <= q) ++wi;
+        const int pr = q - p.pair_start[wi];
+        const WindowGeom& g = p.win.w[wi];
+        w.vis_start = g.start;
+        w.vis_len = g.te * g.he * g.we;
+        w.wi = wi;
+        w.seg0 = w.seg1 = 0;
+        w.row0 = g.start + 2 * kBlockM * pr;
+        w.row1 = w.row0 + kBlockM;
+        w.has1 = 2 * kBlockM * pr + kBlockM < w.vis_len;
+    }
+    w.h = bh % p.H;
+    w.b = bh / p.H;
+    return w;
+}
+
+// Output row of query row `row` of stream seg, or -1 if the row is not stored
+// (past the end of the stream, or of window wi's rows [vis_start,
+// vis_start + vis_len) in window mode).
+__device__ __forceinline__ int out_row(const Params& p, int seg, int row, int wi, int vis_start,
+                                       int vis_len) {
+    if (seg == 1 || wi < 0) return row < p.N[seg] ? row : -1;
+    const int local = row - vis_start;
+    if (local >= vis_len) return -1;
+    return window_to_raster(p.win.w[wi], local, p.win.Hg, p.win.Wg);
 }
 
 __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Bars* bars) {
@@ -142,18 +231,18 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t tile, int s) {
 }
 
 // Streams the n_kv 128-key tiles of one operand (K or V) of the joint key
-// sequence (visual tiles first, then conditioning tiles) through its ring of
-// kStages shared-memory slots.  On an abort, waits (bounded) for the copies
+// sequence (kv_vis visual tiles from row vis_start on, then conditioning
+// tiles) through its ring of kStages shared-memory slots.  On an abort, waits (bounded) for the copies
 // it issued before returning.
 __device__ __forceinline__ void stream_tiles(const CUtensorMap* tm, uint8_t* ring, uint64_t* full,
-                                             uint64_t* empty, int n_kv, int kv_vis, int h, int b,
-                                             Bars* bars) {
+                                             uint64_t* empty, int n_kv, int kv_vis, int vis_start,
+                                             int h, int b, Bars* bars) {
     int issued = 0;
     for (int j = 0; j < n_kv; ++j) {
         const int st = j % kStages;
         const uint32_t ph = (j / kStages) & 1;
         const int seg = j < kv_vis ? 0 : 1;
-        const int row = (seg == 0 ? j : j - kv_vis) * kBlockN;
+        const int row = seg == 0 ? vis_start + j * kBlockN : (j - kv_vis) * kBlockN;
         if (!wait(&empty[st], ph ^ 1, bars)) break;
         uint8_t* t = ring + st * kTileBytes;
         mbar_arrive_expect_tx(&full[st], kTileBytes);
@@ -213,19 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int h = blockIdx.y;
-    const int b = blockIdx.z;
-    const int t0 = 2 * blockIdx.x;
-    const bool has1 = t0 + 1 < p.q_tiles;
-    int L = p.N[1];
-    if (p.ctx_len) {
-        L = p.ctx_len[b];
-        L = L < 0 ? 0 : (L > p.N[1] ? p.N[1] : L);
-    }
-    const int kv_vis = (p.N[0] + kBlockN - 1) / kBlockN;
-    const int n_kv = kv_vis + (L + kBlockN - 1) / kBlockN;
 
     if (threadIdx.x == 0) {
+        bars->work = decode_work(p);
         mbar_init(&bars->q_full, 1);
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&bars->k_full[i], 1);
@@ -244,6 +323,20 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         bars->wait_ns = p.wait_ns;
         fence_barrier_init();
     }
+    __syncthreads();
+    // The work item is read back from shared memory where it is needed, so
+    // that it holds no registers through the main loop.
+    const volatile Work* vwk = &bars->work;
+    const int h = vwk->h;
+    const int b = vwk->b;
+    const bool has1 = vwk->has1;
+    int L = p.N[1];
+    if (p.ctx_len) {
+        L = p.ctx_len[b];
+        L = L < 0 ? 0 : (L > p.N[1] ? p.N[1] : L);
+    }
+    const int kv_vis = (vwk->vis_len + kBlockN - 1) / kBlockN;
+    const int n_kv = kv_vis + (L + kBlockN - 1) / kBlockN;
     if (warp == kWarpLoad && n_kv > 0) {
         tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
@@ -260,13 +353,13 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         // no valid key at all: every output row of this CTA is zero
         for (int tt = 0; tt < 2; ++tt) {
             if (tt == 1 && !has1) break;
-            int s, row0;
-            tile_of(p, t0 + tt, s, row0);
+            const int s = tt ? vwk->seg1 : vwk->seg0;
+            const int row0 = tt ? vwk->row1 : vwk->row0;
             for (int r = threadIdx.x; r < kBlockM * 16; r += kThreads) {
-                const int row = row0 + r / 16;
-                if (row < p.N[s]) {
+                const int orow = out_row(p, s, row0 + r / 16, vwk->wi, vwk->vis_start, vwk->vis_len);
+                if (orow >= 0) {
                     uint4* dst = reinterpret_cast<uint4*>(
-                        p.out[s] + ((size_t)(b * (size_t)p.N[s] + row) * p.H + h) * kHeadDim);
+                        p.out[s] + ((size_t)(b * (size_t)p.N[s] + orow) * p.H + h) * kHeadDim);
                     dst[r % 16] = make_uint4(0, 0, 0, 0);
                 }
             }
@@ -287,9 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                     tma_prefetch_desc(&p.tm_k[seg]);
                 }
             }
-            int s0, r0, s1 = 0, r1 = 0;
-            tile_of(p, t0, s0, r0);
-            if (has1) tile_of(p, t0 + 1, s1, r1);
+            const int s0 = vwk->seg0, r0 = vwk->row0, s1 = vwk->seg1, r1 = vwk->row1;
             mbar_arrive_expect_tx(&bars->q_full, (has1 ? 2 : 1) * kTileBytes);
             tma_load_4d(smem + Smem::q_off, &p.tm_q[s0], &bars->q_full, 0, h, r0, b);
             tma_load_4d(smem + Smem::q_off + kHalfBytes, &p.tm_q[s0], &bars->q_full, 64, h, r0, b);
@@ -298,8 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                 tma_load_4d(smem + Smem::q_off + kTileBytes + kHalfBytes, &p.tm_q[s1], &bars->q_full,
                             64, h, r1, b);
             }
-            stream_tiles(p.tm_k, smem + Smem::k_off, bars->k_full, bars->k_empty, n_kv, kv_vis, h,
-                         b, bars);
+            stream_tiles(p.tm_k, smem + Smem::k_off, bars->k_full, bars->k_empty, n_kv, kv_vis,
+                         vwk->vis_start, h, b, bars);
             if (bars->abort) mbar_wait_bounded(&bars->q_full, 0, nullptr, kDrainLimitNs);
         }
     } else if (warp == kWarpLoadV) {
@@ -307,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         if (lane == 0) {
             for (int seg = 0; seg < 2; ++seg)
                 if (p.N[seg] > 0) tma_prefetch_desc(&p.tm_v[seg]);
-            stream_tiles(p.tm_v, smem + Smem::v_off, bars->v_full, bars->v_empty, n_kv, kv_vis, h,
-                         b, bars);
+            stream_tiles(p.tm_v, smem + Smem::v_off, bars->v_full, bars->v_empty, n_kv, kv_vis,
+                         vwk->vis_start, h, b, bars);
         }
     } else if (warp == kWarpMma && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
@@ -395,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         // ------------------------------------------------------------ softmax warpgroups
         const int i = warp >> 2;        // query tile of this warpgroup
         const int quarter = warp & 3;   // TMEM lanes [32 quarter, 32 quarter + 32)
-        if (i == 0 || has1) {
+        if (i == 0 || vwk->has1) {
             const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
             const uint32_t tS = tmem + i * 128 + lane_off;
             const uint32_t tO = tmem + 256 + i * 128 + lane_off;
@@ -410,7 +501,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
                 tmem_wait_ld();
-                const int valid = j < kv_vis ? p.N[0] - j * kBlockN : L - (j - kv_vis) * kBlockN;
+                const int valid =
+                    j < kv_vis ? vwk->vis_len - j * kBlockN : L - (j - kv_vis) * kBlockN;
                 float sv[128];
 #pragma unroll
                 for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(r[c >> 5][c & 31]);
@@ -463,14 +555,15 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
             // epilogue: O / l  ->  bf16 row of the owning stream
             if (ok) ok = wait_warp(&bars->o_done[i], 0, bars);
             tc_fence_after();
-            int s, row0;
-            tile_of(p, t0 + i, s, row0);
-            const int row = row0 + quarter * 32 + lane;
-            const bool store = row < p.N[s];
+            const int s = i ? vwk->seg1 : vwk->seg0;
+            const int row = (i ? vwk->row1 : vwk->row0) + quarter * 32 + lane;
+            const int orow = out_row(p, s, row, vwk->wi, vwk->vis_start, vwk->vis_len);
+            const bool store = orow >= 0;
             const bool zero = !ok || (s == 1 && row >= L);
             const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
             uint4* dst = reinterpret_cast<uint4*>(
-                p.out[s] + ((size_t)((size_t)b * p.N[s] + (store ? row : 0)) * p.H + h) * kHeadDim);
+                p.out[s] +
+                ((size_t)((size_t)vwk->b * p.N[s] + (store ? orow : 0)) * p.H + vwk->h) * kHeadDim);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
@@ -554,13 +647,30 @@ bool encode_tokens(CUtensorMap* m, const void* base, int B, int N, int H) {
 int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, const void* qc,
                                 const void* kc, const void* vc, const int32_t* ctx_len, void* ov,
                                 void* oc, int B, int Nv, int Nc, int H, float softmax_scale,
-                                cudaStream_t s) {
+                                const WindowTable* win, cudaStream_t s) {
     using namespace attn;
     if (!encode_fn()) return -1;
     const int q_tiles = (Nv + kBlockM - 1) / kBlockM + (Nc + kBlockM - 1) / kBlockM;
     if (B == 0 || q_tiles == 0) return 0;
     Params p;
     std::memset(&p, 0, sizeof(p));
+    long long items = 0;  // window mode: CTAs of the one-dimensional grid
+    if (win) {
+        p.windowed = 1;
+        p.B = B;
+        p.win = *win;
+        p.cond_pairs = ((Nc + kBlockM - 1) / kBlockM + 1) / 2;
+        int pairs = 0;
+        for (int w = 0; w < win->count; ++w) {
+            p.pair_start[w] = pairs;
+            const int len = win->w[w].te * win->w[w].he * win->w[w].we;
+            pairs += ((len + kBlockM - 1) / kBlockM + 1) / 2;
+        }
+        p.pair_start[win->count] = pairs;
+        p.vis_pairs = pairs;
+        items = (long long)B * H * (p.cond_pairs + p.vis_pairs);
+        if (items >= (1LL << 31)) return (int)cudaErrorInvalidConfiguration;
+    }
     if (Nv > 0) {
         if (!encode_tokens(&p.tm_q[0], qv, B, Nv, H) || !encode_tokens(&p.tm_k[0], kv, B, Nv, H) ||
             !encode_tokens(&p.tm_v[0], vv, B, Nv, H))
@@ -600,7 +710,7 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
         if (e != cudaSuccess) return (int)e;
         attr_set[dev] = true;
     }
-    dim3 grid((q_tiles + 1) / 2, H, B);
+    const dim3 grid = win ? dim3((unsigned)items, 1, 1) : dim3((q_tiles + 1) / 2, H, B);
     joint_attn_bf16_kernel<<<grid, kThreads, smem, s>>>(p);
     return (int)cudaGetLastError();
 }

@@ -106,8 +106,46 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
     return (__umulhi(n, f.m) + n) >> f.l;
 }
 
+// One axis of a 3D window partition (see window.h): the first r windows have
+// q + 1 positions and cover [0, big), big = r (q + 1); the others have q.
+struct AxisSplit {
+    uint32_t q, big;
+    FastDiv dq1, dq;
+};
+AxisSplit make_axis_split(int extent, int parts) {
+    AxisSplit s;
+    s.q = (uint32_t)(extent / parts);
+    s.big = (uint32_t)(extent % parts) * (s.q + 1);
+    s.dq1 = make_fastdiv(s.q + 1);
+    s.dq = make_fastdiv(s.q);
+    return s;
+}
+__device__ __forceinline__ void axis_window(uint32_t x, const AxisSplit& s, uint32_t& start,
+                                            uint32_t& ext) {
+    if (x < s.big) {
+        start = fdiv(x, s.dq1) * (s.q + 1);
+        ext = s.q + 1;
+    } else {
+        start = s.big + fdiv(x - s.big, s.dq) * s.q;
+        ext = s.q;
+    }
+}
+// Window-major index of the visual token at grid cell (t, h, w); HW = Hg * Wg.
+struct WinMap {
+    AxisSplit ax[3];
+};
+__device__ __forceinline__ uint32_t raster_to_window(uint32_t t, uint32_t h, uint32_t w,
+                                                     uint32_t Wg, uint32_t HW, const WinMap& m) {
+    uint32_t ts, te, hs, he, ws, we;
+    axis_window(t, m.ax[0], ts, te);
+    axis_window(h, m.ax[1], hs, he);
+    axis_window(w, m.ax[2], ws, we);
+    return ts * HW + te * (hs * Wg + he * ws) + ((t - ts) * he + (h - hs)) * we + (w - ws);
+}
+
 struct RopeParams {
     FastDiv H, N, HW, W;   // heads, tokens per sample, Hg*Wg, Wg
+    WinMap win;            // output order when the kernel permutes to window-major
     int Hg;
     int split[3];
     int off[3];        // first head dim of each axis chunk
@@ -134,7 +172,9 @@ constexpr int kRopeText = 2;   // text tokens, MM-RoPE: one position shared by t
 // 480p (5.5 TB/s, vs 3.6 TB/s with one unit per group and 64-bit index math).
 constexpr int kQkUnroll = 8;
 
-template <typename T, int ROPE, bool TABLE, int UNR>
+// PERM (grid mode only): rows are stored in window-major order instead of in
+// place of the input rows.
+template <typename T, int ROPE, bool TABLE, bool PERM, int UNR>
 __global__ void __launch_bounds__(256, 2)
 qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
                     const float* __restrict__ gq, const float* __restrict__ gk, uint32_t units,
@@ -216,6 +256,7 @@ qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
                 xq[i] *= iq * wq[i];
                 xk[i] *= ik * wk[i];
             }
+            uint32_t delta = 0;  // output unit - input unit
             if (ROPE != kRopeNone) {
                 const uint32_t uu = u < units ? u : 0;
                 const uint32_t bn = fdiv(uu, rp.H);
@@ -226,6 +267,11 @@ qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
                     const uint32_t rem = n - t * rp.HW.d;
                     const uint32_t hh = fdiv(rem, rp.W);
                     const uint32_t pos = axis == 0 ? t : (axis == 1 ? hh : rem - hh * rp.W.d);
+                    if (PERM)
+                        delta = (raster_to_window(t, hh, rem - hh * rp.W.d, rp.W.d, rp.HW.d,
+                                                  rp.win) -
+                                 n) *
+                                rp.H.d;
                     if (TABLE) {
                         const float4* p4 = reinterpret_cast<const float4*>(
                             tab + rp.tab_off[axis] + pos * rp.stride[axis] + jb);
@@ -265,7 +311,7 @@ qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
                 }
             }
             if (u < units) {
-                const size_t base = (size_t)u * kHeadDim + d0;
+                const size_t base = (size_t)(u + delta) * kHeadDim + d0;
                 st16(q_out + base, pack(xq));
                 st16(k_out + base, pack(xk));
             }
@@ -273,12 +319,13 @@ qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
     }
 }
 
-template <typename T, int ROPE, bool TABLE>
+template <typename T, int ROPE, bool TABLE, bool PERM = false>
 cudaError_t run_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, const float* gq,
                    const float* gk, uint32_t units, float eps, const RopeParams& rp, size_t smem,
                    cudaStream_t s) {
-    constexpr int UNR = kQkUnroll;
-    auto kern = qk_norm_rope_kernel<T, ROPE, TABLE, UNR>;
+    // the permuted store next to in-register sin/cos needs more registers
+    constexpr int UNR = (PERM && !TABLE) ? kQkUnroll / 2 : kQkUnroll;
+    auto kern = qk_norm_rope_kernel<T, ROPE, TABLE, PERM, UNR>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -297,6 +344,46 @@ cudaError_t run_qk(const void* q_in, const void* k_in, void* q_out, void* k_out,
         static_cast<const T*>(q_in), static_cast<const T*>(k_in), static_cast<T*>(q_out),
         static_cast<T*>(k_out), gq, gk, units, eps, rp);
     return cudaGetLastError();
+}
+
+// ======================================================================
+// Row permutation between raster and window-major order
+// ======================================================================
+
+// One warp per row of `chunks` 16-byte pieces: forward, row n of sample b
+// moves to window-major position perm(n); inverse, position perm(n) moves back
+// to n.  Each lane issues all its loads of a row before its stores.
+constexpr int kPermUnroll = 4;
+
+__global__ void __launch_bounds__(256)
+window_permute_kernel(const uint4* __restrict__ x, uint4* __restrict__ y, uint32_t rows,
+                      uint32_t chunks, FastDiv N, FastDiv HW, FastDiv W, WinMap wm, bool inverse) {
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t row = warp0; row < rows; row += nwarps) {
+        const uint32_t b = fdiv(row, N);
+        const uint32_t n = row - b * N.d;
+        const uint32_t t = fdiv(n, HW);
+        const uint32_t rem = n - t * HW.d;
+        const uint32_t h = fdiv(rem, W);
+        const uint32_t other = b * N.d + raster_to_window(t, h, rem - h * W.d, W.d, HW.d, wm);
+        const uint4* src = x + (size_t)(inverse ? other : row) * chunks;
+        uint4* dst = y + (size_t)(inverse ? row : other) * chunks;
+        for (uint32_t c0 = lane; c0 < chunks; c0 += 32 * kPermUnroll) {
+            uint4 v[kPermUnroll];
+#pragma unroll
+            for (int k = 0; k < kPermUnroll; ++k) {
+                const uint32_t c = c0 + 32 * k;
+                if (c < chunks) v[k] = __ldcs(src + c);
+            }
+#pragma unroll
+            for (int k = 0; k < kPermUnroll; ++k) {
+                const uint32_t c = c0 + 32 * k;
+                if (c < chunks) __stcs(dst + c, v[k]);
+            }
+        }
+    }
 }
 
 // ======================================================================
@@ -625,8 +712,8 @@ cudaError_t run_residual(const void* x, const void* br, const float* gate, void*
 // ----------------------------------------------------------------------
 cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
                                 const float* gq, const float* gk, int B, int N, int H,
-                                const RopeGrid* grid, const RopeText* text, float eps, bool bf16,
-                                cudaStream_t s) {
+                                const RopeGrid* grid, const RopeText* text, const int* win_parts,
+                                float eps, bool bf16, cudaStream_t s) {
     const long long units_ll = (long long)B * N * H;
     if (units_ll == 0) return cudaSuccess;
     if (units_ll >= (1LL << 31)) return cudaErrorInvalidValue;  // rejected by the C-ABI layer
@@ -655,6 +742,8 @@ cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out,
             off += grid->split[a];
         }
         rp.tab_entries = toff;
+        if (win_parts)
+            for (int a = 0; a < 3; ++a) rp.win.ax[a] = make_axis_split(extent[a], win_parts[a]);
         smem = (size_t)toff * sizeof(float2);
         table = smem <= 64 * 1024;
         if (!table) smem = 0;
@@ -682,6 +771,12 @@ cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out,
     if (!grid)                                                                                 \
         return run_qk<T, kRopeNone, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, \
                                            s);                                                  \
+    if (win_parts && table)                                                                    \
+        return run_qk<T, kRopeGrid, true, true>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, \
+                                                smem, s);                                       \
+    if (win_parts)                                                                             \
+        return run_qk<T, kRopeGrid, false, true>(q_in, k_in, q_out, k_out, gq, gk, units, eps,   \
+                                                 rp, 0, s);                                     \
     if (table)                                                                                 \
         return run_qk<T, kRopeGrid, true>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp,     \
                                           smem, s);                                             \
@@ -738,6 +833,25 @@ cudaError_t launch_gated_residual(const void* x, const void* branch, const float
                                   void* out, int B, int N, int C, bool bf16, cudaStream_t s) {
     return bf16 ? run_residual<__nv_bfloat16>(x, branch, gate, out, B, N, C, s)
                 : run_residual<float>(x, branch, gate, out, B, N, C, s);
+}
+
+cudaError_t launch_window_permute(const void* x, void* y, int B, int N, int row_bytes,
+                                  const RopeGrid& grid, const int* parts, bool inverse,
+                                  cudaStream_t s) {
+    const long long rows_ll = (long long)B * N;
+    if (rows_ll == 0) return cudaSuccess;
+    WinMap wm;
+    const int extent[3] = {grid.T, grid.H, grid.W};
+    for (int a = 0; a < 3; ++a) wm.ax[a] = make_axis_split(extent[a], parts[a]);
+    const uint32_t rows = (uint32_t)rows_ll;
+    long long blocks = ((long long)rows + 7) / 8;  // 8 warps per block, one row each
+    const long long cap = (long long)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    window_permute_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+        static_cast<const uint4*>(x), static_cast<uint4*>(y), rows, (uint32_t)(row_bytes / 16),
+        make_fastdiv((uint32_t)N), make_fastdiv((uint32_t)(grid.H * grid.W)),
+        make_fastdiv((uint32_t)grid.W), wm, inverse);
+    return cudaGetLastError();
 }
 
 }  // namespace mmdit

@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "window.h"
+
 namespace mmdit {
 
 struct RopeGrid {
@@ -21,10 +23,18 @@ struct RopeText {
 };
 
 // 0 or a cudaError_t value.  At most one of grid / text is non-null.
+// win_parts (grid mode only, else null): store the rows in the window-major
+// order of that 3D window partition (window.h) instead of in place.
 cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
                                 const float* gq, const float* gk, int B, int N, int H,
-                                const RopeGrid* grid, const RopeText* text, float eps, bool bf16,
-                                cudaStream_t s);
+                                const RopeGrid* grid, const RopeText* text, const int* win_parts,
+                                float eps, bool bf16, cudaStream_t s);
+
+// Rows of row_bytes (a multiple of 16) of [B, N] between raster order and the
+// window-major order of `parts` (window.h); inverse: window-major -> raster.
+cudaError_t launch_window_permute(const void* x, void* y, int B, int N, int row_bytes,
+                                  const RopeGrid& grid, const int* parts, bool inverse,
+                                  cudaStream_t s);
 
 cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float* scale,
                                   void* y, int B, int N, int C, float eps, bool bf16,
@@ -39,16 +49,20 @@ cudaError_t launch_gated_residual(const void* x, const void* branch, const float
 
 // Returns 0 on success, a cudaError_t value on CUDA failure, or -1 if the
 // driver entry point for tensor-map encoding is unavailable.
+// win (null: full joint attention): 3D window attention; the visual inputs
+// are then in the table's window-major order and o_vis is written in raster
+// order.
 int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv,
                                 const void* qc, const void* kc, const void* vc,
                                 const int32_t* ctx_len, void* ov, void* oc, int B, int Nv,
-                                int Nc, int H, float softmax_scale, cudaStream_t s);
+                                int Nc, int H, float softmax_scale, const WindowTable* win,
+                                cudaStream_t s);
 
 cudaError_t launch_joint_attention_f32(const float* qv, const float* kv, const float* vv,
                                        const float* qc, const float* kc, const float* vc,
                                        const int32_t* ctx_len, float* ov, float* oc, int B,
                                        int Nv, int Nc, int H, float softmax_scale,
-                                       cudaStream_t s);
+                                       const WindowTable* win, cudaStream_t s);
 
 // Limit of one bounded pipeline wait in the attention kernel (0 = default).
 void set_wait_timeout_ns(unsigned long long ns);

@@ -98,3 +98,37 @@ def test_qk_norm_rope_text_validation(L):
     r.pos_offset = float("inf")
     assert f(P, P, P, P, P, P, 1, 8, 2, 128, ctypes.byref(r), 1e-6, 1, None) == -1
     assert f(U, P, P, P, P, P, 1, 8, 2, 128, ctypes.byref(r), 1e-6, 1, None) == -3
+
+
+def test_window_validation(L):
+    g = _lib.Grid(5, 8, 8, (ctypes.c_float * 3)(1, 1, 1), 10000.0, (ctypes.c_int * 3)(16, 56, 56))
+    w = _lib.Window((ctypes.c_int * 3)(1, 2, 2))
+    R = ctypes.byref
+    f = L.mmdit_joint_window_attention
+    Q = ctypes.c_void_p(1 << 20)
+    assert f(P, P, P, P, P, P, None, Q, Q, 1, 320, 8, 2, 128, None, R(w), 0.1, 1, None) == -1
+    assert f(P, P, P, P, P, P, None, Q, Q, 1, 321, 8, 2, 128, R(g), R(w), 0.1, 1, None) == -2
+    for bad in ((0, 1, 1), (6, 1, 1), (1, 9, 1), (1, 1, -1)):
+        wb = _lib.Window((ctypes.c_int * 3)(*bad))
+        assert f(P, P, P, P, P, P, None, Q, Q, 1, 320, 8, 2, 128, R(g), R(wb), 0.1, 1, None) == -2
+    many = _lib.Window((ctypes.c_int * 3)(5, 8, 2))   # 80 windows > 64
+    assert f(P, P, P, P, P, P, None, Q, Q, 1, 320, 8, 2, 128, R(g), R(many), 0.1, 1, None) == -4
+    assert f(P, P, P, P, P, P, None, Q, Q, 1, 320, 8, 2, 64, R(g), R(w), 0.1, 1, None) == -4
+    assert f(P, P, P, P, P, P, None, U, Q, 1, 320, 8, 2, 128, R(g), R(w), 0.1, 1, None) == -3
+
+    p = L.mmdit_window_permute
+    assert p(P, Q, 1, 320, 250, R(g), R(w), 0, 1, None) == -4     # 500-byte rows
+    assert p(P, Q, 1, 321, 256, R(g), R(w), 0, 1, None) == -2
+    assert p(P, P, 1, 320, 256, R(g), R(w), 0, 1, None) == -1     # y overlaps x
+    assert p(U, Q, 1, 320, 256, R(g), R(w), 0, 1, None) == -3
+    assert p(P, Q, 1, 320, 256, None, R(w), 0, 1, None) == -1
+    assert p(None, None, 0, 320, 256, R(g), R(w), 0, 1, None) == 0   # empty batch
+
+    q = L.mmdit_qk_norm_rope_window
+    Q2 = ctypes.c_void_p(1 << 24)
+    assert q(P, P, P, Q2, P, P, 1, 320, 2, 128, R(g), R(w), 1e-6, 1, None) == -1   # q_out == q_in
+    assert q(P, Q, Q2, ctypes.c_void_p((1 << 24) + 16), P, P, 1, 320, 2, 128, R(g), R(w), 1e-6, 1,
+             None) == -1                                                              # outputs overlap
+    assert q(P, P, Q, Q2, P, P, 1, 320, 2, 128, None, R(w), 1e-6, 1, None) == -1
+    assert q(P, P, Q, Q2, P, P, 1, 320, 2, 128, R(g), None, 1e-6, 1, None) == -1
+    assert q(P, P, Q, Q2, P, P, 1, 321, 2, 128, R(g), R(w), 1e-6, 1, None) == -2
