@@ -56,6 +56,12 @@ def _configure(lib):
         [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [ctypes.c_int] * 5 +
         [ctypes.POINTER(_Grid), ctypes.POINTER(ctypes.c_int)] +
         [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp])
+    lib.oracle_joint_attention_bwd.argtypes = (
+        [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [dp] * 2 + [ctypes.c_int] * 5 +
+        [ctypes.c_double] + [dp] * 7)
+    lib.oracle_joint_attention_dq_rows.argtypes = (
+        [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [dp] * 2 + [ctypes.c_int] * 5 +
+        [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp, dp])
     lib.oracle_adaln_modulate.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3 + [ctypes.c_double]
     lib.oracle_gated_residual.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3
     return lib
@@ -170,6 +176,55 @@ def joint_attention(qv, kv, vv, qc, kc, vc, ctx_len=None, scale: Optional[float]
     out = joint_attention_rows(qv, kv, vv, qc, kc, vc, ctx_len, rows, scale)
     out = out.reshape(B, H, Nv + Nc, D).transpose(0, 2, 1, 3)
     return np.ascontiguousarray(out[:, :Nv]), np.ascontiguousarray(out[:, Nv:])
+
+
+def _ctx_ptr(ctx_len):
+    if ctx_len is None:
+        return ctypes.POINTER(ctypes.c_int)(), None
+    cl = np.ascontiguousarray(ctx_len, dtype=np.int32)
+    return cl.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), cl
+
+
+def joint_attention_bwd(qv, kv, vv, qc, kc, vc, dov, doc, ctx_len=None,
+                        scale: Optional[float] = None) -> dict:
+    """Gradients of the joint attention for upstream gradients (dov, doc) on
+    (o_vis, o_ctx): returns dq_vis, dk_vis, dv_vis, dq_ctx, dk_ctx, dv_ctx
+    (shapes of the inputs) and lse [B, H, Nv + Nc] (natural log of the softmax
+    denominator including the max; +inf for rows without an output)."""
+    qv, kv, vv, qc, kc, vc, dov, doc = (_f64(a) for a in (qv, kv, vv, qc, kc, vc, dov, doc))
+    B, Nv, H, D = qv.shape
+    Nc = qc.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = {k: np.empty_like(qv) for k in ("dq_vis", "dk_vis", "dv_vis")}
+    out.update({k: np.empty_like(qc) for k in ("dq_ctx", "dk_ctx", "dv_ctx")})
+    out["lse"] = np.empty((B, H, Nv + Nc), dtype=np.float64)
+    cl_p, _keep = _ctx_ptr(ctx_len)
+    _load().oracle_joint_attention_bwd(
+        _p(qv), _p(kv), _p(vv), _p(qc), _p(kc), _p(vc), cl_p, _p(dov), _p(doc), B, Nv, Nc, H, D,
+        scale, _p(out["dq_vis"]), _p(out["dk_vis"]), _p(out["dv_vis"]), _p(out["dq_ctx"]),
+        _p(out["dk_ctx"]), _p(out["dv_ctx"]), _p(out["lse"]))
+    return out
+
+
+def joint_attention_dq_rows(qv, kv, vv, qc, kc, vc, dov, doc, ctx_len, rows,
+                            scale: Optional[float] = None):
+    """(dq [nrows, D], lse [nrows]) of selected (b, h, joint row) triplets."""
+    qv, kv, vv, qc, kc, vc, dov, doc = (_f64(a) for a in (qv, kv, vv, qc, kc, vc, dov, doc))
+    B, Nv, H, D = qv.shape
+    Nc = qc.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    dq = np.zeros((rows.shape[0], D), dtype=np.float64)
+    lse = np.zeros(rows.shape[0], dtype=np.float64)
+    cl_p, _keep = _ctx_ptr(ctx_len)
+    if rows.shape[0]:
+        _load().oracle_joint_attention_dq_rows(
+            _p(qv), _p(kv), _p(vv), _p(qc), _p(kc), _p(vc), cl_p, _p(dov), _p(doc), B, Nv, Nc,
+            H, D, scale, rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), rows.shape[0],
+            _p(dq), _p(lse))
+    return dq, lse
 
 
 def _grid_struct(grid) -> _Grid:

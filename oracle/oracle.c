@@ -308,3 +308,152 @@ void oracle_window_attention_rows(const double* qv, const double* kv, const doub
     }
     free(win);
 }
+
+/* ---- joint attention backward [V], non-causal [W4] -------------------------
+ * Gradients of the joint attention above for an upstream gradient dO on every
+ * output row (the reverse-mode derivative of the definition; the Seaweed-7B
+ * report, section 3.4, trains forward and backward of this attention).  With
+ * s_ij = scale q_i . k_j over valid keys, p_ij = softmax_j(s_ij),
+ * o_i = sum_j p_ij v_j and D_i = dO_i . o_i:
+ *   dv_j += p_ij dO_i
+ *   dP_ij = dO_i . v_j,   dS_ij = p_ij (dP_ij - D_i)
+ *   dq_i  = scale sum_j dS_ij k_j,   dk_j += scale dS_ij q_i
+ * Padded conditioning query rows have a constant (zero) output: they add
+ * nothing, and their dq is zero; padded keys get zero dk and dv.
+ * lse (if not NULL) [B, H, Nv + Nc] receives log sum_j exp(s_ij) per joint row,
+ * +infinity for rows without an output.                                      */
+static const double* oracle_row(const double* vis, const double* ctx, long b, long j, int Nv,
+                                int Nc, int H, long h, int D)
+{
+    return (j < Nv) ? vis + ((b * Nv + j) * H + h) * (long)D
+                    : ctx + ((b * Nc + (j - Nv)) * H + h) * (long)D;
+}
+
+void oracle_joint_attention_bwd(const double* qv, const double* kv, const double* vv,
+                                const double* qc, const double* kc, const double* vc,
+                                const int* ctx_len, const double* dov, const double* doc,
+                                int B, int Nv, int Nc, int H, int D, double scale,
+                                double* dqv, double* dkv, double* dvv,
+                                double* dqc, double* dkc, double* dvc, double* lse)
+{
+    const long nv = (long)B * Nv * H * D, nc = (long)B * Nc * H * D;
+    memset(dqv, 0, sizeof(double) * (size_t)nv);
+    memset(dkv, 0, sizeof(double) * (size_t)nv);
+    memset(dvv, 0, sizeof(double) * (size_t)nv);
+    memset(dqc, 0, sizeof(double) * (size_t)nc);
+    memset(dkc, 0, sizeof(double) * (size_t)nc);
+    memset(dvc, 0, sizeof(double) * (size_t)nc);
+    #pragma omp parallel
+    {
+        double* p = (double*)malloc(sizeof(double) * (size_t)(Nv + Nc + 1));
+        double* o = (double*)malloc(sizeof(double) * (size_t)D);
+        /* each (b, h) owns its rows of every gradient: no two threads write
+         * the same element */
+        #pragma omp for schedule(dynamic, 1)
+        for (long bh = 0; bh < (long)B * H; ++bh) {
+            const long b = bh / H, h = bh % H;
+            const int L = ctx_len ? ctx_len[b] : Nc;
+            const int nk = L + Nv;  /* valid keys */
+            for (long i = 0; i < Nv + Nc; ++i) {
+                if (lse) lse[bh * (long)(Nv + Nc) + i] = INFINITY;
+                if (i >= nk || nk == 0) continue;    /* padded query row */
+                const double* q = oracle_row(qv, qc, b, i, Nv, Nc, H, h, D);
+                const double* dO = oracle_row(dov, doc, b, i, Nv, Nc, H, h, D);
+                double m = -INFINITY;
+                for (int j = 0; j < nk; ++j) {
+                    const double* k = oracle_row(kv, kc, b, j, Nv, Nc, H, h, D);
+                    double acc = 0.0;
+                    for (int d = 0; d < D; ++d) acc += q[d] * k[d];
+                    p[j] = acc * scale;
+                    if (p[j] > m) m = p[j];
+                }
+                double den = 0.0;
+                for (int j = 0; j < nk; ++j) den += exp(p[j] - m);
+                if (lse) lse[bh * (long)(Nv + Nc) + i] = m + log(den);
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (int j = 0; j < nk; ++j) {
+                    p[j] = exp(p[j] - m) / den;
+                    const double* v = oracle_row(vv, vc, b, j, Nv, Nc, H, h, D);
+                    for (int d = 0; d < D; ++d) o[d] += p[j] * v[d];
+                }
+                double Di = 0.0;
+                for (int d = 0; d < D; ++d) Di += dO[d] * o[d];
+                double* dq = (double*)oracle_row(dqv, dqc, b, i, Nv, Nc, H, h, D);
+                for (int j = 0; j < nk; ++j) {
+                    const double* k = oracle_row(kv, kc, b, j, Nv, Nc, H, h, D);
+                    const double* v = oracle_row(vv, vc, b, j, Nv, Nc, H, h, D);
+                    double* dk = (double*)oracle_row(dkv, dkc, b, j, Nv, Nc, H, h, D);
+                    double* dv = (double*)oracle_row(dvv, dvc, b, j, Nv, Nc, H, h, D);
+                    double dP = 0.0;
+                    for (int d = 0; d < D; ++d) dP += dO[d] * v[d];
+                    const double dS = p[j] * (dP - Di);
+                    for (int d = 0; d < D; ++d) {
+                        dv[d] += p[j] * dO[d];
+                        dq[d] += scale * dS * k[d];
+                        dk[d] += scale * dS * q[d];
+                    }
+                }
+            }
+        }
+        free(o);
+        free(p);
+    }
+}
+
+/* dq and lse of selected query rows (b, h, i) only, for sizes where the full
+ * backward is out of reach: the same definitions, row by row.  dq_out is
+ * [nrows, D]; lse_out [nrows].                                                */
+void oracle_joint_attention_dq_rows(const double* qv, const double* kv, const double* vv,
+                                    const double* qc, const double* kc, const double* vc,
+                                    const int* ctx_len, const double* dov, const double* doc,
+                                    int B, int Nv, int Nc, int H, int D, double scale,
+                                    const long* rows, long nrows, double* dq_out, double* lse_out)
+{
+    (void)B;
+    #pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)(Nv + Nc + 1));
+        double* o = (double*)malloc(sizeof(double) * (size_t)D);
+        #pragma omp for schedule(dynamic, 4)
+        for (long r = 0; r < nrows; ++r) {
+            const long b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+            const int L = ctx_len ? ctx_len[b] : Nc;
+            const int nk = L + Nv;  /* valid keys */
+            double* dq = dq_out + r * (long)D;
+            for (int d = 0; d < D; ++d) dq[d] = 0.0;
+            lse_out[r] = INFINITY;
+            if (i >= nk || nk == 0) continue;
+            const double* q = oracle_row(qv, qc, b, i, Nv, Nc, H, h, D);
+            const double* dO = oracle_row(dov, doc, b, i, Nv, Nc, H, h, D);
+            double mx = -INFINITY;
+            for (int j = 0; j < nk; ++j) {
+                const double* k = oracle_row(kv, kc, b, j, Nv, Nc, H, h, D);
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += q[d] * k[d];
+                s[j] = scale * acc;
+                mx = s[j] > mx ? s[j] : mx;
+            }
+            double sum = 0.0;
+            for (int j = 0; j < nk; ++j) sum += exp(s[j] - mx);
+            lse_out[r] = mx + log(sum);
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            for (int j = 0; j < nk; ++j) {
+                s[j] = exp(s[j] - mx) / sum;             /* now p_ij */
+                const double* v = oracle_row(vv, vc, b, j, Nv, Nc, H, h, D);
+                for (int d = 0; d < D; ++d) o[d] += s[j] * v[d];
+            }
+            double Dsum = 0.0;
+            for (int d = 0; d < D; ++d) Dsum += dO[d] * o[d];
+            for (int j = 0; j < nk; ++j) {
+                const double* k = oracle_row(kv, kc, b, j, Nv, Nc, H, h, D);
+                const double* v = oracle_row(vv, vc, b, j, Nv, Nc, H, h, D);
+                double g = 0.0;
+                for (int d = 0; d < D; ++d) g += dO[d] * v[d];
+                const double w = scale * s[j] * (g - Dsum);
+                for (int d = 0; d < D; ++d) dq[d] += w * k[d];
+            }
+        }
+        free(o);
+        free(s);
+    }
+}

@@ -27,6 +27,17 @@ void oracle_window_attention_rows(const double* qv, const double* kv, const doub
                                   const int* ctx_len, int B, int Nv, int Nc, int H, int D,
                                   const oracle_grid* grid, const int* parts, double scale,
                                   const long* rows, long nrows, double* out);
+void oracle_joint_attention_bwd(const double* qv, const double* kv, const double* vv,
+                                const double* qc, const double* kc, const double* vc,
+                                const int* ctx_len, const double* dov, const double* doc,
+                                int B, int Nv, int Nc, int H, int D, double scale,
+                                double* dqv, double* dkv, double* dvv,
+                                double* dqc, double* dkc, double* dvc, double* lse);
+void oracle_joint_attention_dq_rows(const double* qv, const double* kv, const double* vv,
+                                    const double* qc, const double* kc, const double* vc,
+                                    const int* ctx_len, const double* dov, const double* doc,
+                                    int B, int Nv, int Nc, int H, int D, double scale,
+                                    const long* rows, long nrows, double* dq_out, double* lse_out);
 void oracle_adaln_modulate(const double* x, const double* shift, const double* scale,
                            double* y, int B, int N, int C, double eps);
 void oracle_gated_residual(const double* x, const double* branch, const double* gate,

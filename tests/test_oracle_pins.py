@@ -7,7 +7,10 @@ the definition reduces to (torch float64 scaled_dot_product_attention and
 layer_norm), closed forms (tests/golden/rope_closed_form.json) and invariants
 (RoPE preserves norms and is relative; softmax rows sum to one; identical keys
 give mean(V); masked keys have no influence; constant-scale RMSNorm has RMS
-equal to the scale; a window sees nothing outside itself).  Sources: Vimoo
+equal to the scale; a window sees nothing outside itself), and for the
+attention backward: central finite differences of sum(dO * O), torch float64
+autograd, scipy's logsumexp, and the gradient sums fixed by softmax rows
+summing to one.  Sources: Vimoo
 1.0 research page, section 2.2; Wan 2.1 report sections 4.2.1 and 4.3.1;
 Seaweed-7B report, section 3.2.
 
@@ -530,6 +533,101 @@ def pin_window_sizes():
     assert win[23 * 80 + 40] == 3 and win[22 * 80 + 39] == 0
 
 
+# ------------------------------------------------------------ attention backward
+
+def _bwd_case(seed, B=2, Nv=5, Nc=3, H=2, D=8, ctx_len=(3, 1)):
+    r = RNG(seed)
+    t = [r.standard_normal((B, Nv, H, D)) for _ in range(3)] + \
+        [r.standard_normal((B, Nc, H, D)) for _ in range(3)]
+    do = (r.standard_normal((B, Nv, H, D)), r.standard_normal((B, Nc, H, D)))
+    return t, do, (None if ctx_len is None else np.array(ctx_len, np.int32))
+
+
+@pin
+def pin_bwd_finite_differences():
+    """Every gradient entry equals the central difference of L = sum(dO * O)
+    computed with the forward oracle (step 1e-6)."""
+    t, (dov, doc), cl = _bwd_case(50)
+    g = oracle.joint_attention_bwd(*t, dov, doc, cl)
+
+    def loss(tt):
+        ov, oc = oracle.joint_attention(*tt, cl)
+        return float(np.sum(ov * dov) + np.sum(oc * doc))
+
+    names = ["dq_vis", "dk_vis", "dv_vis", "dq_ctx", "dk_ctx", "dv_ctx"]
+    h = 1e-6
+    for a, name in enumerate(names):
+        num = np.zeros_like(t[a])
+        for idx in np.ndindex(t[a].shape):
+            tp = [x.copy() for x in t]
+            tm = [x.copy() for x in t]
+            tp[a][idx] += h
+            tm[a][idx] -= h
+            num[idx] = (loss(tp) - loss(tm)) / (2 * h)
+        _close(g[name], num, 1e-7)
+
+
+@pin
+def pin_bwd_torch_autograd():
+    """torch float64 autograd through scaled_dot_product_attention on the
+    concatenated sequence with a boolean key mask; the padded cond query rows
+    get dO = 0 (their output is a constant).  Also the row log-sum-exp
+    against scipy's logsumexp of the masked scores."""
+    from scipy.special import logsumexp
+    t, (dov, doc), cl = _bwd_case(51, B=2, Nv=7, Nc=4, H=3, D=16, ctx_len=(4, 2))
+    g = oracle.joint_attention_bwd(*t, dov, doc, cl)
+    B, Nv, H, D = t[0].shape
+    Nc = t[3].shape[1]
+    qkv = [torch.tensor(np.concatenate([t[i], t[i + 3]], axis=1).transpose(0, 2, 1, 3),
+                        requires_grad=True) for i in range(3)]
+    valid = np.concatenate([np.ones((B, Nv), bool), np.arange(Nc)[None, :] < cl[:, None]], 1)
+    mask = torch.from_numpy(valid)[:, None, None, :]
+    out = torch.nn.functional.scaled_dot_product_attention(*qkv, attn_mask=mask)
+    dO = np.concatenate([dov, doc], axis=1).transpose(0, 2, 1, 3) * valid[:, None, :, None]
+    out.backward(torch.from_numpy(dO))
+    for i, n in enumerate("qkv"):
+        grad = qkv[i].grad.numpy().transpose(0, 2, 1, 3)
+        _close(g["d%s_vis" % n], grad[:, :Nv], 1e-12)
+        _close(g["d%s_ctx" % n], grad[:, Nv:], 1e-12)
+    q = np.concatenate([t[0], t[3]], 1).transpose(0, 2, 1, 3)
+    k = np.concatenate([t[1], t[4]], 1).transpose(0, 2, 1, 3)
+    sc = q @ k.transpose(0, 1, 3, 2) / math.sqrt(D)
+    sc = np.where(valid[:, None, None, :], sc, -np.inf)
+    want = logsumexp(sc, axis=-1)
+    want = np.where(valid[:, None, :], want, np.inf)
+    _close(np.where(np.isinf(g["lse"]), 0, g["lse"]), np.where(np.isinf(want), 0, want), 1e-12)
+    assert np.array_equal(np.isinf(g["lse"]), np.isinf(want))
+    # the row function gives the same dq and lse as autograd and scipy
+    rows = np.array([[b, h, i] for b in range(B) for h in range(H) for i in range(Nv + Nc)])
+    dq, lse = oracle.joint_attention_dq_rows(*t, dov, doc, cl, rows)
+    gq = qkv[0].grad.numpy()
+    _close(dq, gq[rows[:, 0], rows[:, 1], rows[:, 2]], 1e-12)
+    _close(np.where(np.isinf(lse), 0, lse),
+           np.where(np.isinf(want), 0, want)[rows[:, 0], rows[:, 1], rows[:, 2]], 1e-12)
+
+
+@pin
+def pin_bwd_invariants():
+    """Softmax rows sum to one, so sum_j dv_j = sum of dO over the rows with
+    an output; sum_j dS_ij = 0, so sum_j dk_j = 0; identical keys make every
+    dq zero."""
+    t, (dov, doc), cl = _bwd_case(52, B=2, Nv=9, Nc=5, H=2, D=16, ctx_len=(5, 2))
+    g = oracle.joint_attention_bwd(*t, dov, doc, cl)
+    for b in range(2):
+        L = cl[b]
+        want = dov[b].sum(axis=0) + doc[b, :L].sum(axis=0)
+        got = g["dv_vis"][b].sum(axis=0) + g["dv_ctx"][b].sum(axis=0)
+        _close(got, want, 1e-12)
+        _close(g["dk_vis"][b].sum(axis=0) + g["dk_ctx"][b].sum(axis=0), np.zeros((2, 16)), 1e-12)
+        assert np.all(g["dk_ctx"][b, L:] == 0) and np.all(g["dv_ctx"][b, L:] == 0)
+        assert np.all(g["dq_ctx"][b, L:] == 0)
+    t2 = [x.copy() for x in t]
+    t2[1][:] = t2[1][:, :1]
+    t2[4][:] = t2[1][:, :1]
+    g2 = oracle.joint_attention_bwd(*t2, dov, doc, cl)
+    _close(g2["dq_vis"], np.zeros_like(g2["dq_vis"]), 1e-12)
+
+
 @pytest.mark.parametrize("name", sorted(PINS))
 def test_pin(name):
     PINS[name]()
@@ -565,6 +663,16 @@ MUTANTS = {
     "window_cond_queries_windowed": ("if (i >= Nv || win[j] == win[i]) key[nk++] = j;",
                                      "if (win[j] == win[i < Nv ? i : 0]) key[nk++] = j;"),
     "window_padded_rows_not_zero": ("if (i >= Nv + L) continue;", "if (i >= Nv + Nc) continue;"),
+    "bwd_no_delta": ("const double dS = p[j] * (dP - Di);", "const double dS = p[j] * dP;"),
+    "bwd_dq_no_scale": ("dq[d] += scale * dS * k[d];", "dq[d] += dS * k[d];"),
+    "bwd_dv_uses_dp": ("dv[d] += p[j] * dO[d];", "dv[d] += dP * dO[d];"),
+    "bwd_dk_from_k": ("dk[d] += scale * dS * q[d];", "dk[d] += scale * dS * k[d];"),
+    "bwd_lse_no_max": ("if (lse) lse[bh * (long)(Nv + Nc) + i] = m + log(den);",
+                       "if (lse) lse[bh * (long)(Nv + Nc) + i] = log(den);"),
+    "bwd_padded_rows_counted": ("if (i >= nk || nk == 0) continue;    /* padded query row */",
+                                "if (nk == 0) continue;"),
+    "dqrows_no_delta": ("const double w = scale * s[j] * (g - Dsum);",
+                        "const double w = scale * s[j] * g;"),
     "window_no_cond_keys": ("for (int j = 0; j < L; ++j) key[nk++] = Nv + j;",
                             "for (int j = 0; j < L && i >= Nv; ++j) key[nk++] = Nv + j;"),
 }
