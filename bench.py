@@ -427,6 +427,30 @@ def run_ours(args):
     txt_ms = time_ms(lambda: api.qk_norm_rope_text(
         t["q_ctx"], t["k_ctx"], t["gq_ctx"], t["gk_ctx"], pos_offset=float(max(w.grid)),
         q_out=q_txt, k_out=k_txt))
+    # backward: forward with the row log-sum-exp, then D, dQ and dK/dV
+    gen = torch.Generator(device=dev).manual_seed(1000 + rank)
+    do_vis = torch.randn(t["q_vis"].shape, generator=gen, device=dev).to(torch.bfloat16)
+    do_ctx = torch.randn(t["q_ctx"].shape, generator=gen, device=dev).to(torch.bfloat16)
+    lse = torch.empty((B, H, Nv + Nc), dtype=torch.float32, device=dev)
+    delta = torch.empty_like(lse)
+    grads = {k: torch.empty_like(t["q_" + k[-3:]]) for k in
+             ("dq_vis", "dk_vis", "dv_vis", "dq_ctx", "dk_ctx", "dv_ctx")}
+    qkv = (t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"], t["v_ctx"])
+    fwd_lse_ms = time_ms(lambda: api.joint_attention_fwd(
+        *qkv, t["ctx_len"], o_vis=t["o_vis"], o_ctx=t["o_ctx"], lse=lse), reps=10)
+    bwd_ms = time_ms(lambda: api.joint_attention_bwd(
+        *qkv, t["o_vis"], t["o_ctx"], do_vis, do_ctx, lse, t["ctx_len"], delta=delta,
+        grads=grads), reps=5)
+    pairs = H * sum((Nv + L) ** 2 for L in w.ctx_lengths())
+    bwd_rows = {"backward": {
+        "ms": bwd_ms, "fwd_with_lse_ms": fwd_lse_ms,
+        "TFLOP/s_beta8": 8.0 * D * pairs / (bwd_ms * 1e-3) / 1e12,
+        "TFLOP/s_executed": 14.0 * D * pairs / (bwd_ms * 1e-3) / 1e12,
+        "frac_bf16_sustained_executed": 14.0 * D * pairs / (bwd_ms * 1e-3) / 1e12 / float(
+            peaks()[0]["bf16_tflops_sustained"]),
+        "flops_beta8": 8.0 * D * pairs, "flops_executed": 14.0 * D * pairs}}
+    del do_vis, do_ctx, grads, lse, delta
+
     # 3D window attention (1x2x2 and 4x1x1 windows): permuting prologue for
     # q/k, row permutation of v, windowed attention back to raster order
     win_rows = {}
@@ -511,7 +535,7 @@ def run_ours(args):
                               Nv / (Nv + Nc)},
             "qk_norm_rope_text_ctx": {
                 "ms": txt_ms, "GB/s": 4 * B * Nc * C * 2 / (txt_ms * 1e-3) / 1e9},
-            **win_rows},
+            **win_rows, **bwd_rows},
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,

@@ -132,6 +132,50 @@ MMDIT_API int mmdit_joint_attention(const void* q_vis, const void* k_vis, const 
                           int B, int Nv, int Nc, int H, int D, float softmax_scale,
                           mmdit_dtype dt, void* stream);
 
+/* mmdit_joint_attention that also writes, for training, the row log-sum-exp
+ * the backward pass needs [Vimoo §2.2 joint attention; the Seaweed-7B report,
+ * section 3.4, trains its forward and backward]:
+ *   lse[b, h, i] = log sum_j exp(Q_i . K_j * softmax_scale) over valid keys j
+ * (natural log) for every joint row i (i < Nv visual, then conditioning), and
+ * +infinity for rows without an output (padded conditioning rows, or no
+ * valid key at all).
+ *   lse: DEVICE fp32 [B, H, Nv + Nc], written; 4-byte aligned, not NULL
+ *   everything else as mmdit_joint_attention.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_joint_attention_fwd(const void* q_vis, const void* k_vis, const void* v_vis,
+                                        const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                        const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                                        float* lse, int B, int Nv, int Nc, int H, int D,
+                                        float softmax_scale, mmdit_dtype dt, void* stream);
+
+/* Backward of the joint attention [the reverse-mode derivative of the joint
+ * attention of Vimoo §2.2; Seaweed-7B, section 3.4]: for the upstream
+ * gradients do_vis / do_ctx of o_vis / o_ctx, with P the softmax of the
+ * forward recomputed from lse and D_i = dO_i . O_i:
+ *   dV_j = sum_i P_ij dO_i
+ *   dS_ij = P_ij (dO_i . V_j - D_i)
+ *   dQ_i = softmax_scale sum_j dS_ij K_j,   dK_j = softmax_scale sum_i dS_ij Q_i
+ * over valid keys and over the query rows that have an output; padded
+ * conditioning rows get zero dQ, dK and dV.
+ *   q/k/v/o_vis, do_vis, dq/dk/dv_vis [B, Nv, H, D] dt (the d* written)
+ *   q/k/v/o_ctx, do_ctx, dq/dk/dv_ctx [B, Nc, H, D] dt
+ *   lse    DEVICE fp32 [B, H, Nv + Nc] from mmdit_joint_attention_fwd
+ *   delta  DEVICE fp32 [B, H, Nv + Nc] caller-owned workspace, overwritten
+ *          with D_i (contents on entry ignored)
+ *   ctx_len, softmax_scale, dt: as mmdit_joint_attention (3D windows are
+ *   not supported here).  Gradients must not alias any input.
+ * bf16 runs three kernels: D, then dQ (query-stationary) and dK/dV
+ * (key-stationary) on the tcgen05 tensor cores; f32 runs CUDA-core kernels.
+ * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_joint_attention_bwd(const void* q_vis, const void* k_vis, const void* v_vis,
+                                        const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                        const int32_t* ctx_len, const void* o_vis,
+                                        const void* o_ctx, const void* do_vis, const void* do_ctx,
+                                        const float* lse, float* delta, void* dq_vis,
+                                        void* dk_vis, void* dv_vis, void* dq_ctx, void* dk_ctx,
+                                        void* dv_ctx, int B, int Nv, int Nc, int H, int D,
+                                        float softmax_scale, mmdit_dtype dt, void* stream);
+
 /* 3D window partition of the visual grid ["Seaweed-7B", section 3.2: attention
  * restricted to w_t x w_h x w_w windows, e.g. 1x2x2 and 4x1x1 in alternating
  * layers].  parts[a] is the number of windows along axis a (T, H, W), each in
@@ -229,8 +273,9 @@ MMDIT_API int mmdit_residual_modulate(const void* x, const void* branch, const f
  * MMDIT_ERR_CUDA if the synchronisation failed. */
 MMDIT_API int mmdit_device_status(void* stream);
 
-/* Sets the limit of one bounded wait inside the attention kernel for launches
- * made after the call, process-wide: 0 restores the default (2 s).  A wait that
+/* Sets the limit of one bounded wait inside the attention kernels (forward and
+ * backward) for launches made after the call, process-wide: 0 restores the
+ * default (2 s).  A wait that
  * runs out makes every role of the kernel stop (outputs undefined), drain the
  * copies and tensor-core work it issued, free its tensor memory and return;
  * the next mmdit_device_status() then reports MMDIT_ERR_TIMEOUT.  No fault or

@@ -81,6 +81,8 @@ def lib():
         L.mmdit_window_permute.argtypes = [_vp, _vp, _i, _i, _i, ctypes.POINTER(Grid),
                                            ctypes.POINTER(Window), _i, _i, _vp]
         L.mmdit_joint_attention.argtypes = [_vp] * 9 + [_i] * 5 + [_f, _i, _vp]
+        L.mmdit_joint_attention_fwd.argtypes = [_vp] * 10 + [_i] * 5 + [_f, _i, _vp]
+        L.mmdit_joint_attention_bwd.argtypes = [_vp] * 19 + [_i] * 5 + [_f, _i, _vp]
         L.mmdit_joint_window_attention.argtypes = ([_vp] * 9 + [_i] * 5 +
                                                    [ctypes.POINTER(Grid), ctypes.POINTER(Window),
                                                     _f, _i, _vp])
@@ -96,6 +98,7 @@ def lib():
         L.mmdit_status_string.restype = ctypes.c_char_p
         for name in ("mmdit_qk_norm_rope", "mmdit_qk_norm_rope_text", "mmdit_qk_norm_rope_window",
                      "mmdit_window_permute", "mmdit_joint_attention",
+                     "mmdit_joint_attention_fwd", "mmdit_joint_attention_bwd",
                      "mmdit_joint_window_attention", "mmdit_adaln_modulate",
                      "mmdit_gated_residual", "mmdit_residual_modulate", "mmdit_device_status"):
             getattr(L, name).restype = ctypes.c_int

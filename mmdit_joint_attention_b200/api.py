@@ -132,6 +132,63 @@ def joint_attention(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
     return o_vis, o_ctx
 
 
+def joint_attention_fwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
+                        softmax_scale: Optional[float] = None, o_vis=None, o_ctx=None, lse=None,
+                        stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """joint_attention that also returns the row log-sum-exp lse [B, H, Nv + Nc]
+    (fp32, natural log, +inf for rows without an output) for the backward."""
+    dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx)
+    B, Nv, H, D = q_vis.shape
+    Nc = q_ctx.shape[1]
+    o_vis = torch.empty_like(q_vis) if o_vis is None else o_vis
+    o_ctx = torch.empty_like(q_ctx) if o_ctx is None else o_ctx
+    if lse is None:
+        lse = torch.empty((B, H, Nv + Nc), dtype=torch.float32, device=q_vis.device)
+    _f32(lse)
+    if ctx_len is not None and (ctx_len.dtype != torch.int32 or not ctx_len.is_cuda):
+        raise TypeError("ctx_len must be an int32 CUDA tensor")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    st = _lib.lib().mmdit_joint_attention_fwd(
+        _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(lse), B, Nv, Nc, H, D, softmax_scale, dt,
+        _stream(stream))
+    check("mmdit_joint_attention_fwd", st)
+    return o_vis, o_ctx, lse
+
+
+def joint_attention_bwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, o_ctx, do_vis, do_ctx,
+                        lse, ctx_len=None, softmax_scale: Optional[float] = None, delta=None,
+                        grads: Optional[dict] = None, stream=None) -> dict:
+    """Gradients dq/dk/dv of both streams for upstream gradients do_vis, do_ctx
+    of the joint attention, given its outputs and lse (joint_attention_fwd).
+    ``delta`` is the fp32 [B, H, Nv + Nc] workspace (allocated here if None);
+    ``grads`` may hold preallocated outputs under the returned keys."""
+    dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, o_ctx, do_vis, do_ctx)
+    B, Nv, H, D = q_vis.shape
+    Nc = q_ctx.shape[1]
+    if delta is None:
+        delta = torch.empty((B, H, Nv + Nc), dtype=torch.float32, device=q_vis.device)
+    _f32(lse, delta)
+    g = dict(grads or {})
+    for k, ref in (("dq_vis", q_vis), ("dk_vis", k_vis), ("dv_vis", v_vis), ("dq_ctx", q_ctx),
+                   ("dk_ctx", k_ctx), ("dv_ctx", v_ctx)):
+        if k not in g:
+            g[k] = torch.empty_like(ref)
+    if ctx_len is not None and (ctx_len.dtype != torch.int32 or not ctx_len.is_cuda):
+        raise TypeError("ctx_len must be an int32 CUDA tensor")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    st = _lib.lib().mmdit_joint_attention_bwd(
+        _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(do_vis), _ptr(do_ctx), _ptr(lse),
+        _ptr(delta), _ptr(g["dq_vis"]), _ptr(g["dk_vis"]), _ptr(g["dv_vis"]), _ptr(g["dq_ctx"]),
+        _ptr(g["dk_ctx"]), _ptr(g["dv_ctx"]), B, Nv, Nc, H, D, softmax_scale, dt,
+        _stream(stream))
+    check("mmdit_joint_attention_bwd", st)
+    return g
+
+
 def make_window(parts: Sequence[int]) -> _lib.Window:
     w = _lib.Window()
     for a in range(3):

@@ -1,0 +1,1053 @@
+// Backward of the joint (concatenated) attention: bf16 in / bf16 out on the
+// sm_100a tensor cores, and an fp32 version on the CUDA cores.
+//
+// What it computes: the reverse-mode derivative of the joint attention of the
+// "Vimoo 1.0" research page, section 2.2 (the Seaweed-7B report, section 3.4,
+// trains forward and backward of this attention).  With s_ij = scale q_i.k_j
+// over valid keys, P = softmax_j(s), O = P V, the upstream gradient dO and
+// D_i = dO_i . O_i:
+//   dV_j = sum_i P_ij dO_i,   dP_ij = dO_i . v_j,   dS_ij = P_ij (dP_ij - D_i),
+//   dQ_i = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i.
+// P is recomputed from the forward's row log-sum-exp, P_ij = exp(s_ij - lse_i).
+// Rows without an output (padded conditioning rows) carry lse = +inf, so all
+// their P are 0 and they contribute nothing; padded keys get zero dK and dV.
+//
+// Three launches:
+//   1. delta_kernel: D_i into the caller's fp32 workspace (one read of O, dO).
+//   2. dq_kernel, query-stationary: a CTA owns 128 query rows of one (b, h)
+//      and streams the 128-key K/V tiles.  S = Q K^T and dP = dO V^T go to
+//      tensor memory, dS goes back over S in bf16, and dQ += dS K.  S is
+//      double-buffered, so the tensor core computes the next tile's S while
+//      the softmax warps turn this tile's S and dP into dS.
+//   3. dkdv_kernel, key-stationary: a CTA owns 128 keys of one (b, h) and
+//      streams 64-row query tiles.  S^T = K Q^T and dP^T = V dO^T (both
+//      double-buffered), P^T and dS^T in bf16 back over them, dV += P^T dO and
+//      dK += dS^T Q.  Query tiles of 64 keep the four accumulators inside the
+//      512 tensor-memory columns.
+// Splitting dQ from dK/dV computes S and dP twice but needs no atomics and no
+// fp32 dQ accumulator in global memory.
+//
+// Every wait is bounded as in the forward kernel: a wait that runs out sets an
+// abort flag and the backward status word, every role leaves its loop, copies
+// and MMAs in flight are drained (bounded), and tensor memory is freed.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "tensor_map.h"
+
+namespace mmdit {
+
+// Bit 0: a bounded wait expired in a backward kernel.
+__device__ unsigned int g_bwd_status = 0;
+
+namespace bwd {
+
+constexpr int kThreads = 384;
+// Register split: launched with 168 per thread; the producer warpgroup (TMA,
+// MMA issue, the lse / D loader) takes 88, the softmax warpgroups 208.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsProducer = 88;
+constexpr int kRegsSoftmax = 208;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsProducer == kThreads * kRegsLaunch,
+              "register split must add up to the launch allocation");
+constexpr uint64_t kDrainLimitNs = 200000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kTileBytes = 128 * 128 * 2;   // 128 rows x 128 bf16
+constexpr int kHalf128 = kTileBytes / 2;    // one 64-column box of a 128-row tile
+constexpr int kQ64Bytes = 64 * 128 * 2;     // 64 rows x 128 bf16
+constexpr int kHalf64 = kQ64Bytes / 2;
+
+// Abort flag, wait limit and tensor-memory base shared by a CTA's roles.
+struct Ctl {
+    uint64_t wait_ns;
+    uint32_t abort;
+    uint32_t tmem_base;
+};
+
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Ctl* c) {
+    if (mbar_wait_bounded(bar, parity, &c->abort, c->wait_ns)) return true;
+    c->abort = 1;
+    atomicOr(&g_bwd_status, 1u);
+    return false;
+}
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Ctl* c) {
+    const bool ok = wait(bar, parity, c);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// K-major operand: k-step s (16 columns of the 128-wide head dim) lies in the
+// 64-column half s / 4, 32 bytes * (s % 4) into each 128-byte row.
+__device__ __forceinline__ uint64_t kdesc(uint32_t addr) { return smem_desc_sw128(addr, 16, 1024); }
+__host__ __device__ constexpr uint64_t koff(int s, int half_bytes) {
+    return (uint64_t)((s >> 2) * (half_bytes >> 4) + (s & 3) * 2);
+}
+// MN-major B operand of `rows` x 128 (rows along K): k-step s = rows
+// [16 s, 16 s + 16) = 2048 bytes further; the two 64-wide halves of N are one
+// box apart (leading byte offset), 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t mndesc(uint32_t addr, int half_bytes) {
+    return smem_desc_sw128(addr, half_bytes, 1024);
+}
+constexpr uint64_t kMnStep = 2048 >> 4;
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ======================================================================
+// 1. D_i = dO_i . O_i
+// ======================================================================
+
+// 128 / E lanes own one (sample, joint row, head) unit; E elements per 16 bytes.
+template <typename T>
+__global__ void __launch_bounds__(256)
+delta_kernel(const T* __restrict__ ov, const T* __restrict__ dov, const T* __restrict__ oc,
+             const T* __restrict__ doc, const int32_t* __restrict__ ctx_len,
+             float* __restrict__ delta, int Nv, int Nc, int H, uint32_t units) {
+    constexpr int E = 16 / sizeof(T);
+    constexpr int LPR = 128 / E;
+    constexpr int GPW = 32 / LPR;
+    constexpr int UNR = 4;
+    const int Nt = Nv + Nc;
+    const int lane = threadIdx.x & 31;
+    const int g = lane % LPR;
+    const int grp = lane / LPR;
+    const uint32_t warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t uw = warp0 * (GPW * UNR); uw < units; uw += nwarps * (GPW * UNR)) {
+        uint4 a[UNR], d[UNR];
+        uint32_t jr[UNR], bb[UNR], hh[UNR];
+        bool live[UNR];
+#pragma unroll
+        for (int r = 0; r < UNR; ++r) {
+            const uint32_t u = uw + r * GPW + grp;
+            live[r] = u < units;
+            const uint32_t uu = live[r] ? u : 0;
+            hh[r] = uu % H;
+            const uint32_t bj = uu / H;
+            jr[r] = bj % Nt;
+            bb[r] = bj / Nt;
+            const bool vis = (int)jr[r] < Nv;
+            const size_t row = vis ? ((size_t)bb[r] * Nv + jr[r]) * H + hh[r]
+                                   : ((size_t)bb[r] * Nc + (jr[r] - Nv)) * H + hh[r];
+            const T* o = (vis ? ov : oc) + row * 128 + g * E;
+            const T* dO = (vis ? dov : doc) + row * 128 + g * E;
+            a[r] = live[r] ? __ldcs(reinterpret_cast<const uint4*>(o)) : make_uint4(0, 0, 0, 0);
+            d[r] = live[r] ? __ldcs(reinterpret_cast<const uint4*>(dO)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int r = 0; r < UNR; ++r) {
+            const uint32_t aw[4] = {a[r].x, a[r].y, a[r].z, a[r].w};
+            const uint32_t dw[4] = {d[r].x, d[r].y, d[r].z, d[r].w};
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (sizeof(T) == 2) {
+                    acc = fmaf(bf_lo(aw[i]), bf_lo(dw[i]), acc);
+                    acc = fmaf(bf_hi(aw[i]), bf_hi(dw[i]), acc);
+                } else {
+                    acc = fmaf(__uint_as_float(aw[i]), __uint_as_float(dw[i]), acc);
+                }
+            }
+#pragma unroll
+            for (int o = LPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (live[r] && g == 0) {
+                int L = Nc;
+                if (ctx_len) {
+                    L = ctx_len[bb[r]];
+                    L = L < 0 ? 0 : (L > Nc ? Nc : L);
+                }
+                const bool out = (int)jr[r] < Nv + L;
+                delta[((size_t)bb[r] * H + hh[r]) * Nt + jr[r]] = out ? acc : 0.f;
+            }
+        }
+    }
+}
+
+// ======================================================================
+// 2. dQ (query-stationary)
+// ======================================================================
+namespace dq {
+
+struct Smem {
+    static constexpr int q_off = 0;
+    static constexpr int do_off = kTileBytes;
+    static constexpr int k_off = 2 * kTileBytes;   // 2 stages
+    static constexpr int v_off = 4 * kTileBytes;   // 2 stages
+    static constexpr int bar_off = 6 * kTileBytes;
+    static constexpr int total = bar_off + 256;
+};
+
+struct Params {
+    CUtensorMap tm_q[2];   // [0] visual, [1] conditioning; 128-row boxes
+    CUtensorMap tm_k[2];
+    CUtensorMap tm_v[2];
+    CUtensorMap tm_do[2];
+    __nv_bfloat16* dq[2];
+    const float* lse;
+    const float* delta;
+    const int32_t* ctx_len;
+    int N[2];
+    int H;
+    int q_tiles_vis;
+    float sl2;      // softmax_scale * log2(e)
+    float scale;
+    uint64_t wait_ns;
+};
+
+struct Bars {
+    uint64_t q_full;
+    uint64_t k_full[2], k_empty[2];
+    uint64_t v_full[2], v_empty[2];
+    uint64_t s_full[2];    // S and dP of the tile with this S buffer are in tensor memory
+    uint64_t dp_free;      // every softmax warp has read dP
+    uint64_t ds_full[4];   // [2 buf + wg]: that warpgroup's half of dS is in tensor memory
+    uint64_t o_done;
+    uint64_t drain;
+    Ctl ctl;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block must fit its shared-memory slot");
+
+// Tensor memory: S0 [0,128) S1 [128,256) dP [256,384) dQ [384,512).  dS of
+// key half w is written over S at columns [64 w, 64 w + 32).
+__global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + Smem::bar_off);
+    Ctl* ctl = &bars->ctl;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x;
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const int seg = t < p.q_tiles_vis ? 0 : 1;
+    const int row0 = (seg ? t - p.q_tiles_vis : t) * 128;
+    int L = p.N[1];
+    if (p.ctx_len) {
+        L = p.ctx_len[b];
+        L = L < 0 ? 0 : (L > p.N[1] ? p.N[1] : L);
+    }
+    const int kv_vis = (p.N[0] + 127) / 128;
+    const int n_kv = kv_vis + (L + 127) / 128;
+    const bool idle = n_kv == 0 || (seg == 1 && row0 >= L);   // no row of this tile has an output
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->k_full[i], 1);
+            mbar_init(&bars->k_empty[i], 1);
+            mbar_init(&bars->v_full[i], 1);
+            mbar_init(&bars->v_empty[i], 1);
+            mbar_init(&bars->s_full[i], 1);
+        }
+        mbar_init(&bars->dp_free, 8);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars->ds_full[i], 4);
+        mbar_init(&bars->o_done, 1);
+        mbar_init(&bars->drain, 1);
+        ctl->abort = 0;
+        ctl->wait_ns = p.wait_ns;
+        fence_barrier_init();
+    }
+    if (warp == 8 && !idle) {
+        tmem_alloc(&ctl->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (idle) {
+        for (int r = threadIdx.x; r < 128 * 16; r += kThreads) {
+            const int row = row0 + r / 16;
+            if (row < p.N[seg])
+                reinterpret_cast<uint4*>(
+                    p.dq[seg] + ((size_t)((size_t)b * p.N[seg] + row) * p.H + h) * 128)[r % 16] =
+                    make_uint4(0, 0, 0, 0);
+        }
+        return;
+    }
+    const uint32_t tmem = ctl->tmem_base;
+    const uint32_t sQ = smem_u32(smem + Smem::q_off);
+    const uint32_t sDO = smem_u32(smem + Smem::do_off);
+    const uint32_t sK = smem_u32(smem + Smem::k_off);
+    const uint32_t sV = smem_u32(smem + Smem::v_off);
+
+    if (warp >= 8) {
+        regs_dec<kRegsProducer>();
+        if ((warp == 8 || warp == 10) && lane == 0) {
+            // ---------------------------------------------- TMA: Q, dO, K (warp 8) / V (warp 10)
+            const bool is_k = warp == 8;
+            const CUtensorMap* tm = is_k ? p.tm_k : p.tm_v;
+            uint8_t* ring = smem + (is_k ? Smem::k_off : Smem::v_off);
+            uint64_t* full = is_k ? bars->k_full : bars->v_full;
+            uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
+            if (is_k) {
+                mbar_arrive_expect_tx(&bars->q_full, 2 * kTileBytes);
+                tma_load_4d(smem + Smem::q_off, &p.tm_q[seg], &bars->q_full, 0, h, row0, b);
+                tma_load_4d(smem + Smem::q_off + kHalf128, &p.tm_q[seg], &bars->q_full, 64, h, row0,
+                            b);
+                tma_load_4d(smem + Smem::do_off, &p.tm_do[seg], &bars->q_full, 0, h, row0, b);
+                tma_load_4d(smem + Smem::do_off + kHalf128, &p.tm_do[seg], &bars->q_full, 64, h,
+                            row0, b);
+            }
+            int issued = 0;
+            for (int j = 0; j < n_kv; ++j) {
+                const int st = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                const int ks = j < kv_vis ? 0 : 1;
+                const int row = (ks ? j - kv_vis : j) * 128;
+                if (!wait(&empty[st], ph ^ 1, ctl)) break;
+                uint8_t* dst = ring + st * kTileBytes;
+                mbar_arrive_expect_tx(&full[st], kTileBytes);
+                tma_load_4d(dst, &tm[ks], &full[st], 0, h, row, b);
+                tma_load_4d(dst + kHalf128, &tm[ks], &full[st], 64, h, row, b);
+                ++issued;
+            }
+            if (ctl->abort) {
+                for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
+                    mbar_wait_bounded(&full[j & 1], (j >> 1) & 1, nullptr, kDrainLimitNs);
+                if (is_k) mbar_wait_bounded(&bars->q_full, 0, nullptr, kDrainLimitNs);
+            }
+        } else if (warp == 9 && lane == 0) {
+            // ---------------------------------------------- MMA issuer
+            constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t id_mn = idesc_bf16_f32(128, 128, 0, 1);
+            bool ok = wait(&bars->q_full, 0, ctl);
+            const uint64_t dq_d = kdesc(sQ), ddo_d = kdesc(sDO);
+            const uint64_t dk0 = kdesc(sK), dk1 = kdesc(sK + kTileBytes);
+            const uint64_t dv0 = kdesc(sV), dv1 = kdesc(sV + kTileBytes);
+            const uint64_t km0 = mndesc(sK, kHalf128), km1 = mndesc(sK + kTileBytes, kHalf128);
+            // dQ += dS(jj) K(jj), key half by key half as the softmax releases them
+            auto dq_mma = [&](int jj) -> bool {
+                const int pb = jj & 1;
+                const uint64_t km = pb ? km1 : km0;
+                const uint32_t sb = tmem + 128 * pb;
+#pragma unroll
+                for (int wg = 0; wg < 2; ++wg) {
+                    if (!wait(&bars->ds_full[2 * pb + wg], (jj >> 1) & 1, ctl)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int s = 4 * wg + q;
+                        mma_ts(tmem + 384, sb + 64 * wg + 8 * q, km + (uint64_t)s * kMnStep, id_mn,
+                               (jj > 0 || s > 0) ? 1u : 0u);
+                    }
+                }
+                return true;
+            };
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int st = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                if (!(ok = wait(&bars->k_full[st], ph, ctl))) break;
+                tc_fence_after();
+                const uint64_t dk = st ? dk1 : dk0;
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint64_t off = koff(s, kHalf128);
+                    mma_ss(tmem + 128 * st, dq_d + off, dk + off, id_kk, s > 0 ? 1u : 0u);
+                }
+                if (!(ok = wait(&bars->v_full[st], ph, ctl))) break;
+                if (j > 0 && !(ok = wait(&bars->dp_free, (j - 1) & 1, ctl))) break;
+                tc_fence_after();
+                const uint64_t dv = st ? dv1 : dv0;
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint64_t off = koff(s, kHalf128);
+                    mma_ss(tmem + 256, ddo_d + off, dv + off, id_kk, s > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars->s_full[st]);
+                mma_commit(&bars->v_empty[st]);
+                if (j > 0) {
+                    if (!(ok = dq_mma(j - 1))) break;
+                    mma_commit(&bars->k_empty[(j - 1) & 1]);
+                }
+            }
+            if (ok && (ok = dq_mma(n_kv - 1))) {
+                mma_commit(&bars->k_empty[(n_kv - 1) & 1]);
+                mma_commit(&bars->o_done);
+            }
+            mma_commit(&bars->drain);
+            if (!mbar_wait_bounded(&bars->drain, 0, nullptr, kDrainLimitNs))
+                atomicOr(&g_bwd_status, 1u);
+        }
+    } else {
+        regs_inc<kRegsSoftmax>();
+        // -------------------------------------------------- dS = P (dP - D)
+        const int wg = warp >> 2;        // key columns [64 wg, 64 wg + 64) of every tile
+        const int quarter = warp & 3;    // tensor-memory lanes (query rows) of this warp
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int row = row0 + quarter * 32 + lane;
+        const bool has_out = row < p.N[seg] && (seg == 0 || row < L);
+        const size_t lrow =
+            ((size_t)b * p.H + h) * (size_t)(p.N[0] + p.N[1]) + (seg ? p.N[0] + row : row);
+        const float lse2 = has_out ? p.lse[lrow] * kLog2e : INFINITY;
+        const float dl = has_out ? p.delta[lrow] : 0.f;
+        const uint64_t sl2x2 = f2_pack(p.sl2, p.sl2);
+        const uint64_t nl2 = f2_pack(-lse2, -lse2);
+        const uint64_t ndl = f2_pack(-dl, -dl);
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            const int buf = j & 1;
+            if (!(ok = wait_warp(&bars->s_full[buf], (j >> 1) & 1, ctl))) break;
+            tc_fence_after();
+            uint32_t sr[2][32], dr[2][32];
+            const uint32_t tS = tmem + 128 * buf + 64 * wg + lane_off;
+            const uint32_t tP = tmem + 256 + 64 * wg + lane_off;
+            tmem_ld32(tS, sr[0]);
+            tmem_ld32(tS + 32, sr[1]);
+            tmem_ld32(tP, dr[0]);
+            tmem_ld32(tP + 32, dr[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->dp_free);
+            const int valid =
+                (j < kv_vis ? p.N[0] - j * 128 : L - (j - kv_vis) * 128) - 64 * wg;
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const int k = 2 * c;
+                uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[k >> 5][k & 31]),
+                                            __uint_as_float(sr[k >> 5][(k & 31) + 1])),
+                                    sl2x2, nl2);
+                float x0, x1;
+                f2_unpack(x, x0, x1);
+                if (valid < 64) {
+                    if (k >= valid) x0 = -INFINITY;
+                    if (k + 1 >= valid) x1 = -INFINITY;
+                }
+                const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+                const uint64_t dd = f2_add(f2_pack(__uint_as_float(dr[k >> 5][k & 31]),
+                                                   __uint_as_float(dr[k >> 5][(k & 31) + 1])),
+                                           ndl);
+                float d0, d1;
+                f2_unpack(f2_mul(pp, dd), d0, d1);
+                pk[c] = pack_bf16x2(d0, d1);
+            }
+            tmem_st32(tS, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->ds_full[2 * buf + wg]);
+        }
+        if (ok) ok = wait_warp(&bars->o_done, 0, ctl);
+        tc_fence_after();
+        const bool store = row < p.N[seg];
+        const bool zero = !ok || !has_out;
+        uint4* dst = reinterpret_cast<uint4*>(
+            p.dq[seg] + ((size_t)((size_t)b * p.N[seg] + (store ? row : 0)) * p.H + h) * 128 +
+            64 * wg);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + 384 + 64 * wg + 32 * c + lane_off, o);
+            tmem_wait_ld();
+            if (store) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        f[e] = zero ? 0.f : __uint_as_float(o[8 * v + e]) * p.scale;
+                    dst[4 * c + v] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace dq
+
+// ======================================================================
+// 3. dK, dV (key-stationary)
+// ======================================================================
+namespace dkv {
+
+constexpr int kStages = 4;   // Q / dO / (lse, D) ring depth
+
+struct Smem {
+    static constexpr int k_off = 0;
+    static constexpr int v_off = kTileBytes;
+    static constexpr int q_off = 2 * kTileBytes;                  // kStages x 64 rows
+    static constexpr int do_off = q_off + kStages * kQ64Bytes;    // kStages x 64 rows
+    static constexpr int l_off = do_off + kStages * kQ64Bytes;    // kStages x 64 float2
+    static constexpr int bar_off = l_off + kStages * 512;
+    static constexpr int total = bar_off + 512;
+};
+
+struct Params {
+    CUtensorMap tm_k[2];   // 128-row boxes
+    CUtensorMap tm_v[2];
+    CUtensorMap tm_q[2];   // 64-row boxes
+    CUtensorMap tm_do[2];
+    __nv_bfloat16* dk[2];
+    __nv_bfloat16* dv[2];
+    const float* lse;
+    const float* delta;
+    const int32_t* ctx_len;
+    int N[2];
+    int H;
+    int k_tiles_vis;
+    float sl2;
+    float scale;
+    uint64_t wait_ns;
+};
+
+struct Bars {
+    uint64_t kv_full;
+    uint64_t q_full[kStages], q_empty[kStages];
+    uint64_t do_full[kStages], do_empty[kStages];
+    uint64_t l_full[kStages], l_empty[kStages];
+    uint64_t s_full[2];   // S^T and dP^T of the tile with this buffer are in tensor memory
+    uint64_t p_full[2];   // every softmax warp has written its P^T and dS^T
+    uint64_t o_done;
+    uint64_t drain;
+    Ctl ctl;
+};
+static_assert(sizeof(Bars) <= 512, "barrier block must fit its shared-memory slot");
+
+// Tensor memory: S^T buffers [0,64) [64,128), dP^T buffers [128,192)
+// [192,256), dV [256,384), dK [384,512).  Warpgroup w handles query columns
+// [32 w, 32 w + 32) of a tile and writes its packed P^T / dS^T at columns
+// [32 w, 32 w + 16) of the same buffer.
+__host__ __device__ constexpr int packed_col(int s) { return s < 2 ? 8 * s : 32 + 8 * (s - 2); }
+
+__global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + Smem::bar_off);
+    Ctl* ctl = &bars->ctl;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x;
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const int seg = t < p.k_tiles_vis ? 0 : 1;
+    const int krow0 = (seg ? t - p.k_tiles_vis : t) * 128;
+    int L = p.N[1];
+    if (p.ctx_len) {
+        L = p.ctx_len[b];
+        L = L < 0 ? 0 : (L > p.N[1] ? p.N[1] : L);
+    }
+    const int nq_vis = (p.N[0] + 63) / 64;
+    const int nq = nq_vis + (L + 63) / 64;
+    const bool idle = nq == 0 || (seg == 1 && krow0 >= L);   // no valid key or no query
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->kv_full, 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&bars->q_full[i], 1);
+            mbar_init(&bars->q_empty[i], 1);
+            mbar_init(&bars->do_full[i], 1);
+            mbar_init(&bars->do_empty[i], 1);
+            mbar_init(&bars->l_full[i], 32);   // every lane of the loader warp
+            mbar_init(&bars->l_empty[i], 8);   // one elected lane per softmax warp
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->p_full[i], 8);
+        }
+        mbar_init(&bars->o_done, 1);
+        mbar_init(&bars->drain, 1);
+        ctl->abort = 0;
+        ctl->wait_ns = p.wait_ns;
+        fence_barrier_init();
+    }
+    if (warp == 8 && !idle) {
+        tmem_alloc(&ctl->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (idle) {
+        for (int r = threadIdx.x; r < 128 * 16; r += kThreads) {
+            const int key = krow0 + r / 16;
+            if (key < p.N[seg]) {
+                const size_t off = ((size_t)((size_t)b * p.N[seg] + key) * p.H + h) * 128;
+                reinterpret_cast<uint4*>(p.dk[seg] + off)[r % 16] = make_uint4(0, 0, 0, 0);
+                reinterpret_cast<uint4*>(p.dv[seg] + off)[r % 16] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        return;
+    }
+    const uint32_t tmem = ctl->tmem_base;
+    const uint32_t sK = smem_u32(smem + Smem::k_off);
+    const uint32_t sV = smem_u32(smem + Smem::v_off);
+    const uint32_t sQ = smem_u32(smem + Smem::q_off);
+    const uint32_t sDO = smem_u32(smem + Smem::do_off);
+    float2* lbuf = reinterpret_cast<float2*>(smem + Smem::l_off);   // (lse * log2 e, D)
+
+    if (warp >= 8) {
+        regs_dec<kRegsProducer>();
+        if ((warp == 8 || warp == 10) && lane == 0) {
+            // ---------------------------------------------- TMA: K, V, then Q (warp 8) / dO (warp 10)
+            const bool is_q = warp == 8;
+            const CUtensorMap* tm = is_q ? p.tm_q : p.tm_do;
+            uint8_t* ring = smem + (is_q ? Smem::q_off : Smem::do_off);
+            uint64_t* full = is_q ? bars->q_full : bars->do_full;
+            uint64_t* empty = is_q ? bars->q_empty : bars->do_empty;
+            if (is_q) {
+                mbar_arrive_expect_tx(&bars->kv_full, 2 * kTileBytes);
+                tma_load_4d(smem + Smem::k_off, &p.tm_k[seg], &bars->kv_full, 0, h, krow0, b);
+                tma_load_4d(smem + Smem::k_off + kHalf128, &p.tm_k[seg], &bars->kv_full, 64, h,
+                            krow0, b);
+                tma_load_4d(smem + Smem::v_off, &p.tm_v[seg], &bars->kv_full, 0, h, krow0, b);
+                tma_load_4d(smem + Smem::v_off + kHalf128, &p.tm_v[seg], &bars->kv_full, 64, h,
+                            krow0, b);
+            }
+            int issued = 0;
+            for (int i = 0; i < nq; ++i) {
+                const int st = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                const int qs = i < nq_vis ? 0 : 1;
+                const int row = (qs ? i - nq_vis : i) * 64;
+                if (!wait(&empty[st], ph ^ 1, ctl)) break;
+                uint8_t* dst = ring + st * kQ64Bytes;
+                mbar_arrive_expect_tx(&full[st], kQ64Bytes);
+                tma_load_4d(dst, &tm[qs], &full[st], 0, h, row, b);
+                tma_load_4d(dst + kHalf64, &tm[qs], &full[st], 64, h, row, b);
+                ++issued;
+            }
+            if (ctl->abort) {
+                for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+                    mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1, nullptr,
+                                      kDrainLimitNs);
+                if (is_q) mbar_wait_bounded(&bars->kv_full, 0, nullptr, kDrainLimitNs);
+            }
+        } else if (warp == 11) {
+            // ---------------------------------------------- (lse * log2 e, D) of each query tile
+            const size_t base = ((size_t)b * p.H + h) * (size_t)(p.N[0] + p.N[1]);
+            for (int i = 0; i < nq; ++i) {
+                const int st = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!wait_warp(&bars->l_empty[st], ph ^ 1, ctl)) break;
+                const int qs = i < nq_vis ? 0 : 1;
+                const int row0q = (qs ? i - nq_vis : i) * 64;
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int q = lane + 32 * r;
+                    const int row = row0q + q;
+                    const bool has = row < p.N[qs] && (qs == 0 || row < L);
+                    const size_t jr = base + (qs ? p.N[0] + row : row);
+                    lbuf[st * 64 + q] =
+                        has ? make_float2(p.lse[jr] * kLog2e, p.delta[jr]) : make_float2(INFINITY, 0.f);
+                }
+                mbar_arrive(&bars->l_full[st]);
+            }
+        } else if (warp == 9 && lane == 0) {
+            // ---------------------------------------------- MMA issuer
+            constexpr uint32_t id_n64 = idesc_bf16_f32(128, 64, 0, 0);
+            constexpr uint32_t id_mn = idesc_bf16_f32(128, 128, 0, 1);
+            bool ok = wait(&bars->kv_full, 0, ctl);
+            const uint64_t kd = kdesc(sK), vd = kdesc(sV);
+            // dV += P^T dO and dK += dS^T Q of query tile ii
+            auto grad_mma = [&](int ii) -> bool {
+                const int pb = ii & 1;
+                const int pst = ii % kStages;
+                if (!wait(&bars->p_full[pb], (ii >> 1) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint64_t dom = mndesc(sDO + pst * kQ64Bytes, kHalf64);
+                const uint64_t qm = mndesc(sQ + pst * kQ64Bytes, kHalf64);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ts(tmem + 256, tmem + 64 * pb + packed_col(s), dom + (uint64_t)s * kMnStep,
+                           id_mn, (ii > 0 || s > 0) ? 1u : 0u);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ts(tmem + 384, tmem + 128 + 64 * pb + packed_col(s),
+                           qm + (uint64_t)s * kMnStep, id_mn, (ii > 0 || s > 0) ? 1u : 0u);
+                mma_commit(&bars->q_empty[pst]);
+                mma_commit(&bars->do_empty[pst]);
+                return true;
+            };
+            for (int i = 0; ok && i < nq; ++i) {
+                const int st = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                const int buf = i & 1;
+                if (!(ok = wait(&bars->q_full[st], ph, ctl))) break;
+                if (!(ok = wait(&bars->do_full[st], ph, ctl))) break;
+                tc_fence_after();
+                const uint64_t qd = kdesc(sQ + st * kQ64Bytes);
+                const uint64_t dod = kdesc(sDO + st * kQ64Bytes);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_ss(tmem + 64 * buf, kd + koff(s, kHalf128), qd + koff(s, kHalf64), id_n64,
+                           s > 0 ? 1u : 0u);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_ss(tmem + 128 + 64 * buf, vd + koff(s, kHalf128), dod + koff(s, kHalf64),
+                           id_n64, s > 0 ? 1u : 0u);
+                mma_commit(&bars->s_full[buf]);
+                if (i > 0 && !(ok = grad_mma(i - 1))) break;
+            }
+            if (ok && (ok = grad_mma(nq - 1))) mma_commit(&bars->o_done);
+            mma_commit(&bars->drain);
+            if (!mbar_wait_bounded(&bars->drain, 0, nullptr, kDrainLimitNs))
+                atomicOr(&g_bwd_status, 1u);
+        }
+    } else {
+        regs_inc<kRegsSoftmax>();
+        // -------------------------------------------------- P^T, dS^T = P^T (dP^T - D)
+        const int wg = warp >> 2;        // query columns [32 wg, 32 wg + 32) of every tile
+        const int quarter = warp & 3;    // tensor-memory lanes (keys) of this warp
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint64_t sl2x2 = f2_pack(p.sl2, p.sl2);
+        bool ok = true;
+        for (int i = 0; i < nq; ++i) {
+            const int buf = i & 1;
+            const int st = i % kStages;
+            if (!(ok = wait_warp(&bars->s_full[buf], (i >> 1) & 1, ctl))) break;
+            if (!(ok = wait_warp(&bars->l_full[st], (i / kStages) & 1, ctl))) break;
+            tc_fence_after();
+            uint32_t sr[32], dr[32];
+            const uint32_t tS = tmem + 64 * buf + 32 * wg + lane_off;
+            const uint32_t tD = tmem + 128 + 64 * buf + 32 * wg + lane_off;
+            tmem_ld32(tS, sr);
+            tmem_ld32(tD, dr);
+            tmem_wait_ld();
+            const float2* lq = lbuf + st * 64 + 32 * wg;
+            uint32_t pp[16], pd[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const float2 l0 = lq[2 * c], l1 = lq[2 * c + 1];
+                const uint64_t x = f2_fma(
+                    f2_pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2,
+                    f2_pack(-l0.x, -l1.x));
+                float x0, x1;
+                f2_unpack(x, x0, x1);
+                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                const uint64_t dd =
+                    f2_sub(f2_pack(__uint_as_float(dr[2 * c]), __uint_as_float(dr[2 * c + 1])),
+                           f2_pack(l0.y, l1.y));
+                float d0, d1;
+                f2_unpack(f2_mul(f2_pack(p0, p1), dd), d0, d1);
+                pp[c] = pack_bf16x2(p0, p1);
+                pd[c] = pack_bf16x2(d0, d1);
+            }
+            tmem_st16(tS, pp);
+            tmem_st16(tD, pd);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars->p_full[buf]);
+                mbar_arrive(&bars->l_empty[st]);
+            }
+        }
+        if (ok) ok = wait_warp(&bars->o_done, 0, ctl);
+        tc_fence_after();
+        const int key = krow0 + quarter * 32 + lane;
+        const bool store = key < p.N[seg];
+        const bool zero = !ok || (seg == 1 && key >= L);
+        const size_t off =
+            ((size_t)((size_t)b * p.N[seg] + (store ? key : 0)) * p.H + h) * 128 + 64 * wg;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {   // 0: dV, 1: dK (times scale)
+            uint4* dst = reinterpret_cast<uint4*>((which ? p.dk[seg] : p.dv[seg]) + off);
+            const float mul = which ? p.scale : 1.f;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tmem + 256 + 128 * which + 64 * wg + 32 * c + lane_off, o);
+                tmem_wait_ld();
+                if (store) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            f[e] = zero ? 0.f : __uint_as_float(o[8 * v + e]) * mul;
+                        dst[4 * c + v] =
+                            make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                       pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace dkv
+
+// ======================================================================
+// fp32 CUDA-core backward (fp32 inputs, 1e-4 accuracy)
+// ======================================================================
+
+// One warp per query row: dQ_i = scale sum_j P_ij (dO_i.v_j - D_i) k_j.
+__global__ void __launch_bounds__(256)
+dq_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv,
+              const float* __restrict__ vv, const float* __restrict__ qc,
+              const float* __restrict__ kc, const float* __restrict__ vc,
+              const int32_t* __restrict__ ctx_len, const float* __restrict__ dov,
+              const float* __restrict__ doc, const float* __restrict__ lse,
+              const float* __restrict__ delta, float* dqv, float* dqc, int Nv, int Nc, int H,
+              float scale) {
+    const int lane = threadIdx.x & 31;
+    const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    if (i >= Nv + Nc) return;
+    int L = Nc;
+    if (ctx_len) {
+        L = ctx_len[b];
+        L = L < 0 ? 0 : (L > Nc ? Nc : L);
+    }
+    const bool vis = i < Nv;
+    const size_t qrow = vis ? ((size_t)b * Nv + i) * H + h : ((size_t)b * Nc + (i - Nv)) * H + h;
+    float4* dst = reinterpret_cast<float4*>((vis ? dqv : dqc) + qrow * 128) + lane;
+    if (!vis && i - Nv >= L) {
+        *dst = make_float4(0.f, 0.f, 0.f, 0.f);
+        return;
+    }
+    const size_t lr = ((size_t)b * H + h) * (size_t)(Nv + Nc) + i;
+    const float li = lse[lr], di = delta[lr];
+    const float4 q = reinterpret_cast<const float4*>((vis ? qv : qc) + qrow * 128)[lane];
+    const float4 g = reinterpret_cast<const float4*>((vis ? dov : doc) + qrow * 128)[lane];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int seg = 0; seg < 2; ++seg) {
+        const int nk = seg == 0 ? Nv : L;
+        const int Ns = seg == 0 ? Nv : Nc;
+        const float* K = seg == 0 ? kv : kc;
+        const float* V = seg == 0 ? vv : vc;
+        for (int j = 0; j < nk; ++j) {
+            const size_t kr = ((size_t)b * Ns + j) * H + h;
+            const float4 k = reinterpret_cast<const float4*>(K + kr * 128)[lane];
+            const float4 v = reinterpret_cast<const float4*>(V + kr * 128)[lane];
+            float s = q.x * k.x + q.y * k.y + q.z * k.z + q.w * k.w;
+            float dp = g.x * v.x + g.y * v.y + g.z * v.z + g.w * v.w;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                s += __shfl_xor_sync(0xffffffffu, s, o);
+                dp += __shfl_xor_sync(0xffffffffu, dp, o);
+            }
+            const float ds = expf(s * scale - li) * (dp - di);
+            acc.x += ds * k.x;
+            acc.y += ds * k.y;
+            acc.z += ds * k.z;
+            acc.w += ds * k.w;
+        }
+    }
+    *dst = make_float4(acc.x * scale, acc.y * scale, acc.z * scale, acc.w * scale);
+}
+
+// One warp per key row: dV_j = sum_i P_ij dO_i, dK_j = scale sum_i dS_ij q_i.
+__global__ void __launch_bounds__(256)
+dkdv_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv,
+                const float* __restrict__ vv, const float* __restrict__ qc,
+                const float* __restrict__ kc, const float* __restrict__ vc,
+                const int32_t* __restrict__ ctx_len, const float* __restrict__ dov,
+                const float* __restrict__ doc, const float* __restrict__ lse,
+                const float* __restrict__ delta, float* dkv, float* dvv, float* dkc, float* dvc,
+                int Nv, int Nc, int H, float scale) {
+    const int lane = threadIdx.x & 31;
+    const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    if (j >= Nv + Nc) return;
+    int L = Nc;
+    if (ctx_len) {
+        L = ctx_len[b];
+        L = L < 0 ? 0 : (L > Nc ? Nc : L);
+    }
+    const bool vis = j < Nv;
+    const size_t kr = vis ? ((size_t)b * Nv + j) * H + h : ((size_t)b * Nc + (j - Nv)) * H + h;
+    float4* dk_dst = reinterpret_cast<float4*>((vis ? dkv : dkc) + kr * 128) + lane;
+    float4* dv_dst = reinterpret_cast<float4*>((vis ? dvv : dvc) + kr * 128) + lane;
+    if (!vis && j - Nv >= L) {
+        *dk_dst = make_float4(0.f, 0.f, 0.f, 0.f);
+        *dv_dst = make_float4(0.f, 0.f, 0.f, 0.f);
+        return;
+    }
+    const float4 k = reinterpret_cast<const float4*>((vis ? kv : kc) + kr * 128)[lane];
+    const float4 v = reinterpret_cast<const float4*>((vis ? vv : vc) + kr * 128)[lane];
+    float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), av = ak;
+    const size_t lb = ((size_t)b * H + h) * (size_t)(Nv + Nc);
+    for (int seg = 0; seg < 2; ++seg) {
+        const int nq = seg == 0 ? Nv : L;
+        const int Ns = seg == 0 ? Nv : Nc;
+        const float* Q = seg == 0 ? qv : qc;
+        const float* G = seg == 0 ? dov : doc;
+        for (int i = 0; i < nq; ++i) {
+            const size_t qr = ((size_t)b * Ns + i) * H + h;
+            const float4 q = reinterpret_cast<const float4*>(Q + qr * 128)[lane];
+            const float4 g = reinterpret_cast<const float4*>(G + qr * 128)[lane];
+            float s = q.x * k.x + q.y * k.y + q.z * k.z + q.w * k.w;
+            float dp = g.x * v.x + g.y * v.y + g.z * v.z + g.w * v.w;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                s += __shfl_xor_sync(0xffffffffu, s, o);
+                dp += __shfl_xor_sync(0xffffffffu, dp, o);
+            }
+            const size_t li = lb + (seg ? Nv + i : i);
+            const float pij = expf(s * scale - lse[li]);
+            const float ds = pij * (dp - delta[li]);
+            av.x += pij * g.x;
+            av.y += pij * g.y;
+            av.z += pij * g.z;
+            av.w += pij * g.w;
+            ak.x += ds * q.x;
+            ak.y += ds * q.y;
+            ak.z += ds * q.z;
+            ak.w += ds * q.w;
+        }
+    }
+    *dk_dst = make_float4(ak.x * scale, ak.y * scale, ak.z * scale, ak.w * scale);
+    *dv_dst = av;
+}
+
+template <typename T>
+cudaError_t run_delta(const void* ov, const void* dov, const void* oc, const void* doc,
+                      const int32_t* ctx_len, float* delta, int B, int Nv, int Nc, int H,
+                      cudaStream_t s) {
+    const long long units = (long long)B * (Nv + Nc) * H;
+    if (units == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    constexpr int GPW = 32 / (128 / (16 / sizeof(T)));
+    long long blocks = (units + 8LL * GPW * 4 - 1) / (8LL * GPW * 4);
+    if (blocks > 8LL * sms) blocks = 8LL * sms;
+    delta_kernel<T><<<(unsigned)blocks, 256, 0, s>>>(
+        static_cast<const T*>(ov), static_cast<const T*>(dov), static_cast<const T*>(oc),
+        static_cast<const T*>(doc), ctx_len, delta, Nv, Nc, H, (uint32_t)units);
+    return cudaGetLastError();
+}
+
+// Refuses to launch unless the compiled kernel uses exactly kRegsLaunch
+// registers per thread (the register split would otherwise wait for ever),
+// and raises its shared-memory limit once per device.
+template <typename K>
+cudaError_t prepare(K kernel, int smem, bool* done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (done[dev]) return cudaSuccess;
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidKernelImage;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    done[dev] = true;
+    return cudaSuccess;
+}
+
+}  // namespace bwd
+
+int launch_joint_attention_bwd_bf16(const void* qv, const void* kv, const void* vv,
+                                    const void* qc, const void* kc, const void* vc,
+                                    const int32_t* ctx_len, const void* ov, const void* oc,
+                                    const void* dov, const void* doc, const float* lse,
+                                    float* delta, void* dqv, void* dkv, void* dvv, void* dqc,
+                                    void* dkc, void* dvc, int B, int Nv, int Nc, int H,
+                                    float softmax_scale, cudaStream_t s) {
+    using namespace bwd;
+    if (!encode_fn()) return -1;
+    if (B == 0 || Nv + Nc == 0) return 0;
+    cudaError_t e = run_delta<__nv_bfloat16>(ov, dov, oc, doc, ctx_len, delta, B, Nv, Nc, H, s);
+    if (e != cudaSuccess) return (int)e;
+
+    dq::Params pq;
+    dkv::Params pk;
+    std::memset(&pq, 0, sizeof(pq));
+    std::memset(&pk, 0, sizeof(pk));
+    const void* src[2][4] = {{qv, kv, vv, dov}, {qc, kc, vc, doc}};
+    const int N[2] = {Nv, Nc};
+    for (int sg = 0; sg < 2; ++sg) {
+        if (N[sg] == 0) continue;
+        bool good = encode_tokens(&pq.tm_q[sg], src[sg][0], B, N[sg], H, 128) &&
+                    encode_tokens(&pq.tm_k[sg], src[sg][1], B, N[sg], H, 128) &&
+                    encode_tokens(&pq.tm_v[sg], src[sg][2], B, N[sg], H, 128) &&
+                    encode_tokens(&pq.tm_do[sg], src[sg][3], B, N[sg], H, 128) &&
+                    encode_tokens(&pk.tm_k[sg], src[sg][1], B, N[sg], H, 128) &&
+                    encode_tokens(&pk.tm_v[sg], src[sg][2], B, N[sg], H, 128) &&
+                    encode_tokens(&pk.tm_q[sg], src[sg][0], B, N[sg], H, 64) &&
+                    encode_tokens(&pk.tm_do[sg], src[sg][3], B, N[sg], H, 64);
+        if (!good) return 1000 + (int)cudaErrorInvalidValue;
+    }
+    const float sl2 = softmax_scale * kLog2e;
+    pq.dq[0] = static_cast<__nv_bfloat16*>(dqv);
+    pq.dq[1] = static_cast<__nv_bfloat16*>(dqc);
+    pk.dk[0] = static_cast<__nv_bfloat16*>(dkv);
+    pk.dk[1] = static_cast<__nv_bfloat16*>(dkc);
+    pk.dv[0] = static_cast<__nv_bfloat16*>(dvv);
+    pk.dv[1] = static_cast<__nv_bfloat16*>(dvc);
+    pq.lse = pk.lse = lse;
+    pq.delta = pk.delta = delta;
+    pq.ctx_len = pk.ctx_len = ctx_len;
+    pq.N[0] = pk.N[0] = Nv;
+    pq.N[1] = pk.N[1] = Nc;
+    pq.H = pk.H = H;
+    pq.q_tiles_vis = pk.k_tiles_vis = (Nv + 127) / 128;
+    pq.sl2 = pk.sl2 = sl2;
+    pq.scale = pk.scale = softmax_scale;
+    pq.wait_ns = pk.wait_ns = wait_timeout_ns();
+
+    static bool dq_ready[64] = {false}, dkv_ready[64] = {false};
+    const int smem_q = dq::Smem::total + 1024;
+    const int smem_k = dkv::Smem::total + 1024;
+    if ((e = prepare(dq::dq_kernel, smem_q, dq_ready)) != cudaSuccess) return (int)e;
+    if ((e = prepare(dkv::dkdv_kernel, smem_k, dkv_ready)) != cudaSuccess) return (int)e;
+    const dim3 grid((Nv + 127) / 128 + (Nc + 127) / 128, H, B);
+    dq::dq_kernel<<<grid, kThreads, smem_q, s>>>(pq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return (int)e;
+    dkv::dkdv_kernel<<<grid, kThreads, smem_k, s>>>(pk);
+    return (int)cudaGetLastError();
+}
+
+cudaError_t launch_joint_attention_bwd_f32(const float* qv, const float* kv, const float* vv,
+                                           const float* qc, const float* kc, const float* vc,
+                                           const int32_t* ctx_len, const float* ov,
+                                           const float* oc, const float* dov, const float* doc,
+                                           const float* lse, float* delta, float* dqv, float* dkv,
+                                           float* dvv, float* dqc, float* dkc, float* dvc, int B,
+                                           int Nv, int Nc, int H, float softmax_scale,
+                                           cudaStream_t s) {
+    using namespace bwd;
+    const int rows = Nv + Nc;
+    if (rows == 0 || B == 0) return cudaSuccess;
+    cudaError_t e = run_delta<float>(ov, dov, oc, doc, ctx_len, delta, B, Nv, Nc, H, s);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((rows + 7) / 8, H, B);
+    dq_f32_kernel<<<grid, 256, 0, s>>>(qv, kv, vv, qc, kc, vc, ctx_len, dov, doc, lse, delta, dqv,
+                                       dqc, Nv, Nc, H, softmax_scale);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    dkdv_f32_kernel<<<grid, 256, 0, s>>>(qv, kv, vv, qc, kc, vc, ctx_len, dov, doc, lse, delta,
+                                         dkv, dvv, dkc, dvc, Nv, Nc, H, softmax_scale);
+    return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_bwd_status(unsigned int* out) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_bwd_status, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_bwd_status, &zero, sizeof(unsigned int));
+}
+
+}  // namespace mmdit

@@ -27,8 +27,9 @@ __global__ void __launch_bounds__(256)
 joint_attn_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv,
                       const float* __restrict__ vv, const float* __restrict__ qc,
                       const float* __restrict__ kc, const float* __restrict__ vc,
-                      const int32_t* __restrict__ ctx_len, float* ov, float* oc, int Nv, int Nc,
-                      int H, float scale, bool windowed, const __grid_constant__ WindowTable win) {
+                      const int32_t* __restrict__ ctx_len, float* ov, float* oc,
+                      float* __restrict__ lse, int Nv, int Nc, int H, float scale, bool windowed,
+                      const __grid_constant__ WindowTable win) {
     const int lane = threadIdx.x & 31;
     const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // joint query row
     const int h = blockIdx.y;
@@ -43,17 +44,21 @@ joint_attn_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv
     const size_t qrow = vis ? ((size_t)b * Nv + i) * H + h : ((size_t)b * Nc + (i - Nv)) * H + h;
     int k0 = 0, k1 = Nv;   // visual keys [k0, k1)
     size_t orow = qrow;    // output row
+    int jrow = i;          // joint row index of the output (raster order)
     if (windowed && vis) {
         int w = 0;
         while (w + 1 < win.count && win.w[w + 1].start <= i) ++w;
         const WindowGeom& g = win.w[w];
         k0 = g.start;
         k1 = g.start + g.te * g.he * g.we;
-        orow = ((size_t)b * Nv + window_to_raster(g, i - g.start, win.Hg, win.Wg)) * H + h;
+        jrow = window_to_raster(g, i - g.start, win.Hg, win.Wg);
+        orow = ((size_t)b * Nv + jrow) * H + h;
     }
     float4* dst = reinterpret_cast<float4*>((vis ? ov : oc) + orow * kHeadDim) + lane;
+    float* lse_row = lse ? lse + ((size_t)b * H + h) * (size_t)(Nv + Nc) + jrow : nullptr;
     if (!vis && i - Nv >= L) {  // padded conditioning query: zero output
         *dst = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lse_row && lane == 0) *lse_row = INFINITY;
         return;
     }
     const float4 q = reinterpret_cast<const float4*>((vis ? qv : qc) + qrow * kHeadDim)[lane];
@@ -86,22 +91,23 @@ joint_attn_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
     *dst = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (lse_row && lane == 0) *lse_row = l > 0.f ? m + logf(l) : INFINITY;
 }
 
 }  // namespace
 
 cudaError_t launch_joint_attention_f32(const float* qv, const float* kv, const float* vv,
                                        const float* qc, const float* kc, const float* vc,
-                                       const int32_t* ctx_len, float* ov, float* oc, int B,
-                                       int Nv, int Nc, int H, float softmax_scale,
+                                       const int32_t* ctx_len, float* ov, float* oc, float* lse,
+                                       int B, int Nv, int Nc, int H, float softmax_scale,
                                        const WindowTable* win, cudaStream_t s) {
     const int rows = Nv + Nc;
     if (rows == 0 || B == 0) return cudaSuccess;
     dim3 grid((rows + 7) / 8, H, B);
     WindowTable tab{};
     if (win) tab = *win;
-    joint_attn_f32_kernel<<<grid, 256, 0, s>>>(qv, kv, vv, qc, kc, vc, ctx_len, ov, oc, Nv, Nc, H,
-                                               softmax_scale, win != nullptr, tab);
+    joint_attn_f32_kernel<<<grid, 256, 0, s>>>(qv, kv, vv, qc, kc, vc, ctx_len, ov, oc, lse, Nv,
+                                               Nc, H, softmax_scale, win != nullptr, tab);
     return cudaGetLastError();
 }
 

@@ -44,6 +44,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "tensor_map.h"
 
 namespace mmdit {
 
@@ -90,6 +91,7 @@ struct Params {
     CUtensorMap tm_k[2];
     CUtensorMap tm_v[2];
     __nv_bfloat16* out[2];
+    float* lse;         // [B, H, Nv + Nc] row log-sum-exp, or null
     const int32_t* ctx_len;
     int N[2];           // Nv, Nc
     int H;
@@ -361,6 +363,9 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                     uint4* dst = reinterpret_cast<uint4*>(
                         p.out[s] + ((size_t)(b * (size_t)p.N[s] + orow) * p.H + h) * kHeadDim);
                     dst[r % 16] = make_uint4(0, 0, 0, 0);
+                    if (p.lse && r % 16 == 0)
+                        p.lse[((size_t)b * p.H + h) * (size_t)(p.N[0] + p.N[1]) +
+                              (s ? p.N[0] + row0 + r / 16 : orow)] = INFINITY;
                 }
             }
         }
@@ -561,6 +566,14 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
             const bool store = orow >= 0;
             const bool zero = !ok || (s == 1 && row >= L);
             const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
+            if (p.lse && store) {
+                // natural-log row log-sum-exp of the scaled scores; m_run and
+                // the exponents are in log2 units
+                const int jrow = s == 0 ? orow : p.N[0] + row;
+                p.lse[((size_t)vwk->b * p.H + vwk->h) * (size_t)(p.N[0] + p.N[1]) + jrow] =
+                    (zero || !(l_run > 0.f)) ? INFINITY
+                                             : (m_run + log2f(l_run)) * 0.6931471805599453f;
+            }
             uint4* dst = reinterpret_cast<uint4*>(
                 p.out[s] +
                 ((size_t)((size_t)vwk->b * p.N[s] + (store ? orow : 0)) * p.H + vwk->h) * kHeadDim);
@@ -602,52 +615,18 @@ namespace {
 
 std::atomic<unsigned long long> g_wait_timeout_ns{0};  // 0: default
 
+
+}  // namespace
+
 uint64_t wait_timeout_ns() {
     const unsigned long long v = g_wait_timeout_ns.load(std::memory_order_relaxed);
     return v ? v : attn::kWaitLimitNs;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-// [B, N, H, 128] bf16 tensor, boxes of 128 tokens x 64 head-dim elements
-// (128 bytes, 128-byte swizzle).  Tokens past N read as zero.
-bool encode_tokens(CUtensorMap* m, const void* base, int B, int N, int H) {
-    const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)H * kHeadDim * 2,
-                                   (cuuint64_t)N * H * kHeadDim * 2};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
-                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-}  // namespace
-
 int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, const void* qc,
                                 const void* kc, const void* vc, const int32_t* ctx_len, void* ov,
-                                void* oc, int B, int Nv, int Nc, int H, float softmax_scale,
-                                const WindowTable* win, cudaStream_t s) {
+                                void* oc, float* lse, int B, int Nv, int Nc, int H,
+                                float softmax_scale, const WindowTable* win, cudaStream_t s) {
     using namespace attn;
     if (!encode_fn()) return -1;
     const int q_tiles = (Nv + kBlockM - 1) / kBlockM + (Nc + kBlockM - 1) / kBlockM;
@@ -672,17 +651,20 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
         if (items >= (1LL << 31)) return (int)cudaErrorInvalidConfiguration;
     }
     if (Nv > 0) {
-        if (!encode_tokens(&p.tm_q[0], qv, B, Nv, H) || !encode_tokens(&p.tm_k[0], kv, B, Nv, H) ||
-            !encode_tokens(&p.tm_v[0], vv, B, Nv, H))
+        if (!encode_tokens(&p.tm_q[0], qv, B, Nv, H, kBlockM) ||
+            !encode_tokens(&p.tm_k[0], kv, B, Nv, H, kBlockN) ||
+            !encode_tokens(&p.tm_v[0], vv, B, Nv, H, kBlockN))
             return 1000 + (int)cudaErrorInvalidValue;
     }
     if (Nc > 0) {
-        if (!encode_tokens(&p.tm_q[1], qc, B, Nc, H) || !encode_tokens(&p.tm_k[1], kc, B, Nc, H) ||
-            !encode_tokens(&p.tm_v[1], vc, B, Nc, H))
+        if (!encode_tokens(&p.tm_q[1], qc, B, Nc, H, kBlockM) ||
+            !encode_tokens(&p.tm_k[1], kc, B, Nc, H, kBlockN) ||
+            !encode_tokens(&p.tm_v[1], vc, B, Nc, H, kBlockN))
             return 1000 + (int)cudaErrorInvalidValue;
     }
     p.out[0] = static_cast<__nv_bfloat16*>(ov);
     p.out[1] = static_cast<__nv_bfloat16*>(oc);
+    p.lse = lse;
     p.ctx_len = ctx_len;
     p.N[0] = Nv;
     p.N[1] = Nc;

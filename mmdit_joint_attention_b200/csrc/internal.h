@@ -52,23 +52,49 @@ cudaError_t launch_gated_residual(const void* x, const void* branch, const float
 // win (null: full joint attention): 3D window attention; the visual inputs
 // are then in the table's window-major order and o_vis is written in raster
 // order.
+// lse (null: not written): [B, H, Nv + Nc] natural-log row log-sum-exp of
+// the scaled scores, +infinity for rows without an output.
 int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv,
                                 const void* qc, const void* kc, const void* vc,
-                                const int32_t* ctx_len, void* ov, void* oc, int B, int Nv,
-                                int Nc, int H, float softmax_scale, const WindowTable* win,
-                                cudaStream_t s);
+                                const int32_t* ctx_len, void* ov, void* oc, float* lse, int B,
+                                int Nv, int Nc, int H, float softmax_scale,
+                                const WindowTable* win, cudaStream_t s);
 
 cudaError_t launch_joint_attention_f32(const float* qv, const float* kv, const float* vv,
                                        const float* qc, const float* kc, const float* vc,
-                                       const int32_t* ctx_len, float* ov, float* oc, int B,
-                                       int Nv, int Nc, int H, float softmax_scale,
+                                       const int32_t* ctx_len, float* ov, float* oc, float* lse,
+                                       int B, int Nv, int Nc, int H, float softmax_scale,
                                        const WindowTable* win, cudaStream_t s);
+
+// Joint-attention backward (no windows).  delta: caller workspace
+// [B, H, Nv + Nc] fp32 (row sums of dO * O, written here); lse from the
+// forward.  Return convention of launch_joint_attention_bf16.
+int launch_joint_attention_bwd_bf16(const void* qv, const void* kv, const void* vv,
+                                    const void* qc, const void* kc, const void* vc,
+                                    const int32_t* ctx_len, const void* ov, const void* oc,
+                                    const void* dov, const void* doc, const float* lse,
+                                    float* delta, void* dqv, void* dkv, void* dvv, void* dqc,
+                                    void* dkc, void* dvc, int B, int Nv, int Nc, int H,
+                                    float softmax_scale, cudaStream_t s);
+cudaError_t launch_joint_attention_bwd_f32(const float* qv, const float* kv, const float* vv,
+                                           const float* qc, const float* kc, const float* vc,
+                                           const int32_t* ctx_len, const float* ov,
+                                           const float* oc, const float* dov, const float* doc,
+                                           const float* lse, float* delta, float* dqv, float* dkv,
+                                           float* dvv, float* dqc, float* dkc, float* dvc, int B,
+                                           int Nv, int Nc, int H, float softmax_scale,
+                                           cudaStream_t s);
+
+// Limit of one bounded pipeline wait (set_wait_timeout_ns, else the default).
+uint64_t wait_timeout_ns();
 
 // Limit of one bounded pipeline wait in the attention kernel (0 = default).
 void set_wait_timeout_ns(unsigned long long ns);
 
 // Device status word (bit set = a bounded wait expired): read-and-clear.
 cudaError_t read_and_clear_device_status(unsigned int* out, cudaStream_t s);
+// The same for the backward kernels' own status word.
+cudaError_t read_and_clear_bwd_status(unsigned int* out);
 
 constexpr int kHeadDim = 128;
 

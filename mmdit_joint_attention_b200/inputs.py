@@ -152,6 +152,15 @@ def _draw_normal(rng: np.random.Generator, shape, dtype: str, std: float = 1.0) 
     return Tensor(a, "f32")
 
 
+def make_grad_outputs(w: Workload, seed: int = 0) -> Dict[str, Tensor]:
+    """Upstream gradients do_vis [B,Nv,H,D] and do_ctx [B,Nc,H,D] of the
+    attention outputs for a backward pass: N(0,1) in the workload's dtype,
+    from their own PCG64 stream (seed + 1000)."""
+    rng = np.random.Generator(np.random.PCG64(seed + 1000))
+    return {"do_vis": _draw_normal(rng, (w.B, w.Nv, w.H, w.D), w.dtype),
+            "do_ctx": _draw_normal(rng, (w.B, w.Nc, w.H, w.D), w.dtype)}
+
+
 def make_inputs(w: Workload, seed: int = 0, parts=("qkv", "scales", "adaln")) -> Dict[str, object]:
     """Draw every input of one block pass for workload ``w``.
 

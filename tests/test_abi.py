@@ -132,3 +132,25 @@ def test_window_validation(L):
     assert q(P, P, Q, Q2, P, P, 1, 320, 2, 128, None, R(w), 1e-6, 1, None) == -1
     assert q(P, P, Q, Q2, P, P, 1, 320, 2, 128, R(g), None, 1e-6, 1, None) == -1
     assert q(P, P, Q, Q2, P, P, 1, 321, 2, 128, R(g), R(w), 1e-6, 1, None) == -2
+
+
+def test_backward_validation(L):
+    f = L.mmdit_joint_attention_bwd
+    Q = ctypes.c_void_p(1 << 20)
+    ptrs = [P] * 6 + [None] + [P] * 4 + [Q, Q] + [P] * 6       # q..v, ctx_len, o, do, lse, delta, grads
+    bad = list(ptrs)
+    bad[11] = None                                             # lse missing
+    assert f(*bad, 1, 8, 8, 2, 128, 0.1, 1, None) == -1
+    bad = list(ptrs)
+    bad[12] = ctypes.c_void_p((1 << 20) + 2)                   # delta misaligned
+    assert f(*bad, 1, 8, 8, 2, 128, 0.1, 1, None) == -3
+    bad = list(ptrs)
+    bad[13] = U                                                # dq_vis misaligned
+    assert f(*bad, 1, 8, 8, 2, 128, 0.1, 1, None) == -3
+    assert f(*ptrs, 1, 8, 8, 2, 64, 0.1, 1, None) == -4         # D != 128
+    assert f(*ptrs, 1, 8, 8, 2, 128, 0.0, 1, None) == -1        # scale
+    assert f(*([None] * 19), 0, 8, 8, 2, 128, 0.1, 1, None) == 0  # empty
+    g = L.mmdit_joint_attention_fwd
+    assert g(P, P, P, P, P, P, None, P, P, None, 1, 8, 8, 2, 128, 0.1, 1, None) == -1  # no lse
+    assert g(P, P, P, P, P, P, None, P, P, ctypes.c_void_p(18), 1, 8, 8, 2, 128, 0.1, 1,
+             None) == -3

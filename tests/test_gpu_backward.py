@@ -1,0 +1,136 @@
+"""GPU parity of the joint-attention backward (and of the forward's row
+log-sum-exp) through the C ABI, against the float64 oracle on the same seeded
+inputs and upstream gradients.
+
+Small and medium cases compare every gradient element; the full 480p and
+ragged workloads compare dq and lse on sampled query rows (each against the
+full key set) and dk / dv through sum rules that hold at any size."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mmdit_joint_attention_b200 import api
+from mmdit_joint_attention_b200 import inputs as I
+from helpers import device_inputs, from_dev, parity, to_dev
+
+pytestmark = pytest.mark.gpu
+
+W = I.WORKLOADS
+
+
+def _ws(w: I.Workload, **kw) -> I.Workload:
+    import dataclasses
+    return dataclasses.replace(w, **kw)
+
+
+def _run(w: I.Workload, seed=0):
+    inp = I.make_inputs(w, seed=seed, parts=("qkv",))
+    gin = I.make_grad_outputs(w, seed=seed)
+    t = device_inputs(inp)
+    do_vis, do_ctx = to_dev(gin["do_vis"]), to_dev(gin["do_ctx"])
+    cl = t["ctx_len"] if w.ctx_len is not None else None
+    ov, oc, lse = api.joint_attention_fwd(t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"],
+                                          t["k_ctx"], t["v_ctx"], cl)
+    g = api.joint_attention_bwd(t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"],
+                                t["v_ctx"], ov, oc, do_vis, do_ctx, lse, cl)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    return inp, gin, {k: from_dev(v) for k, v in g.items()}, from_dev(lse), (ov, oc)
+
+
+def _check_lse(got, ref, name):
+    assert np.array_equal(np.isinf(got), np.isinf(ref)), f"{name}: +inf rows differ"
+    fin = ~np.isinf(ref)
+    if fin.any():
+        err = np.max(np.abs(got[fin] - ref[fin]))
+        assert err <= 1e-3, f"{name}: lse max err {err}"
+
+
+SMALL = {
+    "tiny_f32": W["tiny"],
+    "f32_ragged": _ws(W["tiny"], B=2, H=3, grid=(2, 5, 9), Nc=33, ctx_len=(30, 0)),
+    "block": W["block"],
+    "ragged_small": _ws(W["block"], B=2, H=3, grid=(3, 10, 10), Nc=77, ctx_len=(77, 5)),
+    "odd_tiles": _ws(W["block"], H=2, grid=(1, 1, 257), Nc=0),
+    "cond_all_masked": _ws(W["block"], H=2, grid=(2, 10, 10), Nc=130, ctx_len=(0,)),
+    "batch3_mixed": _ws(W["block"], B=3, H=2, grid=(1, 13, 20), Nc=200, ctx_len=(0, 1, 200)),
+    "medium_2k": _ws(W["block"], H=2, grid=(2, 32, 32), Nc=256),
+}
+
+
+@pytest.mark.parametrize("case", sorted(SMALL))
+def test_backward_full(case):
+    w = SMALL[case]
+    inp, gin, g, lse, _ = _run(w)
+    ref = oracle.joint_attention_bwd(inp["q_vis"].f64, inp["k_vis"].f64, inp["v_vis"].f64,
+                                     inp["q_ctx"].f64, inp["k_ctx"].f64, inp["v_ctx"].f64,
+                                     gin["do_vis"].f64, gin["do_ctx"].f64, inp["ctx_len"])
+    _check_lse(lse, ref["lse"], case)
+    for k in ("dq_vis", "dk_vis", "dv_vis", "dq_ctx", "dk_ctx", "dv_ctx"):
+        parity(g[k], ref[k], w.dtype, f"{case} {k}")
+    for b, L in enumerate(w.ctx_lengths()):
+        for k in ("dq_ctx", "dk_ctx", "dv_ctx"):
+            assert np.all(g[k][b, L:] == 0.0), f"{case} {k}: padded rows must be zero"
+
+
+@pytest.mark.parametrize("name", ["480p", "ragged"])
+def test_backward_sampled_full_size(name):
+    w = W[name]
+    inp, gin, g, lse, _ = _run(w)
+    trip = []
+    for b in range(w.B):
+        for h in range(w.H):
+            rows = I.parity_rows(w, b, h, n_random=128)
+            trip.append(np.stack([np.full_like(rows, b), np.full_like(rows, h), rows], axis=1))
+    trip = np.concatenate(trip)
+    dq, lref = oracle.joint_attention_dq_rows(
+        inp["q_vis"].f64, inp["k_vis"].f64, inp["v_vis"].f64, inp["q_ctx"].f64,
+        inp["k_ctx"].f64, inp["v_ctx"].f64, gin["do_vis"].f64, gin["do_ctx"].f64,
+        inp["ctx_len"], trip)
+    full = np.concatenate([g["dq_vis"], g["dq_ctx"]], axis=1)
+    got = full[trip[:, 0], trip[:, 2], trip[:, 1]]
+    vis = trip[:, 2] < w.Nv
+    parity(got[vis], dq[vis], w.dtype, f"{name} dq_vis rows")
+    parity(got[~vis], dq[~vis], w.dtype, f"{name} dq_ctx rows")
+    _check_lse(lse[trip[:, 0], trip[:, 1], trip[:, 2]], lref, f"{name} lse rows")
+    # Sum rules, per (sample, head, dim): softmax rows sum to one, so
+    # sum_j dv_j = sum_i dO_i over rows with an output, and sum_j dS_ij = 0, so
+    # sum_j dk_j = 0.  Two bf16 roundings of random sign (P before the dV
+    # product, and each stored gradient; relative 2^-8 at most) leave a
+    # deviation of about 0.35 % of the root-sum-square of the terms per entry,
+    # so about 1.2 % at the largest of the 3072 entries of a sample.  The bound
+    # allows 3 %; one missing 128-key tile at 480p moves a sum by about 6 %.
+    for b, L in enumerate(w.ctx_lengths()):
+        do_sum = gin["do_vis"].f64[b].sum(0) + gin["do_ctx"].f64[b, :L].sum(0)
+        dv = np.concatenate([g["dv_vis"][b], g["dv_ctx"][b]], 0)
+        dk = np.concatenate([g["dk_vis"][b], g["dk_ctx"][b]], 0)
+        rss_v = np.sqrt((dv ** 2).sum(0))
+        rss_k = np.sqrt((dk ** 2).sum(0))
+        assert np.all(np.abs(dv.sum(0) - do_sum) <= 3e-2 * rss_v + 1e-6), "sum of dv"
+        assert np.all(np.abs(dk.sum(0)) <= 3e-2 * rss_k + 1e-6), "sum of dk"
+        assert np.all(g["dk_ctx"][b, L:] == 0) and np.all(g["dv_ctx"][b, L:] == 0)
+
+
+def test_forward_with_lse_matches_forward():
+    """The forward with the lse output writes the same o as the plain one."""
+    w = _ws(W["block"], B=2, H=3, grid=(3, 10, 11), Nc=200, ctx_len=(200, 17))
+    t = device_inputs(I.make_inputs(w, seed=4, parts=("qkv",)))
+    args = (t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"], t["v_ctx"], t["ctx_len"])
+    a_v, a_c = api.joint_attention(*args)
+    b_v, b_c, _ = api.joint_attention_fwd(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(a_v, b_v) and torch.equal(a_c, b_c)
+
+
+def test_backward_rejects_bad_arguments():
+    w = W["block"]
+    t = device_inputs(I.make_inputs(w, seed=0, parts=("qkv",)))
+    args = (t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"], t["v_ctx"])
+    ov, oc, lse = api.joint_attention_fwd(*args)
+    with pytest.raises(api._lib.MmditError):
+        api.joint_attention_bwd(*args, ov, oc, ov, oc, lse, softmax_scale=-1.0)
+    bad = torch.empty(t["q_vis"].numel() + 8, dtype=torch.bfloat16, device="cuda")[1:]
+    with pytest.raises(api._lib.MmditError):        # dq_vis not 16-byte aligned
+        api.joint_attention_bwd(*args, ov, oc, ov, oc, lse,
+                                grads={"dq_vis": bad[:t["q_vis"].numel()].view(t["q_vis"].shape)})
