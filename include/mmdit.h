@@ -176,6 +176,33 @@ MMDIT_API int mmdit_joint_attention_bwd(const void* q_vis, const void* k_vis, co
                                         void* dv_ctx, int B, int Nv, int Nc, int H, int D,
                                         float softmax_scale, mmdit_dtype dt, void* stream);
 
+/* Largest B * H * (Nv + Nc) that mmdit_joint_attention_bwd_noalloc accepts:
+ * 4,194,304 rows (its built-in workspace is 16 MiB of fp32 per GPU). */
+#define MMDIT_NOALLOC_MAX_ROWS (1 << 22)
+
+/* mmdit_joint_attention_bwd for callers that cannot allocate device memory.
+ * No passage of the papers corresponds to this entry point: it exists for
+ * callers that must not call cudaMalloc at the point where they run the
+ * backward, for example because another allocator owns the device memory, an
+ * engine forbids allocation once it runs, or a stream is being captured.
+ * Instead of the caller's `delta` workspace it uses a fixed array built into
+ * the library (MMDIT_NOALLOC_MAX_ROWS floats, held on every GPU that loads the
+ * library until the process exits), so the call allocates nothing.
+ *   Arguments, results and errors: as mmdit_joint_attention_bwd without
+ *   `delta`.  B * H * (Nv + Nc) above MMDIT_NOALLOC_MAX_ROWS returns
+ *   MMDIT_ERR_UNSUPPORTED.
+ *   All calls on one GPU share the array: calls whose kernels can overlap on
+ *   the GPU (different streams) race and must be ordered by the caller.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture. */
+MMDIT_API int mmdit_joint_attention_bwd_noalloc(
+    const void* q_vis, const void* k_vis, const void* v_vis, const void* q_ctx, const void* k_ctx,
+    const void* v_ctx, const int32_t* ctx_len, const void* o_vis, const void* o_ctx,
+    const void* do_vis, const void* do_ctx, const float* lse, void* dq_vis, void* dk_vis,
+    void* dv_vis, void* dq_ctx, void* dk_ctx, void* dv_ctx, int B, int Nv, int Nc, int H, int D,
+    float softmax_scale, mmdit_dtype dt, void* stream);
+
 /* 3D window partition of the visual grid ["Seaweed-7B", section 3.2: attention
  * restricted to w_t x w_h x w_w windows, e.g. 1x2x2 and 4x1x1 in alternating
  * layers].  parts[a] is the number of windows along axis a (T, H, W), each in

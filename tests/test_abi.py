@@ -154,3 +154,12 @@ def test_backward_validation(L):
     assert g(P, P, P, P, P, P, None, P, P, None, 1, 8, 8, 2, 128, 0.1, 1, None) == -1  # no lse
     assert g(P, P, P, P, P, P, None, P, P, ctypes.c_void_p(18), 1, 8, 8, 2, 128, 0.1, 1,
              None) == -3
+
+
+def test_noalloc_backward_rejects_sizes_beyond_its_workspace(L):
+    f = L.mmdit_joint_attention_bwd_noalloc
+    f.restype = ctypes.c_int
+    rows = (1 << 22) // 24 + 1            # B = 1, H = 24: one row too many
+    args = [P] * 6 + [None] + [P] * 5 + [P] * 6
+    assert f(*args, 1, rows, 0, 24, 128, ctypes.c_float(0.1), 1, None) == -4
+    assert f(*([None] * 18), 0, 8, 8, 2, 128, ctypes.c_float(0.1), 1, None) == 0
