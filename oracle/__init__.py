@@ -62,6 +62,9 @@ def _configure(lib):
     lib.oracle_joint_attention_dq_rows.argtypes = (
         [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [dp] * 2 + [ctypes.c_int] * 5 +
         [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp, dp])
+    lib.oracle_rmsnorm_rope_bwd.argtypes = [dp, dp, dp, dp, ctypes.c_double,
+                                            ctypes.POINTER(ctypes.c_int), ctypes.c_long,
+                                            ctypes.c_int, ctypes.c_double, dp, dp]
     lib.oracle_adaln_modulate.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3 + [ctypes.c_double]
     lib.oracle_gated_residual.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3
     return lib
@@ -225,6 +228,47 @@ def joint_attention_dq_rows(qv, kv, vv, qc, kc, vc, dov, doc, ctx_len, rows,
             H, D, scale, rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), rows.shape[0],
             _p(dq), _p(lse))
     return dq, lse
+
+
+def grid_positions(grid, pos_scale=(1.0, 1.0, 1.0)) -> np.ndarray:
+    """Scaled (t, h, w) RoPE positions [T*H*W, 3] of the visual tokens in raster
+    order (token n at t = n / (H W), h = (n / W) % H, w = n % W)."""
+    T, Hg, Wg = grid
+    n = np.arange(T * Hg * Wg)
+    p = np.stack([n // (Hg * Wg), (n // Wg) % Hg, n % Wg], axis=1).astype(np.float64)
+    return p * np.asarray(pos_scale, dtype=np.float64)
+
+
+def rmsnorm_rope_bwd(x, g, dy, pos=None, eps: float = 1e-6, base: float = 10000.0,
+                     split=(16, 56, 56)):
+    """Backward of y = RoPE(pos)(rmsnorm(x) * g) for x, dy [B, N, H, D] and
+    positions pos [N, 3] (None: no rotation).  Returns (dx, dg [D])."""
+    x = _f64(x)
+    dy = _f64(dy)
+    g = _f64(g)
+    B, N, H, D = x.shape
+    dx = np.empty_like(x)
+    dg = np.zeros(D, dtype=np.float64)
+    if pos is not None:
+        # one (t, h, w) triple per (b, n, h) row
+        pr = np.ascontiguousarray(np.broadcast_to(_f64(pos).reshape(1, N, 1, 3), (B, N, H, 3)))
+        pp = _p(pr)
+    else:
+        pr = None
+        pp = ctypes.POINTER(ctypes.c_double)()
+    sp = (ctypes.c_int * 3)(*split)
+    _load().oracle_rmsnorm_rope_bwd(_p(x), _p(g), _p(dy), pp, base, sp, B * N * H, D, eps,
+                                    _p(dx), _p(dg))
+    return dx, dg
+
+
+def qk_norm_rope_bwd(q, k, gq, gk, dq_out, dk_out, grid=None, pos_scale=(1.0, 1.0, 1.0),
+                     eps: float = 1e-6, base: float = 10000.0, split=(16, 56, 56)):
+    """Backward of qk_norm_rope: returns dq, dk (inputs' shapes), dgq, dgk [D]."""
+    pos = grid_positions(grid, pos_scale) if grid is not None else None
+    dq, dgq = rmsnorm_rope_bwd(q, gq, dq_out, pos, eps, base, split)
+    dk, dgk = rmsnorm_rope_bwd(k, gk, dk_out, pos, eps, base, split)
+    return dq, dk, dgq, dgk
 
 
 def _grid_struct(grid) -> _Grid:

@@ -457,3 +457,59 @@ void oracle_joint_attention_dq_rows(const double* qv, const double* kv, const do
         free(s);
     }
 }
+
+/* ---- QK-RMSNorm + RoPE backward [V], [S] ----------------------------------
+ * Reverse-mode derivative of y = R(pos) (x / r * g), r = sqrt(mean(x^2) + eps),
+ * for rows x [rows, D] whose RoPE positions are pos [rows, 3] (already scaled;
+ * pos == NULL: no rotation, the conditioning stream), given dy [rows, D]:
+ *   u  = R(pos)^T dy                         (rotation by the opposite angle)
+ *   dg += u * x / r                          (summed over rows)
+ *   dx = g * u / r - x * sum_d(g * u * x) / (D r^3)
+ * dg [D] is accumulated into (caller zeroes it).                             */
+void oracle_rmsnorm_rope_bwd(const double* x, const double* g, const double* dy,
+                             const double* pos, double rope_base, const int* split,
+                             long rows, int D, double eps, double* dx, double* dg)
+{
+    double* part = (double*)calloc((size_t)D, sizeof(double));
+    #pragma omp parallel
+    {
+        double* u = (double*)malloc(sizeof(double) * (size_t)D);
+        double* acc = (double*)calloc((size_t)D, sizeof(double));
+        #pragma omp for schedule(static)
+        for (long r = 0; r < rows; ++r) {
+            const double* xr = x + r * (long)D;
+            const double* dr = dy + r * (long)D;
+            for (int d = 0; d < D; ++d) u[d] = dr[d];
+            if (pos) {
+                int off = 0;
+                for (int a = 0; a < 3; ++a) {
+                    const int d_a = split[a];
+                    for (int j = 0; j < d_a / 2; ++j) {
+                        const double ang = pos[3 * r + a] * pow(rope_base, -2.0 * (double)j / (double)d_a);
+                        const double c = cos(ang), s = sin(ang);
+                        const double a0 = dr[off + 2 * j], a1 = dr[off + 2 * j + 1];
+                        u[off + 2 * j] = a0 * c + a1 * s;        /* transpose of the rotation */
+                        u[off + 2 * j + 1] = -a0 * s + a1 * c;
+                    }
+                    off += d_a;
+                }
+            }
+            double ms = 0.0;
+            for (int d = 0; d < D; ++d) ms += xr[d] * xr[d];
+            const double rr = sqrt(ms / (double)D + eps);
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d) dot += g[d] * u[d] * xr[d];
+            double* dxr = dx + r * (long)D;
+            for (int d = 0; d < D; ++d) {
+                dxr[d] = g[d] * u[d] / rr - xr[d] * dot / ((double)D * rr * rr * rr);
+                acc[d] += u[d] * xr[d] / rr;
+            }
+        }
+        #pragma omp critical
+        for (int d = 0; d < D; ++d) part[d] += acc[d];
+        free(acc);
+        free(u);
+    }
+    for (int d = 0; d < D; ++d) dg[d] += part[d];
+    free(part);
+}

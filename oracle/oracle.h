@@ -38,6 +38,9 @@ void oracle_joint_attention_dq_rows(const double* qv, const double* kv, const do
                                     const int* ctx_len, const double* dov, const double* doc,
                                     int B, int Nv, int Nc, int H, int D, double scale,
                                     const long* rows, long nrows, double* dq_out, double* lse_out);
+void oracle_rmsnorm_rope_bwd(const double* x, const double* g, const double* dy,
+                             const double* pos, double rope_base, const int* split,
+                             long rows, int D, double eps, double* dx, double* dg);
 void oracle_adaln_modulate(const double* x, const double* shift, const double* scale,
                            double* y, int B, int N, int C, double eps);
 void oracle_gated_residual(const double* x, const double* branch, const double* gate,

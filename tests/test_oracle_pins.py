@@ -10,7 +10,8 @@ give mean(V); masked keys have no influence; constant-scale RMSNorm has RMS
 equal to the scale; a window sees nothing outside itself), and for the
 attention backward: central finite differences of sum(dO * O), torch float64
 autograd, scipy's logsumexp, and the gradient sums fixed by softmax rows
-summing to one.  Sources: Vimoo
+summing to one; for the QK-norm + RoPE backward: finite differences through
+the forward oracle and torch autograd through the brute-force rotations.  Sources: Vimoo
 1.0 research page, section 2.2; Wan 2.1 report sections 4.2.1 and 4.3.1;
 Seaweed-7B report, section 3.2.
 
@@ -628,6 +629,63 @@ def pin_bwd_invariants():
     _close(g2["dq_vis"], np.zeros_like(g2["dq_vis"]), 1e-12)
 
 
+# ------------------------------------------------- QK-RMSNorm + RoPE backward
+
+@pin
+def pin_norm_rope_bwd_finite_differences():
+    """dx and dg equal central differences of L = sum(dy * y), y the forward
+    oracle (RMSNorm then 3D RoPE, and RMSNorm alone for the cond stream)."""
+    r = RNG(60)
+    grid = (1, 2, 2)
+    x = r.standard_normal((1, 4, 1, 128))
+    dy = r.standard_normal((1, 4, 1, 128))
+    g = r.uniform(0.5, 1.5, 128)
+    for pos_grid in (grid, None):
+        def loss(xx, gg):
+            y = oracle.rmsnorm(xx, gg, 1e-6)
+            if pos_grid is not None:
+                y = oracle.rope3d(y, pos_grid, (1.0, 1.0, 1.0))
+            return float(np.sum(y * dy))
+        pos = oracle.grid_positions(grid) if pos_grid is not None else None
+        dx, dg = oracle.rmsnorm_rope_bwd(x, g, dy, pos)
+        h = 1e-6
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            num[idx] = (loss(xp, g) - loss(xm, g)) / (2 * h)
+        _close(dx, num, 1e-7)
+        numg = np.zeros_like(g)
+        for d in range(128):
+            gp, gm = g.copy(), g.copy()
+            gp[d] += h
+            gm[d] -= h
+            numg[d] = (loss(x, gp) - loss(x, gm)) / (2 * h)
+        _close(dg, numg, 1e-7)
+
+
+@pin
+def pin_norm_rope_bwd_torch_autograd():
+    """torch float64 autograd through RMSNorm and the explicit rotation
+    matrices of the brute force, at 720p-style scaled positions."""
+    r = RNG(61)
+    grid, ps = (2, 3, 2), (1.0, 1 / 1.5, 1 / 1.5)
+    B, N, H = 2, 12, 3
+    x = r.standard_normal((B, N, H, 128)) * 2.0
+    dy = r.standard_normal((B, N, H, 128))
+    g = r.uniform(0.5, 1.5, 128)
+    R = np.stack([brute.rotation_matrix(p, pos_scale=ps) for p in brute.grid_positions(grid)])
+    xt = torch.tensor(x, requires_grad=True)
+    gt = torch.tensor(g, requires_grad=True)
+    rms = torch.sqrt((xt * xt).mean(-1, keepdim=True) + 1e-6)
+    y = torch.einsum("nde,bnhe->bnhd", torch.from_numpy(R), xt / rms * gt)
+    y.backward(torch.from_numpy(dy))
+    dx, dg = oracle.rmsnorm_rope_bwd(x, g, dy, oracle.grid_positions(grid, ps))
+    _close(dx, xt.grad.numpy(), 1e-12)
+    _close(dg, gt.grad.numpy(), 1e-11)
+
+
 @pytest.mark.parametrize("name", sorted(PINS))
 def test_pin(name):
     PINS[name]()
@@ -673,6 +731,13 @@ MUTANTS = {
                                 "if (nk == 0) continue;"),
     "dqrows_no_delta": ("const double w = scale * s[j] * (g - Dsum);",
                         "const double w = scale * s[j] * g;"),
+    "nrbwd_rotation_not_transposed": ("u[off + 2 * j] = a0 * c + a1 * s;        /* transpose of the rotation */",
+                                      "u[off + 2 * j] = a0 * c - a1 * s;"),
+    "nrbwd_no_dot_term": ("dxr[d] = g[d] * u[d] / rr - xr[d] * dot / ((double)D * rr * rr * rr);",
+                          "dxr[d] = g[d] * u[d] / rr;"),
+    "nrbwd_r_squared": ("dxr[d] = g[d] * u[d] / rr - xr[d] * dot / ((double)D * rr * rr * rr);",
+                        "dxr[d] = g[d] * u[d] / rr - xr[d] * dot / ((double)D * rr * rr);"),
+    "nrbwd_dg_no_norm": ("acc[d] += u[d] * xr[d] / rr;", "acc[d] += u[d] * xr[d];"),
     "window_no_cond_keys": ("for (int j = 0; j < L; ++j) key[nk++] = Nv + j;",
                             "for (int j = 0; j < L && i >= Nv; ++j) key[nk++] = Nv + j;"),
 }
