@@ -441,8 +441,16 @@ def run_ours(args):
     bwd_ms = time_ms(lambda: api.joint_attention_bwd(
         *qkv, t["o_vis"], t["o_ctx"], do_vis, do_ctx, lse, t["ctx_len"], delta=delta,
         grads=grads), reps=5)
+    nr_ms = time_ms(lambda: api.qk_norm_rope_bwd(
+        t["q_vis"], t["k_vis"], t["gq_vis"], t["gk_vis"], do_vis, do_vis, grid=w.grid,
+        pos_scale=w.pos_scale, dq=grads["dq_vis"], dk=grads["dk_vis"]))
+    nr_bytes = 6 * B * Nv * C * 2
     pairs = H * sum((Nv + L) ** 2 for L in w.ctx_lengths())
-    bwd_rows = {"backward": {
+    bwd_rows = {"qk_norm_rope_bwd_vis": {"ms": nr_ms, "GB/s": nr_bytes / (nr_ms * 1e-3) / 1e9,
+                                         "frac_hbm": nr_bytes / (nr_ms * 1e-3) / 1e9 /
+                                                     float(peaks()[0]["hbm_gbs"]),
+                                         "bytes": nr_bytes},
+                "backward": {
         "ms": bwd_ms, "fwd_with_lse_ms": fwd_lse_ms,
         "TFLOP/s_beta8": 8.0 * D * pairs / (bwd_ms * 1e-3) / 1e12,
         "TFLOP/s_executed": 14.0 * D * pairs / (bwd_ms * 1e-3) / 1e12,

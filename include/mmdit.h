@@ -83,6 +83,28 @@ MMDIT_API int mmdit_qk_norm_rope(const void* q_in, const void* k_in, void* q_out
                        int B, int N, int H, int D, const mmdit_grid* grid, float eps,
                        mmdit_dtype dt, void* stream);
 
+/* Backward of mmdit_qk_norm_rope [the reverse-mode derivative of the QK-RMSNorm
+ * + RoPE of Vimoo §2.2; the Seaweed-7B report, section 3.4, fuses the norm and
+ * RoPE of both passes]: for each row x of q_in / k_in with r = sqrt(mean(x^2)
+ * + eps), scale g and upstream gradient dy of the row of q_out / k_out:
+ *   u  = R^T dy      (the RoPE rotation of the row, reversed; u = dy if grid is NULL)
+ *   dx = g * u / r - x * sum_d(g * u * x) / (D r^3)
+ *   dg = sum over all rows of u * x / r
+ *   q_in, k_in       [B, N, H, D] dt, the forward's inputs
+ *   dq_out, dk_out   [B, N, H, D] dt, gradients of the forward's outputs
+ *   dq_in, dk_in     [B, N, H, D] dt, written (may equal dq_out / dk_out)
+ *   q_scale, k_scale [D] fp32;  dq_scale, dk_scale [D] fp32, written
+ *   grid, eps: as mmdit_qk_norm_rope (MM-RoPE text positions not supported).
+ * dq_scale / dk_scale are summed with floating-point atomics, so their last
+ * bits may differ from run to run.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_qk_norm_rope_bwd(const void* q_in, const void* k_in, const void* dq_out,
+                                     const void* dk_out, const float* q_scale,
+                                     const float* k_scale, void* dq_in, void* dk_in,
+                                     float* dq_scale, float* dk_scale, int B, int N, int H, int D,
+                                     const mmdit_grid* grid, float eps, mmdit_dtype dt,
+                                     void* stream);
+
 /* Text-token positions of MM-RoPE ["Seaweed-7B: Cost-Effective Training of
  * Video Generation Foundation Model", section 3.2: text tokens get a 1D
  * position compatible with the video's 3D one, shared by its three

@@ -82,6 +82,30 @@ def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, q_scale: torch.Tensor, k_scal
     return q_out, k_out
 
 
+def qk_norm_rope_bwd(q: torch.Tensor, k: torch.Tensor, q_scale: torch.Tensor,
+                     k_scale: torch.Tensor, dq_out: torch.Tensor, dk_out: torch.Tensor,
+                     grid: Optional[Sequence[int]] = None, pos_scale=(1.0, 1.0, 1.0),
+                     eps: float = 1e-6, rope_base: float = 10000.0, split=(16, 56, 56),
+                     dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+                     stream=None):
+    """Backward of qk_norm_rope: (dq, dk, dq_scale, dk_scale) for the forward
+    inputs q, k and the gradients dq_out, dk_out of its outputs."""
+    dt = _dtype(q, k, dq_out, dk_out)
+    _f32(q_scale, k_scale)
+    B, N, H, D = q.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dgq = torch.empty(D, dtype=torch.float32, device=q.device)
+    dgk = torch.empty(D, dtype=torch.float32, device=q.device)
+    g = make_grid(grid, pos_scale, rope_base, split) if grid is not None else None
+    st = _lib.lib().mmdit_qk_norm_rope_bwd(
+        _ptr(q), _ptr(k), _ptr(dq_out), _ptr(dk_out), _ptr(q_scale), _ptr(k_scale), _ptr(dq),
+        _ptr(dk), _ptr(dgq), _ptr(dgk), B, N, H, D, ctypes.byref(g) if g is not None else None,
+        eps, dt, _stream(stream))
+    check("mmdit_qk_norm_rope_bwd", st)
+    return dq, dk, dgq, dgk
+
+
 def qk_norm_rope_text(q: torch.Tensor, k: torch.Tensor, q_scale: torch.Tensor,
                       k_scale: torch.Tensor, pos_offset: float = 0.0, eps: float = 1e-6,
                       rope_base: float = 10000.0, split=(16, 56, 56),

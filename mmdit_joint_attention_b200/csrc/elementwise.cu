@@ -346,6 +346,190 @@ cudaError_t run_qk(const void* q_in, const void* k_in, void* q_out, void* k_out,
     return cudaGetLastError();
 }
 
+// ----------------------------------------------------------------------
+// Backward of QK-RMSNorm + RoPE.  For a row x with r = sqrt(mean(x^2) + eps),
+// forward y = R (g * x / r), and the upstream gradient dy:
+//   u  = R^T dy                      (each pair turned by the opposite angle)
+//   dx = g * u / r - x * sum(g * u * x) / (D r^3)
+//   dg = sum over rows of u * x / r
+// Same lane mapping, angle table and rows-in-flight structure as the forward
+// kernel.  Each lane keeps the dg partial sums of its E head dims in registers
+// for the whole grid-stride loop; at the end they are summed over the block in
+// shared memory and added to dg with one atomic per dim per block (dg is
+// zeroed on the stream before the launch).
+// ----------------------------------------------------------------------
+constexpr int kQkBwdUnroll = 2;   // rows in flight per lane group (x and dy of q and k each)
+
+template <typename T, int ROPE, bool TABLE, int UNR>
+__global__ void __launch_bounds__(256, 2)
+qk_norm_rope_bwd_kernel(const T* __restrict__ q_in, const T* __restrict__ k_in,
+                        const T* __restrict__ dq_out, const T* __restrict__ dk_out,
+                        T* __restrict__ dq_in, T* __restrict__ dk_in,
+                        const float* __restrict__ gq, const float* __restrict__ gk,
+                        float* __restrict__ dgq, float* __restrict__ dgk, uint32_t units,
+                        float eps, const RopeParams rp) {
+    constexpr int E = Elems<T>::E;
+    constexpr int LPR = kHeadDim / E;
+    constexpr int GPW = 32 / LPR;
+    extern __shared__ float4 rope_tab4[];
+    const float2* tab = reinterpret_cast<const float2*>(rope_tab4);
+    __shared__ float dg_block[2 * kHeadDim];
+
+    for (int i = threadIdx.x; i < 2 * kHeadDim; i += blockDim.x) dg_block[i] = 0.f;
+    if (ROPE == kRopeGrid && TABLE) {
+        float2* wtab = reinterpret_cast<float2*>(rope_tab4);
+        for (int e = threadIdx.x; e < rp.tab_entries; e += blockDim.x) {
+            const int a = e < rp.tab_off[1] ? 0 : (e < rp.tab_off[2] ? 1 : 2);
+            const int local = e - rp.tab_off[a];
+            const int pos = local / rp.stride[a];
+            const int j = local - pos * rp.stride[a];
+            float c = 1.f, sn = 0.f;
+            if (j < rp.split[a] / 2) {
+                const float ang =
+                    (float)((double)pos * rp.pos_scale[a] * rp.freq[rp.off[a] / 2 + j]);
+                sincosf(ang, &sn, &c);
+            }
+            wtab[e] = make_float2(c, sn);
+        }
+    }
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int g = lane % LPR;
+    const int grp = lane / LPR;
+    const int d0 = g * E;
+    float wq[E], wk[E], aq[E], ak[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        wq[i] = gq[d0 + i];
+        wk[i] = gk[d0 + i];
+        aq[i] = 0.f;
+        ak[i] = 0.f;
+    }
+    const int axis = d0 < rp.off[1] ? 0 : (d0 < rp.off[2] ? 1 : 2);
+    const int jb = (d0 - rp.off[axis]) >> 1;
+
+    const uint32_t warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t uw = warp0 * (GPW * UNR); uw < units; uw += nwarps * (GPW * UNR)) {
+        uint4 rq[UNR], rk[UNR], rdq[UNR], rdk[UNR];
+#pragma unroll
+        for (int r = 0; r < UNR; ++r) {
+            const uint32_t u = uw + r * GPW + grp;
+            const bool live = u < units;
+            const size_t base = (size_t)(live ? u : 0) * kHeadDim + d0;
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            rq[r] = live ? ld16(q_in + base) : z;
+            rk[r] = live ? ld16(k_in + base) : z;
+            rdq[r] = live ? ld16(dq_out + base) : z;
+            rdk[r] = live ? ld16(dk_out + base) : z;
+        }
+#pragma unroll
+        for (int r = 0; r < UNR; ++r) {
+            const uint32_t u = uw + r * GPW + grp;
+            float xq[E], xk[E], uq[E], uk[E];
+            unpack(rq[r], xq);
+            unpack(rk[r], xk);
+            unpack(rdq[r], uq);
+            unpack(rdk[r], uk);
+            if (ROPE == kRopeGrid) {
+                const uint32_t uu = u < units ? u : 0;
+                const uint32_t bn = fdiv(uu, rp.H);
+                const uint32_t n = bn - fdiv(bn, rp.N) * rp.N.d;
+                const uint32_t t = fdiv(n, rp.HW);
+                const uint32_t rem = n - t * rp.HW.d;
+                const uint32_t hh = fdiv(rem, rp.W);
+                const uint32_t pos = axis == 0 ? t : (axis == 1 ? hh : rem - hh * rp.W.d);
+                float cs[E];
+                if (TABLE) {
+                    const float4* p4 = reinterpret_cast<const float4*>(
+                        tab + rp.tab_off[axis] + pos * rp.stride[axis] + jb);
+#pragma unroll
+                    for (int i = 0; i < E / 4; ++i) {
+                        const float4 v = p4[i];
+                        cs[4 * i] = v.x;
+                        cs[4 * i + 1] = v.y;
+                        cs[4 * i + 2] = v.z;
+                        cs[4 * i + 3] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int pp = 0; pp < E / 2; ++pp) {
+                        const float ang = (float)((double)pos * rp.pos_scale[axis] *
+                                                  rp.freq[rp.off[axis] / 2 + jb + pp]);
+                        sincosf(ang, &cs[2 * pp + 1], &cs[2 * pp]);
+                    }
+                }
+#pragma unroll
+                for (int pp = 0; pp < E / 2; ++pp) {
+                    const float c = cs[2 * pp], sn = cs[2 * pp + 1];
+                    const float q0 = uq[2 * pp], q1 = uq[2 * pp + 1];
+                    const float k0 = uk[2 * pp], k1 = uk[2 * pp + 1];
+                    uq[2 * pp] = q0 * c + q1 * sn;
+                    uq[2 * pp + 1] = q1 * c - q0 * sn;
+                    uk[2 * pp] = k0 * c + k1 * sn;
+                    uk[2 * pp + 1] = k1 * c - k0 * sn;
+                }
+            }
+            // row sums: mean square of x and sum(g * u * x), for q and k
+            float sq = 0.f, sk = 0.f, tq = 0.f, tk = 0.f;
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                sq = fmaf(xq[i], xq[i], sq);
+                sk = fmaf(xk[i], xk[i], sk);
+                tq = fmaf(wq[i] * uq[i], xq[i], tq);
+                tk = fmaf(wk[i] * uk[i], xk[i], tk);
+            }
+#pragma unroll
+            for (int o = LPR / 2; o >= 1; o >>= 1) {
+                sq += __shfl_xor_sync(kFull, sq, o);
+                sk += __shfl_xor_sync(kFull, sk, o);
+                tq += __shfl_xor_sync(kFull, tq, o);
+                tk += __shfl_xor_sync(kFull, tk, o);
+            }
+            const float iq = rsqrtf(sq * (1.0f / kHeadDim) + eps);   // 1 / r
+            const float ik = rsqrtf(sk * (1.0f / kHeadDim) + eps);
+            const float cq = tq * iq * iq * iq * (1.0f / kHeadDim);    // sum(g u x) / (D r^3)
+            const float ck = tk * ik * ik * ik * (1.0f / kHeadDim);
+            const bool live = u < units;
+            float oq[E], ok[E];
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                oq[i] = wq[i] * uq[i] * iq - xq[i] * cq;
+                ok[i] = wk[i] * uk[i] * ik - xk[i] * ck;
+                if (live) {
+                    aq[i] = fmaf(uq[i] * xq[i], iq, aq[i]);
+                    ak[i] = fmaf(uk[i] * xk[i], ik, ak[i]);
+                }
+            }
+            if (live) {
+                const size_t base = (size_t)u * kHeadDim + d0;
+                st16(dq_in + base, pack(oq));
+                st16(dk_in + base, pack(ok));
+            }
+        }
+    }
+    // dg: lanes with the same head dims (g, g + LPR, ...) first, then the block
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+#pragma unroll
+        for (int o = LPR; o < 32; o <<= 1) {
+            aq[i] += __shfl_xor_sync(kFull, aq[i], o);
+            ak[i] += __shfl_xor_sync(kFull, ak[i], o);
+        }
+    }
+    if (grp == 0) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            atomicAdd(&dg_block[d0 + i], aq[i]);
+            atomicAdd(&dg_block[kHeadDim + d0 + i], ak[i]);
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 2 * kHeadDim; i += blockDim.x)
+        atomicAdd(i < kHeadDim ? &dgq[i] : &dgk[i - kHeadDim], dg_block[i]);
+}
+
 // ======================================================================
 // Row permutation between raster and window-major order
 // ======================================================================
@@ -786,6 +970,93 @@ cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out,
     }
     MMDIT_QK_DISPATCH(float)
 #undef MMDIT_QK_DISPATCH
+}
+
+template <typename T, int ROPE, bool TABLE>
+cudaError_t run_qk_bwd(const void* q_in, const void* k_in, const void* dq_out, const void* dk_out,
+                       const float* gq, const float* gk, void* dq_in, void* dk_in, float* dgq,
+                       float* dgk, uint32_t units, float eps, const RopeParams& rp, size_t smem,
+                       cudaStream_t s) {
+    constexpr int UNR = kQkBwdUnroll;
+    auto kern = qk_norm_rope_bwd_kernel<T, ROPE, TABLE, UNR>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    constexpr int GPW = 32 / (kHeadDim / Elems<T>::E);
+    const long long need = ((long long)units + 8LL * GPW * UNR - 1) / (8LL * GPW * UNR);
+    long long blocks = (long long)sm_count() * per_sm;
+    if (need < blocks) blocks = need;
+    if (blocks < 1) blocks = 1;
+    kern<<<(unsigned)blocks, 256, smem, s>>>(
+        static_cast<const T*>(q_in), static_cast<const T*>(k_in), static_cast<const T*>(dq_out),
+        static_cast<const T*>(dk_out), static_cast<T*>(dq_in), static_cast<T*>(dk_in), gq, gk, dgq,
+        dgk, units, eps, rp);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_qk_norm_rope_bwd(const void* q_in, const void* k_in, const void* dq_out,
+                                    const void* dk_out, const float* gq, const float* gk,
+                                    void* dq_in, void* dk_in, float* dgq, float* dgk, int B, int N,
+                                    int H, const RopeGrid* grid, float eps, bool bf16,
+                                    cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(dgq, 0, kHeadDim * sizeof(float), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dgk, 0, kHeadDim * sizeof(float), s);
+    if (e != cudaSuccess) return e;
+    const long long units_ll = (long long)B * N * H;
+    if (units_ll == 0) return cudaSuccess;
+    const uint32_t units = (uint32_t)units_ll;
+    RopeParams rp{};
+    rp.H = make_fastdiv((uint32_t)H);
+    rp.N = make_fastdiv((uint32_t)N);
+    size_t smem = 0;
+    bool table = false;
+    if (grid) {
+        rp.Hg = grid->H;
+        rp.HW = make_fastdiv((uint32_t)grid->H * (uint32_t)grid->W);
+        rp.W = make_fastdiv((uint32_t)grid->W);
+        const int extent[3] = {grid->T, grid->H, grid->W};
+        int off = 0, toff = 0;
+        for (int a = 0; a < 3; ++a) {
+            rp.split[a] = grid->split[a];
+            rp.off[a] = off;
+            rp.pos_scale[a] = grid->pos_scale[a];
+            const int half = grid->split[a] / 2;
+            for (int j = 0; j < half; ++j)
+                rp.freq[off / 2 + j] = std::pow(grid->base, -2.0 * j / (double)grid->split[a]);
+            rp.stride[a] = (half + 1) & ~1;
+            rp.tab_off[a] = toff;
+            toff += extent[a] * rp.stride[a];
+            off += grid->split[a];
+        }
+        rp.tab_entries = toff;
+        smem = (size_t)toff * sizeof(float2);
+        table = smem <= 64 * 1024;
+        if (!table) smem = 0;
+    } else {
+        rp.off[1] = rp.off[2] = kHeadDim;
+        rp.Hg = 1;
+        rp.HW = rp.W = make_fastdiv(1);
+    }
+#define MMDIT_QK_BWD(T)                                                                       \
+    if (!grid)                                                                               \
+        return run_qk_bwd<T, kRopeNone, false>(q_in, k_in, dq_out, dk_out, gq, gk, dq_in, dk_in, \
+                                               dgq, dgk, units, eps, rp, 0, s);               \
+    if (table)                                                                               \
+        return run_qk_bwd<T, kRopeGrid, true>(q_in, k_in, dq_out, dk_out, gq, gk, dq_in, dk_in,  \
+                                              dgq, dgk, units, eps, rp, smem, s);             \
+    return run_qk_bwd<T, kRopeGrid, false>(q_in, k_in, dq_out, dk_out, gq, gk, dq_in, dk_in,     \
+                                           dgq, dgk, units, eps, rp, 0, s);
+    if (bf16) {
+        MMDIT_QK_BWD(__nv_bfloat16)
+    }
+    MMDIT_QK_BWD(float)
+#undef MMDIT_QK_BWD
 }
 
 cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float* scale,

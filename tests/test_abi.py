@@ -163,3 +163,14 @@ def test_noalloc_backward_rejects_sizes_beyond_its_workspace(L):
     args = [P] * 6 + [None] + [P] * 5 + [P] * 6
     assert f(*args, 1, rows, 0, 24, 128, ctypes.c_float(0.1), 1, None) == -4
     assert f(*([None] * 18), 0, 8, 8, 2, 128, ctypes.c_float(0.1), 1, None) == 0
+
+
+def test_qk_norm_rope_bwd_validation(L):
+    f = L.mmdit_qk_norm_rope_bwd
+    g = _lib.Grid(2, 4, 4, (ctypes.c_float * 3)(1, 1, 1), 10000.0, (ctypes.c_int * 3)(16, 56, 56))
+    R = ctypes.byref
+    assert f(P, P, P, P, P, P, P, P, P, P, 1, 32, 2, 64, R(g), 1e-6, 1, None) == -4   # D
+    assert f(P, P, P, P, P, P, P, P, None, P, 1, 32, 2, 128, R(g), 1e-6, 1, None) == -1
+    assert f(P, P, P, P, P, P, U, P, P, P, 1, 32, 2, 128, R(g), 1e-6, 1, None) == -3
+    assert f(P, P, P, P, P, P, P, P, P, P, 1, 31, 2, 128, R(g), 1e-6, 1, None) == -2  # N != THW
+    assert f(P, P, P, P, P, P, P, P, P, P, 1, 32, 2, 128, R(g), -1.0, 1, None) == -1  # eps

@@ -134,3 +134,29 @@ def test_backward_rejects_bad_arguments():
     with pytest.raises(api._lib.MmditError):        # dq_vis not 16-byte aligned
         api.joint_attention_bwd(*args, ov, oc, ov, oc, lse,
                                 grads={"dq_vis": bad[:t["q_vis"].numel()].view(t["q_vis"].shape)})
+
+
+# ------------------------------------------------------ QK-RMSNorm + RoPE backward
+
+@pytest.mark.parametrize("name", ["tiny", "block", "480p", "720p", "ragged"])
+def test_qk_norm_rope_bwd(name):
+    """dx against the oracle in full (bf16 / fp32 criterion); dg, a sum over
+    every row, within 1e-3 of its largest entry."""
+    w = W[name]
+    inp = I.make_inputs(w, seed=2, parts=("qkv", "scales"))
+    gin = I.make_grad_outputs(w, seed=2)
+    t = device_inputs(inp)
+    for stream, grid, dO in (("vis", w.grid, gin["do_vis"]), ("ctx", None, gin["do_ctx"])):
+        dy = to_dev(dO)
+        dq, dk, dgq, dgk = api.qk_norm_rope_bwd(
+            t["q_" + stream], t["k_" + stream], t["gq_" + stream], t["gk_" + stream], dy, dy,
+            grid=grid, pos_scale=w.pos_scale)
+        torch.cuda.synchronize()
+        rq, rk, rgq, rgk = oracle.qk_norm_rope_bwd(
+            inp["q_" + stream].f64, inp["k_" + stream].f64, inp["gq_" + stream],
+            inp["gk_" + stream], dO.f64, dO.f64, grid=grid, pos_scale=w.pos_scale)
+        parity(from_dev(dq), rq, w.dtype, f"{name} dq_{stream}")
+        parity(from_dev(dk), rk, w.dtype, f"{name} dk_{stream}")
+        for got, ref, n in ((dgq, rgq, "dgq"), (dgk, rgk, "dgk")):
+            err = np.max(np.abs(from_dev(got) - ref)) if ref.size else 0.0
+            assert err <= 1e-3 * max(np.abs(ref).max(), 1e-30), (name, stream, n, err)
