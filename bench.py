@@ -417,6 +417,8 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         return a.elapsed_time(z) / reps
 
+    k_n_vis = torch.empty_like(t["k_vis"])
+    k_n_ctx = torch.empty_like(t["k_ctx"])
     y_next = torch.empty_like(t["x_vis"])
     x_next = torch.empty_like(t["x_vis"])
     rm_ms = time_ms(lambda: api.residual_modulate(
@@ -427,6 +429,21 @@ def run_ours(args):
     txt_ms = time_ms(lambda: api.qk_norm_rope_text(
         t["q_ctx"], t["k_ctx"], t["gq_ctx"], t["gk_ctx"], pos_offset=float(max(w.grid)),
         q_out=q_txt, k_out=k_txt))
+    # q normalised inside the attention kernel: k alone through the prologue
+    kq_ms = time_ms(lambda: (
+        api.k_norm_rope(t["k_vis"], t["gk_vis"], grid=w.grid, pos_scale=w.pos_scale,
+                        k_out=k_n_vis),
+        api.k_norm_rope(t["k_ctx"], t["gk_ctx"], k_out=k_n_ctx)))
+    qn_ms = time_ms(lambda: api.joint_attention_qnorm(
+        t["q_vis"], k_n_vis, t["v_vis"], t["q_ctx"], k_n_ctx, t["v_ctx"], t["gq_vis"],
+        t["gq_ctx"], grid=w.grid, pos_scale=w.pos_scale, ctx_len=t["ctx_len"],
+        o_vis=t["o_vis"], o_ctx=t["o_ctx"]), reps=10)
+    qn_rows = {"qnorm_in_attention": {
+        "k_norm_rope_ms": kq_ms, "attention_qnorm_ms": qn_ms,
+        "attention_qnorm_TFLOP/s": w.attention_flops() / (qn_ms * 1e-3) / 1e12,
+        "fused_ms": kq_ms + qn_ms,
+        "unfused_ms": kern_ms["qk_norm_rope"] + kern_ms["joint_attention"]}}
+
     # backward: forward with the row log-sum-exp, then D, dQ and dK/dV
     gen = torch.Generator(device=dev).manual_seed(1000 + rank)
     do_vis = torch.randn(t["q_vis"].shape, generator=gen, device=dev).to(torch.bfloat16)
@@ -543,7 +560,7 @@ def run_ours(args):
                               Nv / (Nv + Nc)},
             "qk_norm_rope_text_ctx": {
                 "ms": txt_ms, "GB/s": 4 * B * Nc * C * 2 / (txt_ms * 1e-3) / 1e9},
-            **win_rows, **bwd_rows},
+            **win_rows, **bwd_rows, **qn_rows},
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,

@@ -154,6 +154,35 @@ MMDIT_API int mmdit_joint_attention(const void* q_vis, const void* k_vis, const 
                           int B, int Nv, int Nc, int H, int D, float softmax_scale,
                           mmdit_dtype dt, void* stream);
 
+/* mmdit_qk_norm_rope for k alone: the RMSNorm (scale k_scale) and, with a
+ * grid, the 3D RoPE of every row of k_in into k_out (may equal k_in).  Pairs
+ * with mmdit_joint_attention_qnorm, which normalises q itself.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_k_norm_rope(const void* k_in, void* k_out, const float* k_scale, int B, int N,
+                                int H, int D, const mmdit_grid* grid, float eps, mmdit_dtype dt,
+                                void* stream);
+
+/* mmdit_joint_attention with the QK-RMSNorm and 3D RoPE of q done inside the
+ * attention kernel [Vimoo §2.2 QK-norm and RoPE; the Seaweed-7B report,
+ * section 3.4, fuses the attention preprocessing]: q_vis / q_ctx are the RAW
+ * queries; each query tile is normalised (q_scale_vis / q_scale_ctx, [D] fp32,
+ * eps) and, for visual rows when grid is not NULL, rotated by its grid
+ * position, right after it is loaded and before any product reads it.  k_vis /
+ * k_ctx must already be normalised and rotated (mmdit_k_norm_rope).  Saves
+ * one write and one read of q against mmdit_qk_norm_rope + the attention.
+ *   grid: host pointer as for mmdit_qk_norm_rope (Nv == T*H*W), or NULL for
+ *   no rotation.  bf16 only (MMDIT_ERR_UNSUPPORTED otherwise).
+ *   Other arguments as mmdit_joint_attention.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_joint_attention_qnorm(const void* q_vis, const void* k_vis,
+                                          const void* v_vis, const void* q_ctx,
+                                          const void* k_ctx, const void* v_ctx,
+                                          const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                                          const float* q_scale_vis, const float* q_scale_ctx,
+                                          const mmdit_grid* grid, float eps, int B, int Nv,
+                                          int Nc, int H, int D, float softmax_scale,
+                                          mmdit_dtype dt, void* stream);
+
 /* mmdit_joint_attention that also writes, for training, the row log-sum-exp
  * the backward pass needs [Vimoo §2.2 joint attention; the Seaweed-7B report,
  * section 3.4, trains its forward and backward]:

@@ -156,6 +156,52 @@ def joint_attention(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
     return o_vis, o_ctx
 
 
+def k_norm_rope(k: torch.Tensor, k_scale: torch.Tensor, grid: Optional[Sequence[int]] = None,
+                pos_scale=(1.0, 1.0, 1.0), eps: float = 1e-6, rope_base: float = 10000.0,
+                split=(16, 56, 56), k_out: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """RMSNorm (+ 3D RoPE with a grid) of k alone, in place unless k_out is given;
+    for joint_attention_qnorm, which normalises q itself."""
+    dt = _dtype(k)
+    _f32(k_scale)
+    B, N, H, D = k.shape
+    k_out = k if k_out is None else k_out
+    g = make_grid(grid, pos_scale, rope_base, split) if grid is not None else None
+    st = _lib.lib().mmdit_k_norm_rope(_ptr(k), _ptr(k_out), _ptr(k_scale), B, N, H, D,
+                                      ctypes.byref(g) if g is not None else None, eps, dt,
+                                      _stream(stream))
+    check("mmdit_k_norm_rope", st)
+    return k_out
+
+
+def joint_attention_qnorm(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, q_scale_vis, q_scale_ctx,
+                          grid: Optional[Sequence[int]] = None, pos_scale=(1.0, 1.0, 1.0),
+                          ctx_len=None, eps: float = 1e-6, rope_base: float = 10000.0,
+                          split=(16, 56, 56), softmax_scale: Optional[float] = None, o_vis=None,
+                          o_ctx=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """joint_attention on raw q: the kernel RMS-normalises q (and rotates the
+    visual rows when ``grid`` is given) after loading it.  k must already be
+    normalised (k_norm_rope)."""
+    dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx)
+    _f32(q_scale_vis, q_scale_ctx)
+    B, Nv, H, D = q_vis.shape
+    Nc = q_ctx.shape[1]
+    o_vis = torch.empty_like(q_vis) if o_vis is None else o_vis
+    o_ctx = torch.empty_like(q_ctx) if o_ctx is None else o_ctx
+    if ctx_len is not None and (ctx_len.dtype != torch.int32 or not ctx_len.is_cuda):
+        raise TypeError("ctx_len must be an int32 CUDA tensor")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    g = make_grid(grid, pos_scale, rope_base, split) if grid is not None else None
+    st = _lib.lib().mmdit_joint_attention_qnorm(
+        _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(q_scale_vis), _ptr(q_scale_ctx),
+        ctypes.byref(g) if g is not None else None, eps, B, Nv, Nc, H, D, softmax_scale, dt,
+        _stream(stream))
+    check("mmdit_joint_attention_qnorm", st)
+    return o_vis, o_ctx
+
+
 def joint_attention_fwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
                         softmax_scale: Optional[float] = None, o_vis=None, o_ctx=None, lse=None,
                         stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:

@@ -111,6 +111,26 @@ int mmdit_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_
                        "qk_norm_rope");
 }
 
+int mmdit_k_norm_rope(const void* k_in, void* k_out, const float* k_scale, int B, int N, int H,
+                      int D, const mmdit_grid* grid, float eps, mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || N < 0 || H < 0 || !(eps >= 0.f) || !std::isfinite(eps))
+        return MMDIT_ERR_ARG;
+    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * N * H == 0) return MMDIT_OK;
+    if (!k_in || !k_out || !k_scale) return MMDIT_ERR_ARG;
+    if (!aligned16(k_in) || !aligned16(k_out) || !aligned16(k_scale)) return MMDIT_ERR_ALIGN;
+    if ((long long)B * N * H >= (1LL << 31)) return MMDIT_ERR_UNSUPPORTED;
+    RopeGrid g{};
+    if (grid) {
+        const int r = check_grid(grid, N, D, dt, g);
+        if (r != MMDIT_OK) return r;
+    }
+    return cuda_status(launch_qk_norm_rope(nullptr, k_in, nullptr, k_out, k_scale, k_scale, B, N,
+                                           H, grid ? &g : nullptr, nullptr, nullptr, eps,
+                                           dt == MMDIT_BF16, static_cast<cudaStream_t>(stream)),
+                       "k_norm_rope");
+}
+
 int mmdit_qk_norm_rope_bwd(const void* q_in, const void* k_in, const void* dq_out,
                            const void* dk_out, const float* q_scale, const float* k_scale,
                            void* dq_in, void* dk_in, float* dq_scale, float* dk_scale, int B,
@@ -280,6 +300,49 @@ int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vi
                           int H, int D, float softmax_scale, mmdit_dtype dt, void* stream) {
     return joint_attention_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx,
                                 nullptr, B, Nv, Nc, H, D, softmax_scale, nullptr, dt, stream);
+}
+
+int mmdit_joint_attention_qnorm(const void* q_vis, const void* k_vis, const void* v_vis,
+                                const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                                const float* q_scale_vis, const float* q_scale_ctx,
+                                const mmdit_grid* grid, float eps, int B, int Nv, int Nc, int H,
+                                int D, float softmax_scale, mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || Nv < 0 || Nc < 0 || H < 0) return MMDIT_ERR_ARG;
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return MMDIT_ERR_ARG;
+    if (dt != MMDIT_BF16) return MMDIT_ERR_UNSUPPORTED;
+    if ((Nv > 0 && !q_scale_vis) || (Nc > 0 && !q_scale_ctx)) return MMDIT_ERR_ARG;
+    if ((q_scale_vis && !aligned16(q_scale_vis)) || (q_scale_ctx && !aligned16(q_scale_ctx)))
+        return MMDIT_ERR_ALIGN;
+    RopeGrid g{};
+    if (grid) {
+        const int r = check_grid(grid, Nv, D, dt, g);
+        if (r != MMDIT_OK) return r;
+    }
+    const QNormArgs qn{{q_scale_vis, q_scale_ctx}, grid ? &g : nullptr, eps};
+    // the remaining checks and the launch are those of the joint attention
+    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * H * (Nv + (long long)Nc) == 0) return MMDIT_OK;
+    if (B > 65535 || H > 65535) return MMDIT_ERR_UNSUPPORTED;
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MMDIT_ERR_ARG;
+    if (Nv > 0) {
+        if (!q_vis || !k_vis || !v_vis || !o_vis) return MMDIT_ERR_ARG;
+        if (!aligned16(q_vis) || !aligned16(k_vis) || !aligned16(v_vis) || !aligned16(o_vis))
+            return MMDIT_ERR_ALIGN;
+    }
+    if (Nc > 0) {
+        if (!q_ctx || !k_ctx || !v_ctx || !o_ctx) return MMDIT_ERR_ARG;
+        if (!aligned16(q_ctx) || !aligned16(k_ctx) || !aligned16(v_ctx) || !aligned16(o_ctx))
+            return MMDIT_ERR_ALIGN;
+    }
+    if (ctx_len && (reinterpret_cast<uintptr_t>(ctx_len) & 3u)) return MMDIT_ERR_ALIGN;
+    if ((long long)Nv + Nc > (1LL << 30)) return MMDIT_ERR_UNSUPPORTED;
+    const int r = launch_joint_attention_bf16(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len,
+                                              o_vis, o_ctx, nullptr, B, Nv, Nc, H, softmax_scale,
+                                              nullptr, static_cast<cudaStream_t>(stream), &qn);
+    if (r == 0) return MMDIT_OK;
+    set_last_error("joint_attention_qnorm", r);
+    return MMDIT_ERR_CUDA;
 }
 
 int mmdit_joint_attention_fwd(const void* q_vis, const void* k_vis, const void* v_vis,

@@ -34,11 +34,20 @@
 // conditioning query tiles stream every key.  The grid is one-dimensional with
 // the conditioning tiles first (they run longest), and the epilogue writes
 // each visual row back at its raster position.
+//
+// Q-norm mode (the fusion of the Seaweed-7B report, section 3.4, of the
+// attention preprocessing into the attention): q arrives raw, and the softmax
+// warpgroups, idle until the first S tile, RMS-normalise and rotate (3D RoPE
+// on visual rows) their own query row in the swizzled shared-memory Q tile
+// before the first MMA reads it.  The cos/sin of every (axis position, pair)
+// sit in a shared-memory table built by the same warps while the Q tile is in
+// flight.  This saves the write and the re-read of the normalised q.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 
@@ -83,8 +92,13 @@ struct Smem {
     static constexpr int k_off = q_off + 2 * kTileBytes;          // kStages tiles
     static constexpr int v_off = k_off + kStages * kTileBytes;    // kStages tiles
     static constexpr int bar_off = v_off + kStages * kTileBytes;
-    static constexpr int total = bar_off + 256;
+    static constexpr int tab_off = bar_off + 256;                 // Q-norm mode: RoPE table
+    static constexpr int total = tab_off;                         // + the table's bytes
 };
+// Largest RoPE table (float2 entries) that fits beside the tiles in the
+// 227 KB a CTA may use (alignment slack included); larger grids compute
+// sin / cos per element.
+constexpr int kMaxTabEntries = (232448 - Smem::total - 1024) / 8;
 
 struct Params {
     CUtensorMap tm_q[2];  // [0] visual, [1] conditioning
@@ -106,6 +120,16 @@ struct Params {
     int vis_pairs;      // query-tile pairs of all windows per (b, h)
     int pair_start[kMaxWindows + 1];  // first pair of each window
     WindowTable win;
+    // Q-norm mode only
+    int qnorm;
+    float eps;
+    const float* gq[2];        // RMSNorm scale of q per stream [128]
+    int rope;                  // visual rows get 3D RoPE
+    int gT, gH, gW;            // visual grid
+    int off[3], split[3];      // first head dim and width of each axis chunk
+    int tab_off[3], tab_stride[3], tab_entries;   // table layout; 0 entries: no table
+    double pos_scale[3];
+    double freq[64];           // frequency of pair j of axis a at off[a] / 2 + j
 };
 
 
@@ -127,6 +151,7 @@ struct Bars {
     uint64_t s_full[2], o_done[2];
     uint64_t p_full[4];  // [2 i + h]: half h (keys 64h..64h+63) of P_i is in tensor memory
     uint64_t drain;
+    uint64_t q_ready;   // Q-norm mode: every softmax warp has rewritten its Q rows
     uint64_t wait_ns;   // limit of one pipeline wait (copied from the parameters)
     uint32_t tmem_base;
     uint32_t abort;
@@ -296,6 +321,118 @@ __device__ __forceinline__ float exp_half(const float (&sv)[128], uint32_t (&rh)
     return lo + hi;
 }
 
+// Q-norm mode: RMS-normalise (and, on visual rows, rotate) query row r of
+// tile i in place in shared memory, then release it to the MMA issuer.  Run by
+// all 256 softmax threads (thread = row of its warpgroup's tile).
+__device__ __forceinline__ void q_prologue(const Params& p, uint8_t* smem, Bars* bars,
+                                        const volatile Work* vwk, int i, int r) {
+    float2* tab = reinterpret_cast<float2*>(smem + Smem::tab_off);
+    const bool use_tab = p.rope && p.tab_entries > 0;
+    if (use_tab) {
+        for (int e = threadIdx.x; e < p.tab_entries; e += 256) {
+            const int a = e < p.tab_off[1] ? 0 : (e < p.tab_off[2] ? 1 : 2);
+            const int local = e - p.tab_off[a];
+            const int pos = local / p.tab_stride[a];
+            const int j = local - pos * p.tab_stride[a];
+            float c = 1.f, sn = 0.f;
+            if (j < p.split[a] / 2) {
+                const float ang = (float)((double)pos * p.pos_scale[a] * p.freq[p.off[a] / 2 + j]);
+                sincosf(ang, &sn, &c);
+            }
+            tab[e] = make_float2(c, sn);
+        }
+        named_barrier_sync(1, 256);
+    }
+    const bool has_tile = i == 0 || vwk->has1;
+    if (has_tile && wait(&bars->q_full, 0, bars)) {
+        const int seg = i ? vwk->seg1 : vwk->seg0;
+        const int qrow = (i ? vwk->row1 : vwk->row0) + r;
+        uint8_t* row = smem + Smem::q_off + i * kTileBytes + r * 128;
+        const float* g = p.gq[seg];
+        // mean square: 16 partial sums of 8 dims, then a butterfly over them
+        float part[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(row + (c >> 3) * kHalfBytes +
+                                                            (((c & 7) ^ (r & 7)) << 4));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
+                acc = fmaf(lo, lo, acc);
+                acc = fmaf(hi, hi, acc);
+            }
+            part[c] = acc;
+        }
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1)
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                if (!(c & o)) part[c] += part[c | o];
+        const float inv = rsqrtf(part[0] * (1.0f / kHeadDim) + p.eps);
+        // position of the row (visual rows with RoPE only)
+        bool rot = seg == 0 && p.rope;
+        int pt = 0, ph = 0, pw = 0;   // grid position (t, h, w)
+        if (rot) {
+            int n = qrow;
+            if (vwk->wi >= 0) {
+                const int local = qrow - vwk->vis_start;
+                rot = local < vwk->vis_len;
+                n = rot ? window_to_raster(p.win.w[vwk->wi], local, p.win.Hg, p.win.Wg) : 0;
+            } else {
+                rot = qrow < p.N[0];
+            }
+            const int hw = p.gH * p.gW;
+            pt = n / hw;
+            ph = (n / p.gW) % p.gH;
+            pw = n % p.gW;
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            uint4* addr = reinterpret_cast<uint4*>(row + (c >> 3) * kHalfBytes +
+                                                   (((c & 7) ^ (r & 7)) << 4));
+            const uint4 v = *addr;
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x[2 * e] = __uint_as_float(w[e] << 16);
+                x[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+            }
+            const int d0 = 8 * c;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] *= inv * __ldg(g + d0 + e);
+            if (rot) {
+                const int a = d0 < p.off[1] ? 0 : (d0 < p.off[2] ? 1 : 2);
+                const int pa = a == 0 ? pt : (a == 1 ? ph : pw);
+                const int jb = (d0 - p.off[a]) >> 1;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float cs, sn;
+                    if (use_tab) {
+                        const float2 t = tab[p.tab_off[a] + pa * p.tab_stride[a] + jb + q];
+                        cs = t.x;
+                        sn = t.y;
+                    } else {
+                        const float ang = (float)((double)pa * p.pos_scale[a] *
+                                                  p.freq[p.off[a] / 2 + jb + q]);
+                        sincosf(ang, &sn, &cs);
+                    }
+                    const float x0 = x[2 * q], x1 = x[2 * q + 1];
+                    x[2 * q] = x0 * cs - x1 * sn;
+                    x[2 * q + 1] = x0 * sn + x1 * cs;
+                }
+            }
+            *addr = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                               pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+        }
+        fence_proxy_async_smem();
+    }
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&bars->q_ready);
+}
+
 __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -321,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
             mbar_init(&bars->o_done[i], 1);
         }
         mbar_init(&bars->drain, 1);
+        mbar_init(&bars->q_ready, 8);
         bars->abort = 0;
         bars->wait_ns = p.wait_ns;
         fence_barrier_init();
@@ -416,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
         const int ntile = has1 ? 2 : 1;
-        bool ok = wait(&bars->q_full, 0, bars);
+        bool ok = wait(p.qnorm ? &bars->q_ready : &bars->q_full, 0, bars);
         // Descriptor bases are computed once; a k-step only adds a constant to
         // the start-address field (shared addresses stay below 256 KB, so the
         // 14-bit field never carries).  This keeps the issuing thread, which
@@ -491,6 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         // ------------------------------------------------------------ softmax warpgroups
         const int i = warp >> 2;        // query tile of this warpgroup
         const int quarter = warp & 3;   // TMEM lanes [32 quarter, 32 quarter + 32)
+        if (p.qnorm) q_prologue(p, smem, bars, vwk, i, quarter * 32 + lane);
         if (i == 0 || vwk->has1) {
             const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
             const uint32_t tS = tmem + i * 128 + lane_off;
@@ -626,7 +765,8 @@ uint64_t wait_timeout_ns() {
 int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, const void* qc,
                                 const void* kc, const void* vc, const int32_t* ctx_len, void* ov,
                                 void* oc, float* lse, int B, int Nv, int Nc, int H,
-                                float softmax_scale, const WindowTable* win, cudaStream_t s) {
+                                float softmax_scale, const WindowTable* win, cudaStream_t s,
+                                const QNormArgs* qn) {
     using namespace attn;
     if (!encode_fn()) return -1;
     const int q_tiles = (Nv + kBlockM - 1) / kBlockM + (Nc + kBlockM - 1) / kBlockM;
@@ -673,7 +813,38 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
     p.q_tiles = q_tiles;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.wait_ns = wait_timeout_ns();
-    const int smem = Smem::total + 1024;
+    int tab_bytes = 0;
+    if (qn) {
+        p.qnorm = 1;
+        p.eps = qn->eps;
+        p.gq[0] = qn->gq[0];
+        p.gq[1] = qn->gq[1];
+        if (qn->grid) {
+            const RopeGrid& g = *qn->grid;
+            p.rope = 1;
+            p.gT = g.T;
+            p.gH = g.H;
+            p.gW = g.W;
+            const int extent[3] = {g.T, g.H, g.W};
+            int off = 0, toff = 0;
+            for (int a = 0; a < 3; ++a) {
+                p.off[a] = off;
+                p.split[a] = g.split[a];
+                p.pos_scale[a] = g.pos_scale[a];
+                const int half = g.split[a] / 2;
+                for (int j = 0; j < half; ++j)
+                    p.freq[off / 2 + j] = std::pow(g.base, -2.0 * j / (double)g.split[a]);
+                p.tab_stride[a] = (half + 1) & ~1;
+                p.tab_off[a] = toff;
+                toff += extent[a] * p.tab_stride[a];
+                off += g.split[a];
+            }
+            p.tab_entries = toff <= kMaxTabEntries ? toff : 0;
+            tab_bytes = p.tab_entries * 8;
+        }
+    }
+    const int smem = Smem::total + tab_bytes + 1024;
+    const int smem_max = Smem::total + kMaxTabEntries * 8 + 1024;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return (int)e;
@@ -688,7 +859,7 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
         if (e != cudaSuccess) return (int)e;
         if (fa.numRegs != kRegsLaunch) return (int)cudaErrorInvalidKernelImage;
         e = cudaFuncSetAttribute(joint_attn_bf16_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
         if (e != cudaSuccess) return (int)e;
         attr_set[dev] = true;
     }

@@ -173,8 +173,9 @@ constexpr int kRopeText = 2;   // text tokens, MM-RoPE: one position shared by t
 constexpr int kQkUnroll = 8;
 
 // PERM (grid mode only): rows are stored in window-major order instead of in
-// place of the input rows.
-template <typename T, int ROPE, bool TABLE, bool PERM, int UNR>
+// place of the input rows.  KONLY: k alone (q is normalised inside the
+// attention kernel); q_in / q_out are not touched.
+template <typename T, int ROPE, bool TABLE, bool PERM, int UNR, bool KONLY = false>
 __global__ void __launch_bounds__(256, 2)
 qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
                     const float* __restrict__ gq, const float* __restrict__ gk, uint32_t units,
@@ -225,7 +226,7 @@ qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
             const uint32_t u = uw + r * GPW + grp;
             if (u < units) {
                 const size_t base = (size_t)u * kHeadDim + d0;
-                rq[r] = ld16(q_in + base);
+                rq[r] = KONLY ? make_uint4(0, 0, 0, 0) : ld16(q_in + base);
                 rk[r] = ld16(k_in + base);
             } else {
                 rq[r] = make_uint4(0, 0, 0, 0);
@@ -312,20 +313,20 @@ qk_norm_rope_kernel(const T* q_in, const T* k_in, T* q_out, T* k_out,
             }
             if (u < units) {
                 const size_t base = (size_t)(u + delta) * kHeadDim + d0;
-                st16(q_out + base, pack(xq));
+                if (!KONLY) st16(q_out + base, pack(xq));
                 st16(k_out + base, pack(xk));
             }
         }
     }
 }
 
-template <typename T, int ROPE, bool TABLE, bool PERM = false>
+template <typename T, int ROPE, bool TABLE, bool PERM = false, bool KONLY = false>
 cudaError_t run_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, const float* gq,
                    const float* gk, uint32_t units, float eps, const RopeParams& rp, size_t smem,
                    cudaStream_t s) {
     // the permuted store next to in-register sin/cos needs more registers
     constexpr int UNR = (PERM && !TABLE) ? kQkUnroll / 2 : kQkUnroll;
-    auto kern = qk_norm_rope_kernel<T, ROPE, TABLE, PERM, UNR>;
+    auto kern = qk_norm_rope_kernel<T, ROPE, TABLE, PERM, UNR, KONLY>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -949,6 +950,15 @@ cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out,
         rp.HW = rp.W = make_fastdiv(1);
     }
 #define MMDIT_QK_DISPATCH(T)                                                                   \
+    if (!q_in && !grid)                                                                        \
+        return run_qk<T, kRopeNone, false, false, true>(q_in, k_in, q_out, k_out, gq, gk, units,  \
+                                                       eps, rp, 0, s);                          \
+    if (!q_in && table)                                                                        \
+        return run_qk<T, kRopeGrid, true, false, true>(q_in, k_in, q_out, k_out, gq, gk, units,   \
+                                                      eps, rp, smem, s);                        \
+    if (!q_in)                                                                                 \
+        return run_qk<T, kRopeGrid, false, false, true>(q_in, k_in, q_out, k_out, gq, gk, units,  \
+                                                       eps, rp, 0, s);                          \
     if (text)                                                                                  \
         return run_qk<T, kRopeText, false>(q_in, k_in, q_out, k_out, gq, gk, units, eps, rp, 0, \
                                            s);                                                  \

@@ -23,6 +23,7 @@ struct RopeText {
 };
 
 // 0 or a cudaError_t value.  At most one of grid / text is non-null.
+// q_in == null: k alone (no text positions, no permutation).
 // win_parts (grid mode only, else null): store the rows in the window-major
 // order of that 3D window partition (window.h) instead of in place.
 cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
@@ -60,13 +61,24 @@ cudaError_t launch_gated_residual(const void* x, const void* branch, const float
 // win (null: full joint attention): 3D window attention; the visual inputs
 // are then in the table's window-major order and o_vis is written in raster
 // order.
+// Q-norm mode of the attention kernel: q arrives raw and is RMS-normalised
+// (scale gq[stream]) and, on visual rows when grid is set, rotated in the
+// kernel.
+struct QNormArgs {
+    const float* gq[2];
+    const RopeGrid* grid;
+    float eps;
+};
+
 // lse (null: not written): [B, H, Nv + Nc] natural-log row log-sum-exp of
-// the scaled scores, +infinity for rows without an output.
+// the scaled scores, +infinity for rows without an output.  qn (null: q is
+// already normalised).
 int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv,
                                 const void* qc, const void* kc, const void* vc,
                                 const int32_t* ctx_len, void* ov, void* oc, float* lse, int B,
                                 int Nv, int Nc, int H, float softmax_scale,
-                                const WindowTable* win, cudaStream_t s);
+                                const WindowTable* win, cudaStream_t s,
+                                const QNormArgs* qn = nullptr);
 
 cudaError_t launch_joint_attention_f32(const float* qv, const float* kv, const float* vv,
                                        const float* qc, const float* kc, const float* vc,

@@ -74,6 +74,16 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, ui
         : "memory");
 }
 
+// Makes this thread's generic-proxy shared-memory writes visible to later
+// async-proxy reads (tcgen05.mma operands, TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Named barrier for `count` threads (a multiple of 32), id 1..15.
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ---------------------------------------------------------------- register split
 // Every warp of a warpgroup executes these together.  Increases draw on the
 // registers the block was launched with, released by the decreases.

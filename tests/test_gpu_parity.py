@@ -295,3 +295,67 @@ def test_attention_identical_keys_give_mean_v_and_unit_v_gives_one():
     ov, oc = api.joint_attention(t["q_vis"], t["k_vis"], ones_v, t["q_ctx"], t["k_ctx"], ones_c,
                                  t["ctx_len"])
     parity(from_dev(ov), np.ones(ov.shape), "bf16", "rows sum to one")
+
+
+# ------------------------------------------- q normalised inside the attention kernel
+
+def _qnorm_paths(w: I.Workload, seed=6):
+    inp = I.make_inputs(w, seed=seed, parts=("qkv", "scales"))
+    t = device_inputs(inp)
+    cl = t["ctx_len"] if w.ctx_len is not None else None
+    # unfused: q and k through the prologue kernel, then the attention
+    qv, kv = api.qk_norm_rope(t["q_vis"].clone(), t["k_vis"].clone(), t["gq_vis"], t["gk_vis"],
+                              grid=w.grid, pos_scale=w.pos_scale)
+    qc, kc = api.qk_norm_rope(t["q_ctx"].clone(), t["k_ctx"].clone(), t["gq_ctx"], t["gk_ctx"])
+    a_v, a_c = api.joint_attention(qv, kv, t["v_vis"], qc, kc, t["v_ctx"], cl)
+    # fused: k alone through the prologue, raw q into the attention kernel
+    kv2 = api.k_norm_rope(t["k_vis"].clone(), t["gk_vis"], grid=w.grid, pos_scale=w.pos_scale)
+    kc2 = api.k_norm_rope(t["k_ctx"].clone(), t["gk_ctx"])
+    f_v, f_c = api.joint_attention_qnorm(t["q_vis"], kv2, t["v_vis"], t["q_ctx"], kc2, t["v_ctx"],
+                                         t["gq_vis"], t["gq_ctx"], grid=w.grid,
+                                         pos_scale=w.pos_scale, ctx_len=cl)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    assert torch.equal(kv, kv2) and torch.equal(kc, kc2), "k alone must match the pair kernel"
+    return inp, (a_v, a_c), (f_v, f_c)
+
+
+@pytest.mark.parametrize("case", ["block", "ragged_small", "batch3_mixed", "long_2k"])
+def test_attention_qnorm_full(case):
+    w = SMALL[case]
+    inp, (a_v, a_c), (f_v, f_c) = _qnorm_paths(w)
+    rq, rk = oracle.qk_norm_rope(inp["q_vis"].f64, inp["k_vis"].f64, inp["gq_vis"],
+                                 inp["gk_vis"], grid=w.grid, pos_scale=w.pos_scale)
+    cq, ck = oracle.qk_norm_rope(inp["q_ctx"].f64, inp["k_ctx"].f64, inp["gq_ctx"],
+                                 inp["gk_ctx"], grid=None)
+    rq, rk, cq, ck = (I.round_f64_to_bf16(a) for a in (rq, rk, cq, ck))
+    rv, rc = oracle.joint_attention(rq, rk, inp["v_vis"].f64, cq, ck, inp["v_ctx"].f64,
+                                    inp["ctx_len"])
+    parity(from_dev(f_v), rv, w.dtype, f"{case} fused o_vis")
+    parity(from_dev(f_c), rc, w.dtype, f"{case} fused o_ctx")
+    # the fused and the unfused path agree to within the same bound
+    parity(from_dev(f_v), from_dev(a_v), w.dtype, f"{case} fused vs unfused o_vis")
+    parity(from_dev(f_c), from_dev(a_c), w.dtype, f"{case} fused vs unfused o_ctx")
+
+
+@pytest.mark.parametrize("name", ["480p", "720p"])
+def test_attention_qnorm_sampled_full_size(name):
+    w = W[name]
+    inp, _, (f_v, f_c) = _qnorm_paths(w)
+    full = np.concatenate([from_dev(f_v), from_dev(f_c)], axis=1)
+    rq, rk = oracle.qk_norm_rope(inp["q_vis"].f64, inp["k_vis"].f64, inp["gq_vis"],
+                                 inp["gk_vis"], grid=w.grid, pos_scale=w.pos_scale)
+    cq, ck = oracle.qk_norm_rope(inp["q_ctx"].f64, inp["k_ctx"].f64, inp["gq_ctx"],
+                                 inp["gk_ctx"], grid=None)
+    rq, rk, cq, ck = (I.round_f64_to_bf16(a) for a in (rq, rk, cq, ck))
+    trip = []
+    for h in range(w.H):
+        rows = I.parity_rows(w, 0, h, n_random=128)
+        trip.append(np.stack([np.zeros_like(rows), np.full_like(rows, h), rows], axis=1))
+    trip = np.concatenate(trip)
+    ref = oracle.joint_attention_rows(rq, rk, inp["v_vis"].f64, cq, ck, inp["v_ctx"].f64,
+                                      inp["ctx_len"], trip)
+    got = full[trip[:, 0], trip[:, 2], trip[:, 1]]
+    vis = trip[:, 2] < w.Nv
+    parity(got[vis], ref[vis], w.dtype, f"{name} fused o_vis rows")
+    parity(got[~vis], ref[~vis], w.dtype, f"{name} fused o_ctx rows")
