@@ -65,6 +65,21 @@ def _configure(lib):
     lib.oracle_rmsnorm_rope_bwd.argtypes = [dp, dp, dp, dp, ctypes.c_double,
                                             ctypes.POINTER(ctypes.c_int), ctypes.c_long,
                                             ctypes.c_int, ctypes.c_double, dp, dp]
+    lib.oracle_e4m3_round.argtypes = [ctypes.c_double]
+    lib.oracle_e4m3_round.restype = ctypes.c_double
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+    lib.oracle_e4m3_encode.restype = ctypes.c_ubyte
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_ubyte]
+    lib.oracle_e4m3_decode.restype = ctypes.c_double
+    i8p = ctypes.POINTER(ctypes.c_byte)
+    u8p = ctypes.POINTER(ctypes.c_ubyte)
+    fp = ctypes.POINTER(ctypes.c_float)
+    lib.oracle_quant_int8.argtypes = [dp] + [ctypes.c_int] * 5 + [i8p, fp]
+    lib.oracle_quant_v_e4m3.argtypes = [dp, dp, ctypes.POINTER(ctypes.c_int)] + \
+        [ctypes.c_int] * 5 + [u8p, u8p, fp]
+    lib.oracle_attention_q8_rows.argtypes = [i8p, i8p, fp, fp, i8p, i8p, fp, fp, u8p, u8p, fp,
+                                             ctypes.POINTER(ctypes.c_int)] + [ctypes.c_int] * 5 + \
+        [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp]
     lib.oracle_adaln_modulate.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3 + [ctypes.c_double]
     lib.oracle_gated_residual.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3
     return lib
@@ -269,6 +284,112 @@ def qk_norm_rope_bwd(q, k, gq, gk, dq_out, dk_out, grid=None, pos_scale=(1.0, 1.
     dq, dgq = rmsnorm_rope_bwd(q, gq, dq_out, pos, eps, base, split)
     dk, dgk = rmsnorm_rope_bwd(k, gk, dk_out, pos, eps, base, split)
     return dq, dk, dgq, dgk
+
+
+# ------------------------------------------------------------ 8-bit attention
+
+def e4m3_round(x) -> np.ndarray:
+    """Round to the nearest E4M3 value (half-even, saturating at +-448)."""
+    f = _load().oracle_e4m3_round
+    a = np.asarray(x, dtype=np.float64)
+    return np.array([f(float(v)) for v in a.ravel()]).reshape(a.shape)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    f = _load().oracle_e4m3_encode
+    a = np.asarray(x, dtype=np.float64)
+    return np.array([f(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
+
+
+def e4m3_decode(c) -> np.ndarray:
+    f = _load().oracle_e4m3_decode
+    a = np.asarray(c, dtype=np.uint8)
+    return np.array([f(int(v)) for v in a.ravel()]).reshape(a.shape)
+
+
+def quant_int8(x, block: int):
+    """Symmetric int8 codes of x [B, N, H, D] with one fp32 scale per block of
+    ``block`` consecutive tokens of a (sample, head): (codes, scales [B, H, nblk])."""
+    x = _f64(x)
+    B, N, H, D = x.shape
+    nblk = (N + block - 1) // block
+    codes = np.zeros(x.shape, dtype=np.int8)
+    scales = np.zeros((B, H, max(nblk, 0)), dtype=np.float32)
+    if x.size:
+        _load().oracle_quant_int8(_p(x), B, N, H, D, block,
+                                  codes.ctypes.data_as(ctypes.POINTER(ctypes.c_byte)),
+                                  scales.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    return codes, scales
+
+
+def quant_v_e4m3(vv, vc, ctx_len=None):
+    """E4M3 codes of v (both streams) with one fp32 scale per (sample, head,
+    channel) over the valid tokens: (codes_vis, codes_ctx, scales [B, H, D])."""
+    vv, vc = _f64(vv), _f64(vc)
+    B, Nv, H, D = vv.shape
+    Nc = vc.shape[1]
+    cv = np.zeros(vv.shape, dtype=np.uint8)
+    cc = np.zeros(vc.shape, dtype=np.uint8)
+    sv = np.zeros((B, H, D), dtype=np.float32)
+    cl_p, _keep = _ctx_ptr(ctx_len)
+    u8 = ctypes.POINTER(ctypes.c_ubyte)
+    _load().oracle_quant_v_e4m3(_p(vv), _p(vc), cl_p, B, Nv, Nc, H, D, cv.ctypes.data_as(u8),
+                                cc.ctypes.data_as(u8),
+                                sv.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    return cv, cc, sv
+
+
+def attention_q8_rows(qv8, qc8, sqv, sqc, kv8, kc8, skv, skc, vv8, vc8, sv, ctx_len, rows,
+                      scale: Optional[float] = None):
+    """Output rows (b, h, joint i) of the 8-bit joint attention (Wan 2.1
+    report, section 4.4.3) from quantised operands (see oracle.c)."""
+    arrs = [np.ascontiguousarray(a) for a in (qv8, qc8, kv8, kc8)]
+    qv8, qc8, kv8, kc8 = (a.astype(np.int8, copy=False) for a in arrs)
+    vv8 = np.ascontiguousarray(vv8, dtype=np.uint8)
+    vc8 = np.ascontiguousarray(vc8, dtype=np.uint8)
+    sqv, sqc, skv, skc, sv = (np.ascontiguousarray(a, dtype=np.float32)
+                              for a in (sqv, sqc, skv, skc, sv))
+    B, Nv, H, D = qv8.shape
+    Nc = qc8.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    out = np.zeros((rows.shape[0], D), dtype=np.float64)
+    cl_p, _keep = _ctx_ptr(ctx_len)
+    i8 = ctypes.POINTER(ctypes.c_byte)
+    u8 = ctypes.POINTER(ctypes.c_ubyte)
+    f = ctypes.POINTER(ctypes.c_float)
+    if rows.shape[0]:
+        _load().oracle_attention_q8_rows(
+            qv8.ctypes.data_as(i8), qc8.ctypes.data_as(i8), sqv.ctypes.data_as(f),
+            sqc.ctypes.data_as(f), kv8.ctypes.data_as(i8), kc8.ctypes.data_as(i8),
+            skv.ctypes.data_as(f), skc.ctypes.data_as(f), vv8.ctypes.data_as(u8),
+            vc8.ctypes.data_as(u8), sv.ctypes.data_as(f), cl_p, B, Nv, Nc, H, D, scale,
+            rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), rows.shape[0], _p(out))
+    return out
+
+
+def attention_q8(qv, kv, vv, qc, kc, vc, ctx_len=None, rows=None, scale=None):
+    """The whole 8-bit method from unquantised q, k, v: quantise (q per token,
+    k per 128-token block, v per channel), then attend.  Returns (o_vis, o_ctx)
+    when ``rows`` is None, else the requested rows."""
+    qv8, sqv = quant_int8(qv, 1)
+    qc8, sqc = quant_int8(qc, 1)
+    kv8, skv = quant_int8(kv, 128)
+    kc8, skc = quant_int8(kc, 128)
+    vv8, vc8, sv = quant_v_e4m3(vv, vc, ctx_len)
+    B, Nv, H, D = np.shape(qv)
+    Nc = np.shape(qc)[1]
+    full = rows is None
+    if full:
+        bb, hh, ii = np.meshgrid(np.arange(B), np.arange(H), np.arange(Nv + Nc), indexing="ij")
+        rows = np.stack([bb.ravel(), hh.ravel(), ii.ravel()], axis=1)
+    out = attention_q8_rows(qv8, qc8, sqv.reshape(B, H, -1), sqc.reshape(B, H, -1), kv8, kc8,
+                            skv, skc, vv8, vc8, sv, ctx_len, rows, scale)
+    if not full:
+        return out
+    out = out.reshape(B, H, Nv + Nc, D).transpose(0, 2, 1, 3)
+    return np.ascontiguousarray(out[:, :Nv]), np.ascontiguousarray(out[:, Nv:])
 
 
 def _grid_struct(grid) -> _Grid:

@@ -11,7 +11,9 @@ to pin the C oracle (``oracle.c``).  It shares no code with it:
   * LayerNorm uses numpy's mean / var;
   * window attention physically gathers each window's tokens (numpy's
     array_split of the (T, H, W) grid along each axis) and runs the
-    concatenated-sequence attention above on every window separately.
+    concatenated-sequence attention above on every window separately;
+  * the 8-bit attention quantises with numpy float32 arithmetic and torch's
+    float8_e4m3fn conversion, and runs its tiled softmax with numpy arrays.
 
 Sources: Vimoo 1.0 research page, section 2.2 (dual-stream joint attention,
 QK-RMSNorm, 3D RoPE 16/56/56, adaLN, gated residual); Wan 2.1 report section
@@ -120,3 +122,79 @@ def adaln_modulate(x, shift, scale, eps=1e-6):
 
 def gated_residual(x, branch, gate):
     return np.asarray(x, np.float64) + np.asarray(gate, np.float64)[:, None, :] * np.asarray(branch, np.float64)
+
+
+# ------------------------------------------------------------ 8-bit attention
+
+def e4m3(x):
+    """Nearest E4M3 value through torch's float8_e4m3fn (half-even), after
+    saturating to +-448."""
+    import torch
+    a = np.clip(np.asarray(x, dtype=np.float64), -448.0, 448.0)
+    return torch.from_numpy(a).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def quant_int8(x, block):
+    x32 = np.asarray(x, dtype=np.float64).astype(np.float32)
+    B, N, H, D = x32.shape
+    codes = np.zeros(x32.shape, dtype=np.float64)
+    nblk = -(-N // block)
+    scales = np.zeros((B, H, nblk), dtype=np.float32)
+    for b in range(B):
+        for h in range(H):
+            for k in range(nblk):
+                blk = x32[b, k * block:(k + 1) * block, h]
+                s = np.float32(np.abs(blk).max()) / np.float32(127.0)
+                scales[b, h, k] = s
+                if s > 0:
+                    codes[b, k * block:(k + 1) * block, h] = np.clip(np.rint(blk / s), -127, 127)
+    return codes, scales
+
+
+def attention_q8(qv, kv, vv, qc, kc, vc, ctx_len=None, scale=None):
+    qv, kv, vv, qc, kc, vc = (np.asarray(a, dtype=np.float64) for a in (qv, kv, vv, qc, kc, vc))
+    B, Nv, H, D = qv.shape
+    Nc = qc.shape[1]
+    if scale is None:
+        scale = D ** -0.5
+    if ctx_len is None:
+        ctx_len = [Nc] * B
+    q8v, sqv = quant_int8(qv, 1)
+    q8c, sqc = quant_int8(qc, 1)
+    k8v, skv = quant_int8(kv, 128)
+    k8c, skc = quant_int8(kc, 128)
+    out_v = np.zeros_like(qv)
+    out_c = np.zeros_like(qc)
+    for b in range(B):
+        L = ctx_len[b]
+        vals = np.concatenate([vv[b], vc[b, :L]], axis=0).astype(np.float32)     # [Nk, H, D]
+        sv = np.abs(vals).max(axis=0) / np.float32(448.0)                          # [H, D]
+        v8 = np.where(sv > 0, e4m3(np.where(sv > 0, vals / np.where(sv > 0, sv, 1), 0)), 0)
+        # key tiles: visual blocks of 128, then conditioning blocks of 128
+        tiles = [(j, min(j + 128, Nv), skv[b, :, j // 128], 0) for j in range(0, Nv, 128)]
+        tiles += [(Nv + j, Nv + min(j + 128, L), skc[b, :, j // 128], 1) for j in range(0, L, 128)]
+        K8 = np.concatenate([k8v[b], k8c[b, :L]], axis=0)
+        for i in range(Nv + L):
+            q8 = q8v[b, i] if i < Nv else q8c[b, i - Nv]
+            sq = sqv[b, :, i] if i < Nv else sqc[b, :, i - Nv]
+            for h in range(H):
+                m, acc, l = None, np.zeros(D), 0.0
+                for j0, j1, sk, _ in tiles:
+                    x = (K8[j0:j1, h] @ q8[h]) * float(sq[h]) * float(sk[h]) * scale * np.log2(np.e)
+                    mt = x.max()
+                    if m is None:
+                        m = np.ceil(mt)
+                    elif mt > m + 2:
+                        mn = np.ceil(mt)
+                        acc *= 2.0 ** (m - mn)
+                        l *= 2.0 ** (m - mn)
+                        m = mn
+                    p = 2.0 ** (x - m + 6)
+                    l += p.sum()
+                    acc += e4m3(p) @ v8[j0:j1, h]
+                o = acc * sv[h] / l
+                if i < Nv:
+                    out_v[b, i, h] = o
+                else:
+                    out_c[b, i - Nv, h] = o
+    return out_v, out_c

@@ -513,3 +513,198 @@ void oracle_rmsnorm_rope_bwd(const double* x, const double* g, const double* dy,
     for (int d = 0; d < D; ++d) dg[d] += part[d];
     free(part);
 }
+
+/* ---- 8-bit joint attention [W4] ---------------------------------------------
+ * Wan 2.1 report, section 4.4.3: Int8 for S = Q K^T, FP8 (E4M3) for O = P V,
+ * accumulation across key blocks in fp32.  Readings where the report is
+ * silent (each also listed in the design notes):
+ *   - q is quantised per (sample, token, head) row, k per block of 128
+ *     consecutive tokens of one (sample, head, stream), symmetric:
+ *     scale = max|x| / 127 (fp32), code = round-half-even(x / scale) (fp32),
+ *     clamped to [-127, 127]; scale 0 gives codes 0;
+ *   - v is quantised to E4M3 per (sample, head, channel) over the valid
+ *     tokens of both streams: scale = max|v| / 448 (fp32), code = E4M3
+ *     rounding (half-even, saturating at 448) of v / scale (fp32);
+ *   - the softmax runs over key tiles of 128 (visual tiles, then the valid
+ *     conditioning tiles) with a running maximum m in log2 units that is an
+ *     integer (the ceiling of a tile maximum) and is raised only when a
+ *     tile's maximum exceeds it by more than 2; P' = 2^(x - m + 6), with x the
+ *     score in log2 units, is rounded to E4M3 for the P V product, while the
+ *     row sum takes P' unrounded; o = scale_v * sum(E4M3(P') v8) / sum(P').
+ * Because m is an integer, two schedules of raising it give P' that differ by
+ * exact powers of two, which E4M3 rounding commutes with (up to subnormals). */
+
+/* E4M3: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits; no infinity; the
+ * largest finite magnitude is 1.75 * 2^8 = 448; subnormals step 2^-9.       */
+double oracle_e4m3_round(double x)
+{
+    const double a = fabs(x);
+    if (!(a == a)) return x;
+    if (a >= 448.0) return copysign(448.0, x);                  /* saturate */
+    double quantum;
+    if (a < ldexp(1.0, -6)) {
+        quantum = ldexp(1.0, -9);                               /* subnormal range */
+    } else {
+        int e;
+        frexp(a, &e);                                           /* a = f 2^e, f in [0.5, 1) */
+        quantum = ldexp(1.0, e - 1 - 3);                        /* 3 mantissa bits */
+    }
+    double r = nearbyint(a / quantum) * quantum;                /* half-even */
+    if (r > 448.0) r = 448.0;
+    return copysign(r, x);                                      /* keeps the sign of zero */
+}
+
+unsigned char oracle_e4m3_encode(double x)
+{
+    const double r = oracle_e4m3_round(x);
+    const unsigned char sign = signbit(r) ? 0x80 : 0;
+    const double a = fabs(r);
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -6)) return sign | (unsigned char)nearbyint(a / ldexp(1.0, -9));
+    int e;
+    const double f = frexp(a, &e);                              /* a = (2f) 2^(e-1) */
+    const int exp_field = e - 1 + 7;
+    const int mant = (int)nearbyint((2.0 * f - 1.0) * 8.0);
+    return sign | (unsigned char)(exp_field << 3) | (unsigned char)mant;
+}
+
+double oracle_e4m3_decode(unsigned char c)
+{
+    const int exp_field = (c >> 3) & 15, mant = c & 7;
+    const double a = exp_field == 0 ? ldexp((double)mant, -9)
+                                    : ldexp(1.0 + mant / 8.0, exp_field - 7);
+    return (c & 0x80) ? -a : a;
+}
+
+/* x [B, N, H, D] -> codes [B, N, H, D], scales [B, H, ceil(N / block)]       */
+void oracle_quant_int8(const double* x, int B, int N, int H, int D, int block,
+                       signed char* codes, float* scales)
+{
+    const int nblk = (N + block - 1) / block;
+    #pragma omp parallel for schedule(static)
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const long b = bh / H, h = bh % H;
+        for (int k = 0; k < nblk; ++k) {
+            const int n0 = k * block, n1 = (n0 + block < N) ? n0 + block : N;
+            float amax = 0.0f;
+            for (int n = n0; n < n1; ++n)
+                for (int d = 0; d < D; ++d) {
+                    const float v = fabsf((float)x[((b * N + n) * H + h) * (long)D + d]);
+                    if (v > amax) amax = v;
+                }
+            const float s = amax / 127.0f;
+            scales[bh * nblk + k] = s;
+            for (int n = n0; n < n1; ++n)
+                for (int d = 0; d < D; ++d) {
+                    const long idx = ((b * N + n) * H + h) * (long)D + d;
+                    float q = s > 0.0f ? rintf((float)x[idx] / s) : 0.0f;
+                    q = q > 127.0f ? 127.0f : (q < -127.0f ? -127.0f : q);
+                    codes[idx] = (signed char)q;
+                }
+        }
+    }
+}
+
+/* v [B, N_s, H, D] of both streams -> E4M3 codes, scales [B, H, D]           */
+void oracle_quant_v_e4m3(const double* vv, const double* vc, const int* ctx_len, int B, int Nv,
+                         int Nc, int H, int D, unsigned char* cv, unsigned char* cc,
+                         float* scales)
+{
+    #pragma omp parallel for schedule(static)
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const long b = bh / H, h = bh % H;
+        const int L = ctx_len ? ctx_len[b] : Nc;
+        for (int d = 0; d < D; ++d) {
+            float amax = 0.0f;
+            for (int n = 0; n < Nv; ++n) {
+                const float v = fabsf((float)vv[((b * Nv + n) * H + h) * (long)D + d]);
+                if (v > amax) amax = v;
+            }
+            for (int n = 0; n < L; ++n) {
+                const float v = fabsf((float)vc[((b * Nc + n) * H + h) * (long)D + d]);
+                if (v > amax) amax = v;
+            }
+            const float s = amax / 448.0f;
+            scales[bh * D + d] = s;
+            for (int n = 0; n < Nv; ++n) {
+                const long idx = ((b * Nv + n) * H + h) * (long)D + d;
+                cv[idx] = s > 0.0f ? oracle_e4m3_encode((double)((float)vv[idx] / s)) : 0;
+            }
+            for (int n = 0; n < Nc; ++n) {
+                const long idx = ((b * Nc + n) * H + h) * (long)D + d;
+                cc[idx] = s > 0.0f ? oracle_e4m3_encode((double)((float)vc[idx] / s)) : 0;
+            }
+        }
+    }
+}
+
+/* Attention output rows (b, h, i) of the 8-bit method from the quantised
+ * operands: q codes / scales [B, H, N_s] per stream, k codes / block scales
+ * [B, H, ceil(N_s / 128)] per stream, v codes and channel scales [B, H, D]. */
+void oracle_attention_q8_rows(const signed char* qv, const signed char* qc, const float* sqv,
+                              const float* sqc, const signed char* kv, const signed char* kc,
+                              const float* skv, const float* skc, const unsigned char* vv,
+                              const unsigned char* vc, const float* sv, const int* ctx_len,
+                              int B, int Nv, int Nc, int H, int D, double scale,
+                              const long* rows, long nrows, double* out)
+{
+    (void)B;
+    const double log2e = 1.4426950408889634;
+    const int tv = (Nv + 127) / 128, tc = (Nc + 127) / 128;
+    #pragma omp parallel
+    {
+        double* x = (double*)malloc(sizeof(double) * 128);
+        double* acc = (double*)malloc(sizeof(double) * (size_t)D);
+        #pragma omp for schedule(dynamic, 4)
+        for (long r = 0; r < nrows; ++r) {
+            const long b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+            const int L = ctx_len ? ctx_len[b] : Nc;
+            double* o = out + r * (long)D;
+            for (int d = 0; d < D; ++d) { o[d] = 0.0; acc[d] = 0.0; }
+            if (i >= Nv + L || Nv + L == 0) continue;     /* no output */
+            const signed char* q = (i < Nv) ? qv + ((b * Nv + i) * H + h) * (long)D
+                                            : qc + ((b * Nc + (i - Nv)) * H + h) * (long)D;
+            const double sq = (i < Nv) ? sqv[(b * H + h) * (long)Nv + i]
+                                       : sqc[(b * H + h) * (long)Nc + (i - Nv)];
+            double m = 0.0, l = 0.0;
+            int first = 1;
+            for (int seg = 0; seg < 2; ++seg) {
+                const int nk = seg ? L : Nv, Ns = seg ? Nc : Nv, nt = seg ? tc : tv;
+                const signed char* K = seg ? kc : kv;
+                const unsigned char* V = seg ? vc : vv;
+                const float* sk = seg ? skc : skv;
+                for (int t = 0; t * 128 < nk; ++t) {
+                    const int j0 = t * 128, j1 = (j0 + 128 < nk) ? j0 + 128 : nk;
+                    const double skb = sk[(b * H + h) * (long)nt + t];
+                    double mt = -INFINITY;
+                    for (int j = j0; j < j1; ++j) {
+                        const signed char* k = K + ((b * Ns + j) * H + h) * (long)D;
+                        long dot = 0;
+                        for (int d = 0; d < D; ++d) dot += (long)q[d] * (long)k[d];
+                        x[j - j0] = (double)dot * sq * skb * scale * log2e;
+                        if (x[j - j0] > mt) mt = x[j - j0];
+                    }
+                    if (first) {
+                        m = ceil(mt);
+                        first = 0;
+                    } else if (mt > m + 2.0) {
+                        const double mn = ceil(mt), f = exp2(m - mn);
+                        for (int d = 0; d < D; ++d) acc[d] *= f;
+                        l *= f;
+                        m = mn;
+                    }
+                    for (int j = j0; j < j1; ++j) {
+                        const double p = exp2(x[j - j0] - m + 6.0);
+                        l += p;
+                        const double pq = oracle_e4m3_round(p);
+                        const unsigned char* v = V + ((b * Ns + j) * H + h) * (long)D;
+                        for (int d = 0; d < D; ++d) acc[d] += pq * oracle_e4m3_decode(v[d]);
+                    }
+                }
+            }
+            for (int d = 0; d < D; ++d) o[d] = acc[d] * sv[(b * H + h) * (long)D + d] / l;
+        }
+        free(acc);
+        free(x);
+    }
+}

@@ -41,6 +41,20 @@ void oracle_joint_attention_dq_rows(const double* qv, const double* kv, const do
 void oracle_rmsnorm_rope_bwd(const double* x, const double* g, const double* dy,
                              const double* pos, double rope_base, const int* split,
                              long rows, int D, double eps, double* dx, double* dg);
+double oracle_e4m3_round(double x);
+unsigned char oracle_e4m3_encode(double x);
+double oracle_e4m3_decode(unsigned char c);
+void oracle_quant_int8(const double* x, int B, int N, int H, int D, int block,
+                       signed char* codes, float* scales);
+void oracle_quant_v_e4m3(const double* vv, const double* vc, const int* ctx_len, int B, int Nv,
+                         int Nc, int H, int D, unsigned char* cv, unsigned char* cc,
+                         float* scales);
+void oracle_attention_q8_rows(const signed char* qv, const signed char* qc, const float* sqv,
+                              const float* sqc, const signed char* kv, const signed char* kc,
+                              const float* skv, const float* skc, const unsigned char* vv,
+                              const unsigned char* vc, const float* sv, const int* ctx_len,
+                              int B, int Nv, int Nc, int H, int D, double scale,
+                              const long* rows, long nrows, double* out);
 void oracle_adaln_modulate(const double* x, const double* shift, const double* scale,
                            double* y, int B, int N, int C, double eps);
 void oracle_gated_residual(const double* x, const double* branch, const double* gate,

@@ -686,6 +686,108 @@ def pin_norm_rope_bwd_torch_autograd():
     _close(dg, gt.grad.numpy(), 1e-11)
 
 
+# ---------------------------------------------------------------- 8-bit attention
+
+@pin
+def pin_e4m3_against_torch():
+    """E4M3 rounding equals torch's float8_e4m3fn conversion below the
+    saturation point (including the subnormal range and halfway cases); every
+    finite code decodes to torch's value and encodes back to itself; larger
+    magnitudes saturate to 448."""
+    r = RNG(70)
+    x = np.concatenate([r.standard_normal(3000) * 60, r.standard_normal(1000) * 0.01,
+                        (np.arange(-64, 64) + 0.5) * 2.0 ** -9,          # subnormal halfway
+                        (8 + np.arange(8) + 0.5) * 2.0 ** -3])            # halfway at 1..2
+    x = x[np.abs(x) < 448]
+    want = torch.tensor(x, dtype=torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    _close(oracle.e4m3_round(x), want, 0.0)
+    codes = np.arange(256, dtype=np.uint8)
+    tv = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    fin = ~np.isnan(tv)
+    _close(oracle.e4m3_decode(codes)[fin], tv[fin], 0.0)
+    assert np.array_equal(oracle.e4m3_encode(tv[fin]), codes[fin])
+    _close(oracle.e4m3_round([448.0, 460.0, 1e6, -500.0]), [448.0, 448.0, 448.0, -448.0], 0.0)
+
+
+@pin
+def pin_int8_quantisation():
+    """Codes equal torch's half-even rounding of x / scale in float32 with
+    scale = max|x| / 127; the largest entry of a block maps to +-127; the
+    reconstruction error is at most half a step (plus the rounding of the
+    float32 quotient)."""
+    r = RNG(71)
+    x = I.round_f64_to_bf16(r.standard_normal((2, 300, 3, 128)) * 2.0)
+    for block in (1, 128):
+        codes, scales = oracle.quant_int8(x, block)
+        x32 = torch.from_numpy(x).float()
+        for b in range(2):
+            for h in range(3):
+                for k in range(scales.shape[2]):
+                    blk = x32[b, k * block:(k + 1) * block, h]
+                    s = torch.tensor(blk.abs().max().item(), dtype=torch.float32) / 127.0
+                    assert np.float32(scales[b, h, k]) == np.float32(s.item())
+                    want = torch.clamp(torch.round(blk / s), -127, 127).numpy()
+                    got = codes[b, k * block:(k + 1) * block, h]
+                    assert np.array_equal(got, want)
+                    assert np.abs(got).max() == 127
+                    # half a step, plus the float32 rounding of x / scale
+                    # (at most 127 * 2^-24 of a step)
+                    err = np.abs(got * float(s) - blk.double().numpy()).max()
+                    assert err <= float(s) * (0.5 + 127 * 2.0 ** -24)
+
+
+@pin
+def pin_q8_uniform_scores():
+    """q = 0 makes every score 0, so every P' is exactly 2^6 and the output is
+    the mean of the dequantised v over the valid keys; v built from E4M3 values
+    with a channel maximum of 448 dequantises exactly, so that mean is the mean
+    of v itself."""
+    r = RNG(72)
+    B, Nv, Nc, H, D = 2, 200, 40, 2, 128
+    vals = oracle.e4m3_round(r.standard_normal((B, Nv + Nc, H, D)) * 40)
+    vals[:, 0] = 448.0                        # channel maximum 448 -> scale 1
+    vv, vc = vals[:, :Nv], vals[:, Nv:]
+    z = np.zeros((B, Nv, H, D)), np.zeros((B, Nc, H, D))
+    k = r.standard_normal((B, Nv, H, D)), r.standard_normal((B, Nc, H, D))
+    cl = np.array([40, 7], np.int32)
+    ov, oc = oracle.attention_q8(z[0], k[0], vv, z[1], k[1], vc, cl)
+    for b in range(B):
+        mean = np.concatenate([vv[b], vc[b, :cl[b]]], 0).mean(0)
+        _close(ov[b], np.broadcast_to(mean, ov[b].shape), 1e-12)
+        _close(oc[b, :cl[b]], np.broadcast_to(mean, oc[b, :cl[b]].shape), 1e-12)
+        assert np.all(oc[b, cl[b]:] == 0)
+
+
+@pin
+def pin_q8_brute():
+    """The 8-bit method equals a numpy restatement (float32 quantisation,
+    torch E4M3 conversion, array softmax tiles) on ragged small inputs."""
+    r = RNG(73)
+    B, Nv, Nc, H, D = 2, 300, 140, 2, 128
+    t = [I.round_f64_to_bf16(r.standard_normal((B, n, H, D)) * sd)
+         for n, sd in ((Nv, 1.5), (Nv, 1.5), (Nv, 1.0), (Nc, 1.5), (Nc, 1.5), (Nc, 1.0))]
+    cl = np.array([140, 70], np.int32)
+    ov, oc = oracle.attention_q8(t[0], t[1], t[2], t[3], t[4], t[5], cl)
+    bv, bc = brute.attention_q8(t[0], t[1], t[2], t[3], t[4], t[5], cl)
+    _close(ov, bv, 1e-12)
+    _close(oc, bc, 1e-12)
+
+
+@pin
+def pin_q8_close_to_exact():
+    """The 8-bit method stays close to the exact attention: max error under 8 %
+    of the largest output and mean error under 1 % of it on N(0,1) inputs."""
+    r = RNG(74)
+    B, Nv, Nc, H, D = 1, 400, 100, 2, 128
+    t = [I.round_f64_to_bf16(r.standard_normal((B, n, H, D))) for n in (Nv, Nv, Nv, Nc, Nc, Nc)]
+    ov, oc = oracle.attention_q8(t[0], t[1], t[2], t[3], t[4], t[5])
+    rv, rc = oracle.joint_attention(t[0], t[1], t[2], t[3], t[4], t[5])
+    got, ref = np.concatenate([ov, oc], 1), np.concatenate([rv, rc], 1)
+    mx = np.abs(ref).max()
+    assert np.abs(got - ref).max() <= 0.08 * mx
+    assert np.abs(got - ref).mean() <= 0.01 * mx
+
+
 @pytest.mark.parametrize("name", sorted(PINS))
 def test_pin(name):
     PINS[name]()
@@ -738,6 +840,14 @@ MUTANTS = {
     "nrbwd_r_squared": ("dxr[d] = g[d] * u[d] / rr - xr[d] * dot / ((double)D * rr * rr * rr);",
                         "dxr[d] = g[d] * u[d] / rr - xr[d] * dot / ((double)D * rr * rr);"),
     "nrbwd_dg_no_norm": ("acc[d] += u[d] * xr[d] / rr;", "acc[d] += u[d] * xr[d];"),
+    "q8_no_offset": ("const double p = exp2(x[j - j0] - m + 6.0);",
+                     "const double p = exp2(x[j - j0] - m);"),
+    "q8_no_rescale": ("for (int d = 0; d < D; ++d) acc[d] *= f;", "(void)f;"),
+    "q8_int8_step": ("const float s = amax / 127.0f;", "const float s = amax / 128.0f;"),
+    "q8_v_scale": ("const float s = amax / 448.0f;", "const float s = amax / 256.0f;"),
+    "q8_sum_rounded": ("        l += p;\n", "        l += oracle_e4m3_round(p);\n"),
+    "q8_subnormal_step": ("        quantum = ldexp(1.0, -9);                               /* subnormal range */",
+                          "        quantum = ldexp(1.0, -10);"),
     "window_no_cond_keys": ("for (int j = 0; j < L; ++j) key[nk++] = Nv + j;",
                             "for (int j = 0; j < L && i >= Nv; ++j) key[nk++] = Nv + j;"),
 }
