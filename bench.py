@@ -444,6 +444,23 @@ def run_ours(args):
         "fused_ms": kq_ms + qn_ms,
         "unfused_ms": kern_ms["qk_norm_rope"] + kern_ms["joint_attention"]}}
 
+    # 8-bit attention: quantisers, then Int8 QK^T / E4M3 PV
+    qkv8 = (t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"], t["v_ctx"])
+    _, _, parts8 = api.joint_attention_8bit(*qkv8, t["ctx_len"])
+    quant_ms = time_ms(lambda: api.joint_attention_8bit(*qkv8, t["ctx_len"]), reps=5)
+    q8_ms = time_ms(lambda: api.joint_attention_q8(
+        (parts8["q_vis"], parts8["q_ctx"]), (parts8["k_vis"], parts8["k_ctx"]),
+        (parts8["v_vis"], parts8["v_ctx"]), parts8, t["ctx_len"], o_vis=t["o_vis"],
+        o_ctx=t["o_ctx"]), reps=10)
+    fp8_peak = 2.0 * float(peaks()[0]["bf16_tflops_sustained"])
+    q8_rows = {"attention_8bit": {
+        "attention_ms": q8_ms, "TFLOP/s": w.attention_flops() / (q8_ms * 1e-3) / 1e12,
+        "frac_8bit_sustained": w.attention_flops() / (q8_ms * 1e-3) / 1e12 / fp8_peak,
+        "peak_note": "8-bit peak = 2 x measured bf16 sustained (nominal dense ratio)",
+        "quantise_and_attend_ms": quant_ms,
+        "speedup_vs_bf16_attention": kern_ms["joint_attention"] / q8_ms}}
+    del parts8
+
     # backward: forward with the row log-sum-exp, then D, dQ and dK/dV
     gen = torch.Generator(device=dev).manual_seed(1000 + rank)
     do_vis = torch.randn(t["q_vis"].shape, generator=gen, device=dev).to(torch.bfloat16)
@@ -560,7 +577,7 @@ def run_ours(args):
                               Nv / (Nv + Nc)},
             "qk_norm_rope_text_ctx": {
                 "ms": txt_ms, "GB/s": 4 * B * Nc * C * 2 / (txt_ms * 1e-3) / 1e9},
-            **win_rows, **bwd_rows, **qn_rows},
+            **win_rows, **bwd_rows, **qn_rows, **q8_rows},
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,

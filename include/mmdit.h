@@ -183,6 +183,49 @@ MMDIT_API int mmdit_joint_attention_qnorm(const void* q_vis, const void* k_vis,
                                           int Nc, int H, int D, float softmax_scale,
                                           mmdit_dtype dt, void* stream);
 
+/* Symmetric int8 quantisation for the 8-bit attention ["Wan 2.1" report,
+ * section 4.4.3: Int8 for S = Q K^T]: x [B, N, H, D] bf16 -> codes [B, N, H, D]
+ * int8 and one fp32 scale per `block` consecutive tokens of a (sample, head):
+ * block = 1 (q: per token) or 128 (k: the attention's key tile).
+ *   scale = max|x| / 127, code = round-half-even(x / scale) clamped to
+ *   [-127, 127], both in fp32 (scale 0: codes 0); scales [B, H, ceil(N / block)].
+ * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_quantize_int8(const void* x, void* codes, float* scales, int B, int N, int H,
+                                  int D, int block, void* stream);
+
+/* FP8 E4M3 quantisation of v for the 8-bit attention [Wan 2.1, section 4.4.3:
+ * FP8 for O = P V]: one fp32 scale per (sample, head, channel) over the valid
+ * tokens of both streams (visual, and conditioning below ctx_len[b]):
+ *   scale = max|v| / 448, code = E4M3(v / scale), half-even with saturation.
+ *   v_vis [B, Nv, H, D], v_ctx [B, Nc, H, D] bf16 -> c_vis, c_ctx one byte per
+ *   element (padded conditioning rows are encoded too); scales [B, H, D]
+ *   (16-byte aligned; used as scratch during the call).
+ * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_quantize_v_e4m3(const void* v_vis, const void* v_ctx, const int32_t* ctx_len,
+                                    void* c_vis, void* c_ctx, float* scales, int B, int Nv,
+                                    int Nc, int H, int D, void* stream);
+
+/* 8-bit joint attention [Wan 2.1, section 4.4.3: Int8 S = Q K^T, FP8 O = P V,
+ * fp32 accumulation across key blocks; the joint streams of Vimoo §2.2]:
+ *   S_ij = s_q[i] s_k[block(j)] (q8_i . k8_j), exactly in integers;
+ *   online softmax over 128-key tiles with an integer running maximum m (log2
+ *   units, raised to the ceiling of a tile maximum once that exceeds it by more
+ *   than 2); P' = 2^(S_ij softmax_scale log2(e) - m + 6) rounded to E4M3 for
+ *   the P V product, unrounded in the row sum;
+ *   O_i = s_v * sum_j E4M3(P'_ij) v8_j / sum_j P'_ij over valid keys.
+ *   q/k/v_vis [B, Nv, H, D], q/k/v_ctx [B, Nc, H, D]: codes from
+ *   mmdit_quantize_int8 (q block 1, k block 128) and mmdit_quantize_v_e4m3;
+ *   sq_vis / sq_ctx, sk_vis / sk_ctx, sv: their scales.
+ *   o_vis, o_ctx: bf16 outputs as mmdit_joint_attention (padded rows zero).
+ * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_joint_attention_q8(const void* q_vis, const void* k_vis, const void* v_vis,
+                                       const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                       const float* sq_vis, const float* sq_ctx,
+                                       const float* sk_vis, const float* sk_ctx, const float* sv,
+                                       const int32_t* ctx_len, void* o_vis, void* o_ctx, int B,
+                                       int Nv, int Nc, int H, int D, float softmax_scale,
+                                       void* stream);
+
 /* mmdit_joint_attention that also writes, for training, the row log-sum-exp
  * the backward pass needs [Vimoo §2.2 joint attention; the Seaweed-7B report,
  * section 3.4, trains its forward and backward]:

@@ -259,6 +259,77 @@ def joint_attention_bwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, o_ctx, 
     return g
 
 
+def quantize_int8(x: torch.Tensor, block: int, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Symmetric int8 codes of bf16 x [B, N, H, 128] with one scale per ``block``
+    (1 or 128) tokens of a (sample, head): (codes int8, scales [B, H, blocks])."""
+    if x.dtype != torch.bfloat16:
+        raise TypeError("quantize_int8 takes bf16")
+    _dtype(x)
+    B, N, H, D = x.shape
+    codes = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    scales = torch.empty((B, H, (N + block - 1) // block), dtype=torch.float32, device=x.device)
+    st = _lib.lib().mmdit_quantize_int8(_ptr(x), _ptr(codes), _ptr(scales), B, N, H, D, block,
+                                        _stream(stream))
+    check("mmdit_quantize_int8", st)
+    return codes, scales
+
+
+def quantize_v_e4m3(v_vis: torch.Tensor, v_ctx: torch.Tensor, ctx_len=None, stream=None):
+    """E4M3 codes (uint8) of v for both streams and the per-(sample, head,
+    channel) scales [B, H, 128]."""
+    _dtype(v_vis, v_ctx)
+    B, Nv, H, D = v_vis.shape
+    Nc = v_ctx.shape[1]
+    cv = torch.empty(v_vis.shape, dtype=torch.uint8, device=v_vis.device)
+    cc = torch.empty(v_ctx.shape, dtype=torch.uint8, device=v_vis.device)
+    sv = torch.empty((B, H, D), dtype=torch.float32, device=v_vis.device)
+    st = _lib.lib().mmdit_quantize_v_e4m3(_ptr(v_vis), _ptr(v_ctx), _ptr(ctx_len), _ptr(cv),
+                                          _ptr(cc), _ptr(sv), B, Nv, Nc, H, D, _stream(stream))
+    check("mmdit_quantize_v_e4m3", st)
+    return cv, cc, sv
+
+
+def joint_attention_q8(q8, k8, v8, scales: dict, ctx_len=None,
+                       softmax_scale: Optional[float] = None, o_vis=None, o_ctx=None,
+                       stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """8-bit joint attention.  q8, k8, v8: (vis, ctx) pairs of code tensors;
+    scales: dict with sq_vis, sq_ctx, sk_vis, sk_ctx, sv."""
+    qv, qc = q8
+    kv, kc = k8
+    vv, vc = v8
+    B, Nv, H, D = qv.shape
+    Nc = qc.shape[1]
+    o_vis = torch.empty(qv.shape, dtype=torch.bfloat16, device=qv.device) if o_vis is None else o_vis
+    o_ctx = torch.empty(qc.shape, dtype=torch.bfloat16, device=qv.device) if o_ctx is None else o_ctx
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    st = _lib.lib().mmdit_joint_attention_q8(
+        _ptr(qv), _ptr(kv), _ptr(vv), _ptr(qc), _ptr(kc), _ptr(vc), _ptr(scales["sq_vis"]),
+        _ptr(scales["sq_ctx"]), _ptr(scales["sk_vis"]), _ptr(scales["sk_ctx"]),
+        _ptr(scales["sv"]), _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), B, Nv, Nc, H, D,
+        softmax_scale, _stream(stream))
+    check("mmdit_joint_attention_q8", st)
+    return o_vis, o_ctx
+
+
+def joint_attention_8bit(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
+                         softmax_scale: Optional[float] = None, stream=None):
+    """Quantise bf16 q, k, v (q per token, k per 128-token block, v per
+    channel) and run the 8-bit joint attention.  Returns (o_vis, o_ctx, parts)
+    with the codes and scales in ``parts``."""
+    qv8, sqv = quantize_int8(q_vis, 1, stream)
+    qc8, sqc = quantize_int8(q_ctx, 1, stream)
+    kv8, skv = quantize_int8(k_vis, 128, stream)
+    kc8, skc = quantize_int8(k_ctx, 128, stream)
+    vv8, vc8, sv = quantize_v_e4m3(v_vis, v_ctx, ctx_len, stream)
+    sc = {"sq_vis": sqv, "sq_ctx": sqc, "sk_vis": skv, "sk_ctx": skc, "sv": sv}
+    ov, oc = joint_attention_q8((qv8, qc8), (kv8, kc8), (vv8, vc8), sc, ctx_len, softmax_scale,
+                                stream=stream)
+    parts = {"q_vis": qv8, "q_ctx": qc8, "k_vis": kv8, "k_ctx": kc8, "v_vis": vv8, "v_ctx": vc8,
+             **sc}
+    return ov, oc, parts
+
+
 def make_window(parts: Sequence[int]) -> _lib.Window:
     w = _lib.Window()
     for a in range(3):

@@ -345,6 +345,74 @@ int mmdit_joint_attention_qnorm(const void* q_vis, const void* k_vis, const void
     return MMDIT_ERR_CUDA;
 }
 
+int mmdit_quantize_int8(const void* x, void* codes, float* scales, int B, int N, int H, int D,
+                        int block, void* stream) {
+    if (B < 0 || N < 0 || H < 0) return MMDIT_ERR_ARG;
+    if (D != kHeadDim || (block != 1 && block != 128)) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * N * H == 0) return MMDIT_OK;
+    if (!x || !codes || !scales) return MMDIT_ERR_ARG;
+    if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return MMDIT_ERR_ALIGN;
+    if ((long long)B * N * H >= (1LL << 31) || B > 65535 || H > 65535) return MMDIT_ERR_UNSUPPORTED;
+    return cuda_status(launch_quant_int8(x, codes, scales, B, N, H, block,
+                                         static_cast<cudaStream_t>(stream)),
+                       "quantize_int8");
+}
+
+int mmdit_quantize_v_e4m3(const void* v_vis, const void* v_ctx, const int32_t* ctx_len,
+                          void* c_vis, void* c_ctx, float* scales, int B, int Nv, int Nc, int H,
+                          int D, void* stream) {
+    if (B < 0 || Nv < 0 || Nc < 0 || H < 0) return MMDIT_ERR_ARG;
+    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * H == 0) return MMDIT_OK;
+    if (!scales) return MMDIT_ERR_ARG;
+    if (!aligned16(scales)) return MMDIT_ERR_ALIGN;
+    if (Nv > 0 && (!v_vis || !c_vis)) return MMDIT_ERR_ARG;
+    if (Nc > 0 && (!v_ctx || !c_ctx)) return MMDIT_ERR_ARG;
+    if ((Nv > 0 && (!aligned16(v_vis) || !aligned16(c_vis))) ||
+        (Nc > 0 && (!aligned16(v_ctx) || !aligned16(c_ctx))) ||
+        (ctx_len && (reinterpret_cast<uintptr_t>(ctx_len) & 3u)))
+        return MMDIT_ERR_ALIGN;
+    if ((long long)B * (Nv + (long long)Nc) * H >= (1LL << 31) || B > 65535 || H > 65535)
+        return MMDIT_ERR_UNSUPPORTED;
+    return cuda_status(launch_quant_v_e4m3(v_vis, v_ctx, ctx_len, c_vis, c_ctx, scales, B, Nv, Nc,
+                                           H, static_cast<cudaStream_t>(stream)),
+                       "quantize_v_e4m3");
+}
+
+int mmdit_joint_attention_q8(const void* q_vis, const void* k_vis, const void* v_vis,
+                             const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                             const float* sq_vis, const float* sq_ctx, const float* sk_vis,
+                             const float* sk_ctx, const float* sv, const int32_t* ctx_len,
+                             void* o_vis, void* o_ctx, int B, int Nv, int Nc, int H, int D,
+                             float softmax_scale, void* stream) {
+    if (B < 0 || Nv < 0 || Nc < 0 || H < 0) return MMDIT_ERR_ARG;
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MMDIT_ERR_ARG;
+    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * H * (Nv + (long long)Nc) == 0) return MMDIT_OK;
+    if (B > 65535 || H > 65535 || (long long)Nv + Nc > (1LL << 30)) return MMDIT_ERR_UNSUPPORTED;
+    if (!sv) return MMDIT_ERR_ARG;
+    if (Nv > 0) {
+        if (!q_vis || !k_vis || !v_vis || !o_vis || !sq_vis || !sk_vis) return MMDIT_ERR_ARG;
+        if (!aligned16(q_vis) || !aligned16(k_vis) || !aligned16(v_vis) || !aligned16(o_vis))
+            return MMDIT_ERR_ALIGN;
+    }
+    if (Nc > 0) {
+        if (!q_ctx || !k_ctx || !v_ctx || !o_ctx || !sq_ctx || !sk_ctx) return MMDIT_ERR_ARG;
+        if (!aligned16(q_ctx) || !aligned16(k_ctx) || !aligned16(v_ctx) || !aligned16(o_ctx))
+            return MMDIT_ERR_ALIGN;
+    }
+    for (const void* f : {(const void*)sq_vis, (const void*)sq_ctx, (const void*)sk_vis,
+                          (const void*)sk_ctx, (const void*)sv, (const void*)ctx_len})
+        if (f && (reinterpret_cast<uintptr_t>(f) & 3u)) return MMDIT_ERR_ALIGN;
+    const int r = launch_joint_attention_q8(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, sq_vis, sq_ctx,
+                                            sk_vis, sk_ctx, sv, ctx_len, o_vis, o_ctx, B, Nv, Nc,
+                                            H, softmax_scale, static_cast<cudaStream_t>(stream));
+    if (r == 0) return MMDIT_OK;
+    set_last_error("joint_attention_q8", r);
+    return MMDIT_ERR_CUDA;
+}
+
 int mmdit_joint_attention_fwd(const void* q_vis, const void* k_vis, const void* v_vis,
                               const void* q_ctx, const void* k_ctx, const void* v_ctx,
                               const int32_t* ctx_len, void* o_vis, void* o_ctx, float* lse, int B,
@@ -472,7 +540,9 @@ int mmdit_device_status(void* stream) {
     cudaError_t e = read_and_clear_device_status(&w, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_status(e, "device_status");
     if ((e = read_and_clear_bwd_status(&wb)) != cudaSuccess) return cuda_status(e, "device_status");
-    return (w | wb) ? MMDIT_ERR_TIMEOUT : MMDIT_OK;
+    unsigned int wq = 0;
+    if ((e = read_and_clear_q8_status(&wq)) != cudaSuccess) return cuda_status(e, "device_status");
+    return (w | wb | wq) ? MMDIT_ERR_TIMEOUT : MMDIT_OK;
 }
 
 void mmdit_set_wait_timeout_ns(unsigned long long ns) { set_wait_timeout_ns(ns); }

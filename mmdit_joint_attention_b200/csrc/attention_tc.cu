@@ -324,7 +324,9 @@ __device__ __forceinline__ float exp_half(const float (&sv)[128], uint32_t (&rh)
 // Q-norm mode: RMS-normalise (and, on visual rows, rotate) query row r of
 // tile i in place in shared memory, then release it to the MMA issuer.  Run by
 // all 256 softmax threads (thread = row of its warpgroup's tile).
-__device__ __forceinline__ void q_prologue(const Params& p, uint8_t* smem, Bars* bars,
+// Kept out of line: inlined, it measured slower (the main loop's schedule
+// changed).
+__device__ __noinline__ void q_prologue(const Params& p, uint8_t* smem, Bars* bars,
                                         const volatile Work* vwk, int i, int r) {
     float2* tab = reinterpret_cast<float2*>(smem + Smem::tab_off);
     const bool use_tab = p.rope && p.tab_entries > 0;

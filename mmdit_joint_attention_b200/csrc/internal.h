@@ -105,6 +105,25 @@ cudaError_t launch_joint_attention_bwd_f32(const float* qv, const float* kv, con
                                            int Nv, int Nc, int H, float softmax_scale,
                                            cudaStream_t s);
 
+// 8-bit joint attention: int8 q / k codes with q row scales [B, H, N_s] and k
+// block scales [B, H, ceil(N_s / 128)], E4M3 v codes with channel scales
+// [B, H, 128]; bf16 outputs.  Return convention of the bf16 launcher.
+int launch_joint_attention_q8(const void* qv, const void* kv, const void* vv, const void* qc,
+                              const void* kc, const void* vc, const float* sqv, const float* sqc,
+                              const float* skv, const float* skc, const float* sv,
+                              const int32_t* ctx_len, void* ov, void* oc, int B, int Nv, int Nc,
+                              int H, float softmax_scale, cudaStream_t s);
+// int8 codes of bf16 x [B, N, H, 128] with one scale per `block` (1 or 128)
+// consecutive tokens of a (sample, head): scales [B, H, ceil(N / block)].
+cudaError_t launch_quant_int8(const void* x, void* codes, float* scales, int B, int N, int H,
+                              int block, cudaStream_t s);
+// E4M3 codes of bf16 v of both streams with one scale per (sample, head,
+// channel) over the valid tokens: scales [B, H, 128].
+cudaError_t launch_quant_v_e4m3(const void* vv, const void* vc, const int32_t* ctx_len, void* cv,
+                                void* cc, float* scales, int B, int Nv, int Nc, int H,
+                                cudaStream_t s);
+cudaError_t read_and_clear_q8_status(unsigned int* out);
+
 // Limit of one bounded pipeline wait (set_wait_timeout_ns, else the default).
 uint64_t wait_timeout_ns();
 

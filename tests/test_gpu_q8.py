@@ -1,0 +1,90 @@
+"""GPU parity of the 8-bit joint attention (Wan 2.1 report, section 4.4.3:
+Int8 S = Q K^T, FP8 E4M3 O = P V) through the C ABI.
+
+The quantisers must reproduce the oracle's codes and scales exactly (integer
+and byte work).  The attention is compared with the oracle's whole 8-bit
+method run from the unquantised inputs (the oracle quantises by itself), with
+the bf16 criterion; small cases in full, 480p on sampled rows."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mmdit_joint_attention_b200 import api
+from mmdit_joint_attention_b200 import inputs as I
+from helpers import device_inputs, from_dev, parity
+
+pytestmark = pytest.mark.gpu
+
+W = I.WORKLOADS
+
+
+def _ws(w: I.Workload, **kw) -> I.Workload:
+    import dataclasses
+    return dataclasses.replace(w, **kw)
+
+
+CASES = {
+    "block": W["block"],
+    "ragged_small": _ws(W["block"], B=2, H=3, grid=(3, 10, 10), Nc=77, ctx_len=(77, 5)),
+    "cond_all_masked": _ws(W["block"], H=2, grid=(2, 10, 10), Nc=130, ctx_len=(0,)),
+    "long_2k": _ws(W["block"], H=2, grid=(4, 16, 32), Nc=64),
+}
+
+
+@pytest.mark.parametrize("case", sorted(CASES) + ["480p"])
+def test_quantisers_match_the_oracle(case):
+    w = CASES.get(case) or W[case]
+    inp = I.make_inputs(w, seed=8, parts=("qkv",))
+    t = device_inputs(inp)
+    cl = t["ctx_len"] if w.ctx_len is not None else None
+    for name, block in (("q_vis", 1), ("q_ctx", 1), ("k_vis", 128), ("k_ctx", 128)):
+        codes, scales = api.quantize_int8(t[name], block)
+        rc, rs = oracle.quant_int8(inp[name].f64, block)
+        assert np.array_equal(codes.cpu().numpy(), rc), f"{case} {name} codes"
+        assert np.array_equal(scales.cpu().numpy(), rs), f"{case} {name} scales"
+    cv, cc, sv = api.quantize_v_e4m3(t["v_vis"], t["v_ctx"], cl)
+    rv, rcc, rsv = oracle.quant_v_e4m3(inp["v_vis"].f64, inp["v_ctx"].f64, inp["ctx_len"])
+    assert np.array_equal(sv.cpu().numpy(), rsv), f"{case} v scales"
+    assert np.array_equal(cv.cpu().numpy(), rv), f"{case} v codes (visual)"
+    assert np.array_equal(cc.cpu().numpy(), rcc), f"{case} v codes (cond)"
+
+
+def _run(w, seed=9):
+    inp = I.make_inputs(w, seed=seed, parts=("qkv",))
+    t = device_inputs(inp)
+    cl = t["ctx_len"] if w.ctx_len is not None else None
+    ov, oc, _ = api.joint_attention_8bit(t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"],
+                                         t["k_ctx"], t["v_ctx"], cl)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    return inp, from_dev(ov), from_dev(oc)
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_attention_q8_full(case):
+    w = CASES[case]
+    inp, ov, oc = _run(w)
+    args = [inp[k].f64 for k in ("q_vis", "k_vis", "v_vis", "q_ctx", "k_ctx", "v_ctx")]
+    rv, rc = oracle.attention_q8(*args, ctx_len=inp["ctx_len"])
+    parity(ov, rv, "bf16", f"{case} o_vis")
+    parity(oc, rc, "bf16", f"{case} o_ctx")
+    for b, L in enumerate(w.ctx_lengths()):
+        assert np.all(oc[b, L:] == 0.0)
+
+
+def test_attention_q8_sampled_480p():
+    w = W["480p"]
+    inp, ov, oc = _run(w)
+    full = np.concatenate([ov, oc], axis=1)
+    trip = []
+    for h in range(w.H):
+        rows = I.parity_rows(w, 0, h, n_random=64)
+        trip.append(np.stack([np.zeros_like(rows), np.full_like(rows, h), rows], axis=1))
+    trip = np.concatenate(trip)
+    args = [inp[k].f64 for k in ("q_vis", "k_vis", "v_vis", "q_ctx", "k_ctx", "v_ctx")]
+    ref = oracle.attention_q8(*args, ctx_len=inp["ctx_len"], rows=trip)
+    got = full[trip[:, 0], trip[:, 2], trip[:, 1]]
+    vis = trip[:, 2] < w.Nv
+    parity(got[vis], ref[vis], "bf16", "480p q8 o_vis rows")
+    parity(got[~vis], ref[~vis], "bf16", "480p q8 o_ctx rows")
