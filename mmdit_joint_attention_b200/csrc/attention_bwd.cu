@@ -173,12 +173,18 @@ delta_kernel(const T* __restrict__ ov, const T* __restrict__ dov, const T* __res
 // ======================================================================
 namespace dq {
 
+// K is read twice per tile (S = Q K^T, then dQ += dS K one tile later), so its
+// ring has a third stage: with two, the next K's load could only start just
+// before the product that needs it.  V is read once (dP = dO V^T).
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+
 struct Smem {
     static constexpr int q_off = 0;
     static constexpr int do_off = kTileBytes;
-    static constexpr int k_off = 2 * kTileBytes;   // 2 stages
-    static constexpr int v_off = 4 * kTileBytes;   // 2 stages
-    static constexpr int bar_off = 6 * kTileBytes;
+    static constexpr int k_off = 2 * kTileBytes;                        // kKStages tiles
+    static constexpr int v_off = k_off + kKStages * kTileBytes;         // kVStages tiles
+    static constexpr int bar_off = v_off + kVStages * kTileBytes;
     static constexpr int total = bar_off + 256;
 };
 
@@ -201,8 +207,8 @@ struct Params {
 
 struct Bars {
     uint64_t q_full;
-    uint64_t k_full[2], k_empty[2];
-    uint64_t v_full[2], v_empty[2];
+    uint64_t k_full[kKStages], k_empty[kKStages];
+    uint64_t v_full[kVStages], v_empty[kVStages];
     uint64_t s_full[2];    // S and dP of the tile with this S buffer are in tensor memory
     uint64_t dp_free;      // every softmax warp has read dP
     uint64_t ds_full[4];   // [2 buf + wg]: that warpgroup's half of dS is in tensor memory
@@ -211,6 +217,34 @@ struct Bars {
     Ctl ctl;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block must fit its shared-memory slot");
+
+// dS = exp2(S * scale log2 e - lse log2 e) * (dP - D) for 64 keys of one row,
+// packed in bf16 pairs; keys at or past `valid` get dS = 0.  (A variant that
+// masks only tail tiles duplicated this loop and made the softmax spill.)
+__device__ __forceinline__ void ds_half(const uint32_t (&sr)[2][32], const uint32_t (&dr)[2][32],
+                                        uint32_t (&pk)[32], uint64_t sl2x2, uint64_t nl2,
+                                        uint64_t ndl, int valid) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const int k = 2 * c;
+        const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[k >> 5][k & 31]),
+                                          __uint_as_float(sr[k >> 5][(k & 31) + 1])),
+                                  sl2x2, nl2);
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        if (valid < 64) {
+            if (k >= valid) x0 = -INFINITY;
+            if (k + 1 >= valid) x1 = -INFINITY;
+        }
+        const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        const uint64_t dd = f2_add(f2_pack(__uint_as_float(dr[k >> 5][k & 31]),
+                                           __uint_as_float(dr[k >> 5][(k & 31) + 1])),
+                                   ndl);
+        float d0, d1;
+        f2_unpack(f2_mul(pp, dd), d0, d1);
+        pk[c] = pack_bf16x2(d0, d1);
+    }
+}
 
 // Tensor memory: S0 [0,128) S1 [128,256) dP [256,384) dQ [384,512).  dS of
 // key half w is written over S at columns [64 w, 64 w + 32).
@@ -239,13 +273,15 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kKStages; ++i) {
             mbar_init(&bars->k_full[i], 1);
             mbar_init(&bars->k_empty[i], 1);
+        }
+        for (int i = 0; i < kVStages; ++i) {
             mbar_init(&bars->v_full[i], 1);
             mbar_init(&bars->v_empty[i], 1);
-            mbar_init(&bars->s_full[i], 1);
         }
+        for (int i = 0; i < 2; ++i) mbar_init(&bars->s_full[i], 1);
         mbar_init(&bars->dp_free, 8);
         for (int i = 0; i < 4; ++i) mbar_init(&bars->ds_full[i], 4);
         mbar_init(&bars->o_done, 1);
@@ -296,10 +332,11 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 tma_load_4d(smem + Smem::do_off + kHalf128, &p.tm_do[seg], &bars->q_full, 64, h,
                             row0, b);
             }
+            const int stages = is_k ? kKStages : kVStages;
             int issued = 0;
             for (int j = 0; j < n_kv; ++j) {
-                const int st = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
+                const int st = j % stages;
+                const uint32_t ph = (j / stages) & 1;
                 const int ks = j < kv_vis ? 0 : 1;
                 const int row = (ks ? j - kv_vis : j) * 128;
                 if (!wait(&empty[st], ph ^ 1, ctl)) break;
@@ -310,8 +347,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 ++issued;
             }
             if (ctl->abort) {
-                for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-                    mbar_wait_bounded(&full[j & 1], (j >> 1) & 1, nullptr, kDrainLimitNs);
+                for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j)
+                    mbar_wait_bounded(&full[j % stages], (j / stages) & 1, nullptr,
+                                      kDrainLimitNs);
                 if (is_k) mbar_wait_bounded(&bars->q_full, 0, nullptr, kDrainLimitNs);
             }
         } else if (warp == 9 && lane == 0) {
@@ -320,13 +358,16 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             constexpr uint32_t id_mn = idesc_bf16_f32(128, 128, 0, 1);
             bool ok = wait(&bars->q_full, 0, ctl);
             const uint64_t dq_d = kdesc(sQ), ddo_d = kdesc(sDO);
-            const uint64_t dk0 = kdesc(sK), dk1 = kdesc(sK + kTileBytes);
             const uint64_t dv0 = kdesc(sV), dv1 = kdesc(sV + kTileBytes);
-            const uint64_t km0 = mndesc(sK, kHalf128), km1 = mndesc(sK + kTileBytes, kHalf128);
+            // K stage st: K-major for S, MN-major for dQ (descriptor start
+            // addresses differ by whole tiles)
+            const uint64_t dk0 = kdesc(sK);
+            const uint64_t km0 = mndesc(sK, kHalf128);
+            constexpr uint64_t kTileStep = kTileBytes >> 4;
             // dQ += dS(jj) K(jj), key half by key half as the softmax releases them
-            auto dq_mma = [&](int jj) -> bool {
+            auto dq_mma = [&](int jj, int kst_jj) -> bool {
                 const int pb = jj & 1;
-                const uint64_t km = pb ? km1 : km0;
+                const uint64_t km = km0 + (uint64_t)kst_jj * kTileStep;
                 const uint32_t sb = tmem + 128 * pb;
 #pragma unroll
                 for (int wg = 0; wg < 2; ++wg) {
@@ -341,12 +382,13 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 }
                 return true;
             };
+            int kst = 0, kph = 0, kst_prev = 0;      // K stage of tile j, its phase, and of j - 1
             for (int j = 0; ok && j < n_kv; ++j) {
-                const int st = j & 1;
+                const int st = j & 1;                // S buffer and V stage
                 const uint32_t ph = (j >> 1) & 1;
-                if (!(ok = wait(&bars->k_full[st], ph, ctl))) break;
+                if (!(ok = wait(&bars->k_full[kst], kph, ctl))) break;
                 tc_fence_after();
-                const uint64_t dk = st ? dk1 : dk0;
+                const uint64_t dk = dk0 + (uint64_t)kst * kTileStep;
 #pragma unroll
                 for (int s = 0; s < 8; ++s) {
                     const uint64_t off = koff(s, kHalf128);
@@ -364,12 +406,17 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 mma_commit(&bars->s_full[st]);
                 mma_commit(&bars->v_empty[st]);
                 if (j > 0) {
-                    if (!(ok = dq_mma(j - 1))) break;
-                    mma_commit(&bars->k_empty[(j - 1) & 1]);
+                    if (!(ok = dq_mma(j - 1, kst_prev))) break;
+                    mma_commit(&bars->k_empty[kst_prev]);
+                }
+                kst_prev = kst;
+                if (++kst == kKStages) {
+                    kst = 0;
+                    kph ^= 1;
                 }
             }
-            if (ok && (ok = dq_mma(n_kv - 1))) {
-                mma_commit(&bars->k_empty[(n_kv - 1) & 1]);
+            if (ok && (ok = dq_mma(n_kv - 1, kst_prev))) {
+                mma_commit(&bars->k_empty[kst_prev]);
                 mma_commit(&bars->o_done);
             }
             mma_commit(&bars->drain);
@@ -410,26 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             const int valid =
                 (j < kv_vis ? p.N[0] - j * 128 : L - (j - kv_vis) * 128) - 64 * wg;
             uint32_t pk[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const int k = 2 * c;
-                uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[k >> 5][k & 31]),
-                                            __uint_as_float(sr[k >> 5][(k & 31) + 1])),
-                                    sl2x2, nl2);
-                float x0, x1;
-                f2_unpack(x, x0, x1);
-                if (valid < 64) {
-                    if (k >= valid) x0 = -INFINITY;
-                    if (k + 1 >= valid) x1 = -INFINITY;
-                }
-                const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
-                const uint64_t dd = f2_add(f2_pack(__uint_as_float(dr[k >> 5][k & 31]),
-                                                   __uint_as_float(dr[k >> 5][(k & 31) + 1])),
-                                           ndl);
-                float d0, d1;
-                f2_unpack(f2_mul(pp, dd), d0, d1);
-                pk[c] = pack_bf16x2(d0, d1);
-            }
+            ds_half(sr, dr, pk, sl2x2, nl2, ndl, valid);
             tmem_st32(tS, pk);
             tmem_wait_st();
             tc_fence_before();
