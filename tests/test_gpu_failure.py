@@ -1,8 +1,9 @@
 """Failure detection on the GPU without a fault: every wait in the attention
-kernel is bounded; when one runs out the kernel drains, frees its tensor
-memory, returns, and the status word reports MMDIT_ERR_TIMEOUT.  The test
-shortens the wait limit so that the waits of an ordinary launch run out, then
-checks the status, and that the context is healthy afterwards."""
+kernels (forward, backward, 8-bit) is bounded; when one runs out the kernel
+drains, frees its tensor memory, returns, and the status word reports
+MMDIT_ERR_TIMEOUT.  The tests shorten the wait limit so that the waits of an
+ordinary launch run out, then check the status, and that the context is
+healthy afterwards."""
 import pytest
 import torch
 
@@ -40,3 +41,44 @@ def test_wait_timeout_is_reported_and_context_survives():
                                     inp["q_ctx"].f64, inp["k_ctx"].f64, inp["v_ctx"].f64)
     parity(from_dev(ov), rv, "bf16", "o_vis after a timed-out launch")
     parity(from_dev(oc), rc, "bf16", "o_ctx after a timed-out launch")
+
+
+def test_backward_and_q8_wait_timeouts_are_reported():
+    """The same for the backward kernels and the 8-bit attention kernel: with
+    the waits cut short both report MMDIT_ERR_TIMEOUT, and the next call at the
+    default limit is correct."""
+    w = I.WORKLOADS["block"]
+    inp = I.make_inputs(w, seed=3, parts=("qkv",))
+    gin = I.make_grad_outputs(w, seed=3)
+    t = device_inputs(inp)
+    from helpers import to_dev
+    do_vis, do_ctx = to_dev(gin["do_vis"]), to_dev(gin["do_ctx"])
+    qkv = (t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"], t["v_ctx"])
+    ov, oc, lse = api.joint_attention_fwd(*qkv)
+    torch.cuda.synchronize()
+    L = _lib.lib()
+    for call in ("bwd", "q8"):
+        assert api.device_status() == 0
+        try:
+            L.mmdit_set_wait_timeout_ns(1)
+            if call == "bwd":
+                api.joint_attention_bwd(*qkv, ov, oc, do_vis, do_ctx, lse)
+            else:
+                api.joint_attention_8bit(*qkv)
+            status = api.device_status()
+        finally:
+            L.mmdit_set_wait_timeout_ns(0)
+        assert status == _lib.STATUS_CODES["MMDIT_ERR_TIMEOUT"], call
+        assert api.device_status() == 0
+    g = api.joint_attention_bwd(*qkv, ov, oc, do_vis, do_ctx, lse)
+    q8v, q8c, _ = api.joint_attention_8bit(*qkv)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    ref = oracle.joint_attention_bwd(inp["q_vis"].f64, inp["k_vis"].f64, inp["v_vis"].f64,
+                                     inp["q_ctx"].f64, inp["k_ctx"].f64, inp["v_ctx"].f64,
+                                     gin["do_vis"].f64, gin["do_ctx"].f64)
+    for k in ("dq_vis", "dk_vis", "dv_vis"):
+        parity(from_dev(g[k]), ref[k], "bf16", f"{k} after a timed-out launch")
+    rv, _ = oracle.attention_q8(inp["q_vis"].f64, inp["k_vis"].f64, inp["v_vis"].f64,
+                                inp["q_ctx"].f64, inp["k_ctx"].f64, inp["v_ctx"].f64)
+    parity(from_dev(q8v), rv, "bf16", "8-bit o_vis after a timed-out launch")
