@@ -1,7 +1,7 @@
 """Shared test helpers: device transfer of synthetic inputs and the parity
 criterion.
 
-Parity criterion (tolerances of the benchmark spec):
+Parity criterion (the tolerances stated for this path):
   * fp32 outputs: max |gpu - exact| <= 1e-4, exact = float64 oracle result;
   * bf16 outputs: the reference is the float64 oracle result rounded (RNE) to
     bf16, the storage type of the output buffer, i.e. the best answer a bf16
