@@ -55,3 +55,13 @@ def test_parity_rows_cover_boundaries():
     for r in (0, 127, 128, Nv - 1, (Nv // 128) * 128, Nv + 299, Nv + 300):
         assert r in rows
     assert rows.min() >= 0 and rows.max() < Nv + w.Nc
+
+
+def test_grad_outputs_deterministic_and_independent():
+    w = I.WORKLOADS["block"]
+    a = I.make_grad_outputs(w, seed=4)
+    b = I.make_grad_outputs(w, seed=4)
+    assert np.array_equal(a["do_vis"].storage, b["do_vis"].storage)
+    assert a["do_vis"].shape == (w.B, w.Nv, w.H, w.D) and a["do_ctx"].shape == (w.B, w.Nc, w.H, w.D)
+    q = I.make_inputs(w, seed=4, parts=("qkv",))["q_vis"]
+    assert not np.array_equal(a["do_vis"].storage, q.storage)   # its own random stream
