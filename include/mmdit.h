@@ -8,7 +8,8 @@
  * stream follows the patchify-and-flatten step of the Wan 2.1 report, section
  * 4.2.1, and the attention is non-causal (Wan 2.1 report, section 4.3.1).
  *
- * Conventions shared by every entry point:
+ * Conventions shared by every entry point (the host-buffer executor at the
+ * end, mmdit_block_forward_host, differs where its comment says so):
  *   - All tensor pointers are DEVICE pointers to contiguous row-major arrays,
  *     16-byte aligned.  The caller owns all memory; the library allocates no
  *     device memory and keeps no state between calls.
@@ -387,6 +388,94 @@ MMDIT_API int mmdit_residual_modulate(const void* x, const void* branch, const f
                                       const float* shift, const float* scale, void* x_out,
                                       void* y, int B, int N, int C, float eps, mmdit_dtype dt,
                                       void* stream);
+
+/* ---- Host-buffer executor -------------------------------------------------
+ *
+ * Runs the whole path of one block, step after step, from HOST buffers
+ * [Vimoo §2.2, the dual-stream block]:
+ *   y   = adaLN modulate of x                    (mmdit_adaln_modulate, both streams)
+ *   q,k = QK-RMSNorm (+ 3D RoPE on the visual stream)   (mmdit_qk_norm_rope)
+ *   o   = joint attention over both streams      (mmdit_joint_attention)
+ *   x'  = x + gate * o                           (mmdit_gated_residual, both streams)
+ * The projections of a full block (QKV, output, MLP) are outside this library:
+ * q, k, v arrive as inputs and the attention output is the gated branch.  Each
+ * step is the same computation, with the same kernels and results, as these
+ * seven calls made one after the other on device buffers.
+ *
+ * Unlike the rest of this header, the executor moves data between host and
+ * device itself: it copies a step's inputs in, runs the kernels and copies the
+ * outputs back.  It pipelines the steps over three CUDA streams of its own, so
+ * that one step's input copy, another step's kernels and a third step's output
+ * copy run at the same time.  Device memory comes from a caller-provided
+ * workspace cut into slots of mmdit_block_slot_bytes() bytes; each step takes a
+ * slot, and a slot is reused only once the step that held it has copied its
+ * outputs out.  Three slots keep the copies and the kernels all busy; one slot
+ * runs the steps one after the other. */
+
+/* Sizes and constants shared by every step. */
+typedef struct {
+    int B, Nv, Nc, H, D;      /* batch, visual tokens, cond tokens, heads, head dim (128);
+                                 C = H * D */
+    mmdit_grid grid;          /* visual token grid (T*H*W == Nv) and its RoPE */
+    const float* gq_vis;      /* DEVICE [D] fp32 RMSNorm scales of q and k per stream */
+    const float* gk_vis;
+    const float* gq_ctx;      /* may be NULL when Nc == 0 */
+    const float* gk_ctx;
+    float norm_eps;           /* QK-RMSNorm eps */
+    float ln_eps;             /* adaLN LayerNorm eps */
+    float softmax_scale;      /* > 0 (1/sqrt(D) in the usual form) */
+    mmdit_dtype dt;
+} mmdit_block_config;
+
+/* HOST buffers of one step, laid out as in the device entry points above.
+ * Page-locked (pinned) memory lets the copies run asynchronously and overlap
+ * the kernels; pageable memory gives the same results without the overlap. */
+typedef struct {
+    const void* q_vis;         /* [B, Nv, H, D] dt */
+    const void* k_vis;
+    const void* v_vis;
+    const void* q_ctx;         /* [B, Nc, H, D] dt (unused when Nc == 0) */
+    const void* k_ctx;
+    const void* v_ctx;
+    const void* x_vis;         /* [B, Nv, C] dt residual stream */
+    const void* x_ctx;         /* [B, Nc, C] dt */
+    const float* shift_vis;    /* [B, C] fp32 adaLN shift, scale and gate per stream */
+    const float* scale_vis;
+    const float* gate_vis;
+    const float* shift_ctx;
+    const float* scale_ctx;
+    const float* gate_ctx;
+    const int32_t* ctx_len;    /* [B], or NULL: all Nc cond tokens valid */
+    void* y_vis;               /* out [B, Nv, C] dt: modulated x, or NULL: not copied back */
+    void* y_ctx;
+    void* o_vis;               /* out [B, Nv, H, D] dt: attention output, or NULL */
+    void* o_ctx;
+    void* x_out_vis;           /* out [B, Nv, C] dt: x + gate * o (required) */
+    void* x_out_ctx;           /* required when Nc > 0 */
+} mmdit_block_step;
+
+/* Device bytes one step's slot needs, or a negative MMDIT_ERR_* code if the
+ * configuration is invalid.  Makes no CUDA call. */
+MMDIT_API long long mmdit_block_slot_bytes(const mmdit_block_config* cfg);
+
+/* Runs steps[0..n_steps) in order, each from and to its own host buffers.
+ *   workspace: DEVICE memory, 256-byte aligned, workspace_bytes long; the
+ *     executor uses floor(workspace_bytes / slot bytes) slots (at most 4, at
+ *     most n_steps) and must not be given less than one slot.
+ *   stream: the work starts after what is already queued on `stream`, and
+ *     everything queued on `stream` afterwards waits for the last output copy.
+ *     The call returns once the work is enqueued; synchronise `stream` before
+ *     reading the host outputs or reusing the host inputs.
+ * Host input buffers may be shared between steps; output buffers of different
+ * steps may also coincide (the output copies run in step order, so the last
+ * step's values remain).  The workspace must not be used by anything else
+ * until the work has finished.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED before anything is
+ * enqueued; MMDIT_ERR_CUDA if a CUDA call fails while enqueueing (work already
+ * enqueued still completes before later work on `stream`). */
+MMDIT_API int mmdit_block_forward_host(const mmdit_block_config* cfg,
+                                       const mmdit_block_step* steps, int n_steps,
+                                       void* workspace, long long workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device: MMDIT_OK, or MMDIT_ERR_TIMEOUT if a kernel gave up on a

@@ -41,6 +41,26 @@ class Window(ctypes.Structure):
     _fields_ = [("parts", ctypes.c_int * 3)]
 
 
+class BlockConfig(ctypes.Structure):
+    """mmdit_block_config: sizes and constants of the host-buffer executor."""
+    _fields_ = [("B", ctypes.c_int), ("Nv", ctypes.c_int), ("Nc", ctypes.c_int),
+                ("H", ctypes.c_int), ("D", ctypes.c_int), ("grid", Grid),
+                ("gq_vis", ctypes.c_void_p), ("gk_vis", ctypes.c_void_p),
+                ("gq_ctx", ctypes.c_void_p), ("gk_ctx", ctypes.c_void_p),
+                ("norm_eps", ctypes.c_float), ("ln_eps", ctypes.c_float),
+                ("softmax_scale", ctypes.c_float), ("dt", ctypes.c_int)]
+
+
+BLOCK_STEP_FIELDS = ("q_vis", "k_vis", "v_vis", "q_ctx", "k_ctx", "v_ctx", "x_vis", "x_ctx",
+                     "shift_vis", "scale_vis", "gate_vis", "shift_ctx", "scale_ctx", "gate_ctx",
+                     "ctx_len", "y_vis", "y_ctx", "o_vis", "o_ctx", "x_out_vis", "x_out_ctx")
+
+
+class BlockStep(ctypes.Structure):
+    """mmdit_block_step: host buffers of one step (every field a pointer)."""
+    _fields_ = [(name, ctypes.c_void_p) for name in BLOCK_STEP_FIELDS]
+
+
 class MmditError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
@@ -60,7 +80,7 @@ def declared_functions():
     """Names of the functions include/mmdit.h declares."""
     with open(HEADER) as f:
         text = f.read()
-    return sorted(set(re.findall(r"^MMDIT_API\s+(?:int|void|const char\*)\s+(mmdit_\w+)\s*\(",
+    return sorted(set(re.findall(r"^MMDIT_API\s+(?:int|void|long long|const char\*)\s+(mmdit_\w+)\s*\(",
                                  text, re.M)))
 
 
@@ -99,6 +119,11 @@ def lib():
         L.mmdit_gated_residual.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
         L.mmdit_residual_modulate.argtypes = [_vp] * 7 + [_i, _i, _i, _f, _i, _vp]
         L.mmdit_device_status.argtypes = [_vp]
+        L.mmdit_block_slot_bytes.argtypes = [ctypes.POINTER(BlockConfig)]
+        L.mmdit_block_slot_bytes.restype = ctypes.c_longlong
+        L.mmdit_block_forward_host.argtypes = [ctypes.POINTER(BlockConfig),
+                                               ctypes.POINTER(BlockStep), _i, _vp,
+                                               ctypes.c_longlong, _vp]
         L.mmdit_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
         L.mmdit_set_wait_timeout_ns.restype = None
         L.mmdit_last_error.argtypes = []
@@ -111,7 +136,8 @@ def lib():
                      "mmdit_window_permute", "mmdit_joint_attention",
                      "mmdit_joint_attention_fwd", "mmdit_joint_attention_bwd",
                      "mmdit_joint_window_attention", "mmdit_adaln_modulate",
-                     "mmdit_gated_residual", "mmdit_residual_modulate", "mmdit_device_status"):
+                     "mmdit_gated_residual", "mmdit_residual_modulate", "mmdit_device_status",
+                     "mmdit_block_forward_host"):
             getattr(L, name).restype = ctypes.c_int
         _LIB = L
     return _LIB

@@ -485,3 +485,73 @@ def block_forward(t: dict, grid: Sequence[int], pos_scale=(1.0, 1.0, 1.0), eps: 
         out["x_" + s] = gated_residual(t["x_" + s], out["o_" + s].view(B, n, H * D),
                                        t["gate_" + s], stream=stream)
     return out
+
+
+class BlockHostExecutor:
+    """``block_forward``'s path run step after step from HOST tensors, through
+    mmdit_block_forward_host: the library copies each step's inputs in, runs the
+    seven kernels and copies the outputs back, overlapping the copies of some
+    steps with the kernels of others on streams of its own.
+
+    The device workspace (``slots`` slots, one step each) is allocated here
+    with torch; the RMSNorm scales are device tensors kept for the executor's
+    lifetime.  A step is a dict of CPU tensors keyed like ``mmdit_block_step``
+    (``_lib.BLOCK_STEP_FIELDS``); ``y_*`` and ``o_*`` may be left out (not
+    copied back), ``ctx_len`` too (every cond token valid).  Pinned host memory
+    lets the copies overlap the kernels."""
+
+    def __init__(self, B: int, Nv: int, Nc: int, H: int, grid: Sequence[int],
+                 gq_vis: torch.Tensor, gk_vis: torch.Tensor, gq_ctx: torch.Tensor,
+                 gk_ctx: torch.Tensor, pos_scale=(1.0, 1.0, 1.0), rope_base: float = 10000.0,
+                 split=(16, 56, 56), eps: float = 1e-6, softmax_scale: Optional[float] = None,
+                 dtype: torch.dtype = torch.bfloat16, slots: int = 3):
+        _f32(gq_vis, gk_vis, gq_ctx, gk_ctx)
+        if dtype not in _DT:
+            raise TypeError(f"unsupported dtype {dtype}")
+        D = gq_vis.shape[0]
+        self.dtype, self.B, self.N, self.C = dtype, B, {"vis": Nv, "ctx": Nc}, H * D
+        c = _lib.BlockConfig()
+        c.B, c.Nv, c.Nc, c.H, c.D = B, Nv, Nc, H, D
+        c.grid = make_grid(grid, pos_scale, rope_base, split)
+        c.gq_vis, c.gk_vis = gq_vis.data_ptr(), gk_vis.data_ptr()
+        c.gq_ctx, c.gk_ctx = gq_ctx.data_ptr(), gk_ctx.data_ptr()
+        c.norm_eps = c.ln_eps = eps
+        c.softmax_scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
+        c.dt = _DT[dtype]
+        self.cfg = c
+        self._scales = (gq_vis, gk_vis, gq_ctx, gk_ctx)
+        nbytes = _lib.lib().mmdit_block_slot_bytes(ctypes.byref(c))
+        if nbytes < 0:
+            raise _lib.MmditError("mmdit_block_slot_bytes", int(nbytes))
+        self.slot_bytes = int(nbytes)
+        self.workspace = torch.empty(slots * self.slot_bytes, dtype=torch.uint8,
+                                     device=gq_vis.device)
+
+    def _host(self, name: str, t: torch.Tensor) -> int:
+        s = name.rsplit("_", 1)[1]
+        if name == "ctx_len":
+            want, dt = self.B, torch.int32
+        elif name.split("_")[0] in ("shift", "scale", "gate"):
+            want, dt = self.B * self.C, torch.float32
+        else:
+            want, dt = self.B * self.N[s] * self.C, self.dtype
+        if t.is_cuda or not t.is_contiguous() or t.dtype != dt or t.numel() != want:
+            raise ValueError(f"step[{name!r}] must be a contiguous CPU {dt} tensor of "
+                             f"{want} elements")
+        return t.data_ptr()
+
+    def run(self, steps: Sequence[dict], stream=None) -> None:
+        """Enqueues every step on ``stream`` (default: the current stream);
+        synchronise it before reading the outputs."""
+        arr = (_lib.BlockStep * max(1, len(steps)))()
+        for i, st in enumerate(steps):
+            unknown = set(st) - set(_lib.BLOCK_STEP_FIELDS)
+            if unknown:
+                raise KeyError(f"unknown step fields {sorted(unknown)}")
+            for name, t in st.items():
+                if t is not None:
+                    setattr(arr[i], name, self._host(name, t))
+        status = _lib.lib().mmdit_block_forward_host(
+            ctypes.byref(self.cfg), arr, len(steps), ctypes.c_void_p(self.workspace.data_ptr()),
+            self.workspace.numel(), _stream(stream))
+        check("mmdit_block_forward_host", status)

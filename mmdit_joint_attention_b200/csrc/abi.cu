@@ -46,8 +46,10 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
+}  // namespace
+
 // Validates a RoPE grid for N tokens of head dim D and converts it.
-int check_grid(const mmdit_grid* grid, long long N, int D, mmdit_dtype dt, RopeGrid& g) {
+int mmdit::check_grid(const mmdit_grid* grid, long long N, int D, mmdit_dtype dt, RopeGrid& g) {
     if (grid->T < 1 || grid->H < 1 || grid->W < 1) return MMDIT_ERR_SHAPE;
     if ((long long)grid->T * grid->H * grid->W != N) return MMDIT_ERR_SHAPE;
     int sum = 0;
@@ -71,6 +73,8 @@ int check_grid(const mmdit_grid* grid, long long N, int D, mmdit_dtype dt, RopeG
     g.base = grid->rope_base;
     return MMDIT_OK;
 }
+
+namespace {
 
 // Validates a window partition of the grid's T, H, W extents.
 int check_window(const mmdit_grid* grid, const mmdit_window* win) {

@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "../../include/mmdit.h"
 #include "window.h"
 
 namespace mmdit {
@@ -21,6 +22,10 @@ struct RopeText {
     double base;
     int split[3];
 };
+
+// Validates a RoPE grid for N tokens of head dim D and converts it: MMDIT_OK
+// or the MMDIT_ERR_* code the entry points return for it.
+int check_grid(const mmdit_grid* grid, long long N, int D, mmdit_dtype dt, RopeGrid& g);
 
 // 0 or a cudaError_t value.  At most one of grid / text is non-null.
 // q_in == null: k alone (no text positions, no permutation).

@@ -174,3 +174,75 @@ def test_qk_norm_rope_bwd_validation(L):
     assert f(P, P, P, P, P, P, U, P, P, P, 1, 32, 2, 128, R(g), 1e-6, 1, None) == -3
     assert f(P, P, P, P, P, P, P, P, P, P, 1, 31, 2, 128, R(g), 1e-6, 1, None) == -2  # N != THW
     assert f(P, P, P, P, P, P, P, P, P, P, 1, 32, 2, 128, R(g), -1.0, 1, None) == -1  # eps
+
+
+def _block_cfg(B=1, Nv=32, Nc=8, H=2, dt=1):
+    c = _lib.BlockConfig()
+    c.B, c.Nv, c.Nc, c.H, c.D = B, Nv, Nc, H, 128
+    c.grid = _lib.Grid(2, 4, 4, (ctypes.c_float * 3)(1, 1, 1), 10000.0,
+                       (ctypes.c_int * 3)(16, 56, 56))
+    c.gq_vis = c.gk_vis = c.gq_ctx = c.gk_ctx = 16
+    c.norm_eps = c.ln_eps = 1e-6
+    c.softmax_scale = 128 ** -0.5
+    c.dt = dt
+    return c
+
+
+def test_block_slot_bytes_layout(L):
+    """A slot holds q, k, v, x, y, o of both streams, the three [B, C] fp32
+    vectors of both streams and ctx_len, each region rounded up to 256 bytes."""
+    r256 = lambda n: (n + 255) // 256 * 256
+    for B, Nv, Nc, H, dt, esz in ((1, 32, 8, 2, 1, 2), (3, 32, 0, 4, 1, 2), (2, 32, 5, 1, 0, 4)):
+        C = H * 128
+        want = sum(6 * r256(B * n * C * esz) + 3 * r256(B * C * 4) for n in (Nv, Nc)) + r256(4 * B)
+        assert L.mmdit_block_slot_bytes(ctypes.byref(_block_cfg(B, Nv, Nc, H, dt))) == want
+
+
+def test_block_config_validation(L):
+    f = L.mmdit_block_slot_bytes
+    assert f(None) == -1
+    c = _block_cfg(); c.D = 64
+    assert f(ctypes.byref(c)) == -4
+    c = _block_cfg(); c.dt = 5
+    assert f(ctypes.byref(c)) == -1
+    c = _block_cfg(Nv=31)
+    assert f(ctypes.byref(c)) == -2                       # Nv != T*H*W
+    c = _block_cfg(); c.grid.split[1] = 58
+    assert f(ctypes.byref(c)) == -2                       # split sum != D
+    c = _block_cfg(); c.softmax_scale = 0.0
+    assert f(ctypes.byref(c)) == -1
+    c = _block_cfg(); c.ln_eps = float("nan")
+    assert f(ctypes.byref(c)) == -1
+    c = _block_cfg(H=40)
+    assert f(ctypes.byref(c)) == -4                       # C = 5120 > 4096 bf16 per LN row
+    c = _block_cfg(); c.gk_ctx = None
+    assert f(ctypes.byref(c)) == -1
+    c = _block_cfg(Nc=0); c.gq_ctx = c.gk_ctx = None
+    assert f(ctypes.byref(c)) > 0                         # no cond stream: no cond scales
+    c = _block_cfg(); c.gq_vis = 18
+    assert f(ctypes.byref(c)) == -3
+
+
+def test_block_forward_host_validation(L):
+    """Every rejection happens before any CUDA call, so this runs without a GPU."""
+    f = L.mmdit_block_forward_host
+    c = _block_cfg()
+    slot = L.mmdit_block_slot_bytes(ctypes.byref(c))
+    steps = (_lib.BlockStep * 2)()
+    for s in steps:
+        for name in _lib.BLOCK_STEP_FIELDS:
+            setattr(s, name, 64)
+    ws = ctypes.c_void_p(256)
+    assert f(ctypes.byref(c), steps, 0, None, 0, None) == 0            # nothing to do
+    assert f(ctypes.byref(c), steps, -1, ws, slot, None) == -1
+    assert f(ctypes.byref(c), None, 2, ws, slot, None) == -1
+    assert f(ctypes.byref(c), steps, 2, None, slot, None) == -1
+    assert f(ctypes.byref(c), steps, 2, ctypes.c_void_p(272), slot, None) == -3  # 256-byte rule
+    assert f(ctypes.byref(c), steps, 2, ws, slot - 1, None) == -1      # less than one slot
+    steps[1].x_out_vis = None
+    assert f(ctypes.byref(c), steps, 2, ws, slot, None) == -1          # required output
+    steps[1].x_out_vis = 64
+    steps[0].gate_ctx = None
+    assert f(ctypes.byref(c), steps, 2, ws, slot, None) == -1          # cond input missing
+    c.D = 64
+    assert f(ctypes.byref(c), steps, 2, ws, slot, None) == -4
