@@ -292,8 +292,10 @@ def config_of(w: I.Workload, n: int):
 # ---------------------------------------------------------------------------- our arm
 
 def run_ours(args):
+    import ctypes
+
     import torch
-    from mmdit_joint_attention_b200 import api
+    from mmdit_joint_attention_b200 import _lib, api
 
     rank, world, local, group = dist_setup(args.gpus)
     if not torch.cuda.is_available():
@@ -329,6 +331,8 @@ def run_ours(args):
     host_out = {k: torch.empty(t[k].shape, dtype=t[k].dtype).pin_memory() for k in out_names}
 
     KERNELS = ["adaln_modulate", "qk_norm_rope", "joint_attention", "gated_residual"]
+    # split-tail workspace of the attention (21 MB, allocated once)
+    attn_ws = api.attention_workspace(dev)
 
     def step(ev=None):
         """One pass of the path; ``ev`` collects per-kernel event pairs."""
@@ -346,13 +350,19 @@ def run_ours(args):
         api.qk_norm_rope(t["q_ctx"], t["k_ctx"], t["gq_ctx"], t["gk_ctx"])
         mark(2)
         api.joint_attention(t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"],
-                            t["v_ctx"], t["ctx_len"], o_vis=t["o_vis"], o_ctx=t["o_ctx"])
+                            t["v_ctx"], t["ctx_len"], o_vis=t["o_vis"], o_ctx=t["o_ctx"],
+                            workspace=attn_ws)
         mark(3)
         api.gated_residual(t["x_vis"], t["o_vis"].view(B, Nv, C), t["gate_vis"])
         api.gated_residual(t["x_ctx"], t["o_ctx"].view(B, Nc, C), t["gate_ctx"])
         mark(4)
 
-    launches_per_step = 7
+    # 7 launches, plus the merge of the attention's split tail when it splits
+    plan = (ctypes.c_longlong * 4)()
+    _lib.check("mmdit_joint_attention_split_plan", _lib.lib().mmdit_joint_attention_split_plan(
+        B, Nv, Nc, H, torch.cuda.get_device_properties(dev).multi_processor_count,
+        attn_ws.numel(), plan))
+    launches_per_step = 7 + (1 if plan[1] >= 2 else 0)
 
     for _ in range(args.warmup):
         step()

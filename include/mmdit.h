@@ -243,6 +243,47 @@ MMDIT_API int mmdit_joint_attention_fwd(const void* q_vis, const void* k_vis, co
                                         float* lse, int B, int Nv, int Nc, int H, int D,
                                         float softmax_scale, mmdit_dtype dt, void* stream);
 
+/* Joint attention with a device workspace for the split tail (a scheduling
+ * choice of this library, not a step of the method): the same results as
+ * mmdit_joint_attention / mmdit_joint_attention_fwd up to the order of the
+ * floating-point sums [Vimoo §2.2 joint attention].
+ *
+ * The bf16 kernel runs one CTA per SM, one item (b, h, pair of 128-row query
+ * tiles) each, and every item costs the same.  The items beyond the last whole
+ * wave would run as a short wave on a few SMs; with a workspace, each of them
+ * is split over its keys into pieces that run side by side, and a second
+ * kernel merges the pieces' partial rows (rescaling them to a common maximum,
+ * as between key tiles).  Problems with fewer items than SMs split every item.
+ *   lse: DEVICE fp32 [B, H, Nv + Nc] as mmdit_joint_attention_fwd, or NULL
+ *   workspace: DEVICE memory, 256-byte aligned, of workspace_bytes bytes, or
+ *     NULL; MMDIT_ATTENTION_WORKSPACE_BYTES suffice for every problem.  The
+ *     tail is split only when the workspace holds the plan's partials; else
+ *     the call equals mmdit_joint_attention(_fwd).  Contents need no
+ *     initialisation; calls overlapping on the GPU need separate workspaces.
+ *   dt == MMDIT_F32 ignores the workspace.
+ *   everything else as mmdit_joint_attention.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+#define MMDIT_ATTENTION_SPLIT_MAX_PIECES 160
+#define MMDIT_ATTENTION_WORKSPACE_BYTES (MMDIT_ATTENTION_SPLIT_MAX_PIECES * 256LL * 130 * 4)
+MMDIT_API int mmdit_joint_attention_ws(const void* q_vis, const void* k_vis, const void* v_vis,
+                                       const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                       const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                                       float* lse, void* workspace, long long workspace_bytes,
+                                       int B, int Nv, int Nc, int H, int D, float softmax_scale,
+                                       mmdit_dtype dt, void* stream);
+
+/* The split-tail plan mmdit_joint_attention_ws follows for bf16 on a GPU of
+ * num_sms SMs with a workspace of workspace_bytes (host arithmetic, no CUDA
+ * call):
+ *   plan[0]  items split (the last ones of the launch), 0: no split
+ *   plan[1]  pieces per split item (0 when nothing is split)
+ *   plan[2]  key tiles of 128 keys per piece (the last may hold fewer)
+ *   plan[3]  CTAs of the attention launch
+ * A split launch is followed by one merging launch.
+ * Errors: MMDIT_ERR_ARG (negative size, num_sms < 1, plan NULL). */
+MMDIT_API int mmdit_joint_attention_split_plan(int B, int Nv, int Nc, int H, int num_sms,
+                                               long long workspace_bytes, long long* plan);
+
 /* Backward of the joint attention [the reverse-mode derivative of the joint
  * attention of Vimoo §2.2; Seaweed-7B, section 3.4]: for the upstream
  * gradients do_vis / do_ctx of o_vis / o_ctx, with P the softmax of the
@@ -395,12 +436,13 @@ MMDIT_API int mmdit_residual_modulate(const void* x, const void* branch, const f
  * [Vimoo §2.2, the dual-stream block]:
  *   y   = adaLN modulate of x                    (mmdit_adaln_modulate, both streams)
  *   q,k = QK-RMSNorm (+ 3D RoPE on the visual stream)   (mmdit_qk_norm_rope)
- *   o   = joint attention over both streams      (mmdit_joint_attention)
+ *   o   = joint attention over both streams      (mmdit_joint_attention_ws)
  *   x'  = x + gate * o                           (mmdit_gated_residual, both streams)
  * The projections of a full block (QKV, output, MLP) are outside this library:
  * q, k, v arrive as inputs and the attention output is the gated branch.  Each
  * step is the same computation, with the same kernels and results, as these
- * seven calls made one after the other on device buffers.
+ * seven calls made one after the other on device buffers (the attention with a
+ * workspace of MMDIT_ATTENTION_WORKSPACE_BYTES, which each slot holds).
  *
  * Unlike the rest of this header, the executor moves data between host and
  * device itself: it copies a step's inputs in, runs the kernels and copies the

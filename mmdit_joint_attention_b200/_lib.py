@@ -22,6 +22,9 @@ STATUS = {0: "MMDIT_OK", -1: "MMDIT_ERR_ARG", -2: "MMDIT_ERR_SHAPE", -3: "MMDIT_
 
 STATUS_CODES = {v: k for k, v in STATUS.items()}
 
+# MMDIT_ATTENTION_WORKSPACE_BYTES: 160 split pieces x 256 rows x (128 + 2) fp32
+ATTENTION_WORKSPACE_BYTES = 160 * 256 * 130 * 4
+
 
 class Grid(ctypes.Structure):
     """mmdit_grid: visual token grid (T, H, W) and RoPE parameters."""
@@ -111,6 +114,9 @@ def lib():
                                            ctypes.POINTER(Window), _i, _i, _vp]
         L.mmdit_joint_attention.argtypes = [_vp] * 9 + [_i] * 5 + [_f, _i, _vp]
         L.mmdit_joint_attention_fwd.argtypes = [_vp] * 10 + [_i] * 5 + [_f, _i, _vp]
+        L.mmdit_joint_attention_ws.argtypes = ([_vp] * 11 + [ctypes.c_longlong] + [_i] * 5 +
+                                               [_f, _i, _vp])
+        L.mmdit_joint_attention_split_plan.argtypes = [_i] * 5 + [ctypes.c_longlong, _vp]
         L.mmdit_joint_attention_bwd.argtypes = [_vp] * 19 + [_i] * 5 + [_f, _i, _vp]
         L.mmdit_joint_window_attention.argtypes = ([_vp] * 9 + [_i] * 5 +
                                                    [ctypes.POINTER(Grid), ctypes.POINTER(Window),
@@ -135,6 +141,7 @@ def lib():
                      "mmdit_quantize_int8", "mmdit_quantize_v_e4m3", "mmdit_joint_attention_q8",
                      "mmdit_window_permute", "mmdit_joint_attention",
                      "mmdit_joint_attention_fwd", "mmdit_joint_attention_bwd",
+                     "mmdit_joint_attention_ws", "mmdit_joint_attention_split_plan",
                      "mmdit_joint_window_attention", "mmdit_adaln_modulate",
                      "mmdit_gated_residual", "mmdit_residual_modulate", "mmdit_device_status",
                      "mmdit_block_forward_host"):

@@ -132,27 +132,55 @@ def qk_norm_rope_text(q: torch.Tensor, k: torch.Tensor, q_scale: torch.Tensor,
     return q_out, k_out
 
 
-def joint_attention(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
-                    softmax_scale: Optional[float] = None, o_vis=None, o_ctx=None,
-                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Non-causal attention over the concatenation [visual; cond] of both
-    streams, output split back into (o_vis, o_ctx)."""
+def attention_workspace(device=None) -> torch.Tensor:
+    """A device workspace for the split tail of joint_attention(_fwd):
+    MMDIT_ATTENTION_WORKSPACE_BYTES bytes, enough for every problem."""
+    return torch.empty(_lib.ATTENTION_WORKSPACE_BYTES, dtype=torch.uint8,
+                       device=device if device is not None else torch.cuda.current_device())
+
+
+def _attention_call(name, q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx, lse,
+                    workspace, softmax_scale, stream):
     dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx)
     B, Nv, H, D = q_vis.shape
     Nc = q_ctx.shape[1]
-    if o_vis is None:
-        o_vis = torch.empty_like(q_vis)
-    if o_ctx is None:
-        o_ctx = torch.empty_like(q_ctx)
     if ctx_len is not None and (ctx_len.dtype != torch.int32 or not ctx_len.is_cuda):
         raise TypeError("ctx_len must be an int32 CUDA tensor")
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
-    st = _lib.lib().mmdit_joint_attention(
-        _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
-        _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), B, Nv, Nc, H, D, softmax_scale, dt,
-        _stream(stream))
-    check("mmdit_joint_attention", st)
+    ptrs = [_ptr(t) for t in (q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx)]
+    if workspace is None:
+        if lse is None:
+            st = _lib.lib().mmdit_joint_attention(*ptrs, B, Nv, Nc, H, D, softmax_scale, dt,
+                                                  _stream(stream))
+        else:
+            name = "mmdit_joint_attention_fwd"
+            st = _lib.lib().mmdit_joint_attention_fwd(*ptrs, _ptr(lse), B, Nv, Nc, H, D,
+                                                      softmax_scale, dt, _stream(stream))
+    else:
+        if workspace.dtype != torch.uint8 or not workspace.is_cuda or not workspace.is_contiguous():
+            raise TypeError("workspace must be a contiguous uint8 CUDA tensor")
+        name = "mmdit_joint_attention_ws"
+        st = _lib.lib().mmdit_joint_attention_ws(*ptrs, _ptr(lse), _ptr(workspace),
+                                                 workspace.numel(), B, Nv, Nc, H, D,
+                                                 softmax_scale, dt, _stream(stream))
+    check(name, st)
+
+
+def joint_attention(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
+                    softmax_scale: Optional[float] = None, o_vis=None, o_ctx=None,
+                    stream=None, workspace: Optional[torch.Tensor] = None
+                    ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Non-causal attention over the concatenation [visual; cond] of both
+    streams, output split back into (o_vis, o_ctx).  With a ``workspace``
+    (``attention_workspace()``) the items past the last whole wave of CTAs are
+    split over their keys (mmdit_joint_attention_ws)."""
+    if o_vis is None:
+        o_vis = torch.empty_like(q_vis)
+    if o_ctx is None:
+        o_ctx = torch.empty_like(q_ctx)
+    _attention_call("mmdit_joint_attention", q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len,
+                    o_vis, o_ctx, None, workspace, softmax_scale, stream)
     return o_vis, o_ctx
 
 
@@ -204,10 +232,10 @@ def joint_attention_qnorm(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, q_scale_vis,
 
 def joint_attention_fwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
                         softmax_scale: Optional[float] = None, o_vis=None, o_ctx=None, lse=None,
-                        stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+                        stream=None, workspace: Optional[torch.Tensor] = None
+                        ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """joint_attention that also returns the row log-sum-exp lse [B, H, Nv + Nc]
     (fp32, natural log, +inf for rows without an output) for the backward."""
-    dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx)
     B, Nv, H, D = q_vis.shape
     Nc = q_ctx.shape[1]
     o_vis = torch.empty_like(q_vis) if o_vis is None else o_vis
@@ -215,15 +243,8 @@ def joint_attention_fwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
     if lse is None:
         lse = torch.empty((B, H, Nv + Nc), dtype=torch.float32, device=q_vis.device)
     _f32(lse)
-    if ctx_len is not None and (ctx_len.dtype != torch.int32 or not ctx_len.is_cuda):
-        raise TypeError("ctx_len must be an int32 CUDA tensor")
-    if softmax_scale is None:
-        softmax_scale = 1.0 / math.sqrt(D)
-    st = _lib.lib().mmdit_joint_attention_fwd(
-        _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
-        _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(lse), B, Nv, Nc, H, D, softmax_scale, dt,
-        _stream(stream))
-    check("mmdit_joint_attention_fwd", st)
+    _attention_call("mmdit_joint_attention_fwd", q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx,
+                    ctx_len, o_vis, o_ctx, lse, workspace, softmax_scale, stream)
     return o_vis, o_ctx, lse
 
 
@@ -461,14 +482,18 @@ def device_status(stream=None) -> int:
 
 
 def block_forward(t: dict, grid: Sequence[int], pos_scale=(1.0, 1.0, 1.0), eps: float = 1e-6,
-                  stream=None) -> dict:
+                  stream=None, workspace: Optional[torch.Tensor] = None) -> dict:
     """One pass of the whole path on device tensors ``t`` (keys as produced by
     ``inputs.make_inputs``): adaLN modulate of both streams (y_vis, y_ctx),
     QK-RMSNorm (+ RoPE on the visual stream) in place on q/k, joint attention
     (o_vis, o_ctx), and the gated residual x += gate * o in place, with the
     attention output standing in for the branch (the projections around
-    attention are not part of this path).  Returns the output tensors."""
+    attention are not part of this path).  The attention splits its tail
+    (``joint_attention``'s ``workspace``; one is allocated when none is given),
+    as the host-buffer executor does.  Returns the output tensors."""
     B, Nv, H, D = t["q_vis"].shape
+    if workspace is None:
+        workspace = attention_workspace(t["q_vis"].device)
     Nc = t["q_ctx"].shape[1]
     out = {}
     for s in ("vis", "ctx"):
@@ -480,7 +505,8 @@ def block_forward(t: dict, grid: Sequence[int], pos_scale=(1.0, 1.0, 1.0), eps: 
                  stream=stream)
     out["o_vis"], out["o_ctx"] = joint_attention(
         t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"], t["v_ctx"],
-        t.get("ctx_len"), o_vis=t.get("o_vis"), o_ctx=t.get("o_ctx"), stream=stream)
+        t.get("ctx_len"), o_vis=t.get("o_vis"), o_ctx=t.get("o_ctx"), stream=stream,
+        workspace=workspace)
     for s, n in (("vis", Nv), ("ctx", Nc)):
         out["x_" + s] = gated_residual(t["x_" + s], out["o_" + s].view(B, n, H * D),
                                        t["gate_" + s], stream=stream)

@@ -259,7 +259,8 @@ int joint_attention_impl(const void* q_vis, const void* k_vis, const void* v_vis
                          const void* q_ctx, const void* k_ctx, const void* v_ctx,
                          const int32_t* ctx_len, void* o_vis, void* o_ctx, float* lse, int B,
                          int Nv, int Nc, int H, int D, float softmax_scale, const WindowTable* win,
-                         mmdit_dtype dt, void* stream) {
+                         mmdit_dtype dt, void* stream, void* ws = nullptr,
+                         long long ws_bytes = 0) {
     if (!dtype_ok(dt) || B < 0 || Nv < 0 || Nc < 0 || H < 0) return MMDIT_ERR_ARG;
     if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MMDIT_ERR_ARG;
     if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
@@ -288,7 +289,7 @@ int joint_attention_impl(const void* q_vis, const void* k_vis, const void* v_vis
             softmax_scale, win, s), "joint_attention_f32");
     const int r = launch_joint_attention_bf16(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len,
                                               o_vis, o_ctx, lse, B, Nv, Nc, H, softmax_scale, win,
-                                              s);
+                                              s, nullptr, static_cast<float*>(ws), ws_bytes);
     if (r == 0) return MMDIT_OK;
     set_last_error("joint_attention_bf16", r);
     return MMDIT_ERR_CUDA;
@@ -425,6 +426,30 @@ int mmdit_joint_attention_fwd(const void* q_vis, const void* k_vis, const void* 
     if (!lse && (long long)B * H * (Nv + (long long)Nc) > 0) return MMDIT_ERR_ARG;
     return joint_attention_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx,
                                 lse, B, Nv, Nc, H, D, softmax_scale, nullptr, dt, stream);
+}
+
+int mmdit_joint_attention_ws(const void* q_vis, const void* k_vis, const void* v_vis,
+                             const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                             const int32_t* ctx_len, void* o_vis, void* o_ctx, float* lse,
+                             void* workspace, long long workspace_bytes, int B, int Nv, int Nc,
+                             int H, int D, float softmax_scale, mmdit_dtype dt, void* stream) {
+    if (workspace_bytes < 0) return MMDIT_ERR_ARG;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MMDIT_ERR_ALIGN;
+    return joint_attention_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx,
+                                lse, B, Nv, Nc, H, D, softmax_scale, nullptr, dt, stream,
+                                workspace, workspace ? workspace_bytes : 0);
+}
+
+int mmdit_joint_attention_split_plan(int B, int Nv, int Nc, int H, int num_sms,
+                                     long long workspace_bytes, long long* plan) {
+    if (B < 0 || Nv < 0 || Nc < 0 || H < 0 || num_sms < 1 || workspace_bytes < 0 || !plan)
+        return MMDIT_ERR_ARG;
+    const SplitPlan sp = split_plan(B, Nv, Nc, H, num_sms, workspace_bytes);
+    plan[0] = sp.tail;
+    plan[1] = sp.parts;
+    plan[2] = sp.per;
+    plan[3] = sp.ctas;
+    return MMDIT_OK;
 }
 
 int mmdit_joint_attention_bwd(const void* q_vis, const void* k_vis, const void* v_vis,

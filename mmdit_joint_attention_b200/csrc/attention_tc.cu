@@ -46,6 +46,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -83,6 +84,10 @@ constexpr int kRegsProducer = 72;
 constexpr int kRegsSoftmax = 216;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsProducer == kThreads * kRegsLaunch,
               "register split must add up to the launch allocation");
+// Split tail: at most kMaxSplitPieces pieces (the workspace bound of the
+// public header), each at least kMinSplitTiles key tiles long.
+constexpr int kMaxSplitPieces = MMDIT_ATTENTION_SPLIT_MAX_PIECES;
+constexpr int kMinSplitTiles = 2;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // default: 2 s per pipeline wait
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s per drain wait after an abort
 
@@ -130,6 +135,15 @@ struct Params {
     int tab_off[3], tab_stride[3], tab_entries;   // table layout; 0 entries: no table
     double pos_scale[3];
     double freq[64];           // frequency of pair j of axis a at off[a] / 2 + j
+    // split tail (full mode only; split_parts == 0: off).  The grid is then
+    // one-dimensional: items (b, h, query-tile pair) in the order of the
+    // three-dimensional grid, the first split_first of them whole, each later
+    // one as split_parts pieces of split_per key tiles.  A piece writes its
+    // rows' unnormalised O and (m, l) to part_o / part_ml at index
+    // piece * 256 + row; attn_combine_kernel then finishes those rows.
+    int split_first, split_parts, split_per, pairs;
+    float* part_o;             // [pieces][256][128]
+    float2* part_ml;           // [pieces][256]: running max (log2 units), sum
 };
 
 
@@ -142,6 +156,8 @@ struct Work {
     bool has1;
     int vis_start, vis_len;
     int wi;
+    int kv_lo, kv_hi;   // key tiles [kv_lo, kv_hi) of the joint sequence (valid ones only)
+    int piece;          // split-tail piece index, or -1 (the CTA stores finished rows)
 };
 
 struct Bars {
@@ -176,10 +192,29 @@ __device__ __forceinline__ Work decode_work(const Params& p) {
     w.vis_start = 0;
     w.vis_len = p.N[0];
     w.wi = -1;
+    w.kv_lo = 0;
+    w.kv_hi = 1 << 30;
+    w.piece = -1;
     if (!p.windowed) {
+        int pair = blockIdx.x;
         w.h = blockIdx.y;
         w.b = blockIdx.z;
-        const int t0 = 2 * blockIdx.x;
+        if (p.split_parts > 0) {
+            int item = blockIdx.x;
+            if (item >= p.split_first) {
+                const int q = item - p.split_first;
+                const int t = q / p.split_parts;
+                w.piece = q;
+                w.kv_lo = (q - t * p.split_parts) * p.split_per;
+                w.kv_hi = w.kv_lo + p.split_per;
+                item = p.split_first + t;
+            }
+            pair = item % p.pairs;
+            const int bh = item / p.pairs;
+            w.h = bh % p.H;
+            w.b = bh / p.H;
+        }
+        const int t0 = 2 * pair;
         w.has1 = t0 + 1 < p.q_tiles;
         tile_of(p, t0, w.seg0, w.row0);
         w.seg1 = w.seg0;
@@ -257,17 +292,18 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t tile, int s) {
     return smem_desc_sw128(tile + s * 2048, kHalfBytes, 1024);
 }
 
-// Streams the n_kv 128-key tiles of one operand (K or V) of the joint key
-// sequence (kv_vis visual tiles from row vis_start on, then conditioning
-// tiles) through its ring of kStages shared-memory slots.  On an abort, waits (bounded) for the copies
-// it issued before returning.
+// Streams key tiles [j_lo, j_lo + n_it) of one operand (K or V) of the joint
+// key sequence (kv_vis visual tiles from row vis_start on, then conditioning
+// tiles) through its ring of kStages shared-memory slots.  On an abort, waits
+// (bounded) for the copies it issued before returning.
 __device__ __forceinline__ void stream_tiles(const CUtensorMap* tm, uint8_t* ring, uint64_t* full,
-                                             uint64_t* empty, int n_kv, int kv_vis, int vis_start,
-                                             int h, int b, Bars* bars) {
+                                             uint64_t* empty, int j_lo, int n_it, int kv_vis,
+                                             int vis_start, int h, int b, Bars* bars) {
     int issued = 0;
-    for (int j = 0; j < n_kv; ++j) {
-        const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
+    for (int it = 0; it < n_it; ++it) {
+        const int j = j_lo + it;
+        const int st = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
         const int seg = j < kv_vis ? 0 : 1;
         const int row = seg == 0 ? vis_start + j * kBlockN : (j - kv_vis) * kBlockN;
         if (!wait(&empty[st], ph ^ 1, bars)) break;
@@ -479,7 +515,10 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
     }
     const int kv_vis = (vwk->vis_len + kBlockN - 1) / kBlockN;
     const int n_kv = kv_vis + (L + kBlockN - 1) / kBlockN;
-    if (warp == kWarpLoad && n_kv > 0) {
+    // this CTA's key tiles: all of them, or a split-tail piece's range
+    const int j_lo = vwk->kv_lo < n_kv ? vwk->kv_lo : n_kv;
+    const int n_it = (vwk->kv_hi < n_kv ? vwk->kv_hi : n_kv) - j_lo;
+    if (warp == kWarpLoad && n_it > 0) {
         tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
     }
@@ -491,7 +530,14 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
     const uint32_t sK = smem_u32(smem + Smem::k_off);
     const uint32_t sV = smem_u32(smem + Smem::v_off);
 
-    if (n_kv == 0) {
+    if (n_it == 0 && vwk->piece >= 0) {
+        // a split-tail piece whose key range holds no valid key: an empty
+        // partial (the combine skips it)
+        for (int r = threadIdx.x; r < 2 * kBlockM; r += kThreads)
+            p.part_ml[(size_t)vwk->piece * (2 * kBlockM) + r] = make_float2(-INFINITY, 0.f);
+        return;
+    }
+    if (n_it == 0) {
         // no valid key at all: every output row of this CTA is zero
         for (int tt = 0; tt < 2; ++tt) {
             if (tt == 1 && !has1) break;
@@ -534,8 +580,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                 tma_load_4d(smem + Smem::q_off + kTileBytes + kHalfBytes, &p.tm_q[s1], &bars->q_full,
                             64, h, r1, b);
             }
-            stream_tiles(p.tm_k, smem + Smem::k_off, bars->k_full, bars->k_empty, n_kv, kv_vis,
-                         vwk->vis_start, h, b, bars);
+            stream_tiles(p.tm_k, smem + Smem::k_off, bars->k_full, bars->k_empty, j_lo, n_it,
+                         kv_vis, vwk->vis_start, h, b, bars);
             if (bars->abort) mbar_wait_bounded(&bars->q_full, 0, nullptr, kDrainLimitNs);
         }
     } else if (warp == kWarpLoadV) {
@@ -543,8 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         if (lane == 0) {
             for (int seg = 0; seg < 2; ++seg)
                 if (p.N[seg] > 0) tma_prefetch_desc(&p.tm_v[seg]);
-            stream_tiles(p.tm_v, smem + Smem::v_off, bars->v_full, bars->v_empty, n_kv, kv_vis,
-                         vwk->vis_start, h, b, bars);
+            stream_tiles(p.tm_v, smem + Smem::v_off, bars->v_full, bars->v_empty, j_lo, n_it,
+                         kv_vis, vwk->vis_start, h, b, bars);
         }
     } else if (warp == kWarpMma && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
@@ -593,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
             }
             return true;
         };
-        for (int j = 0; ok && j < n_kv; ++j) {
+        for (int j = 0; ok && j < n_it; ++j) {
             const int st = j % kStages;
             const uint32_t ph = (j / kStages) & 1;
             const int pst = (j + kStages - 1) % kStages;
@@ -611,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
             mma_commit(&bars->k_empty[st]);
         }
         if (ok) {
-            const int j = n_kv;
+            const int j = n_it;
             const int pst = (j - 1) % kStages;
             const uint32_t pph = ((j - 1) / kStages) & 1;
             ok = wait(&bars->v_full[pst], pph, bars);
@@ -640,13 +686,15 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
             float m_run = -INFINITY, l_run = 0.f;
             bool ok = true;
-            for (int j = 0; j < n_kv; ++j) {
-                if (!(ok = wait_warp(&bars->s_full[i], j & 1, bars))) break;
+            for (int it = 0; it < n_it; ++it) {
+                if (!(ok = wait_warp(&bars->s_full[i], it & 1, bars))) break;
                 tc_fence_after();
                 uint32_t r[4][32];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
                 tmem_wait_ld();
+                // key tile of this iteration (j_lo equals kv_lo whenever the loop runs)
+                const int j = it + vwk->kv_lo;
                 const int valid =
                     j < kv_vis ? vwk->vis_len - j * kBlockN : L - (j - kv_vis) * kBlockN;
                 float sv[128];
@@ -674,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                 // by more than 8 (log2 units); O (which holds PV up to the
                 // previous tile: S(j) ready implies it completed) is rescaled
                 // before any half of this tile's P is released to the MMA.
-                if (j == 0) {
+                if (it == 0) {
                     m_run = m_tile;
                 } else if (__any_sync(0xffffffffu, m_tile > m_run + 8.0f)) {
                     const float m_new = fmaxf(m_run, m_tile);
@@ -698,44 +746,65 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                 }
                 l_run += sum;
             }
-            // epilogue: O / l  ->  bf16 row of the owning stream
+            // epilogue: O / l  ->  bf16 row of the owning stream (or, for a
+            // split-tail piece, the partial row for the combine)
             if (ok) ok = wait_warp(&bars->o_done[i], 0, bars);
             tc_fence_after();
-            const int s = i ? vwk->seg1 : vwk->seg0;
-            const int row = (i ? vwk->row1 : vwk->row0) + quarter * 32 + lane;
-            const int orow = out_row(p, s, row, vwk->wi, vwk->vis_start, vwk->vis_len);
-            const bool store = orow >= 0;
-            const bool zero = !ok || (s == 1 && row >= L);
-            const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
-            if (p.lse && store) {
-                // natural-log row log-sum-exp of the scaled scores; m_run and
-                // the exponents are in log2 units
-                const int jrow = s == 0 ? orow : p.N[0] + row;
-                p.lse[((size_t)vwk->b * p.H + vwk->h) * (size_t)(p.N[0] + p.N[1]) + jrow] =
-                    (zero || !(l_run > 0.f)) ? INFINITY
-                                             : (m_run + log2f(l_run)) * 0.6931471805599453f;
-            }
-            uint4* dst = reinterpret_cast<uint4*>(
-                p.out[s] +
-                ((size_t)((size_t)vwk->b * p.N[s] + (store ? orow : 0)) * p.H + vwk->h) * kHeadDim);
+            if (vwk->piece >= 0) {
+                // split-tail piece: this row's unnormalised O and (m, l) for
+                // the combine
+                const size_t prow = (size_t)vwk->piece * (2 * kBlockM) + i * kBlockM +
+                                    quarter * 32 + lane;
+                float4* dst = reinterpret_cast<float4*>(p.part_o + prow * kHeadDim);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tO + 32 * c, o);
-                tmem_wait_ld();
-                if (store) {
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + 32 * c, o);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint4 w;
-                        float f[8];
+                    for (int v = 0; v < 8; ++v)
+                        dst[8 * c + v] = make_float4(
+                            __uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                            __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+                }
+                p.part_ml[prow] = ok ? make_float2(m_run, l_run) : make_float2(-INFINITY, 0.f);
+            } else {
+                const int s = i ? vwk->seg1 : vwk->seg0;
+                const int row = (i ? vwk->row1 : vwk->row0) + quarter * 32 + lane;
+                const int orow = out_row(p, s, row, vwk->wi, vwk->vis_start, vwk->vis_len);
+                const bool store = orow >= 0;
+                const bool zero = !ok || (s == 1 && row >= L);
+                const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
+                if (p.lse && store) {
+                    // natural-log row log-sum-exp of the scaled scores; m_run and
+                    // the exponents are in log2 units
+                    const int jrow = s == 0 ? orow : p.N[0] + row;
+                    p.lse[((size_t)vwk->b * p.H + vwk->h) * (size_t)(p.N[0] + p.N[1]) + jrow] =
+                        (zero || !(l_run > 0.f)) ? INFINITY
+                                                 : (m_run + log2f(l_run)) * 0.6931471805599453f;
+                }
+                uint4* dst = reinterpret_cast<uint4*>(
+                    p.out[s] + ((size_t)((size_t)vwk->b * p.N[s] + (store ? orow : 0)) * p.H +
+                                vwk->h) * kHeadDim);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            f[e] = zero ? 0.f : __uint_as_float(o[8 * v + e]) * inv;
-                        w.x = pack_bf16x2(f[0], f[1]);
-                        w.y = pack_bf16x2(f[2], f[3]);
-                        w.z = pack_bf16x2(f[4], f[5]);
-                        w.w = pack_bf16x2(f[6], f[7]);
-                        dst[4 * c + v] = w;
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + 32 * c, o);
+                    tmem_wait_ld();
+                    if (store) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 w;
+                            float f[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                f[e] = zero ? 0.f : __uint_as_float(o[8 * v + e]) * inv;
+                            w.x = pack_bf16x2(f[0], f[1]);
+                            w.y = pack_bf16x2(f[2], f[3]);
+                            w.z = pack_bf16x2(f[4], f[5]);
+                            w.w = pack_bf16x2(f[6], f[7]);
+                            dst[4 * c + v] = w;
+                        }
                     }
                 }
             }
@@ -748,6 +817,64 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+// Finishes the rows of the split-tail items.  Piece p of a row holds
+// O_p = sum over its keys of 2^(x - m_p) v and l_p = sum of the same weights
+// (x: scaled score in log2 units, m_p the piece's running maximum); the row is
+//   M = max_p m_p,  l = sum_p 2^(m_p - M) l_p,  O = sum_p 2^(m_p - M) O_p / l,
+// the rescaling the main loop applies between key tiles.  Pieces without a
+// valid key (m_p = -inf) drop out.  One warp per row, four head dims a lane.
+__global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant__ Params p,
+                                                           int tail_items) {
+    const int row_id = blockIdx.x * 8 + (threadIdx.x >> 5);   // tail item * 256 + row
+    const int lane = threadIdx.x & 31;
+    const int t = row_id / (2 * kBlockM);
+    const int r = row_id - t * (2 * kBlockM);
+    if (t >= tail_items) return;
+    const int item = p.split_first + t;
+    const int pair = item % p.pairs;
+    const int bh = item / p.pairs;
+    const int h = bh % p.H, b = bh / p.H;
+    const int tt = 2 * pair + r / kBlockM;
+    if (tt >= p.q_tiles) return;          // the last pair has one tile
+    int s, row0;
+    tile_of(p, tt, s, row0);
+    const int row = row0 + r % kBlockM;
+    if (row >= p.N[s]) return;            // past the end of the stream: not stored
+    int L = p.N[1];
+    if (p.ctx_len) {
+        L = p.ctx_len[b];
+        L = L < 0 ? 0 : (L > p.N[1] ? p.N[1] : L);
+    }
+    const bool zero = s == 1 && row >= L;
+    const size_t first = (size_t)t * p.split_parts * (2 * kBlockM) + r;   // piece 0's row
+    float M = -INFINITY;
+    for (int q = 0; q < p.split_parts; ++q)
+        M = fmaxf(M, p.part_ml[first + (size_t)q * (2 * kBlockM)].x);
+    float l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!zero && M > -INFINITY) {
+        for (int q = 0; q < p.split_parts; ++q) {
+            const size_t pr = first + (size_t)q * (2 * kBlockM);
+            const float2 ml = p.part_ml[pr];
+            if (!(ml.x > -INFINITY)) continue;
+            const float w = exp2f(ml.x - M);
+            l += w * ml.y;
+            const float4 o = reinterpret_cast<const float4*>(p.part_o + pr * kHeadDim)[lane];
+            acc.x += w * o.x;
+            acc.y += w * o.y;
+            acc.z += w * o.z;
+            acc.w += w * o.w;
+        }
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    reinterpret_cast<uint2*>(p.out[s] + ((size_t)((size_t)b * p.N[s] + row) * p.H + h) *
+                                            kHeadDim)[lane] =
+        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+    if (p.lse && lane == 0)
+        p.lse[((size_t)b * p.H + h) * (size_t)(p.N[0] + p.N[1]) + (s ? p.N[0] + row : row)] =
+            (zero || !(l > 0.f)) ? INFINITY : (M + log2f(l)) * 0.6931471805599453f;
 }
 
 }  // namespace attn
@@ -764,11 +891,35 @@ uint64_t wait_timeout_ns() {
     return v ? v : attn::kWaitLimitNs;
 }
 
+SplitPlan split_plan(int B, int Nv, int Nc, int H, int num_sms, long long ws_bytes) {
+    using namespace attn;
+    SplitPlan sp{};
+    const long long q_tiles = (Nv + kBlockM - 1) / kBlockM + (Nc + kBlockM - 1) / kBlockM;
+    const long long total = (long long)B * H * ((q_tiles + 1) / 2);
+    const int kv_max = (int)((Nv + (long long)kBlockN - 1) / kBlockN +
+                             (Nc + (long long)kBlockN - 1) / kBlockN);
+    sp.ctas = total;
+    if (num_sms < 1 || total == 0 || total >= (1LL << 31)) return sp;
+    const int t = (int)(total % num_sms);
+    if (t == 0) return sp;
+    int parts = std::min(num_sms / t, std::min(kv_max / kMinSplitTiles, kMaxSplitPieces / t));
+    if (parts < 2) return sp;
+    const int per = (kv_max + parts - 1) / parts;
+    parts = (kv_max + per - 1) / per;
+    if ((long long)t * parts * 2 * kBlockM * (kHeadDim + 2) * 4 > ws_bytes) return sp;
+    sp.tail = t;
+    sp.parts = parts;
+    sp.per = per;
+    sp.first = (int)(total - t);
+    sp.ctas = total - t + (long long)t * parts;
+    return sp;
+}
+
 int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, const void* qc,
                                 const void* kc, const void* vc, const int32_t* ctx_len, void* ov,
                                 void* oc, float* lse, int B, int Nv, int Nc, int H,
                                 float softmax_scale, const WindowTable* win, cudaStream_t s,
-                                const QNormArgs* qn) {
+                                const QNormArgs* qn, float* split_ws, long long split_ws_bytes) {
     using namespace attn;
     if (!encode_fn()) return -1;
     const int q_tiles = (Nv + kBlockM - 1) / kBlockM + (Nc + kBlockM - 1) / kBlockM;
@@ -851,8 +1002,11 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return (int)e;
     static bool attr_set[64] = {false};
+    static int sm_count[64] = {0};
     if (dev < 0 || dev >= 64) return (int)cudaErrorInvalidDevice;
     if (!attr_set[dev]) {
+        e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return (int)e;
         // The register split inside the kernel assumes the launch allocation
         // is exactly kRegsLaunch per thread; refuse to launch otherwise (a
         // smaller allocation would leave the increase waiting for ever).
@@ -865,8 +1019,32 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
         if (e != cudaSuccess) return (int)e;
         attr_set[dev] = true;
     }
-    const dim3 grid = win ? dim3((unsigned)items, 1, 1) : dim3((q_tiles + 1) / 2, H, B);
+    dim3 grid = win ? dim3((unsigned)items, 1, 1) : dim3((q_tiles + 1) / 2, H, B);
+    // Split tail.  One CTA runs per SM, and every item of a full launch costs
+    // the same, so the items beyond the last whole wave (total mod #SMs) would
+    // run as a wave of their own on a few SMs.  With a workspace, each of them
+    // is split over its key tiles into as many pieces as fill the SMs (at
+    // least kMinSplitTiles tiles a piece, kMaxSplitPieces pieces in all), and
+    // attn_combine_kernel merges the pieces.
+    int tail = 0;
+    if (!win && split_ws) {
+        SplitPlan sp = split_plan(B, Nv, Nc, H, sm_count[dev], split_ws_bytes);
+        if (sp.parts >= 2) {
+            tail = sp.tail;
+            p.split_first = sp.first;
+            p.split_parts = sp.parts;
+            p.split_per = sp.per;
+            p.pairs = (q_tiles + 1) / 2;
+            p.part_o = split_ws;
+            const size_t o_floats = (size_t)sp.tail * sp.parts * 2 * kBlockM * kHeadDim;
+            p.part_ml = reinterpret_cast<float2*>(split_ws + o_floats);
+            grid = dim3((unsigned)sp.ctas, 1, 1);
+        }
+    }
     joint_attn_bf16_kernel<<<grid, kThreads, smem, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || tail == 0) return (int)e;
+    attn_combine_kernel<<<tail * 2 * kBlockM / 8, 256, 0, s>>>(p, tail);
     return (int)cudaGetLastError();
 }
 

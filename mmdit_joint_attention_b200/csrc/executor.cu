@@ -4,13 +4,14 @@
 //
 // A step is the seven launches of the device entry points, in this order:
 // adaLN modulate of both streams, QK-RMSNorm + RoPE of both streams (in
-// place), the joint attention, and the gated residual of both streams (in
-// place on x).  Every buffer a step touches on the device lives in its slot of
+// place), the joint attention (with its split-tail workspace), and the gated
+// residual of both streams (in place on x).  Every buffer a step touches on the device lives in its slot of
 // the workspace:
 //
 //   per stream s in (vis, ctx), N_s tokens:  q, k, v, x, y, o   [B, N_s, C] dt
 //   per stream:                              shift, scale, gate [B, C] fp32
 //   ctx_len                                  [B] int32
+//   attention workspace                      MMDIT_ATTENTION_WORKSPACE_BYTES
 //
 // each region starting on a 256-byte boundary.
 //
@@ -46,6 +47,7 @@ struct SlotLayout {
     long long q[2], k[2], v[2], x[2], y[2], o[2];
     long long shift[2], scale[2], gate[2];
     long long ctx_len;
+    long long attn_ws;      // split-tail workspace of the attention
     long long bytes;        // slot size (a multiple of 256)
     long long tok_bytes[2]; // bytes of one [B, N_s, C] tensor
     long long vec_bytes;    // bytes of one [B, C] fp32 vector
@@ -101,6 +103,8 @@ int check_config(const mmdit_block_config* c, SlotLayout& L) {
     }
     L.ctx_len = off;
     off += round256((long long)c->B * 4);
+    L.attn_ws = off;
+    off += round256(MMDIT_ATTENTION_WORKSPACE_BYTES);
     L.bytes = off;
     return MMDIT_OK;
 }
@@ -250,12 +254,12 @@ extern "C" int mmdit_block_forward_host(const mmdit_block_config* cfg,
                                         c.gq_ctx, c.gk_ctx, B, N[1], H, D, nullptr, c.norm_eps,
                                         c.dt, cs);
         if (status == MMDIT_OK)
-            status = mmdit_joint_attention(
+            status = mmdit_joint_attention_ws(
                 dev(L.q[0]), dev(L.k[0]), dev(L.v[0]), has_ctx ? dev(L.q[1]) : nullptr,
                 has_ctx ? dev(L.k[1]) : nullptr, has_ctx ? dev(L.v[1]) : nullptr,
                 st.ctx_len ? reinterpret_cast<const int32_t*>(dev(L.ctx_len)) : nullptr,
-                dev(L.o[0]), has_ctx ? dev(L.o[1]) : nullptr, B, N[0], N[1], H, D,
-                c.softmax_scale, c.dt, cs);
+                dev(L.o[0]), has_ctx ? dev(L.o[1]) : nullptr, nullptr, dev(L.attn_ws),
+                MMDIT_ATTENTION_WORKSPACE_BYTES, B, N[0], N[1], H, D, c.softmax_scale, c.dt, cs);
         if (status != MMDIT_OK) break;
         if ((e = cudaEventRecord(h.o_done[k], h.cmp)) != cudaSuccess) break;
         for (int s = 0; s < 2 && status == MMDIT_OK; ++s)

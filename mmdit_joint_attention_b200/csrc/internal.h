@@ -75,15 +75,27 @@ struct QNormArgs {
     float eps;
 };
 
+// Split-tail plan of a full bf16 launch on num_sms SMs with a workspace of
+// ws_bytes: `tail` items (the last ones) in `parts` pieces of `per` key tiles
+// each, the first `first` items whole, `ctas` CTAs in all (the plain
+// launch's count when parts == 0: no split).  Host arithmetic only.
+struct SplitPlan {
+    int tail, parts, per, first;
+    long long ctas;
+};
+SplitPlan split_plan(int B, int Nv, int Nc, int H, int num_sms, long long ws_bytes);
+
 // lse (null: not written): [B, H, Nv + Nc] natural-log row log-sum-exp of
 // the scaled scores, +infinity for rows without an output.  qn (null: q is
-// already normalised).
+// already normalised).  split_ws (null: off; full mode only): workspace of
+// split_ws_bytes for the split tail, used when the plan's partials fit.
 int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv,
                                 const void* qc, const void* kc, const void* vc,
                                 const int32_t* ctx_len, void* ov, void* oc, float* lse, int B,
                                 int Nv, int Nc, int H, float softmax_scale,
                                 const WindowTable* win, cudaStream_t s,
-                                const QNormArgs* qn = nullptr);
+                                const QNormArgs* qn = nullptr, float* split_ws = nullptr,
+                                long long split_ws_bytes = 0);
 
 cudaError_t launch_joint_attention_f32(const float* qv, const float* kv, const float* vv,
                                        const float* qc, const float* kc, const float* vc,

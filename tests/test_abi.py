@@ -190,11 +190,13 @@ def _block_cfg(B=1, Nv=32, Nc=8, H=2, dt=1):
 
 def test_block_slot_bytes_layout(L):
     """A slot holds q, k, v, x, y, o of both streams, the three [B, C] fp32
-    vectors of both streams and ctx_len, each region rounded up to 256 bytes."""
+    vectors of both streams, ctx_len and the attention's split-tail workspace,
+    each region rounded up to 256 bytes."""
     r256 = lambda n: (n + 255) // 256 * 256
     for B, Nv, Nc, H, dt, esz in ((1, 32, 8, 2, 1, 2), (3, 32, 0, 4, 1, 2), (2, 32, 5, 1, 0, 4)):
         C = H * 128
         want = sum(6 * r256(B * n * C * esz) + 3 * r256(B * C * 4) for n in (Nv, Nc)) + r256(4 * B)
+        want += r256(_lib.ATTENTION_WORKSPACE_BYTES)
         assert L.mmdit_block_slot_bytes(ctypes.byref(_block_cfg(B, Nv, Nc, H, dt))) == want
 
 
@@ -246,3 +248,67 @@ def test_block_forward_host_validation(L):
     assert f(ctypes.byref(c), steps, 2, ws, slot, None) == -1          # cond input missing
     c.D = 64
     assert f(ctypes.byref(c), steps, 2, ws, slot, None) == -4
+
+
+def test_attention_workspace_constant_matches_header():
+    import re
+    text = open(_lib.HEADER).read()
+    pieces = int(re.search(r"#define MMDIT_ATTENTION_SPLIT_MAX_PIECES (\d+)", text).group(1))
+    assert re.search(r"#define MMDIT_ATTENTION_WORKSPACE_BYTES \(MMDIT_ATTENTION_SPLIT_MAX_PIECES "
+                     r"\* 256LL \* 130 \* 4\)", text)
+    assert _lib.ATTENTION_WORKSPACE_BYTES == pieces * 256 * 130 * 4
+
+
+def test_attention_ws_validation(L):
+    f = L.mmdit_joint_attention_ws
+    args = lambda ws, n: (P, P, P, P, P, P, None, P, P, None, ws, n, 1, 8, 8, 2, 128, 0.1, 1, None)
+    assert f(*args(ctypes.c_void_p(272), 1 << 20)) == -3          # workspace not 256-aligned
+    assert f(*args(ctypes.c_void_p(256), -1)) == -1
+    a = list(args(None, 0)); a[16] = 64                              # D != 128
+    assert f(*a) == -4
+    a = list(args(None, 0)); a[13] = -1                              # Nv < 0
+    assert f(*a) == -1
+    a = list(args(None, 0)); a[12] = 0                               # B = 0: nothing to do
+    assert f(*a) == 0
+
+
+def _plan_rule(B, Nv, Nc, H, nsm, ws):
+    """The split-tail rule restated: the items past the last whole wave
+    (total mod nsm) are split into as many pieces as fill the SMs, at least 2
+    key tiles a piece and 160 pieces in all; pieces then get equal tile counts."""
+    tiles = -(-Nv // 128) + -(-Nc // 128)
+    total = B * H * ((tiles + 1) // 2)
+    t = total % nsm
+    parts = min(nsm // t, tiles // 2, 160 // t) if t else 0
+    if parts < 2:
+        return [0, 0, 0, total]
+    per = -(-tiles // parts)
+    parts = -(-tiles // per)
+    if t * parts * 256 * 130 * 4 > ws:
+        return [0, 0, 0, total]
+    return [t, parts, per, total - t + t * parts]
+
+
+def test_split_plan(L):
+    plan = (ctypes.c_longlong * 4)()
+    f = L.mmdit_joint_attention_split_plan
+    ws = _lib.ATTENTION_WORKSPACE_BYTES
+    # 480p (32,760 + 512 tokens, 24 heads): 3,120 items = 21 waves of 148 + 12,
+    # the 12 split into 12 pieces of 22 key tiles
+    assert f(1, 32760, 512, 24, 148, ws, plan) == 0
+    assert list(plan) == [12, 12, 22, 3108 + 144]
+    assert f(1, 32760, 512, 24, 148, 0, plan) == 0 and list(plan) == [0, 0, 0, 3120]
+    for B, Nv, Nc, H, nsm in [(b, nv, nc, h, n) for b in (1, 2, 3) for h in (1, 2, 24, 40)
+                              for nv in (0, 1, 128, 305, 1024, 32760) for nc in (0, 77, 512)
+                              for n in (1, 7, 148)]:
+        assert f(B, Nv, Nc, H, nsm, ws, plan) == 0
+        got = list(plan)
+        assert got == _plan_rule(B, Nv, Nc, H, nsm, ws), (B, Nv, Nc, H, nsm, got)
+        t, parts, per, ctas = got
+        if parts:
+            tiles = -(-Nv // 128) + -(-Nc // 128)
+            assert parts * per >= tiles > (parts - 1) * per     # every tile in one piece
+            assert t * parts <= min(nsm, 160)
+    assert f(-1, 8, 8, 2, 148, ws, plan) == -1
+    assert f(1, 8, 8, 2, 0, ws, plan) == -1
+    assert f(1, 8, 8, 2, 148, ws, None) == -1
