@@ -79,6 +79,16 @@ def recorded_traffic():
     return float(m.group(1))
 
 
+# softmax work per (query, key) score: scale, max, subtract, exp, sum
+SOFTMAX_FLOPS_PER_SCORE = 5
+
+
+def attention_scores(w) -> int:
+    """(query, key) scores of the joint attention over valid tokens: one
+    exponential each."""
+    return w.H * sum((w.Nv + L) ** 2 for L in w.ctx_lengths())
+
+
 def window_sizes(grid, parts):
     """Token counts of the 3D windows (parts windows per axis, the first
     extent % parts of an axis one position longer)."""
@@ -547,12 +557,14 @@ def run_ours(args):
     attn_tflops = flops / (kern_ms["joint_attention"] * 1e-3) / 1e12
     bytes_ = workload_bytes(w)
     hbm = float(pk["hbm_gbs"])
+    scores = attention_scores(w)
     kernels = {"joint_attention": {
         "ms": kern_ms["joint_attention"], "TFLOP/s": attn_tflops,
         "frac_bf16_burst": attn_tflops / float(pk["bf16_tflops"]),
         "frac_bf16_sustained": attn_tflops / float(pk["bf16_tflops_sustained"]),
-        "exp_per_s": H * sum((Nv + L) ** 2 for L in w.ctx_lengths()) /
-                     (kern_ms["joint_attention"] * 1e-3)}}
+        "exp_per_s": scores / (kern_ms["joint_attention"] * 1e-3),
+        "TFLOP/s_incl_softmax": (flops + SOFTMAX_FLOPS_PER_SCORE * scores) /
+                                (kern_ms["joint_attention"] * 1e-3) / 1e12}}
     for name in ("qk_norm_rope", "adaln_modulate", "gated_residual"):
         gbs = bytes_[name] / (kern_ms[name] * 1e-3) / 1e9
         kernels[name] = {"ms": kern_ms[name], "GB/s": gbs, "frac_hbm": gbs / hbm,

@@ -31,3 +31,13 @@ def test_full_attention_flops_are_the_one_window_case():
     for name in ("block", "ragged", "480p"):
         w = I.WORKLOADS[name]
         assert bench.window_attention_flops(w, (1, 1, 1)) == w.attention_flops()
+
+
+def test_scores_are_the_attention_flops_over_4d():
+    """One exponential per valid (query, key) score: 4 * D FLOPs of the two
+    products per score, so the count is the FLOP count / (4 D); 480p holds
+    2.66e10 of them (24 heads x 33,272^2)."""
+    for name in ("tiny", "block", "ragged", "480p", "720p"):
+        w = I.WORKLOADS[name]
+        assert bench.attention_scores(w) * 4 * w.D == w.attention_flops(), name
+    assert bench.attention_scores(I.WORKLOADS["480p"]) == 24 * 33272 ** 2
