@@ -121,16 +121,55 @@ def workload_bytes(w: I.Workload):
     }
 
 
-class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+CLOCK_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+
+def summarize_clocks(lines, t0=None, t1=None):
+    """Clock record of nvidia-smi lines (timestamp, clocks.sm, clocks.max.sm,
+    power.draw, then the four reasons of CLOCK_REASONS as Active / Not Active).
+    Only samples stamped inside the timed region [t0, t1] (host epoch seconds)
+    count; the median SM clock is then the clock under load.  If none fell
+    inside (a region shorter than the sampling period), every sample counts
+    and ``window`` says so."""
+    import datetime
+    rows = []
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 8:
+            continue
+        try:
+            ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            ts = None        # an unexpected stamp: the sample still counts for the whole run
+        try:
+            rows.append((ts, float(parts[1]), float(parts[2]), parts[4:8]))
+        except ValueError:
+            continue
+    if not rows:
+        return None
+    inside = [r for r in rows
+              if t0 is not None and t1 is not None and r[0] is not None and t0 <= r[0] <= t1]
+    use = inside if inside else rows
+    reasons = sorted({CLOCK_REASONS[i] for r in use for i in range(4) if r[3][i] == "Active"})
+    return {"sm_mhz": statistics.median(r[1] for r in use),
+            "sm_min_mhz": min(r[1] for r in use),
+            "sm_max_mhz": max(r[2] for r in use), "reasons": reasons, "samples": len(use),
+            "window": "timed region" if inside else "whole sampling (no sample inside the "
+                                                    "timed region)"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling around the timed region; mark()
+    brackets the region so that the summary keeps the samples under load."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.t0 = self.t1 = None
         self.path = os.path.join("/tmp", f"mmdit_clocks_{os.getpid()}.csv")
 
     def start(self):
@@ -138,10 +177,17 @@ class ClockSampler:
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.out,
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.out,
                 stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+
+    def mark(self, which: str):
+        """Host time of the start ("start") or end ("end") of the timed region."""
+        if which == "start":
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
 
     def stop(self):
         if self.proc is None:
@@ -153,23 +199,10 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.out.close()
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                rows.append((float(parts[0]), float(parts[1]), parts[3:7]))
-            except ValueError:
-                continue
+        with open(self.path) as f:
+            lines = f.readlines()
         os.unlink(self.path)
-        if not rows:
-            return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i] == "Active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows),
-                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
-                "samples": len(rows)}
+        return summarize_clocks(lines, self.t0, self.t1)
 
 
 def dist_setup(n_gpus: int):
@@ -389,11 +422,13 @@ def run_ours(args):
     ev = [[] for _ in range(5)]
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
+    clocks.mark("start")
     start.record(stream)
     for _ in range(args.steps):
         step(ev)
     stop.record(stream)
     torch.cuda.synchronize(dev)
+    clocks.mark("end")
     barrier(group, dev)
     clk = clocks.stop()
     local_ms = start.elapsed_time(stop)
