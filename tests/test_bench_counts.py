@@ -41,3 +41,11 @@ def test_scores_are_the_attention_flops_over_4d():
         w = I.WORKLOADS[name]
         assert bench.attention_scores(w) * 4 * w.D == w.attention_flops(), name
     assert bench.attention_scores(I.WORKLOADS["480p"]) == 24 * 33272 ** 2
+
+
+def test_l2_note_follows_the_workload():
+    assert "201 MB each, above" in bench.l2_note(I.WORKLOADS["480p"])
+    assert "464 MB each, above" in bench.l2_note(I.WORKLOADS["720p"])
+    assert "249 MB each, above" in bench.l2_note(I.WORKLOADS["ragged"])
+    assert "fit in the 126 MB L2" in bench.l2_note(I.WORKLOADS["block"])
+    assert bench.config_of(I.WORKLOADS["480p"], 1)["l2"] == bench.l2_note(I.WORKLOADS["480p"])
