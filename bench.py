@@ -4,11 +4,12 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload 480p]
 
-A step is one pass of the whole path over one 480p/81-frame sample (21x30x52 =
-32,760 visual + 512 cond tokens, 24 heads x 128): adaLN modulate of both
-streams, QK-RMSNorm + 3D RoPE (visual) / QK-RMSNorm (cond), joint attention,
-and the gated residual of both streams.  Inputs are synthetic (seeded PCG64,
-N(0,1) bf16; see mmdit_joint_attention_b200/inputs.py) and resident in HBM;
+A step is one pass of the whole path over one sample of the workload (by
+default 480p/81 frames: 21x30x52 = 32,760 visual + 512 cond tokens, 24 heads x
+128): adaLN modulate of both streams, QK-RMSNorm + 3D RoPE (visual) /
+QK-RMSNorm (cond), joint attention (with the merge of its split tail), and the
+gated residual of both streams.  Inputs are synthetic (seeded PCG64, N(0,1)
+bf16; see mmdit_joint_attention_b200/inputs.py) and resident in HBM; at 480p
 q/k/v are 201 MB each, larger than the 126 MB L2, so no flush is needed.
 
 The metric is joint-attention TFLOP/s (4 * N^2 * 128 per head, the Wan
@@ -65,9 +66,12 @@ def attn_source_hash() -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def recorded_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, if it
-    was taken on the current kernel source (else None)."""
+def recorded_traffic(w):
+    """DRAM bytes per attention launch from the committed ncu summary of the
+    480p workload, if it was taken on the current kernel source and the run
+    is that workload (else None)."""
+    if w.name != "480p":
+        return None
     try:
         text = open(TRAFFIC_FILE).read()
     except OSError:
@@ -641,11 +645,11 @@ def run_ours(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded PCG64, N(0,1) inputs of the 480p/81f latent shape)",
+        "data": f"synthetic (seeded PCG64, N(0,1) inputs of the {w.name} latent shape)",
         "config": config_of(w, world),
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": attn_tflops / peak,
-                     "traffic": recorded_traffic(),
+                     "traffic": recorded_traffic(w),
                      "peak_kind": f"bf16_tflops_sustained ({pk_src}); attention is timed "
                                   f"inside a multi-second loop of steps"},
         "kernels": kernels,

@@ -49,3 +49,10 @@ def test_l2_note_follows_the_workload():
     assert "249 MB each, above" in bench.l2_note(I.WORKLOADS["ragged"])
     assert "fit in the 126 MB L2" in bench.l2_note(I.WORKLOADS["block"])
     assert bench.config_of(I.WORKLOADS["480p"], 1)["l2"] == bench.l2_note(I.WORKLOADS["480p"])
+
+
+def test_recorded_traffic_only_for_the_captured_workload():
+    """The committed ncu traffic is the 480p launch's: other workloads get none."""
+    assert bench.recorded_traffic(I.WORKLOADS["720p"]) is None
+    t = bench.recorded_traffic(I.WORKLOADS["480p"])
+    assert t is None or t > 8.0e8      # 480p moves at least its 817.8 MB of Q, K, V and O
