@@ -458,7 +458,7 @@ def run_ours(args):
 
     # ---- end-to-end through the public API with host buffers: the library's
     # host-buffer executor copies each step's inputs in from pinned memory, runs
-    # the same seven kernels and copies the outputs back, pipelining the steps
+    # the same seven calls and copies the outputs back, pipelining the steps
     # over three slots of device workspace.
     ex = api.BlockHostExecutor(B, Nv, Nc, H, w.grid, t["gq_vis"], t["gk_vis"], t["gq_ctx"],
                                t["gk_ctx"], pos_scale=w.pos_scale, slots=3)

@@ -516,7 +516,7 @@ def block_forward(t: dict, grid: Sequence[int], pos_scale=(1.0, 1.0, 1.0), eps: 
 class BlockHostExecutor:
     """``block_forward``'s path run step after step from HOST tensors, through
     mmdit_block_forward_host: the library copies each step's inputs in, runs the
-    seven kernels and copies the outputs back, overlapping the copies of some
+    seven calls and copies the outputs back, overlapping the copies of some
     steps with the kernels of others on streams of its own.
 
     The device workspace (``slots`` slots, one step each) is allocated here

@@ -2,11 +2,11 @@
 // buffers, with the copies in, the kernels and the copies out of different
 // steps overlapped on three streams.
 //
-// A step is the seven launches of the device entry points, in this order:
-// adaLN modulate of both streams, QK-RMSNorm + RoPE of both streams (in
-// place), the joint attention (with its split-tail workspace), and the gated
-// residual of both streams (in place on x).  Every buffer a step touches on the device lives in its slot of
-// the workspace:
+// A step is seven calls of the device entry points, in this order: adaLN
+// modulate of both streams, QK-RMSNorm + RoPE of both streams (in place), the
+// joint attention (with its split-tail workspace), and the gated residual of
+// both streams (in place on x).  Every buffer a step touches on the device
+// lives in its slot of the workspace:
 //
 //   per stream s in (vis, ctx), N_s tokens:  q, k, v, x, y, o   [B, N_s, C] dt
 //   per stream:                              shift, scale, gate [B, C] fp32
