@@ -320,8 +320,10 @@ def joint_attention_q8(q8, k8, v8, scales: dict, ctx_len=None,
     vv, vc = v8
     B, Nv, H, D = qv.shape
     Nc = qc.shape[1]
-    o_vis = torch.empty(qv.shape, dtype=torch.bfloat16, device=qv.device) if o_vis is None else o_vis
-    o_ctx = torch.empty(qc.shape, dtype=torch.bfloat16, device=qv.device) if o_ctx is None else o_ctx
+    if o_vis is None:
+        o_vis = torch.empty(qv.shape, dtype=torch.bfloat16, device=qv.device)
+    if o_ctx is None:
+        o_ctx = torch.empty(qc.shape, dtype=torch.bfloat16, device=qv.device)
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
     st = _lib.lib().mmdit_joint_attention_q8(
