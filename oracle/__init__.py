@@ -82,6 +82,9 @@ def _configure(lib):
         [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp]
     lib.oracle_adaln_modulate.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3 + [ctypes.c_double]
     lib.oracle_gated_residual.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3
+    lib.oracle_adaln_modulate_bwd.argtypes = [dp, dp, dp] + [ctypes.c_int] * 3 + [
+        ctypes.c_double, dp, dp, dp]
+    lib.oracle_gated_residual_bwd.argtypes = [dp, dp, dp] + [ctypes.c_int] * 3 + [dp, dp, dp]
     return lib
 
 
@@ -474,6 +477,30 @@ def gated_residual(x, branch, gate) -> np.ndarray:
     B, N, C = x.shape
     out = np.empty_like(x)
     _load().oracle_gated_residual(_p(x), _p(branch), _p(gate), _p(out), B, N, C)
+    return out
+
+
+def adaln_modulate_bwd(x, scale, dy, eps: float = 1e-6) -> dict:
+    """Backward of adaln_modulate for the upstream gradient dy [B, N, C]:
+    dx [B, N, C], dshift and dscale [B, C] (the shift does not enter any of
+    them)."""
+    x, scale, dy = _f64(x), _f64(scale), _f64(dy)
+    B, N, C = x.shape
+    out = {"dx": np.empty_like(x), "dshift": np.empty((B, C)), "dscale": np.empty((B, C))}
+    _load().oracle_adaln_modulate_bwd(_p(x), _p(scale), _p(dy), B, N, C, eps, _p(out["dx"]),
+                                      _p(out["dshift"]), _p(out["dscale"]))
+    return out
+
+
+def gated_residual_bwd(branch, gate, dout) -> dict:
+    """Backward of gated_residual for the upstream gradient dout [B, N, C]:
+    dx, dbranch [B, N, C] and dgate [B, C]."""
+    branch, gate, dout = _f64(branch), _f64(gate), _f64(dout)
+    B, N, C = branch.shape
+    out = {"dx": np.empty_like(branch), "dbranch": np.empty_like(branch),
+           "dgate": np.empty((B, C))}
+    _load().oracle_gated_residual_bwd(_p(branch), _p(gate), _p(dout), B, N, C, _p(out["dx"]),
+                                      _p(out["dbranch"]), _p(out["dgate"]))
     return out
 
 

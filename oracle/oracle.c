@@ -215,6 +215,74 @@ void oracle_gated_residual(const double* x, const double* branch, const double* 
     }
 }
 
+/* ---- backward of adaLN modulate [V] -------------------------------------------
+ * Reverse-mode derivative of y = xh * (1 + scale[b, c]) + shift[b, c], with
+ * xh = (x - mu) * rstd and rstd = 1 / sqrt(var + eps) over the C values of a
+ * row (biased variance).  For the upstream gradient dy of a row:
+ *   g  = dy * (1 + scale[b, c])
+ *   dx = rstd * (g - mean_c(g) - xh * mean_c(g * xh))
+ *   dshift[b, c] = sum over the rows of sample b of dy
+ *   dscale[b, c] = sum over the rows of sample b of dy * xh
+ * dshift and dscale [B, C] are written, not accumulated.                      */
+void oracle_adaln_modulate_bwd(const double* x, const double* scale, const double* dy,
+                               int B, int N, int C, double eps, double* dx, double* dshift,
+                               double* dscale)
+{
+    for (long i = 0; i < (long)B * C; ++i) {
+        dshift[i] = 0.0;
+        dscale[i] = 0.0;
+    }
+    double* xh = (double*)malloc(sizeof(double) * (size_t)C);
+    for (int b = 0; b < B; ++b) {
+        for (int n = 0; n < N; ++n) {
+            const long row = ((long)b * N + n) * C;
+            const double* xr = x + row;
+            const double* dr = dy + row;
+            double sum = 0.0;
+            for (int c = 0; c < C; ++c) sum += xr[c];
+            const double mean = sum / (double)C;
+            double ss = 0.0;
+            for (int c = 0; c < C; ++c) ss += (xr[c] - mean) * (xr[c] - mean);
+            const double rstd = 1.0 / sqrt(ss / (double)C + eps);
+            double mg = 0.0, mgx = 0.0;
+            for (int c = 0; c < C; ++c) {
+                xh[c] = (xr[c] - mean) * rstd;
+                const double g = dr[c] * (1.0 + scale[(long)b * C + c]);
+                mg += g;
+                mgx += g * xh[c];
+                dshift[(long)b * C + c] += dr[c];
+                dscale[(long)b * C + c] += dr[c] * xh[c];
+            }
+            mg /= (double)C;
+            mgx /= (double)C;
+            for (int c = 0; c < C; ++c) {
+                const double g = dr[c] * (1.0 + scale[(long)b * C + c]);
+                dx[row + c] = rstd * (g - mg - xh[c] * mgx);
+            }
+        }
+    }
+    free(xh);
+}
+
+/* ---- backward of the gated residual [V] ------------------------------------
+ * out = x + gate[b, c] * branch:  dx = dout,  dbranch = gate[b, c] * dout,
+ * dgate[b, c] = sum over the rows of sample b of dout * branch (written).      */
+void oracle_gated_residual_bwd(const double* branch, const double* gate, const double* dout,
+                               int B, int N, int C, double* dx, double* dbranch, double* dgate)
+{
+    for (long i = 0; i < (long)B * C; ++i) dgate[i] = 0.0;
+    for (int b = 0; b < B; ++b) {
+        for (int n = 0; n < N; ++n) {
+            const long row = ((long)b * N + n) * C;
+            for (int c = 0; c < C; ++c) {
+                dx[row + c] = dout[row + c];
+                dbranch[row + c] = gate[(long)b * C + c] * dout[row + c];
+                dgate[(long)b * C + c] += dout[row + c] * branch[row + c];
+            }
+        }
+    }
+}
+
 /* ---- 3D window attention [S] ----------------------------------------------
  * Seaweed-7B report, section 3.2: the visual tokens are partitioned into
  * w_t x w_h x w_w windows and attention is computed only within a window

@@ -59,5 +59,10 @@ void oracle_adaln_modulate(const double* x, const double* shift, const double* s
                            double* y, int B, int N, int C, double eps);
 void oracle_gated_residual(const double* x, const double* branch, const double* gate,
                            double* out, int B, int N, int C);
+void oracle_adaln_modulate_bwd(const double* x, const double* scale, const double* dy,
+                               int B, int N, int C, double eps, double* dx, double* dshift,
+                               double* dscale);
+void oracle_gated_residual_bwd(const double* branch, const double* gate, const double* dout,
+                               int B, int N, int C, double* dx, double* dbranch, double* dgate);
 
 #endif

@@ -686,6 +686,91 @@ def pin_norm_rope_bwd_torch_autograd():
     _close(dg, gt.grad.numpy(), 1e-11)
 
 
+# ------------------------------------------------ modulate / residual backward
+
+@pin
+def pin_modulate_bwd_finite_differences():
+    """dx, dshift and dscale equal central differences of L = sum(dy * y),
+    y the forward modulate oracle, for every entry."""
+    r = RNG(70)
+    B, N, C = 2, 3, 16
+    x = r.standard_normal((B, N, C)) * 1.5 + 0.3
+    sh, sc = r.standard_normal((B, C)) * 0.1, r.standard_normal((B, C)) * 0.1
+    dy = r.standard_normal((B, N, C))
+    got = oracle.adaln_modulate_bwd(x, sc, dy)
+    loss = lambda xx, hh, ss: float(np.sum(dy * oracle.adaln_modulate(xx, hh, ss)))  # noqa: E731
+    h = 1e-6
+    for name, arr, f in (("dx", x, lambda a: loss(a, sh, sc)),
+                         ("dshift", sh, lambda a: loss(x, a, sc)),
+                         ("dscale", sc, lambda a: loss(x, sh, a))):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            ap, am = arr.copy(), arr.copy()
+            ap[idx] += h
+            am[idx] -= h
+            num[idx] = (f(ap) - f(am)) / (2 * h)
+        _close(got[name], num, 1e-7)
+
+
+@pin
+def pin_modulate_bwd_torch_autograd():
+    """torch float64 autograd through layer_norm (no affine), the (1 + scale)
+    multiply and the shift."""
+    r = RNG(71)
+    B, N, C = 2, 5, 64
+    x = r.standard_normal((B, N, C)) * 2.0
+    sh, sc = r.standard_normal((B, C)) * 0.1, r.standard_normal((B, C)) * 0.1
+    dy = r.standard_normal((B, N, C))
+    xt, sht, sct = (torch.tensor(a, requires_grad=True) for a in (x, sh, sc))
+    y = torch.nn.functional.layer_norm(xt, (C,), eps=1e-6) * (1 + sct[:, None, :]) + sht[:, None, :]
+    y.backward(torch.from_numpy(dy))
+    got = oracle.adaln_modulate_bwd(x, sc, dy, 1e-6)
+    _close(got["dx"], xt.grad.numpy(), 1e-12)
+    _close(got["dshift"], sht.grad.numpy(), 1e-12)
+    _close(got["dscale"], sct.grad.numpy(), 1e-12)
+
+
+@pin
+def pin_modulate_bwd_invariants():
+    """LayerNorm ignores adding a constant to a row and, with eps = 0,
+    scaling it: so dx is orthogonal to the ones vector and to x - mean; an
+    upstream gradient constant along a row (scale 0) gives dx = 0."""
+    r = RNG(72)
+    B, N, C = 2, 4, 32
+    x = r.standard_normal((B, N, C))
+    sc = r.standard_normal((B, C)) * 0.2
+    dy = r.standard_normal((B, N, C))
+    dx = oracle.adaln_modulate_bwd(x, sc, dy, 0.0)["dx"]
+    xc = x - x.mean(-1, keepdims=True)
+    assert np.max(np.abs(dx.sum(-1))) < 1e-12
+    assert np.max(np.abs((dx * xc).sum(-1))) < 1e-12
+    const = np.repeat(r.standard_normal((B, N, 1)), C, axis=-1)
+    dx0 = oracle.adaln_modulate_bwd(x, np.zeros((B, C)), const, 1e-6)["dx"]
+    assert np.max(np.abs(dx0)) < 1e-13
+
+
+@pin
+def pin_residual_bwd_finite_differences():
+    """dx, dbranch and dgate equal central differences of L = sum(dout * out),
+    out the forward gated-residual oracle."""
+    r = RNG(73)
+    B, N, C = 2, 3, 8
+    x, br, dout = (r.standard_normal((B, N, C)) for _ in range(3))
+    g = r.standard_normal((B, C)) * 0.5
+    got = oracle.gated_residual_bwd(br, g, dout)
+    loss = lambda xx, bb, gg: float(np.sum(dout * oracle.gated_residual(xx, bb, gg)))  # noqa: E731
+    h = 1e-6
+    for name, arr, f in (("dx", x, lambda a: loss(a, br, g)), ("dbranch", br, lambda a: loss(x, a, g)),
+                         ("dgate", g, lambda a: loss(x, br, a))):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            ap, am = arr.copy(), arr.copy()
+            ap[idx] += h
+            am[idx] -= h
+            num[idx] = (f(ap) - f(am)) / (2 * h)
+        _close(got[name], num, 1e-8)
+
+
 # ---------------------------------------------------------------- 8-bit attention
 
 @pin
@@ -848,6 +933,22 @@ MUTANTS = {
     "q8_sum_rounded": ("        l += p;\n", "        l += oracle_e4m3_round(p);\n"),
     "q8_subnormal_step": ("        quantum = ldexp(1.0, -9);                               /* subnormal range */",
                           "        quantum = ldexp(1.0, -10);"),
+    "modbwd_no_mean_g": ("dx[row + c] = rstd * (g - mg - xh[c] * mgx);",
+                         "dx[row + c] = rstd * (g - xh[c] * mgx);"),
+    "modbwd_no_xh_term": ("dx[row + c] = rstd * (g - mg - xh[c] * mgx);",
+                          "dx[row + c] = rstd * (g - mg);"),
+    "modbwd_rstd_squared": ("dx[row + c] = rstd * (g - mg - xh[c] * mgx);",
+                            "dx[row + c] = rstd * rstd * (g - mg - xh[c] * mgx);"),
+    "modbwd_no_one_plus": ("const double g = dr[c] * (1.0 + scale[(long)b * C + c]);\n"
+                           "                dx[row + c]",
+                           "const double g = dr[c] * scale[(long)b * C + c];\n"
+                           "                dx[row + c]"),
+    "modbwd_dscale_no_xh": ("dscale[(long)b * C + c] += dr[c] * xh[c];",
+                            "dscale[(long)b * C + c] += dr[c];"),
+    "resbwd_dbranch_no_gate": ("dbranch[row + c] = gate[(long)b * C + c] * dout[row + c];",
+                               "dbranch[row + c] = dout[row + c];"),
+    "resbwd_dgate_no_branch": ("dgate[(long)b * C + c] += dout[row + c] * branch[row + c];",
+                               "dgate[(long)b * C + c] += dout[row + c];"),
     "window_no_cond_keys": ("for (int j = 0; j < L; ++j) key[nk++] = Nv + j;",
                             "for (int j = 0; j < L && i >= Nv; ++j) key[nk++] = Nv + j;"),
 }
