@@ -412,6 +412,35 @@ MMDIT_API int mmdit_adaln_modulate(const void* x, const float* shift, const floa
 MMDIT_API int mmdit_gated_residual(const void* x, const void* branch, const float* gate, void* out,
                          int B, int N, int C, mmdit_dtype dt, void* stream);
 
+/* Backward of mmdit_adaln_modulate [the reverse-mode derivative of the adaLN
+ * modulate of Vimoo §2.2]: for the upstream gradient dy of y, with
+ * xh = (x - mean) / sqrt(var + eps) per row of C values,
+ *   g  = dy * (1 + scale[b])
+ *   dx = (g - mean_c(g) - xh * mean_c(g * xh)) / sqrt(var + eps)
+ *   dshift[b, c] = sum over the rows of sample b of dy
+ *   dscale[b, c] = sum over the rows of sample b of dy * xh
+ *   x, dy [B, N, C] dt read;  dx [B, N, C] dt written (may equal dy, not x)
+ *   scale [B, C] fp32;  dshift, dscale [B, C] fp32 written (zeroed, then summed
+ *   with floating-point atomics: their last bits may differ from run to run)
+ *   C % 8 == 0 and C <= 4096 (bf16) / 2048 (f32)
+ * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_adaln_modulate_bwd(const void* x, const float* scale, const void* dy,
+                                       void* dx, float* dshift, float* dscale, int B, int N,
+                                       int C, float eps, mmdit_dtype dt, void* stream);
+
+/* Backward of mmdit_gated_residual [the reverse-mode derivative of the gated
+ * residual of Vimoo §2.2]: for the upstream gradient dout of out,
+ *   dx = dout,  dbranch = gate[b] * dout,
+ *   dgate[b, c] = sum over the rows of sample b of dout * branch
+ *   branch, dout [B, N, C] dt read;  dbranch [B, N, C] dt written (may equal
+ *   dout, not branch);  dx [B, N, C] dt written, or NULL (it equals dout)
+ *   gate [B, C] fp32;  dgate [B, C] fp32 written (zeroed, then summed with
+ *   floating-point atomics);  C % 8 == 0 and C <= 4096 (bf16) / 2048 (f32)
+ * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_gated_residual_bwd(const void* branch, const float* gate, const void* dout,
+                                       void* dx, void* dbranch, float* dgate, int B, int N,
+                                       int C, mmdit_dtype dt, void* stream);
+
 /* Gated residual fused with the adaLN modulate that follows it, in one pass
  * over memory [Vimoo §2.2: a branch's gated contribution is added to the
  * residual stream, and the next branch starts from a LayerNorm of that stream

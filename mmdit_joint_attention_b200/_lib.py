@@ -124,6 +124,8 @@ def lib():
         L.mmdit_adaln_modulate.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp]
         L.mmdit_gated_residual.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
         L.mmdit_residual_modulate.argtypes = [_vp] * 7 + [_i, _i, _i, _f, _i, _vp]
+        L.mmdit_adaln_modulate_bwd.argtypes = [_vp] * 6 + [_i, _i, _i, _f, _i, _vp]
+        L.mmdit_gated_residual_bwd.argtypes = [_vp] * 6 + [_i, _i, _i, _i, _vp]
         L.mmdit_device_status.argtypes = [_vp]
         L.mmdit_block_slot_bytes.argtypes = [ctypes.POINTER(BlockConfig)]
         L.mmdit_block_slot_bytes.restype = ctypes.c_longlong
@@ -144,6 +146,7 @@ def lib():
                      "mmdit_joint_attention_ws", "mmdit_joint_attention_split_plan",
                      "mmdit_joint_window_attention", "mmdit_adaln_modulate",
                      "mmdit_gated_residual", "mmdit_residual_modulate", "mmdit_device_status",
+                     "mmdit_adaln_modulate_bwd", "mmdit_gated_residual_bwd",
                      "mmdit_block_forward_host"):
             getattr(L, name).restype = ctypes.c_int
         _LIB = L

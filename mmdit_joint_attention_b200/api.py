@@ -460,6 +460,39 @@ def gated_residual(x: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor,
     return out
 
 
+def adaln_modulate_bwd(x: torch.Tensor, scale: torch.Tensor, dy: torch.Tensor,
+                       eps: float = 1e-6, stream=None
+                       ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Backward of adaln_modulate: (dx, dshift, dscale) for the gradient dy of y."""
+    dt = _dtype(x, dy)
+    _f32(scale)
+    B, N, C = x.shape
+    dx = torch.empty_like(x)
+    dshift = torch.empty((B, C), dtype=torch.float32, device=x.device)
+    dscale = torch.empty_like(dshift)
+    st = _lib.lib().mmdit_adaln_modulate_bwd(_ptr(x), _ptr(scale), _ptr(dy), _ptr(dx),
+                                             _ptr(dshift), _ptr(dscale), B, N, C, eps, dt,
+                                             _stream(stream))
+    check("mmdit_adaln_modulate_bwd", st)
+    return dx, dshift, dscale
+
+
+def gated_residual_bwd(branch: torch.Tensor, gate: torch.Tensor, dout: torch.Tensor,
+                       stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Backward of gated_residual: (dbranch, dgate) for the gradient dout of
+    the output; the gradient of x is dout itself."""
+    dt = _dtype(branch, dout)
+    _f32(gate)
+    B, N, C = branch.shape
+    dbranch = torch.empty_like(branch)
+    dgate = torch.empty((B, C), dtype=torch.float32, device=branch.device)
+    st = _lib.lib().mmdit_gated_residual_bwd(_ptr(branch), _ptr(gate), _ptr(dout), None,
+                                             _ptr(dbranch), _ptr(dgate), B, N, C, dt,
+                                             _stream(stream))
+    check("mmdit_gated_residual_bwd", st)
+    return dbranch, dgate
+
+
 def residual_modulate(x: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor,
                       shift: torch.Tensor, scale: torch.Tensor, eps: float = 1e-6,
                       x_out: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,

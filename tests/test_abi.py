@@ -312,3 +312,23 @@ def test_split_plan(L):
     assert f(-1, 8, 8, 2, 148, ws, plan) == -1
     assert f(1, 8, 8, 2, 0, ws, plan) == -1
     assert f(1, 8, 8, 2, 148, ws, None) == -1
+
+
+def test_elementwise_bwd_validation(L):
+    fm, fr = L.mmdit_adaln_modulate_bwd, L.mmdit_gated_residual_bwd
+    # modulate: x, scale, dy, dx, dshift, dscale, B, N, C, eps, dt, stream
+    assert fm(P, P, P, ctypes.c_void_p(4096), P, P, 1, 4, 60, 1e-6, 1, None) == -4   # C % 8
+    assert fm(P, P, P, ctypes.c_void_p(4096), P, P, 1, 4, 4104, 1e-6, 1, None) == -4  # C > 4096
+    assert fm(P, P, P, ctypes.c_void_p(4096), P, P, 1, 4, 64, -1.0, 1, None) == -1   # eps
+    assert fm(P, P, P, ctypes.c_void_p(4096), P, P, 1, 4, 64, 1e-6, 9, None) == -1   # dtype
+    assert fm(P, None, P, ctypes.c_void_p(4096), P, P, 1, 4, 64, 1e-6, 1, None) == -1
+    assert fm(P, P, P, ctypes.c_void_p(4097), P, P, 1, 4, 64, 1e-6, 1, None) == -3
+    assert fm(P, P, P, P, ctypes.c_void_p(4096), P, 1, 4, 64, 1e-6, 1, None) == -1   # dx aliases x
+    assert fm(None, None, None, None, None, None, 0, 4, 64, 1e-6, 1, None) == 0      # B = 0
+    # residual: branch, gate, dout, dx, dbranch, dgate, B, N, C, dt, stream
+    assert fr(P, P, P, None, ctypes.c_void_p(4096), P, 1, 4, 60, 1, None) == -4
+    assert fr(P, None, P, None, ctypes.c_void_p(4096), P, 1, 4, 64, 1, None) == -1
+    assert fr(P, P, P, None, None, P, 1, 4, 64, 1, None) == -1
+    assert fr(P, P, P, ctypes.c_void_p(18), ctypes.c_void_p(4096), P, 1, 4, 64, 1, None) == -3
+    assert fr(P, P, P, None, P, P, 1, 4, 64, 1, None) == -1                          # dbranch aliases branch
+    assert fr(None, None, None, None, None, None, 0, 4, 64, 1, None) == 0
