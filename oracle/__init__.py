@@ -62,6 +62,9 @@ def _configure(lib):
     lib.oracle_joint_attention_dq_rows.argtypes = (
         [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [dp] * 2 + [ctypes.c_int] * 5 +
         [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp, dp])
+    lib.oracle_joint_attention_dkdv_rows.argtypes = (
+        [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [dp] * 2 + [ctypes.c_int] * 5 +
+        [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp, dp])
     lib.oracle_rmsnorm_rope_bwd.argtypes = [dp, dp, dp, dp, ctypes.c_double,
                                             ctypes.POINTER(ctypes.c_int), ctypes.c_long,
                                             ctypes.c_int, ctypes.c_double, dp, dp]
@@ -246,6 +249,27 @@ def joint_attention_dq_rows(qv, kv, vv, qc, kc, vc, dov, doc, ctx_len, rows,
             H, D, scale, rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), rows.shape[0],
             _p(dq), _p(lse))
     return dq, lse
+
+
+def joint_attention_dkdv_rows(qv, kv, vv, qc, kc, vc, dov, doc, ctx_len, keys,
+                              scale: Optional[float] = None):
+    """(dk [nkeys, D], dv [nkeys, D]) of selected (b, h, joint key index)
+    triplets; padded keys give zeros."""
+    qv, kv, vv, qc, kc, vc, dov, doc = (_f64(a) for a in (qv, kv, vv, qc, kc, vc, dov, doc))
+    B, Nv, H, D = qv.shape
+    Nc = qc.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    keys = np.ascontiguousarray(keys, dtype=np.int64).reshape(-1, 3)
+    dk = np.zeros((keys.shape[0], D), dtype=np.float64)
+    dv = np.zeros((keys.shape[0], D), dtype=np.float64)
+    cl_p, _keep = _ctx_ptr(ctx_len)
+    if keys.shape[0]:
+        _load().oracle_joint_attention_dkdv_rows(
+            _p(qv), _p(kv), _p(vv), _p(qc), _p(kc), _p(vc), cl_p, _p(dov), _p(doc), B, Nv, Nc,
+            H, D, scale, keys.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), keys.shape[0],
+            _p(dk), _p(dv))
+    return dk, dv
 
 
 def grid_positions(grid, pos_scale=(1.0, 1.0, 1.0)) -> np.ndarray:

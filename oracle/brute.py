@@ -13,7 +13,8 @@ to pin the C oracle (``oracle.c``).  It shares no code with it:
     array_split of the (T, H, W) grid along each axis) and runs the
     concatenated-sequence attention above on every window separately;
   * the 8-bit attention quantises with numpy float32 arithmetic and torch's
-    float8_e4m3fn conversion, and runs its tiled softmax with numpy arrays.
+    float8_e4m3fn conversion, dequantises k block by block, and forms each
+    row's whole score vector with one matrix product.
 
 Sources: Vimoo 1.0 research page, section 2.2 (dual-stream joint attention,
 QK-RMSNorm, 3D RoPE 16/56/56, adaLN, gated residual); Wan 2.1 report section
@@ -152,6 +153,9 @@ def quant_int8(x, block):
 
 
 def attention_q8(qv, kv, vv, qc, kc, vc, ctx_len=None, scale=None):
+    """The 8-bit method with numpy arrays: float32 quantisation, torch's E4M3
+    conversion, and for each (row, head) the whole score vector at once (the
+    concatenated valid keys), m = ceil of its maximum, P' = 2^(x - m + 6)."""
     qv, kv, vv, qc, kc, vc = (np.asarray(a, dtype=np.float64) for a in (qv, kv, vv, qc, kc, vc))
     B, Nv, H, D = qv.shape
     Nc = qc.shape[1]
@@ -170,29 +174,17 @@ def attention_q8(qv, kv, vv, qc, kc, vc, ctx_len=None, scale=None):
         vals = np.concatenate([vv[b], vc[b, :L]], axis=0).astype(np.float32)     # [Nk, H, D]
         sv = np.abs(vals).max(axis=0) / np.float32(448.0)                          # [H, D]
         v8 = np.where(sv > 0, e4m3(np.where(sv > 0, vals / np.where(sv > 0, sv, 1), 0)), 0)
-        # key tiles: visual blocks of 128, then conditioning blocks of 128
-        tiles = [(j, min(j + 128, Nv), skv[b, :, j // 128], 0) for j in range(0, Nv, 128)]
-        tiles += [(Nv + j, Nv + min(j + 128, L), skc[b, :, j // 128], 1) for j in range(0, L, 128)]
-        K8 = np.concatenate([k8v[b], k8c[b, :L]], axis=0)
+        # dequantised keys: codes times the scale of their 128-token block
+        kd = np.concatenate([k8v[b] * np.repeat(skv[b].T, 128, axis=0)[:Nv, :, None],
+                             k8c[b, :L] * np.repeat(skc[b].T, 128, axis=0)[:L, :, None]], axis=0)
         for i in range(Nv + L):
             q8 = q8v[b, i] if i < Nv else q8c[b, i - Nv]
             sq = sqv[b, :, i] if i < Nv else sqc[b, :, i - Nv]
             for h in range(H):
-                m, acc, l = None, np.zeros(D), 0.0
-                for j0, j1, sk, _ in tiles:
-                    x = (K8[j0:j1, h] @ q8[h]) * float(sq[h]) * float(sk[h]) * scale * np.log2(np.e)
-                    mt = x.max()
-                    if m is None:
-                        m = np.ceil(mt)
-                    elif mt > m + 2:
-                        mn = np.ceil(mt)
-                        acc *= 2.0 ** (m - mn)
-                        l *= 2.0 ** (m - mn)
-                        m = mn
-                    p = 2.0 ** (x - m + 6)
-                    l += p.sum()
-                    acc += e4m3(p) @ v8[j0:j1, h]
-                o = acc * sv[h] / l
+                x = (kd[:, h] @ q8[h]) * float(sq[h]) * scale * np.log2(np.e)
+                m = np.ceil(x.max())
+                p = 2.0 ** (x - m + 6)
+                o = (e4m3(p) @ v8[:, h]) * sv[h] / p.sum()
                 if i < Nv:
                     out_v[b, i, h] = o
                 else:

@@ -526,6 +526,95 @@ void oracle_joint_attention_dq_rows(const double* qv, const double* kv, const do
     }
 }
 
+/* dK and dV of selected keys (b, h, joint key index j), for the checks at
+ * sizes where the whole backward is too slow [the reverse-mode derivative of
+ * the joint attention, as oracle_joint_attention_bwd]:
+ *   dV_j = sum_i P_ij dO_i,   dK_j = scale * sum_i P_ij (dO_i . V_j - D_i) Q_i
+ * over the query rows i that have an output (i < Nv + ctx_len[b]), with
+ * P_ij = exp(s_ij - lse_i), s_ij = scale Q_i . K_j and D_i = dO_i . O_i.
+ * For every (b, h) that holds a selected key, lse_i and D_i of all its query
+ * rows come first, each row computed as the forward defines it; then the sums
+ * over i for each selected key.  Padded keys (j >= Nv + ctx_len[b]) get 0. */
+void oracle_joint_attention_dkdv_rows(const double* qv, const double* kv, const double* vv,
+                                      const double* qc, const double* kc, const double* vc,
+                                      const int* ctx_len, const double* dov, const double* doc,
+                                      int B, int Nv, int Nc, int H, int D, double scale,
+                                      const long* keys, long nkeys, double* dk_out,
+                                      double* dv_out)
+{
+    double* lse = (double*)malloc(sizeof(double) * (size_t)(Nv + Nc + 1));
+    double* Dr = (double*)malloc(sizeof(double) * (size_t)(Nv + Nc + 1));
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const long b = bh / H, h = bh % H;
+        int any = 0;
+        for (long r = 0; r < nkeys; ++r)
+            if (keys[3 * r] == b && keys[3 * r + 1] == h) { any = 1; break; }
+        if (!any) continue;
+        const int L = ctx_len ? ctx_len[b] : Nc;
+        const int nval = Nv + L;    /* valid keys, and the query rows with an output */
+        #pragma omp parallel
+        {
+            double* s = (double*)malloc(sizeof(double) * (size_t)(nval + 1));
+            double* o = (double*)malloc(sizeof(double) * (size_t)D);
+            #pragma omp for schedule(dynamic, 16)
+            for (int i = 0; i < nval; ++i) {
+                const double* q = oracle_row(qv, qc, b, i, Nv, Nc, H, h, D);
+                const double* dO = oracle_row(dov, doc, b, i, Nv, Nc, H, h, D);
+                double mx = -INFINITY;
+                for (int j = 0; j < nval; ++j) {
+                    const double* k = oracle_row(kv, kc, b, j, Nv, Nc, H, h, D);
+                    double acc = 0.0;
+                    for (int d = 0; d < D; ++d) acc += q[d] * k[d];
+                    s[j] = scale * acc;
+                    mx = s[j] > mx ? s[j] : mx;
+                }
+                double sum = 0.0;
+                for (int j = 0; j < nval; ++j) sum += exp(s[j] - mx);
+                lse[i] = mx + log(sum);
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (int j = 0; j < nval; ++j) {
+                    const double p = exp(s[j] - mx) / sum;
+                    const double* v = oracle_row(vv, vc, b, j, Nv, Nc, H, h, D);
+                    for (int d = 0; d < D; ++d) o[d] += p * v[d];
+                }
+                double Di = 0.0;
+                for (int d = 0; d < D; ++d) Di += dO[d] * o[d];
+                Dr[i] = Di;
+            }
+            free(o);
+            free(s);
+        }
+        #pragma omp parallel for schedule(dynamic, 1)
+        for (long r = 0; r < nkeys; ++r) {
+            if (keys[3 * r] != b || keys[3 * r + 1] != h) continue;
+            const long j = keys[3 * r + 2];
+            double* dk = dk_out + r * (long)D;
+            double* dv = dv_out + r * (long)D;
+            for (int d = 0; d < D; ++d) { dk[d] = 0.0; dv[d] = 0.0; }
+            if (j >= nval) continue;                          /* padded key */
+            const double* k = oracle_row(kv, kc, b, j, Nv, Nc, H, h, D);
+            const double* v = oracle_row(vv, vc, b, j, Nv, Nc, H, h, D);
+            for (int i = 0; i < nval; ++i) {
+                const double* qi = oracle_row(qv, qc, b, i, Nv, Nc, H, h, D);
+                const double* dOi = oracle_row(dov, doc, b, i, Nv, Nc, H, h, D);
+                double sij = 0.0, dP = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    sij += qi[d] * k[d];
+                    dP += dOi[d] * v[d];
+                }
+                const double p = exp(scale * sij - lse[i]);
+                const double dS = p * (dP - Dr[i]);
+                for (int d = 0; d < D; ++d) {
+                    dv[d] += p * dOi[d];
+                    dk[d] += scale * dS * qi[d];
+                }
+            }
+        }
+    }
+    free(Dr);
+    free(lse);
+}
+
 /* ---- QK-RMSNorm + RoPE backward [V], [S] ----------------------------------
  * Reverse-mode derivative of y = R(pos) (x / r * g), r = sqrt(mean(x^2) + eps),
  * for rows x [rows, D] whose RoPE positions are pos [rows, 3] (already scaled;
@@ -593,14 +682,16 @@ void oracle_rmsnorm_rope_bwd(const double* x, const double* g, const double* dy,
  *   - v is quantised to E4M3 per (sample, head, channel) over the valid
  *     tokens of both streams: scale = max|v| / 448 (fp32), code = E4M3
  *     rounding (half-even, saturating at 448) of v / scale (fp32);
- *   - the softmax runs over key tiles of 128 (visual tiles, then the valid
- *     conditioning tiles) with a running maximum m in log2 units that is an
- *     integer (the ceiling of a tile maximum) and is raised only when a
- *     tile's maximum exceeds it by more than 2; P' = 2^(x - m + 6), with x the
- *     score in log2 units, is rounded to E4M3 for the P V product, while the
- *     row sum takes P' unrounded; o = scale_v * sum(E4M3(P') v8) / sum(P').
- * Because m is an integer, two schedules of raising it give P' that differ by
- * exact powers of two, which E4M3 rounding commutes with (up to subnormals). */
+ *   - the softmax of a row, written plainly: x_j is the score of valid key j
+ *     in log2 units (the exact integer dot product of the codes times both
+ *     scales, the softmax scale and log2 e), m = ceil(max_j x_j) an integer,
+ *     P'_j = 2^(x_j - m + 6) <= 2^6, rounded to E4M3 for the P V product and
+ *     unrounded in the row sum:  o = scale_v * sum_j E4M3(P'_j) v8_j / sum_j P'_j.
+ * A tiled schedule that keeps an integer running maximum and rescales by
+ * 2^(old - new) computes the same values: every P' it rounds differs from the
+ * one here by an exact power of two, which E4M3 rounding commutes with, except
+ * for keys whose P' here falls in E4M3's subnormal range (x_j < m - 12, a
+ * weight below 2^-12 of the largest). */
 
 /* E4M3: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits; no infinity; the
  * largest finite magnitude is 1.75 * 2^8 = 448; subnormals step 2^-9.       */
@@ -721,54 +812,40 @@ void oracle_attention_q8_rows(const signed char* qv, const signed char* qc, cons
     const int tv = (Nv + 127) / 128, tc = (Nc + 127) / 128;
     #pragma omp parallel
     {
-        double* x = (double*)malloc(sizeof(double) * 128);
+        double* x = (double*)malloc(sizeof(double) * (size_t)(Nv + Nc + 1));
         double* acc = (double*)malloc(sizeof(double) * (size_t)D);
         #pragma omp for schedule(dynamic, 4)
         for (long r = 0; r < nrows; ++r) {
             const long b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
             const int L = ctx_len ? ctx_len[b] : Nc;
+            const int nval = Nv + L;                /* valid keys: visual, then cond */
             double* o = out + r * (long)D;
             for (int d = 0; d < D; ++d) { o[d] = 0.0; acc[d] = 0.0; }
-            if (i >= Nv + L || Nv + L == 0) continue;     /* no output */
+            if (i >= nval || nval == 0) continue;   /* no output */
             const signed char* q = (i < Nv) ? qv + ((b * Nv + i) * H + h) * (long)D
                                             : qc + ((b * Nc + (i - Nv)) * H + h) * (long)D;
             const double sq = (i < Nv) ? sqv[(b * H + h) * (long)Nv + i]
                                        : sqc[(b * H + h) * (long)Nc + (i - Nv)];
-            double m = 0.0, l = 0.0;
-            int first = 1;
-            for (int seg = 0; seg < 2; ++seg) {
-                const int nk = seg ? L : Nv, Ns = seg ? Nc : Nv, nt = seg ? tc : tv;
-                const signed char* K = seg ? kc : kv;
-                const unsigned char* V = seg ? vc : vv;
-                const float* sk = seg ? skc : skv;
-                for (int t = 0; t * 128 < nk; ++t) {
-                    const int j0 = t * 128, j1 = (j0 + 128 < nk) ? j0 + 128 : nk;
-                    const double skb = sk[(b * H + h) * (long)nt + t];
-                    double mt = -INFINITY;
-                    for (int j = j0; j < j1; ++j) {
-                        const signed char* k = K + ((b * Ns + j) * H + h) * (long)D;
-                        long dot = 0;
-                        for (int d = 0; d < D; ++d) dot += (long)q[d] * (long)k[d];
-                        x[j - j0] = (double)dot * sq * skb * scale * log2e;
-                        if (x[j - j0] > mt) mt = x[j - j0];
-                    }
-                    if (first) {
-                        m = ceil(mt);
-                        first = 0;
-                    } else if (mt > m + 2.0) {
-                        const double mn = ceil(mt), f = exp2(m - mn);
-                        for (int d = 0; d < D; ++d) acc[d] *= f;
-                        l *= f;
-                        m = mn;
-                    }
-                    for (int j = j0; j < j1; ++j) {
-                        const double p = exp2(x[j - j0] - m + 6.0);
-                        l += p;
-                        const double pq = oracle_e4m3_round(p);
-                        const unsigned char* v = V + ((b * Ns + j) * H + h) * (long)D;
-                        for (int d = 0; d < D; ++d) acc[d] += pq * oracle_e4m3_decode(v[d]);
-                    }
-                }
+            /* scores in log2 units */
+            double mx = -INFINITY;
+            for (int j = 0; j < nval; ++j) {
+                const int seg = j >= Nv, jj = seg ? j - Nv : j, Ns = seg ? Nc : Nv;
+                const signed char* k = (seg ? kc : kv) + ((b * Ns + jj) * H + h) * (long)D;
+                const double skb = (seg ? skc : skv)[(b * H + h) * (long)(seg ? tc : tv) + jj / 128];
+                long dot = 0;
+                for (int d = 0; d < D; ++d) dot += (long)q[d] * (long)k[d];
+                x[j] = (double)dot * sq * skb * scale * log2e;
+                if (x[j] > mx) mx = x[j];
+            }
+            const double m = ceil(mx);
+            double l = 0.0;
+            for (int j = 0; j < nval; ++j) {
+                const int seg = j >= Nv, jj = seg ? j - Nv : j, Ns = seg ? Nc : Nv;
+                const double p = exp2(x[j] - m + 6.0);
+                l += p;
+                const double pq = oracle_e4m3_round(p);
+                const unsigned char* v = (seg ? vc : vv) + ((b * Ns + jj) * H + h) * (long)D;
+                for (int d = 0; d < D; ++d) acc[d] += pq * oracle_e4m3_decode(v[d]);
             }
             for (int d = 0; d < D; ++d) o[d] = acc[d] * sv[(b * H + h) * (long)D + d] / l;
         }

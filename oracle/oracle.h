@@ -38,6 +38,12 @@ void oracle_joint_attention_dq_rows(const double* qv, const double* kv, const do
                                     const int* ctx_len, const double* dov, const double* doc,
                                     int B, int Nv, int Nc, int H, int D, double scale,
                                     const long* rows, long nrows, double* dq_out, double* lse_out);
+void oracle_joint_attention_dkdv_rows(const double* qv, const double* kv, const double* vv,
+                                      const double* qc, const double* kc, const double* vc,
+                                      const int* ctx_len, const double* dov, const double* doc,
+                                      int B, int Nv, int Nc, int H, int D, double scale,
+                                      const long* keys, long nkeys, double* dk_out,
+                                      double* dv_out);
 void oracle_rmsnorm_rope_bwd(const double* x, const double* g, const double* dy,
                              const double* pos, double rope_base, const int* split,
                              long rows, int D, double eps, double* dx, double* dg);

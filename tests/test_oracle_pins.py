@@ -605,6 +605,11 @@ def pin_bwd_torch_autograd():
     _close(dq, gq[rows[:, 0], rows[:, 1], rows[:, 2]], 1e-12)
     _close(np.where(np.isinf(lse), 0, lse),
            np.where(np.isinf(want), 0, want)[rows[:, 0], rows[:, 1], rows[:, 2]], 1e-12)
+    # the key-row function gives autograd's dk and dv (zero on padded keys)
+    dk, dv = oracle.joint_attention_dkdv_rows(*t, dov, doc, cl, rows)
+    gk, gv = qkv[1].grad.numpy(), qkv[2].grad.numpy()
+    _close(dk, gk[rows[:, 0], rows[:, 1], rows[:, 2]], 1e-12)
+    _close(dv, gv[rows[:, 0], rows[:, 1], rows[:, 2]], 1e-12)
 
 
 @pin
@@ -846,7 +851,8 @@ def pin_q8_uniform_scores():
 @pin
 def pin_q8_brute():
     """The 8-bit method equals a numpy restatement (float32 quantisation,
-    torch E4M3 conversion, array softmax tiles) on ragged small inputs."""
+    torch E4M3 conversion, whole score vectors as matrix products) on ragged
+    small inputs."""
     r = RNG(73)
     B, Nv, Nc, H, D = 2, 300, 140, 2, 128
     t = [I.round_f64_to_bf16(r.standard_normal((B, n, H, D)) * sd)
@@ -860,17 +866,20 @@ def pin_q8_brute():
 
 @pin
 def pin_q8_close_to_exact():
-    """The 8-bit method stays close to the exact attention: max error under 8 %
-    of the largest output and mean error under 1 % of it on N(0,1) inputs."""
+    """The 8-bit method stays within its own rounding-error model of the exact
+    attention (tests/helpers.py: every element within 6 sigma of the error
+    that int8 scores and E4M3 rounding of P' and v allow, and a mean of
+    |error| / sigma at most 1), on N(0,1) inputs with ragged conditioning."""
+    from helpers import q8_close_to_exact, q8_exact_rows
     r = RNG(74)
-    B, Nv, Nc, H, D = 1, 400, 100, 2, 128
+    B, Nv, Nc, H, D = 2, 400, 100, 2, 128
     t = [I.round_f64_to_bf16(r.standard_normal((B, n, H, D))) for n in (Nv, Nv, Nv, Nc, Nc, Nc)]
-    ov, oc = oracle.attention_q8(t[0], t[1], t[2], t[3], t[4], t[5])
-    rv, rc = oracle.joint_attention(t[0], t[1], t[2], t[3], t[4], t[5])
-    got, ref = np.concatenate([ov, oc], 1), np.concatenate([rv, rc], 1)
-    mx = np.abs(ref).max()
-    assert np.abs(got - ref).max() <= 0.08 * mx
-    assert np.abs(got - ref).mean() <= 0.01 * mx
+    cl = np.array([100, 37], np.int32)
+    ov, oc = oracle.attention_q8(t[0], t[1], t[2], t[3], t[4], t[5], cl)
+    got = np.concatenate([ov, oc], 1)
+    trip = np.array([(b, h, i) for b in range(B) for h in range(H) for i in range(Nv + Nc)])
+    o, sig = q8_exact_rows(*t, cl, trip)
+    q8_close_to_exact(got[trip[:, 0], trip[:, 2], trip[:, 1]], o, sig, "q8 vs exact")
 
 
 @pytest.mark.parametrize("name", sorted(PINS))
@@ -918,6 +927,10 @@ MUTANTS = {
                                 "if (nk == 0) continue;"),
     "dqrows_no_delta": ("const double w = scale * s[j] * (g - Dsum);",
                         "const double w = scale * s[j] * g;"),
+    "dkdv_no_delta": ("const double dS = p * (dP - Dr[i]);", "const double dS = p * dP;"),
+    "dkdv_padded_queries_counted": (
+        "const int nval = Nv + L;    /* valid keys, and the query rows with an output */",
+        "const int nval = Nv + Nc;"),
     "nrbwd_rotation_not_transposed": ("u[off + 2 * j] = a0 * c + a1 * s;        /* transpose of the rotation */",
                                       "u[off + 2 * j] = a0 * c - a1 * s;"),
     "nrbwd_no_dot_term": ("dxr[d] = g[d] * u[d] / rr - xr[d] * dot / ((double)D * rr * rr * rr);",
@@ -925,12 +938,15 @@ MUTANTS = {
     "nrbwd_r_squared": ("dxr[d] = g[d] * u[d] / rr - xr[d] * dot / ((double)D * rr * rr * rr);",
                         "dxr[d] = g[d] * u[d] / rr - xr[d] * dot / ((double)D * rr * rr);"),
     "nrbwd_dg_no_norm": ("acc[d] += u[d] * xr[d] / rr;", "acc[d] += u[d] * xr[d];"),
-    "q8_no_offset": ("const double p = exp2(x[j - j0] - m + 6.0);",
-                     "const double p = exp2(x[j - j0] - m);"),
-    "q8_no_rescale": ("for (int d = 0; d < D; ++d) acc[d] *= f;", "(void)f;"),
+    "q8_no_offset": ("const double p = exp2(x[j] - m + 6.0);",
+                     "const double p = exp2(x[j] - m);"),
+    "q8_no_kscale": ("x[j] = (double)dot * sq * skb * scale * log2e;",
+                     "x[j] = (double)dot * sq * scale * log2e;"),
+    "q8_cond_kscale_block": ("[(b * H + h) * (long)(seg ? tc : tv) + jj / 128];",
+                             "[(b * H + h) * (long)(seg ? tc : tv) + j / 128];"),
     "q8_int8_step": ("const float s = amax / 127.0f;", "const float s = amax / 128.0f;"),
     "q8_v_scale": ("const float s = amax / 448.0f;", "const float s = amax / 256.0f;"),
-    "q8_sum_rounded": ("        l += p;\n", "        l += oracle_e4m3_round(p);\n"),
+    "q8_sum_rounded": ("                l += p;\n", "                l += oracle_e4m3_round(p);\n"),
     "q8_subnormal_step": ("        quantum = ldexp(1.0, -9);                               /* subnormal range */",
                           "        quantum = ldexp(1.0, -10);"),
     "modbwd_no_mean_g": ("dx[row + c] = rstd * (g - mg - xh[c] * mgx);",
