@@ -331,7 +331,9 @@ MMDIT_API int mmdit_joint_attention_bwd(const void* q_vis, const void* k_vis, co
  *   the GPU (different streams) race and must be ordered by the caller.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture. */
+ *   before any stream capture.  The address is kept for the life of the
+ *   process, so resetting a device (cudaDeviceReset) after that first call is
+ *   not supported: the kept address would then point into a released module. */
 MMDIT_API int mmdit_joint_attention_bwd_noalloc(
     const void* q_vis, const void* k_vis, const void* v_vis, const void* q_ctx, const void* k_ctx,
     const void* v_ctx, const int32_t* ctx_len, const void* o_vis, const void* o_ctx,
@@ -403,6 +405,23 @@ MMDIT_API int mmdit_joint_window_attention(const void* q_vis, const void* k_vis,
 MMDIT_API int mmdit_adaln_modulate(const void* x, const float* shift, const float* scale, void* y,
                          int B, int N, int C, float eps, mmdit_dtype dt, void* stream);
 
+/* mmdit_adaln_modulate of both streams of a block in ONE launch [Vimoo §2.2:
+ * each stream has its own LayerNorm and its own shift and scale]: rows of the
+ * visual stream use (shift_vis, scale_vis), rows of the conditioning stream
+ * (shift_ctx, scale_ctx).  The results equal two mmdit_adaln_modulate calls
+ * bit for bit; one launch keeps the short conditioning stream from costing a
+ * launch of its own.
+ *   x_vis, y_vis [B, N_vis, C] dt;  x_ctx, y_ctx [B, N_ctx, C] dt (y may
+ *   equal its own x); shift_*, scale_* [B, C] fp32.  N_vis or N_ctx may be 0
+ *   (that stream's pointers are then not read).  C, eps, dt as
+ *   mmdit_adaln_modulate.
+ * Errors: MMDIT_ERR_ARG / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_adaln_modulate_pair(const void* x_vis, const float* shift_vis,
+                                        const float* scale_vis, void* y_vis, int N_vis,
+                                        const void* x_ctx, const float* shift_ctx,
+                                        const float* scale_ctx, void* y_ctx, int N_ctx, int B,
+                                        int C, float eps, mmdit_dtype dt, void* stream);
+
 /* Gated residual [Vimoo §2.2: a per-channel gate from the timestep embedding
  * weighs each branch before it is added back to the residual stream]:
  *   out = x + gate[b] * branch.
@@ -463,14 +482,14 @@ MMDIT_API int mmdit_residual_modulate(const void* x, const void* branch, const f
  *
  * Runs the whole path of one block, step after step, from HOST buffers
  * [Vimoo §2.2, the dual-stream block]:
- *   y   = adaLN modulate of x                    (mmdit_adaln_modulate, both streams)
+ *   y   = adaLN modulate of x                    (mmdit_adaln_modulate_pair)
  *   q,k = QK-RMSNorm (+ 3D RoPE on the visual stream)   (mmdit_qk_norm_rope)
  *   o   = joint attention over both streams      (mmdit_joint_attention_ws)
  *   x'  = x + gate * o                           (mmdit_gated_residual, both streams)
  * The projections of a full block (QKV, output, MLP) are outside this library:
  * q, k, v arrive as inputs and the attention output is the gated branch.  Each
  * step is the same computation, with the same kernels and results, as these
- * seven calls made one after the other on device buffers (the attention with a
+ * six calls made one after the other on device buffers (the attention with a
  * workspace of MMDIT_ATTENTION_WORKSPACE_BYTES, which each slot holds).
  *
  * Unlike the rest of this header, the executor moves data between host and

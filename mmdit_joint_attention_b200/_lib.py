@@ -122,6 +122,8 @@ def lib():
                                                    [ctypes.POINTER(Grid), ctypes.POINTER(Window),
                                                     _f, _i, _vp])
         L.mmdit_adaln_modulate.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp]
+        L.mmdit_adaln_modulate_pair.argtypes = ([_vp] * 4 + [_i] + [_vp] * 4 + [_i] * 3 +
+                                                [_f, _i, _vp])
         L.mmdit_gated_residual.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
         L.mmdit_residual_modulate.argtypes = [_vp] * 7 + [_i, _i, _i, _f, _i, _vp]
         L.mmdit_adaln_modulate_bwd.argtypes = [_vp] * 6 + [_i, _i, _i, _f, _i, _vp]
@@ -145,7 +147,7 @@ def lib():
                      "mmdit_joint_attention_fwd", "mmdit_joint_attention_bwd",
                      "mmdit_joint_attention_ws", "mmdit_joint_attention_split_plan",
                      "mmdit_joint_window_attention", "mmdit_adaln_modulate",
-                     "mmdit_gated_residual", "mmdit_residual_modulate", "mmdit_device_status",
+                     "mmdit_adaln_modulate_pair", "mmdit_gated_residual", "mmdit_residual_modulate", "mmdit_device_status",
                      "mmdit_adaln_modulate_bwd", "mmdit_gated_residual_bwd",
                      "mmdit_block_forward_host"):
             getattr(L, name).restype = ctypes.c_int

@@ -447,6 +447,28 @@ def adaln_modulate(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
     return y
 
 
+def adaln_modulate_pair(x_vis: torch.Tensor, shift_vis: torch.Tensor, scale_vis: torch.Tensor,
+                        x_ctx: torch.Tensor, shift_ctx: torch.Tensor, scale_ctx: torch.Tensor,
+                        eps: float = 1e-6, out_vis: Optional[torch.Tensor] = None,
+                        out_ctx: Optional[torch.Tensor] = None,
+                        stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """adaln_modulate of the visual and the conditioning stream in one launch,
+    each with its own (shift, scale); same results as two calls."""
+    dt = _dtype(x_vis, x_ctx)
+    _f32(shift_vis, scale_vis, shift_ctx, scale_ctx)
+    B, Nv, C = x_vis.shape
+    Bc, Nc, Cc = x_ctx.shape
+    if (Bc, Cc) != (B, C):
+        raise ValueError("the two streams differ in batch or width")
+    y_vis = torch.empty_like(x_vis) if out_vis is None else out_vis
+    y_ctx = torch.empty_like(x_ctx) if out_ctx is None else out_ctx
+    st = _lib.lib().mmdit_adaln_modulate_pair(
+        _ptr(x_vis), _ptr(shift_vis), _ptr(scale_vis), _ptr(y_vis), Nv, _ptr(x_ctx),
+        _ptr(shift_ctx), _ptr(scale_ctx), _ptr(y_ctx), Nc, B, C, eps, dt, _stream(stream))
+    check("mmdit_adaln_modulate_pair", st)
+    return y_vis, y_ctx
+
+
 def gated_residual(x: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor,
                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """x + gate * branch (in place into x unless ``out`` is given)."""
@@ -519,7 +541,7 @@ def device_status(stream=None) -> int:
 def block_forward(t: dict, grid: Sequence[int], pos_scale=(1.0, 1.0, 1.0), eps: float = 1e-6,
                   stream=None, workspace: Optional[torch.Tensor] = None) -> dict:
     """One pass of the whole path on device tensors ``t`` (keys as produced by
-    ``inputs.make_inputs``): adaLN modulate of both streams (y_vis, y_ctx),
+    ``inputs.make_inputs``): adaLN modulate of both streams in one launch (y_vis, y_ctx),
     QK-RMSNorm (+ RoPE on the visual stream) in place on q/k, joint attention
     (o_vis, o_ctx), and the gated residual x += gate * o in place, with the
     attention output standing in for the branch (the projections around
@@ -531,9 +553,9 @@ def block_forward(t: dict, grid: Sequence[int], pos_scale=(1.0, 1.0, 1.0), eps: 
         workspace = attention_workspace(t["q_vis"].device)
     Nc = t["q_ctx"].shape[1]
     out = {}
-    for s in ("vis", "ctx"):
-        out["y_" + s] = adaln_modulate(t["x_" + s], t["shift_" + s], t["scale_" + s], eps,
-                                       out=t.get("y_" + s), stream=stream)
+    out["y_vis"], out["y_ctx"] = adaln_modulate_pair(
+        t["x_vis"], t["shift_vis"], t["scale_vis"], t["x_ctx"], t["shift_ctx"], t["scale_ctx"],
+        eps, out_vis=t.get("y_vis"), out_ctx=t.get("y_ctx"), stream=stream)
     qk_norm_rope(t["q_vis"], t["k_vis"], t["gq_vis"], t["gk_vis"], grid=grid,
                  pos_scale=pos_scale, eps=eps, stream=stream)
     qk_norm_rope(t["q_ctx"], t["k_ctx"], t["gq_ctx"], t["gk_ctx"], grid=None, eps=eps,
@@ -551,7 +573,7 @@ def block_forward(t: dict, grid: Sequence[int], pos_scale=(1.0, 1.0, 1.0), eps: 
 class BlockHostExecutor:
     """``block_forward``'s path run step after step from HOST tensors, through
     mmdit_block_forward_host: the library copies each step's inputs in, runs the
-    seven calls and copies the outputs back, overlapping the copies of some
+    six calls and copies the outputs back, overlapping the copies of some
     steps with the kernels of others on streams of its own.
 
     The device workspace (``slots`` slots, one step each) is allocated here

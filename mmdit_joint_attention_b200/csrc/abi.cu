@@ -531,6 +531,40 @@ int mmdit_adaln_modulate(const void* x, const float* shift, const float* scale, 
                        "adaln_modulate");
 }
 
+int mmdit_adaln_modulate_pair(const void* x_vis, const float* shift_vis, const float* scale_vis,
+                              void* y_vis, int N_vis, const void* x_ctx, const float* shift_ctx,
+                              const float* scale_ctx, void* y_ctx, int N_ctx, int B, int C,
+                              float eps, mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || N_vis < 0 || N_ctx < 0 || C < 0 || !(eps >= 0.f) ||
+        !std::isfinite(eps))
+        return MMDIT_ERR_ARG;
+    const int E = vec_elems(dt);
+    if (C == 0 || C % 8 != 0 || C / E > 512) return MMDIT_ERR_UNSUPPORTED;
+    if (B > 65535) return MMDIT_ERR_UNSUPPORTED;
+    ModStreamsHost h{};
+    const void* xs[2] = {x_vis, x_ctx};
+    void* ys[2] = {y_vis, y_ctx};
+    const float* shifts[2] = {shift_vis, shift_ctx};
+    const float* scales[2] = {scale_vis, scale_ctx};
+    const int Ns[2] = {N_vis, N_ctx};
+    for (int k = 0; k < 2; ++k) {
+        if ((long long)B * Ns[k] == 0) continue;
+        if (!xs[k] || !shifts[k] || !scales[k] || !ys[k]) return MMDIT_ERR_ARG;
+        if (!aligned16(xs[k]) || !aligned16(shifts[k]) || !aligned16(scales[k]) ||
+            !aligned16(ys[k]))
+            return MMDIT_ERR_ALIGN;
+        h.x[k] = xs[k];
+        h.y[k] = ys[k];
+        h.shift[k] = shifts[k];
+        h.scale[k] = scales[k];
+        h.N[k] = Ns[k];
+    }
+    // one launch holds at most 2^31 - 1 CTAs: far above B * (2 * #SMs)
+    return cuda_status(launch_adaln_modulate_pair(h, B, C, eps, dt == MMDIT_BF16,
+                                                  static_cast<cudaStream_t>(stream)),
+                       "adaln_modulate_pair");
+}
+
 int mmdit_gated_residual(const void* x, const void* branch, const float* gate, void* out, int B,
                          int N, int C, mmdit_dtype dt, void* stream) {
     if (!dtype_ok(dt) || B < 0 || N < 0 || C < 0) return MMDIT_ERR_ARG;

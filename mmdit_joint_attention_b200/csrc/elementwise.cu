@@ -13,6 +13,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 
@@ -663,17 +664,43 @@ __device__ __forceinline__ void mod_row(const uint4 (&raw)[CPL], T* y, size_t ro
     }
 }
 
+// The rows of up to two streams (the visual and the conditioning stream of a
+// block) in one launch: each CTA works on one (stream, sample) and stages that
+// pair's (1 + scale, shift) in shared memory.  A short stream (512 cond rows)
+// then rides along with the long one instead of paying a launch of its own.
+template <typename T>
+struct ModStreams {
+    const T* x[2];
+    T* y[2];
+    const float* shift[2];
+    const float* scale[2];
+    int N[2];    // rows per sample of each stream (0: stream absent)
+    int bx[2];   // CTAs per sample of each stream
+    int B;
+};
+
 // Two CTAs of 256 threads per SM (about 127 registers, 16 warps): measured
 // best at 480p among 1-3 CTAs per SM with and without double-buffered rows.
 template <typename T, int CPL>
 __global__ void __launch_bounds__(256, 2)
-adaln_modulate_kernel(const T* x, const float* __restrict__ shift,
-                      const float* __restrict__ scale, T* y, int N, int C, float eps) {
+adaln_modulate_kernel(const __grid_constant__ ModStreams<T> a, int C, float eps) {
     using L = ModLayout<T>;
     constexpr int E = L::E;
     constexpr int P = L::PIECES;
     extern __shared__ float4 mod[];
-    const int b = blockIdx.y;
+    int id = blockIdx.x;
+    int sidx = 0;
+    if (id >= a.B * a.bx[0]) {
+        id -= a.B * a.bx[0];
+        sidx = 1;
+    }
+    const int b = id / a.bx[sidx];
+    const int cx = id - b * a.bx[sidx];
+    const float* shift = a.shift[sidx];
+    const float* scale = a.scale[sidx];
+    const T* x = a.x[sidx];
+    T* y = a.y[sidx];
+    const int N = a.N[sidx];
     const int nch = C / E;
     for (int idx = threadIdx.x; idx < nch * P; idx += blockDim.x) {
         const int c = idx / P, k = idx - (idx / P) * P;
@@ -694,15 +721,14 @@ adaln_modulate_kernel(const T* x, const float* __restrict__ shift,
     const int lane = threadIdx.x & 31;
     const int warps = blockDim.x >> 5;
     const float invC = 1.0f / (float)C;
-    const int stride = gridDim.x * warps;
+    const int stride = a.bx[sidx] * warps;
     const size_t base = (size_t)b * N * (size_t)C;
-    int n = blockIdx.x * warps + (threadIdx.x >> 5);
+    int n = cx * warps + (threadIdx.x >> 5);
     for (; n < N; n += stride) {
         uint4 buf[CPL];
         mod_load<T, CPL>(buf, x, base + (size_t)n * C, nch, lane);
         mod_row<T, CPL>(buf, y, base + (size_t)n * C, nch, lane, invC, eps, mod);
     }
-
 }
 
 // Gated residual followed by the next adaLN modulate, one pass over memory:
@@ -797,8 +823,7 @@ cudaError_t run_residual_modulate(const void* x, const void* br, const float* ga
 }
 
 template <typename T, int CPL>
-cudaError_t run_modulate(const void* x, const float* shift, const float* scale, void* y, int B,
-                         int N, int C, float eps, cudaStream_t s) {
+cudaError_t run_modulate(const ModStreamsHost& h, int B, int C, float eps, cudaStream_t s) {
     auto kern = adaln_modulate_kernel<T, CPL>;
     const size_t smem = (size_t)C * 8;  // (1 + scale, shift) per column, fp32
     if (smem > 48 * 1024) {
@@ -810,13 +835,29 @@ cudaError_t run_modulate(const void* x, const float* shift, const float* scale, 
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
-    long long bx = ((long long)sm_count() * per_sm + B - 1) / B;
-    const long long need = (N + 7) / 8;
-    if (need < bx) bx = need;
-    if (bx < 1) bx = 1;
-    dim3 grid((unsigned)bx, (unsigned)B);
-    kern<<<grid, 256, smem, s>>>(static_cast<const T*>(x), shift, scale, static_cast<T*>(y), N, C,
-                                 eps);
+    ModStreams<T> a;
+    a.B = B;
+    // CTAs of one sample's share of a full wave, split between the streams in
+    // proportion to their rows; at least one CTA per present stream and at
+    // most one per 8 rows (a row per warp).
+    const long long per_sample = std::max<long long>(1, (long long)sm_count() * per_sm / B);
+    const long long rows = (long long)h.N[0] + h.N[1];
+    for (int k = 0; k < 2; ++k) {
+        a.x[k] = static_cast<const T*>(h.x[k]);
+        a.y[k] = static_cast<T*>(h.y[k]);
+        a.shift[k] = h.shift[k];
+        a.scale[k] = h.scale[k];
+        a.N[k] = h.N[k];
+        long long bx = 0;
+        if (h.N[k] > 0) {
+            bx = (long long)((double)per_sample * h.N[k] / (double)rows + 0.5);
+            bx = std::min<long long>(std::max<long long>(bx, 1), (h.N[k] + 7) / 8);
+        }
+        a.bx[k] = (int)bx;
+    }
+    const long long ctas = (long long)B * (a.bx[0] + a.bx[1]);
+    if (ctas == 0) return cudaSuccess;
+    kern<<<(unsigned)ctas, 256, smem, s>>>(a, C, eps);
     return cudaGetLastError();
 }
 
@@ -1069,16 +1110,15 @@ cudaError_t launch_qk_norm_rope_bwd(const void* q_in, const void* k_in, const vo
 #undef MMDIT_QK_BWD
 }
 
-cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float* scale,
-                                  void* y, int B, int N, int C, float eps, bool bf16,
-                                  cudaStream_t s) {
-    if ((long long)B * N == 0) return cudaSuccess;
+cudaError_t launch_adaln_modulate_pair(const ModStreamsHost& h, int B, int C, float eps,
+                                       bool bf16, cudaStream_t s) {
+    if ((long long)B * ((long long)h.N[0] + h.N[1]) == 0) return cudaSuccess;
     const int E = bf16 ? 8 : 4;
     const int cpl = (C / E + 31) / 32;
-#define MMDIT_MOD_CASE(V)                                                                 \
-    if (cpl <= V)                                                                         \
-        return bf16 ? run_modulate<__nv_bfloat16, V>(x, shift, scale, y, B, N, C, eps, s) \
-                    : run_modulate<float, V>(x, shift, scale, y, B, N, C, eps, s);
+#define MMDIT_MOD_CASE(V)                                                          \
+    if (cpl <= V)                                                                  \
+        return bf16 ? run_modulate<__nv_bfloat16, V>(h, B, C, eps, s)              \
+                    : run_modulate<float, V>(h, B, C, eps, s);
     MMDIT_MOD_CASE(1)
     MMDIT_MOD_CASE(2)
     MMDIT_MOD_CASE(4)
@@ -1087,6 +1127,18 @@ cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float
     MMDIT_MOD_CASE(16)
 #undef MMDIT_MOD_CASE
     return cudaErrorInvalidValue;  // the C-ABI layer rejects such C before this point
+}
+
+cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float* scale,
+                                  void* y, int B, int N, int C, float eps, bool bf16,
+                                  cudaStream_t s) {
+    ModStreamsHost h{};
+    h.x[0] = x;
+    h.y[0] = y;
+    h.shift[0] = shift;
+    h.scale[0] = scale;
+    h.N[0] = N;
+    return launch_adaln_modulate_pair(h, B, C, eps, bf16, s);
 }
 
 cudaError_t launch_residual_modulate(const void* x, const void* branch, const float* gate,

@@ -10,13 +10,14 @@
 // gated residual, out = x + gate[b] * branch, for the upstream gradient dout:
 //   dx = dout,  dbranch = gate[b] * dout,  dgate[b, c] = sum_n dout * branch
 //
-// One warp per row (the row's 16-byte chunks spread over the lanes and held
-// in registers between the passes), CTAs of one sample per grid row.  The
-// per-(b, c) sums are gathered per CTA in shared memory, then added to the
-// [B, C] outputs with one global atomic per column and CTA: the outputs are
-// zeroed first, and their last bits depend on the order of those atomics.
-// HBM-bound: modulate reads x and dy and writes dx; residual reads branch
-// and dout and writes dbranch (and dx when asked for: it equals dout).
+// A CTA works on one sample; each thread owns one 16-byte column chunk of all
+// the CTA's rows, so the per-(b, c) sums stay in registers and are added to
+// the [B, C] outputs with one global atomic per column and CTA at the end: the
+// outputs are zeroed first, and their last bits depend on the order of those
+// atomics.  The LayerNorm statistics of a row are CTA-wide sums, taken for
+// several rows at once.  HBM-bound: modulate reads x and dy and writes dx;
+// residual reads branch and dout and writes dbranch (and dx when asked for:
+// it equals dout).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -28,8 +29,6 @@
 
 namespace mmdit {
 namespace {
-
-constexpr int kThreads = 256;   // 8 warps, one row each at a time
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8], __nv_bfloat16) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -74,138 +73,181 @@ __host__ __device__ constexpr int chunk_elems() {
     return 16 / (int)sizeof(T);
 }
 
+// Layout of both kernels: a CTA works on one sample and owns a set of rows,
+// kRows at a time; thread t owns the 16-byte column chunk t of every one of
+// those rows (blockDim = the chunks of a row rounded up to a warp).  The
+// per-column sums (dshift / dscale, dgate) therefore stay in the owning
+// thread's registers over all of the CTA's rows, and reach the [B, C] output
+// with one global atomic per column and CTA at the end.  kRows rows are loaded
+// before any is used, so a CTA keeps kRows rows of loads in flight.
+constexpr int kRows = 4;
+
+// Sum over the CTA of V values per thread; every thread gets the totals.
+// red: shared scratch of (warps * V) floats, one array per call site so that
+// consecutive reductions never overwrite values still being read.
+template <int V>
+__device__ __forceinline__ void cta_sum(float (&v)[V], float* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, warps = blockDim.x >> 5;
+#pragma unroll
+    for (int k = 0; k < V; ++k) v[k] = warp_sum(v[k]);
+    if (lane == 0)
+#pragma unroll
+        for (int k = 0; k < V; ++k) red[warp * V + k] = v[k];
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < V; ++k) v[k] = 0.f;
+    for (int w = 0; w < warps; ++w)
+#pragma unroll
+        for (int k = 0; k < V; ++k) v[k] += red[w * V + k];
+}
+
 // ---------------------------------------------------------------- modulate bwd
-template <typename T, int CPL>
-__global__ void __launch_bounds__(kThreads)
+// Per row: both moments in one pass, shifted by the row's first element (so a
+// large common offset does not cancel), one CTA reduction for the kRows rows
+// of an iteration; then mean_c(g) and mean_c(g * xh), a second reduction.
+// MAXT: the largest block the instantiation serves (384 threads leave room
+// for 168 registers a thread, which C <= 3072 bf16 needs without spilling).
+template <typename T, int MAXT>
+__global__ void __launch_bounds__(MAXT)
 adaln_modulate_bwd_kernel(const T* x, const float* __restrict__ scale, const T* dy, T* dx,
                           float* dshift, float* dscale, int N, int C, float eps) {
     constexpr int E = chunk_elems<T>();
-    extern __shared__ float acc[];          // [0, C): dshift part, [C, 2C): dscale part
+    __shared__ float red0[16 * 2 * kRows], red1[16 * 2 * kRows];
     const int b = blockIdx.y;
-    for (int i = threadIdx.x; i < 2 * C; i += kThreads) acc[i] = 0.f;
-    __syncthreads();
-    const int lane = threadIdx.x & 31;
-    const int nch = C / E;
+    const int c = threadIdx.x;               // this thread's chunk
+    const bool own = c < C / E;
     const float invC = 1.f / (float)C;
-    const float* sc = scale + (size_t)b * C;
-    for (int n = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); n < N;
-         n += gridDim.x * (kThreads / 32)) {
-        const size_t row = ((size_t)b * N + n) * (size_t)C;
-        uint4 rx[CPL], rd[CPL];
+    float sc1[E], ash[E], asc[E];            // 1 + scale, dshift and dscale partials
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int c = lane + 32 * i;
-            if (c < nch) {
-                rx[i] = *reinterpret_cast<const uint4*>(x + row + (size_t)c * E);
-                rd[i] = *reinterpret_cast<const uint4*>(dy + row + (size_t)c * E);
+    for (int e = 0; e < E; ++e) {
+        sc1[e] = own ? 1.f + __ldg(scale + (size_t)b * C + c * E + e) : 0.f;
+        ash[e] = 0.f;
+        asc[e] = 0.f;
+    }
+    const size_t sample = (size_t)b * N * (size_t)C;
+    for (int n0 = blockIdx.x * kRows; n0 < N; n0 += gridDim.x * kRows) {
+        uint4 rx[kRows], rd[kRows];
+        float pivot[kRows];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+            const bool row_ok = n0 + r < N;
+            const size_t row = sample + (size_t)(row_ok ? n0 + r : n0) * C;
+            rx[r] = make_uint4(0, 0, 0, 0);
+            rd[r] = make_uint4(0, 0, 0, 0);
+            if (own && row_ok) {
+                rx[r] = *reinterpret_cast<const uint4*>(x + row + (size_t)c * E);
+                rd[r] = *reinterpret_cast<const uint4*>(dy + row + (size_t)c * E);
             }
+            pivot[r] = row_ok ? (float)x[row] : 0.f;
         }
-        // mean, then the centred sum of squares (two passes over the registers)
-        float s = 0.f;
+        float st[2 * kRows];                 // per row: sum(x - p), sum((x - p)^2)
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            if (lane + 32 * i < nch) {
-                float f[8];
-                unpack8(rx[i], f, T());
+        for (int r = 0; r < kRows; ++r) {
+            float f[8];
+            unpack8(rx[r], f, T());
+            float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-                for (int e = 0; e < E; ++e) s += f[e];
+            for (int e = 0; e < E; ++e) {
+                const float d = own ? f[e] - pivot[r] : 0.f;
+                s1 += d;
+                s2 = fmaf(d, d, s2);
             }
+            st[2 * r] = s1;
+            st[2 * r + 1] = s2;
         }
-        const float mean = warp_sum(s) * invC;
-        float ss = 0.f;
+        cta_sum(st, red0);
+        float mean[kRows], rstd[kRows], gm[2 * kRows];   // gm: per row sum(g), sum(g * xh)
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            if (lane + 32 * i < nch) {
-                float f[8];
-                unpack8(rx[i], f, T());
+        for (int r = 0; r < kRows; ++r) {
+            const float dm = st[2 * r] * invC;
+            mean[r] = pivot[r] + dm;
+            rstd[r] = rsqrtf(fmaxf(st[2 * r + 1] * invC - dm * dm, 0.f) + eps);
+            float fx[8], fd[8];
+            unpack8(rx[r], fx, T());
+            unpack8(rd[r], fd, T());
+            float a = 0.f, bgx = 0.f;
 #pragma unroll
-                for (int e = 0; e < E; ++e) ss += (f[e] - mean) * (f[e] - mean);
+            for (int e = 0; e < E; ++e) {
+                const float xh = (fx[e] - mean[r]) * rstd[r];
+                const float g = fd[e] * sc1[e];
+                a += g;
+                bgx = fmaf(g, xh, bgx);
             }
+            gm[2 * r] = a;
+            gm[2 * r + 1] = bgx;
         }
-        const float rstd = rsqrtf(warp_sum(ss) * invC + eps);
-        // mean_c(g), mean_c(g * xh), and this row's share of dshift / dscale
-        float mg = 0.f, mgx = 0.f;
+        cta_sum(gm, red1);
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int c = lane + 32 * i;
-            if (c < nch) {
-                float fx[8], fd[8];
-                unpack8(rx[i], fx, T());
-                unpack8(rd[i], fd, T());
+        for (int r = 0; r < kRows; ++r) {
+            if (!own || n0 + r >= N) continue;
+            const float mg = gm[2 * r] * invC, mgx = gm[2 * r + 1] * invC;
+            float fx[8], fd[8], o[8];
+            unpack8(rx[r], fx, T());
+            unpack8(rd[r], fd, T());
 #pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const float xh = (fx[e] - mean) * rstd;
-                    const float g = fd[e] * (1.f + __ldg(sc + c * E + e));
-                    mg += g;
-                    mgx += g * xh;
-                    atomicAdd(&acc[c * E + e], fd[e]);
-                    atomicAdd(&acc[C + c * E + e], fd[e] * xh);
-                }
+            for (int e = 0; e < E; ++e) {
+                const float xh = (fx[e] - mean[r]) * rstd[r];
+                o[e] = rstd[r] * (fd[e] * sc1[e] - mg - xh * mgx);
+                ash[e] += fd[e];
+                asc[e] = fmaf(fd[e], xh, asc[e]);
             }
-        }
-        mg = warp_sum(mg) * invC;
-        mgx = warp_sum(mgx) * invC;
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int c = lane + 32 * i;
-            if (c < nch) {
-                float fx[8], fd[8], o[8];
-                unpack8(rx[i], fx, T());
-                unpack8(rd[i], fd, T());
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const float xh = (fx[e] - mean) * rstd;
-                    const float g = fd[e] * (1.f + __ldg(sc + c * E + e));
-                    o[e] = rstd * (g - mg - xh * mgx);
-                }
-                *reinterpret_cast<uint4*>(dx + row + (size_t)c * E) = pack8(o, T());
-            }
+            *reinterpret_cast<uint4*>(dx + sample + (size_t)(n0 + r) * C + (size_t)c * E) =
+                pack8(o, T());
         }
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < C; i += kThreads) {
-        atomicAdd(dshift + (size_t)b * C + i, acc[i]);
-        atomicAdd(dscale + (size_t)b * C + i, acc[C + i]);
+    if (own) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            atomicAdd(dshift + (size_t)b * C + c * E + e, ash[e]);
+            atomicAdd(dscale + (size_t)b * C + c * E + e, asc[e]);
+        }
     }
 }
 
 // ---------------------------------------------------------------- residual bwd
-template <typename T, int CPL>
-__global__ void __launch_bounds__(kThreads)
+template <typename T>
+__global__ void __launch_bounds__(512)
 gated_residual_bwd_kernel(const T* branch, const float* __restrict__ gate, const T* dout,
                           T* dx, T* dbranch, float* dgate, int N, int C) {
     constexpr int E = chunk_elems<T>();
-    extern __shared__ float acc[];          // [0, C): dgate part
     const int b = blockIdx.y;
-    for (int i = threadIdx.x; i < C; i += kThreads) acc[i] = 0.f;
-    __syncthreads();
-    const int lane = threadIdx.x & 31;
-    const int nch = C / E;
-    const float* gt = gate + (size_t)b * C;
-    for (int n = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); n < N;
-         n += gridDim.x * (kThreads / 32)) {
-        const size_t row = ((size_t)b * N + n) * (size_t)C;
+    const int c = threadIdx.x;
+    if (c >= C / E) return;                 // no barrier below: idle threads may leave
+    float g[E], acc[E];
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int c = lane + 32 * i;
-            if (c < nch) {
-                const uint4 rb = *reinterpret_cast<const uint4*>(branch + row + (size_t)c * E);
-                const uint4 rd = *reinterpret_cast<const uint4*>(dout + row + (size_t)c * E);
-                float fb[8], fd[8], o[8];
-                unpack8(rb, fb, T());
-                unpack8(rd, fd, T());
+    for (int e = 0; e < E; ++e) {
+        g[e] = __ldg(gate + (size_t)b * C + c * E + e);
+        acc[e] = 0.f;
+    }
+    const size_t sample = (size_t)b * N * (size_t)C;
+    for (int n0 = blockIdx.x * kRows; n0 < N; n0 += gridDim.x * kRows) {
+        uint4 rb[kRows], rd[kRows];
 #pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    o[e] = __ldg(gt + c * E + e) * fd[e];
-                    atomicAdd(&acc[c * E + e], fd[e] * fb[e]);
-                }
-                *reinterpret_cast<uint4*>(dbranch + row + (size_t)c * E) = pack8(o, T());
-                if (dx) *reinterpret_cast<uint4*>(dx + row + (size_t)c * E) = rd;
+        for (int r = 0; r < kRows; ++r) {
+            if (n0 + r < N) {
+                const size_t at = sample + (size_t)(n0 + r) * C + (size_t)c * E;
+                rb[r] = *reinterpret_cast<const uint4*>(branch + at);
+                rd[r] = *reinterpret_cast<const uint4*>(dout + at);
             }
         }
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+            if (n0 + r >= N) continue;
+            const size_t at = sample + (size_t)(n0 + r) * C + (size_t)c * E;
+            float fb[8], fd[8], o[8];
+            unpack8(rb[r], fb, T());
+            unpack8(rd[r], fd, T());
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                o[e] = g[e] * fd[e];
+                acc[e] = fmaf(fd[e], fb[e], acc[e]);
+            }
+            *reinterpret_cast<uint4*>(dbranch + at) = pack8(o, T());
+            if (dx) *reinterpret_cast<uint4*>(dx + at) = rd[r];
+        }
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < C; i += kThreads) atomicAdd(dgate + (size_t)b * C + i, acc[i]);
+#pragma unroll
+    for (int e = 0; e < E; ++e) atomicAdd(dgate + (size_t)b * C + c * E + e, acc[e]);
 }
 
 int num_sms() {
@@ -220,63 +262,51 @@ int num_sms() {
     return cached[dev];
 }
 
-// CTAs per sample: two per SM over the whole grid, no more than the rows need.
-dim3 grid_for(int B, int N) {
-    long long bx = ((long long)num_sms() * 2 + B - 1) / B;
-    const long long need = ((long long)N + 7) / 8;
+// Threads of a CTA: one per 16-byte chunk of a row, rounded up to a warp.
+int threads_for(int C, int E) { return ((C / E + 31) / 32) * 32; }
+
+// CTAs per sample: as many as the SMs hold at once (occupancy of the kernel at
+// this block size), but at least 4 * kRows rows per CTA so that the final
+// atomics stay few against the rows.
+template <typename K>
+cudaError_t grid_for(K kern, int threads, int B, int N, dim3& grid) {
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
+    if (e != cudaSuccess) return e;
+    long long bx = ((long long)num_sms() * (per_sm > 0 ? per_sm : 1) + B - 1) / B;
+    const long long need = ((long long)N + 4 * kRows - 1) / (4 * kRows);
     if (need < bx) bx = need;
     if (bx < 1) bx = 1;
-    return dim3((unsigned)bx, (unsigned)B);
-}
-
-template <typename T, int CPL>
-cudaError_t run_modulate_bwd(const void* x, const float* scale, const void* dy, void* dx,
-                             float* dshift, float* dscale, int B, int N, int C, float eps,
-                             cudaStream_t s) {
-    const size_t smem = (size_t)C * 8;
-    adaln_modulate_bwd_kernel<T, CPL><<<grid_for(B, N), kThreads, smem, s>>>(
-        static_cast<const T*>(x), scale, static_cast<const T*>(dy), static_cast<T*>(dx),
-        dshift, dscale, N, C, eps);
-    return cudaGetLastError();
-}
-
-template <typename T, int CPL>
-cudaError_t run_residual_bwd(const void* br, const float* gate, const void* dout, void* dx,
-                             void* dbr, float* dgate, int B, int N, int C, cudaStream_t s) {
-    const size_t smem = (size_t)C * 4;
-    gated_residual_bwd_kernel<T, CPL><<<grid_for(B, N), kThreads, smem, s>>>(
-        static_cast<const T*>(br), gate, static_cast<const T*>(dout), static_cast<T*>(dx),
-        static_cast<T*>(dbr), dgate, N, C);
-    return cudaGetLastError();
-}
-
-// Chunks of 16 bytes per lane, rounded up to a compiled width.
-int cpl_for(int nch) {
-    const int need = (nch + 31) / 32;
-    return need <= 4 ? 4 : need <= 8 ? 8 : need <= 12 ? 12 : 16;
+    grid = dim3((unsigned)bx, (unsigned)B);
+    return cudaSuccess;
 }
 
 template <typename T>
 cudaError_t dispatch_modulate_bwd(const void* x, const float* scale, const void* dy, void* dx,
                                   float* dshift, float* dscale, int B, int N, int C, float eps,
                                   cudaStream_t s) {
-    switch (cpl_for(C / chunk_elems<T>())) {
-        case 4: return run_modulate_bwd<T, 4>(x, scale, dy, dx, dshift, dscale, B, N, C, eps, s);
-        case 8: return run_modulate_bwd<T, 8>(x, scale, dy, dx, dshift, dscale, B, N, C, eps, s);
-        case 12: return run_modulate_bwd<T, 12>(x, scale, dy, dx, dshift, dscale, B, N, C, eps, s);
-        default: return run_modulate_bwd<T, 16>(x, scale, dy, dx, dshift, dscale, B, N, C, eps, s);
-    }
+    const int threads = threads_for(C, chunk_elems<T>());
+    auto kern = threads <= 384 ? adaln_modulate_bwd_kernel<T, 384>
+                               : adaln_modulate_bwd_kernel<T, 512>;
+    dim3 grid;
+    cudaError_t e = grid_for(kern, threads, B, N, grid);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, threads, 0, s>>>(static_cast<const T*>(x), scale, static_cast<const T*>(dy),
+                                  static_cast<T*>(dx), dshift, dscale, N, C, eps);
+    return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t dispatch_residual_bwd(const void* br, const float* gate, const void* dout, void* dx,
                                   void* dbr, float* dgate, int B, int N, int C, cudaStream_t s) {
-    switch (cpl_for(C / chunk_elems<T>())) {
-        case 4: return run_residual_bwd<T, 4>(br, gate, dout, dx, dbr, dgate, B, N, C, s);
-        case 8: return run_residual_bwd<T, 8>(br, gate, dout, dx, dbr, dgate, B, N, C, s);
-        case 12: return run_residual_bwd<T, 12>(br, gate, dout, dx, dbr, dgate, B, N, C, s);
-        default: return run_residual_bwd<T, 16>(br, gate, dout, dx, dbr, dgate, B, N, C, s);
-    }
+    const int threads = threads_for(C, chunk_elems<T>());
+    dim3 grid;
+    cudaError_t e = grid_for(gated_residual_bwd_kernel<T>, threads, B, N, grid);
+    if (e != cudaSuccess) return e;
+    gated_residual_bwd_kernel<T><<<grid, threads, 0, s>>>(
+        static_cast<const T*>(br), gate, static_cast<const T*>(dout), static_cast<T*>(dx),
+        static_cast<T*>(dbr), dgate, N, C);
+    return cudaGetLastError();
 }
 
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -320,7 +350,10 @@ extern "C" int mmdit_adaln_modulate_bwd(const void* x, const float* scale, const
         if (!x || !dy || !dx) return MMDIT_ERR_ARG;
         if (!al16(x) || !al16(dy) || !al16(dx)) return MMDIT_ERR_ALIGN;
         const size_t bytes = (size_t)B * N * C * (dt == MMDIT_BF16 ? 2 : 4);
-        if (overlaps(dx, x, bytes)) return MMDIT_ERR_ARG;   // dx may replace dy, not x
+        // dx may replace dy exactly (a thread reads its chunks of a row before
+        // writing them), but must not overlap x or be shifted against dy
+        if (overlaps(dx, x, bytes) || (dx != dy && overlaps(dx, dy, bytes)))
+            return MMDIT_ERR_ARG;
     }
     cudaError_t e = cudaMemsetAsync(dshift, 0, vec, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(dscale, 0, vec, s);
@@ -346,7 +379,12 @@ extern "C" int mmdit_gated_residual_bwd(const void* branch, const float* gate, c
         if (!al16(branch) || !al16(dout) || !al16(dbranch) || (dx && !al16(dx)))
             return MMDIT_ERR_ALIGN;
         const size_t bytes = (size_t)B * N * C * (dt == MMDIT_BF16 ? 2 : 4);
-        if (overlaps(dbranch, branch, bytes) || (dx && overlaps(dx, branch, bytes)))
+        // outputs: not over branch, not over each other, and over dout only
+        // exactly (a thread reads its chunk of dout before writing there)
+        if (overlaps(dbranch, branch, bytes) || (dx && overlaps(dx, branch, bytes)) ||
+            (dx && overlaps(dx, dbranch, bytes)) ||
+            (dbranch != dout && overlaps(dbranch, dout, bytes)) ||
+            (dx && dx != dout && overlaps(dx, dout, bytes)))
             return MMDIT_ERR_ARG;
     }
     cudaError_t e = cudaMemsetAsync(dgate, 0, (size_t)B * C * sizeof(float), s);

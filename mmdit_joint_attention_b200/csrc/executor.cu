@@ -2,8 +2,8 @@
 // buffers, with the copies in, the kernels and the copies out of different
 // steps overlapped on three streams.
 //
-// A step is seven calls of the device entry points, in this order: adaLN
-// modulate of both streams, QK-RMSNorm + RoPE of both streams (in place), the
+// A step is six calls of the device entry points, in this order: adaLN
+// modulate of both streams (one launch), QK-RMSNorm + RoPE of both streams (in place), the
 // joint attention (with its split-tail workspace), and the gated residual of
 // both streams (in place on x).  Every buffer a step touches on the device
 // lives in its slot of the workspace:
@@ -58,7 +58,7 @@ long long round256(long long n) { return (n + 255) & ~255LL; }
 bool aligned(const void* p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // MMDIT_OK and the layout, or the MMDIT_ERR_* code of an invalid configuration.
-// Covers every check the seven entry points make on sizes and constants, so
+// Covers every check the six entry points make on sizes and constants, so
 // that a step cannot fail validation half-way through the enqueue.
 int check_config(const mmdit_block_config* c, SlotLayout& L) {
     if (!c) return MMDIT_ERR_ARG;
@@ -241,10 +241,11 @@ extern "C" int mmdit_block_forward_host(const mmdit_block_config* cfg,
         // ---- kernels
         if ((e = cudaStreamWaitEvent(h.cmp, h.ready[k], 0)) != cudaSuccess) break;
         void* cs = static_cast<void*>(h.cmp);
-        for (int s = 0; s < 2 && status == MMDIT_OK; ++s)
-            if (N[s] > 0)
-                status = mmdit_adaln_modulate(dev(L.x[s]), devf(L.shift[s]), devf(L.scale[s]),
-                                              dev(L.y[s]), B, N[s], C, c.ln_eps, c.dt, cs);
+        status = mmdit_adaln_modulate_pair(
+            dev(L.x[0]), devf(L.shift[0]), devf(L.scale[0]), dev(L.y[0]), N[0],
+            has_ctx ? dev(L.x[1]) : nullptr, has_ctx ? devf(L.shift[1]) : nullptr,
+            has_ctx ? devf(L.scale[1]) : nullptr, has_ctx ? dev(L.y[1]) : nullptr, N[1], B, C,
+            c.ln_eps, c.dt, cs);
         if (status != MMDIT_OK) break;
         if ((e = cudaEventRecord(h.y_done[k], h.cmp)) != cudaSuccess) break;
         status = mmdit_qk_norm_rope(dev(L.q[0]), dev(L.k[0]), dev(L.q[0]), dev(L.k[0]), c.gq_vis,

@@ -54,6 +54,18 @@ cudaError_t launch_adaln_modulate(const void* x, const float* shift, const float
                                   void* y, int B, int N, int C, float eps, bool bf16,
                                   cudaStream_t s);
 
+// The adaLN modulate of two streams (index 0 visual, 1 conditioning) with the
+// same B and C in one launch; a stream with N == 0 is absent.
+struct ModStreamsHost {
+    const void* x[2];
+    void* y[2];
+    const float* shift[2];
+    const float* scale[2];
+    int N[2];
+};
+cudaError_t launch_adaln_modulate_pair(const ModStreamsHost& h, int B, int C, float eps,
+                                       bool bf16, cudaStream_t s);
+
 cudaError_t launch_residual_modulate(const void* x, const void* branch, const float* gate,
                                      const float* shift, const float* scale, void* x_out, void* y,
                                      int B, int N, int C, float eps, bool bf16, cudaStream_t s);

@@ -20,7 +20,8 @@
 // Host code cannot use the array's name as a device address: the device
 // address comes from cudaGetSymbolAddress, done once per device by the first
 // call made with that device current.  That first call should therefore come
-// before any stream capture.
+// before any stream capture.  The address is kept until the process exits: a
+// device reset after the first call is not supported.
 #include <cuda_runtime.h>
 
 #include <cstdint>

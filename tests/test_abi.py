@@ -72,6 +72,20 @@ def test_modulate_residual_validation(L):
     assert r(P, P, None, P, 1, 4, 3072, 1, None) == -1
     assert r(P, P, P, U, 1, 4, 3072, 1, None) == -3
     assert r(P, P, P, P, 1, 0, 3072, 1, None) == 0
+    # both streams in one launch: x, shift, scale, y, N for each stream, then B, C
+    mp = L.mmdit_adaln_modulate_pair
+    assert mp(P, P, P, P, 4, P, P, P, P, 2, 1, 3070, 1e-6, 1, None) == -4    # C % 8
+    assert mp(P, P, P, P, 4, P, P, P, P, 2, 1, 8192, 1e-6, 1, None) == -4    # register budget
+    assert mp(P, P, P, P, -1, P, P, P, P, 2, 1, 3072, 1e-6, 1, None) == -1   # N_vis < 0
+    assert mp(P, P, P, P, 4, P, P, P, P, -2, 1, 3072, 1e-6, 1, None) == -1   # N_ctx < 0
+    assert mp(P, P, P, P, 4, P, P, P, P, 2, 1, 3072, -1.0, 1, None) == -1    # eps
+    assert mp(P, P, P, P, 4, P, P, P, P, 2, 1, 3072, 1e-6, 7, None) == -1    # dtype
+    assert mp(P, P, P, P, 4, P, None, P, P, 2, 1, 3072, 1e-6, 1, None) == -1  # ctx shift
+    assert mp(P, P, P, U, 4, P, P, P, P, 2, 1, 3072, 1e-6, 1, None) == -3    # y_vis unaligned
+    assert mp(P, P, P, P, 4, U, P, P, P, 2, 1, 3072, 1e-6, 1, None) == -3    # x_ctx unaligned
+    assert mp(None, None, None, None, 0, None, None, None, None, 0, 1, 3072, 1e-6, 1,
+              None) == 0                                                      # both empty
+    assert mp(P, P, P, P, 4, P, P, P, P, 2, 0, 3072, 1e-6, 1, None) == 0     # B = 0
 
 
 def test_residual_modulate_validation(L):
@@ -325,6 +339,8 @@ def test_elementwise_bwd_validation(L):
     assert fm(P, P, P, ctypes.c_void_p(4097), P, P, 1, 4, 64, 1e-6, 1, None) == -3
     assert fm(P, P, P, P, ctypes.c_void_p(4096), P, 1, 4, 64, 1e-6, 1, None) == -1   # dx aliases x
     assert fm(None, None, None, None, None, None, 0, 4, 64, 1e-6, 1, None) == 0      # B = 0
+    dy0, dy16 = ctypes.c_void_p(8192), ctypes.c_void_p(8192 + 16)
+    assert fm(P, P, dy0, dy16, P, P, 1, 4, 64, 1e-6, 1, None) == -1   # dx shifted against dy
     # residual: branch, gate, dout, dx, dbranch, dgate, B, N, C, dt, stream
     assert fr(P, P, P, None, ctypes.c_void_p(4096), P, 1, 4, 60, 1, None) == -4
     assert fr(P, None, P, None, ctypes.c_void_p(4096), P, 1, 4, 64, 1, None) == -1
@@ -332,3 +348,8 @@ def test_elementwise_bwd_validation(L):
     assert fr(P, P, P, ctypes.c_void_p(18), ctypes.c_void_p(4096), P, 1, 4, 64, 1, None) == -3
     assert fr(P, P, P, None, P, P, 1, 4, 64, 1, None) == -1                          # dbranch aliases branch
     assert fr(None, None, None, None, None, None, 0, 4, 64, 1, None) == 0
+    do0, a0, a16 = ctypes.c_void_p(8192), ctypes.c_void_p(16384), ctypes.c_void_p(16384 + 16)
+    assert fr(P, P, do0, a0, a16, P, 1, 4, 64, 1, None) == -1   # dx overlaps dbranch
+    assert fr(P, P, do0, a0, a0, P, 1, 4, 64, 1, None) == -1    # dx is dbranch
+    assert fr(P, P, do0, None, ctypes.c_void_p(8192 + 16), P, 1, 4, 64, 1, None) == -1
+    assert fr(P, P, do0, ctypes.c_void_p(8192 + 32), a0, P, 1, 4, 64, 1, None) == -1

@@ -4,7 +4,8 @@ inputs and upstream gradients.
 
 Small and medium cases compare every gradient element; the full 480p and
 ragged workloads compare dq and lse on sampled query rows (each against the
-full key set) and dk / dv through sum rules that hold at any size."""
+full key set), dk and dv on sampled key rows of a few heads (each against every
+query row), and dk / dv of every key through sum rules that hold at any size."""
 import numpy as np
 import pytest
 import torch
@@ -94,6 +95,27 @@ def test_backward_sampled_full_size(name):
     parity(got[vis], dq[vis], w.dtype, f"{name} dq_vis rows")
     parity(got[~vis], dq[~vis], w.dtype, f"{name} dq_ctx rows")
     _check_lse(lse[trip[:, 0], trip[:, 1], trip[:, 2]], lref, f"{name} lse rows")
+    # dk and dv element by element on sampled key rows (the query-row sampler
+    # applied to keys: every cond key, both visual tails, the tile and padding
+    # boundaries, 128 random keys), 2 heads at 480p and 1 head per sample of
+    # the ragged batch; each key against every query row
+    heads = {"480p": [(0, 0), (0, 17)], "ragged": [(0, 5), (1, 11)]}[name]
+    keys = []
+    for b, h in heads:
+        rows = I.parity_rows(w, b, h, n_random=128)
+        keys.append(np.stack([np.full_like(rows, b), np.full_like(rows, h), rows], axis=1))
+    keys = np.concatenate(keys)
+    dk, dv = oracle.joint_attention_dkdv_rows(
+        inp["q_vis"].f64, inp["k_vis"].f64, inp["v_vis"].f64, inp["q_ctx"].f64,
+        inp["k_ctx"].f64, inp["v_ctx"].f64, gin["do_vis"].f64, gin["do_ctx"].f64,
+        inp["ctx_len"], keys)
+    vis = keys[:, 2] < w.Nv
+    for grad, ref, n in ((g["dk_vis"], g["dk_ctx"], "dk"), (g["dv_vis"], g["dv_ctx"], "dv")):
+        full = np.concatenate([grad, ref], axis=1)
+        got = full[keys[:, 0], keys[:, 2], keys[:, 1]]
+        want = dk if n == "dk" else dv
+        parity(got[vis], want[vis], w.dtype, f"{name} {n}_vis keys")
+        parity(got[~vis], want[~vis], w.dtype, f"{name} {n}_ctx keys")
     # Sum rules, per (sample, head, dim): softmax rows sum to one, so
     # sum_j dv_j = sum_i dO_i over rows with an output, and sum_j dS_ij = 0, so
     # sum_j dk_j = 0.  Two bf16 roundings of random sign (P before the dV

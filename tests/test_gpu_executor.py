@@ -1,7 +1,7 @@
 """mmdit_block_forward_host, the host-buffer executor: several steps from and
 to host buffers, pipelined over the library's own streams and a workspace of
 one or more slots.  Each step's outputs must equal, bit for bit, the same
-seven calls run on device buffers (api.block_forward), and match the
+six calls run on device buffers (api.block_forward), and match the
 oracle's whole-path result within the stated tolerances."""
 import dataclasses
 

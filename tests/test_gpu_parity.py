@@ -60,10 +60,15 @@ def test_qk_norm_rope_odd_grid_and_base():
 
 # ---------------------------------------------------------------- modulate / residual
 
-@pytest.mark.parametrize("name", ["tiny", "block", "480p", "ragged"])
+@pytest.mark.parametrize("name", ["tiny", "block", "480p", "720p", "ragged"])
 def test_modulate_and_residual(name):
     w = W[name]
     inp = I.make_inputs(w, parts=("qkv", "adaln"))
+    # both streams in one launch: bit-equal to one launch per stream
+    yv, yc = api.adaln_modulate_pair(
+        to_dev(inp["x_vis"]), to_dev(inp["shift_vis"]), to_dev(inp["scale_vis"]),
+        to_dev(inp["x_ctx"]), to_dev(inp["shift_ctx"]), to_dev(inp["scale_ctx"]))
+    pair = {"vis": yv, "ctx": yc}
     for s in ("vis", "ctx"):
         n = w.Nv if s == "vis" else w.Nc
         x = to_dev(inp["x_" + s])
@@ -76,6 +81,26 @@ def test_modulate_and_residual(name):
                                    inp["gate_" + s])
         parity(from_dev(y), ry, w.dtype, f"{name} y_{s}")
         parity(from_dev(out), rr, w.dtype, f"{name} residual_{s}")
+        assert torch.equal(pair[s], y), f"{name} y_{s}: the pair launch differs"
+
+
+def test_modulate_pair_one_stream_empty_and_in_place():
+    """The pair launch with an empty conditioning stream equals the single
+    launch; y may overwrite its own x."""
+    w = _ws(W["block"], B=2, ctx_len=None)
+    inp = I.make_inputs(w, parts=("adaln",))
+    xv = to_dev(inp["x_vis"])
+    sv, cv = to_dev(inp["shift_vis"]), to_dev(inp["scale_vis"])
+    empty = torch.empty((w.B, 0, w.C), dtype=xv.dtype, device=xv.device)
+    yv, _ = api.adaln_modulate_pair(xv, sv, cv, empty, sv, cv)
+    assert torch.equal(yv, api.adaln_modulate(xv, sv, cv))
+    xc = to_dev(inp["x_ctx"])
+    yc_ref = api.adaln_modulate(xc, to_dev(inp["shift_ctx"]), to_dev(inp["scale_ctx"]))
+    xv2, xc2 = xv.clone(), xc.clone()
+    api.adaln_modulate_pair(xv2, sv, cv, xc2, to_dev(inp["shift_ctx"]), to_dev(inp["scale_ctx"]),
+                            out_vis=xv2, out_ctx=xc2)
+    torch.cuda.synchronize()
+    assert torch.equal(xv2, yv) and torch.equal(xc2, yc_ref)
 
 
 def test_modulate_large_mean_rows():

@@ -4,7 +4,10 @@ Int8 S = Q K^T, FP8 E4M3 O = P V) through the C ABI.
 The quantisers must reproduce the oracle's codes and scales exactly (integer
 and byte work).  The attention is compared with the oracle's whole 8-bit
 method run from the unquantised inputs (the oracle quantises by itself), with
-the bf16 criterion; small cases in full, 480p on sampled rows."""
+the bf16 criterion; small cases in full, 480p on sampled rows.  It is also
+compared with the EXACT attention, within the error the method's own rounding
+steps allow (tests/helpers.py: int8 scores, E4M3 P' and v; every element
+within 6 sigma, mean |error| / sigma at most 0.8)."""
 import numpy as np
 import pytest
 import torch
@@ -12,7 +15,7 @@ import torch
 import oracle
 from mmdit_joint_attention_b200 import api
 from mmdit_joint_attention_b200 import inputs as I
-from helpers import device_inputs, from_dev, parity
+from helpers import device_inputs, from_dev, parity, q8_close_to_exact, q8_exact_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -71,6 +74,12 @@ def test_attention_q8_full(case):
     parity(oc, rc, "bf16", f"{case} o_ctx")
     for b, L in enumerate(w.ctx_lengths()):
         assert np.all(oc[b, L:] == 0.0)
+    # against the exact attention, within the 8-bit method's error model
+    trip = np.array([(b, h, i) for b in range(w.B) for h in range(w.H)
+                     for i in range(w.Nv + w.Nc)])
+    o, sig = q8_exact_rows(*args, inp["ctx_len"], trip)
+    full = np.concatenate([ov, oc], axis=1)
+    q8_close_to_exact(full[trip[:, 0], trip[:, 2], trip[:, 1]], o, sig, f"{case} vs exact")
 
 
 def test_attention_q8_sampled_480p():
@@ -88,3 +97,7 @@ def test_attention_q8_sampled_480p():
     vis = trip[:, 2] < w.Nv
     parity(got[vis], ref[vis], "bf16", "480p q8 o_vis rows")
     parity(got[~vis], ref[~vis], "bf16", "480p q8 o_ctx rows")
+    # against the exact attention on two heads, within the method's error model
+    sub = trip[np.isin(trip[:, 1], (0, 13))]
+    o, sig = q8_exact_rows(*args, inp["ctx_len"], sub)
+    q8_close_to_exact(full[sub[:, 0], sub[:, 2], sub[:, 1]], o, sig, "480p q8 vs exact")

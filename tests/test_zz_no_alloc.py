@@ -15,7 +15,7 @@ import torch
 
 from mmdit_joint_attention_b200 import _lib, api
 from mmdit_joint_attention_b200 import inputs as I
-from helpers import device_inputs, from_dev, parity, to_dev
+from helpers import device_inputs, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -51,5 +51,7 @@ def test_noalloc_backward_matches_the_workspace_entry_point():
         assert st == 0, _lib.STATUS.get(st, st)
         torch.cuda.synchronize()
         assert api.device_status() == 0
+        # the same kernels on the same inputs: bit for bit, so that a stale
+        # value left in the built-in workspace cannot hide inside a tolerance
         for k in KEYS:
-            parity(from_dev(out[k]), from_dev(ref[k]), "bf16", f"call {call} {k}")
+            assert torch.equal(out[k], ref[k]), f"call {call} {k} differs"
