@@ -672,7 +672,18 @@ def run_ours(args):
         "frac_bf16_burst_executed": 14.0 * D * pairs / (bwd_ms * 1e-3) / 1e12 / float(
             peaks()[0]["bf16_tflops"]),
         "flops_beta8": 8.0 * D * pairs, "flops_executed": 14.0 * D * pairs}}
-    del do_vis, do_ctx, grads, lse, delta
+    # modulate and residual backward on the visual stream: x and dy read, dx
+    # written; branch and dout read, dbranch written (dx = dout not asked for)
+    dy_x = torch.randn(t["x_vis"].shape, generator=gen, device=dev).to(torch.bfloat16)
+    mb_ms = time_ms(lambda: api.adaln_modulate_bwd(t["x_vis"], t["scale_vis"], dy_x))
+    rb_ms = time_ms(lambda: api.gated_residual_bwd(t["o_vis"].view(B, Nv, C), t["gate_vis"],
+                                                   dy_x))
+    eb = 3 * B * Nv * C * 2
+    for key, ms_ in (("adaln_modulate_bwd_vis", mb_ms), ("gated_residual_bwd_vis", rb_ms)):
+        bwd_rows[key] = {"ms": ms_, "GB/s": eb / (ms_ * 1e-3) / 1e9,
+                         "frac_hbm": eb / (ms_ * 1e-3) / 1e9 / float(peaks()[0]["hbm_gbs"]),
+                         "bytes": eb}
+    del do_vis, do_ctx, grads, lse, delta, dy_x
 
     # 3D window attention (1x2x2 and 4x1x1 windows): permuting prologue for
     # q/k, row permutation of v, windowed attention back to raster order

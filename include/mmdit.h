@@ -95,7 +95,7 @@ MMDIT_API int mmdit_qk_norm_rope(const void* q_in, const void* k_in, void* q_out
  *   dq_out, dk_out   [B, N, H, D] dt, gradients of the forward's outputs
  *   dq_in, dk_in     [B, N, H, D] dt, written (may equal dq_out / dk_out)
  *   q_scale, k_scale [D] fp32;  dq_scale, dk_scale [D] fp32, written
- *   grid, eps: as mmdit_qk_norm_rope (MM-RoPE text positions not supported).
+ *   grid, eps: as mmdit_qk_norm_rope (text positions: mmdit_qk_norm_rope_text_bwd).
  * dq_scale / dk_scale are summed with floating-point atomics, so their last
  * bits may differ from run to run.
  * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
@@ -129,6 +129,22 @@ MMDIT_API int mmdit_qk_norm_rope_text(const void* q_in, const void* k_in, void* 
                                       void* k_out, const float* q_scale, const float* k_scale,
                                       int B, int N, int H, int D, const mmdit_text_rope* rope,
                                       float eps, mmdit_dtype dt, void* stream);
+
+/* Backward of mmdit_qk_norm_rope_text [the reverse-mode derivative of the
+ * QK-RMSNorm and of the MM-RoPE text rotation, Seaweed-7B, section 3.2; the
+ * same report's section 3.4 trains forward and backward]: as
+ * mmdit_qk_norm_rope_bwd, with R the rotation of token n by the shared text
+ * position pos_offset + n on every axis chunk.
+ *   Arguments as mmdit_qk_norm_rope_bwd, with rope (host pointer, read during
+ *   the call only; as mmdit_qk_norm_rope_text) in place of grid.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_qk_norm_rope_text_bwd(const void* q_in, const void* k_in,
+                                          const void* dq_out, const void* dk_out,
+                                          const float* q_scale, const float* k_scale,
+                                          void* dq_in, void* dk_in, float* dq_scale,
+                                          float* dk_scale, int B, int N, int H, int D,
+                                          const mmdit_text_rope* rope, float eps, mmdit_dtype dt,
+                                          void* stream);
 
 /* Joint non-causal attention over the concatenated streams, output split back
  * [Vimoo §2.2: each stream projects its own Q/K/V, one attention runs over the

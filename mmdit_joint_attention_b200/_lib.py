@@ -107,6 +107,8 @@ def lib():
         L.mmdit_joint_attention_q8.argtypes = [_vp] * 14 + [_i] * 5 + [_f, _vp]
         L.mmdit_qk_norm_rope_bwd.argtypes = [_vp] * 10 + [_i] * 4 + [ctypes.POINTER(Grid), _f,
                                                                    _i, _vp]
+        L.mmdit_qk_norm_rope_text_bwd.argtypes = [_vp] * 10 + [_i] * 4 + [
+            ctypes.POINTER(TextRope), _f, _i, _vp]
         L.mmdit_qk_norm_rope_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                                 ctypes.POINTER(Grid), ctypes.POINTER(Window),
                                                 _f, _i, _vp]
@@ -141,7 +143,8 @@ def lib():
         L.mmdit_status_string.argtypes = [_i]
         L.mmdit_status_string.restype = ctypes.c_char_p
         for name in ("mmdit_qk_norm_rope", "mmdit_qk_norm_rope_text", "mmdit_qk_norm_rope_window",
-                     "mmdit_qk_norm_rope_bwd", "mmdit_k_norm_rope", "mmdit_joint_attention_qnorm",
+                     "mmdit_qk_norm_rope_bwd", "mmdit_qk_norm_rope_text_bwd", "mmdit_k_norm_rope",
+                     "mmdit_joint_attention_qnorm",
                      "mmdit_quantize_int8", "mmdit_quantize_v_e4m3", "mmdit_joint_attention_q8",
                      "mmdit_window_permute", "mmdit_joint_attention",
                      "mmdit_joint_attention_fwd", "mmdit_joint_attention_bwd",

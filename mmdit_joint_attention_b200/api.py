@@ -132,6 +132,31 @@ def qk_norm_rope_text(q: torch.Tensor, k: torch.Tensor, q_scale: torch.Tensor,
     return q_out, k_out
 
 
+def qk_norm_rope_text_bwd(q: torch.Tensor, k: torch.Tensor, q_scale: torch.Tensor,
+                          k_scale: torch.Tensor, dq_out: torch.Tensor, dk_out: torch.Tensor,
+                          pos_offset: float = 0.0, eps: float = 1e-6, rope_base: float = 10000.0,
+                          split=(16, 56, 56), dq: Optional[torch.Tensor] = None,
+                          dk: Optional[torch.Tensor] = None, stream=None):
+    """Backward of qk_norm_rope_text: (dq, dk, dq_scale, dk_scale)."""
+    dt = _dtype(q, k, dq_out, dk_out)
+    _f32(q_scale, k_scale)
+    B, N, H, D = q.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dgq = torch.empty(D, dtype=torch.float32, device=q.device)
+    dgk = torch.empty(D, dtype=torch.float32, device=q.device)
+    r = _lib.TextRope()
+    r.pos_offset = float(pos_offset)
+    r.rope_base = float(rope_base)
+    for a in range(3):
+        r.split[a] = int(split[a])
+    st = _lib.lib().mmdit_qk_norm_rope_text_bwd(
+        _ptr(q), _ptr(k), _ptr(dq_out), _ptr(dk_out), _ptr(q_scale), _ptr(k_scale), _ptr(dq),
+        _ptr(dk), _ptr(dgq), _ptr(dgk), B, N, H, D, ctypes.byref(r), eps, dt, _stream(stream))
+    check("mmdit_qk_norm_rope_text_bwd", st)
+    return dq, dk, dgq, dgk
+
+
 def attention_workspace(device=None) -> torch.Tensor:
     """A device workspace for the split tail of joint_attention(_fwd):
     MMDIT_ATTENTION_WORKSPACE_BYTES bytes, enough for every problem."""

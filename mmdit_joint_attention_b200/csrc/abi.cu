@@ -161,9 +161,49 @@ int mmdit_qk_norm_rope_bwd(const void* q_in, const void* k_in, const void* dq_ou
     }
     return cuda_status(launch_qk_norm_rope_bwd(q_in, k_in, dq_out, dk_out, q_scale, k_scale, dq_in,
                                                dk_in, dq_scale, dk_scale, B, N, H,
-                                               grid ? &g : nullptr, eps, dt == MMDIT_BF16,
+                                               grid ? &g : nullptr, nullptr, eps,
+                                               dt == MMDIT_BF16,
                                                static_cast<cudaStream_t>(stream)),
                        "qk_norm_rope_bwd");
+}
+
+int mmdit_qk_norm_rope_text_bwd(const void* q_in, const void* k_in, const void* dq_out,
+                                const void* dk_out, const float* q_scale, const float* k_scale,
+                                void* dq_in, void* dk_in, float* dq_scale, float* dk_scale, int B,
+                                int N, int H, int D, const mmdit_text_rope* rope, float eps,
+                                mmdit_dtype dt, void* stream) {
+    if (!dtype_ok(dt) || B < 0 || N < 0 || H < 0 || !(eps >= 0.f) || !std::isfinite(eps) || !rope)
+        return MMDIT_ERR_ARG;
+    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
+    if (!dq_scale || !dk_scale) return MMDIT_ERR_ARG;
+    if (!aligned16(dq_scale) || !aligned16(dk_scale)) return MMDIT_ERR_ALIGN;
+    if (!std::isfinite(rope->pos_offset)) return MMDIT_ERR_ARG;
+    if (!(rope->rope_base > 0.f) || !std::isfinite(rope->rope_base)) return MMDIT_ERR_ARG;
+    int sum = 0;
+    for (int a = 0; a < 3; ++a) {
+        if (rope->split[a] < 0 || (rope->split[a] & 1)) return MMDIT_ERR_SHAPE;
+        sum += rope->split[a];
+    }
+    if (sum != D) return MMDIT_ERR_SHAPE;
+    const int E = vec_elems(dt);
+    if (rope->split[0] % E || (rope->split[0] + rope->split[1]) % E) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * N * H != 0) {
+        if (!q_in || !k_in || !dq_out || !dk_out || !q_scale || !k_scale || !dq_in || !dk_in)
+            return MMDIT_ERR_ARG;
+        if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(dq_out) || !aligned16(dk_out) ||
+            !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(dq_in) || !aligned16(dk_in))
+            return MMDIT_ERR_ALIGN;
+        if ((long long)B * N * H >= (1LL << 31)) return MMDIT_ERR_UNSUPPORTED;
+    }
+    RopeText t{};
+    t.pos_offset = rope->pos_offset;
+    t.base = rope->rope_base;
+    for (int a = 0; a < 3; ++a) t.split[a] = rope->split[a];
+    return cuda_status(launch_qk_norm_rope_bwd(q_in, k_in, dq_out, dk_out, q_scale, k_scale, dq_in,
+                                               dk_in, dq_scale, dk_scale, B, N, H, nullptr, &t,
+                                               eps, dt == MMDIT_BF16,
+                                               static_cast<cudaStream_t>(stream)),
+                       "qk_norm_rope_text_bwd");
 }
 
 int mmdit_qk_norm_rope_window(const void* q_in, const void* k_in, void* q_out, void* k_out,

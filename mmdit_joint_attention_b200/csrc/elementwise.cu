@@ -434,15 +434,24 @@ qk_norm_rope_bwd_kernel(const T* __restrict__ q_in, const T* __restrict__ k_in,
             unpack(rk[r], xk);
             unpack(rdq[r], uq);
             unpack(rdk[r], uk);
-            if (ROPE == kRopeGrid) {
+            if (ROPE != kRopeNone) {
                 const uint32_t uu = u < units ? u : 0;
                 const uint32_t bn = fdiv(uu, rp.H);
                 const uint32_t n = bn - fdiv(bn, rp.N) * rp.N.d;
+                float cs[E];
+                if (ROPE == kRopeText) {
+                    // MM-RoPE text position: pos_offset + n on every axis chunk
+                    const double tpos = rp.pos_offset + (double)n;
+#pragma unroll
+                    for (int pp = 0; pp < E / 2; ++pp) {
+                        const float ang = (float)(tpos * rp.freq[rp.off[axis] / 2 + jb + pp]);
+                        sincosf(ang, &cs[2 * pp + 1], &cs[2 * pp]);
+                    }
+                } else {
                 const uint32_t t = fdiv(n, rp.HW);
                 const uint32_t rem = n - t * rp.HW.d;
                 const uint32_t hh = fdiv(rem, rp.W);
                 const uint32_t pos = axis == 0 ? t : (axis == 1 ? hh : rem - hh * rp.W.d);
-                float cs[E];
                 if (TABLE) {
                     const float4* p4 = reinterpret_cast<const float4*>(
                         tab + rp.tab_off[axis] + pos * rp.stride[axis] + jb);
@@ -461,6 +470,7 @@ qk_norm_rope_bwd_kernel(const T* __restrict__ q_in, const T* __restrict__ k_in,
                                                   rp.freq[rp.off[axis] / 2 + jb + pp]);
                         sincosf(ang, &cs[2 * pp + 1], &cs[2 * pp]);
                     }
+                }
                 }
 #pragma unroll
                 for (int pp = 0; pp < E / 2; ++pp) {
@@ -1054,8 +1064,8 @@ cudaError_t run_qk_bwd(const void* q_in, const void* k_in, const void* dq_out, c
 cudaError_t launch_qk_norm_rope_bwd(const void* q_in, const void* k_in, const void* dq_out,
                                     const void* dk_out, const float* gq, const float* gk,
                                     void* dq_in, void* dk_in, float* dgq, float* dgk, int B, int N,
-                                    int H, const RopeGrid* grid, float eps, bool bf16,
-                                    cudaStream_t s) {
+                                    int H, const RopeGrid* grid, const RopeText* text, float eps,
+                                    bool bf16, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(dgq, 0, kHeadDim * sizeof(float), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(dgk, 0, kHeadDim * sizeof(float), s);
     if (e != cudaSuccess) return e;
@@ -1089,12 +1099,27 @@ cudaError_t launch_qk_norm_rope_bwd(const void* q_in, const void* k_in, const vo
         smem = (size_t)toff * sizeof(float2);
         table = smem <= 64 * 1024;
         if (!table) smem = 0;
+    } else if (text) {
+        int off = 0;
+        for (int a = 0; a < 3; ++a) {
+            rp.split[a] = text->split[a];
+            rp.off[a] = off;
+            for (int j = 0; j < text->split[a] / 2; ++j)
+                rp.freq[off / 2 + j] = std::pow(text->base, -2.0 * j / (double)text->split[a]);
+            off += text->split[a];
+        }
+        rp.pos_offset = text->pos_offset;
+        rp.Hg = 1;
+        rp.HW = rp.W = make_fastdiv(1);
     } else {
         rp.off[1] = rp.off[2] = kHeadDim;
         rp.Hg = 1;
         rp.HW = rp.W = make_fastdiv(1);
     }
 #define MMDIT_QK_BWD(T)                                                                       \
+    if (text)                                                                                \
+        return run_qk_bwd<T, kRopeText, false>(q_in, k_in, dq_out, dk_out, gq, gk, dq_in, dk_in, \
+                                               dgq, dgk, units, eps, rp, 0, s);               \
     if (!grid)                                                                               \
         return run_qk_bwd<T, kRopeNone, false>(q_in, k_in, dq_out, dk_out, gq, gk, dq_in, dk_in, \
                                                dgq, dgk, units, eps, rp, 0, s);               \

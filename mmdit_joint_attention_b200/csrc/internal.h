@@ -36,13 +36,14 @@ cudaError_t launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out,
                                 const RopeGrid* grid, const RopeText* text, const int* win_parts,
                                 float eps, bool bf16, cudaStream_t s);
 
-// Backward of launch_qk_norm_rope (grid or none; no text positions, no
-// permutation): dq_in / dk_in written, dgq / dgk [128] zeroed then summed.
+// Backward of launch_qk_norm_rope (grid, text positions or none, at most one
+// of them; no permutation): dq_in / dk_in written, dgq / dgk [128] zeroed
+// then summed.
 cudaError_t launch_qk_norm_rope_bwd(const void* q_in, const void* k_in, const void* dq_out,
                                     const void* dk_out, const float* gq, const float* gk,
                                     void* dq_in, void* dk_in, float* dgq, float* dgk, int B, int N,
-                                    int H, const RopeGrid* grid, float eps, bool bf16,
-                                    cudaStream_t s);
+                                    int H, const RopeGrid* grid, const RopeText* text, float eps,
+                                    bool bf16, cudaStream_t s);
 
 // Rows of row_bytes (a multiple of 16) of [B, N] between raster order and the
 // window-major order of `parts` (window.h); inverse: window-major -> raster.

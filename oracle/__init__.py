@@ -313,6 +313,15 @@ def qk_norm_rope_bwd(q, k, gq, gk, dq_out, dk_out, grid=None, pos_scale=(1.0, 1.
     return dq, dk, dgq, dgk
 
 
+def qk_norm_rope_text_bwd(q, k, gq, gk, dq_out, dk_out, offset: float = 0.0,
+                          eps: float = 1e-6, base: float = 10000.0, split=(16, 56, 56)):
+    """Backward of qk_norm_rope_text (MM-RoPE text positions): dq, dk, dgq, dgk."""
+    pos = text_positions(np.shape(q)[1], offset)
+    dq, dgq = rmsnorm_rope_bwd(q, gq, dq_out, pos, eps, base, split)
+    dk, dgk = rmsnorm_rope_bwd(k, gk, dk_out, pos, eps, base, split)
+    return dq, dk, dgq, dgk
+
+
 # ------------------------------------------------------------ 8-bit attention
 
 def e4m3_round(x) -> np.ndarray:

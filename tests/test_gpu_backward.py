@@ -182,3 +182,27 @@ def test_qk_norm_rope_bwd(name):
         for got, ref, n in ((dgq, rgq, "dgq"), (dgk, rgk, "dgk")):
             err = np.max(np.abs(from_dev(got) - ref)) if ref.size else 0.0
             assert err <= 1e-3 * max(np.abs(ref).max(), 1e-30), (name, stream, n, err)
+
+
+@pytest.mark.parametrize("name", ["block", "480p", "ragged"])
+def test_qk_norm_rope_text_bwd(name):
+    """The backward with MM-RoPE text positions (cond token n at offset + n on
+    every axis chunk): dx in full against the oracle, dg within 1e-3 of its
+    largest entry."""
+    w = W[name]
+    inp = I.make_inputs(w, seed=3, parts=("qkv", "scales"))
+    gin = I.make_grad_outputs(w, seed=3)
+    t = device_inputs(inp)
+    off = float(max(w.grid))
+    dy = to_dev(gin["do_ctx"])
+    dq, dk, dgq, dgk = api.qk_norm_rope_text_bwd(t["q_ctx"], t["k_ctx"], t["gq_ctx"],
+                                                 t["gk_ctx"], dy, dy, pos_offset=off)
+    torch.cuda.synchronize()
+    rq, rk, rgq, rgk = oracle.qk_norm_rope_text_bwd(
+        inp["q_ctx"].f64, inp["k_ctx"].f64, inp["gq_ctx"], inp["gk_ctx"], gin["do_ctx"].f64,
+        gin["do_ctx"].f64, offset=off)
+    parity(from_dev(dq), rq, w.dtype, f"{name} dq_ctx text")
+    parity(from_dev(dk), rk, w.dtype, f"{name} dk_ctx text")
+    for got, ref, n in ((dgq, rgq, "dgq"), (dgk, rgk, "dgk")):
+        err = np.max(np.abs(from_dev(got) - ref))
+        assert err <= 1e-3 * max(np.abs(ref).max(), 1e-30), (name, n, err)

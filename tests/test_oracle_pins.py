@@ -691,6 +691,30 @@ def pin_norm_rope_bwd_torch_autograd():
     _close(dg, gt.grad.numpy(), 1e-11)
 
 
+@pin
+def pin_text_rope_bwd_torch_autograd():
+    """The backward with MM-RoPE text positions (token n at offset + n on all
+    three axes) equals torch float64 autograd through RMSNorm and the brute
+    force's explicit rotation matrices at those positions."""
+    r = RNG(62)
+    B, N, H, off = 2, 9, 2, 31.0
+    q = r.standard_normal((B, N, H, 128)) * 1.5
+    k = r.standard_normal((B, N, H, 128))
+    dq_o, dk_o = r.standard_normal((B, N, H, 128)), r.standard_normal((B, N, H, 128))
+    gq, gk = r.uniform(0.5, 1.5, 128), r.uniform(0.5, 1.5, 128)
+    R = torch.from_numpy(np.stack([brute.rotation_matrix((off + n, off + n, off + n))
+                                   for n in range(N)]))
+    got = oracle.qk_norm_rope_text_bwd(q, k, gq, gk, dq_o, dk_o, offset=off)
+    for x, g, dy, dx_got, dg_got in ((q, gq, dq_o, got[0], got[2]), (k, gk, dk_o, got[1], got[3])):
+        xt = torch.tensor(x, requires_grad=True)
+        gt = torch.tensor(g, requires_grad=True)
+        rms = torch.sqrt((xt * xt).mean(-1, keepdim=True) + 1e-6)
+        y = torch.einsum("nde,bnhe->bnhd", R, xt / rms * gt)
+        y.backward(torch.from_numpy(dy))
+        _close(dx_got, xt.grad.numpy(), 1e-12)
+        _close(dg_got, gt.grad.numpy(), 1e-11)
+
+
 # ------------------------------------------------ modulate / residual backward
 
 @pin
