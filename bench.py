@@ -710,6 +710,27 @@ def run_ours(args):
             "qk_norm_rope_window_ms": pro_ms,
             "qk_norm_rope_window_GB/s": 2 * vbytes / (pro_ms * 1e-3) / 1e9,
             "v_permute_ms": perm_ms, "v_permute_GB/s": vbytes / (perm_ms * 1e-3) / 1e9}
+        if parts == (1, 2, 2):
+            # window backward: forward with lse, then dQ / dK / dV of the windowed
+            # attention (o and its gradient already window-major), beta = 8 over
+            # the windowed (query, key) pairs
+            wgen = torch.Generator(device=dev).manual_seed(2000 + rank)
+            dow = torch.randn(t["q_vis"].shape, generator=wgen, device=dev).to(torch.bfloat16)
+            doc_w = torch.randn(t["q_ctx"].shape, generator=wgen, device=dev).to(torch.bfloat16)
+            ow, ocw, lw = api.joint_window_attention_fwd(qw, kw, vw, t["q_ctx"], t["k_ctx"],
+                                                         t["v_ctx"], w.grid, parts, t["ctx_len"])
+            ow = api.window_permute(ow, w.grid, parts)
+            wdelta = torch.empty_like(lw)
+            wgrads = {k: torch.empty_like(t["q_" + k[-3:]]) for k in
+                      ("dq_vis", "dk_vis", "dv_vis", "dq_ctx", "dk_ctx", "dv_ctx")}
+            wb_ms = time_ms(lambda: api.joint_window_attention_bwd(
+                qw, kw, vw, t["q_ctx"], t["k_ctx"], t["v_ctx"], ow, ocw, dow, doc_w, lw, w.grid,
+                parts, t["ctx_len"], delta=wdelta, grads=wgrads, raster_in=False), reps=5)
+            win_rows["window_" + tag].update({
+                "backward_ms": wb_ms,
+                "backward_TFLOP/s_beta8": 2 * wfl / (wb_ms * 1e-3) / 1e12,
+                "backward_TFLOP/s_executed": 3.5 * wfl / (wb_ms * 1e-3) / 1e12})
+            del dow, doc_w, ow, ocw, lw, wdelta, wgrads
         del qw, kw, vw
     if api.device_status() != 0:
         raise SystemExit("device-side wait timed out in the next-row kernels")

@@ -411,6 +411,47 @@ MMDIT_API int mmdit_joint_window_attention(const void* q_vis, const void* k_vis,
                                            const mmdit_grid* grid, const mmdit_window* win,
                                            float softmax_scale, mmdit_dtype dt, void* stream);
 
+/* mmdit_joint_window_attention that also writes, for training, the row
+ * log-sum-exp the window backward needs [Seaweed-7B, section 3.2 windows;
+ * section 3.4 trains forward and backward]:
+ *   lse[b, h, r] = log sum_j exp(Q_r . K_j * softmax_scale) over the keys row r
+ *   sees (natural log), +infinity for rows without an output.  Rows are in
+ *   the order of the INPUTS: r < Nv is the window-major visual row (as q_vis),
+ *   then the conditioning rows.
+ *   lse: DEVICE fp32 [B, H, Nv + Nc], written; 4-byte aligned, not NULL
+ *   everything else as mmdit_joint_window_attention (o_vis in raster order).
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_joint_window_attention_fwd(const void* q_vis, const void* k_vis,
+                                               const void* v_vis, const void* q_ctx,
+                                               const void* k_ctx, const void* v_ctx,
+                                               const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                                               float* lse, int B, int Nv, int Nc, int H, int D,
+                                               const mmdit_grid* grid, const mmdit_window* win,
+                                               float softmax_scale, mmdit_dtype dt,
+                                               void* stream);
+
+/* Backward of the 3D window joint attention [the reverse-mode derivative of
+ * mmdit_joint_window_attention; Seaweed-7B, section 3.2 windows, section 3.4
+ * forward and backward]: the gradients of mmdit_joint_attention_bwd with each
+ * row's key set restricted as the window forward restricts it (a visual row
+ * sees its own window's visual keys and the valid conditioning keys; a
+ * conditioning row sees every valid key).
+ *   Every VISUAL tensor is in window-major order (the order of q_vis): q_vis,
+ *   k_vis, v_vis, o_vis, do_vis (permute the raster o and its gradient with
+ *   mmdit_window_permute), the outputs dq_vis, dk_vis, dv_vis (the inverse
+ *   mmdit_window_permute returns them to raster order), and the visual rows
+ *   of lse (from mmdit_joint_window_attention_fwd) and of delta.
+ *   grid, win: as mmdit_joint_window_attention; everything else as
+ *   mmdit_joint_attention_bwd.
+ * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_joint_window_attention_bwd(
+    const void* q_vis, const void* k_vis, const void* v_vis, const void* q_ctx, const void* k_ctx,
+    const void* v_ctx, const int32_t* ctx_len, const void* o_vis, const void* o_ctx,
+    const void* do_vis, const void* do_ctx, const float* lse, float* delta, void* dq_vis,
+    void* dk_vis, void* dv_vis, void* dq_ctx, void* dk_ctx, void* dv_ctx, int B, int Nv, int Nc,
+    int H, int D, const mmdit_grid* grid, const mmdit_window* win, float softmax_scale,
+    mmdit_dtype dt, void* stream);
+
 /* adaLN modulate [Vimoo §2.2: a LayerNorm sits before attention and the FFN,
  * and the timestep embedding supplies a shift and a scale for its output]:
  *   y = LN(x) * (1 + scale[b]) + shift[b], LN over C without an affine,

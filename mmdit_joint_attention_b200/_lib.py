@@ -123,6 +123,12 @@ def lib():
         L.mmdit_joint_window_attention.argtypes = ([_vp] * 9 + [_i] * 5 +
                                                    [ctypes.POINTER(Grid), ctypes.POINTER(Window),
                                                     _f, _i, _vp])
+        L.mmdit_joint_window_attention_fwd.argtypes = ([_vp] * 10 + [_i] * 5 +
+                                                       [ctypes.POINTER(Grid),
+                                                        ctypes.POINTER(Window), _f, _i, _vp])
+        L.mmdit_joint_window_attention_bwd.argtypes = ([_vp] * 19 + [_i] * 5 +
+                                                       [ctypes.POINTER(Grid),
+                                                        ctypes.POINTER(Window), _f, _i, _vp])
         L.mmdit_adaln_modulate.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp]
         L.mmdit_adaln_modulate_pair.argtypes = ([_vp] * 4 + [_i] + [_vp] * 4 + [_i] * 3 +
                                                 [_f, _i, _vp])
@@ -149,7 +155,8 @@ def lib():
                      "mmdit_window_permute", "mmdit_joint_attention",
                      "mmdit_joint_attention_fwd", "mmdit_joint_attention_bwd",
                      "mmdit_joint_attention_ws", "mmdit_joint_attention_split_plan",
-                     "mmdit_joint_window_attention", "mmdit_adaln_modulate",
+                     "mmdit_joint_window_attention", "mmdit_joint_window_attention_fwd",
+                     "mmdit_joint_window_attention_bwd", "mmdit_adaln_modulate",
                      "mmdit_adaln_modulate_pair", "mmdit_gated_residual", "mmdit_residual_modulate", "mmdit_device_status",
                      "mmdit_adaln_modulate_bwd", "mmdit_gated_residual_bwd",
                      "mmdit_block_forward_host"):

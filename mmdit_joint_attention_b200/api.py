@@ -458,6 +458,76 @@ def joint_window_attention(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, grid: Seque
     return o_vis, o_ctx
 
 
+def joint_window_attention_fwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, grid: Sequence[int],
+                               parts: Sequence[int], ctx_len=None,
+                               softmax_scale: Optional[float] = None, o_vis=None, o_ctx=None,
+                               lse=None, stream=None):
+    """joint_window_attention that also returns the row log-sum-exp for the
+    window backward: (o_vis [raster order], o_ctx, lse [B, H, Nv + Nc] with the
+    visual rows in window-major order)."""
+    dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx)
+    B, Nv, H, D = q_vis.shape
+    Nc = q_ctx.shape[1]
+    o_vis = torch.empty_like(q_vis) if o_vis is None else o_vis
+    o_ctx = torch.empty_like(q_ctx) if o_ctx is None else o_ctx
+    if lse is None:
+        lse = torch.empty((B, H, Nv + Nc), dtype=torch.float32, device=q_vis.device)
+    _f32(lse)
+    if ctx_len is not None and (ctx_len.dtype != torch.int32 or not ctx_len.is_cuda):
+        raise TypeError("ctx_len must be an int32 CUDA tensor")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    g = make_grid(grid)
+    w = make_window(parts)
+    st = _lib.lib().mmdit_joint_window_attention_fwd(
+        _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(lse), B, Nv, Nc, H, D, ctypes.byref(g),
+        ctypes.byref(w), softmax_scale, dt, _stream(stream))
+    check("mmdit_joint_window_attention_fwd", st)
+    return o_vis, o_ctx, lse
+
+
+def joint_window_attention_bwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, o_ctx, do_vis,
+                               do_ctx, lse, grid: Sequence[int], parts: Sequence[int],
+                               ctx_len=None, softmax_scale: Optional[float] = None, delta=None,
+                               grads: Optional[dict] = None, raster_in: bool = True,
+                               stream=None) -> dict:
+    """Gradients of the 3D window joint attention.  q/k/v_vis are window-major
+    (as for joint_window_attention) and lse comes from
+    joint_window_attention_fwd.  With ``raster_in`` (the default) o_vis and
+    do_vis are in raster order, as the forward writes o_vis, and are permuted
+    to window-major here; the returned dq/dk/dv_vis are window-major, like
+    q/k/v_vis."""
+    dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, o_ctx, do_vis, do_ctx)
+    B, Nv, H, D = q_vis.shape
+    Nc = q_ctx.shape[1]
+    if raster_in:
+        o_vis = window_permute(o_vis, grid, parts, stream=stream)
+        do_vis = window_permute(do_vis, grid, parts, stream=stream)
+    if delta is None:
+        delta = torch.empty((B, H, Nv + Nc), dtype=torch.float32, device=q_vis.device)
+    _f32(lse, delta)
+    g = dict(grads or {})
+    for k, ref in (("dq_vis", q_vis), ("dk_vis", k_vis), ("dv_vis", v_vis), ("dq_ctx", q_ctx),
+                   ("dk_ctx", k_ctx), ("dv_ctx", v_ctx)):
+        if k not in g:
+            g[k] = torch.empty_like(ref)
+    if ctx_len is not None and (ctx_len.dtype != torch.int32 or not ctx_len.is_cuda):
+        raise TypeError("ctx_len must be an int32 CUDA tensor")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    gr = make_grid(grid)
+    w = make_window(parts)
+    st = _lib.lib().mmdit_joint_window_attention_bwd(
+        _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(do_vis), _ptr(do_ctx), _ptr(lse),
+        _ptr(delta), _ptr(g["dq_vis"]), _ptr(g["dk_vis"]), _ptr(g["dv_vis"]), _ptr(g["dq_ctx"]),
+        _ptr(g["dk_ctx"]), _ptr(g["dv_ctx"]), B, Nv, Nc, H, D, ctypes.byref(gr), ctypes.byref(w),
+        softmax_scale, dt, _stream(stream))
+    check("mmdit_joint_window_attention_bwd", st)
+    return g
+
+
 def adaln_modulate(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
                    eps: float = 1e-6, out: Optional[torch.Tensor] = None,
                    stream=None) -> torch.Tensor:

@@ -335,6 +335,56 @@ int joint_attention_impl(const void* q_vis, const void* k_vis, const void* v_vis
     return MMDIT_ERR_CUDA;
 }
 
+// The attention backward of both entry points (win: null, or the 3D window
+// partition of the window-major visual inputs).
+int joint_attention_bwd_impl(const void* q_vis, const void* k_vis, const void* v_vis,
+                             const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                             const int32_t* ctx_len, const void* o_vis, const void* o_ctx,
+                             const void* do_vis, const void* do_ctx, const float* lse,
+                             float* delta, void* dq_vis, void* dk_vis, void* dv_vis,
+                             void* dq_ctx, void* dk_ctx, void* dv_ctx, int B, int Nv, int Nc,
+                             int H, int D, float softmax_scale, mmdit_dtype dt, void* stream,
+                             const WindowTable* win) {
+    if (!dtype_ok(dt) || B < 0 || Nv < 0 || Nc < 0 || H < 0) return MMDIT_ERR_ARG;
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MMDIT_ERR_ARG;
+    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * H * (Nv + (long long)Nc) == 0) return MMDIT_OK;
+    if (B > 65535 || H > 65535) return MMDIT_ERR_UNSUPPORTED;
+    if ((long long)B * H * (Nv + (long long)Nc) >= (1LL << 31)) return MMDIT_ERR_UNSUPPORTED;
+    const void* vis[] = {q_vis, k_vis, v_vis, o_vis, do_vis, dq_vis, dk_vis, dv_vis};
+    const void* ctx[] = {q_ctx, k_ctx, v_ctx, o_ctx, do_ctx, dq_ctx, dk_ctx, dv_ctx};
+    for (int i = 0; i < 8; ++i) {
+        if (Nv > 0 && !vis[i]) return MMDIT_ERR_ARG;
+        if (Nc > 0 && !ctx[i]) return MMDIT_ERR_ARG;
+        if (Nv > 0 && !aligned16(vis[i])) return MMDIT_ERR_ALIGN;
+        if (Nc > 0 && !aligned16(ctx[i])) return MMDIT_ERR_ALIGN;
+    }
+    if (!lse || !delta) return MMDIT_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(delta) & 3u) ||
+        (ctx_len && (reinterpret_cast<uintptr_t>(ctx_len) & 3u)))
+        return MMDIT_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == MMDIT_F32)
+        return cuda_status(
+            launch_joint_attention_bwd_f32(
+                static_cast<const float*>(q_vis), static_cast<const float*>(k_vis),
+                static_cast<const float*>(v_vis), static_cast<const float*>(q_ctx),
+                static_cast<const float*>(k_ctx), static_cast<const float*>(v_ctx), ctx_len,
+                static_cast<const float*>(o_vis), static_cast<const float*>(o_ctx),
+                static_cast<const float*>(do_vis), static_cast<const float*>(do_ctx), lse, delta,
+                static_cast<float*>(dq_vis), static_cast<float*>(dk_vis),
+                static_cast<float*>(dv_vis), static_cast<float*>(dq_ctx),
+                static_cast<float*>(dk_ctx), static_cast<float*>(dv_ctx), B, Nv, Nc, H,
+                softmax_scale, s, win),
+            "joint_attention_bwd_f32");
+    const int r = launch_joint_attention_bwd_bf16(
+        q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx, do_vis, do_ctx, lse, delta,
+        dq_vis, dk_vis, dv_vis, dq_ctx, dk_ctx, dv_ctx, B, Nv, Nc, H, softmax_scale, s, win);
+    if (r == 0) return MMDIT_OK;
+    set_last_error("joint_attention_bwd_bf16", r);
+    return MMDIT_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -499,44 +549,10 @@ int mmdit_joint_attention_bwd(const void* q_vis, const void* k_vis, const void* 
                               float* delta, void* dq_vis, void* dk_vis, void* dv_vis,
                               void* dq_ctx, void* dk_ctx, void* dv_ctx, int B, int Nv, int Nc,
                               int H, int D, float softmax_scale, mmdit_dtype dt, void* stream) {
-    if (!dtype_ok(dt) || B < 0 || Nv < 0 || Nc < 0 || H < 0) return MMDIT_ERR_ARG;
-    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MMDIT_ERR_ARG;
-    if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
-    if ((long long)B * H * (Nv + (long long)Nc) == 0) return MMDIT_OK;
-    if (B > 65535 || H > 65535) return MMDIT_ERR_UNSUPPORTED;
-    if ((long long)B * H * (Nv + (long long)Nc) >= (1LL << 31)) return MMDIT_ERR_UNSUPPORTED;
-    const void* vis[] = {q_vis, k_vis, v_vis, o_vis, do_vis, dq_vis, dk_vis, dv_vis};
-    const void* ctx[] = {q_ctx, k_ctx, v_ctx, o_ctx, do_ctx, dq_ctx, dk_ctx, dv_ctx};
-    for (int i = 0; i < 8; ++i) {
-        if (Nv > 0 && !vis[i]) return MMDIT_ERR_ARG;
-        if (Nc > 0 && !ctx[i]) return MMDIT_ERR_ARG;
-        if (Nv > 0 && !aligned16(vis[i])) return MMDIT_ERR_ALIGN;
-        if (Nc > 0 && !aligned16(ctx[i])) return MMDIT_ERR_ALIGN;
-    }
-    if (!lse || !delta) return MMDIT_ERR_ARG;
-    if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(delta) & 3u) ||
-        (ctx_len && (reinterpret_cast<uintptr_t>(ctx_len) & 3u)))
-        return MMDIT_ERR_ALIGN;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dt == MMDIT_F32)
-        return cuda_status(
-            launch_joint_attention_bwd_f32(
-                static_cast<const float*>(q_vis), static_cast<const float*>(k_vis),
-                static_cast<const float*>(v_vis), static_cast<const float*>(q_ctx),
-                static_cast<const float*>(k_ctx), static_cast<const float*>(v_ctx), ctx_len,
-                static_cast<const float*>(o_vis), static_cast<const float*>(o_ctx),
-                static_cast<const float*>(do_vis), static_cast<const float*>(do_ctx), lse, delta,
-                static_cast<float*>(dq_vis), static_cast<float*>(dk_vis),
-                static_cast<float*>(dv_vis), static_cast<float*>(dq_ctx),
-                static_cast<float*>(dk_ctx), static_cast<float*>(dv_ctx), B, Nv, Nc, H,
-                softmax_scale, s),
-            "joint_attention_bwd_f32");
-    const int r = launch_joint_attention_bwd_bf16(
-        q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx, do_vis, do_ctx, lse, delta,
-        dq_vis, dk_vis, dv_vis, dq_ctx, dk_ctx, dv_ctx, B, Nv, Nc, H, softmax_scale, s);
-    if (r == 0) return MMDIT_OK;
-    set_last_error("joint_attention_bwd_bf16", r);
-    return MMDIT_ERR_CUDA;
+    return joint_attention_bwd_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis,
+                                    o_ctx, do_vis, do_ctx, lse, delta, dq_vis, dk_vis, dv_vis,
+                                    dq_ctx, dk_ctx, dv_ctx, B, Nv, Nc, H, D, softmax_scale, dt,
+                                    stream, nullptr);
 }
 
 int mmdit_joint_window_attention(const void* q_vis, const void* k_vis, const void* v_vis,
@@ -553,6 +569,43 @@ int mmdit_joint_window_attention(const void* q_vis, const void* k_vis, const voi
     const WindowTable tab = make_window_table(grid->T, grid->H, grid->W, win->parts);
     return joint_attention_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx,
                                 nullptr, B, Nv, Nc, H, D, softmax_scale, &tab, dt, stream);
+}
+
+int mmdit_joint_window_attention_fwd(const void* q_vis, const void* k_vis, const void* v_vis,
+                                     const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                     const int32_t* ctx_len, void* o_vis, void* o_ctx, float* lse,
+                                     int B, int Nv, int Nc, int H, int D,
+                                     const mmdit_grid* grid, const mmdit_window* win,
+                                     float softmax_scale, mmdit_dtype dt, void* stream) {
+    if (!grid || !win || !lse || Nv < 0) return MMDIT_ERR_ARG;
+    if (grid->T < 1 || grid->H < 1 || grid->W < 1) return MMDIT_ERR_SHAPE;
+    if ((long long)grid->T * grid->H * grid->W != (long long)Nv) return MMDIT_ERR_SHAPE;
+    const int r = check_window(grid, win);
+    if (r != MMDIT_OK) return r;
+    const WindowTable tab = make_window_table(grid->T, grid->H, grid->W, win->parts);
+    return joint_attention_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx,
+                                lse, B, Nv, Nc, H, D, softmax_scale, &tab, dt, stream);
+}
+
+int mmdit_joint_window_attention_bwd(const void* q_vis, const void* k_vis, const void* v_vis,
+                                     const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                     const int32_t* ctx_len, const void* o_vis,
+                                     const void* o_ctx, const void* do_vis, const void* do_ctx,
+                                     const float* lse, float* delta, void* dq_vis, void* dk_vis,
+                                     void* dv_vis, void* dq_ctx, void* dk_ctx, void* dv_ctx,
+                                     int B, int Nv, int Nc, int H, int D, const mmdit_grid* grid,
+                                     const mmdit_window* win, float softmax_scale, mmdit_dtype dt,
+                                     void* stream) {
+    if (!grid || !win || Nv < 0) return MMDIT_ERR_ARG;
+    if (grid->T < 1 || grid->H < 1 || grid->W < 1) return MMDIT_ERR_SHAPE;
+    if ((long long)grid->T * grid->H * grid->W != (long long)Nv) return MMDIT_ERR_SHAPE;
+    const int r = check_window(grid, win);
+    if (r != MMDIT_OK) return r;
+    const WindowTable tab = make_window_table(grid->T, grid->H, grid->W, win->parts);
+    return joint_attention_bwd_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis,
+                                    o_ctx, do_vis, do_ctx, lse, delta, dq_vis, dk_vis, dv_vis,
+                                    dq_ctx, dk_ctx, dv_ctx, B, Nv, Nc, H, D, softmax_scale, dt,
+                                    stream, &tab);
 }
 
 int mmdit_adaln_modulate(const void* x, const float* shift, const float* scale, void* y, int B,

@@ -203,7 +203,15 @@ struct Params {
     float sl2;      // softmax_scale * log2(e)
     float scale;
     uint64_t wait_ns;
+    // 3D window mode (visual rows in window-major order): the grid holds the
+    // conditioning query tiles first, then the query tiles of each window;
+    // a visual tile streams its window's keys, a conditioning tile every key
+    int windowed;
+    int cond_tiles;
+    int tile_start[kMaxWindows + 1];   // first tile of each window after the cond tiles
+    WindowTable win;
 };
+static_assert(sizeof(Params) <= 4096, "kernel parameters must fit the 4 KB parameter space");
 
 struct Bars {
     uint64_t q_full;
@@ -260,14 +268,34 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     const int t = blockIdx.x;
     const int h = blockIdx.y;
     const int b = blockIdx.z;
-    const int seg = t < p.q_tiles_vis ? 0 : 1;
-    const int row0 = (seg ? t - p.q_tiles_vis : t) * 128;
+    // query tile: stream seg, first row row0, rows stored below rend; visual
+    // keys [vs, vs + vl) (all of them, or the query's window)
+    int seg, row0, rend, vs = 0, vl = p.N[0];
+    if (!p.windowed) {
+        seg = t < p.q_tiles_vis ? 0 : 1;
+        row0 = (seg ? t - p.q_tiles_vis : t) * 128;
+        rend = p.N[seg];
+    } else if (t < p.cond_tiles) {
+        seg = 1;
+        row0 = 128 * t;
+        rend = p.N[1];
+    } else {
+        const int tt = t - p.cond_tiles;
+        int w = 0;
+        while (w + 1 < p.win.count && p.tile_start[w + 1] <= tt) ++w;
+        const WindowGeom& g = p.win.w[w];
+        seg = 0;
+        vs = g.start;
+        vl = g.te * g.he * g.we;
+        row0 = vs + 128 * (tt - p.tile_start[w]);
+        rend = vs + vl;
+    }
     int L = p.N[1];
     if (p.ctx_len) {
         L = p.ctx_len[b];
         L = L < 0 ? 0 : (L > p.N[1] ? p.N[1] : L);
     }
-    const int kv_vis = (p.N[0] + 127) / 128;
+    const int kv_vis = (vl + 127) / 128;
     const int n_kv = kv_vis + (L + 127) / 128;
     const bool idle = n_kv == 0 || (seg == 1 && row0 >= L);   // no row of this tile has an output
 
@@ -301,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     if (idle) {
         for (int r = threadIdx.x; r < 128 * 16; r += kThreads) {
             const int row = row0 + r / 16;
-            if (row < p.N[seg])
+            if (row < rend)
                 reinterpret_cast<uint4*>(
                     p.dq[seg] + ((size_t)((size_t)b * p.N[seg] + row) * p.H + h) * 128)[r % 16] =
                     make_uint4(0, 0, 0, 0);
@@ -338,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                 const int st = j % stages;
                 const uint32_t ph = (j / stages) & 1;
                 const int ks = j < kv_vis ? 0 : 1;
-                const int row = (ks ? j - kv_vis : j) * 128;
+                const int row = ks ? (j - kv_vis) * 128 : vs + j * 128;
                 if (!wait(&empty[st], ph ^ 1, ctl)) break;
                 uint8_t* dst = ring + st * kTileBytes;
                 mbar_arrive_expect_tx(&full[st], kTileBytes);
@@ -430,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         const int quarter = warp & 3;    // tensor-memory lanes (query rows) of this warp
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int row = row0 + quarter * 32 + lane;
-        const bool has_out = row < p.N[seg] && (seg == 0 || row < L);
+        const bool has_out = row < rend && (seg == 0 || row < L);
         const size_t lrow =
             ((size_t)b * p.H + h) * (size_t)(p.N[0] + p.N[1]) + (seg ? p.N[0] + row : row);
         const float lse2 = has_out ? p.lse[lrow] * kLog2e : INFINITY;
@@ -455,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->dp_free);
             const int valid =
-                (j < kv_vis ? p.N[0] - j * 128 : L - (j - kv_vis) * 128) - 64 * wg;
+                (j < kv_vis ? vl - j * 128 : L - (j - kv_vis) * 128) - 64 * wg;
             uint32_t pk[32];
             ds_half(sr, dr, pk, sl2x2, nl2, ndl, valid);
             tmem_st32(tS, pk);
@@ -466,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         }
         if (ok) ok = wait_warp(&bars->o_done, 0, ctl);
         tc_fence_after();
-        const bool store = row < p.N[seg];
+        const bool store = row < rend;
         const bool zero = !ok || !has_out;
         uint4* dst = reinterpret_cast<uint4*>(
             p.dq[seg] + ((size_t)((size_t)b * p.N[seg] + (store ? row : 0)) * p.H + h) * 128 +
@@ -533,7 +561,15 @@ struct Params {
     float sl2;
     float scale;
     uint64_t wait_ns;
+    // 3D window mode (visual rows in window-major order): the grid holds the
+    // conditioning key tiles first (every query sees them), then the key
+    // tiles of each window (seen by that window's queries and the cond ones)
+    int windowed;
+    int cond_tiles;
+    int tile_start[kMaxWindows + 1];
+    WindowTable win;
 };
+static_assert(sizeof(Params) <= 4096, "kernel parameters must fit the 4 KB parameter space");
 
 struct Bars {
     uint64_t kv_full;
@@ -566,14 +602,34 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     const int t = blockIdx.x;
     const int h = blockIdx.y;
     const int b = blockIdx.z;
-    const int seg = t < p.k_tiles_vis ? 0 : 1;
-    const int krow0 = (seg ? t - p.k_tiles_vis : t) * 128;
+    // key tile: stream seg, first key krow0, keys stored below kend; visual
+    // query rows [qvs, qvs + qvl) that see it (all, or the keys' window)
+    int seg, krow0, kend, qvs = 0, qvl = p.N[0];
+    if (!p.windowed) {
+        seg = t < p.k_tiles_vis ? 0 : 1;
+        krow0 = (seg ? t - p.k_tiles_vis : t) * 128;
+        kend = p.N[seg];
+    } else if (t < p.cond_tiles) {
+        seg = 1;
+        krow0 = 128 * t;
+        kend = p.N[1];
+    } else {
+        const int tt = t - p.cond_tiles;
+        int w = 0;
+        while (w + 1 < p.win.count && p.tile_start[w + 1] <= tt) ++w;
+        const WindowGeom& g = p.win.w[w];
+        seg = 0;
+        qvs = g.start;
+        qvl = g.te * g.he * g.we;
+        krow0 = qvs + 128 * (tt - p.tile_start[w]);
+        kend = qvs + qvl;
+    }
     int L = p.N[1];
     if (p.ctx_len) {
         L = p.ctx_len[b];
         L = L < 0 ? 0 : (L > p.N[1] ? p.N[1] : L);
     }
-    const int nq_vis = (p.N[0] + 63) / 64;
+    const int nq_vis = (qvl + 63) / 64;
     const int nq = nq_vis + (L + 63) / 64;
     const bool idle = nq == 0 || (seg == 1 && krow0 >= L);   // no valid key or no query
 
@@ -608,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     if (idle) {
         for (int r = threadIdx.x; r < 128 * 16; r += kThreads) {
             const int key = krow0 + r / 16;
-            if (key < p.N[seg]) {
+            if (key < kend) {
                 const size_t off = ((size_t)((size_t)b * p.N[seg] + key) * p.H + h) * 128;
                 reinterpret_cast<uint4*>(p.dk[seg] + off)[r % 16] = make_uint4(0, 0, 0, 0);
                 reinterpret_cast<uint4*>(p.dv[seg] + off)[r % 16] = make_uint4(0, 0, 0, 0);
@@ -646,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 const int st = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
                 const int qs = i < nq_vis ? 0 : 1;
-                const int row = (qs ? i - nq_vis : i) * 64;
+                const int row = qs ? (i - nq_vis) * 64 : qvs + i * 64;
                 if (!wait(&empty[st], ph ^ 1, ctl)) break;
                 uint8_t* dst = ring + st * kQ64Bytes;
                 mbar_arrive_expect_tx(&full[st], kQ64Bytes);
@@ -668,12 +724,15 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 const uint32_t ph = (i / kStages) & 1;
                 if (!wait_warp(&bars->l_empty[st], ph ^ 1, ctl)) break;
                 const int qs = i < nq_vis ? 0 : 1;
-                const int row0q = (qs ? i - nq_vis : i) * 64;
+                const int row0q = qs ? (i - nq_vis) * 64 : qvs + i * 64;
+                // rows outside the range that sees these keys (past the
+                // stream, past the window, or padding) get lse = +inf: P = 0
+                const int rlim = qs ? L : qvs + qvl;
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
                     const int q = lane + 32 * r;
                     const int row = row0q + q;
-                    const bool has = row < p.N[qs] && (qs == 0 || row < L);
+                    const bool has = row < rlim && row < p.N[qs];
                     const size_t jr = base + (qs ? p.N[0] + row : row);
                     lbuf[st * 64 + q] =
                         has ? make_float2(p.lse[jr] * kLog2e, p.delta[jr]) : make_float2(INFINITY, 0.f);
@@ -783,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
         if (ok) ok = wait_warp(&bars->o_done, 0, ctl);
         tc_fence_after();
         const int key = krow0 + quarter * 32 + lane;
-        const bool store = key < p.N[seg];
+        const bool store = key < kend;
         const bool zero = !ok || (seg == 1 && key >= L);
         const size_t off =
             ((size_t)((size_t)b * p.N[seg] + (store ? key : 0)) * p.H + h) * 128 + 64 * wg;
@@ -834,7 +893,7 @@ dq_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv,
               const int32_t* __restrict__ ctx_len, const float* __restrict__ dov,
               const float* __restrict__ doc, const float* __restrict__ lse,
               const float* __restrict__ delta, float* dqv, float* dqc, int Nv, int Nc, int H,
-              float scale) {
+              float scale, bool windowed, const __grid_constant__ WindowTable win) {
     const int lane = threadIdx.x & 31;
     const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int h = blockIdx.y;
@@ -856,13 +915,20 @@ dq_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv,
     const float li = lse[lr], di = delta[lr];
     const float4 q = reinterpret_cast<const float4*>((vis ? qv : qc) + qrow * 128)[lane];
     const float4 g = reinterpret_cast<const float4*>((vis ? dov : doc) + qrow * 128)[lane];
+    int k0 = 0, k1 = Nv;   // visual keys [k0, k1): all, or the query's window (window-major)
+    if (windowed && vis) {
+        int w = 0;
+        while (w + 1 < win.count && win.w[w + 1].start <= i) ++w;
+        k0 = win.w[w].start;
+        k1 = k0 + win.w[w].te * win.w[w].he * win.w[w].we;
+    }
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int seg = 0; seg < 2; ++seg) {
-        const int nk = seg == 0 ? Nv : L;
+        const int nk = seg == 0 ? k1 : L;
         const int Ns = seg == 0 ? Nv : Nc;
         const float* K = seg == 0 ? kv : kc;
         const float* V = seg == 0 ? vv : vc;
-        for (int j = 0; j < nk; ++j) {
+        for (int j = seg == 0 ? k0 : 0; j < nk; ++j) {
             const size_t kr = ((size_t)b * Ns + j) * H + h;
             const float4 k = reinterpret_cast<const float4*>(K + kr * 128)[lane];
             const float4 v = reinterpret_cast<const float4*>(V + kr * 128)[lane];
@@ -891,7 +957,8 @@ dkdv_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv,
                 const int32_t* __restrict__ ctx_len, const float* __restrict__ dov,
                 const float* __restrict__ doc, const float* __restrict__ lse,
                 const float* __restrict__ delta, float* dkv, float* dvv, float* dkc, float* dvc,
-                int Nv, int Nc, int H, float scale) {
+                int Nv, int Nc, int H, float scale, bool windowed,
+                const __grid_constant__ WindowTable win) {
     const int lane = threadIdx.x & 31;
     const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int h = blockIdx.y;
@@ -915,12 +982,19 @@ dkdv_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv,
     const float4 v = reinterpret_cast<const float4*>((vis ? vv : vc) + kr * 128)[lane];
     float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), av = ak;
     const size_t lb = ((size_t)b * H + h) * (size_t)(Nv + Nc);
+    int q0 = 0, q1 = Nv;   // visual queries [q0, q1) that see this key
+    if (windowed && vis) {
+        int w = 0;
+        while (w + 1 < win.count && win.w[w + 1].start <= j) ++w;
+        q0 = win.w[w].start;
+        q1 = q0 + win.w[w].te * win.w[w].he * win.w[w].we;
+    }
     for (int seg = 0; seg < 2; ++seg) {
-        const int nq = seg == 0 ? Nv : L;
+        const int nq = seg == 0 ? q1 : L;
         const int Ns = seg == 0 ? Nv : Nc;
         const float* Q = seg == 0 ? qv : qc;
         const float* G = seg == 0 ? dov : doc;
-        for (int i = 0; i < nq; ++i) {
+        for (int i = seg == 0 ? q0 : 0; i < nq; ++i) {
             const size_t qr = ((size_t)b * Ns + i) * H + h;
             const float4 q = reinterpret_cast<const float4*>(Q + qr * 128)[lane];
             const float4 g = reinterpret_cast<const float4*>(G + qr * 128)[lane];
@@ -994,7 +1068,7 @@ int launch_joint_attention_bwd_bf16(const void* qv, const void* kv, const void* 
                                     const void* dov, const void* doc, const float* lse,
                                     float* delta, void* dqv, void* dkv, void* dvv, void* dqc,
                                     void* dkc, void* dvc, int B, int Nv, int Nc, int H,
-                                    float softmax_scale, cudaStream_t s) {
+                                    float softmax_scale, cudaStream_t s, const WindowTable* win) {
     using namespace bwd;
     if (!encode_fn()) return -1;
     if (B == 0 || Nv + Nc == 0) return 0;
@@ -1042,7 +1116,21 @@ int launch_joint_attention_bwd_bf16(const void* qv, const void* kv, const void* 
     const int smem_k = dkv::Smem::total + 1024;
     if ((e = prepare(dq::dq_kernel, smem_q, dq_ready)) != cudaSuccess) return (int)e;
     if ((e = prepare(dkv::dkdv_kernel, smem_k, dkv_ready)) != cudaSuccess) return (int)e;
-    const dim3 grid((Nv + 127) / 128 + (Nc + 127) / 128, H, B);
+    dim3 grid((Nv + 127) / 128 + (Nc + 127) / 128, H, B);
+    if (win) {
+        // window mode: the conditioning tiles first, then each window's tiles
+        // of 128 rows (queries for dq_kernel, keys for dkdv_kernel)
+        pq.windowed = pk.windowed = 1;
+        pq.win = pk.win = *win;
+        pq.cond_tiles = pk.cond_tiles = (Nc + 127) / 128;
+        int tiles = 0;
+        for (int w = 0; w < win->count; ++w) {
+            pq.tile_start[w] = pk.tile_start[w] = tiles;
+            tiles += (win->w[w].te * win->w[w].he * win->w[w].we + 127) / 128;
+        }
+        pq.tile_start[win->count] = pk.tile_start[win->count] = tiles;
+        grid.x = (unsigned)(pq.cond_tiles + tiles);
+    }
     dq::dq_kernel<<<grid, kThreads, smem_q, s>>>(pq);
     if ((e = cudaGetLastError()) != cudaSuccess) return (int)e;
     dkv::dkdv_kernel<<<grid, kThreads, smem_k, s>>>(pk);
@@ -1056,18 +1144,21 @@ cudaError_t launch_joint_attention_bwd_f32(const float* qv, const float* kv, con
                                            const float* lse, float* delta, float* dqv, float* dkv,
                                            float* dvv, float* dqc, float* dkc, float* dvc, int B,
                                            int Nv, int Nc, int H, float softmax_scale,
-                                           cudaStream_t s) {
+                                           cudaStream_t s, const WindowTable* win) {
     using namespace bwd;
     const int rows = Nv + Nc;
     if (rows == 0 || B == 0) return cudaSuccess;
     cudaError_t e = run_delta<float>(ov, dov, oc, doc, ctx_len, delta, B, Nv, Nc, H, s);
     if (e != cudaSuccess) return e;
+    WindowTable tab{};
+    if (win) tab = *win;
     const dim3 grid((rows + 7) / 8, H, B);
     dq_f32_kernel<<<grid, 256, 0, s>>>(qv, kv, vv, qc, kc, vc, ctx_len, dov, doc, lse, delta, dqv,
-                                       dqc, Nv, Nc, H, softmax_scale);
+                                       dqc, Nv, Nc, H, softmax_scale, win != nullptr, tab);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     dkdv_f32_kernel<<<grid, 256, 0, s>>>(qv, kv, vv, qc, kc, vc, ctx_len, dov, doc, lse, delta,
-                                         dkv, dvv, dkc, dvc, Nv, Nc, H, softmax_scale);
+                                         dkv, dvv, dkc, dvc, Nv, Nc, H, softmax_scale,
+                                         win != nullptr, tab);
     return cudaGetLastError();
 }
 

@@ -55,7 +55,8 @@ joint_attn_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv
         orow = ((size_t)b * Nv + jrow) * H + h;
     }
     float4* dst = reinterpret_cast<float4*>((vis ? ov : oc) + orow * kHeadDim) + lane;
-    float* lse_row = lse ? lse + ((size_t)b * H + h) * (size_t)(Nv + Nc) + jrow : nullptr;
+    // lse rows in the order of the inputs (window-major in window mode)
+    float* lse_row = lse ? lse + ((size_t)b * H + h) * (size_t)(Nv + Nc) + i : nullptr;
     if (!vis && i - Nv >= L) {  // padded conditioning query: zero output
         *dst = make_float4(0.f, 0.f, 0.f, 0.f);
         if (lse_row && lane == 0) *lse_row = INFINITY;

@@ -549,9 +549,10 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                     uint4* dst = reinterpret_cast<uint4*>(
                         p.out[s] + ((size_t)(b * (size_t)p.N[s] + orow) * p.H + h) * kHeadDim);
                     dst[r % 16] = make_uint4(0, 0, 0, 0);
+                    // lse rows in the order of the inputs (window-major in window mode)
                     if (p.lse && r % 16 == 0)
                         p.lse[((size_t)b * p.H + h) * (size_t)(p.N[0] + p.N[1]) +
-                              (s ? p.N[0] + row0 + r / 16 : orow)] = INFINITY;
+                              (s ? p.N[0] : 0) + row0 + r / 16] = INFINITY;
                 }
             }
         }
@@ -777,8 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                 const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
                 if (p.lse && store) {
                     // natural-log row log-sum-exp of the scaled scores; m_run and
-                    // the exponents are in log2 units
-                    const int jrow = s == 0 ? orow : p.N[0] + row;
+                    // the exponents are in log2 units.  Rows in the order of the
+                    // inputs (window-major in window mode)
+                    const int jrow = s == 0 ? row : p.N[0] + row;
                     p.lse[((size_t)vwk->b * p.H + vwk->h) * (size_t)(p.N[0] + p.N[1]) + jrow] =
                         (zero || !(l_run > 0.f)) ? INFINITY
                                                  : (m_run + log2f(l_run)) * 0.6931471805599453f;

@@ -116,16 +116,20 @@ cudaError_t launch_joint_attention_f32(const float* qv, const float* kv, const f
                                        int B, int Nv, int Nc, int H, float softmax_scale,
                                        const WindowTable* win, cudaStream_t s);
 
-// Joint-attention backward (no windows).  delta: caller workspace
-// [B, H, Nv + Nc] fp32 (row sums of dO * O, written here); lse from the
-// forward.  Return convention of launch_joint_attention_bf16.
+// Joint-attention backward.  delta: caller workspace [B, H, Nv + Nc] fp32
+// (row sums of dO * O, written here); lse from the forward.  win (null: full
+// joint attention): 3D window attention, with every visual tensor
+// (q, k, v, o, dO, the d* outputs, and the visual rows of lse and delta) in
+// the table's window-major order.  Return convention of
+// launch_joint_attention_bf16.
 int launch_joint_attention_bwd_bf16(const void* qv, const void* kv, const void* vv,
                                     const void* qc, const void* kc, const void* vc,
                                     const int32_t* ctx_len, const void* ov, const void* oc,
                                     const void* dov, const void* doc, const float* lse,
                                     float* delta, void* dqv, void* dkv, void* dvv, void* dqc,
                                     void* dkc, void* dvc, int B, int Nv, int Nc, int H,
-                                    float softmax_scale, cudaStream_t s);
+                                    float softmax_scale, cudaStream_t s,
+                                    const WindowTable* win = nullptr);
 cudaError_t launch_joint_attention_bwd_f32(const float* qv, const float* kv, const float* vv,
                                            const float* qc, const float* kc, const float* vc,
                                            const int32_t* ctx_len, const float* ov,
@@ -133,7 +137,7 @@ cudaError_t launch_joint_attention_bwd_f32(const float* qv, const float* kv, con
                                            const float* lse, float* delta, float* dqv, float* dkv,
                                            float* dvv, float* dqc, float* dkc, float* dvc, int B,
                                            int Nv, int Nc, int H, float softmax_scale,
-                                           cudaStream_t s);
+                                           cudaStream_t s, const WindowTable* win = nullptr);
 
 // 8-bit joint attention: int8 q / k codes with q row scales [B, H, N_s] and k
 // block scales [B, H, ceil(N_s / 128)], E4M3 v codes with channel scales

@@ -59,6 +59,9 @@ def _configure(lib):
     lib.oracle_joint_attention_bwd.argtypes = (
         [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [dp] * 2 + [ctypes.c_int] * 5 +
         [ctypes.c_double] + [dp] * 7)
+    lib.oracle_window_attention_bwd.argtypes = (
+        [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [dp] * 2 + [ctypes.c_int] * 5 +
+        [ctypes.POINTER(_Grid), ctypes.POINTER(ctypes.c_int), ctypes.c_double] + [dp] * 7)
     lib.oracle_joint_attention_dq_rows.argtypes = (
         [dp] * 6 + [ctypes.POINTER(ctypes.c_int)] + [dp] * 2 + [ctypes.c_int] * 5 +
         [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp, dp])
@@ -489,6 +492,33 @@ def window_attention(qv, kv, vv, qc, kc, vc, grid, parts, ctx_len=None,
     out = window_attention_rows(qv, kv, vv, qc, kc, vc, ctx_len, grid, parts, rows, scale)
     out = out.reshape(B, H, Nv + Nc, D).transpose(0, 2, 1, 3)
     return np.ascontiguousarray(out[:, :Nv]), np.ascontiguousarray(out[:, Nv:])
+
+
+def window_attention_bwd(qv, kv, vv, qc, kc, vc, dov, doc, grid, parts, ctx_len=None,
+                         scale: Optional[float] = None) -> dict:
+    """Gradients of the 3D window joint attention (raster order in and out):
+    dq/dk/dv of both streams and lse [B, H, Nv + Nc] (+inf for rows without
+    an output)."""
+    qv, kv, vv, qc, kc, vc, dov, doc = (_f64(a) for a in (qv, kv, vv, qc, kc, vc, dov, doc))
+    B, Nv, H, D = qv.shape
+    Nc = qc.shape[1]
+    if Nv != grid[0] * grid[1] * grid[2]:
+        raise ValueError("grid does not match Nv")
+    if any(p < 1 or p > e for p, e in zip(parts, grid)):
+        raise ValueError("each axis needs 1 <= parts <= extent")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = {k: np.empty_like(qv) for k in ("dq_vis", "dk_vis", "dv_vis")}
+    out.update({k: np.empty_like(qc) for k in ("dq_ctx", "dk_ctx", "dv_ctx")})
+    out["lse"] = np.empty((B, H, Nv + Nc), dtype=np.float64)
+    cl_p, _keep = _ctx_ptr(ctx_len)
+    gr = _grid_struct(grid)
+    pa = (ctypes.c_int * 3)(*parts)
+    _load().oracle_window_attention_bwd(
+        _p(qv), _p(kv), _p(vv), _p(qc), _p(kc), _p(vc), cl_p, _p(dov), _p(doc), B, Nv, Nc, H, D,
+        ctypes.byref(gr), pa, scale, _p(out["dq_vis"]), _p(out["dk_vis"]), _p(out["dv_vis"]),
+        _p(out["dq_ctx"]), _p(out["dk_ctx"]), _p(out["dv_ctx"]), _p(out["lse"]))
+    return out
 
 
 def adaln_modulate(x, shift, scale, eps: float = 1e-6) -> np.ndarray:

@@ -468,6 +468,94 @@ void oracle_joint_attention_bwd(const double* qv, const double* kv, const double
     }
 }
 
+/* ---- 3D window attention backward [S] --------------------------------------
+ * The reverse-mode derivative of oracle_window_attention_rows (the Seaweed-7B
+ * report, section 3.2, restricts the attention to windows; its section 3.4
+ * trains forward and backward): the joint backward above with the key set of
+ * each query row restricted as the window forward restricts it (a visual query
+ * sees its own window's visual keys and every valid conditioning key; a
+ * conditioning query sees every valid key).  Inputs and outputs in raster
+ * order; lse as in oracle_joint_attention_bwd.                                */
+void oracle_window_attention_bwd(const double* qv, const double* kv, const double* vv,
+                                 const double* qc, const double* kc, const double* vc,
+                                 const int* ctx_len, const double* dov, const double* doc,
+                                 int B, int Nv, int Nc, int H, int D, const oracle_grid* grid,
+                                 const int* parts, double scale, double* dqv, double* dkv,
+                                 double* dvv, double* dqc, double* dkc, double* dvc, double* lse)
+{
+    const long nv = (long)B * Nv * H * D, nc = (long)B * Nc * H * D;
+    memset(dqv, 0, sizeof(double) * (size_t)nv);
+    memset(dkv, 0, sizeof(double) * (size_t)nv);
+    memset(dvv, 0, sizeof(double) * (size_t)nv);
+    memset(dqc, 0, sizeof(double) * (size_t)nc);
+    memset(dkc, 0, sizeof(double) * (size_t)nc);
+    memset(dvc, 0, sizeof(double) * (size_t)nc);
+    int* win = (int*)malloc(sizeof(int) * (size_t)(Nv > 0 ? Nv : 1));
+    oracle_window_of_tokens(grid, parts, win);
+    #pragma omp parallel
+    {
+        double* p = (double*)malloc(sizeof(double) * (size_t)(Nv + Nc + 1));
+        int* key = (int*)malloc(sizeof(int) * (size_t)(Nv + Nc + 1));
+        double* o = (double*)malloc(sizeof(double) * (size_t)D);
+        /* each (b, h) owns its rows of every gradient */
+        #pragma omp for schedule(dynamic, 1)
+        for (long bh = 0; bh < (long)B * H; ++bh) {
+            const long b = bh / H, h = bh % H;
+            const int L = ctx_len ? ctx_len[b] : Nc;
+            for (long i = 0; i < Nv + Nc; ++i) {
+                if (lse != NULL) lse[bh * (long)(Nv + Nc) + i] = INFINITY;
+                if (i >= (long)Nv + L) continue;       /* padded query row */
+                int nkeys = 0;                         /* the keys this query sees */
+                for (int j = 0; j < Nv; ++j)
+                    if (i >= Nv || win[j] == win[i]) key[nkeys++] = j;
+                for (int j = 0; j < L; ++j) key[nkeys++] = Nv + j;
+                if (nkeys == 0) continue;
+                const double* q = oracle_row(qv, qc, b, i, Nv, Nc, H, h, D);
+                const double* dO = oracle_row(dov, doc, b, i, Nv, Nc, H, h, D);
+                double m = -INFINITY;
+                for (int e = 0; e < nkeys; ++e) {
+                    const double* k = oracle_row(kv, kc, b, key[e], Nv, Nc, H, h, D);
+                    double acc = 0.0;
+                    for (int d = 0; d < D; ++d) acc += q[d] * k[d];
+                    p[e] = acc * scale;
+                    if (p[e] > m) m = p[e];
+                }
+                double den = 0.0;
+                for (int e = 0; e < nkeys; ++e) den += exp(p[e] - m);
+                if (lse != NULL) lse[bh * (long)(Nv + Nc) + i] = m + log(den);
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (int e = 0; e < nkeys; ++e) {
+                    p[e] = exp(p[e] - m) / den;
+                    const double* v = oracle_row(vv, vc, b, key[e], Nv, Nc, H, h, D);
+                    for (int d = 0; d < D; ++d) o[d] += p[e] * v[d];
+                }
+                double Di = 0.0;
+                for (int d = 0; d < D; ++d) Di += dO[d] * o[d];
+                double* dq = (double*)oracle_row(dqv, dqc, b, i, Nv, Nc, H, h, D);
+                for (int e = 0; e < nkeys; ++e) {
+                    const int j = key[e];
+                    const double* k = oracle_row(kv, kc, b, j, Nv, Nc, H, h, D);
+                    const double* v = oracle_row(vv, vc, b, j, Nv, Nc, H, h, D);
+                    double* dk = (double*)oracle_row(dkv, dkc, b, j, Nv, Nc, H, h, D);
+                    double* dv = (double*)oracle_row(dvv, dvc, b, j, Nv, Nc, H, h, D);
+                    double dPw = 0.0;
+                    for (int d = 0; d < D; ++d) dPw += dO[d] * v[d];
+                    const double dSw = p[e] * (dPw - Di);
+                    for (int d = 0; d < D; ++d) {
+                        dv[d] += p[e] * dO[d];
+                        dq[d] += scale * dSw * k[d];
+                        dk[d] += scale * dSw * q[d];
+                    }
+                }
+            }
+        }
+        free(o);
+        free(key);
+        free(p);
+    }
+    free(win);
+}
+
 /* dq and lse of selected query rows (b, h, i) only, for sizes where the full
  * backward is out of reach: the same definitions, row by row.  dq_out is
  * [nrows, D]; lse_out [nrows].                                                */

@@ -33,6 +33,12 @@ void oracle_joint_attention_bwd(const double* qv, const double* kv, const double
                                 int B, int Nv, int Nc, int H, int D, double scale,
                                 double* dqv, double* dkv, double* dvv,
                                 double* dqc, double* dkc, double* dvc, double* lse);
+void oracle_window_attention_bwd(const double* qv, const double* kv, const double* vv,
+                                 const double* qc, const double* kc, const double* vc,
+                                 const int* ctx_len, const double* dov, const double* doc,
+                                 int B, int Nv, int Nc, int H, int D, const oracle_grid* grid,
+                                 const int* parts, double scale, double* dqv, double* dkv,
+                                 double* dvv, double* dqc, double* dkc, double* dvc, double* lse);
 void oracle_joint_attention_dq_rows(const double* qv, const double* kv, const double* vv,
                                     const double* qc, const double* kc, const double* vc,
                                     const int* ctx_len, const double* dov, const double* doc,

@@ -130,6 +130,28 @@ def test_window_validation(L):
     assert f(P, P, P, P, P, P, None, Q, Q, 1, 320, 8, 2, 64, R(g), R(w), 0.1, 1, None) == -4
     assert f(P, P, P, P, P, P, None, U, Q, 1, 320, 8, 2, 128, R(g), R(w), 0.1, 1, None) == -3
 
+    # forward with lse: lse required, 4-byte aligned
+    ff = L.mmdit_joint_window_attention_fwd
+    assert ff(P, P, P, P, P, P, None, Q, Q, None, 1, 320, 8, 2, 128, R(g), R(w), 0.1, 1,
+              None) == -1
+    assert ff(P, P, P, P, P, P, None, Q, Q, ctypes.c_void_p(4098), 1, 320, 8, 2, 128, R(g),
+              R(w), 0.1, 1, None) == -3
+    assert ff(P, P, P, P, P, P, None, Q, Q, P, 1, 321, 8, 2, 128, R(g), R(w), 0.1, 1, None) == -2
+    assert ff(P, P, P, P, P, P, None, Q, Q, P, 1, 320, 8, 2, 128, None, R(w), 0.1, 1, None) == -1
+    # backward: the window checks first, then those of the joint backward
+    fb = L.mmdit_joint_window_attention_bwd
+    args = [P] * 6 + [None] + [P] * 12
+
+    def bwd(*rest):
+        return fb(*args, *rest)
+    assert bwd(1, 320, 8, 2, 128, None, R(w), 0.1, 1, None) == -1
+    assert bwd(1, 321, 8, 2, 128, R(g), R(w), 0.1, 1, None) == -2
+    assert bwd(1, 320, 8, 2, 128, R(g), R(many), 0.1, 1, None) == -4
+    assert bwd(1, 320, 8, 2, 64, R(g), R(w), 0.1, 1, None) == -4
+    assert bwd(1, 320, 8, 2, 128, R(g), R(w), -0.1, 1, None) == -1
+    bad = [P] * 6 + [None] + [P] * 4 + [None] + [P] * 7                      # lse NULL
+    assert fb(*bad, 1, 320, 8, 2, 128, R(g), R(w), 0.1, 1, None) == -1
+
     p = L.mmdit_window_permute
     assert p(P, Q, 1, 320, 250, R(g), R(w), 0, 1, None) == -4     # 500-byte rows
     assert p(P, Q, 1, 321, 256, R(g), R(w), 0, 1, None) == -2

@@ -1,6 +1,7 @@
 """GPU parity of 3D window attention (Seaweed-7B report, section 3.2) through
-the C ABI: the row permutation, the permuting QK-norm + RoPE prologue and the
-windowed joint attention, against the float64 oracle on raster-order inputs.
+the C ABI: the row permutation, the permuting QK-norm + RoPE prologue, the
+windowed joint attention and its backward, against the float64 oracle on
+raster-order inputs.
 
 Small grids compare every output element; the 480p grid compares sampled
 query rows (every cond row, the first and last tokens and the tile
@@ -200,3 +201,79 @@ def test_window_api_rejects_bad_arguments():
     with pytest.raises(api._lib.MmditError):                       # permuting in place
         api.qk_norm_rope_window(t["q_vis"], t["k_vis"], t["gq_vis"], t["gk_vis"], w.grid,
                                 (1, 2, 2), q_out=t["q_vis"])
+
+
+# ------------------------------------------------------------- window backward
+
+def _window_bwd_run(w: I.Workload, parts, seed=0):
+    """Window forward with lse, then the window backward; gradients returned
+    to raster order, lse as written (window-major visual rows)."""
+    inp = I.make_inputs(w, seed=seed, parts=("qkv",))
+    gin = I.make_grad_outputs(w, seed=seed)
+    t = device_inputs(inp)
+    cl = t["ctx_len"] if w.ctx_len is not None else None
+    q, k, v = (api.window_permute(t[n], w.grid, parts) for n in ("q_vis", "k_vis", "v_vis"))
+    ov, oc, lse = api.joint_window_attention_fwd(q, k, v, t["q_ctx"], t["k_ctx"], t["v_ctx"],
+                                                 w.grid, parts, cl)
+    g = api.joint_window_attention_bwd(q, k, v, t["q_ctx"], t["k_ctx"], t["v_ctx"], ov, oc,
+                                       to_dev(gin["do_vis"]), to_dev(gin["do_ctx"]), lse, w.grid,
+                                       parts, cl)
+    for n in ("dq_vis", "dk_vis", "dv_vis"):
+        g[n] = api.window_permute(g[n], w.grid, parts, inverse=True)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    return inp, gin, {n: from_dev(x) for n, x in g.items()}, from_dev(lse)
+
+
+BWD = {
+    "tiny_f32_122": (W["tiny"], (1, 2, 2)),
+    "f32_ragged_232": (_ws(W["tiny"], B=2, H=3, grid=(2, 6, 9), Nc=33, ctx_len=(30, 0)), (2, 3, 2)),
+    "block_122": (W["block"], (1, 2, 2)),
+    "block_411": (W["block"], (4, 1, 1)),
+    "ragged_311": (_ws(W["block"], B=2, H=2, grid=(5, 9, 11), Nc=130, ctx_len=(0, 129)), (3, 1, 1)),
+    "uneven_235": (_ws(W["block"], H=2, grid=(7, 9, 11), Nc=64), (2, 3, 5)),
+    "no_cond_122": (_ws(W["block"], H=2, grid=(2, 20, 20), Nc=0), (1, 2, 2)),
+    "medium_2k_122": (_ws(W["block"], H=2, grid=(2, 32, 32), Nc=256), (1, 2, 2)),
+}
+
+
+@pytest.mark.parametrize("case", sorted(BWD))
+def test_window_backward_full(case):
+    w, parts = BWD[case]
+    inp, gin, g, lse = _window_bwd_run(w, parts)
+    ref = oracle.window_attention_bwd(inp["q_vis"].f64, inp["k_vis"].f64, inp["v_vis"].f64,
+                                      inp["q_ctx"].f64, inp["k_ctx"].f64, inp["v_ctx"].f64,
+                                      gin["do_vis"].f64, gin["do_ctx"].f64, w.grid, parts,
+                                      inp["ctx_len"])
+    for n in ("dq_vis", "dk_vis", "dv_vis", "dq_ctx", "dk_ctx", "dv_ctx"):
+        parity(g[n], ref[n], w.dtype, f"{case} {n}")
+    # lse: the oracle's raster rows, reordered to the window-major order of q_vis
+    order = _order(w.grid, parts)
+    want = np.concatenate([ref["lse"][:, :, order], ref["lse"][:, :, w.Nv:]], axis=2)
+    assert np.array_equal(np.isinf(lse), np.isinf(want)), f"{case}: +inf rows differ"
+    fin = ~np.isinf(want)
+    if fin.any():
+        assert np.abs(lse[fin] - want[fin]).max() <= 1e-3, f"{case}: lse"
+    for b, L in enumerate(w.ctx_lengths()):
+        for n in ("dq_ctx", "dk_ctx", "dv_ctx"):
+            assert np.all(g[n][b, L:] == 0.0), f"{case} {n}: padded rows must be zero"
+
+
+def test_single_window_backward_is_the_joint_backward_bitwise():
+    """With one window the window backward runs the joint backward's per-row
+    arithmetic in the same order: bit for bit the same gradients."""
+    w = _ws(W["block"], B=2, H=3, grid=(3, 10, 11), Nc=200, ctx_len=(200, 17))
+    inp = I.make_inputs(w, seed=6, parts=("qkv",))
+    gin = I.make_grad_outputs(w, seed=6)
+    t = device_inputs(inp)
+    args = (t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"], t["v_ctx"])
+    do_v, do_c = to_dev(gin["do_vis"]), to_dev(gin["do_ctx"])
+    jv, jc, jl = api.joint_attention_fwd(*args, t["ctx_len"])
+    jg = api.joint_attention_bwd(*args, jv, jc, do_v, do_c, jl, t["ctx_len"])
+    wv, wc, wl = api.joint_window_attention_fwd(*args, w.grid, (1, 1, 1), t["ctx_len"])
+    wg = api.joint_window_attention_bwd(*args, wv, wc, do_v, do_c, wl, w.grid, (1, 1, 1),
+                                        t["ctx_len"])
+    torch.cuda.synchronize()
+    assert torch.equal(jl, wl)
+    for n in jg:
+        assert torch.equal(jg[n], wg[n]), n

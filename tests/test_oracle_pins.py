@@ -569,6 +569,60 @@ def pin_bwd_finite_differences():
 
 
 @pin
+def pin_window_bwd_finite_differences():
+    """Every gradient of the 3D window attention equals the central difference
+    of L = sum(dO * O) through the window forward oracle (grid 2x2x3 in 1x2x2
+    windows of uneven size, ragged conditioning), and the row log-sum-exp is
+    scipy's logsumexp over each row's visible keys."""
+    from scipy.special import logsumexp
+    grid, parts = (2, 2, 3), (1, 2, 2)
+    t, (dov, doc), cl = _bwd_case(53, Nv=12, Nc=3, H=2, D=8, ctx_len=(3, 1))
+    g = oracle.window_attention_bwd(*t, dov, doc, grid, parts, cl)
+
+    def loss(tt):
+        ov, oc = oracle.window_attention(*tt, grid, parts, cl)
+        return float(np.sum(ov * dov) + np.sum(oc * doc))
+
+    names = ["dq_vis", "dk_vis", "dv_vis", "dq_ctx", "dk_ctx", "dv_ctx"]
+    h = 1e-6
+    for a, name in enumerate(names):
+        num = np.zeros_like(t[a])
+        for idx in np.ndindex(t[a].shape):
+            tp = [x.copy() for x in t]
+            tm = [x.copy() for x in t]
+            tp[a][idx] += h
+            tm[a][idx] -= h
+            num[idx] = (loss(tp) - loss(tm)) / (2 * h)
+        _close(g[name], num, 1e-7)
+    win = oracle.window_of_tokens(grid, parts)
+    B, Nv, H, D = t[0].shape
+    for b in range(B):
+        for hh in range(H):
+            q = np.concatenate([t[0][b, :, hh], t[3][b, :, hh]])
+            k = np.concatenate([t[1][b, :, hh], t[4][b, :cl[b], hh]])
+            for i in range(Nv + 3):
+                if i >= Nv + cl[b]:
+                    assert np.isinf(g["lse"][b, hh, i])
+                    continue
+                vis_ok = (win == win[i]) if i < Nv else np.ones(Nv, bool)
+                sel = np.concatenate([vis_ok, np.ones(cl[b], bool)])
+                want = logsumexp(k[sel] @ q[i] / math.sqrt(D))
+                assert abs(g["lse"][b, hh, i] - want) <= 1e-12
+
+
+@pin
+def pin_window_bwd_one_window_is_joint():
+    """With one window over the whole grid the window backward is the joint
+    attention backward."""
+    t, (dov, doc), cl = _bwd_case(54, Nv=12, Nc=5, H=2, D=16, ctx_len=(5, 2))
+    g = oracle.window_attention_bwd(*t, dov, doc, (2, 3, 2), (1, 1, 1), cl)
+    j = oracle.joint_attention_bwd(*t, dov, doc, cl)
+    for k in ("dq_vis", "dk_vis", "dv_vis", "dq_ctx", "dk_ctx", "dv_ctx"):
+        _close(g[k], j[k], 1e-12)
+    assert np.array_equal(np.isinf(g["lse"]), np.isinf(j["lse"]))
+
+
+@pin
 def pin_bwd_torch_autograd():
     """torch float64 autograd through scaled_dot_product_attention on the
     concatenated sequence with a boolean key mask; the padded cond query rows
@@ -989,6 +1043,10 @@ MUTANTS = {
                                "dbranch[row + c] = dout[row + c];"),
     "resbwd_dgate_no_branch": ("dgate[(long)b * C + c] += dout[row + c] * branch[row + c];",
                                "dgate[(long)b * C + c] += dout[row + c];"),
+    "wbwd_cond_queries_windowed": ("if (i >= Nv || win[j] == win[i]) key[nkeys++] = j;",
+                                   "if (win[j] == win[i < Nv ? i : 0]) key[nkeys++] = j;"),
+    "wbwd_window_ignored": ("if (i >= Nv || win[j] == win[i]) key[nkeys++] = j;",
+                            "key[nkeys++] = j;"),
     "window_no_cond_keys": ("for (int j = 0; j < L; ++j) key[nk++] = Nv + j;",
                             "for (int j = 0; j < L && i >= Nv; ++j) key[nk++] = Nv + j;"),
 }
