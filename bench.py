@@ -512,6 +512,46 @@ def kernel_rates(w: I.Workload, kern_ms: dict, pk: dict, sm_mhz=None) -> dict:
     return out
 
 
+def run_attention_only(args):
+    """The step's attention launch alone (normalised q and k, split-tail
+    workspace), ``warmup`` + ``steps`` times on one GPU; one JSON line with the
+    mean time.  For profiler captures, which need a short program around the
+    kernel they replay."""
+    import torch
+    from mmdit_joint_attention_b200 import api
+    if not torch.cuda.is_available():
+        raise SystemExit("no CUDA device: the product path has no CPU fallback")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = I.WORKLOADS[args.workload]
+    t = device_inputs(w, seed=0, dev=dev)
+    api.qk_norm_rope(t["q_vis"], t["k_vis"], t["gq_vis"], t["gk_vis"], grid=w.grid,
+                     pos_scale=w.pos_scale)
+    api.qk_norm_rope(t["q_ctx"], t["k_ctx"], t["gq_ctx"], t["gk_ctx"])
+    ws = api.attention_workspace(dev)
+    o_vis, o_ctx = torch.empty_like(t["q_vis"]), torch.empty_like(t["q_ctx"])
+
+    def call():
+        api.joint_attention(t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"],
+                            t["v_ctx"], t["ctx_len"], o_vis=o_vis, o_ctx=o_ctx, workspace=ws)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    z = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        call()
+    z.record()
+    torch.cuda.synchronize(dev)
+    if api.device_status() != 0:
+        raise SystemExit("device-side wait timed out")
+    ms = a.elapsed_time(z) / args.steps
+    print(json.dumps({"only": "attention", "workload": w.name, "ms": ms,
+                      "TFLOP/s": w.attention_flops() / (ms * 1e-3) / 1e12}), flush=True)
+    return 0
+
+
 def run_ours(args):
     import ctypes
 
@@ -531,12 +571,12 @@ def run_ours(args):
     t = {k: host[k].to(dev, non_blocking=True) for k in STEP_INPUTS}
     torch.cuda.synchronize(dev)
     stream = torch.cuda.current_stream(dev)
-    out_names = ["y_vis", "y_ctx", "o_vis", "o_ctx", "x_vis", "x_ctx"]
-    host_out = {k: torch.empty(t[k].shape, dtype=t[k].dtype).pin_memory() for k in out_names}
 
     # split-tail workspace of the attention (21 MB, allocated once)
     attn_ws = api.attention_workspace(dev)
     step, launches_per_step = make_step(w, t, attn_ws, stream, dev)
+    out_names = ["y_vis", "y_ctx", "o_vis", "o_ctx", "x_vis", "x_ctx"]
+    host_out = {k: torch.empty(t[k].shape, dtype=t[k].dtype).pin_memory() for k in out_names}
 
     for _ in range(args.warmup):
         step()
@@ -837,10 +877,14 @@ def main(argv=None):
     ap.add_argument("--extra-workloads", default="720p",
                     help="comma-separated workloads timed after the main one (own sub-record)")
     ap.add_argument("--extra-steps", type=int, default=5)
+    ap.add_argument("--only-attention", action="store_true",
+                    help="time the attention launch alone (for profiler captures)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps, always
     if args.impl == "reference":
         return run_reference(args)
+    if args.only_attention:
+        return run_attention_only(args)
     return run_ours(args)
 
 

@@ -73,7 +73,10 @@ class Workload:
 
 # The five workloads: tiny fp32 parity case; one 17-frame 128x128 block;
 # 81-frame 480p; 81-frame 720p with per-axis position scaling; a batch of two
-# 49-frame 480p samples with ragged conditioning lengths.
+# 49-frame 480p samples with ragged conditioning lengths.  "medium" is a
+# quarter of the 480p grid (81 frames of 240x416: 21x15x26 = 8190 visual
+# tokens), the smallest case whose q, k and v (50 MB each) still exceed the
+# L2 together: the size for profiler captures that replay a launch many times.
 WORKLOADS: Dict[str, Workload] = {
     "tiny": Workload("tiny", "f32", B=1, H=2, grid=(2, 4, 4), Nc=8),
     "block": Workload("block", "bf16", B=1, H=24, grid=(5, 8, 8), Nc=256),
@@ -82,6 +85,7 @@ WORKLOADS: Dict[str, Workload] = {
                      pos_scale=(1.0, 1.0 / 1.5, 1.0 / 1.5)),
     "ragged": Workload("ragged", "bf16", B=2, H=24, grid=(13, 30, 52), Nc=320,
                        ctx_len=(77, 300)),
+    "medium": Workload("medium", "bf16", B=1, H=24, grid=(21, 15, 26), Nc=512),
 }
 
 

@@ -31,6 +31,7 @@ def test_workload_sizes():
     assert abs(W["480p"].attention_flops() - 13.60e12) < 0.01e12
     assert abs(W["720p"].attention_flops() - 71.18e12) < 0.01e12
     assert abs(W["ragged"].attention_flops() - 10.30e12) < 0.01e12
+    assert W["medium"].Nv == 8190 and W["medium"].Nv * W["medium"].C * 2 * 3 > 126e6
 
 
 def test_make_inputs_deterministic_and_shaped():
