@@ -65,17 +65,19 @@ namespace attn {
 
 constexpr int kBlockM = 128;         // query rows per tile
 constexpr int kBlockN = 128;         // keys per tile
-constexpr int kStages = 2;           // K and V ring depth (the MMA issuer assumes 2)
+constexpr int kStages = 2;           // K/V ring: stage j % 2 holds K(j) and V(j - 1)
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kHalfBytes = kTileBytes / 2;  // one 64-column TMA box (128 B per row)
 // Warpgroups: 0 = softmax of query tile 0 (warps 0-3), 1 = softmax of tile 1
-// (warps 4-7), 2 = warp 8 TMA of Q and K, warp 9 MMA issuer, warp 10 TMA of V,
-// warp 11 idle.  K and V have their own producers so that neither waits for
-// the other's ring slot: a tile takes about one KV iteration to arrive.
+// (warps 4-7), 2 = warp 8 TMA of Q, K and V, warp 9 MMA issuer, warps 10-11
+// idle (they give the producer warpgroup its 128 threads of the register split).
+// K(j) and V(j - 1), the operands of one iteration of the MMA issuer, travel
+// together under one barrier, so the issuer waits once per key tile: its
+// waits, not the tensor core, set the pace of this kernel on B200 (a separate
+// V ring with its own barrier measured 2-3 % slower).
 constexpr int kThreads = 384;
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
-constexpr int kWarpLoadV = 10;
 // Register split: launched with kRegsLaunch per thread (64512 in total); the
 // producer warpgroup drops to kRegsProducer, the softmax warpgroups rise to
 // kRegsSoftmax: 2*128*216 + 128*72 = 64512, the launch total.
@@ -162,10 +164,9 @@ struct Work {
 
 struct Bars {
     uint64_t q_full;
-    uint64_t k_full[kStages], k_empty[kStages];
-    uint64_t v_full[kStages], v_empty[kStages];
+    uint64_t k_full[kStages], k_empty[kStages];   // the K/V ring
     uint64_t s_full[2], o_done[2];
-    uint64_t p_full[4];  // [2 i + h]: half h (keys 64h..64h+63) of P_i is in tensor memory
+    uint64_t p_full[2];  // [i]: all of P_i is in tensor memory
     uint64_t drain;
     uint64_t q_ready;   // Q-norm mode: every softmax warp has rewritten its Q rows
     uint64_t wait_ns;   // limit of one pipeline wait (copied from the parameters)
@@ -292,30 +293,34 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t tile, int s) {
     return smem_desc_sw128(tile + s * 2048, kHalfBytes, 1024);
 }
 
-// Streams key tiles [j_lo, j_lo + n_it) of one operand (K or V) of the joint
-// key sequence (kv_vis visual tiles from row vis_start on, then conditioning
-// tiles) through its ring of kStages shared-memory slots.  On an abort, waits
-// (bounded) for the copies it issued before returning.
-__device__ __forceinline__ void stream_tiles(const CUtensorMap* tm, uint8_t* ring, uint64_t* full,
-                                             uint64_t* empty, int j_lo, int n_it, int kv_vis,
-                                             int vis_start, int h, int b, Bars* bars) {
+// Streams key tiles [j_lo, j_lo + n_it) of the joint key sequence (kv_vis
+// visual tiles from row vis_start on, then conditioning tiles) through the
+// K/V ring: stage j % 2 receives K(j) and V(j - 1) under one barrier (only
+// K(0) at j = 0, only V(n_it - 1) at j = n_it).  On an abort, waits (bounded)
+// for the copies it issued before returning.
+__device__ __forceinline__ void stream_kv(const Params& p, uint8_t* smem, Bars* bars, int j_lo,
+                                          int n_it, int kv_vis, int vis_start, int h, int b) {
     int issued = 0;
-    for (int it = 0; it < n_it; ++it) {
-        const int j = j_lo + it;
-        const int st = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        const int seg = j < kv_vis ? 0 : 1;
-        const int row = seg == 0 ? vis_start + j * kBlockN : (j - kv_vis) * kBlockN;
-        if (!wait(&empty[st], ph ^ 1, bars)) break;
-        uint8_t* t = ring + st * kTileBytes;
-        mbar_arrive_expect_tx(&full[st], kTileBytes);
-        tma_load_4d(t, &tm[seg], &full[st], 0, h, row, b);
-        tma_load_4d(t + kHalfBytes, &tm[seg], &full[st], 64, h, row, b);
+    for (int j = 0; j <= n_it; ++j) {
+        const int st = j & 1;
+        if (!wait(&bars->k_empty[st], ((j >> 1) & 1) ^ 1, bars)) break;
+        const int bytes = (j < n_it ? kTileBytes : 0) + (j > 0 ? kTileBytes : 0);
+        mbar_arrive_expect_tx(&bars->k_full[st], bytes);
+        for (int w = 0; w < 2; ++w) {    // w = 0: K(j), w = 1: V(j - 1)
+            if ((w == 0 && j == n_it) || (w == 1 && j == 0)) continue;
+            const int jj = j_lo + j - w;
+            const int seg = jj < kv_vis ? 0 : 1;
+            const int row = seg == 0 ? vis_start + jj * kBlockN : (jj - kv_vis) * kBlockN;
+            const CUtensorMap* tm = w == 0 ? &p.tm_k[seg] : &p.tm_v[seg];
+            uint8_t* t = smem + (w == 0 ? Smem::k_off : Smem::v_off) + st * kTileBytes;
+            tma_load_4d(t, tm, &bars->k_full[st], 0, h, row, b);
+            tma_load_4d(t + kHalfBytes, tm, &bars->k_full[st], 64, h, row, b);
+        }
         ++issued;
     }
     if (bars->abort) {
         for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-            mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1, nullptr, kDrainLimitNs);
+            mbar_wait_bounded(&bars->k_full[j & 1], (j >> 1) & 1, nullptr, kDrainLimitNs);
     }
 }
 
@@ -486,13 +491,10 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&bars->k_full[i], 1);
             mbar_init(&bars->k_empty[i], 1);
-            mbar_init(&bars->v_full[i], 1);
-            mbar_init(&bars->v_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->s_full[i], 1);
-            mbar_init(&bars->p_full[2 * i], 4);      // one elected lane per softmax warp
-            mbar_init(&bars->p_full[2 * i + 1], 4);
+            mbar_init(&bars->p_full[i], 4);          // one elected lane per softmax warp
             mbar_init(&bars->o_done[i], 1);
         }
         mbar_init(&bars->drain, 1);
@@ -564,12 +566,13 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
     if (warp >= 8) {
         regs_dec<kRegsProducer>();
     if (warp == kWarpLoad) {
-        // ------------------------------------------------------------ TMA: Q and K
+        // ------------------------------------------------------------ TMA: Q, K and V
         if (lane == 0) {
             for (int seg = 0; seg < 2; ++seg) {
                 if (p.N[seg] > 0) {
                     tma_prefetch_desc(&p.tm_q[seg]);
                     tma_prefetch_desc(&p.tm_k[seg]);
+                    tma_prefetch_desc(&p.tm_v[seg]);
                 }
             }
             const int s0 = vwk->seg0, r0 = vwk->row0, s1 = vwk->seg1, r1 = vwk->row1;
@@ -581,17 +584,8 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                 tma_load_4d(smem + Smem::q_off + kTileBytes + kHalfBytes, &p.tm_q[s1], &bars->q_full,
                             64, h, r1, b);
             }
-            stream_tiles(p.tm_k, smem + Smem::k_off, bars->k_full, bars->k_empty, j_lo, n_it,
-                         kv_vis, vwk->vis_start, h, b, bars);
+            stream_kv(p, smem, bars, j_lo, n_it, kv_vis, vwk->vis_start, h, b);
             if (bars->abort) mbar_wait_bounded(&bars->q_full, 0, nullptr, kDrainLimitNs);
-        }
-    } else if (warp == kWarpLoadV) {
-        // ------------------------------------------------------------ TMA: V
-        if (lane == 0) {
-            for (int seg = 0; seg < 2; ++seg)
-                if (p.N[seg] > 0) tma_prefetch_desc(&p.tm_v[seg]);
-            stream_tiles(p.tm_v, smem + Smem::v_off, bars->v_full, bars->v_empty, j_lo, n_it,
-                         kv_vis, vwk->vis_start, h, b, bars);
         }
     } else if (warp == kWarpMma && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
@@ -623,50 +617,39 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                 mma_ss(d, dq + off, dk + off, idesc_qk, s > 0 ? 1u : 0u);
             }
         };
-        // O_i += P_i V in two halves of 64 keys, each issued as soon as the
-        // softmax has written that half of P_i; false if a wait gave up.
+        // O_i += P_i V once the softmax has written all of P_i; false if the
+        // wait gave up.  (Releasing P in halves, so that the first half's MMAs
+        // start early, measured 1-3 % slower: one more wait per tile for the
+        // issuing thread.)
         auto pv = [&](int i, int st, bool acc, uint32_t par) -> bool {
             const uint64_t dv = st == 0 ? dv0 : dv1;
             const uint32_t d = tmem + 256 + 128 * i;
             const uint32_t a = tmem + 128 * i;
+            if (!wait(&bars->p_full[i], par, bars)) return false;
+            tc_fence_after();
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                if (!wait(&bars->p_full[2 * i + hh], par, bars)) return false;
-                tc_fence_after();
-#pragma unroll
-                for (int s = 4 * hh; s < 4 * hh + 4; ++s)
-                    mma_ts(d, a + s * 8, dv + (uint64_t)(s * (2048 >> 4)), idesc_pv,
-                           (acc || s > 0) ? 1u : 0u);
-            }
+            for (int s = 0; s < 8; ++s)
+                mma_ts(d, a + s * 8, dv + (uint64_t)(s * (2048 >> 4)), idesc_pv,
+                       (acc || s > 0) ? 1u : 0u);
             return true;
         };
-        for (int j = 0; ok && j < n_it; ++j) {
-            const int st = j % kStages;
-            const uint32_t ph = (j / kStages) & 1;
-            const int pst = (j + kStages - 1) % kStages;
-            const uint32_t pph = ((j - 1) / kStages) & 1;
-            if (!(ok = wait(&bars->k_full[st], ph, bars))) break;
-            if (j > 0 && !(ok = wait(&bars->v_full[pst], pph, bars))) break;
+        // Iteration j: stage j % 2 holds K(j) and V(j - 1); PV_i(j - 1) then
+        // QK_i(j) per tile, and the stage is released when both have run.
+        for (int j = 0; ok && j <= n_it; ++j) {
+            const int st = j & 1;
+            if (!(ok = wait(&bars->k_full[st], (j >> 1) & 1, bars))) break;
             for (int i = 0; i < ntile; ++i) {
-                if (j > 0 && !(ok = pv(i, pst, j > 1, (j - 1) & 1))) break;
-                tc_fence_after();
-                qk(i, st);
-                mma_commit(&bars->s_full[i]);
+                if (j > 0 && !(ok = pv(i, st, j > 1, (j - 1) & 1))) break;
+                if (j < n_it) {
+                    if (j == 0) tc_fence_after();
+                    qk(i, st);
+                    mma_commit(&bars->s_full[i]);
+                } else {
+                    mma_commit(&bars->o_done[i]);
+                }
             }
             if (!ok) break;
-            if (j > 0) mma_commit(&bars->v_empty[pst]);
             mma_commit(&bars->k_empty[st]);
-        }
-        if (ok) {
-            const int j = n_it;
-            const int pst = (j - 1) % kStages;
-            const uint32_t pph = ((j - 1) / kStages) & 1;
-            ok = wait(&bars->v_full[pst], pph, bars);
-            for (int i = 0; ok && i < ntile; ++i) {
-                if (!(ok = pv(i, pst, j > 1, (j - 1) & 1))) break;
-                mma_commit(&bars->o_done[i]);
-            }
-            if (ok) mma_commit(&bars->v_empty[pst]);
         }
         // make sure nothing this thread issued is still running before TMEM is freed
         mma_commit(&bars->drain);
@@ -722,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                 // Raise the running maximum only when some row of this warp grew
                 // by more than 8 (log2 units); O (which holds PV up to the
                 // previous tile: S(j) ready implies it completed) is rescaled
-                // before any half of this tile's P is released to the MMA.
+                // before this tile's P is released to the MMA.
                 if (it == 0) {
                     m_run = m_tile;
                 } else if (__any_sync(0xffffffffu, m_tile > m_run + 8.0f)) {
@@ -732,19 +715,19 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_bf16_kernel(const __gr
                     l_run *= f;
                     rescale_o(tO, f);
                 }
-                // P in two halves of 64 keys: the MMA starts the first half of
-                // P V while the second half of the exponentials is computed.
+                // P (bf16 pairs) over the first 64 columns of S, released to
+                // the MMA issuer in one piece
                 const uint64_t negm2 = f2_pack(-m_run, -m_run);
                 float sum = 0.f;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     sum += exp_half(sv, r[h], h, sl2x2, negm2);
                     tmem_st32(tS + 32 * h, r[h]);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->p_full[2 * i + h]);
                 }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->p_full[i]);
                 l_run += sum;
             }
             // epilogue: O / l  ->  bf16 row of the owning stream (or, for a
