@@ -631,8 +631,8 @@ MMDIT_API int mmdit_block_forward_host(const mmdit_block_config* cfg,
 MMDIT_API int mmdit_device_status(void* stream);
 
 /* Sets the limit of one bounded wait inside the attention kernels (forward and
- * backward) for launches made after the call, process-wide: 0 restores the
- * default (2 s).  A wait that
+ * backward) and the modulate backward for launches made after the call,
+ * process-wide: 0 restores the default (2 s).  A wait that
  * runs out makes every role of the kernel stop (outputs undefined), drain the
  * copies and tensor-core work it issued, free its tensor memory and return;
  * the next mmdit_device_status() then reports MMDIT_ERR_TIMEOUT.  No fault or

@@ -15,9 +15,10 @@
 // the [B, C] outputs with one global atomic per column and CTA at the end: the
 // outputs are zeroed first, and their last bits depend on the order of those
 // atomics.  The LayerNorm statistics of a row are CTA-wide sums, taken for
-// several rows at once.  HBM-bound: modulate reads x and dy and writes dx;
-// residual reads branch and dout and writes dbranch (and dx when asked for:
-// it equals dout).
+// several rows at once; the modulate backward stages its rows in shared
+// memory with bulk copies, so that loads stay in flight across those sums.
+// HBM-bound: modulate reads x and dy and writes dx; residual reads branch and
+// dout and writes dbranch (and dx when asked for: it equals dout).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -26,6 +27,7 @@
 
 #include "../../include/mmdit.h"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace mmdit {
 namespace {
@@ -61,12 +63,6 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8], float) {
                       __float_as_uint(f[3]));
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
 // Elements of T in one 16-byte chunk.
 template <typename T>
 __host__ __device__ constexpr int chunk_elems() {
@@ -74,134 +70,272 @@ __host__ __device__ constexpr int chunk_elems() {
 }
 
 // Layout of both kernels: a CTA works on one sample and owns a set of rows,
-// kRows at a time; thread t owns the 16-byte column chunk t of every one of
+// a few at a time; thread t owns the 16-byte column chunk t of every one of
 // those rows (blockDim = the chunks of a row rounded up to a warp).  The
 // per-column sums (dshift / dscale, dgate) therefore stay in the owning
 // thread's registers over all of the CTA's rows, and reach the [B, C] output
-// with one global atomic per column and CTA at the end.  kRows rows are loaded
-// before any is used, so a CTA keeps kRows rows of loads in flight.
+// with one global atomic per column and CTA at the end.  The residual
+// backward loads kRows rows into registers before using any, so a CTA keeps
+// kRows rows of loads in flight; the modulate backward stages its rows in
+// shared memory (below).
 constexpr int kRows = 4;
 
-// Sum over the CTA of V values per thread; every thread gets the totals.
-// red: shared scratch of (warps * V) floats, one array per call site so that
-// consecutive reductions never overwrite values still being read.
-template <int V>
-__device__ __forceinline__ void cta_sum(float (&v)[V], float* red) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, warps = blockDim.x >> 5;
-#pragma unroll
-    for (int k = 0; k < V; ++k) v[k] = warp_sum(v[k]);
-    if (lane == 0)
-#pragma unroll
-        for (int k = 0; k < V; ++k) red[warp * V + k] = v[k];
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < V; ++k) v[k] = 0.f;
-    for (int w = 0; w < warps; ++w)
-#pragma unroll
-        for (int k = 0; k < V; ++k) v[k] += red[w * V + k];
+// ---------------------------------------------------------------- modulate bwd
+// Rows reach shared memory through bulk copies (one per row of x and of dy)
+// into a ring of kStages stages of kRows rows each, issued by thread 0, and
+// stay there: both passes over a row read their chunk from shared memory, so
+// that no row data is held in registers across the CTA barrier and the
+// per-element arithmetic runs on the paired fp32 pipe (two elements per
+// instruction).  Pass 1 takes, per row, four moments with the row's first
+// element p as a pivot (d = x - p, so that a large common offset does not
+// cancel): sum d, sum d^2, sum g and sum g d, g = dy * (1 + scale); one
+// CTA-wide sum gives mean = p + sum d / C, the variance, mean_c(g) and
+// mean_c(g xh) = rstd (sum g d - (mean - p) sum g) / C.  Pass 2 writes
+//   dx = rstd g - rstd mean_c(g) - rstd mean_c(g xh) xh
+// and adds dy and dy xh to the column sums.  A stage is refilled at the
+// barrier of the next iteration, when no thread reads it any more; two CTAs
+// share an SM (C <= 3072 bf16 / 1536 fp32), so one CTA's waits are the
+// other's compute time.
+// Measured at 480p (C = 3072 bf16): 4 rows x 2 stages 0.140 ms, 2 rows x 3 or
+// 4 stages 0.153 ms, rows held in registers across the barrier 0.149 ms.
+constexpr int kModRows = 4;                  // rows per iteration (one CTA barrier each)
+constexpr int kStages = 2;
+constexpr int kMods = 4 * kModRows;          // moments summed per iteration
+constexpr int kModBits = kMods == 16 ? 4 : (kMods == 8 ? 3 : 2);
+static_assert((1 << kModBits) == kMods, "moments per iteration: 4, 8 or 16");
+
+// Bit 0: a bounded wait expired in an elementwise backward kernel.
+__device__ unsigned int g_elem_status = 0;
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
-// ---------------------------------------------------------------- modulate bwd
-// Per row: both moments in one pass, shifted by the row's first element (so a
-// large common offset does not cancel), one CTA reduction for the kRows rows
-// of an iteration; then mean_c(g) and mean_c(g * xh), a second reduction.
-// MAXT: the largest block the instantiation serves (384 threads leave room
-// for 168 registers a thread, which C <= 3072 bf16 needs without spilling).
+// Sum of kMods values over the warp: each of the first kModBits steps swaps
+// half of the remaining values with the partner lane (xor 16, 8, ...), the
+// last steps add the partners' single values, so that lane l ends with the
+// warp total of value mod_of_lane(l); the lanes whose low 5 - kModBits bits
+// are zero hold one copy of each.
+__device__ __forceinline__ int mod_of_lane(int l) {
+    int k = 0;
+#pragma unroll
+    for (int s = 0; s < kModBits; ++s) k |= ((l >> (4 - s)) & 1) << (kModBits - 1 - s);
+    return k;
+}
+__device__ __forceinline__ int lane_of_mod(int k) {
+    int l = 0;
+#pragma unroll
+    for (int s = 0; s < kModBits; ++s) l |= ((k >> (kModBits - 1 - s)) & 1) << (4 - s);
+    return l;
+}
+__device__ __forceinline__ float warp_reduce_scatter(float (&v)[kMods], int lane) {
+#pragma unroll
+    for (int step = 0; step < kModBits; ++step) {
+        const int h = (kMods / 2) >> step, o = 16 >> step;
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int k = 0; k < h; ++k) {
+            const float send = up ? v[k] : v[k + h];
+            const float keep = up ? v[k + h] : v[k];
+            v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    float t = v[0];
+#pragma unroll
+    for (int o = 16 >> kModBits; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    return t;
+}
+
+// The 16-byte chunk of a row as packed fp32 pairs.
+template <typename T>
+struct Pairs {
+    static constexpr int N = chunk_elems<T>() / 2;
+};
+__device__ __forceinline__ void to_pairs(const uint4& v, uint64_t (&f)[4], __nv_bfloat16) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        f[e] = f2_pack(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+}
+__device__ __forceinline__ void to_pairs(const uint4& v, uint64_t (&f)[2], float) {
+    f[0] = f2_pack(__uint_as_float(v.x), __uint_as_float(v.y));
+    f[1] = f2_pack(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+__device__ __forceinline__ uint4 from_pairs(const uint64_t (&f)[4], __nv_bfloat16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float lo, hi;
+        f2_unpack(f[e], lo, hi);
+        w[e] = pack_bf16x2(lo, hi);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ uint4 from_pairs(const uint64_t (&f)[2], float) {
+    float a, b, c, d;
+    f2_unpack(f[0], a, b);
+    f2_unpack(f[1], c, d);
+    return make_uint4(__float_as_uint(a), __float_as_uint(b), __float_as_uint(c),
+                      __float_as_uint(d));
+}
+__device__ __forceinline__ float pair_sum(uint64_t v) {
+    float lo, hi;
+    f2_unpack(v, lo, hi);
+    return lo + hi;
+}
+__device__ __forceinline__ uint64_t splat(float v) { return f2_pack(v, v); }
+
 template <typename T, int MAXT>
-__global__ void __launch_bounds__(MAXT)
+__global__ void __launch_bounds__(MAXT, MAXT <= 384 ? 2 : 1)
 adaln_modulate_bwd_kernel(const T* x, const float* __restrict__ scale, const T* dy, T* dx,
-                          float* dshift, float* dscale, int N, int C, float eps) {
+                          float* dshift, float* dscale, int N, int C, float eps,
+                          uint64_t wait_ns) {
     constexpr int E = chunk_elems<T>();
-    __shared__ float red0[16 * 2 * kRows], red1[16 * 2 * kRows];
+    constexpr int NP = Pairs<T>::N;
+    extern __shared__ __align__(128) uint8_t ring[];      // [stage][row][x | dy]
+    __shared__ float red[2][16 * kMods];
+    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ uint32_t abort_flag;
     const int b = blockIdx.y;
     const int c = threadIdx.x;               // this thread's chunk
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, warps = blockDim.x >> 5;
     const bool own = c < C / E;
     const float invC = 1.f / (float)C;
-    float sc1[E], ash[E], asc[E];            // 1 + scale, dshift and dscale partials
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        sc1[e] = own ? 1.f + __ldg(scale + (size_t)b * C + c * E + e) : 0.f;
-        ash[e] = 0.f;
-        asc[e] = 0.f;
-    }
+    const uint32_t row_bytes = (uint32_t)C * sizeof(T);
     const size_t sample = (size_t)b * N * (size_t)C;
-    for (int n0 = blockIdx.x * kRows; n0 < N; n0 += gridDim.x * kRows) {
-        uint4 rx[kRows], rd[kRows];
-        float pivot[kRows];
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-            const bool row_ok = n0 + r < N;
-            const size_t row = sample + (size_t)(row_ok ? n0 + r : n0) * C;
-            rx[r] = make_uint4(0, 0, 0, 0);
-            rd[r] = make_uint4(0, 0, 0, 0);
-            if (own && row_ok) {
-                rx[r] = *reinterpret_cast<const uint4*>(x + row + (size_t)c * E);
-                rd[r] = *reinterpret_cast<const uint4*>(dy + row + (size_t)c * E);
-            }
-            pivot[r] = row_ok ? (float)x[row] : 0.f;
+    // groups of kModRows rows handled by this CTA: n0 = (blockIdx.x + g gridDim.x) kModRows
+    const int groups_all = (N + kModRows - 1) / kModRows;
+    const int G = groups_all > (int)blockIdx.x
+                      ? (groups_all - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                      : 0;
+    auto stage_row = [&](int st, int r, int which) -> const T* {
+        return reinterpret_cast<const T*>(ring +
+                                          ((size_t)(st * kModRows + r) * 2 + which) * row_bytes);
+    };
+    auto issue = [&](int g) {
+        const int st = g % kStages;
+        const int n0 = (blockIdx.x + g * gridDim.x) * kModRows;
+        const int nr = min(kModRows, N - n0);
+        mbar_arrive_expect_tx(&full[st], (uint32_t)nr * 2u * row_bytes);
+        for (int r = 0; r < nr; ++r) {
+            const size_t row = sample + (size_t)(n0 + r) * C;
+            bulk_load(const_cast<T*>(stage_row(st, r, 0)), x + row, row_bytes, &full[st]);
+            bulk_load(const_cast<T*>(stage_row(st, r, 1)), dy + row, row_bytes, &full[st]);
         }
-        float st[2 * kRows];                 // per row: sum(x - p), sum((x - p)^2)
+    };
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    int issued = 0;                          // thread 0: groups whose copies were issued
+    if (threadIdx.x == 0)
+        for (; issued < G && issued < kStages; ++issued) issue(issued);
+
+    uint64_t sc1[NP], ash[NP], asc[NP];      // 1 + scale, dshift and dscale partials (pairs)
 #pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-            float f[8];
-            unpack8(rx[r], f, T());
-            float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const float d = own ? f[e] - pivot[r] : 0.f;
-                s1 += d;
-                s2 = fmaf(d, d, s2);
-            }
-            st[2 * r] = s1;
-            st[2 * r + 1] = s2;
+    for (int k = 0; k < NP; ++k) {
+        const float* sp = scale + (size_t)b * C + c * E + 2 * k;
+        sc1[k] = own ? f2_pack(1.f + __ldg(sp), 1.f + __ldg(sp + 1)) : 0ull;
+        ash[k] = 0ull;
+        asc[k] = 0ull;
+    }
+    for (int g = 0; g < G; ++g) {
+        const int st = g % kStages;
+        const int n0 = (blockIdx.x + g * gridDim.x) * kModRows;
+        if (!mbar_wait_bounded(&full[st], (uint32_t)(g / kStages) & 1u, &abort_flag, wait_ns)) {
+            abort_flag = 1;                   // the rows are garbage from here on; no hang
+            atomicOr(&g_elem_status, 1u);
         }
-        cta_sum(st, red0);
-        float mean[kRows], rstd[kRows], gm[2 * kRows];   // gm: per row sum(g), sum(g * xh)
+        float v[kMods];                      // per row: sum d, sum d^2, sum g, sum g d
 #pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-            const float dm = st[2 * r] * invC;
-            mean[r] = pivot[r] + dm;
-            rstd[r] = rsqrtf(fmaxf(st[2 * r + 1] * invC - dm * dm, 0.f) + eps);
-            float fx[8], fd[8];
-            unpack8(rx[r], fx, T());
-            unpack8(rd[r], fd, T());
-            float a = 0.f, bgx = 0.f;
+        for (int r = 0; r < kModRows; ++r) {
+            uint64_t a1 = 0ull, a2 = 0ull, ag = 0ull, agd = 0ull;
+            if (own && n0 + r < N) {
+                const T* sx = stage_row(st, r, 0);
+                const uint64_t p2 = splat((float)sx[0]);
+                uint64_t fx[NP], fd[NP];
+                to_pairs(reinterpret_cast<const uint4*>(sx)[c], fx, T());
+                to_pairs(reinterpret_cast<const uint4*>(stage_row(st, r, 1))[c], fd, T());
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const float xh = (fx[e] - mean[r]) * rstd[r];
-                const float g = fd[e] * sc1[e];
-                a += g;
-                bgx = fmaf(g, xh, bgx);
+                for (int k = 0; k < NP; ++k) {
+                    const uint64_t d = f2_sub(fx[k], p2);
+                    const uint64_t gg = f2_mul(fd[k], sc1[k]);
+                    a1 = f2_add(a1, d);
+                    a2 = f2_fma(d, d, a2);
+                    ag = f2_add(ag, gg);
+                    agd = f2_fma(gg, d, agd);
+                }
             }
-            gm[2 * r] = a;
-            gm[2 * r + 1] = bgx;
+            v[4 * r] = pair_sum(a1);
+            v[4 * r + 1] = pair_sum(a2);
+            v[4 * r + 2] = pair_sum(ag);
+            v[4 * r + 3] = pair_sum(agd);
         }
-        cta_sum(gm, red1);
+        const float wsum = warp_reduce_scatter(v, lane);
+        float* rb = red[g & 1];              // alternate: no warp can still be reading it
+        if ((lane & ((32 >> kModBits) - 1)) == 0) rb[warp * kMods + mod_of_lane(lane)] = wsum;
+        __syncthreads();                     // also: no thread reads group g - 1's stage any more
+        if (threadIdx.x == 0 && g >= 1 && g + kStages - 1 < G && !abort_flag) {
+            fence_proxy_async_smem();
+            issue(g + kStages - 1);          // into the stage of group g - 1
+            ++issued;
+        }
+        float tot = 0.f;
+        for (int w = 0; w < warps; ++w) tot += rb[w * kMods + mod_of_lane(lane)];
 #pragma unroll
-        for (int r = 0; r < kRows; ++r) {
+        for (int r = 0; r < kModRows; ++r) {
+            const float s1 = __shfl_sync(0xffffffffu, tot, lane_of_mod(4 * r));
+            const float s2 = __shfl_sync(0xffffffffu, tot, lane_of_mod(4 * r + 1));
+            const float sg = __shfl_sync(0xffffffffu, tot, lane_of_mod(4 * r + 2));
+            const float sgd = __shfl_sync(0xffffffffu, tot, lane_of_mod(4 * r + 3));
             if (!own || n0 + r >= N) continue;
-            const float mg = gm[2 * r] * invC, mgx = gm[2 * r + 1] * invC;
-            float fx[8], fd[8], o[8];
-            unpack8(rx[r], fx, T());
-            unpack8(rd[r], fd, T());
+            const float dm = s1 * invC;
+            const float rstd = rsqrtf(fmaxf(s2 * invC - dm * dm, 0.f) + eps);
+            const float mg = sg * invC;
+            const float mgx = rstd * (sgd - dm * sg) * invC;
+            const T* sx = stage_row(st, r, 0);
+            const uint64_t p2 = splat((float)sx[0]);
+            const uint64_t rs2 = splat(rstd);
+            const uint64_t nb2 = splat(-dm * rstd);         // xh = d rstd + nb
+            const uint64_t k0 = splat(-rstd * mg), k1 = splat(-rstd * mgx);
+            uint64_t fx[NP], fd[NP], o[NP];
+            to_pairs(reinterpret_cast<const uint4*>(sx)[c], fx, T());
+            to_pairs(reinterpret_cast<const uint4*>(stage_row(st, r, 1))[c], fd, T());
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const float xh = (fx[e] - mean[r]) * rstd[r];
-                o[e] = rstd[r] * (fd[e] * sc1[e] - mg - xh * mgx);
-                ash[e] += fd[e];
-                asc[e] = fmaf(fd[e], xh, asc[e]);
+            for (int k = 0; k < NP; ++k) {
+                const uint64_t xh = f2_fma(f2_sub(fx[k], p2), rs2, nb2);
+                o[k] = f2_fma(f2_mul(fd[k], sc1[k]), rs2, f2_fma(xh, k1, k0));
+                ash[k] = f2_add(ash[k], fd[k]);
+                asc[k] = f2_fma(fd[k], xh, asc[k]);
             }
             *reinterpret_cast<uint4*>(dx + sample + (size_t)(n0 + r) * C + (size_t)c * E) =
-                pack8(o, T());
+                from_pairs(o, T());
         }
     }
     if (own) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            atomicAdd(dshift + (size_t)b * C + c * E + e, ash[e]);
-            atomicAdd(dscale + (size_t)b * C + c * E + e, asc[e]);
+        for (int k = 0; k < NP; ++k) {
+            float lo, hi;
+            f2_unpack(ash[k], lo, hi);
+            atomicAdd(dshift + (size_t)b * C + c * E + 2 * k, lo);
+            atomicAdd(dshift + (size_t)b * C + c * E + 2 * k + 1, hi);
+            f2_unpack(asc[k], lo, hi);
+            atomicAdd(dscale + (size_t)b * C + c * E + 2 * k, lo);
+            atomicAdd(dscale + (size_t)b * C + c * E + 2 * k + 1, hi);
         }
     }
+    // after an expired wait, copies may still be landing in this CTA's shared
+    // memory: wait for them (bounded) before the CTA exits
+    if (threadIdx.x == 0 && abort_flag)
+        for (int g = issued > kStages ? issued - kStages : 0; g < issued; ++g)
+            mbar_wait_bounded(&full[g % kStages], (uint32_t)(g / kStages) & 1u, nullptr,
+                              200000000ull);
 }
 
 // ---------------------------------------------------------------- residual bwd
@@ -269,9 +403,9 @@ int threads_for(int C, int E) { return ((C / E + 31) / 32) * 32; }
 // this block size), but at least 4 * kRows rows per CTA so that the final
 // atomics stay few against the rows.
 template <typename K>
-cudaError_t grid_for(K kern, int threads, int B, int N, dim3& grid) {
+cudaError_t grid_for(K kern, int threads, size_t smem, int B, int N, dim3& grid) {
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
     if (e != cudaSuccess) return e;
     long long bx = ((long long)num_sms() * (per_sm > 0 ? per_sm : 1) + B - 1) / B;
     const long long need = ((long long)N + 4 * kRows - 1) / (4 * kRows);
@@ -288,11 +422,18 @@ cudaError_t dispatch_modulate_bwd(const void* x, const float* scale, const void*
     const int threads = threads_for(C, chunk_elems<T>());
     auto kern = threads <= 384 ? adaln_modulate_bwd_kernel<T, 384>
                                : adaln_modulate_bwd_kernel<T, 512>;
-    dim3 grid;
-    cudaError_t e = grid_for(kern, threads, B, N, grid);
+    // the ring: kStages stages of kModRows rows of x and dy (at most 128 KB:
+    // C <= 4096 bf16 or 2048 fp32)
+    const size_t smem = (size_t)kStages * kModRows * 2 * C * sizeof(T);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, threads, 0, s>>>(static_cast<const T*>(x), scale, static_cast<const T*>(dy),
-                                  static_cast<T*>(dx), dshift, dscale, N, C, eps);
+    dim3 grid;
+    e = grid_for(kern, threads, smem, B, N, grid);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, threads, smem, s>>>(static_cast<const T*>(x), scale, static_cast<const T*>(dy),
+                                     static_cast<T*>(dx), dshift, dscale, N, C, eps,
+                                     wait_timeout_ns());
     return cudaGetLastError();
 }
 
@@ -301,7 +442,7 @@ cudaError_t dispatch_residual_bwd(const void* br, const float* gate, const void*
                                   void* dbr, float* dgate, int B, int N, int C, cudaStream_t s) {
     const int threads = threads_for(C, chunk_elems<T>());
     dim3 grid;
-    cudaError_t e = grid_for(gated_residual_bwd_kernel<T>, threads, B, N, grid);
+    cudaError_t e = grid_for(gated_residual_bwd_kernel<T>, threads, 0, B, N, grid);
     if (e != cudaSuccess) return e;
     gated_residual_bwd_kernel<T><<<grid, threads, 0, s>>>(
         static_cast<const T*>(br), gate, static_cast<const T*>(dout), static_cast<T*>(dx),
@@ -331,6 +472,14 @@ int check_sizes(int B, int N, int C, mmdit_dtype dt) {
 }
 
 }  // namespace
+
+cudaError_t read_and_clear_elem_status(unsigned int* out) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_elem_status, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_elem_status, &zero, sizeof(unsigned int));
+}
+
 }  // namespace mmdit
 
 using namespace mmdit;

@@ -168,6 +168,8 @@ void set_wait_timeout_ns(unsigned long long ns);
 cudaError_t read_and_clear_device_status(unsigned int* out, cudaStream_t s);
 // The same for the backward kernels' own status word.
 cudaError_t read_and_clear_bwd_status(unsigned int* out);
+// The same for the elementwise backward kernels.
+cudaError_t read_and_clear_elem_status(unsigned int* out);
 
 constexpr int kHeadDim = 128;
 
