@@ -175,7 +175,9 @@ namespace dq {
 
 // K is read twice per tile (S = Q K^T, then dQ += dS K one tile later), so its
 // ring has a third stage: with two, the next K's load could only start just
-// before the product that needs it.  V is read once (dP = dO V^T).
+// before the product that needs it.  V is read once (dP = dO V^T).  K(j) and
+// V(j) arrive under one barrier (that of K's stage), so the MMA issuer waits
+// once per key tile for both.
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
 
@@ -215,11 +217,12 @@ static_assert(sizeof(Params) <= 4096, "kernel parameters must fit the 4 KB param
 
 struct Bars {
     uint64_t q_full;
-    uint64_t k_full[kKStages], k_empty[kKStages];
-    uint64_t v_full[kVStages], v_empty[kVStages];
+    uint64_t kv_full[kKStages];   // K(j) in K stage j % 3 and V(j) in V stage j % 2 landed
+    uint64_t k_empty[kKStages];
+    uint64_t v_empty[kVStages];
     uint64_t s_full[2];    // S and dP of the tile with this S buffer are in tensor memory
     uint64_t dp_free;      // every softmax warp has read dP
-    uint64_t ds_full[4];   // [2 buf + wg]: that warpgroup's half of dS is in tensor memory
+    uint64_t ds_full[2];   // [buf]: all of dS of that buffer is in tensor memory
     uint64_t o_done;
     uint64_t drain;
     Ctl ctl;
@@ -302,16 +305,13 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
         for (int i = 0; i < kKStages; ++i) {
-            mbar_init(&bars->k_full[i], 1);
+            mbar_init(&bars->kv_full[i], 1);
             mbar_init(&bars->k_empty[i], 1);
         }
-        for (int i = 0; i < kVStages; ++i) {
-            mbar_init(&bars->v_full[i], 1);
-            mbar_init(&bars->v_empty[i], 1);
-        }
+        for (int i = 0; i < kVStages; ++i) mbar_init(&bars->v_empty[i], 1);
         for (int i = 0; i < 2; ++i) mbar_init(&bars->s_full[i], 1);
         mbar_init(&bars->dp_free, 8);
-        for (int i = 0; i < 4; ++i) mbar_init(&bars->ds_full[i], 4);
+        for (int i = 0; i < 2; ++i) mbar_init(&bars->ds_full[i], 8);   // one lane per softmax warp
         mbar_init(&bars->o_done, 1);
         mbar_init(&bars->drain, 1);
         ctl->abort = 0;
@@ -344,41 +344,35 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
 
     if (warp >= 8) {
         regs_dec<kRegsProducer>();
-        if ((warp == 8 || warp == 10) && lane == 0) {
-            // ---------------------------------------------- TMA: Q, dO, K (warp 8) / V (warp 10)
-            const bool is_k = warp == 8;
-            const CUtensorMap* tm = is_k ? p.tm_k : p.tm_v;
-            uint8_t* ring = smem + (is_k ? Smem::k_off : Smem::v_off);
-            uint64_t* full = is_k ? bars->k_full : bars->v_full;
-            uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
-            if (is_k) {
-                mbar_arrive_expect_tx(&bars->q_full, 2 * kTileBytes);
-                tma_load_4d(smem + Smem::q_off, &p.tm_q[seg], &bars->q_full, 0, h, row0, b);
-                tma_load_4d(smem + Smem::q_off + kHalf128, &p.tm_q[seg], &bars->q_full, 64, h, row0,
-                            b);
-                tma_load_4d(smem + Smem::do_off, &p.tm_do[seg], &bars->q_full, 0, h, row0, b);
-                tma_load_4d(smem + Smem::do_off + kHalf128, &p.tm_do[seg], &bars->q_full, 64, h,
-                            row0, b);
-            }
-            const int stages = is_k ? kKStages : kVStages;
+        if (warp == 8 && lane == 0) {
+            // ---------------------------------------------- TMA: Q, dO, then K and V
+            mbar_arrive_expect_tx(&bars->q_full, 2 * kTileBytes);
+            tma_load_4d(smem + Smem::q_off, &p.tm_q[seg], &bars->q_full, 0, h, row0, b);
+            tma_load_4d(smem + Smem::q_off + kHalf128, &p.tm_q[seg], &bars->q_full, 64, h, row0, b);
+            tma_load_4d(smem + Smem::do_off, &p.tm_do[seg], &bars->q_full, 0, h, row0, b);
+            tma_load_4d(smem + Smem::do_off + kHalf128, &p.tm_do[seg], &bars->q_full, 64, h, row0,
+                        b);
             int issued = 0;
             for (int j = 0; j < n_kv; ++j) {
-                const int st = j % stages;
-                const uint32_t ph = (j / stages) & 1;
+                const int kst = j % kKStages, vst = j % kVStages;
                 const int ks = j < kv_vis ? 0 : 1;
                 const int row = ks ? (j - kv_vis) * 128 : vs + j * 128;
-                if (!wait(&empty[st], ph ^ 1, ctl)) break;
-                uint8_t* dst = ring + st * kTileBytes;
-                mbar_arrive_expect_tx(&full[st], kTileBytes);
-                tma_load_4d(dst, &tm[ks], &full[st], 0, h, row, b);
-                tma_load_4d(dst + kHalf128, &tm[ks], &full[st], 64, h, row, b);
+                if (!wait(&bars->k_empty[kst], ((j / kKStages) & 1) ^ 1, ctl)) break;
+                if (!wait(&bars->v_empty[vst], ((j / kVStages) & 1) ^ 1, ctl)) break;
+                uint8_t* dk = smem + Smem::k_off + kst * kTileBytes;
+                uint8_t* dv = smem + Smem::v_off + vst * kTileBytes;
+                mbar_arrive_expect_tx(&bars->kv_full[kst], 2 * kTileBytes);
+                tma_load_4d(dk, &p.tm_k[ks], &bars->kv_full[kst], 0, h, row, b);
+                tma_load_4d(dk + kHalf128, &p.tm_k[ks], &bars->kv_full[kst], 64, h, row, b);
+                tma_load_4d(dv, &p.tm_v[ks], &bars->kv_full[kst], 0, h, row, b);
+                tma_load_4d(dv + kHalf128, &p.tm_v[ks], &bars->kv_full[kst], 64, h, row, b);
                 ++issued;
             }
             if (ctl->abort) {
-                for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j)
-                    mbar_wait_bounded(&full[j % stages], (j / stages) & 1, nullptr,
+                for (int j = (issued > kKStages ? issued - kKStages : 0); j < issued; ++j)
+                    mbar_wait_bounded(&bars->kv_full[j % kKStages], (j / kKStages) & 1, nullptr,
                                       kDrainLimitNs);
-                if (is_k) mbar_wait_bounded(&bars->q_full, 0, nullptr, kDrainLimitNs);
+                mbar_wait_bounded(&bars->q_full, 0, nullptr, kDrainLimitNs);
             }
         } else if (warp == 9 && lane == 0) {
             // ---------------------------------------------- MMA issuer
@@ -392,29 +386,25 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             const uint64_t dk0 = kdesc(sK);
             const uint64_t km0 = mndesc(sK, kHalf128);
             constexpr uint64_t kTileStep = kTileBytes >> 4;
-            // dQ += dS(jj) K(jj), key half by key half as the softmax releases them
+            // dQ += dS(jj) K(jj) once the softmax has written all of dS(jj)
+            // (two releases, one per key half, measured slower: one more
+            // wait per tile for the issuing thread)
             auto dq_mma = [&](int jj, int kst_jj) -> bool {
                 const int pb = jj & 1;
                 const uint64_t km = km0 + (uint64_t)kst_jj * kTileStep;
                 const uint32_t sb = tmem + 128 * pb;
+                if (!wait(&bars->ds_full[pb], (jj >> 1) & 1, ctl)) return false;
+                tc_fence_after();
 #pragma unroll
-                for (int wg = 0; wg < 2; ++wg) {
-                    if (!wait(&bars->ds_full[2 * pb + wg], (jj >> 1) & 1, ctl)) return false;
-                    tc_fence_after();
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int s = 4 * wg + q;
-                        mma_ts(tmem + 384, sb + 64 * wg + 8 * q, km + (uint64_t)s * kMnStep, id_mn,
-                               (jj > 0 || s > 0) ? 1u : 0u);
-                    }
-                }
+                for (int s = 0; s < 8; ++s)
+                    mma_ts(tmem + 384, sb + 64 * (s >> 2) + 8 * (s & 3), km + (uint64_t)s * kMnStep,
+                           id_mn, (jj > 0 || s > 0) ? 1u : 0u);
                 return true;
             };
             int kst = 0, kph = 0, kst_prev = 0;      // K stage of tile j, its phase, and of j - 1
             for (int j = 0; ok && j < n_kv; ++j) {
                 const int st = j & 1;                // S buffer and V stage
-                const uint32_t ph = (j >> 1) & 1;
-                if (!(ok = wait(&bars->k_full[kst], kph, ctl))) break;
+                if (!(ok = wait(&bars->kv_full[kst], kph, ctl))) break;   // K(j) and V(j)
                 tc_fence_after();
                 const uint64_t dk = dk0 + (uint64_t)kst * kTileStep;
 #pragma unroll
@@ -422,7 +412,6 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                     const uint64_t off = koff(s, kHalf128);
                     mma_ss(tmem + 128 * st, dq_d + off, dk + off, id_kk, s > 0 ? 1u : 0u);
                 }
-                if (!(ok = wait(&bars->v_full[st], ph, ctl))) break;
                 if (j > 0 && !(ok = wait(&bars->dp_free, (j - 1) & 1, ctl))) break;
                 tc_fence_after();
                 const uint64_t dv = st ? dv1 : dv0;
@@ -490,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->ds_full[2 * buf + wg]);
+            if (lane == 0) mbar_arrive(&bars->ds_full[buf]);
         }
         if (ok) ok = wait_warp(&bars->o_done, 0, ctl);
         tc_fence_after();
@@ -533,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
 // ======================================================================
 namespace dkv {
 
-constexpr int kStages = 4;   // Q / dO / (lse, D) ring depth
+constexpr int kStages = 4;   // Q / dO / (lse, D) ring depth; Q and dO of a tile share a barrier
 
 struct Smem {
     static constexpr int k_off = 0;
@@ -573,8 +562,7 @@ static_assert(sizeof(Params) <= 4096, "kernel parameters must fit the 4 KB param
 
 struct Bars {
     uint64_t kv_full;
-    uint64_t q_full[kStages], q_empty[kStages];
-    uint64_t do_full[kStages], do_empty[kStages];
+    uint64_t qd_full[kStages], qd_empty[kStages];   // Q and dO of query tile i in stage i % 4
     uint64_t l_full[kStages], l_empty[kStages];
     uint64_t s_full[2];   // S^T and dP^T of the tile with this buffer are in tensor memory
     uint64_t p_full[2];   // every softmax warp has written its P^T and dS^T
@@ -636,10 +624,8 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&bars->q_full[i], 1);
-            mbar_init(&bars->q_empty[i], 1);
-            mbar_init(&bars->do_full[i], 1);
-            mbar_init(&bars->do_empty[i], 1);
+            mbar_init(&bars->qd_full[i], 1);
+            mbar_init(&bars->qd_empty[i], 1);
             mbar_init(&bars->l_full[i], 32);   // every lane of the loader warp
             mbar_init(&bars->l_empty[i], 8);   // one elected lane per softmax warp
         }
@@ -681,40 +667,36 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
 
     if (warp >= 8) {
         regs_dec<kRegsProducer>();
-        if ((warp == 8 || warp == 10) && lane == 0) {
-            // ---------------------------------------------- TMA: K, V, then Q (warp 8) / dO (warp 10)
-            const bool is_q = warp == 8;
-            const CUtensorMap* tm = is_q ? p.tm_q : p.tm_do;
-            uint8_t* ring = smem + (is_q ? Smem::q_off : Smem::do_off);
-            uint64_t* full = is_q ? bars->q_full : bars->do_full;
-            uint64_t* empty = is_q ? bars->q_empty : bars->do_empty;
-            if (is_q) {
-                mbar_arrive_expect_tx(&bars->kv_full, 2 * kTileBytes);
-                tma_load_4d(smem + Smem::k_off, &p.tm_k[seg], &bars->kv_full, 0, h, krow0, b);
-                tma_load_4d(smem + Smem::k_off + kHalf128, &p.tm_k[seg], &bars->kv_full, 64, h,
-                            krow0, b);
-                tma_load_4d(smem + Smem::v_off, &p.tm_v[seg], &bars->kv_full, 0, h, krow0, b);
-                tma_load_4d(smem + Smem::v_off + kHalf128, &p.tm_v[seg], &bars->kv_full, 64, h,
-                            krow0, b);
-            }
+        if (warp == 8 && lane == 0) {
+            // ---------------------------------------------- TMA: K, V, then Q and dO
+            mbar_arrive_expect_tx(&bars->kv_full, 2 * kTileBytes);
+            tma_load_4d(smem + Smem::k_off, &p.tm_k[seg], &bars->kv_full, 0, h, krow0, b);
+            tma_load_4d(smem + Smem::k_off + kHalf128, &p.tm_k[seg], &bars->kv_full, 64, h, krow0,
+                        b);
+            tma_load_4d(smem + Smem::v_off, &p.tm_v[seg], &bars->kv_full, 0, h, krow0, b);
+            tma_load_4d(smem + Smem::v_off + kHalf128, &p.tm_v[seg], &bars->kv_full, 64, h, krow0,
+                        b);
             int issued = 0;
             for (int i = 0; i < nq; ++i) {
                 const int st = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
                 const int qs = i < nq_vis ? 0 : 1;
                 const int row = qs ? (i - nq_vis) * 64 : qvs + i * 64;
-                if (!wait(&empty[st], ph ^ 1, ctl)) break;
-                uint8_t* dst = ring + st * kQ64Bytes;
-                mbar_arrive_expect_tx(&full[st], kQ64Bytes);
-                tma_load_4d(dst, &tm[qs], &full[st], 0, h, row, b);
-                tma_load_4d(dst + kHalf64, &tm[qs], &full[st], 64, h, row, b);
+                if (!wait(&bars->qd_empty[st], ph ^ 1, ctl)) break;
+                uint8_t* dq_ = smem + Smem::q_off + st * kQ64Bytes;
+                uint8_t* ddo = smem + Smem::do_off + st * kQ64Bytes;
+                mbar_arrive_expect_tx(&bars->qd_full[st], 2 * kQ64Bytes);
+                tma_load_4d(dq_, &p.tm_q[qs], &bars->qd_full[st], 0, h, row, b);
+                tma_load_4d(dq_ + kHalf64, &p.tm_q[qs], &bars->qd_full[st], 64, h, row, b);
+                tma_load_4d(ddo, &p.tm_do[qs], &bars->qd_full[st], 0, h, row, b);
+                tma_load_4d(ddo + kHalf64, &p.tm_do[qs], &bars->qd_full[st], 64, h, row, b);
                 ++issued;
             }
             if (ctl->abort) {
                 for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-                    mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1, nullptr,
+                    mbar_wait_bounded(&bars->qd_full[i % kStages], (i / kStages) & 1, nullptr,
                                       kDrainLimitNs);
-                if (is_q) mbar_wait_bounded(&bars->kv_full, 0, nullptr, kDrainLimitNs);
+                mbar_wait_bounded(&bars->kv_full, 0, nullptr, kDrainLimitNs);
             }
         } else if (warp == 11) {
             // ---------------------------------------------- (lse * log2 e, D) of each query tile
@@ -761,16 +743,14 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 for (int s = 0; s < 4; ++s)
                     mma_ts(tmem + 384, tmem + 128 + 64 * pb + packed_col(s),
                            qm + (uint64_t)s * kMnStep, id_mn, (ii > 0 || s > 0) ? 1u : 0u);
-                mma_commit(&bars->q_empty[pst]);
-                mma_commit(&bars->do_empty[pst]);
+                mma_commit(&bars->qd_empty[pst]);
                 return true;
             };
             for (int i = 0; ok && i < nq; ++i) {
                 const int st = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
                 const int buf = i & 1;
-                if (!(ok = wait(&bars->q_full[st], ph, ctl))) break;
-                if (!(ok = wait(&bars->do_full[st], ph, ctl))) break;
+                if (!(ok = wait(&bars->qd_full[st], ph, ctl))) break;   // Q and dO of tile i
                 tc_fence_after();
                 const uint64_t qd = kdesc(sQ + st * kQ64Bytes);
                 const uint64_t dod = kdesc(sDO + st * kQ64Bytes);
