@@ -658,7 +658,7 @@ def run_ours(args):
     qn_ms = time_ms(lambda: api.joint_attention_qnorm(
         t["q_vis"], k_n_vis, t["v_vis"], t["q_ctx"], k_n_ctx, t["v_ctx"], t["gq_vis"],
         t["gq_ctx"], grid=w.grid, pos_scale=w.pos_scale, ctx_len=t["ctx_len"],
-        o_vis=t["o_vis"], o_ctx=t["o_ctx"]), reps=10)
+        o_vis=t["o_vis"], o_ctx=t["o_ctx"], workspace=attn_ws), reps=10)
     qn_rows = {"qnorm_in_attention": {
         "k_norm_rope_ms": kq_ms, "attention_qnorm_ms": qn_ms,
         "attention_qnorm_TFLOP/s": w.attention_flops() / (qn_ms * 1e-3) / 1e12,

@@ -200,6 +200,24 @@ MMDIT_API int mmdit_joint_attention_qnorm(const void* q_vis, const void* k_vis,
                                           int Nc, int H, int D, float softmax_scale,
                                           mmdit_dtype dt, void* stream);
 
+/* mmdit_joint_attention_qnorm with the split tail of mmdit_joint_attention_ws:
+ * workspace (device, 256-byte aligned, workspace_bytes long, or NULL) lets the
+ * items past the last whole wave of CTAs be split over their key tiles and
+ * merged by a second kernel (each piece normalises its own copy of the query
+ * tiles).  A NULL or too small workspace gives the unsplit launch.
+ * Other arguments as mmdit_joint_attention_qnorm.
+ * Errors: MMDIT_ERR_ARG (also workspace_bytes < 0) / _SHAPE / _ALIGN /
+ * _UNSUPPORTED / _CUDA. */
+MMDIT_API int mmdit_joint_attention_qnorm_ws(const void* q_vis, const void* k_vis,
+                                             const void* v_vis, const void* q_ctx,
+                                             const void* k_ctx, const void* v_ctx,
+                                             const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                                             const float* q_scale_vis, const float* q_scale_ctx,
+                                             const mmdit_grid* grid, float eps, void* workspace,
+                                             long long workspace_bytes, int B, int Nv, int Nc,
+                                             int H, int D, float softmax_scale, mmdit_dtype dt,
+                                             void* stream);
+
 /* Symmetric int8 quantisation for the 8-bit attention ["Wan 2.1" report,
  * section 4.4.3: Int8 for S = Q K^T]: x [B, N, H, D] bf16 -> codes [B, N, H, D]
  * int8 and one fp32 scale per `block` consecutive tokens of a (sample, head):

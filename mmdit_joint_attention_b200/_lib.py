@@ -102,6 +102,9 @@ def lib():
                                         _i, _vp]
         L.mmdit_joint_attention_qnorm.argtypes = ([_vp] * 11 + [ctypes.POINTER(Grid), _f] +
                                                   [_i] * 5 + [_f, _i, _vp])
+        L.mmdit_joint_attention_qnorm_ws.argtypes = ([_vp] * 11 + [ctypes.POINTER(Grid), _f, _vp,
+                                                      ctypes.c_longlong] + [_i] * 5 +
+                                                     [_f, _i, _vp])
         L.mmdit_quantize_int8.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
         L.mmdit_quantize_v_e4m3.argtypes = [_vp] * 6 + [_i] * 5 + [_vp]
         L.mmdit_joint_attention_q8.argtypes = [_vp] * 14 + [_i] * 5 + [_f, _vp]
@@ -150,7 +153,7 @@ def lib():
         L.mmdit_status_string.restype = ctypes.c_char_p
         for name in ("mmdit_qk_norm_rope", "mmdit_qk_norm_rope_text", "mmdit_qk_norm_rope_window",
                      "mmdit_qk_norm_rope_bwd", "mmdit_qk_norm_rope_text_bwd", "mmdit_k_norm_rope",
-                     "mmdit_joint_attention_qnorm",
+                     "mmdit_joint_attention_qnorm", "mmdit_joint_attention_qnorm_ws",
                      "mmdit_quantize_int8", "mmdit_quantize_v_e4m3", "mmdit_joint_attention_q8",
                      "mmdit_window_permute", "mmdit_joint_attention",
                      "mmdit_joint_attention_fwd", "mmdit_joint_attention_bwd",

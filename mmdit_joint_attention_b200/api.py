@@ -231,10 +231,12 @@ def joint_attention_qnorm(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, q_scale_vis,
                           grid: Optional[Sequence[int]] = None, pos_scale=(1.0, 1.0, 1.0),
                           ctx_len=None, eps: float = 1e-6, rope_base: float = 10000.0,
                           split=(16, 56, 56), softmax_scale: Optional[float] = None, o_vis=None,
-                          o_ctx=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                          o_ctx=None, stream=None, workspace: Optional[torch.Tensor] = None
+                          ) -> Tuple[torch.Tensor, torch.Tensor]:
     """joint_attention on raw q: the kernel RMS-normalises q (and rotates the
     visual rows when ``grid`` is given) after loading it.  k must already be
-    normalised (k_norm_rope)."""
+    normalised (k_norm_rope).  With ``workspace`` (attention_workspace()), the
+    launch's tail is split over its keys as in joint_attention."""
     dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx)
     _f32(q_scale_vis, q_scale_ctx)
     B, Nv, H, D = q_vis.shape
@@ -246,12 +248,20 @@ def joint_attention_qnorm(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, q_scale_vis,
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
     g = make_grid(grid, pos_scale, rope_base, split) if grid is not None else None
-    st = _lib.lib().mmdit_joint_attention_qnorm(
-        _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
-        _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(q_scale_vis), _ptr(q_scale_ctx),
-        ctypes.byref(g) if g is not None else None, eps, B, Nv, Nc, H, D, softmax_scale, dt,
-        _stream(stream))
-    check("mmdit_joint_attention_qnorm", st)
+    args = (_ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
+            _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(q_scale_vis), _ptr(q_scale_ctx),
+            ctypes.byref(g) if g is not None else None, eps)
+    tail = (B, Nv, Nc, H, D, softmax_scale, dt, _stream(stream))
+    if workspace is None:
+        name = "mmdit_joint_attention_qnorm"
+        st = _lib.lib().mmdit_joint_attention_qnorm(*args, *tail)
+    else:
+        if workspace.dtype != torch.uint8 or not workspace.is_cuda or not workspace.is_contiguous():
+            raise TypeError("workspace must be a contiguous uint8 CUDA tensor")
+        name = "mmdit_joint_attention_qnorm_ws"
+        st = _lib.lib().mmdit_joint_attention_qnorm_ws(*args, _ptr(workspace), workspace.numel(),
+                                                       *tail)
+    check(name, st)
     return o_vis, o_ctx
 
 

@@ -397,12 +397,17 @@ int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vi
                                 nullptr, B, Nv, Nc, H, D, softmax_scale, nullptr, dt, stream);
 }
 
-int mmdit_joint_attention_qnorm(const void* q_vis, const void* k_vis, const void* v_vis,
-                                const void* q_ctx, const void* k_ctx, const void* v_ctx,
-                                const int32_t* ctx_len, void* o_vis, void* o_ctx,
-                                const float* q_scale_vis, const float* q_scale_ctx,
-                                const mmdit_grid* grid, float eps, int B, int Nv, int Nc, int H,
-                                int D, float softmax_scale, mmdit_dtype dt, void* stream) {
+namespace {
+
+int joint_attention_qnorm_impl(const void* q_vis, const void* k_vis, const void* v_vis,
+                               const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                               const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                               const float* q_scale_vis, const float* q_scale_ctx,
+                               const mmdit_grid* grid, float eps, int B, int Nv, int Nc, int H,
+                               int D, float softmax_scale, mmdit_dtype dt, void* stream,
+                               void* workspace, long long workspace_bytes) {
+    if (workspace_bytes < 0) return MMDIT_ERR_ARG;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MMDIT_ERR_ALIGN;
     if (!dtype_ok(dt) || B < 0 || Nv < 0 || Nc < 0 || H < 0) return MMDIT_ERR_ARG;
     if (!(eps >= 0.f) || !std::isfinite(eps)) return MMDIT_ERR_ARG;
     if (dt != MMDIT_BF16) return MMDIT_ERR_UNSUPPORTED;
@@ -432,12 +437,38 @@ int mmdit_joint_attention_qnorm(const void* q_vis, const void* k_vis, const void
     }
     if (ctx_len && (reinterpret_cast<uintptr_t>(ctx_len) & 3u)) return MMDIT_ERR_ALIGN;
     if ((long long)Nv + Nc > (1LL << 30)) return MMDIT_ERR_UNSUPPORTED;
-    const int r = launch_joint_attention_bf16(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len,
-                                              o_vis, o_ctx, nullptr, B, Nv, Nc, H, softmax_scale,
-                                              nullptr, static_cast<cudaStream_t>(stream), &qn);
+    const int r = launch_joint_attention_bf16(
+        q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx, nullptr, B, Nv, Nc, H,
+        softmax_scale, nullptr, static_cast<cudaStream_t>(stream), &qn,
+        static_cast<float*>(workspace), workspace ? workspace_bytes : 0);
     if (r == 0) return MMDIT_OK;
     set_last_error("joint_attention_qnorm", r);
     return MMDIT_ERR_CUDA;
+}
+
+}  // namespace
+
+int mmdit_joint_attention_qnorm(const void* q_vis, const void* k_vis, const void* v_vis,
+                                const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                                const float* q_scale_vis, const float* q_scale_ctx,
+                                const mmdit_grid* grid, float eps, int B, int Nv, int Nc, int H,
+                                int D, float softmax_scale, mmdit_dtype dt, void* stream) {
+    return joint_attention_qnorm_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis,
+                                      o_ctx, q_scale_vis, q_scale_ctx, grid, eps, B, Nv, Nc, H, D,
+                                      softmax_scale, dt, stream, nullptr, 0);
+}
+
+int mmdit_joint_attention_qnorm_ws(const void* q_vis, const void* k_vis, const void* v_vis,
+                                   const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                   const int32_t* ctx_len, void* o_vis, void* o_ctx,
+                                   const float* q_scale_vis, const float* q_scale_ctx,
+                                   const mmdit_grid* grid, float eps, void* workspace,
+                                   long long workspace_bytes, int B, int Nv, int Nc, int H, int D,
+                                   float softmax_scale, mmdit_dtype dt, void* stream) {
+    return joint_attention_qnorm_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis,
+                                      o_ctx, q_scale_vis, q_scale_ctx, grid, eps, B, Nv, Nc, H, D,
+                                      softmax_scale, dt, stream, workspace, workspace_bytes);
 }
 
 int mmdit_quantize_int8(const void* x, void* codes, float* scales, int B, int N, int H, int D,

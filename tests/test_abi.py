@@ -308,6 +308,22 @@ def test_attention_ws_validation(L):
     assert f(*a) == 0
 
 
+def test_attention_qnorm_ws_validation(L):
+    f = L.mmdit_joint_attention_qnorm_ws
+    # q, k, v of both streams, ctx_len, o of both streams, q scales, grid, eps,
+    # workspace, bytes, B, Nv, Nc, H, D, softmax_scale, dtype, stream
+    args = lambda ws, n: (P, P, P, P, P, P, None, P, P, P, P, None, 1e-6, ws, n, 1, 8, 8, 2, 128,
+                          0.1, 1, None)
+    assert f(*args(ctypes.c_void_p(272), 1 << 20)) == -3          # workspace not 256-aligned
+    assert f(*args(ctypes.c_void_p(256), -1)) == -1
+    a = list(args(None, 0)); a[19] = 64                              # D != 128
+    assert f(*a) == -4
+    a = list(args(None, 0)); a[21] = 0                               # fp32: bf16 only
+    assert f(*a) == -4
+    a = list(args(None, 0)); a[15] = 0                               # B = 0: nothing to do
+    assert f(*a) == 0
+
+
 def _plan_rule(B, Nv, Nc, H, nsm, ws):
     """The split-tail rule restated: the items past the last whole wave
     (total mod nsm) are split into as many pieces as fill the SMs, at least 2

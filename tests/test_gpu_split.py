@@ -88,3 +88,31 @@ def test_split_tail_close_to_unsplit_and_small_workspace_falls_back():
     fin = torch.isfinite(lse_u)
     assert torch.equal(torch.isfinite(lse_s), fin)
     assert (lse_s[fin] - lse_u[fin]).abs().max().item() <= 1e-4
+
+
+@pytest.mark.parametrize("case", ["all_split", "whole_then_split"])
+def test_split_tail_with_qnorm(case):
+    """The split tail with q normalised and rotated inside the kernel
+    (mmdit_joint_attention_qnorm_ws): every piece normalises its own copy of
+    the query tiles, and the merged rows match the oracle."""
+    w = CASES[case]
+    inp = I.make_inputs(w, seed=7, parts=("qkv", "scales"))
+    t = device_inputs(inp)
+    cl = t["ctx_len"] if w.ctx_len is not None else None
+    kv = api.k_norm_rope(t["k_vis"].clone(), t["gk_vis"], grid=w.grid, pos_scale=w.pos_scale)
+    kc = api.k_norm_rope(t["k_ctx"].clone(), t["gk_ctx"])
+    fv, fc = api.joint_attention_qnorm(t["q_vis"], kv, t["v_vis"], t["q_ctx"], kc, t["v_ctx"],
+                                       t["gq_vis"], t["gq_ctx"], grid=w.grid,
+                                       pos_scale=w.pos_scale, ctx_len=cl,
+                                       workspace=api.attention_workspace())
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+    rq, rk = oracle.qk_norm_rope(inp["q_vis"].f64, inp["k_vis"].f64, inp["gq_vis"],
+                                 inp["gk_vis"], grid=w.grid, pos_scale=w.pos_scale)
+    cq, ck = oracle.qk_norm_rope(inp["q_ctx"].f64, inp["k_ctx"].f64, inp["gq_ctx"],
+                                 inp["gk_ctx"], grid=None)
+    rq, rk, cq, ck = (I.round_f64_to_bf16(a) for a in (rq, rk, cq, ck))
+    rv, rc = oracle.joint_attention(rq, rk, inp["v_vis"].f64, cq, ck, inp["v_ctx"].f64,
+                                    inp["ctx_len"])
+    parity(from_dev(fv), rv, "bf16", f"{case} qnorm split o_vis")
+    parity(from_dev(fc), rc, "bf16", f"{case} qnorm split o_ctx")
