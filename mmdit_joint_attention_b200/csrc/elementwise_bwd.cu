@@ -107,14 +107,6 @@ static_assert((1 << kModBits) == kMods, "moments per iteration: 4, 8 or 16");
 // Bit 0: a bounded wait expired in an elementwise backward kernel.
 __device__ unsigned int g_elem_status = 0;
 
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // Sum of kMods values over the warp: each of the first kModBits steps swaps
 // half of the remaining values with the partner lane (xor 16, 8, ...), the
 // last steps add the partners' single values, so that lane l ends with the

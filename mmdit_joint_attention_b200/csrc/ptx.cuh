@@ -76,6 +76,16 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, ui
 
 // Makes this thread's generic-proxy shared-memory writes visible to later
 // async-proxy reads (tcgen05.mma operands, TMA).
+// Untiled bulk copy global -> this CTA's shared memory, completing on an
+// mbarrier's transaction count.  Both addresses and `bytes` must be multiples
+// of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
