@@ -692,7 +692,8 @@ def run_ours(args):
              ("dq_vis", "dk_vis", "dv_vis", "dq_ctx", "dk_ctx", "dv_ctx")}
     qkv = (t["nq_vis"], t["nk_vis"], t["v_vis"], t["nq_ctx"], t["nk_ctx"], t["v_ctx"])
     fwd_lse_ms = time_ms(lambda: api.joint_attention_fwd(
-        *qkv, t["ctx_len"], o_vis=t["o_vis"], o_ctx=t["o_ctx"], lse=lse), reps=10)
+        *qkv, t["ctx_len"], o_vis=t["o_vis"], o_ctx=t["o_ctx"], lse=lse, workspace=attn_ws),
+        reps=10)
     bwd_ms = time_ms(lambda: api.joint_attention_bwd(
         *qkv, t["o_vis"], t["o_ctx"], do_vis, do_ctx, lse, t["ctx_len"], delta=delta,
         grads=grads), reps=5)
