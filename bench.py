@@ -46,7 +46,7 @@ from mmdit_joint_attention_b200 import inputs as I  # noqa: E402
 METRIC = "joint-attention TFLOP/s and % bf16 peak at 480p/81f; norm/RoPE GB/s % HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ATTN_SRC = os.path.join(ROOT, "mmdit_joint_attention_b200", "csrc", "attention_tc.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "joint_attn_bf16_480p.md")
+PROFILES = os.path.join(ROOT, "profiles")
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -67,13 +67,11 @@ def attn_source_hash() -> str:
 
 
 def recorded_traffic(w):
-    """DRAM bytes per attention launch from the committed ncu summary of the
-    480p workload, if it was taken on the current kernel source and the run
-    is that workload (else None)."""
-    if w.name != "480p":
-        return None
+    """DRAM bytes per attention launch of workload ``w`` from the committed
+    ncu summary of that workload (profiles/joint_attn_bf16_<name>.md), if
+    there is one and it was taken on the current kernel source (else None)."""
     try:
-        text = open(TRAFFIC_FILE).read()
+        text = open(os.path.join(PROFILES, f"joint_attn_bf16_{w.name}.md")).read()
     except OSError:
         return None
     m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
@@ -809,7 +807,7 @@ def run_ours(args):
             "value": xw.attention_flops() * world / (x_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "data": f"synthetic (seeded torch generator on the device, N(0,1) inputs of the "
                     f"{xw.name} latent shape)",
-            "roofline": roofline(xk, pk, pk_src, None),
+            "roofline": roofline(xk, pk, pk_src, recorded_traffic(xw)),
             "kernels": xk, "gpu_launches": xlaunches * args.extra_steps, "clocks": xclk}
         del xt, xstep
 
