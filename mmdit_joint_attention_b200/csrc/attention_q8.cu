@@ -48,7 +48,6 @@ constexpr int kTileBytes = 128 * 128;   // 128 rows x 128 one-byte elements
 constexpr int kThreads = 384;
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
-constexpr int kWarpLoadV = 10;
 constexpr int kRegsLaunch = 168;
 constexpr int kRegsProducer = 72;
 constexpr int kRegsSoftmax = 216;
@@ -83,10 +82,9 @@ struct Params {
 
 struct Bars {
     uint64_t q_full;
-    uint64_t k_full[kStages], k_empty[kStages];
-    uint64_t v_full[kStages], v_empty[kStages];
+    uint64_t k_full[kStages], k_empty[kStages];   // stage j % 2: K(j) and V(j - 1)
     uint64_t s_full[2], o_done[2];
-    uint64_t p_full[4];    // [2 i + h]: keys 64h..64h+63 of P_i are in tensor memory
+    uint64_t p_full[2];    // [i]: all of P_i is in tensor memory
     uint64_t drain;
     uint64_t wait_ns;
     uint32_t tmem_base;
@@ -124,23 +122,31 @@ __device__ __forceinline__ uint64_t vdesc(uint32_t addr) {
     return smem_desc_sw128(addr, kTileBytes, 1024);
 }
 
-__device__ __forceinline__ void stream_tiles(const CUtensorMap* tm, uint8_t* ring, uint64_t* full,
-                                             uint64_t* empty, int n_kv, int kv_vis, int h, int b,
-                                             Bars* bars) {
+// Streams the key tiles through the K/V ring: stage j % 2 receives K(j) and
+// V(j - 1), the operands of the MMA issuer's iteration j, under one barrier
+// (only K(0) at j = 0, only V(n_kv - 1) at j = n_kv), as in the bf16 kernel.
+// On an abort, waits (bounded) for the copies it issued before returning.
+__device__ __forceinline__ void stream_kv(const Params& p, uint8_t* smem, Bars* bars, int n_kv,
+                                          int kv_vis, int h, int b) {
     int issued = 0;
-    for (int j = 0; j < n_kv; ++j) {
-        const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        const int seg = j < kv_vis ? 0 : 1;
-        const int row = (seg == 0 ? j : j - kv_vis) * kBlock;
-        if (!wait(&empty[st], ph ^ 1, bars)) break;
-        mbar_arrive_expect_tx(&full[st], kTileBytes);
-        tma_load_4d(ring + st * kTileBytes, &tm[seg], &full[st], 0, h, row, b);
+    for (int j = 0; j <= n_kv; ++j) {
+        const int st = j & 1;
+        if (!wait(&bars->k_empty[st], ((j >> 1) & 1) ^ 1, bars)) break;
+        const int bytes = (j < n_kv ? kTileBytes : 0) + (j > 0 ? kTileBytes : 0);
+        mbar_arrive_expect_tx(&bars->k_full[st], bytes);
+        for (int w = 0; w < 2; ++w) {    // w = 0: K(j), w = 1: V(j - 1)
+            if ((w == 0 && j == n_kv) || (w == 1 && j == 0)) continue;
+            const int jj = j - w;
+            const int seg = jj < kv_vis ? 0 : 1;
+            const int row = (seg == 0 ? jj : jj - kv_vis) * kBlock;
+            uint8_t* t = smem + (w == 0 ? Smem::k_off : Smem::v_off) + st * kTileBytes;
+            tma_load_4d(t, w == 0 ? &p.tm_k[seg] : &p.tm_v[seg], &bars->k_full[st], 0, h, row, b);
+        }
         ++issued;
     }
     if (bars->abort) {
         for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-            mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1, nullptr, kDrainLimitNs);
+            mbar_wait_bounded(&bars->k_full[j & 1], (j >> 1) & 1, nullptr, kDrainLimitNs);
     }
 }
 
@@ -232,13 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_q8_kernel(const __grid
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&bars->k_full[i], 1);
             mbar_init(&bars->k_empty[i], 1);
-            mbar_init(&bars->v_full[i], 1);
-            mbar_init(&bars->v_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->s_full[i], 1);
-            mbar_init(&bars->p_full[2 * i], 4);
-            mbar_init(&bars->p_full[2 * i + 1], 4);
+            mbar_init(&bars->p_full[i], 4);   // one elected lane per softmax warp
             mbar_init(&bars->o_done[i], 1);
         }
         mbar_init(&bars->drain, 1);
@@ -286,14 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_q8_kernel(const __grid
             if (has1)
                 tma_load_4d(smem + Smem::q_off + kTileBytes, &p.tm_q[s1], &bars->q_full, 0, h, r1,
                             b);
-            stream_tiles(p.tm_k, smem + Smem::k_off, bars->k_full, bars->k_empty, n_kv, kv_vis, h,
-                         b, bars);
+            stream_kv(p, smem, bars, n_kv, kv_vis, h, b);
             if (bars->abort) mbar_wait_bounded(&bars->q_full, 0, nullptr, kDrainLimitNs);
         }
-    } else if (warp == kWarpLoadV) {
-        if (lane == 0)
-            stream_tiles(p.tm_v, smem + Smem::v_off, bars->v_full, bars->v_empty, n_kv, kv_vis, h,
-                         b, bars);
     } else if (warp == kWarpMma && lane == 0) {
         // one thread issues every MMA: PV_0(j-1), QK_0(j), PV_1(j-1), QK_1(j)
         constexpr uint32_t idesc_qk = idesc_s8_s32(128, 128);
@@ -310,47 +308,34 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_q8_kernel(const __grid
             for (int s = 0; s < 4; ++s)
                 mma_ss_i8(tmem + 128 * i, dq + 2 * s, dk + 2 * s, idesc_qk, s > 0 ? 1u : 0u);
         };
-        // O_i += P'_i V, two k-steps of 32 keys per released half of P'_i
+        // O_i += P'_i V (four k-steps of 32 keys) once the softmax has written
+        // all of P'_i
         auto pv = [&](int i, int st, bool acc, uint32_t par) -> bool {
             const uint64_t dv = st == 0 ? dv0 : dv1;
+            if (!wait(&bars->p_full[i], par, bars)) return false;
+            tc_fence_after();
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                if (!wait(&bars->p_full[2 * i + hh], par, bars)) return false;
-                tc_fence_after();
-#pragma unroll
-                for (int s = 2 * hh; s < 2 * hh + 2; ++s)
-                    mma_ts_f8(tmem + 256 + 128 * i, tmem + 128 * i + 8 * s,
-                              dv + (uint64_t)s * (4096 >> 4), idesc_pv, (acc || s > 0) ? 1u : 0u);
-            }
+            for (int s = 0; s < 4; ++s)
+                mma_ts_f8(tmem + 256 + 128 * i, tmem + 128 * i + 8 * s,
+                          dv + (uint64_t)s * (4096 >> 4), idesc_pv, (acc || s > 0) ? 1u : 0u);
             return true;
         };
-        for (int j = 0; ok && j < n_kv; ++j) {
-            const int st = j % kStages;
-            const uint32_t ph = (j / kStages) & 1;
-            const int pst = (j + kStages - 1) % kStages;
-            const uint32_t pph = ((j - 1) / kStages) & 1;
-            if (!(ok = wait(&bars->k_full[st], ph, bars))) break;
-            if (j > 0 && !(ok = wait(&bars->v_full[pst], pph, bars))) break;
+        // iteration j: PV_i(j - 1) then QK_i(j) per tile from stage j % 2
+        for (int j = 0; ok && j <= n_kv; ++j) {
+            const int st = j & 1;
+            if (!(ok = wait(&bars->k_full[st], (j >> 1) & 1, bars))) break;   // K(j), V(j - 1)
             for (int i = 0; i < ntile; ++i) {
-                if (j > 0 && !(ok = pv(i, pst, j > 1, (j - 1) & 1))) break;
-                tc_fence_after();
-                qk(i, st);
-                mma_commit(&bars->s_full[i]);
+                if (j > 0 && !(ok = pv(i, st, j > 1, (j - 1) & 1))) break;
+                if (j < n_kv) {
+                    if (j == 0) tc_fence_after();
+                    qk(i, st);
+                    mma_commit(&bars->s_full[i]);
+                } else {
+                    mma_commit(&bars->o_done[i]);
+                }
             }
             if (!ok) break;
-            if (j > 0) mma_commit(&bars->v_empty[pst]);
             mma_commit(&bars->k_empty[st]);
-        }
-        if (ok) {
-            const int j = n_kv;
-            const int pst = (j - 1) % kStages;
-            const uint32_t pph = ((j - 1) / kStages) & 1;
-            ok = wait(&bars->v_full[pst], pph, bars);
-            for (int i = 0; ok && i < ntile; ++i) {
-                if (!(ok = pv(i, pst, j > 1, (j - 1) & 1))) break;
-                mma_commit(&bars->o_done[i]);
-            }
-            if (ok) mma_commit(&bars->v_empty[pst]);
         }
         mma_commit(&bars->drain);
         if (!mbar_wait_bounded(&bars->drain, 0, nullptr, kDrainLimitNs))
@@ -420,11 +405,11 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_q8_kernel(const __grid
                     sum += valid >= 128 ? p_half<false>(r, pk, hh, c2, b2, 64)
                                         : p_half<true>(r, pk, hh, c2, b2, valid - 64 * hh);
                     tmem_st16(tS + 16 * hh, pk);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->p_full[2 * i + hh]);
                 }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->p_full[i]);
                 l_run += sum;
             }
             if (ok) ok = wait_warp(&bars->o_done[i], 0, bars);
