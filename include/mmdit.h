@@ -346,6 +346,40 @@ MMDIT_API int mmdit_joint_attention_bwd(const void* q_vis, const void* k_vis, co
                                         void* dv_ctx, int B, int Nv, int Nc, int H, int D,
                                         float softmax_scale, mmdit_dtype dt, void* stream);
 
+/* Bytes of the workspace with which mmdit_joint_attention_bwd_ws (and
+ * mmdit_joint_window_attention_bwd_ws) runs the one-pass backward: an fp32
+ * dQ accumulator [B, Nv + Nc, H, 128]. */
+#define MMDIT_BWD_WORKSPACE_BYTES(B, Nv, Nc, H) \
+    ((long long)(B) * ((long long)(Nv) + (long long)(Nc)) * (long long)(H) * 512LL)
+
+/* mmdit_joint_attention_bwd with a workspace for a one-pass backward [same
+ * derivative as mmdit_joint_attention_bwd].  With bf16 and workspace_bytes >=
+ * MMDIT_BWD_WORKSPACE_BYTES(B, Nv, Nc, H), one key-stationary kernel forms
+ * dK, dV and dQ: S and dP are computed once per (key tile, query tile)
+ * instead of once in a dQ kernel and again in a dK/dV kernel (10 N^2 D
+ * executed FLOPs per sample and head instead of 14); each key tile adds its
+ * share of dQ into the workspace with bulk reduce-adds, and a last kernel
+ * scales the sums into bf16 dQ.  The order of those additions varies from
+ * run to run, so dQ is not bit-reproducible (dK and dV are; the gradients of
+ * mmdit_joint_attention_bwd are).  With f32, a NULL workspace or a smaller
+ * one, the call is mmdit_joint_attention_bwd.
+ *   workspace  DEVICE, 256-byte aligned, caller-owned, contents on entry
+ *              ignored and overwritten; must not overlap any other argument
+ *   workspace_bytes  its size
+ *   everything else as mmdit_joint_attention_bwd.
+ * Errors: as mmdit_joint_attention_bwd; MMDIT_ERR_ARG for workspace_bytes < 0,
+ * MMDIT_ERR_ALIGN for a workspace not 256-byte aligned. */
+MMDIT_API int mmdit_joint_attention_bwd_ws(const void* q_vis, const void* k_vis, const void* v_vis,
+                                           const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                           const int32_t* ctx_len, const void* o_vis,
+                                           const void* o_ctx, const void* do_vis,
+                                           const void* do_ctx, const float* lse, float* delta,
+                                           void* workspace, long long workspace_bytes,
+                                           void* dq_vis, void* dk_vis, void* dv_vis, void* dq_ctx,
+                                           void* dk_ctx, void* dv_ctx, int B, int Nv, int Nc,
+                                           int H, int D, float softmax_scale, mmdit_dtype dt,
+                                           void* stream);
+
 /* Largest B * H * (Nv + Nc) that mmdit_joint_attention_bwd_noalloc accepts:
  * 4,194,304 rows (its built-in workspace is 16 MiB of fp32 per GPU). */
 #define MMDIT_NOALLOC_MAX_ROWS (1 << 22)
@@ -469,6 +503,22 @@ MMDIT_API int mmdit_joint_window_attention_bwd(
     void* dk_vis, void* dv_vis, void* dq_ctx, void* dk_ctx, void* dv_ctx, int B, int Nv, int Nc,
     int H, int D, const mmdit_grid* grid, const mmdit_window* win, float softmax_scale,
     mmdit_dtype dt, void* stream);
+
+/* mmdit_joint_window_attention_bwd with the workspace of
+ * mmdit_joint_attention_bwd_ws: the one-pass backward (dQ reduced into the
+ * workspace, not bit-reproducible) when bf16 and workspace_bytes >=
+ * MMDIT_BWD_WORKSPACE_BYTES(B, Nv, Nc, H), else mmdit_joint_window_attention_bwd.
+ * The accumulator's visual rows are in window-major order like dq_vis.
+ *   workspace, workspace_bytes: as mmdit_joint_attention_bwd_ws; everything
+ *   else as mmdit_joint_window_attention_bwd.
+ * Errors: as mmdit_joint_window_attention_bwd and mmdit_joint_attention_bwd_ws. */
+MMDIT_API int mmdit_joint_window_attention_bwd_ws(
+    const void* q_vis, const void* k_vis, const void* v_vis, const void* q_ctx, const void* k_ctx,
+    const void* v_ctx, const int32_t* ctx_len, const void* o_vis, const void* o_ctx,
+    const void* do_vis, const void* do_ctx, const float* lse, float* delta, void* workspace,
+    long long workspace_bytes, void* dq_vis, void* dk_vis, void* dv_vis, void* dq_ctx,
+    void* dk_ctx, void* dv_ctx, int B, int Nv, int Nc, int H, int D, const mmdit_grid* grid,
+    const mmdit_window* win, float softmax_scale, mmdit_dtype dt, void* stream);
 
 /* adaLN modulate [Vimoo §2.2: a LayerNorm sits before attention and the FFN,
  * and the timestep embedding supplies a shift and a scale for its output]:

@@ -123,6 +123,8 @@ def lib():
                                                [_f, _i, _vp])
         L.mmdit_joint_attention_split_plan.argtypes = [_i] * 5 + [ctypes.c_longlong, _vp]
         L.mmdit_joint_attention_bwd.argtypes = [_vp] * 19 + [_i] * 5 + [_f, _i, _vp]
+        L.mmdit_joint_attention_bwd_ws.argtypes = ([_vp] * 14 + [ctypes.c_longlong] + [_vp] * 6 +
+                                                   [_i] * 5 + [_f, _i, _vp])
         L.mmdit_joint_window_attention.argtypes = ([_vp] * 9 + [_i] * 5 +
                                                    [ctypes.POINTER(Grid), ctypes.POINTER(Window),
                                                     _f, _i, _vp])
@@ -132,6 +134,10 @@ def lib():
         L.mmdit_joint_window_attention_bwd.argtypes = ([_vp] * 19 + [_i] * 5 +
                                                        [ctypes.POINTER(Grid),
                                                         ctypes.POINTER(Window), _f, _i, _vp])
+        L.mmdit_joint_window_attention_bwd_ws.argtypes = ([_vp] * 14 + [ctypes.c_longlong] +
+                                                          [_vp] * 6 + [_i] * 5 +
+                                                          [ctypes.POINTER(Grid),
+                                                           ctypes.POINTER(Window), _f, _i, _vp])
         L.mmdit_adaln_modulate.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp]
         L.mmdit_adaln_modulate_pair.argtypes = ([_vp] * 4 + [_i] + [_vp] * 4 + [_i] * 3 +
                                                 [_f, _i, _vp])
@@ -157,6 +163,7 @@ def lib():
                      "mmdit_quantize_int8", "mmdit_quantize_v_e4m3", "mmdit_joint_attention_q8",
                      "mmdit_window_permute", "mmdit_joint_attention",
                      "mmdit_joint_attention_fwd", "mmdit_joint_attention_bwd",
+                     "mmdit_joint_attention_bwd_ws", "mmdit_joint_window_attention_bwd_ws",
                      "mmdit_joint_attention_ws", "mmdit_joint_attention_split_plan",
                      "mmdit_joint_window_attention", "mmdit_joint_window_attention_fwd",
                      "mmdit_joint_window_attention_bwd", "mmdit_adaln_modulate",

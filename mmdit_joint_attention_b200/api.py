@@ -283,13 +283,34 @@ def joint_attention_fwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len=None,
     return o_vis, o_ctx, lse
 
 
+def bwd_workspace_bytes(B: int, Nv: int, Nc: int, H: int) -> int:
+    """Bytes of the one-pass backward's fp32 dQ accumulator [B, Nv + Nc, H, 128]."""
+    return B * (Nv + Nc) * H * 128 * 4
+
+
+def bwd_workspace(B: int, Nv: int, Nc: int, H: int, device=None) -> torch.Tensor:
+    """A workspace with which joint_attention_bwd runs the one-pass backward."""
+    return torch.empty(bwd_workspace_bytes(B, Nv, Nc, H), dtype=torch.uint8,
+                       device=device if device is not None else torch.device("cuda"))
+
+
+def _workspace_arg(workspace):
+    if workspace is None:
+        return None, 0
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise TypeError("workspace must be a contiguous CUDA tensor")
+    return workspace, workspace.numel() * workspace.element_size()
+
+
 def joint_attention_bwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, o_ctx, do_vis, do_ctx,
                         lse, ctx_len=None, softmax_scale: Optional[float] = None, delta=None,
-                        grads: Optional[dict] = None, stream=None) -> dict:
+                        grads: Optional[dict] = None, workspace=None, stream=None) -> dict:
     """Gradients dq/dk/dv of both streams for upstream gradients do_vis, do_ctx
     of the joint attention, given its outputs and lse (joint_attention_fwd).
     ``delta`` is the fp32 [B, H, Nv + Nc] workspace (allocated here if None);
-    ``grads`` may hold preallocated outputs under the returned keys."""
+    ``grads`` may hold preallocated outputs under the returned keys.  With a
+    ``workspace`` of bwd_workspace_bytes (bwd_workspace) a bf16 backward runs
+    in one pass (dQ reduced in fp32, not bit-reproducible)."""
     dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, o_ctx, do_vis, do_ctx)
     B, Nv, H, D = q_vis.shape
     Nc = q_ctx.shape[1]
@@ -305,13 +326,23 @@ def joint_attention_bwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, o_ctx, 
         raise TypeError("ctx_len must be an int32 CUDA tensor")
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(D)
-    st = _lib.lib().mmdit_joint_attention_bwd(
+    if workspace is None:
+        st = _lib.lib().mmdit_joint_attention_bwd(
+            _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
+            _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(do_vis), _ptr(do_ctx), _ptr(lse),
+            _ptr(delta), _ptr(g["dq_vis"]), _ptr(g["dk_vis"]), _ptr(g["dv_vis"]),
+            _ptr(g["dq_ctx"]), _ptr(g["dk_ctx"]), _ptr(g["dv_ctx"]), B, Nv, Nc, H, D,
+            softmax_scale, dt, _stream(stream))
+        check("mmdit_joint_attention_bwd", st)
+        return g
+    ws, nbytes = _workspace_arg(workspace)
+    st = _lib.lib().mmdit_joint_attention_bwd_ws(
         _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
         _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(do_vis), _ptr(do_ctx), _ptr(lse),
-        _ptr(delta), _ptr(g["dq_vis"]), _ptr(g["dk_vis"]), _ptr(g["dv_vis"]), _ptr(g["dq_ctx"]),
-        _ptr(g["dk_ctx"]), _ptr(g["dv_ctx"]), B, Nv, Nc, H, D, softmax_scale, dt,
-        _stream(stream))
-    check("mmdit_joint_attention_bwd", st)
+        _ptr(delta), _ptr(ws), nbytes, _ptr(g["dq_vis"]), _ptr(g["dk_vis"]), _ptr(g["dv_vis"]),
+        _ptr(g["dq_ctx"]), _ptr(g["dk_ctx"]), _ptr(g["dv_ctx"]), B, Nv, Nc, H, D, softmax_scale,
+        dt, _stream(stream))
+    check("mmdit_joint_attention_bwd_ws", st)
     return g
 
 
@@ -501,13 +532,13 @@ def joint_window_attention_bwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, 
                                do_ctx, lse, grid: Sequence[int], parts: Sequence[int],
                                ctx_len=None, softmax_scale: Optional[float] = None, delta=None,
                                grads: Optional[dict] = None, raster_in: bool = True,
-                               stream=None) -> dict:
+                               workspace=None, stream=None) -> dict:
     """Gradients of the 3D window joint attention.  q/k/v_vis are window-major
     (as for joint_window_attention) and lse comes from
     joint_window_attention_fwd.  With ``raster_in`` (the default) o_vis and
     do_vis are in raster order, as the forward writes o_vis, and are permuted
     to window-major here; the returned dq/dk/dv_vis are window-major, like
-    q/k/v_vis."""
+    q/k/v_vis.  ``workspace``: as for joint_attention_bwd."""
     dt = _dtype(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, o_ctx, do_vis, do_ctx)
     B, Nv, H, D = q_vis.shape
     Nc = q_ctx.shape[1]
@@ -528,13 +559,23 @@ def joint_window_attention_bwd(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, o_vis, 
         softmax_scale = 1.0 / math.sqrt(D)
     gr = make_grid(grid)
     w = make_window(parts)
-    st = _lib.lib().mmdit_joint_window_attention_bwd(
+    if workspace is None:
+        st = _lib.lib().mmdit_joint_window_attention_bwd(
+            _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
+            _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(do_vis), _ptr(do_ctx), _ptr(lse),
+            _ptr(delta), _ptr(g["dq_vis"]), _ptr(g["dk_vis"]), _ptr(g["dv_vis"]),
+            _ptr(g["dq_ctx"]), _ptr(g["dk_ctx"]), _ptr(g["dv_ctx"]), B, Nv, Nc, H, D,
+            ctypes.byref(gr), ctypes.byref(w), softmax_scale, dt, _stream(stream))
+        check("mmdit_joint_window_attention_bwd", st)
+        return g
+    ws, nbytes = _workspace_arg(workspace)
+    st = _lib.lib().mmdit_joint_window_attention_bwd_ws(
         _ptr(q_vis), _ptr(k_vis), _ptr(v_vis), _ptr(q_ctx), _ptr(k_ctx), _ptr(v_ctx),
         _ptr(ctx_len), _ptr(o_vis), _ptr(o_ctx), _ptr(do_vis), _ptr(do_ctx), _ptr(lse),
-        _ptr(delta), _ptr(g["dq_vis"]), _ptr(g["dk_vis"]), _ptr(g["dv_vis"]), _ptr(g["dq_ctx"]),
-        _ptr(g["dk_ctx"]), _ptr(g["dv_ctx"]), B, Nv, Nc, H, D, ctypes.byref(gr), ctypes.byref(w),
-        softmax_scale, dt, _stream(stream))
-    check("mmdit_joint_window_attention_bwd", st)
+        _ptr(delta), _ptr(ws), nbytes, _ptr(g["dq_vis"]), _ptr(g["dk_vis"]), _ptr(g["dv_vis"]),
+        _ptr(g["dq_ctx"]), _ptr(g["dk_ctx"]), _ptr(g["dv_ctx"]), B, Nv, Nc, H, D,
+        ctypes.byref(gr), ctypes.byref(w), softmax_scale, dt, _stream(stream))
+    check("mmdit_joint_window_attention_bwd_ws", st)
     return g
 
 

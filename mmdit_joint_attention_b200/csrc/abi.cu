@@ -344,7 +344,10 @@ int joint_attention_bwd_impl(const void* q_vis, const void* k_vis, const void* v
                              float* delta, void* dq_vis, void* dk_vis, void* dv_vis,
                              void* dq_ctx, void* dk_ctx, void* dv_ctx, int B, int Nv, int Nc,
                              int H, int D, float softmax_scale, mmdit_dtype dt, void* stream,
-                             const WindowTable* win) {
+                             const WindowTable* win, void* workspace = nullptr,
+                             long long workspace_bytes = 0) {
+    if (workspace_bytes < 0) return MMDIT_ERR_ARG;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MMDIT_ERR_ALIGN;
     if (!dtype_ok(dt) || B < 0 || Nv < 0 || Nc < 0 || H < 0) return MMDIT_ERR_ARG;
     if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MMDIT_ERR_ARG;
     if (D != kHeadDim) return MMDIT_ERR_UNSUPPORTED;
@@ -377,9 +380,13 @@ int joint_attention_bwd_impl(const void* q_vis, const void* k_vis, const void* v
                 static_cast<float*>(dk_ctx), static_cast<float*>(dv_ctx), B, Nv, Nc, H,
                 softmax_scale, s, win),
             "joint_attention_bwd_f32");
+    // the one-pass form when the workspace holds the fp32 dQ accumulator
+    const bool one_pass =
+        workspace && workspace_bytes >= MMDIT_BWD_WORKSPACE_BYTES(B, Nv, Nc, H);
     const int r = launch_joint_attention_bwd_bf16(
         q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis, o_ctx, do_vis, do_ctx, lse, delta,
-        dq_vis, dk_vis, dv_vis, dq_ctx, dk_ctx, dv_ctx, B, Nv, Nc, H, softmax_scale, s, win);
+        dq_vis, dk_vis, dv_vis, dq_ctx, dk_ctx, dv_ctx, B, Nv, Nc, H, softmax_scale, s, win,
+        one_pass ? static_cast<float*>(workspace) : nullptr);
     if (r == 0) return MMDIT_OK;
     set_last_error("joint_attention_bwd_bf16", r);
     return MMDIT_ERR_CUDA;
@@ -586,6 +593,20 @@ int mmdit_joint_attention_bwd(const void* q_vis, const void* k_vis, const void* 
                                     stream, nullptr);
 }
 
+int mmdit_joint_attention_bwd_ws(const void* q_vis, const void* k_vis, const void* v_vis,
+                                 const void* q_ctx, const void* k_ctx, const void* v_ctx,
+                                 const int32_t* ctx_len, const void* o_vis, const void* o_ctx,
+                                 const void* do_vis, const void* do_ctx, const float* lse,
+                                 float* delta, void* workspace, long long workspace_bytes,
+                                 void* dq_vis, void* dk_vis, void* dv_vis, void* dq_ctx,
+                                 void* dk_ctx, void* dv_ctx, int B, int Nv, int Nc, int H, int D,
+                                 float softmax_scale, mmdit_dtype dt, void* stream) {
+    return joint_attention_bwd_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis,
+                                    o_ctx, do_vis, do_ctx, lse, delta, dq_vis, dk_vis, dv_vis,
+                                    dq_ctx, dk_ctx, dv_ctx, B, Nv, Nc, H, D, softmax_scale, dt,
+                                    stream, nullptr, workspace, workspace_bytes);
+}
+
 int mmdit_joint_window_attention(const void* q_vis, const void* k_vis, const void* v_vis,
                                  const void* q_ctx, const void* k_ctx, const void* v_ctx,
                                  const int32_t* ctx_len, void* o_vis, void* o_ctx, int B, int Nv,
@@ -637,6 +658,25 @@ int mmdit_joint_window_attention_bwd(const void* q_vis, const void* k_vis, const
                                     o_ctx, do_vis, do_ctx, lse, delta, dq_vis, dk_vis, dv_vis,
                                     dq_ctx, dk_ctx, dv_ctx, B, Nv, Nc, H, D, softmax_scale, dt,
                                     stream, &tab);
+}
+
+int mmdit_joint_window_attention_bwd_ws(
+    const void* q_vis, const void* k_vis, const void* v_vis, const void* q_ctx, const void* k_ctx,
+    const void* v_ctx, const int32_t* ctx_len, const void* o_vis, const void* o_ctx,
+    const void* do_vis, const void* do_ctx, const float* lse, float* delta, void* workspace,
+    long long workspace_bytes, void* dq_vis, void* dk_vis, void* dv_vis, void* dq_ctx,
+    void* dk_ctx, void* dv_ctx, int B, int Nv, int Nc, int H, int D, const mmdit_grid* grid,
+    const mmdit_window* win, float softmax_scale, mmdit_dtype dt, void* stream) {
+    if (!grid || !win || Nv < 0) return MMDIT_ERR_ARG;
+    if (grid->T < 1 || grid->H < 1 || grid->W < 1) return MMDIT_ERR_SHAPE;
+    if ((long long)grid->T * grid->H * grid->W != (long long)Nv) return MMDIT_ERR_SHAPE;
+    const int r = check_window(grid, win);
+    if (r != MMDIT_OK) return r;
+    const WindowTable tab = make_window_table(grid->T, grid->H, grid->W, win->parts);
+    return joint_attention_bwd_impl(q_vis, k_vis, v_vis, q_ctx, k_ctx, v_ctx, ctx_len, o_vis,
+                                    o_ctx, do_vis, do_ctx, lse, delta, dq_vis, dk_vis, dv_vis,
+                                    dq_ctx, dk_ctx, dv_ctx, B, Nv, Nc, H, D, softmax_scale, dt,
+                                    stream, &tab, workspace, workspace_bytes);
 }
 
 int mmdit_adaln_modulate(const void* x, const float* shift, const float* scale, void* y, int B,

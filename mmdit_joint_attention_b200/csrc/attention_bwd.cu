@@ -103,11 +103,14 @@ __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 
 // ======================================================================
 
 // 128 / E lanes own one (sample, joint row, head) unit; E elements per 16 bytes.
+// acc (null when unused): the fused backward's fp32 dQ accumulator
+// [B, Nv + Nc, H, 128], whose unit rows are zeroed here.
 template <typename T>
 __global__ void __launch_bounds__(256)
 delta_kernel(const T* __restrict__ ov, const T* __restrict__ dov, const T* __restrict__ oc,
              const T* __restrict__ doc, const int32_t* __restrict__ ctx_len,
-             float* __restrict__ delta, int Nv, int Nc, int H, uint32_t units) {
+             float* __restrict__ delta, float* __restrict__ acc, int Nv, int Nc, int H,
+             uint32_t units) {
     constexpr int E = 16 / sizeof(T);
     constexpr int LPR = 128 / E;
     constexpr int GPW = 32 / LPR;
@@ -138,6 +141,12 @@ delta_kernel(const T* __restrict__ ov, const T* __restrict__ dov, const T* __res
             const T* dO = (vis ? dov : doc) + row * 128 + g * E;
             a[r] = live[r] ? __ldcs(reinterpret_cast<const uint4*>(o)) : make_uint4(0, 0, 0, 0);
             d[r] = live[r] ? __ldcs(reinterpret_cast<const uint4*>(dO)) : make_uint4(0, 0, 0, 0);
+            if (acc && live[r]) {
+                float4* z = reinterpret_cast<float4*>(
+                    acc + (((size_t)bb[r] * Nt + jr[r]) * H + hh[r]) * 128 + g * E);
+#pragma unroll
+                for (int e = 0; e < E / 4; ++e) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
 #pragma unroll
         for (int r = 0; r < UNR; ++r) {
@@ -539,6 +548,7 @@ struct Params {
     CUtensorMap tm_v[2];
     CUtensorMap tm_q[2];   // 64-row boxes
     CUtensorMap tm_do[2];
+    CUtensorMap tm_acc;    // fp32 dQ accumulator [B, Nv + Nc, H, 128] (dkdvq_kernel only)
     __nv_bfloat16* dk[2];
     __nv_bfloat16* dv[2];
     const float* lse;
@@ -572,6 +582,189 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 512, "barrier block must fit its shared-memory slot");
 
+// The key tile a CTA owns and the query tiles that stream past it.
+struct KeyTile {
+    int seg;      // stream of the keys
+    int krow0;    // first key
+    int kend;     // keys stored below this row
+    int qvs;      // visual query rows [qvs, qvs + qvl) see these keys
+    int qvl;
+    int L;        // valid conditioning tokens of the sample
+    int nq_vis;   // 64-row visual query tiles, then the conditioning ones
+    int nq;
+    bool idle;    // no valid key or no query
+};
+
+__device__ __forceinline__ KeyTile key_tile(const Params& p, int t, int b) {
+    KeyTile k;
+    k.qvs = 0;
+    k.qvl = p.N[0];
+    if (!p.windowed) {
+        k.seg = t < p.k_tiles_vis ? 0 : 1;
+        k.krow0 = (k.seg ? t - p.k_tiles_vis : t) * 128;
+        k.kend = p.N[k.seg];
+    } else if (t < p.cond_tiles) {
+        k.seg = 1;
+        k.krow0 = 128 * t;
+        k.kend = p.N[1];
+    } else {
+        const int tt = t - p.cond_tiles;
+        int w = 0;
+        while (w + 1 < p.win.count && p.tile_start[w + 1] <= tt) ++w;
+        const WindowGeom& g = p.win.w[w];
+        k.seg = 0;
+        k.qvs = g.start;
+        k.qvl = g.te * g.he * g.we;
+        k.krow0 = k.qvs + 128 * (tt - p.tile_start[w]);
+        k.kend = k.qvs + k.qvl;
+    }
+    k.L = p.N[1];
+    if (p.ctx_len) {
+        k.L = p.ctx_len[b];
+        k.L = k.L < 0 ? 0 : (k.L > p.N[1] ? p.N[1] : k.L);
+    }
+    k.nq_vis = (k.qvl + 63) / 64;
+    k.nq = k.nq_vis + (k.L + 63) / 64;
+    k.idle = k.nq == 0 || (k.seg == 1 && k.krow0 >= k.L);
+    return k;
+}
+
+// First row of query tile i in its stream (qs: 0 visual, 1 conditioning).
+__device__ __forceinline__ int query_row(const KeyTile& k, int i, int& qs) {
+    qs = i < k.nq_vis ? 0 : 1;
+    return qs ? (i - k.nq_vis) * 64 : k.qvs + i * 64;
+}
+
+// Zero dK and dV of a key tile that no query sees.
+__device__ __forceinline__ void zero_key_tile(const Params& p, const KeyTile& k, int h, int b) {
+    for (int r = threadIdx.x; r < 128 * 16; r += kThreads) {
+        const int key = k.krow0 + r / 16;
+        if (key < k.kend) {
+            const size_t off = ((size_t)((size_t)b * p.N[k.seg] + key) * p.H + h) * 128;
+            reinterpret_cast<uint4*>(p.dk[k.seg] + off)[r % 16] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4*>(p.dv[k.seg] + off)[r % 16] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+// TMA producer (one thread): K and V of the key tile under kv_full, then Q
+// and dO of each 64-row query tile under qd_full of its ring stage.
+template <int S>
+__device__ __forceinline__ void stream_key_tile(const Params& p, const KeyTile& k, uint8_t* smem,
+                                                int q_off, int do_off, uint64_t* kv_full,
+                                                uint64_t* qd_full, uint64_t* qd_empty, Ctl* ctl,
+                                                int h, int b) {
+    mbar_arrive_expect_tx(kv_full, 2 * kTileBytes);
+    tma_load_4d(smem, &p.tm_k[k.seg], kv_full, 0, h, k.krow0, b);
+    tma_load_4d(smem + kHalf128, &p.tm_k[k.seg], kv_full, 64, h, k.krow0, b);
+    tma_load_4d(smem + kTileBytes, &p.tm_v[k.seg], kv_full, 0, h, k.krow0, b);
+    tma_load_4d(smem + kTileBytes + kHalf128, &p.tm_v[k.seg], kv_full, 64, h, k.krow0, b);
+    int issued = 0;
+    for (int i = 0; i < k.nq; ++i) {
+        const int st = i % S;
+        int qs;
+        const int row = query_row(k, i, qs);
+        if (!wait(&qd_empty[st], ((i / S) & 1) ^ 1, ctl)) break;
+        uint8_t* dq_ = smem + q_off + st * kQ64Bytes;
+        uint8_t* ddo = smem + do_off + st * kQ64Bytes;
+        mbar_arrive_expect_tx(&qd_full[st], 2 * kQ64Bytes);
+        tma_load_4d(dq_, &p.tm_q[qs], &qd_full[st], 0, h, row, b);
+        tma_load_4d(dq_ + kHalf64, &p.tm_q[qs], &qd_full[st], 64, h, row, b);
+        tma_load_4d(ddo, &p.tm_do[qs], &qd_full[st], 0, h, row, b);
+        tma_load_4d(ddo + kHalf64, &p.tm_do[qs], &qd_full[st], 64, h, row, b);
+        ++issued;
+    }
+    if (ctl->abort) {
+        for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+            mbar_wait_bounded(&qd_full[i % S], (i / S) & 1, nullptr, kDrainLimitNs);
+        mbar_wait_bounded(kv_full, 0, nullptr, kDrainLimitNs);
+    }
+}
+
+// (lse * log2 e, D) of each query tile (one warp); rows outside the range
+// that sees these keys (past the stream, past the window, or padding) get
+// lse = +inf, so their P is 0.
+template <int S>
+__device__ __forceinline__ void load_lse_delta(const Params& p, const KeyTile& k, float2* lbuf,
+                                               uint64_t* l_full, uint64_t* l_empty, Ctl* ctl,
+                                               int lane, int h, int b) {
+    const size_t base = ((size_t)b * p.H + h) * (size_t)(p.N[0] + p.N[1]);
+    for (int i = 0; i < k.nq; ++i) {
+        const int st = i % S;
+        if (!wait_warp(&l_empty[st], ((i / S) & 1) ^ 1, ctl)) break;
+        int qs;
+        const int row0q = query_row(k, i, qs);
+        const int rlim = qs ? k.L : k.qvs + k.qvl;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int q = lane + 32 * r;
+            const int row = row0q + q;
+            const bool has = row < rlim && row < p.N[qs];
+            const size_t jr = base + (qs ? p.N[0] + row : row);
+            lbuf[st * 64 + q] =
+                has ? make_float2(p.lse[jr] * kLog2e, p.delta[jr]) : make_float2(INFINITY, 0.f);
+        }
+        mbar_arrive(&l_full[st]);
+    }
+}
+
+// P^T and dS^T = P^T (dP^T - D) of 32 queries of one key row, packed in bf16
+// pairs, from S^T and dP^T as read from tensor memory.
+__device__ __forceinline__ void p_ds(const uint32_t (&sr)[32], const uint32_t (&dr)[32],
+                                     const float2* lq, uint64_t sl2x2, uint32_t (&pp)[16],
+                                     uint32_t (&pd)[16]) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        const float2 l0 = lq[2 * c], l1 = lq[2 * c + 1];
+        const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])),
+                                  sl2x2, f2_pack(-l0.x, -l1.x));
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        const uint64_t dd = f2_sub(
+            f2_pack(__uint_as_float(dr[2 * c]), __uint_as_float(dr[2 * c + 1])), f2_pack(l0.y, l1.y));
+        float d0, d1;
+        f2_unpack(f2_mul(f2_pack(p0, p1), dd), d0, d1);
+        pp[c] = pack_bf16x2(p0, p1);
+        pd[c] = pack_bf16x2(d0, d1);
+    }
+}
+
+// dV and dK (times scale) of the key rows of this warp's tensor-memory lanes
+// and 64 head-dim columns of warpgroup wg, to bf16 (zero when !ok or for
+// padded conditioning keys).
+__device__ __forceinline__ void store_dkdv(const Params& p, const KeyTile& k, uint32_t tmem,
+                                           int quarter, int wg, int lane, bool ok, int h, int b) {
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int key = k.krow0 + quarter * 32 + lane;
+    const bool store = key < k.kend;
+    const bool zero = !ok || (k.seg == 1 && key >= k.L);
+    const size_t off =
+        ((size_t)((size_t)b * p.N[k.seg] + (store ? key : 0)) * p.H + h) * 128 + 64 * wg;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {   // 0: dV, 1: dK (times scale)
+        uint4* dst = reinterpret_cast<uint4*>((which ? p.dk[k.seg] : p.dv[k.seg]) + off);
+        const float mul = which ? p.scale : 1.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + 256 + 128 * which + 64 * wg + 32 * c + lane_off, o);
+            tmem_wait_ld();
+            if (store) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        f[e] = zero ? 0.f : __uint_as_float(o[8 * v + e]) * mul;
+                    dst[4 * c + v] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                }
+            }
+        }
+    }
+}
+
 // Tensor memory: S^T buffers [0,64) [64,128), dP^T buffers [128,192)
 // [192,256), dV [256,384), dK [384,512).  Warpgroup w handles query columns
 // [32 w, 32 w + 32) of a tile and writes its packed P^T / dS^T at columns
@@ -587,39 +780,9 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x;
     const int h = blockIdx.y;
     const int b = blockIdx.z;
-    // key tile: stream seg, first key krow0, keys stored below kend; visual
-    // query rows [qvs, qvs + qvl) that see it (all, or the keys' window)
-    int seg, krow0, kend, qvs = 0, qvl = p.N[0];
-    if (!p.windowed) {
-        seg = t < p.k_tiles_vis ? 0 : 1;
-        krow0 = (seg ? t - p.k_tiles_vis : t) * 128;
-        kend = p.N[seg];
-    } else if (t < p.cond_tiles) {
-        seg = 1;
-        krow0 = 128 * t;
-        kend = p.N[1];
-    } else {
-        const int tt = t - p.cond_tiles;
-        int w = 0;
-        while (w + 1 < p.win.count && p.tile_start[w + 1] <= tt) ++w;
-        const WindowGeom& g = p.win.w[w];
-        seg = 0;
-        qvs = g.start;
-        qvl = g.te * g.he * g.we;
-        krow0 = qvs + 128 * (tt - p.tile_start[w]);
-        kend = qvs + qvl;
-    }
-    int L = p.N[1];
-    if (p.ctx_len) {
-        L = p.ctx_len[b];
-        L = L < 0 ? 0 : (L > p.N[1] ? p.N[1] : L);
-    }
-    const int nq_vis = (qvl + 63) / 64;
-    const int nq = nq_vis + (L + 63) / 64;
-    const bool idle = nq == 0 || (seg == 1 && krow0 >= L);   // no valid key or no query
+    const KeyTile kt = key_tile(p, blockIdx.x, b);
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
@@ -639,7 +802,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
         ctl->wait_ns = p.wait_ns;
         fence_barrier_init();
     }
-    if (warp == 8 && !idle) {
+    if (warp == 8 && !kt.idle) {
         tmem_alloc(&ctl->tmem_base, 512);
         tmem_relinquish();
     }
@@ -647,15 +810,8 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     __syncthreads();
     tc_fence_after();
 
-    if (idle) {
-        for (int r = threadIdx.x; r < 128 * 16; r += kThreads) {
-            const int key = krow0 + r / 16;
-            if (key < kend) {
-                const size_t off = ((size_t)((size_t)b * p.N[seg] + key) * p.H + h) * 128;
-                reinterpret_cast<uint4*>(p.dk[seg] + off)[r % 16] = make_uint4(0, 0, 0, 0);
-                reinterpret_cast<uint4*>(p.dv[seg] + off)[r % 16] = make_uint4(0, 0, 0, 0);
-            }
-        }
+    if (kt.idle) {
+        zero_key_tile(p, kt, h, b);
         return;
     }
     const uint32_t tmem = ctl->tmem_base;
@@ -668,59 +824,10 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
     if (warp >= 8) {
         regs_dec<kRegsProducer>();
         if (warp == 8 && lane == 0) {
-            // ---------------------------------------------- TMA: K, V, then Q and dO
-            mbar_arrive_expect_tx(&bars->kv_full, 2 * kTileBytes);
-            tma_load_4d(smem + Smem::k_off, &p.tm_k[seg], &bars->kv_full, 0, h, krow0, b);
-            tma_load_4d(smem + Smem::k_off + kHalf128, &p.tm_k[seg], &bars->kv_full, 64, h, krow0,
-                        b);
-            tma_load_4d(smem + Smem::v_off, &p.tm_v[seg], &bars->kv_full, 0, h, krow0, b);
-            tma_load_4d(smem + Smem::v_off + kHalf128, &p.tm_v[seg], &bars->kv_full, 64, h, krow0,
-                        b);
-            int issued = 0;
-            for (int i = 0; i < nq; ++i) {
-                const int st = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
-                const int qs = i < nq_vis ? 0 : 1;
-                const int row = qs ? (i - nq_vis) * 64 : qvs + i * 64;
-                if (!wait(&bars->qd_empty[st], ph ^ 1, ctl)) break;
-                uint8_t* dq_ = smem + Smem::q_off + st * kQ64Bytes;
-                uint8_t* ddo = smem + Smem::do_off + st * kQ64Bytes;
-                mbar_arrive_expect_tx(&bars->qd_full[st], 2 * kQ64Bytes);
-                tma_load_4d(dq_, &p.tm_q[qs], &bars->qd_full[st], 0, h, row, b);
-                tma_load_4d(dq_ + kHalf64, &p.tm_q[qs], &bars->qd_full[st], 64, h, row, b);
-                tma_load_4d(ddo, &p.tm_do[qs], &bars->qd_full[st], 0, h, row, b);
-                tma_load_4d(ddo + kHalf64, &p.tm_do[qs], &bars->qd_full[st], 64, h, row, b);
-                ++issued;
-            }
-            if (ctl->abort) {
-                for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-                    mbar_wait_bounded(&bars->qd_full[i % kStages], (i / kStages) & 1, nullptr,
-                                      kDrainLimitNs);
-                mbar_wait_bounded(&bars->kv_full, 0, nullptr, kDrainLimitNs);
-            }
+            stream_key_tile<kStages>(p, kt, smem, Smem::q_off, Smem::do_off, &bars->kv_full,
+                                     bars->qd_full, bars->qd_empty, ctl, h, b);
         } else if (warp == 11) {
-            // ---------------------------------------------- (lse * log2 e, D) of each query tile
-            const size_t base = ((size_t)b * p.H + h) * (size_t)(p.N[0] + p.N[1]);
-            for (int i = 0; i < nq; ++i) {
-                const int st = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
-                if (!wait_warp(&bars->l_empty[st], ph ^ 1, ctl)) break;
-                const int qs = i < nq_vis ? 0 : 1;
-                const int row0q = qs ? (i - nq_vis) * 64 : qvs + i * 64;
-                // rows outside the range that sees these keys (past the
-                // stream, past the window, or padding) get lse = +inf: P = 0
-                const int rlim = qs ? L : qvs + qvl;
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int q = lane + 32 * r;
-                    const int row = row0q + q;
-                    const bool has = row < rlim && row < p.N[qs];
-                    const size_t jr = base + (qs ? p.N[0] + row : row);
-                    lbuf[st * 64 + q] =
-                        has ? make_float2(p.lse[jr] * kLog2e, p.delta[jr]) : make_float2(INFINITY, 0.f);
-                }
-                mbar_arrive(&bars->l_full[st]);
-            }
+            load_lse_delta<kStages>(p, kt, lbuf, bars->l_full, bars->l_empty, ctl, lane, h, b);
         } else if (warp == 9 && lane == 0) {
             // ---------------------------------------------- MMA issuer
             constexpr uint32_t id_n64 = idesc_bf16_f32(128, 64, 0, 0);
@@ -746,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 mma_commit(&bars->qd_empty[pst]);
                 return true;
             };
-            for (int i = 0; ok && i < nq; ++i) {
+            for (int i = 0; ok && i < kt.nq; ++i) {
                 const int st = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
                 const int buf = i & 1;
@@ -765,7 +872,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
                 mma_commit(&bars->s_full[buf]);
                 if (i > 0 && !(ok = grad_mma(i - 1))) break;
             }
-            if (ok && (ok = grad_mma(nq - 1))) mma_commit(&bars->o_done);
+            if (ok && (ok = grad_mma(kt.nq - 1))) mma_commit(&bars->o_done);
             mma_commit(&bars->drain);
             if (!mbar_wait_bounded(&bars->drain, 0, nullptr, kDrainLimitNs))
                 atomicOr(&g_bwd_status, 1u);
@@ -778,7 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint64_t sl2x2 = f2_pack(p.sl2, p.sl2);
         bool ok = true;
-        for (int i = 0; i < nq; ++i) {
+        for (int i = 0; i < kt.nq; ++i) {
             const int buf = i & 1;
             const int st = i % kStages;
             if (!(ok = wait_warp(&bars->s_full[buf], (i >> 1) & 1, ctl))) break;
@@ -790,25 +897,8 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
             tmem_ld32(tS, sr);
             tmem_ld32(tD, dr);
             tmem_wait_ld();
-            const float2* lq = lbuf + st * 64 + 32 * wg;
             uint32_t pp[16], pd[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const float2 l0 = lq[2 * c], l1 = lq[2 * c + 1];
-                const uint64_t x = f2_fma(
-                    f2_pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2,
-                    f2_pack(-l0.x, -l1.x));
-                float x0, x1;
-                f2_unpack(x, x0, x1);
-                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                const uint64_t dd =
-                    f2_sub(f2_pack(__uint_as_float(dr[2 * c]), __uint_as_float(dr[2 * c + 1])),
-                           f2_pack(l0.y, l1.y));
-                float d0, d1;
-                f2_unpack(f2_mul(f2_pack(p0, p1), dd), d0, d1);
-                pp[c] = pack_bf16x2(p0, p1);
-                pd[c] = pack_bf16x2(d0, d1);
-            }
+            p_ds(sr, dr, lbuf + st * 64 + 32 * wg, sl2x2, pp, pd);
             tmem_st16(tS, pp);
             tmem_st16(tD, pd);
             tmem_wait_st();
@@ -821,34 +911,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
         }
         if (ok) ok = wait_warp(&bars->o_done, 0, ctl);
         tc_fence_after();
-        const int key = krow0 + quarter * 32 + lane;
-        const bool store = key < kend;
-        const bool zero = !ok || (seg == 1 && key >= L);
-        const size_t off =
-            ((size_t)((size_t)b * p.N[seg] + (store ? key : 0)) * p.H + h) * 128 + 64 * wg;
-#pragma unroll
-        for (int which = 0; which < 2; ++which) {   // 0: dV, 1: dK (times scale)
-            uint4* dst = reinterpret_cast<uint4*>((which ? p.dk[seg] : p.dv[seg]) + off);
-            const float mul = which ? p.scale : 1.f;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tmem + 256 + 128 * which + 64 * wg + 32 * c + lane_off, o);
-                tmem_wait_ld();
-                if (store) {
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        float f[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            f[e] = zero ? 0.f : __uint_as_float(o[8 * v + e]) * mul;
-                        dst[4 * c + v] =
-                            make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                       pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-                    }
-                }
-            }
-        }
+        store_dkdv(p, kt, tmem, quarter, wg, lane, ok, h, b);
     }
 
     tc_fence_before();
@@ -858,6 +921,286 @@ __global__ void __launch_bounds__(kThreads, 1) dkdv_kernel(const __grid_constant
         tmem_dealloc(tmem, 512);
     }
 }
+
+// ----------------------------------------------------------------------
+// 3b. dK, dV and dQ in one key-stationary pass
+// ----------------------------------------------------------------------
+// dkdv_kernel's pipeline extended with dQ.  The softmax warps write dS^T to
+// shared memory (P^T still goes to tensor memory), where it is the A operand
+// of dK += dS^T Q and the B operand of this tile's dQ^T = K^T dS^T (head dim
+// x 64 queries; K^T is the stationary K tile read as an MN-major operand).
+// Each softmax warp then reads its 32 x 32 block of dQ^T and adds it into an
+// fp32 accumulator [B, Nv + Nc, H, 128] in global memory with one bulk tensor
+// reduce-add; dq_convert_kernel scales the sums into bf16 dQ.  S and dP are
+// formed once, so the backward executes 10 N^2 D FLOPs per (sample, head)
+// instead of the 14 of dq_kernel + dkdv_kernel.  The costs: the accumulator
+// (zeroed by delta_kernel; a head's rows are reduced into by all its key tiles
+// at about the same time, so they stay in L2), dP^T single-buffered (it is
+// only read, so the next tile's dP^T waits for the loads, not the softmax),
+// and an order of the dQ sums that changes from run to run.
+namespace fused {
+
+constexpr int kQdStages = 3;                // Q / dO / (lse, D) ring depth
+constexpr int kBlockBytes = 32 * 32 * 4;    // one warp's 32 x 32 fp32 block of dQ^T
+
+struct Smem {
+    static constexpr int k_off = 0;
+    static constexpr int v_off = kTileBytes;
+    static constexpr int q_off = 2 * kTileBytes;
+    static constexpr int do_off = q_off + kQdStages * kQ64Bytes;
+    static constexpr int ds_off = do_off + kQdStages * kQ64Bytes;   // dS^T: 128 keys x 64 queries
+    static constexpr int dq_off = ds_off + kQ64Bytes;               // 8 softmax warps' blocks
+    static constexpr int l_off = dq_off + 8 * kBlockBytes;
+    static constexpr int bar_off = l_off + kQdStages * 512;
+    static constexpr int total = bar_off + 512;
+};
+
+struct Bars {
+    uint64_t kv_full;
+    uint64_t qd_full[kQdStages], qd_empty[kQdStages];
+    uint64_t l_full[kQdStages], l_empty[kQdStages];
+    uint64_t s_full[2];   // S^T (buffer i % 2) and dP^T of query tile i are in tensor memory
+    uint64_t dp_free;     // every softmax warp has read dP^T
+    uint64_t p_full[2];   // P^T in tensor memory, dS^T in shared memory
+    uint64_t dq_full;     // dQ^T formed; dS^T's shared memory free again
+    uint64_t dq_empty;    // every softmax warp has read dQ^T
+    uint64_t o_done;
+    uint64_t drain;
+    Ctl ctl;
+};
+static_assert(sizeof(Bars) <= 512, "barrier block must fit its shared-memory slot");
+
+// Tensor memory: S^T buffers [0,64) [64,128) (P^T packed over them as in
+// dkdv_kernel), dP^T [128,192), dQ^T [192,256), dV [256,384), dK [384,512).
+constexpr uint32_t kColDP = 128;
+constexpr uint32_t kColDQ = 192;
+
+__global__ void __launch_bounds__(kThreads, 1) dkdvq_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + Smem::bar_off);
+    Ctl* ctl = &bars->ctl;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const KeyTile kt = key_tile(p, blockIdx.x, b);
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->kv_full, 1);
+        for (int i = 0; i < kQdStages; ++i) {
+            mbar_init(&bars->qd_full[i], 1);
+            mbar_init(&bars->qd_empty[i], 1);
+            mbar_init(&bars->l_full[i], 32);   // every lane of the loader warp
+            mbar_init(&bars->l_empty[i], 8);   // one elected lane per softmax warp
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->p_full[i], 8);
+        }
+        mbar_init(&bars->dp_free, 8);
+        mbar_init(&bars->dq_full, 1);
+        mbar_init(&bars->dq_empty, 8);
+        mbar_init(&bars->o_done, 1);
+        mbar_init(&bars->drain, 1);
+        ctl->abort = 0;
+        ctl->wait_ns = p.wait_ns;
+        fence_barrier_init();
+    }
+    if (warp == 8 && !kt.idle) {
+        tmem_alloc(&ctl->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (kt.idle) {   // no query sees these keys: they add nothing to dQ
+        zero_key_tile(p, kt, h, b);
+        return;
+    }
+    const uint32_t tmem = ctl->tmem_base;
+    const uint32_t sK = smem_u32(smem + Smem::k_off);
+    const uint32_t sV = smem_u32(smem + Smem::v_off);
+    const uint32_t sQ = smem_u32(smem + Smem::q_off);
+    const uint32_t sDO = smem_u32(smem + Smem::do_off);
+    const uint32_t sDS = smem_u32(smem + Smem::ds_off);
+    float2* lbuf = reinterpret_cast<float2*>(smem + Smem::l_off);   // (lse * log2 e, D)
+
+    if (warp >= 8) {
+        regs_dec<kRegsProducer>();
+        if (warp == 8 && lane == 0) {
+            stream_key_tile<kQdStages>(p, kt, smem, Smem::q_off, Smem::do_off, &bars->kv_full,
+                                       bars->qd_full, bars->qd_empty, ctl, h, b);
+        } else if (warp == 11) {
+            load_lse_delta<kQdStages>(p, kt, lbuf, bars->l_full, bars->l_empty, ctl, lane, h, b);
+        } else if (warp == 9 && lane == 0) {
+            // ---------------------------------------------- MMA issuer
+            constexpr uint32_t id_n64 = idesc_bf16_f32(128, 64, 0, 0);   // S^T, dP^T
+            constexpr uint32_t id_mn = idesc_bf16_f32(128, 128, 0, 1);   // dV, dK
+            constexpr uint32_t id_dq = idesc_bf16_f32(128, 64, 1, 1);    // dQ^T
+            bool ok = wait(&bars->kv_full, 0, ctl);
+            const uint64_t kd = kdesc(sK), vd = kdesc(sV);
+            const uint64_t dsa = kdesc(sDS);   // dS^T as A: M = keys, K = queries
+            // dV += P^T dO, dK += dS^T Q, then dQ^T = K^T dS^T of query tile ii
+            auto grad_mma = [&](int ii) -> bool {
+                const int pb = ii & 1;
+                const int pst = ii % kQdStages;
+                if (!wait(&bars->p_full[pb], (ii >> 1) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint64_t dom = mndesc(sDO + pst * kQ64Bytes, kHalf64);
+                const uint64_t qm = mndesc(sQ + pst * kQ64Bytes, kHalf64);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ts(tmem + 256, tmem + 64 * pb + packed_col(s), dom + (uint64_t)s * kMnStep,
+                           id_mn, (ii > 0 || s > 0) ? 1u : 0u);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ss(tmem + 384, dsa + koff(s, 0), qm + (uint64_t)s * kMnStep, id_mn,
+                           (ii > 0 || s > 0) ? 1u : 0u);
+                mma_commit(&bars->qd_empty[pst]);
+                if (ii > 0) {   // the softmax warps have read dQ^T of tile ii - 1
+                    if (!wait(&bars->dq_empty, (ii - 1) & 1, ctl)) return false;
+                    tc_fence_after();
+                }
+                // A = K^T (M = head dim over K's two boxes), B = dS^T (N = 64
+                // queries, one swizzle atom); k-step s = keys [16 s, 16 s + 16)
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_ss(tmem + kColDQ, mndesc(sK + 2048 * s, kHalf128),
+                           mndesc(sDS + 2048 * s, kQ64Bytes), id_dq, s > 0 ? 1u : 0u);
+                mma_commit(&bars->dq_full);
+                return true;
+            };
+            for (int i = 0; ok && i < kt.nq; ++i) {
+                const int st = i % kQdStages;
+                const int buf = i & 1;
+                if (!(ok = wait(&bars->qd_full[st], (i / kQdStages) & 1, ctl))) break;
+                tc_fence_after();
+                const uint64_t qd = kdesc(sQ + st * kQ64Bytes);
+                const uint64_t dod = kdesc(sDO + st * kQ64Bytes);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_ss(tmem + 64 * buf, kd + koff(s, kHalf128), qd + koff(s, kHalf64), id_n64,
+                           s > 0 ? 1u : 0u);
+                if (i > 0) {   // the softmax warps have read dP^T of tile i - 1
+                    if (!(ok = wait(&bars->dp_free, (i - 1) & 1, ctl))) break;
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_ss(tmem + kColDP, vd + koff(s, kHalf128), dod + koff(s, kHalf64), id_n64,
+                           s > 0 ? 1u : 0u);
+                mma_commit(&bars->s_full[buf]);
+                if (i > 0 && !(ok = grad_mma(i - 1))) break;
+            }
+            if (ok && (ok = grad_mma(kt.nq - 1))) mma_commit(&bars->o_done);
+            mma_commit(&bars->drain);
+            if (!mbar_wait_bounded(&bars->drain, 0, nullptr, kDrainLimitNs))
+                atomicOr(&g_bwd_status, 1u);
+        }
+    } else {
+        regs_inc<kRegsSoftmax>();
+        // -------------------------------------------------- P^T, dS^T, and the dQ reduction
+        const int wg = warp >> 2;        // query columns [32 wg, 32 wg + 32) of every tile
+        const int quarter = warp & 3;    // tensor-memory lanes (keys; head dim for dQ^T)
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint64_t sl2x2 = f2_pack(p.sl2, p.sl2);
+        // this thread's key row of dS^T: 128 bytes (64 queries), 16-byte chunk
+        // c stored at c ^ (row % 8) (the 128-byte swizzle of the operands)
+        const int krow = quarter * 32 + lane;
+        uint8_t* ds_row = smem + Smem::ds_off + (krow >> 3) * 1024 + (krow & 7) * 128;
+        // keys past the tile's end (the next window's, or padding) and padded
+        // conditioning keys are real rows of K: their dS^T must not reach dQ
+        const int key = kt.krow0 + krow;
+        const bool key_ok = key < kt.kend && !(kt.seg == 1 && key >= kt.L);
+        float* blk = reinterpret_cast<float*>(smem + Smem::dq_off + warp * kBlockBytes);
+        // Reduces this warp's block of dQ^T of query tile j (head dim
+        // [32 quarter, +32) x queries [32 wg, +32)) into the accumulator, as
+        // 32 query rows x 32 head-dim floats.
+        auto reduce_dq = [&](int j) {
+            uint32_t r[32];
+            tmem_ld32(tmem + kColDQ + 32 * wg + lane_off, r);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars->dq_empty);
+                bulk_wait_group_read<0>();   // the previous block has left shared memory
+            }
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) blk[q * 32 + lane] = __uint_as_float(r[q]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                int qs;
+                const int row = query_row(kt, j, qs);
+                tma_reduce_add_4d(&p.tm_acc, blk, 32 * quarter, h,
+                                  (qs ? p.N[0] : 0) + row + 32 * wg, b);
+                bulk_commit_group();
+            }
+        };
+        bool ok = true;
+        for (int i = 0; i < kt.nq; ++i) {
+            const int buf = i & 1;
+            const int st = i % kQdStages;
+            if (!(ok = wait_warp(&bars->s_full[buf], (i >> 1) & 1, ctl))) break;
+            if (!(ok = wait_warp(&bars->l_full[st], (i / kQdStages) & 1, ctl))) break;
+            tc_fence_after();
+            uint32_t sr[32], dr[32];
+            const uint32_t tS = tmem + 64 * buf + 32 * wg + lane_off;
+            tmem_ld32(tS, sr);
+            tmem_ld32(tmem + kColDP + 32 * wg + lane_off, dr);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->dp_free);
+            uint32_t pp[16], pd[16];
+            p_ds(sr, dr, lbuf + st * 64 + 32 * wg, sl2x2, pp, pd);
+            if (!key_ok) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) pd[c] = 0u;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->l_empty[st]);
+            if (i > 0) {   // dQ^T of tile i - 1 formed: dS^T's buffer is free
+                if (!(ok = wait_warp(&bars->dq_full, (i - 1) & 1, ctl))) break;
+                tc_fence_after();
+            }
+            tmem_st16(tS, pp);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4*>(ds_row + 16 * ((4 * wg + c) ^ (krow & 7))) =
+                    make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
+            fence_proxy_async_smem();
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->p_full[buf]);
+            if (i > 0) reduce_dq(i - 1);
+        }
+        if (ok && (ok = wait_warp(&bars->dq_full, (kt.nq - 1) & 1, ctl))) {
+            tc_fence_after();
+            reduce_dq(kt.nq - 1);
+        }
+        if (ok) ok = wait_warp(&bars->o_done, 0, ctl);
+        tc_fence_after();
+        store_dkdv(p, kt, tmem, quarter, wg, lane, ok, h, b);
+        if (lane == 0) bulk_wait_group<0>();   // reduce-adds complete before the CTA ends
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace fused
 
 }  // namespace dkv
 
@@ -1005,7 +1348,7 @@ dkdv_f32_kernel(const float* __restrict__ qv, const float* __restrict__ kv,
 template <typename T>
 cudaError_t run_delta(const void* ov, const void* dov, const void* oc, const void* doc,
                       const int32_t* ctx_len, float* delta, int B, int Nv, int Nc, int H,
-                      cudaStream_t s) {
+                      cudaStream_t s, float* acc = nullptr) {
     const long long units = (long long)B * (Nv + Nc) * H;
     if (units == 0) return cudaSuccess;
     int dev = 0, sms = 148;
@@ -1016,8 +1359,34 @@ cudaError_t run_delta(const void* ov, const void* dov, const void* oc, const voi
     if (blocks > 8LL * sms) blocks = 8LL * sms;
     delta_kernel<T><<<(unsigned)blocks, 256, 0, s>>>(
         static_cast<const T*>(ov), static_cast<const T*>(dov), static_cast<const T*>(oc),
-        static_cast<const T*>(doc), ctx_len, delta, Nv, Nc, H, (uint32_t)units);
+        static_cast<const T*>(doc), ctx_len, delta, acc, Nv, Nc, H, (uint32_t)units);
     return cudaGetLastError();
+}
+
+// dQ = softmax_scale * accumulator: fp32 [B, Nv + Nc, H, 128] -> bf16 dq_vis
+// [B, Nv, H, 128] and dq_ctx [B, Nc, H, 128].  16 lanes per (sample, joint
+// row, head) row, 8 elements each.
+__global__ void __launch_bounds__(256)
+dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dqv,
+                  __nv_bfloat16* __restrict__ dqc, int Nv, int Nc, int H, float scale,
+                  uint32_t rows) {
+    const uint32_t Nt = (uint32_t)(Nv + Nc);
+    const int e = (threadIdx.x & 15) * 8;
+    const uint32_t step = gridDim.x * (blockDim.x / 16);
+    for (uint32_t r = blockIdx.x * (blockDim.x / 16) + threadIdx.x / 16; r < rows; r += step) {
+        const uint32_t hh = r % (uint32_t)H;
+        const uint32_t bj = r / (uint32_t)H;
+        const uint32_t jr = bj % Nt;
+        const uint32_t bb = bj / Nt;
+        const float4* src = reinterpret_cast<const float4*>(acc + (size_t)r * 128 + e);
+        const float4 x = __ldcs(src), y = __ldcs(src + 1);
+        __nv_bfloat16* dst =
+            (int)jr < Nv ? dqv + (((size_t)bb * Nv + jr) * H + hh) * 128 + e
+                         : dqc + (((size_t)bb * Nc + (jr - Nv)) * H + hh) * 128 + e;
+        *reinterpret_cast<uint4*>(dst) =
+            make_uint4(pack_bf16x2(x.x * scale, x.y * scale), pack_bf16x2(x.z * scale, x.w * scale),
+                       pack_bf16x2(y.x * scale, y.y * scale), pack_bf16x2(y.z * scale, y.w * scale));
+    }
 }
 
 // Refuses to launch unless the compiled kernel uses exactly kRegsLaunch
@@ -1048,11 +1417,13 @@ int launch_joint_attention_bwd_bf16(const void* qv, const void* kv, const void* 
                                     const void* dov, const void* doc, const float* lse,
                                     float* delta, void* dqv, void* dkv, void* dvv, void* dqc,
                                     void* dkc, void* dvc, int B, int Nv, int Nc, int H,
-                                    float softmax_scale, cudaStream_t s, const WindowTable* win) {
+                                    float softmax_scale, cudaStream_t s, const WindowTable* win,
+                                    float* dq_acc) {
     using namespace bwd;
     if (!encode_fn()) return -1;
     if (B == 0 || Nv + Nc == 0) return 0;
-    cudaError_t e = run_delta<__nv_bfloat16>(ov, dov, oc, doc, ctx_len, delta, B, Nv, Nc, H, s);
+    cudaError_t e =
+        run_delta<__nv_bfloat16>(ov, dov, oc, doc, ctx_len, delta, B, Nv, Nc, H, s, dq_acc);
     if (e != cudaSuccess) return (int)e;
 
     dq::Params pq;
@@ -1091,11 +1462,18 @@ int launch_joint_attention_bwd_bf16(const void* qv, const void* kv, const void* 
     pq.scale = pk.scale = softmax_scale;
     pq.wait_ns = pk.wait_ns = wait_timeout_ns();
 
-    static bool dq_ready[64] = {false}, dkv_ready[64] = {false};
+    static bool dq_ready[64] = {false}, dkv_ready[64] = {false}, fused_ready[64] = {false};
     const int smem_q = dq::Smem::total + 1024;
     const int smem_k = dkv::Smem::total + 1024;
-    if ((e = prepare(dq::dq_kernel, smem_q, dq_ready)) != cudaSuccess) return (int)e;
-    if ((e = prepare(dkv::dkdv_kernel, smem_k, dkv_ready)) != cudaSuccess) return (int)e;
+    const int smem_f = dkv::fused::Smem::total + 1024;
+    if (dq_acc) {
+        if (!encode_acc_f32(&pk.tm_acc, dq_acc, B, Nv + Nc, H)) return 1000 + (int)cudaErrorInvalidValue;
+        if ((e = prepare(dkv::fused::dkdvq_kernel, smem_f, fused_ready)) != cudaSuccess)
+            return (int)e;
+    } else {
+        if ((e = prepare(dq::dq_kernel, smem_q, dq_ready)) != cudaSuccess) return (int)e;
+        if ((e = prepare(dkv::dkdv_kernel, smem_k, dkv_ready)) != cudaSuccess) return (int)e;
+    }
     dim3 grid((Nv + 127) / 128 + (Nc + 127) / 128, H, B);
     if (win) {
         // window mode: the conditioning tiles first, then each window's tiles
@@ -1110,6 +1488,20 @@ int launch_joint_attention_bwd_bf16(const void* qv, const void* kv, const void* 
         }
         pq.tile_start[win->count] = pk.tile_start[win->count] = tiles;
         grid.x = (unsigned)(pq.cond_tiles + tiles);
+    }
+    if (dq_acc) {
+        dkv::fused::dkdvq_kernel<<<grid, kThreads, smem_f, s>>>(pk);
+        if ((e = cudaGetLastError()) != cudaSuccess) return (int)e;
+        const long long rows = (long long)B * (Nv + Nc) * H;
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        long long blocks = (rows + 15) / 16;
+        if (blocks > 8LL * sms) blocks = 8LL * sms;
+        dq_convert_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+            dq_acc, static_cast<__nv_bfloat16*>(dqv), static_cast<__nv_bfloat16*>(dqc), Nv, Nc, H,
+            softmax_scale, (uint32_t)rows);
+        return (int)cudaGetLastError();
     }
     dq::dq_kernel<<<grid, kThreads, smem_q, s>>>(pq);
     if ((e = cudaGetLastError()) != cudaSuccess) return (int)e;

@@ -120,8 +120,10 @@ cudaError_t launch_joint_attention_f32(const float* qv, const float* kv, const f
 // (row sums of dO * O, written here); lse from the forward.  win (null: full
 // joint attention): 3D window attention, with every visual tensor
 // (q, k, v, o, dO, the d* outputs, and the visual rows of lse and delta) in
-// the table's window-major order.  Return convention of
-// launch_joint_attention_bf16.
+// the table's window-major order.  dq_acc (null: the two-kernel form, dQ and
+// dK/dV apart): caller workspace [B, Nv + Nc, H, 128] fp32 for the one-pass
+// form, which reduces dQ into it (contents on entry ignored).  Return
+// convention of launch_joint_attention_bf16.
 int launch_joint_attention_bwd_bf16(const void* qv, const void* kv, const void* vv,
                                     const void* qc, const void* kc, const void* vc,
                                     const int32_t* ctx_len, const void* ov, const void* oc,
@@ -129,7 +131,7 @@ int launch_joint_attention_bwd_bf16(const void* qv, const void* kv, const void* 
                                     float* delta, void* dqv, void* dkv, void* dvv, void* dqc,
                                     void* dkc, void* dvc, int B, int Nv, int Nc, int H,
                                     float softmax_scale, cudaStream_t s,
-                                    const WindowTable* win = nullptr);
+                                    const WindowTable* win = nullptr, float* dq_acc = nullptr);
 cudaError_t launch_joint_attention_bwd_f32(const float* qv, const float* kv, const float* vv,
                                            const float* qc, const float* kc, const float* vc,
                                            const int32_t* ctx_len, const float* ov,

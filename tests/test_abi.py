@@ -324,6 +324,38 @@ def test_attention_qnorm_ws_validation(L):
     assert f(*a) == 0
 
 
+def test_backward_ws_validation(L):
+    f = L.mmdit_joint_attention_bwd_ws
+    Q = ctypes.c_void_p(1 << 20)
+    # q..v, ctx_len, o, do, lse, delta, workspace, bytes, the six gradients
+    args = lambda ws, n: ([P] * 6 + [None] + [P] * 4 + [Q, Q, ws, n] + [P] * 6 +
+                          [1, 8, 8, 2, 128, 0.1, 1, None])
+    assert f(*args(ctypes.c_void_p(272), 1 << 20)) == -3          # workspace not 256-aligned
+    assert f(*args(ctypes.c_void_p(256), -1)) == -1
+    a = args(None, 0); a[11] = None                                 # lse missing
+    assert f(*a) == -1
+    a = args(None, 0); a[25] = 64                                   # D != 128
+    assert f(*a) == -4
+    a = args(None, 0); a[21] = 0                                    # B = 0: nothing to do
+    assert f(*a) == 0
+    w = L.mmdit_joint_window_attention_bwd_ws
+    g, win = _lib.Grid(), _lib.Window()
+    g.T, g.H, g.W = 1, 2, 4                                          # Nv = 8
+    win.parts[0], win.parts[1], win.parts[2] = 1, 1, 2
+    wargs = args(ctypes.c_void_p(272), 1 << 20)
+    wargs = wargs[:26] + [ctypes.byref(g), ctypes.byref(win)] + wargs[26:]
+    assert w(*wargs) == -3                                          # workspace not 256-aligned
+    wargs[26] = None
+    assert w(*wargs) == -1                                          # no grid
+
+
+def test_bwd_workspace_bytes_rule():
+    """The one-pass backward's accumulator: fp32 [B, Nv + Nc, H, 128]."""
+    from mmdit_joint_attention_b200 import api
+    assert api.bwd_workspace_bytes(1, 32760, 512, 24) == 1 * 33272 * 24 * 128 * 4
+    assert api.bwd_workspace_bytes(2, 0, 5, 3) == 2 * 5 * 3 * 512
+
+
 def _plan_rule(B, Nv, Nc, H, nsm, ws):
     """The split-tail rule restated: the items past the last whole wave
     (total mod nsm) are split into as many pieces as fill the SMs, at least 2

@@ -5,7 +5,9 @@ inputs and upstream gradients.
 Small and medium cases compare every gradient element; the full 480p and
 ragged workloads compare dq and lse on sampled query rows (each against the
 full key set), dk and dv on sampled key rows of a few heads (each against every
-query row), and dk / dv of every key through sum rules that hold at any size."""
+query row), and dk / dv of every key through sum rules that hold at any size.
+Each case runs both forms of the bf16 backward: the two-kernel form (dQ, then
+dK / dV) and the one-pass form (dQ reduced into an fp32 workspace)."""
 import numpy as np
 import pytest
 import torch
@@ -25,7 +27,7 @@ def _ws(w: I.Workload, **kw) -> I.Workload:
     return dataclasses.replace(w, **kw)
 
 
-def _run(w: I.Workload, seed=0):
+def _run(w: I.Workload, seed=0, one_pass=False):
     inp = I.make_inputs(w, seed=seed, parts=("qkv",))
     gin = I.make_grad_outputs(w, seed=seed)
     t = device_inputs(inp)
@@ -33,8 +35,11 @@ def _run(w: I.Workload, seed=0):
     cl = t["ctx_len"] if w.ctx_len is not None else None
     ov, oc, lse = api.joint_attention_fwd(t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"],
                                           t["k_ctx"], t["v_ctx"], cl)
+    ws = api.bwd_workspace(w.B, w.Nv, w.Nc, w.H) if one_pass else None
+    if ws is not None:
+        ws.fill_(0xFF)   # NaN bit patterns: the backward must not read stale contents
     g = api.joint_attention_bwd(t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"],
-                                t["v_ctx"], ov, oc, do_vis, do_ctx, lse, cl)
+                                t["v_ctx"], ov, oc, do_vis, do_ctx, lse, cl, workspace=ws)
     torch.cuda.synchronize()
     assert api.device_status() == 0
     return inp, gin, {k: from_dev(v) for k, v in g.items()}, from_dev(lse), (ov, oc)
@@ -60,10 +65,11 @@ SMALL = {
 }
 
 
+@pytest.mark.parametrize("one_pass", [False, True])
 @pytest.mark.parametrize("case", sorted(SMALL))
-def test_backward_full(case):
+def test_backward_full(case, one_pass):
     w = SMALL[case]
-    inp, gin, g, lse, _ = _run(w)
+    inp, gin, g, lse, _ = _run(w, one_pass=one_pass)
     ref = oracle.joint_attention_bwd(inp["q_vis"].f64, inp["k_vis"].f64, inp["v_vis"].f64,
                                      inp["q_ctx"].f64, inp["k_ctx"].f64, inp["v_ctx"].f64,
                                      gin["do_vis"].f64, gin["do_ctx"].f64, inp["ctx_len"])
@@ -75,10 +81,11 @@ def test_backward_full(case):
             assert np.all(g[k][b, L:] == 0.0), f"{case} {k}: padded rows must be zero"
 
 
+@pytest.mark.parametrize("one_pass", [False, True])
 @pytest.mark.parametrize("name", ["480p", "ragged"])
-def test_backward_sampled_full_size(name):
+def test_backward_sampled_full_size(name, one_pass):
     w = W[name]
-    inp, gin, g, lse, _ = _run(w)
+    inp, gin, g, lse, _ = _run(w, one_pass=one_pass)
     trip = []
     for b in range(w.B):
         for h in range(w.H):
@@ -132,6 +139,41 @@ def test_backward_sampled_full_size(name):
         assert np.all(np.abs(dv.sum(0) - do_sum) <= 3e-2 * rss_v + 1e-6), "sum of dv"
         assert np.all(np.abs(dk.sum(0)) <= 3e-2 * rss_k + 1e-6), "sum of dk"
         assert np.all(g["dk_ctx"][b, L:] == 0) and np.all(g["dv_ctx"][b, L:] == 0)
+
+
+@pytest.mark.parametrize("case", ["ragged_small", "batch3_mixed", "medium_2k"])
+def test_one_pass_dk_dv_equal_two_kernel_form(case):
+    """Both forms form the same bf16 P^T and dS^T and the same dV and dK
+    products in the same order (dS^T read from shared memory instead of tensor
+    memory), so dK and dV agree bit for bit; dQ is summed in another order and
+    agrees within the bf16 rounding of the two results."""
+    w = SMALL[case]
+    _, _, g2, _, _ = _run(w, one_pass=False)
+    _, _, g1, _, _ = _run(w, one_pass=True)
+    for k in ("dk_vis", "dv_vis", "dk_ctx", "dv_ctx"):
+        assert np.array_equal(g1[k], g2[k]), f"{case} {k} differs between the forms"
+    for k in ("dq_vis", "dq_ctx"):
+        a, b = g1[k].astype(np.float64), g2[k].astype(np.float64)
+        scale = np.sqrt(np.mean(b ** 2)) + 1e-30
+        assert np.max(np.abs(a - b)) <= 2 ** -6 * scale + 1e-30, f"{case} {k}"
+
+
+def test_one_pass_workspace_too_small_runs_two_kernel_form():
+    w = SMALL["ragged_small"]
+    inp = I.make_inputs(w, seed=0, parts=("qkv",))
+    gin = I.make_grad_outputs(w, seed=0)
+    t = device_inputs(inp)
+    do_vis, do_ctx = to_dev(gin["do_vis"]), to_dev(gin["do_ctx"])
+    args = (t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"], t["v_ctx"])
+    ov, oc, lse = api.joint_attention_fwd(*args, t["ctx_len"])
+    small = torch.empty(api.bwd_workspace_bytes(w.B, w.Nv, w.Nc, w.H) - 256, dtype=torch.uint8,
+                        device="cuda")
+    g_small = api.joint_attention_bwd(*args, ov, oc, do_vis, do_ctx, lse, t["ctx_len"],
+                                      workspace=small)
+    g_two = api.joint_attention_bwd(*args, ov, oc, do_vis, do_ctx, lse, t["ctx_len"])
+    torch.cuda.synchronize()
+    for k in g_two:   # the two-kernel form is deterministic
+        assert torch.equal(g_small[k], g_two[k]), k
 
 
 def test_forward_with_lse_matches_forward():

@@ -205,9 +205,10 @@ def test_window_api_rejects_bad_arguments():
 
 # ------------------------------------------------------------- window backward
 
-def _window_bwd_run(w: I.Workload, parts, seed=0):
-    """Window forward with lse, then the window backward; gradients returned
-    to raster order, lse as written (window-major visual rows)."""
+def _window_bwd_run(w: I.Workload, parts, seed=0, one_pass=False):
+    """Window forward with lse, then the window backward (two-kernel or
+    one-pass form); gradients returned to raster order, lse as written
+    (window-major visual rows)."""
     inp = I.make_inputs(w, seed=seed, parts=("qkv",))
     gin = I.make_grad_outputs(w, seed=seed)
     t = device_inputs(inp)
@@ -215,9 +216,12 @@ def _window_bwd_run(w: I.Workload, parts, seed=0):
     q, k, v = (api.window_permute(t[n], w.grid, parts) for n in ("q_vis", "k_vis", "v_vis"))
     ov, oc, lse = api.joint_window_attention_fwd(q, k, v, t["q_ctx"], t["k_ctx"], t["v_ctx"],
                                                  w.grid, parts, cl)
+    ws = api.bwd_workspace(w.B, w.Nv, w.Nc, w.H) if one_pass else None
+    if ws is not None:
+        ws.fill_(0xFF)
     g = api.joint_window_attention_bwd(q, k, v, t["q_ctx"], t["k_ctx"], t["v_ctx"], ov, oc,
                                        to_dev(gin["do_vis"]), to_dev(gin["do_ctx"]), lse, w.grid,
-                                       parts, cl)
+                                       parts, cl, workspace=ws)
     for n in ("dq_vis", "dk_vis", "dv_vis"):
         g[n] = api.window_permute(g[n], w.grid, parts, inverse=True)
     torch.cuda.synchronize()
@@ -237,10 +241,11 @@ BWD = {
 }
 
 
+@pytest.mark.parametrize("one_pass", [False, True])
 @pytest.mark.parametrize("case", sorted(BWD))
-def test_window_backward_full(case):
+def test_window_backward_full(case, one_pass):
     w, parts = BWD[case]
-    inp, gin, g, lse = _window_bwd_run(w, parts)
+    inp, gin, g, lse = _window_bwd_run(w, parts, one_pass=one_pass)
     ref = oracle.window_attention_bwd(inp["q_vis"].f64, inp["k_vis"].f64, inp["v_vis"].f64,
                                       inp["q_ctx"].f64, inp["k_ctx"].f64, inp["v_ctx"].f64,
                                       gin["do_vis"].f64, gin["do_ctx"].f64, w.grid, parts,
