@@ -961,9 +961,11 @@ struct Bars {
     uint64_t l_full[kQdStages], l_empty[kQdStages];
     uint64_t s_full[2];   // S^T (buffer i % 2) and dP^T of query tile i are in tensor memory
     uint64_t dp_free;     // every softmax warp has read dP^T
-    uint64_t p_full[2];   // P^T in tensor memory, dS^T in shared memory
+    // p_full[i % 2]: every softmax warp has written P^T(i) to tensor memory and
+    // dS^T(i) to shared memory, and has read dQ^T(i - 1) (so the MMA issuer
+    // needs no other wait before overwriting dQ^T)
+    uint64_t p_full[2];
     uint64_t dq_full;     // dQ^T formed; dS^T's shared memory free again
-    uint64_t dq_empty;    // every softmax warp has read dQ^T
     uint64_t o_done;
     uint64_t drain;
     Ctl ctl;
@@ -1002,7 +1004,6 @@ __global__ void __launch_bounds__(kThreads, 1) dkdvq_kernel(const __grid_constan
         }
         mbar_init(&bars->dp_free, 8);
         mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_empty, 8);
         mbar_init(&bars->o_done, 1);
         mbar_init(&bars->drain, 1);
         ctl->abort = 0;
@@ -1045,10 +1046,10 @@ __global__ void __launch_bounds__(kThreads, 1) dkdvq_kernel(const __grid_constan
             const uint64_t kd = kdesc(sK), vd = kdesc(sV);
             const uint64_t dsa = kdesc(sDS);   // dS^T as A: M = keys, K = queries
             // dV += P^T dO, dK += dS^T Q, then dQ^T = K^T dS^T of query tile ii
-            auto grad_mma = [&](int ii) -> bool {
+            // (issued once p_full of tile ii has been seen)
+            auto grad_mma = [&](int ii) {
                 const int pb = ii & 1;
                 const int pst = ii % kQdStages;
-                if (!wait(&bars->p_full[pb], (ii >> 1) & 1, ctl)) return false;
                 tc_fence_after();
                 const uint64_t dom = mndesc(sDO + pst * kQ64Bytes, kHalf64);
                 const uint64_t qm = mndesc(sQ + pst * kQ64Bytes, kHalf64);
@@ -1061,10 +1062,6 @@ __global__ void __launch_bounds__(kThreads, 1) dkdvq_kernel(const __grid_constan
                     mma_ss(tmem + 384, dsa + koff(s, 0), qm + (uint64_t)s * kMnStep, id_mn,
                            (ii > 0 || s > 0) ? 1u : 0u);
                 mma_commit(&bars->qd_empty[pst]);
-                if (ii > 0) {   // the softmax warps have read dQ^T of tile ii - 1
-                    if (!wait(&bars->dq_empty, (ii - 1) & 1, ctl)) return false;
-                    tc_fence_after();
-                }
                 // A = K^T (M = head dim over K's two boxes), B = dS^T (N = 64
                 // queries, one swizzle atom); k-step s = keys [16 s, 16 s + 16)
 #pragma unroll
@@ -1072,8 +1069,10 @@ __global__ void __launch_bounds__(kThreads, 1) dkdvq_kernel(const __grid_constan
                     mma_ss(tmem + kColDQ, mndesc(sK + 2048 * s, kHalf128),
                            mndesc(sDS + 2048 * s, kQ64Bytes), id_dq, s > 0 ? 1u : 0u);
                 mma_commit(&bars->dq_full);
-                return true;
             };
+            // iteration i: S^T(i); once the softmax has read dP^T(i - 1),
+            // dP^T(i); once it is done with tile i - 1, the gradient products
+            // of tile i - 1
             for (int i = 0; ok && i < kt.nq; ++i) {
                 const int st = i % kQdStages;
                 const int buf = i & 1;
@@ -1085,7 +1084,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdvq_kernel(const __grid_constan
                 for (int s = 0; s < 8; ++s)
                     mma_ss(tmem + 64 * buf, kd + koff(s, kHalf128), qd + koff(s, kHalf64), id_n64,
                            s > 0 ? 1u : 0u);
-                if (i > 0) {   // the softmax warps have read dP^T of tile i - 1
+                if (i > 0) {
                     if (!(ok = wait(&bars->dp_free, (i - 1) & 1, ctl))) break;
                     tc_fence_after();
                 }
@@ -1094,9 +1093,15 @@ __global__ void __launch_bounds__(kThreads, 1) dkdvq_kernel(const __grid_constan
                     mma_ss(tmem + kColDP, vd + koff(s, kHalf128), dod + koff(s, kHalf64), id_n64,
                            s > 0 ? 1u : 0u);
                 mma_commit(&bars->s_full[buf]);
-                if (i > 0 && !(ok = grad_mma(i - 1))) break;
+                if (i > 0) {
+                    if (!(ok = wait(&bars->p_full[(i - 1) & 1], ((i - 1) >> 1) & 1, ctl))) break;
+                    grad_mma(i - 1);
+                }
             }
-            if (ok && (ok = grad_mma(kt.nq - 1))) mma_commit(&bars->o_done);
+            if (ok && (ok = wait(&bars->p_full[(kt.nq - 1) & 1], ((kt.nq - 1) >> 1) & 1, ctl))) {
+                grad_mma(kt.nq - 1);
+                mma_commit(&bars->o_done);
+            }
             mma_commit(&bars->drain);
             if (!mbar_wait_bounded(&bars->drain, 0, nullptr, kDrainLimitNs))
                 atomicOr(&g_bwd_status, 1u);
@@ -1117,19 +1122,11 @@ __global__ void __launch_bounds__(kThreads, 1) dkdvq_kernel(const __grid_constan
         const int key = kt.krow0 + krow;
         const bool key_ok = key < kt.kend && !(kt.seg == 1 && key >= kt.L);
         float* blk = reinterpret_cast<float*>(smem + Smem::dq_off + warp * kBlockBytes);
-        // Reduces this warp's block of dQ^T of query tile j (head dim
-        // [32 quarter, +32) x queries [32 wg, +32)) into the accumulator, as
-        // 32 query rows x 32 head-dim floats.
-        auto reduce_dq = [&](int j) {
-            uint32_t r[32];
-            tmem_ld32(tmem + kColDQ + 32 * wg + lane_off, r);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars->dq_empty);
-                bulk_wait_group_read<0>();   // the previous block has left shared memory
-            }
+        // Adds this warp's block of dQ^T of query tile j (head dim [32 quarter,
+        // +32) x queries [32 wg, +32), read from tensor memory into r) into
+        // the accumulator, staged in shared memory as 32 query rows x 32 floats.
+        auto reduce_dq = [&](int j, const uint32_t (&r)[32]) {
+            if (lane == 0) bulk_wait_group_read<0>();   // the previous block has left
             __syncwarp();
 #pragma unroll
             for (int q = 0; q < 32; ++q) blk[q * 32 + lane] = __uint_as_float(r[q]);
@@ -1143,6 +1140,7 @@ __global__ void __launch_bounds__(kThreads, 1) dkdvq_kernel(const __grid_constan
                 bulk_commit_group();
             }
         };
+        const uint32_t tDQ = tmem + kColDQ + 32 * wg + lane_off;
         bool ok = true;
         for (int i = 0; i < kt.nq; ++i) {
             const int buf = i & 1;
@@ -1150,41 +1148,49 @@ __global__ void __launch_bounds__(kThreads, 1) dkdvq_kernel(const __grid_constan
             if (!(ok = wait_warp(&bars->s_full[buf], (i >> 1) & 1, ctl))) break;
             if (!(ok = wait_warp(&bars->l_full[st], (i / kQdStages) & 1, ctl))) break;
             tc_fence_after();
-            uint32_t sr[32], dr[32];
-            const uint32_t tS = tmem + 64 * buf + 32 * wg + lane_off;
-            tmem_ld32(tS, sr);
-            tmem_ld32(tmem + kColDP + 32 * wg + lane_off, dr);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->dp_free);
             uint32_t pp[16], pd[16];
-            p_ds(sr, dr, lbuf + st * 64 + 32 * wg, sl2x2, pp, pd);
+            const uint32_t tS = tmem + 64 * buf + 32 * wg + lane_off;
+            {
+                uint32_t sr[32], dr[32];
+                tmem_ld32(tS, sr);
+                tmem_ld32(tmem + kColDP + 32 * wg + lane_off, dr);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->dp_free);
+                p_ds(sr, dr, lbuf + st * 64 + 32 * wg, sl2x2, pp, pd);
+            }
             if (!key_ok) {
 #pragma unroll
                 for (int c = 0; c < 16; ++c) pd[c] = 0u;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->l_empty[st]);
-            if (i > 0) {   // dQ^T of tile i - 1 formed: dS^T's buffer is free
+            uint32_t r[32];
+            if (i > 0) {   // dQ^T of tile i - 1 formed; dS^T's buffer is free
                 if (!(ok = wait_warp(&bars->dq_full, (i - 1) & 1, ctl))) break;
                 tc_fence_after();
             }
+            tmem_ld32(tDQ, r);   // dQ^T of tile i - 1 (not used at i = 0)
             tmem_st16(tS, pp);
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 *reinterpret_cast<uint4*>(ds_row + 16 * ((4 * wg + c) ^ (krow & 7))) =
                     make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
             fence_proxy_async_smem();
+            tmem_wait_ld();
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->p_full[buf]);
-            if (i > 0) reduce_dq(i - 1);
+            if (i > 0) reduce_dq(i - 1, r);
         }
         if (ok && (ok = wait_warp(&bars->dq_full, (kt.nq - 1) & 1, ctl))) {
             tc_fence_after();
-            reduce_dq(kt.nq - 1);
+            uint32_t r[32];
+            tmem_ld32(tDQ, r);
+            tmem_wait_ld();
+            reduce_dq(kt.nq - 1, r);
         }
         if (ok) ok = wait_warp(&bars->o_done, 0, ctl);
         tc_fence_after();
