@@ -51,8 +51,11 @@ def test_l2_note_follows_the_workload():
     assert bench.config_of(I.WORKLOADS["480p"], 1)["l2"] == bench.l2_note(I.WORKLOADS["480p"])
 
 
-def test_recorded_traffic_only_for_the_captured_workload():
-    """The committed ncu traffic is the 480p launch's: other workloads get none."""
-    assert bench.recorded_traffic(I.WORKLOADS["720p"]) is None
+def test_recorded_traffic_only_for_the_captured_workloads():
+    """The committed ncu traffic covers the 480p and 720p launches; a workload
+    without a capture (ragged) gets none."""
+    assert bench.recorded_traffic(I.WORKLOADS["ragged"]) is None
     t = bench.recorded_traffic(I.WORKLOADS["480p"])
     assert t is None or t > 8.0e8      # 480p moves at least its 817.8 MB of Q, K, V and O
+    t = bench.recorded_traffic(I.WORKLOADS["720p"])
+    assert t is None or t > 1.8e9      # 720p: at least its 1870.5 MB of Q, K, V and O
