@@ -13,8 +13,10 @@
 //   * S_i = Q_i K^T runs as kind::i8 into s32 tensor memory: 4 k-steps of 32
 //     bytes instead of 8 of 16 bf16, at twice the bf16 rate;
 //   * the softmax turns an s32 score into fp32 exactly (|S| < 2^22: add the
-//     magic 1.5 * 2^23 as an integer, subtract it as a float), then
-//     x = S * (s_q s_k scale log2 e) in log2 units;
+//     magic 1.5 * 2^23 as an integer; the FMA that scales S by
+//     s_q s_k scale log2 e takes the magic's share back out of its addend),
+//     so x = S * (s_q s_k scale log2 e) in log2 units costs one integer add
+//     per score and one FMA per score pair;
 //   * the running maximum is an integer, raised to the ceiling of a tile
 //     maximum when that exceeds it by more than 2, so every O rescale is by an
 //     exact power of two; P' = 2^(x - m + 6) <= 2^8 is rounded to E4M3 (four
@@ -182,7 +184,6 @@ constexpr float kMagicF = 12582912.0f;
 template <bool MASK>
 __device__ __forceinline__ float p_half(const uint32_t (&sr)[4][32], uint32_t (&pk)[16], int h,
                                         uint64_t c2, uint64_t b2, int valid) {
-    const uint64_t magic2 = f2_pack(kMagicF, kMagicF);
     uint64_t acc[2] = {0, 0};
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
@@ -191,10 +192,9 @@ __device__ __forceinline__ float p_half(const uint32_t (&sr)[4][32], uint32_t (&
         for (int pr = 0; pr < 2; ++pr) {
             const int k = 64 * h + 4 * c + 2 * pr;
             const uint32_t s0 = sr[k >> 5][k & 31], s1 = sr[k >> 5][(k & 31) + 1];
-            // exact s32 -> fp32 (|S| < 2^22), then x - m + 6 in log2 units
-            const uint64_t sf = f2_sub(f2_pack(__uint_as_float(s0 + kMagic),
-                                               __uint_as_float(s1 + kMagic)),
-                                       magic2);
+            // 1.5 * 2^23 + S exactly in fp32 (|S| < 2^22); b2 takes the offset
+            // back out, so the FMA gives x - m + 6 in log2 units
+            const uint64_t sf = f2_pack(__uint_as_float(s0 + kMagic), __uint_as_float(s1 + kMagic));
             float x0, x1;
             f2_unpack(f2_fma(sf, c2, b2), x0, x1);
             if (MASK) {
@@ -373,19 +373,26 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_q8_kernel(const __grid
                 const float c = sq * sk * p.sl2;   // log2 units per unit of S
                 // tile maximum of the valid s32 scores (c >= 0 keeps the order);
                 // only a tail tile pays for masking
-                int mi = INT32_MIN;
+                // (8 independent chains of 3-way maxima, so the latency of one
+                // dependent chain of 64 does not sit on every row's path)
+                int mk[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mk[k] = INT32_MIN;
                 if (valid < kBlock) {
 #pragma unroll
                     for (int k = 0; k < 128; k += 2) {
                         const int a0 = k < valid ? (int)r[k >> 5][k & 31] : INT32_MIN;
                         const int a1 = k + 1 < valid ? (int)r[k >> 5][(k & 31) + 1] : INT32_MIN;
-                        mi = __vimax3_s32(mi, a0, a1);
+                        mk[(k >> 1) & 7] = __vimax3_s32(mk[(k >> 1) & 7], a0, a1);
                     }
                 } else {
 #pragma unroll
                     for (int k = 0; k < 128; k += 2)
-                        mi = __vimax3_s32(mi, (int)r[k >> 5][k & 31], (int)r[k >> 5][(k & 31) + 1]);
+                        mk[(k >> 1) & 7] = __vimax3_s32(mk[(k >> 1) & 7], (int)r[k >> 5][k & 31],
+                                                        (int)r[k >> 5][(k & 31) + 1]);
                 }
+                const int mi = max(__vimax3_s32(mk[0], mk[1], mk[2]),
+                                   max(__vimax3_s32(mk[3], mk[4], mk[5]), max(mk[6], mk[7])));
                 const float m_tile = ceilf((float)mi * c);
                 if (j == 0) {
                     m_run = m_tile;
@@ -397,7 +404,11 @@ __global__ void __launch_bounds__(kThreads, 1) joint_attn_q8_kernel(const __grid
                     m_run = m_new;
                 }
                 const uint64_t c2 = f2_pack(c, c);
-                const uint64_t b2 = f2_pack(6.0f - m_run, 6.0f - m_run);
+                // (1.5 * 2^23 + S) c + b = S c + 6 - m: one FMA per score pair
+                // instead of a subtraction and an FMA (b's own rounding is
+                // 2^-24 of 1.5 * 2^23 c, far below the E4M3 step of P')
+                const float bm = fmaf(-kMagicF, c, 6.0f - m_run);
+                const uint64_t b2 = f2_pack(bm, bm);
                 float sum = 0.f;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {

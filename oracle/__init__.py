@@ -85,7 +85,7 @@ def _configure(lib):
         [ctypes.c_int] * 5 + [u8p, u8p, fp]
     lib.oracle_attention_q8_rows.argtypes = [i8p, i8p, fp, fp, i8p, i8p, fp, fp, u8p, u8p, fp,
                                              ctypes.POINTER(ctypes.c_int)] + [ctypes.c_int] * 5 + \
-        [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp]
+        [ctypes.c_double, ctypes.POINTER(ctypes.c_long), ctypes.c_long, dp, ctypes.c_double, dp]
     lib.oracle_adaln_modulate.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3 + [ctypes.c_double]
     lib.oracle_gated_residual.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 3
     lib.oracle_adaln_modulate_bwd.argtypes = [dp, dp, dp] + [ctypes.c_int] * 3 + [
@@ -379,9 +379,12 @@ def quant_v_e4m3(vv, vc, ctx_len=None):
 
 
 def attention_q8_rows(qv8, qc8, sqv, sqc, kv8, kc8, skv, skc, vv8, vc8, sv, ctx_len, rows,
-                      scale: Optional[float] = None):
+                      scale: Optional[float] = None, rel: Optional[float] = None):
     """Output rows (b, h, joint i) of the 8-bit joint attention (Wan 2.1
-    report, section 4.4.3) from quantised operands (see oracle.c)."""
+    report, section 4.4.3) from quantised operands (see oracle.c).  With
+    ``rel``, also the bound on how far rounding the P' that lie within a
+    relative ``rel`` of an E4M3 midpoint the other way can move each output
+    element: returns (out, amb)."""
     arrs = [np.ascontiguousarray(a) for a in (qv8, qc8, kv8, kc8)]
     qv8, qc8, kv8, kc8 = (a.astype(np.int8, copy=False) for a in arrs)
     vv8 = np.ascontiguousarray(vv8, dtype=np.uint8)
@@ -394,6 +397,7 @@ def attention_q8_rows(qv8, qc8, sqv, sqc, kv8, kc8, skv, skc, vv8, vc8, sv, ctx_
         scale = 1.0 / math.sqrt(D)
     rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
     out = np.zeros((rows.shape[0], D), dtype=np.float64)
+    amb = np.zeros_like(out) if rel is not None else None
     cl_p, _keep = _ctx_ptr(ctx_len)
     i8 = ctypes.POINTER(ctypes.c_byte)
     u8 = ctypes.POINTER(ctypes.c_ubyte)
@@ -404,14 +408,17 @@ def attention_q8_rows(qv8, qc8, sqv, sqc, kv8, kc8, skv, skc, vv8, vc8, sv, ctx_
             sqc.ctypes.data_as(f), kv8.ctypes.data_as(i8), kc8.ctypes.data_as(i8),
             skv.ctypes.data_as(f), skc.ctypes.data_as(f), vv8.ctypes.data_as(u8),
             vc8.ctypes.data_as(u8), sv.ctypes.data_as(f), cl_p, B, Nv, Nc, H, D, scale,
-            rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), rows.shape[0], _p(out))
-    return out
+            rows.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), rows.shape[0], _p(out),
+            float(rel or 0.0), _p(amb) if amb is not None else None)
+    return out if rel is None else (out, amb)
 
 
-def attention_q8(qv, kv, vv, qc, kc, vc, ctx_len=None, rows=None, scale=None):
+def attention_q8(qv, kv, vv, qc, kc, vc, ctx_len=None, rows=None, scale=None, rel=None):
     """The whole 8-bit method from unquantised q, k, v: quantise (q per token,
     k per 128-token block, v per channel), then attend.  Returns (o_vis, o_ctx)
-    when ``rows`` is None, else the requested rows."""
+    when ``rows`` is None, else the requested rows; with ``rel``, each output
+    comes with its rounding-ambiguity bound (attention_q8_rows):
+    (o_vis, o_ctx, amb_vis, amb_ctx), or (rows, amb)."""
     qv8, sqv = quant_int8(qv, 1)
     qc8, sqc = quant_int8(qc, 1)
     kv8, skv = quant_int8(kv, 128)
@@ -423,12 +430,15 @@ def attention_q8(qv, kv, vv, qc, kc, vc, ctx_len=None, rows=None, scale=None):
     if full:
         bb, hh, ii = np.meshgrid(np.arange(B), np.arange(H), np.arange(Nv + Nc), indexing="ij")
         rows = np.stack([bb.ravel(), hh.ravel(), ii.ravel()], axis=1)
-    out = attention_q8_rows(qv8, qc8, sqv.reshape(B, H, -1), sqc.reshape(B, H, -1), kv8, kc8,
-                            skv, skc, vv8, vc8, sv, ctx_len, rows, scale)
+    res = attention_q8_rows(qv8, qc8, sqv.reshape(B, H, -1), sqc.reshape(B, H, -1), kv8, kc8,
+                            skv, skc, vv8, vc8, sv, ctx_len, rows, scale, rel)
     if not full:
-        return out
-    out = out.reshape(B, H, Nv + Nc, D).transpose(0, 2, 1, 3)
-    return np.ascontiguousarray(out[:, :Nv]), np.ascontiguousarray(out[:, Nv:])
+        return res
+    parts = []
+    for a in (res if rel is not None else (res,)):
+        a = a.reshape(B, H, Nv + Nc, D).transpose(0, 2, 1, 3)
+        parts += [np.ascontiguousarray(a[:, :Nv]), np.ascontiguousarray(a[:, Nv:])]
+    return tuple(parts)
 
 
 def _grid_struct(grid) -> _Grid:

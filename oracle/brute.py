@@ -152,10 +152,12 @@ def quant_int8(x, block):
     return codes, scales
 
 
-def attention_q8(qv, kv, vv, qc, kc, vc, ctx_len=None, scale=None):
+def attention_q8(qv, kv, vv, qc, kc, vc, ctx_len=None, scale=None, round_input=None):
     """The 8-bit method with numpy arrays: float32 quantisation, torch's E4M3
     conversion, and for each (row, head) the whole score vector at once (the
-    concatenated valid keys), m = ceil of its maximum, P' = 2^(x - m + 6)."""
+    concatenated valid keys), m = ceil of its maximum, P' = 2^(x - m + 6).
+    round_input (optional): maps the vector P' to the values that are rounded
+    to E4M3 for the P V product (the row sum keeps P')."""
     qv, kv, vv, qc, kc, vc = (np.asarray(a, dtype=np.float64) for a in (qv, kv, vv, qc, kc, vc))
     B, Nv, H, D = qv.shape
     Nc = qc.shape[1]
@@ -184,7 +186,8 @@ def attention_q8(qv, kv, vv, qc, kc, vc, ctx_len=None, scale=None):
                 x = (kd[:, h] @ q8[h]) * float(sq[h]) * scale * np.log2(np.e)
                 m = np.ceil(x.max())
                 p = 2.0 ** (x - m + 6)
-                o = (e4m3(p) @ v8[:, h]) * sv[h] / p.sum()
+                pr = p if round_input is None else round_input(p)
+                o = (e4m3(pr) @ v8[:, h]) * sv[h] / p.sum()
                 if i < Nv:
                     out_v[b, i, h] = o
                 else:

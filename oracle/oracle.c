@@ -779,7 +779,14 @@ void oracle_rmsnorm_rope_bwd(const double* x, const double* g, const double* dy,
  * 2^(old - new) computes the same values: every P' it rounds differs from the
  * one here by an exact power of two, which E4M3 rounding commutes with, except
  * for keys whose P' here falls in E4M3's subnormal range (x_j < m - 12, a
- * weight below 2^-12 of the largest). */
+ * weight below 2^-12 of the largest).
+ * The report does not fix the precision in which P' is formed before its E4M3
+ * rounding.  An implementation whose P' differs from this one's by a relative
+ * amount up to rel can round a P' that lies that close to a rounding midpoint
+ * the other way.  With amb non-NULL, amb[r][d] bounds what those choices can
+ * move o: sum_j w_j |v8_jd| scale_v,d / sum_j P'_j, where w_j is the larger
+ * distance from E4M3(P'_j) to E4M3(P'_j (1 - rel)) and to E4M3(P'_j (1 + rel))
+ * (0 unless P'_j is within rel of a midpoint). */
 
 /* E4M3: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits; no infinity; the
  * largest finite magnitude is 1.75 * 2^8 = 448; subnormals step 2^-9.       */
@@ -893,7 +900,7 @@ void oracle_attention_q8_rows(const signed char* qv, const signed char* qc, cons
                               const float* skv, const float* skc, const unsigned char* vv,
                               const unsigned char* vc, const float* sv, const int* ctx_len,
                               int B, int Nv, int Nc, int H, int D, double scale,
-                              const long* rows, long nrows, double* out)
+                              const long* rows, long nrows, double* out, double rel, double* amb)
 {
     (void)B;
     const double log2e = 1.4426950408889634;
@@ -902,13 +909,16 @@ void oracle_attention_q8_rows(const signed char* qv, const signed char* qc, cons
     {
         double* x = (double*)malloc(sizeof(double) * (size_t)(Nv + Nc + 1));
         double* acc = (double*)malloc(sizeof(double) * (size_t)D);
+        double* wacc = (double*)malloc(sizeof(double) * (size_t)D);
         #pragma omp for schedule(dynamic, 4)
         for (long r = 0; r < nrows; ++r) {
             const long b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
             const int L = ctx_len ? ctx_len[b] : Nc;
             const int nval = Nv + L;                /* valid keys: visual, then cond */
             double* o = out + r * (long)D;
-            for (int d = 0; d < D; ++d) { o[d] = 0.0; acc[d] = 0.0; }
+            for (int d = 0; d < D; ++d) { o[d] = 0.0; acc[d] = 0.0; wacc[d] = 0.0; }
+            if (amb)
+                for (int d = 0; d < D; ++d) amb[r * (long)D + d] = 0.0;
             if (i >= nval || nval == 0) continue;   /* no output */
             const signed char* q = (i < Nv) ? qv + ((b * Nv + i) * H + h) * (long)D
                                             : qc + ((b * Nc + (i - Nv)) * H + h) * (long)D;
@@ -934,9 +944,20 @@ void oracle_attention_q8_rows(const signed char* qv, const signed char* qc, cons
                 const double pq = oracle_e4m3_round(p);
                 const unsigned char* v = (seg ? vc : vv) + ((b * Ns + jj) * H + h) * (long)D;
                 for (int d = 0; d < D; ++d) acc[d] += pq * oracle_e4m3_decode(v[d]);
+                if (amb) {   /* the other rounding a P' this close to a midpoint can take */
+                    const double wl = fabs(pq - oracle_e4m3_round(p * (1.0 - rel)));
+                    const double wh = fabs(oracle_e4m3_round(p * (1.0 + rel)) - pq);
+                    const double w = wl > wh ? wl : wh;
+                    if (w > 0.0)
+                        for (int d = 0; d < D; ++d) wacc[d] += w * fabs(oracle_e4m3_decode(v[d]));
+                }
             }
             for (int d = 0; d < D; ++d) o[d] = acc[d] * sv[(b * H + h) * (long)D + d] / l;
+            if (amb)
+                for (int d = 0; d < D; ++d)
+                    amb[r * (long)D + d] = wacc[d] * sv[(b * H + h) * (long)D + d] / l;
         }
+        free(wacc);
         free(acc);
         free(x);
     }

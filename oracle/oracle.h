@@ -66,7 +66,8 @@ void oracle_attention_q8_rows(const signed char* qv, const signed char* qc, cons
                               const float* skv, const float* skc, const unsigned char* vv,
                               const unsigned char* vc, const float* sv, const int* ctx_len,
                               int B, int Nv, int Nc, int H, int D, double scale,
-                              const long* rows, long nrows, double* out);
+                              const long* rows, long nrows, double* out, double rel,
+                              double* amb);
 void oracle_adaln_modulate(const double* x, const double* shift, const double* scale,
                            double* y, int B, int N, int C, double eps);
 void oracle_gated_residual(const double* x, const double* branch, const double* gate,

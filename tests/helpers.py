@@ -90,6 +90,50 @@ _R = 2.0 ** -4 / np.sqrt(3.0)
 _A = 2.0 ** -10 / np.sqrt(3.0)
 
 
+def q8_rel(qv, kv, qc, kc, scale=None) -> float:
+    """Relative bound on how far the 8-bit kernel's P' (before its E4M3
+    rounding) can sit from the oracle's float64 P', for the oracle's
+    rounding-ambiguity bound.  The kernel forms x = S c - m + 6 (log2 units,
+    c = s_q s_k scale log2 e from three float32 roundings) as one float32 FMA of
+    1.5 * 2^23 + S (exact) by c with the addend rounded from
+    6 - m - 1.5 * 2^23 c, then P' = ex2.approx(x).  Against the exact x that
+    leaves, in log2 units, at most 2^-24 (1.5 * 2^23 c + m + 6) from the addend,
+    3 * 2^-24 (m + 12) from c over the keys in E4M3's normal range
+    (|S c| <= m + 12) and 2^-24 * 16 from the FMA's result; ex2.approx adds a
+    relative 2^-21.  c and m are bounded from the inputs: every quantisation
+    scale is at most the tensor's max |x| / 127, and |S| <= 127^2 * 128.
+    The bound is doubled."""
+    D = np.shape(qv)[-1]
+    if scale is None:
+        scale = D ** -0.5
+    amax = lambda *xs: max(float(np.abs(x).max()) if np.size(x) else 0.0 for x in xs)
+    c = amax(qv, qc) / 127.0 * amax(kv, kc) / 127.0 * scale * np.log2(np.e)
+    m = 127.0 * 127.0 * 128.0 * c + 1.0
+    dx = 2.0 ** -24 * (1.5 * 2.0 ** 23 * c + m + 6.0 + 3.0 * (m + 12.0) + 16.0)
+    return 2.0 * (np.log(2.0) * dx + 2.0 ** -21)
+
+
+def q8_parity(got: np.ndarray, ref: np.ndarray, amb: np.ndarray, rel: float, name: str = ""):
+    """The 8-bit kernel against the oracle's 8-bit method: the bf16 tolerance
+    of parity(), plus the oracle's bound amb on rounding the P' that lie within
+    rel of an E4M3 midpoint the other way, plus 2 rel of |o| (the row sum
+    takes the kernel's P' unrounded)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite output"
+    if got.size == 0:
+        return {"max_err": 0.0}
+    refr = I.round_f64_to_bf16(ref)
+    err = np.abs(got - refr)
+    scale = float(np.abs(refr).max())
+    allowed = 1e-2 * max(scale, 1e-30) + amb + 2.0 * rel * np.abs(ref)
+    rep = {"max_err": float(err.max()), "max_ref": scale, "max_amb": float(amb.max()),
+           "elements_past_bf16_tol": int((err > 1e-2 * max(scale, 1e-30)).sum())}
+    assert np.all(err <= allowed), (name, rep)
+    return rep
+
+
 def q8_exact_rows(qv, kv, vv, qc, kc, vc, ctx_len, trip, scale=None, chunk=128):
     """Exact attention rows and the 8-bit method's error sigma at the query
     rows ``trip`` [(b, h, i)]: returns (o [R, D], sigma [R, D]), float64."""

@@ -10,7 +10,7 @@ import torch
 import oracle
 from mmdit_joint_attention_b200 import _lib, api
 from mmdit_joint_attention_b200 import inputs as I
-from helpers import device_inputs, from_dev, parity
+from helpers import device_inputs, from_dev, parity, q8_parity, q8_rel
 
 pytestmark = pytest.mark.gpu
 
@@ -79,6 +79,7 @@ def test_backward_and_q8_wait_timeouts_are_reported():
                                      gin["do_vis"].f64, gin["do_ctx"].f64)
     for k in ("dq_vis", "dk_vis", "dv_vis"):
         parity(from_dev(g[k]), ref[k], "bf16", f"{k} after a timed-out launch")
-    rv, _ = oracle.attention_q8(inp["q_vis"].f64, inp["k_vis"].f64, inp["v_vis"].f64,
-                                inp["q_ctx"].f64, inp["k_ctx"].f64, inp["v_ctx"].f64)
-    parity(from_dev(q8v), rv, "bf16", "8-bit o_vis after a timed-out launch")
+    a = [inp[k].f64 for k in ("q_vis", "k_vis", "v_vis", "q_ctx", "k_ctx", "v_ctx")]
+    rel = q8_rel(a[0], a[1], a[3], a[4])
+    rv, _, av, _ = oracle.attention_q8(*a, rel=rel)
+    q8_parity(from_dev(q8v), rv, av, rel, "8-bit o_vis after a timed-out launch")

@@ -4,7 +4,9 @@ Int8 S = Q K^T, FP8 E4M3 O = P V) through the C ABI.
 The quantisers must reproduce the oracle's codes and scales exactly (integer
 and byte work).  The attention is compared with the oracle's whole 8-bit
 method run from the unquantised inputs (the oracle quantises by itself), with
-the bf16 criterion; small cases in full, 480p on sampled rows.  It is also
+the bf16 criterion plus the oracle's bound on the E4M3 roundings of P' that
+the kernel's float32 P' may take the other way (helpers.q8_rel, q8_parity);
+small cases in full, 480p on sampled rows.  It is also
 compared with the EXACT attention, within the error the method's own rounding
 steps allow (tests/helpers.py: int8 scores, E4M3 P' and v; every element
 within 6 sigma, mean |error| / sigma at most 0.8)."""
@@ -15,7 +17,8 @@ import torch
 import oracle
 from mmdit_joint_attention_b200 import api
 from mmdit_joint_attention_b200 import inputs as I
-from helpers import device_inputs, from_dev, parity, q8_close_to_exact, q8_exact_rows
+from helpers import (device_inputs, from_dev, q8_close_to_exact, q8_exact_rows, q8_parity,
+                     q8_rel)
 
 pytestmark = pytest.mark.gpu
 
@@ -69,9 +72,10 @@ def test_attention_q8_full(case):
     w = CASES[case]
     inp, ov, oc = _run(w)
     args = [inp[k].f64 for k in ("q_vis", "k_vis", "v_vis", "q_ctx", "k_ctx", "v_ctx")]
-    rv, rc = oracle.attention_q8(*args, ctx_len=inp["ctx_len"])
-    parity(ov, rv, "bf16", f"{case} o_vis")
-    parity(oc, rc, "bf16", f"{case} o_ctx")
+    rel = q8_rel(args[0], args[1], args[3], args[4])
+    rv, rc, av, ac = oracle.attention_q8(*args, ctx_len=inp["ctx_len"], rel=rel)
+    q8_parity(ov, rv, av, rel, f"{case} o_vis")
+    q8_parity(oc, rc, ac, rel, f"{case} o_ctx")
     for b, L in enumerate(w.ctx_lengths()):
         assert np.all(oc[b, L:] == 0.0)
     # against the exact attention, within the 8-bit method's error model
@@ -92,11 +96,12 @@ def test_attention_q8_sampled_480p():
         trip.append(np.stack([np.zeros_like(rows), np.full_like(rows, h), rows], axis=1))
     trip = np.concatenate(trip)
     args = [inp[k].f64 for k in ("q_vis", "k_vis", "v_vis", "q_ctx", "k_ctx", "v_ctx")]
-    ref = oracle.attention_q8(*args, ctx_len=inp["ctx_len"], rows=trip)
+    rel = q8_rel(args[0], args[1], args[3], args[4])
+    ref, amb = oracle.attention_q8(*args, ctx_len=inp["ctx_len"], rows=trip, rel=rel)
     got = full[trip[:, 0], trip[:, 2], trip[:, 1]]
     vis = trip[:, 2] < w.Nv
-    parity(got[vis], ref[vis], "bf16", "480p q8 o_vis rows")
-    parity(got[~vis], ref[~vis], "bf16", "480p q8 o_ctx rows")
+    q8_parity(got[vis], ref[vis], amb[vis], rel, "480p q8 o_vis rows")
+    q8_parity(got[~vis], ref[~vis], amb[~vis], rel, "480p q8 o_ctx rows")
     # against the exact attention on two heads, within the method's error model
     sub = trip[np.isin(trip[:, 1], (0, 13))]
     o, sig = q8_exact_rows(*args, inp["ctx_len"], sub)

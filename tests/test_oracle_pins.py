@@ -943,6 +943,36 @@ def pin_q8_brute():
 
 
 @pin
+def pin_q8_rounding_ambiguity_bound():
+    """The bound on choosing the other E4M3 rounding for every P' within a
+    relative rel of a midpoint: zero at rel = 0; at rel = 2^-10, outputs of the
+    numpy restatement whose P' are each moved by a relative amount up to rel
+    before rounding (random factors, and the two extremes) stay within it of
+    the oracle's, and some do move (the bound is not vacuous)."""
+    r = RNG(75)
+    B, Nv, Nc, H, D = 2, 300, 140, 2, 128
+    t = [I.round_f64_to_bf16(r.standard_normal((B, n, H, D)) * sd)
+         for n, sd in ((Nv, 1.5), (Nv, 1.5), (Nv, 1.0), (Nc, 1.5), (Nc, 1.5), (Nc, 1.0))]
+    cl = np.array([140, 70], np.int32)
+    _, _, z0, z1 = oracle.attention_q8(*t, cl, rel=0.0)
+    assert not z0.any() and not z1.any()
+    rel = 2.0 ** -10
+    ov, oc, av, ac = oracle.attention_q8(*t, cl, rel=rel)
+    assert av.max() > 0
+    moved = 0.0
+    factors = [lambda p, g=RNG(76 + k): p * (1.0 + rel * g.uniform(-1.0, 1.0, p.shape))
+               for k in range(2)]
+    factors += [lambda p: p * (1.0 + rel), lambda p: p * (1.0 - rel)]
+    for f in factors:
+        bv, bc = brute.attention_q8(*t, cl, round_input=f)
+        for got, ref, bound in ((bv, ov, av), (bc, oc, ac)):
+            dev = np.abs(got - ref)
+            assert np.all(dev <= bound + 1e-12 * (1.0 + np.abs(ref)))
+            moved = max(moved, float(dev.max()))
+    assert moved > 1e-6
+
+
+@pin
 def pin_q8_close_to_exact():
     """The 8-bit method stays within its own rounding-error model of the exact
     attention (tests/helpers.py: every element within 6 sigma of the error
