@@ -724,15 +724,19 @@ def run_ours(args):
     # modulate and residual backward on the visual stream: x and dy read, dx
     # written; branch and dout read, dbranch written (dx = dout not asked for)
     dy_x = torch.randn(t["x_vis"].shape, generator=gen, device=dev).to(torch.bfloat16)
-    mb_ms = time_ms(lambda: api.adaln_modulate_bwd(t["x_vis"], t["scale_vis"], dy_x))
+    dx_x = torch.empty_like(dy_x)   # gradient buffers held across steps, as in training
+    dsh = torch.empty((B, C), dtype=torch.float32, device=dev)
+    dsc = torch.empty_like(dsh)
+    mb_ms = time_ms(lambda: api.adaln_modulate_bwd(t["x_vis"], t["scale_vis"], dy_x, dx=dx_x,
+                                                   dshift=dsh, dscale=dsc))
     rb_ms = time_ms(lambda: api.gated_residual_bwd(t["o_vis"].view(B, Nv, C), t["gate_vis"],
-                                                   dy_x))
+                                                   dy_x, dbranch=dx_x, dgate=dsh))
     eb = 3 * B * Nv * C * 2
     for key, ms_ in (("adaln_modulate_bwd_vis", mb_ms), ("gated_residual_bwd_vis", rb_ms)):
         bwd_rows[key] = {"ms": ms_, "GB/s": eb / (ms_ * 1e-3) / 1e9,
                          "frac_hbm": eb / (ms_ * 1e-3) / 1e9 / float(peaks()[0]["hbm_gbs"]),
                          "bytes": eb}
-    del do_vis, do_ctx, grads, lse, delta, dy_x, bwd_ws
+    del do_vis, do_ctx, grads, lse, delta, dy_x, dx_x, dsh, dsc, bwd_ws
 
     # 3D window attention (1x2x2 and 4x1x1 windows): permuting prologue for
     # q/k, row permutation of v, windowed attention back to raster order

@@ -629,15 +629,22 @@ def gated_residual(x: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor,
 
 
 def adaln_modulate_bwd(x: torch.Tensor, scale: torch.Tensor, dy: torch.Tensor,
-                       eps: float = 1e-6, stream=None
+                       eps: float = 1e-6, dx: Optional[torch.Tensor] = None,
+                       dshift: Optional[torch.Tensor] = None,
+                       dscale: Optional[torch.Tensor] = None, stream=None
                        ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """Backward of adaln_modulate: (dx, dshift, dscale) for the gradient dy of y."""
+    """Backward of adaln_modulate: (dx, dshift, dscale) for the gradient dy of y
+    (each allocated here unless given; dshift and dscale are overwritten)."""
     dt = _dtype(x, dy)
     _f32(scale)
     B, N, C = x.shape
-    dx = torch.empty_like(x)
-    dshift = torch.empty((B, C), dtype=torch.float32, device=x.device)
-    dscale = torch.empty_like(dshift)
+    if dx is None:
+        dx = torch.empty_like(x)
+    if dshift is None:
+        dshift = torch.empty((B, C), dtype=torch.float32, device=x.device)
+    if dscale is None:
+        dscale = torch.empty((B, C), dtype=torch.float32, device=x.device)
+    _f32(dshift, dscale)
     st = _lib.lib().mmdit_adaln_modulate_bwd(_ptr(x), _ptr(scale), _ptr(dy), _ptr(dx),
                                              _ptr(dshift), _ptr(dscale), B, N, C, eps, dt,
                                              _stream(stream))
@@ -646,14 +653,20 @@ def adaln_modulate_bwd(x: torch.Tensor, scale: torch.Tensor, dy: torch.Tensor,
 
 
 def gated_residual_bwd(branch: torch.Tensor, gate: torch.Tensor, dout: torch.Tensor,
+                       dbranch: Optional[torch.Tensor] = None,
+                       dgate: Optional[torch.Tensor] = None,
                        stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Backward of gated_residual: (dbranch, dgate) for the gradient dout of
-    the output; the gradient of x is dout itself."""
+    the output (each allocated here unless given; dgate is overwritten); the
+    gradient of x is dout itself."""
     dt = _dtype(branch, dout)
     _f32(gate)
     B, N, C = branch.shape
-    dbranch = torch.empty_like(branch)
-    dgate = torch.empty((B, C), dtype=torch.float32, device=branch.device)
+    if dbranch is None:
+        dbranch = torch.empty_like(branch)
+    if dgate is None:
+        dgate = torch.empty((B, C), dtype=torch.float32, device=branch.device)
+    _f32(dgate)
     st = _lib.lib().mmdit_gated_residual_bwd(_ptr(branch), _ptr(gate), _ptr(dout), None,
                                              _ptr(dbranch), _ptr(dgate), B, N, C, dt,
                                              _stream(stream))

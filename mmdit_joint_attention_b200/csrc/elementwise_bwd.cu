@@ -394,6 +394,23 @@ int threads_for(int C, int E) { return ((C / E + 31) / 32) * 32; }
 // CTAs per sample: as many as the SMs hold at once (occupancy of the kernel at
 // this block size), but at least 4 * kRows rows per CTA so that the final
 // atomics stay few against the rows.
+// Zeroes the fp32 column-sum outputs (a, and b when not null; n floats each)
+// before the row kernels add their partial sums into them.
+__global__ void __launch_bounds__(256) zero_sums_kernel(float* __restrict__ a,
+                                                        float* __restrict__ b, int n) {
+    for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) {
+        a[i] = 0.f;
+        if (b) b[i] = 0.f;
+    }
+}
+
+cudaError_t zero_sums(float* a, float* b, size_t n, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+    zero_sums_kernel<<<blocks, 256, 0, s>>>(a, b, (int)n);
+    return cudaGetLastError();
+}
+
 template <typename K>
 cudaError_t grid_for(K kern, int threads, size_t smem, int B, int N, dim3& grid) {
     int per_sm = 0;
@@ -496,8 +513,7 @@ extern "C" int mmdit_adaln_modulate_bwd(const void* x, const float* scale, const
         if (overlaps(dx, x, bytes) || (dx != dy && overlaps(dx, dy, bytes)))
             return MMDIT_ERR_ARG;
     }
-    cudaError_t e = cudaMemsetAsync(dshift, 0, vec, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dscale, 0, vec, s);
+    cudaError_t e = zero_sums(dshift, dscale, vec / sizeof(float), s);
     if (e == cudaSuccess && N > 0)
         e = dt == MMDIT_BF16
                 ? dispatch_modulate_bwd<__nv_bfloat16>(x, scale, dy, dx, dshift, dscale, B, N, C,
@@ -528,7 +544,7 @@ extern "C" int mmdit_gated_residual_bwd(const void* branch, const float* gate, c
             (dx && dx != dout && overlaps(dx, dout, bytes)))
             return MMDIT_ERR_ARG;
     }
-    cudaError_t e = cudaMemsetAsync(dgate, 0, (size_t)B * C * sizeof(float), s);
+    cudaError_t e = zero_sums(dgate, nullptr, (size_t)B * C, s);
     if (e == cudaSuccess && N > 0)
         e = dt == MMDIT_BF16
                 ? dispatch_residual_bwd<__nv_bfloat16>(branch, gate, dout, dx, dbranch, dgate, B,

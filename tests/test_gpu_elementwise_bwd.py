@@ -47,7 +47,13 @@ def test_modulate_bwd_matches_oracle(case):
     w = CASES[case]
     inp, dy, _ = _inputs(w, 41)
     x, sc = inp["x_vis"], inp["scale_vis"]
-    dx, dsh, dsc = api.adaln_modulate_bwd(to_dev(x), to_dev(sc), to_dev(dy))
+    # caller-held outputs full of NaN: every element must be written, and the
+    # column sums zeroed before the rows add into them
+    xd = to_dev(x)
+    nan = lambda shape, dt: torch.full(shape, float("nan"), dtype=dt, device=xd.device)
+    dx, dsh, dsc = api.adaln_modulate_bwd(
+        xd, to_dev(sc), to_dev(dy), dx=nan(xd.shape, xd.dtype),
+        dshift=nan((w.B, w.C), torch.float32), dscale=nan((w.B, w.C), torch.float32))
     torch.cuda.synchronize()
     ref = oracle.adaln_modulate_bwd(x.f64, sc, dy.f64)
     parity(from_dev(dx), ref["dx"], w.dtype, f"{case} dx")
@@ -60,7 +66,11 @@ def test_residual_bwd_matches_oracle(case):
     w = CASES[case]
     inp, dout, br = _inputs(w, 43)
     g = inp["gate_vis"]
-    dbr, dg = api.gated_residual_bwd(to_dev(br), to_dev(g), to_dev(dout))
+    brd = to_dev(br)
+    dbr, dg = api.gated_residual_bwd(
+        brd, to_dev(g), to_dev(dout),
+        dbranch=torch.full(brd.shape, float("nan"), dtype=brd.dtype, device=brd.device),
+        dgate=torch.full((w.B, w.C), float("nan"), dtype=torch.float32, device=brd.device))
     torch.cuda.synchronize()
     ref = oracle.gated_residual_bwd(br.f64, g, dout.f64)
     parity(from_dev(dbr), ref["dbranch"], w.dtype, f"{case} dbranch")
