@@ -44,9 +44,9 @@ def test_wait_timeout_is_reported_and_context_survives():
 
 
 def test_backward_and_q8_wait_timeouts_are_reported():
-    """The same for the backward kernels and the 8-bit attention kernel: with
-    the waits cut short both report MMDIT_ERR_TIMEOUT, and the next call at the
-    default limit is correct."""
+    """The same for the backward kernels (both forms) and the 8-bit attention
+    kernel: with the waits cut short each reports MMDIT_ERR_TIMEOUT, and the
+    next call at the default limit is correct."""
     w = I.WORKLOADS["block"]
     inp = I.make_inputs(w, seed=3, parts=("qkv",))
     gin = I.make_grad_outputs(w, seed=3)
@@ -55,14 +55,17 @@ def test_backward_and_q8_wait_timeouts_are_reported():
     do_vis, do_ctx = to_dev(gin["do_vis"]), to_dev(gin["do_ctx"])
     qkv = (t["q_vis"], t["k_vis"], t["v_vis"], t["q_ctx"], t["k_ctx"], t["v_ctx"])
     ov, oc, lse = api.joint_attention_fwd(*qkv)
+    ws = api.bwd_workspace(w.B, w.Nv, w.Nc, w.H)
     torch.cuda.synchronize()
     L = _lib.lib()
-    for call in ("bwd", "q8"):
+    for call in ("bwd", "bwd_one_pass", "q8"):
         assert api.device_status() == 0
         try:
             L.mmdit_set_wait_timeout_ns(1)
             if call == "bwd":
                 api.joint_attention_bwd(*qkv, ov, oc, do_vis, do_ctx, lse)
+            elif call == "bwd_one_pass":
+                api.joint_attention_bwd(*qkv, ov, oc, do_vis, do_ctx, lse, workspace=ws)
             else:
                 api.joint_attention_8bit(*qkv)
             status = api.device_status()
@@ -71,6 +74,7 @@ def test_backward_and_q8_wait_timeouts_are_reported():
         assert status == _lib.STATUS_CODES["MMDIT_ERR_TIMEOUT"], call
         assert api.device_status() == 0
     g = api.joint_attention_bwd(*qkv, ov, oc, do_vis, do_ctx, lse)
+    g1 = api.joint_attention_bwd(*qkv, ov, oc, do_vis, do_ctx, lse, workspace=ws)
     q8v, q8c, _ = api.joint_attention_8bit(*qkv)
     torch.cuda.synchronize()
     assert api.device_status() == 0
@@ -79,6 +83,7 @@ def test_backward_and_q8_wait_timeouts_are_reported():
                                      gin["do_vis"].f64, gin["do_ctx"].f64)
     for k in ("dq_vis", "dk_vis", "dv_vis"):
         parity(from_dev(g[k]), ref[k], "bf16", f"{k} after a timed-out launch")
+        parity(from_dev(g1[k]), ref[k], "bf16", f"one-pass {k} after a timed-out launch")
     a = [inp[k].f64 for k in ("q_vis", "k_vis", "v_vis", "q_ctx", "k_ctx", "v_ctx")]
     rel = q8_rel(a[0], a[1], a[3], a[4])
     rv, _, av, _ = oracle.attention_q8(*a, rel=rel)
