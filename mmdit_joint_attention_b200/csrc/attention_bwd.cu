@@ -12,7 +12,7 @@
 // Rows without an output (padded conditioning rows) carry lse = +inf, so all
 // their P are 0 and they contribute nothing; padded keys get zero dK and dV.
 //
-// Three launches:
+// Two forms, three launches each.  Two-kernel form (deterministic):
 //   1. delta_kernel: D_i into the caller's fp32 workspace (one read of O, dO).
 //   2. dq_kernel, query-stationary: a CTA owns 128 query rows of one (b, h)
 //      and streams the 128-key K/V tiles.  S = Q K^T and dP = dO V^T go to
@@ -26,6 +26,13 @@
 //      512 tensor-memory columns.
 // Splitting dQ from dK/dV computes S and dP twice but needs no atomics and no
 // fp32 dQ accumulator in global memory.
+// One-pass form (a caller workspace holds an fp32 dQ accumulator):
+//   1. delta_kernel, which also zeroes the accumulator;
+//   2. dkdvq_kernel: dkdv_kernel's pipeline that also forms each query tile's
+//      dQ^T = K^T dS^T and reduces it into the accumulator (section 3b);
+//   3. dq_convert_kernel: dQ = scale * accumulator, in bf16.
+// S and dP are formed once (10 N^2 D executed FLOPs per (sample, head)
+// instead of 14); the order of the dQ sums varies from run to run.
 //
 // Every wait is bounded as in the forward kernel: a wait that runs out sets an
 // abort flag and the backward status word, every role leaves its loop, copies
