@@ -7,8 +7,8 @@
 A step is one pass of the whole path over one sample of the workload (by
 default 480p/81 frames: 21x30x52 = 32,760 visual + 512 cond tokens, 24 heads x
 128): adaLN modulate of both streams, QK-RMSNorm + 3D RoPE (visual) /
-QK-RMSNorm (cond), joint attention (with the merge of its split tail), and the
-gated residual of both streams.  Inputs are synthetic (seeded PCG64, N(0,1)
+QK-RMSNorm (cond), joint attention (the pair kernel: CTA pairs sharing one
+MMA-issuing thread), and the gated residual of both streams.  Inputs are synthetic (seeded PCG64, N(0,1)
 bf16; see mmdit_joint_attention_b200/inputs.py) and resident in HBM; at 480p
 q/k/v are 201 MB each, larger than the 126 MB L2, so no flush is needed.
 
@@ -45,7 +45,7 @@ from mmdit_joint_attention_b200 import inputs as I  # noqa: E402
 
 METRIC = "joint-attention TFLOP/s and % bf16 peak at 480p/81f; norm/RoPE GB/s % HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_SRC = os.path.join(ROOT, "mmdit_joint_attention_b200", "csrc", "attention_tc.cu")
+ATTN_SRC = os.path.join(ROOT, "mmdit_joint_attention_b200", "csrc", "attention_pair.cu")
 PROFILES = os.path.join(ROOT, "profiles")
 
 
@@ -68,14 +68,15 @@ def attn_source_hash() -> str:
 
 def recorded_traffic(w):
     """DRAM bytes per attention launch of workload ``w`` from the committed
-    ncu summary of that workload (profiles/joint_attn_bf16_<name>.md), if
-    there is one and it was taken on the current kernel source (else None)."""
+    ncu summary of that workload's pair-kernel launch (the kernel the step's
+    attention runs: profiles/joint_attn_pair_<name>.md), if there is one and
+    it was taken on the current kernel source (else None)."""
     try:
-        text = open(os.path.join(PROFILES, f"joint_attn_bf16_{w.name}.md")).read()
+        text = open(os.path.join(PROFILES, f"joint_attn_pair_{w.name}.md")).read()
     except OSError:
         return None
     m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    h = re.search(r"attention_tc\.cu sha256\[:16\]:\s*([0-9a-f]+)", text)
+    h = re.search(r"attention_pair\.cu sha256\[:16\]:\s*([0-9a-f]+)", text)
     if not m or not h or h.group(1) != attn_source_hash():
         return None
     return float(m.group(1))
@@ -439,7 +440,11 @@ def make_step(w: I.Workload, t: dict, attn_ws, stream, dev):
                            out=t["xo_ctx"])
         mark(4)
 
-    # 6 launches, plus the merge of the attention's split tail when it splits
+    # 6 launches: the attention without lse runs the pair kernel (one launch,
+    # no split tail); with no visual tokens it would run the one-SM kernel,
+    # plus the merge of its split tail when the plan splits
+    if Nv > 0:
+        return step, 6
     plan = (ctypes.c_longlong * 4)()
     _lib.check("mmdit_joint_attention_split_plan", _lib.lib().mmdit_joint_attention_split_plan(
         B, Nv, Nc, H, torch.cuda.get_device_properties(dev).multi_processor_count,

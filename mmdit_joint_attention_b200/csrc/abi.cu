@@ -767,10 +767,11 @@ int mmdit_device_status(void* stream) {
     cudaError_t e = read_and_clear_device_status(&w, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_status(e, "device_status");
     if ((e = read_and_clear_bwd_status(&wb)) != cudaSuccess) return cuda_status(e, "device_status");
-    unsigned int wq = 0, we = 0;
+    unsigned int wq = 0, we = 0, wp = 0;
     if ((e = read_and_clear_q8_status(&wq)) != cudaSuccess) return cuda_status(e, "device_status");
     if ((e = read_and_clear_elem_status(&we)) != cudaSuccess) return cuda_status(e, "device_status");
-    return (w | wb | wq | we) ? MMDIT_ERR_TIMEOUT : MMDIT_OK;
+    if ((e = read_and_clear_pair_status(&wp)) != cudaSuccess) return cuda_status(e, "device_status");
+    return (w | wb | wq | we | wp) ? MMDIT_ERR_TIMEOUT : MMDIT_OK;
 }
 
 void mmdit_set_wait_timeout_ns(unsigned long long ns) { set_wait_timeout_ns(ns); }

@@ -909,6 +909,11 @@ int launch_joint_attention_bf16(const void* qv, const void* kv, const void* vv, 
     if (!encode_fn()) return -1;
     const int q_tiles = (Nv + kBlockM - 1) / kBlockM + (Nc + kBlockM - 1) / kBlockM;
     if (B == 0 || q_tiles == 0) return 0;
+    // the plain form runs on CTA pairs (attention_pair.cu): same outputs, half
+    // the issued products per SM; the split tail's workspace is then unused
+    if (!win && !qn && !lse && Nv > 0)
+        return launch_joint_attention_pair(qv, kv, vv, qc, kc, vc, ctx_len, ov, oc, B, Nv, Nc, H,
+                                           softmax_scale, s);
     Params p;
     std::memset(&p, 0, sizeof(p));
     long long items = 0;  // window mode: CTAs of the one-dimensional grid

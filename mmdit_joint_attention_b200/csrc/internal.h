@@ -159,6 +159,16 @@ cudaError_t launch_quant_v_e4m3(const void* vv, const void* vc, const int32_t* c
                                 void* cc, float* scales, int B, int Nv, int Nc, int H,
                                 cudaStream_t s);
 cudaError_t read_and_clear_q8_status(unsigned int* out);
+// The same for the pair kernel (attention_pair.cu).
+cudaError_t read_and_clear_pair_status(unsigned int* out);
+// Plain bf16 joint attention (no windows, no Q normalisation, no lse) on CTA
+// pairs with one MMA-issuing thread per pair; outputs bit for bit those of
+// launch_joint_attention_bf16's kernel.  Return convention of
+// launch_joint_attention_bf16.
+int launch_joint_attention_pair(const void* qv, const void* kv, const void* vv, const void* qc,
+                                const void* kc, const void* vc, const int32_t* ctx_len, void* ov,
+                                void* oc, int B, int Nv, int Nc, int H, float softmax_scale,
+                                cudaStream_t s);
 
 // Limit of one bounded pipeline wait (set_wait_timeout_ns, else the default).
 uint64_t wait_timeout_ns();
