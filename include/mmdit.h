@@ -161,9 +161,11 @@ MMDIT_API int mmdit_qk_norm_rope_text_bwd(const void* q_in, const void* k_in,
  *   ctx_len  DEVICE int32 [B], each clamped to [0, Nc]; NULL = all Nc valid
  *   o_vis [B, Nv, H, D] dt, o_ctx [B, Nc, H, D] dt  (written; must not alias inputs)
  *   softmax_scale > 0 (1/sqrt(D) in the usual form)
- * bf16 runs on the tcgen05 tensor cores (fp32 accumulation in tensor memory);
- * f32 runs an fp32 CUDA-core kernel.  Nv or Nc may be 0 (the ctx pointers may
- * then be NULL).
+ * bf16 runs on the tcgen05 tensor cores (fp32 accumulation in tensor memory):
+ * with Nv > 0 on clusters of two SMs that share one MMA-issuing thread
+ * (cta_group::2 products of 256 query rows), else on one SM per work item; the
+ * two give the same bits.  f32 runs an fp32 CUDA-core kernel.  Nv or Nc may be
+ * 0 (the ctx pointers may then be NULL).
  * Errors: MMDIT_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED / _CUDA. */
 MMDIT_API int mmdit_joint_attention(const void* q_vis, const void* k_vis, const void* v_vis,
                           const void* q_ctx, const void* k_ctx, const void* v_ctx,
@@ -282,12 +284,15 @@ MMDIT_API int mmdit_joint_attention_fwd(const void* q_vis, const void* k_vis, co
  * mmdit_joint_attention / mmdit_joint_attention_fwd up to the order of the
  * floating-point sums [Vimoo §2.2 joint attention].
  *
- * The bf16 kernel runs one CTA per SM, one item (b, h, pair of 128-row query
- * tiles) each, and every item costs the same.  The items beyond the last whole
- * wave would run as a short wave on a few SMs; with a workspace, each of them
- * is split over its keys into pieces that run side by side, and a second
- * kernel merges the pieces' partial rows (rescaling them to a common maximum,
- * as between key tiles).  Problems with fewer items than SMs split every item.
+ * The split applies to the one-SM bf16 kernel, which runs one CTA per SM,
+ * one item (b, h, pair of 128-row query tiles) each, and every item costs the
+ * same.  The items beyond the last whole wave would run as a short wave on a
+ * few SMs; with a workspace, each of them is split over its keys into pieces
+ * that run side by side, and a second kernel merges the pieces' partial rows
+ * (rescaling them to a common maximum, as between key tiles).  Problems with
+ * fewer items than SMs split every item.  Without lse and with Nv > 0 the call
+ * runs the paired kernel of mmdit_joint_attention instead (faster whole than
+ * the one-SM kernel split), and the workspace is unused.
  *   lse: DEVICE fp32 [B, H, Nv + Nc] as mmdit_joint_attention_fwd, or NULL
  *   workspace: DEVICE memory, 256-byte aligned, of workspace_bytes bytes, or
  *     NULL; MMDIT_ATTENTION_WORKSPACE_BYTES suffice for every problem.  The
