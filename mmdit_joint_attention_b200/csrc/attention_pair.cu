@@ -164,6 +164,10 @@ __device__ __forceinline__ void tile_of(const Params& p, int t, int& s, int& row
     else { s = 1; row0 = (t - p.q_tiles_vis) * kBlockM; }
 }
 
+// The per-row softmax steps below are those of joint_attn_bf16_kernel
+// (attention_tc.cu), kept identical so that both kernels give the same bits
+// (tests/test_gpu_pair.py compares them on every run).
+// O row of this thread *= f, 32 tensor-memory columns at a time.
 __device__ __forceinline__ void rescale_o(uint32_t tO, float f) {
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
@@ -175,6 +179,8 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float f) {
         tmem_st32(tO + 32 * c, o);
     }
 }
+// P = 2^(s * scale_log2 - m) for keys [64 h, 64 h + 64) of one score row,
+// packed two bf16 keys per column into rh; returns their sum.
 __device__ __forceinline__ float exp_half(const float (&sv)[128], uint32_t (&rh)[32], int h,
                                           uint64_t sl2x2, uint64_t negm2) {
     uint64_t acc[4] = {0, 0, 0, 0};
