@@ -9,10 +9,12 @@
 //   * each CTA holds half of every K tile (keys 64 r .. 64 r + 63 of the
 //     128-key tile, r the CTA's rank in the pair) and half of every V tile
 //     (head dims 64 r .. 64 r + 63); a product reads the B operand from both
-//     CTAs, so each CTA loads and stores half the K/V bytes;
-//   * one thread (rank 0, warp 9) issues the pair's products: half the
-//     instructions, commits and waits per SM of the one-SM kernel (the issuing
-//     thread, not the tensor core, bounds that kernel);
+//     CTAs, so each SM's shared memory takes half the K/V fills and serves
+//     half the B-operand reads;
+//   * one thread (rank 0, warp 9) issues the pair's products; an instruction
+//     costs it about what an M = 128 one costs the one-SM kernel's issuer, so
+//     the products reach each SM at about the same rate, each with less
+//     shared-memory traffic behind it;
 //   * both CTAs' copies complete on the leader's barriers (the cta_group::2
 //     form of the TMA load, no multicast); the leader's commits arrive on the
 //     barrier at the same offset in both CTAs; the softmax warps of both CTAs
